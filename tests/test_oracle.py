@@ -1,0 +1,307 @@
+"""Pins of the fp64 oracle against facts the pages and the mathematics fix.
+
+Each test ties the oracle to something other than itself: values worked by
+hand from the defining rule (tests/golden/), closed forms, special cases, the
+convex-gate identity, and invariances that follow from the definition.  The
+tests are chosen so that a plausible slip in the oracle (a dropped term, an
+unsquared or transposed score, an exclusive instead of inclusive causal sum, a
+missing normalisation, a wrong psi index) fails at least one of them; the
+mutation tests at the end plant such slips in copies of the oracle's C source
+and check that the pins catch them.
+"""
+import os
+import subprocess
+import ctypes
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+import oracle
+import workloads
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _read_golden(name):
+    rows = []
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.split("#", 1)[0].strip()
+            if line:
+                rows.append([Fraction(x) for x in line.split()])
+    a = np.array([[float(x) for x in r] for r in rows])
+    q, k, v, o = a[:, 0:2], a[:, 2:4], a[:, 4:6], a[:, 6:8]
+    return (x[None, None] for x in (q, k, v, o))
+
+
+# ---------------------------------------------------------------------------
+# worked examples (tests/golden)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("fn", ["direct", "recurrent"])
+def test_worked_example_p2(fn):
+    q, k, v, o_expected = _read_golden("worked_example_p2.txt")
+    o = getattr(oracle, fn)(q, k, v)
+    np.testing.assert_allclose(o, o_expected, rtol=0, atol=1e-14)
+
+
+@pytest.mark.parametrize("fn", ["direct", "recurrent"])
+def test_zero_denominator_reading(fn):
+    q, k, v, o_expected = _read_golden("zero_denominator.txt")
+    o = getattr(oracle, fn)(q, k, v)
+    np.testing.assert_array_equal(o, o_expected)
+
+
+# ---------------------------------------------------------------------------
+# the four spec identities
+# ---------------------------------------------------------------------------
+
+def _rand(B=2, H=2, T=40, p=5, dv=3, seed=11):
+    rng = np.random.default_rng(seed)
+    return (rng.standard_normal((B, H, T, p)), rng.standard_normal((B, H, T, p)),
+            rng.standard_normal((B, H, T, dv)))
+
+
+@pytest.mark.parametrize("shape", [(1, 1, 1, 1, 1), (2, 3, 37, 4, 5), (1, 2, 64, 16, 16), (1, 1, 9, 32, 2)])
+def test_direct_equals_recurrent(shape):
+    B, H, T, p, dv = shape
+    q, k, v = _rand(B, H, T, p, dv, seed=T + p)
+    np.testing.assert_allclose(oracle.direct(q, k, v), oracle.recurrent(q, k, v), rtol=1e-11, atol=1e-12)
+
+
+def test_first_output_is_first_value():
+    q, k, v = _rand()
+    o = oracle.direct(q, k, v)
+    np.testing.assert_allclose(o[:, :, 0, :], v[:, :, 0, :], rtol=1e-14, atol=0)
+
+
+@pytest.mark.parametrize("fn", ["direct", "recurrent"])
+def test_convex_gate_bounds(fn):
+    """Nonnegative weights: each output coordinate lies in the range of the past values."""
+    q, k, v = _rand(T=80, seed=3)
+    o = getattr(oracle, fn)(q, k, v)
+    lo = np.minimum.accumulate(v, axis=2)
+    hi = np.maximum.accumulate(v, axis=2)
+    eps = 1e-12
+    assert np.all(o >= lo - eps) and np.all(o <= hi + eps)
+    # the bound is tight somewhere only through nonnegativity: also check a
+    # query anti-aligned with keys still gives weights >= 0 (signs cancel)
+    o_neg = getattr(oracle, fn)(-q, k, v)
+    np.testing.assert_allclose(o_neg, o, rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("fn", ["direct", "recurrent"])
+def test_identical_keys_running_mean(fn):
+    rng = np.random.default_rng(5)
+    B, H, T, p, dv = 1, 2, 33, 6, 4
+    kvec = rng.standard_normal(p)
+    k = np.broadcast_to(kvec, (B, H, T, p)).copy()
+    q = rng.standard_normal((B, H, T, p))
+    v = rng.standard_normal((B, H, T, dv))
+    o = getattr(oracle, fn)(q, k, v)
+    mean = np.cumsum(v, axis=2) / np.arange(1, T + 1)[None, None, :, None]
+    np.testing.assert_allclose(o, mean, rtol=1e-12, atol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# the convex output gate, gate form (ai.info summary, Main Findings:
+# o_t = alpha_t r_{t-1} + beta_t v_t with alpha_t = D_{t-1}/D_t,
+# beta_t = c_t/D_t, alpha_t + beta_t = 1)
+# ---------------------------------------------------------------------------
+
+def test_gate_form_identity():
+    q, k, v = _rand(B=1, H=1, T=30, p=4, dv=3, seed=21)
+    T = q.shape[2]
+    o = oracle.direct(q, k, v)
+    for t in range(1, T):
+        # previous readout read with the current query: replace q_{t-1} by q_t
+        # in the length-t prefix and take its last output
+        qq = q[:, :, : t].copy()
+        qq[:, :, t - 1] = q[:, :, t]
+        r_prev, d_prev = oracle.direct_rows(qq, k[:, :, :t], v[:, :, :t], [0], [t - 1], return_d=True)
+        _, d_t = oracle.direct_rows(q, k, v, [0], [t], return_d=True)
+        c_t = float(np.dot(q[0, 0, t], k[0, 0, t]) ** 2)
+        alpha, beta = d_prev[0] / d_t[0], c_t / d_t[0]
+        assert abs(alpha + beta - 1.0) < 1e-12
+        np.testing.assert_allclose(o[0, 0, t], alpha * r_prev[0] + beta * v[0, 0, t], rtol=1e-11, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# closed forms and special cases
+# ---------------------------------------------------------------------------
+
+def test_orthonormal_keys_exact_retrieval():
+    """Keys from an orthonormal basis, query = basis vector j: o_t is the mean
+    of the values stored under e_j so far (0 if none yet)."""
+    rng = np.random.default_rng(7)
+    p, dv, T = 8, 3, 50
+    # signed standard basis: exactly orthonormal in floating point
+    R = np.eye(p) * rng.choice([-1.0, 1.0], size=p)
+    key_ids = rng.integers(0, p, size=T)
+    qry_ids = rng.integers(0, p, size=T)
+    k = R[:, key_ids].T[None, None]
+    q = R[:, qry_ids].T[None, None]
+    v = rng.standard_normal((1, 1, T, dv))
+    o = oracle.direct(q, k, v)
+    for t in range(T):
+        match = [s for s in range(t + 1) if key_ids[s] == qry_ids[t]]
+        want = v[0, 0, match].mean(axis=0) if match else np.zeros(dv)
+        np.testing.assert_allclose(o[0, 0, t], want, rtol=1e-10, atol=1e-10)
+
+
+@pytest.mark.parametrize("fn", ["direct", "recurrent"])
+def test_p1_closed_form(fn):
+    rng = np.random.default_rng(8)
+    T, dv = 25, 4
+    q = rng.standard_normal((1, 1, T, 1)) + 2.0
+    k = rng.standard_normal((1, 1, T, 1))
+    v = rng.standard_normal((1, 1, T, dv))
+    o = getattr(oracle, fn)(q, k, v)
+    k2 = k[0, 0, :, 0] ** 2
+    want = np.cumsum(k2[:, None] * v[0, 0], axis=0) / np.cumsum(k2)[:, None]
+    np.testing.assert_allclose(o[0, 0], want, rtol=1e-12, atol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# invariances that follow from the definition
+# ---------------------------------------------------------------------------
+
+def test_invariances():
+    q, k, v = _rand(B=1, H=2, T=35, p=6, dv=4, seed=9)
+    rng = np.random.default_rng(10)
+    o = oracle.direct(q, k, v)
+    T = q.shape[2]
+    # sign flips of individual queries and keys
+    sq = rng.choice([-1.0, 1.0], size=(1, 2, T, 1))
+    sk = rng.choice([-1.0, 1.0], size=(1, 2, T, 1))
+    np.testing.assert_allclose(oracle.direct(q * sq, k * sk, v), o, rtol=1e-11, atol=1e-12)
+    # per-query scaling and a global key scale
+    cq = rng.uniform(0.1, 10.0, size=(1, 2, T, 1))
+    np.testing.assert_allclose(oracle.direct(q * cq, k * 3.7, v), o, rtol=1e-10, atol=1e-11)
+    # joint rotation of queries and keys
+    Rm, _ = np.linalg.qr(rng.standard_normal((6, 6)))
+    np.testing.assert_allclose(oracle.direct(q @ Rm.T, k @ Rm.T, v), o, rtol=1e-10, atol=1e-11)
+    # affine equivariance in v
+    A = rng.standard_normal((4, 4))
+    b = rng.standard_normal(4)
+    np.testing.assert_allclose(oracle.direct(q, k, v @ A + b), o @ A + b, rtol=1e-10, atol=1e-10)
+
+
+def test_not_invariant_to_per_key_scaling():
+    """Scaling one key changes its weight by c^2: the result must move (guards
+    against an implementation that normalises k internally)."""
+    q, k, v = _rand(B=1, H=1, T=10, p=3, dv=2, seed=12)
+    k2 = k.copy()
+    k2[0, 0, 3] *= 5.0
+    assert np.abs(oracle.direct(q, k2, v) - oracle.direct(q, k, v))[0, 0, 3:].max() > 1e-3
+
+
+# ---------------------------------------------------------------------------
+# state semantics of the recurrence (checkpoint / resume, decode)
+# ---------------------------------------------------------------------------
+
+def test_split_and_resume_and_final_state():
+    q, k, v = _rand(B=2, H=1, T=31, p=4, dv=3, seed=13)
+    o_full, S_full, z_full = oracle.recurrent(q, k, v, return_state=True)
+    t0 = 12
+    o1, S1, z1 = oracle.recurrent(q[:, :, :t0], k[:, :, :t0], v[:, :, :t0], return_state=True)
+    o2, S2, z2 = oracle.recurrent(q[:, :, t0:], k[:, :, t0:], v[:, :, t0:], S1, z1, return_state=True)
+    np.testing.assert_allclose(np.concatenate([o1, o2], axis=2), o_full, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(S2, S_full, rtol=1e-12, atol=1e-12)
+    # the final state is the sum of outer products psi(k_s) v_s^T; check one
+    # entry by brute force with explicit indices (i, j, e)
+    i, j, e = 2, 1, 0
+    want = sum(k[0, 0, s, i] * k[0, 0, s, j] * v[0, 0, s, e] for s in range(31))
+    assert abs(S_full[0, 0, i * 4 + j, e] - want) < 1e-12
+    assert abs(z_full[0, 0, i * 4 + j] - sum(k[0, 0, s, i] * k[0, 0, s, j] for s in range(31))) < 1e-12
+    # decode step continues the sequence
+    o_dec, S3, z3 = oracle.decode_step(q[:, :, -1], k[:, :, -1], v[:, :, -1], S_full, z_full)
+    qe = np.concatenate([q, q[:, :, -1:]], axis=2)
+    ke = np.concatenate([k, k[:, :, -1:]], axis=2)
+    ve = np.concatenate([v, v[:, :, -1:]], axis=2)
+    np.testing.assert_allclose(o_dec, oracle.direct(qe, ke, ve)[:, :, -1], rtol=1e-11, atol=1e-12)
+
+
+def test_direct_rows_matches_full_and_threads_do_not_matter():
+    q, k, v = _rand(B=2, H=3, T=45, p=4, dv=3, seed=14)
+    o = oracle.direct(q, k, v, nthreads=1)
+    o4 = oracle.direct(q, k, v, nthreads=4)
+    np.testing.assert_array_equal(o, o4)
+    bh = np.array([0, 5, 3, 2])
+    t = np.array([0, 44, 17, 30])
+    rows = oracle.direct_rows(q, k, v, bh, t)
+    np.testing.assert_array_equal(rows, o.reshape(6, 45, 3)[bh, t])
+    np.testing.assert_array_equal(oracle.recurrent(q, k, v, nthreads=1), oracle.recurrent(q, k, v, nthreads=3))
+
+
+def test_workload_inputs_shapes_and_bf16_rounding():
+    cfg = workloads.CONFIGS["tiny"]
+    q, k, v = workloads.make_inputs(cfg)
+    assert q.shape == (1, 1, 256, 16) and v.shape == (1, 1, 256, 16)
+    np.testing.assert_allclose(np.linalg.norm(q, axis=-1), 1.0, rtol=1e-6)
+    qb, kb, vb = workloads.normal_qkv(1, 2, 64, 16, 64, seed=1, dtype="bf16")
+    bits = qb.view(np.uint32)
+    assert np.all(bits & 0xFFFF == 0)  # representable in bfloat16
+    # round-to-nearest-even on a few hand-picked cases
+    x = np.array([1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -9, -2.5], np.float32)
+    np.testing.assert_array_equal(workloads.round_bf16(x), np.array([1.0, 1.0, 1.0 + 2 ** -7, -2.5], np.float32))
+    qr, kr, vr = workloads.recall_qkv(1, 1, 2048, 32, 8, seed=3, dtype="f32")
+    # each codeword appears exactly twice per block of 1024 tokens
+    blk = kr[0, 0, :1024]
+    _, counts = np.unique(blk.round(6), axis=0, return_counts=True)
+    assert counts.min() == 2 and counts.max() == 2 and len(counts) == 512
+
+
+# ---------------------------------------------------------------------------
+# mutation check: slips planted in copies of the oracle's C source must fail
+# the pins above (the planted copy is compiled to a temporary library; the
+# committed oracle is never modified)
+# ---------------------------------------------------------------------------
+
+MUTATIONS = {
+    "exclusive causal sum": ("for (int64_t s = 0; s <= t; ++s) {\n    const double *k_s", "for (int64_t s = 0; s < t; ++s) {\n    const double *k_s"),
+    "unsquared score": ("double w = dot * dot;", "double w = dot;"),
+    "missing normalisation": ("o_t[e] = (D > 0.0) ? N[e] / D : 0.0;", "o_t[e] = N[e];"),
+    "transposed operands": ("dot += q_t[i] * k_s[i];", "dot += q_t[i] * (k_s[i] + (i == 0 ? k_s[1] - k_s[0] : 0.0));"),
+}
+
+
+def _build_mutant(tmp_path, name, old, new):
+    src = open(os.path.join(os.path.dirname(oracle.__file__), "kata_oracle.c")).read()
+    assert old in src, name
+    path = tmp_path / ("mut_%d.c" % abs(hash(name)))
+    path.write_text(src.replace(old, new, 1))
+    so = str(path) + ".so"
+    subprocess.check_call(["gcc", "-O1", "-std=c99", "-D_POSIX_C_SOURCE=200809L", "-fPIC", "-shared",
+                           "-o", so, str(path), "-lpthread"])
+    lib = ctypes.CDLL(so)
+    dp = ctypes.POINTER(ctypes.c_double)
+    lib.kata_oracle_direct.argtypes = [dp, dp, dp, dp, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                       ctypes.c_int, ctypes.c_int, ctypes.c_int]
+    return lib
+
+
+def _mutant_direct(lib, q, k, v):
+    q, k, v = (np.ascontiguousarray(x, np.float64) for x in (q, k, v))
+    B, H, T, p = q.shape
+    dv = v.shape[3]
+    o = np.empty((B, H, T, dv))
+    dp = ctypes.POINTER(ctypes.c_double)
+    lib.kata_oracle_direct(q.ctypes.data_as(dp), k.ctypes.data_as(dp), v.ctypes.data_as(dp),
+                           o.ctypes.data_as(dp), B, H, T, p, dv, 1)
+    return o
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_pins_catch_planted_mistakes(tmp_path, name):
+    old, new = MUTATIONS[name]
+    lib = _build_mutant(tmp_path, name, old, new)
+    q, k, v, o_expected = _read_golden("worked_example_p2.txt")
+    caught = not np.allclose(_mutant_direct(lib, q, k, v), o_expected, atol=1e-12)
+    qr, kr, vr = _rand(B=1, H=1, T=20, p=4, dv=3, seed=30)
+    o = _mutant_direct(lib, qr, kr, vr)
+    caught = caught or not np.allclose(o[:, :, 0], vr[:, :, 0], atol=1e-12)
+    lo, hi = np.minimum.accumulate(vr, axis=2), np.maximum.accumulate(vr, axis=2)
+    caught = caught or not (np.all(o >= lo - 1e-12) and np.all(o <= hi + 1e-12))
+    assert caught, "pin set failed to catch: " + name
