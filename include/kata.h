@@ -1,0 +1,159 @@
+/*
+ * kata.h -- C ABI of libkata, the sm_100a (B200) KATA forward library.
+ *
+ * The operation is causal normalized linear attention with the rank-one PSD
+ * feature map psi(u) = vec(u u^T).  For one (batch b, head h) pair, with
+ * q_t, k_t in R^p and v_t in R^dv (t = 1..T):
+ *
+ *   w_{t,s} = <psi(q_t), psi(k_s)> = (q_t . k_s)^2 >= 0
+ *   o_t     = sum_{s<=t} w_{t,s} v_s  /  sum_{s<=t} w_{t,s}
+ *
+ * -- gist.science technical summary of arXiv:2607.17419, sec. 2.2 ("PSD Kegel
+ *    (Rank-One)": the map squares the raw inner product) and sec. 2.1
+ *    ("Output Gating": the denominator is a parameter-free convex output
+ *    gate); ai.info summary, Main Findings ("The readout gate is free").
+ *
+ * Equivalently, with the fixed-size state S_t = sum_{s<=t} psi(k_s) v_s^T
+ * (p^2 x dv) and z_t = sum_{s<=t} psi(k_s) (p^2):
+ *   o_t = psi(q_t)^T S_t / psi(q_t)^T z_t
+ * (ai.info summary, Methodology in Plain English: a recurrence on a
+ * fixed-size state).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Layout     q, k: [B, H, T, p]; v, o: [B, H, T, dv]; row-major, contiguous.
+ *            State S: [B, H, p*p, dv] fp32 with psi index r = i*p + j;
+ *            z: [B, H, p*p] fp32.  A state is symmetric in (i, j).
+ * Dtypes     q, k, v, o share one dtype: KATA_F32 (fp32) or KATA_BF16
+ *            (bfloat16).  Accumulation is fp32.  o is rounded to nearest.
+ * Shapes     p in {16, 32}; dv in {16, 64}; B, H >= 1; T >= 0 (T = 0 is a
+ *            no-op); C in {64, 128}.  Anything else: KATA_ERR_UNSUPPORTED.
+ * Pointers   device pointers, 16-byte aligned (KATA_ERR_MISALIGNED
+ *            otherwise); input and output buffers must not overlap.
+ * Ownership  the caller owns every buffer; the library never allocates,
+ *            frees or retains caller memory.  Workspace is caller-provided.
+ * Streams    `stream` is a cudaStream_t passed as void* (NULL = legacy
+ *            default stream).  Calls enqueue work and return; they never
+ *            synchronise the device.
+ * Errors     argument errors are returned before anything is launched;
+ *            a failed launch returns KATA_ERR_CUDA.  Waits inside kernels are
+ *            bounded: a wait that runs out records KATA_ERR_TIMEOUT in a
+ *            device-side status word, the kernel drains its own copies and
+ *            returns, and kata_get_status() reports it.  No C++ exception
+ *            crosses this boundary.
+ * Scaling    no 1/sqrt(p) or temperature factor is applied, and q, k are
+ *            used as given (the caller normalises them if wanted).
+ * Zero gate  a row whose denominator is exactly 0 (q_t orthogonal to every
+ *            key so far) yields o_t = 0.
+ */
+#ifndef KATA_H_
+#define KATA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  KATA_OK = 0,
+  KATA_ERR_INVALID_ARG = 1,
+  KATA_ERR_UNSUPPORTED = 2,
+  KATA_ERR_MISALIGNED = 3,
+  KATA_ERR_WORKSPACE = 4,
+  KATA_ERR_CUDA = 5,
+  KATA_ERR_TIMEOUT = 6
+} kata_status_t;
+
+typedef enum { KATA_F32 = 0, KATA_BF16 = 1 } kata_dtype_t;
+
+/*
+ * Quadratic (flash-style) operating point: o = causal squared-score attention
+ * over the whole sequence, O(T^2) work, no state is materialised.
+ * (gist.science sec. 2.3, first operating point: a FlashAttention-style
+ * kernel that never materialises the full state.)
+ *
+ * q, k: [B,H,T,p] in; v: [B,H,T,dv] in; o: [B,H,T,dv] out.
+ */
+kata_status_t kata_fwd_quadratic(const void* q, const void* k, const void* v, void* o,
+                                 int B, int H, int T, int p, int dv,
+                                 kata_dtype_t dtype, void* stream);
+
+/*
+ * Bytes of device workspace kata_fwd_chunked needs for these sizes (0 when
+ * T == 0).  The same arguments must be passed to kata_fwd_chunked.
+ */
+size_t kata_fwd_chunked_workspace_size(int B, int H, int T, int p, int dv, int C,
+                                       kata_dtype_t dtype);
+
+/*
+ * Exact O(T) chunked-state operating point (gist.science sec. 2.3, "Chunked
+ * Parallelism" and the second operating point; ai.info Main Findings,
+ * "Chunk recurrence avoids the triangular solve"):
+ *   1. per-chunk states psi(K_c)^T [V_c | 1] built as tensor-core
+ *      contractions and summed over groups of consecutive chunks,
+ *   2. an exclusive associative (parallel prefix) scan of those sums along
+ *      the sequence, depth O(log(T/C)) (gist.science sec. 2.3,
+ *      "Complexiteitsreductie"),
+ *   3. per chunk: intra-chunk squared-score attention plus the readout
+ *      psi(Q_c) . S_prefix, then o = numerator / denominator.
+ * The result equals kata_fwd_quadratic's up to rounding; C is the chunk
+ * length and changes rounding only.
+ *
+ * S0, z0     optional state before token 1 ([B,H,p*p,dv], [B,H,p*p] fp32);
+ *            both NULL means a zero state; exactly one NULL is an error.
+ * S_out,z_out optional state after token T (same layouts); both or neither.
+ * workspace  device buffer of at least kata_fwd_chunked_workspace_size()
+ *            bytes, 256-byte aligned; contents on entry are ignored.
+ */
+kata_status_t kata_fwd_chunked(const void* q, const void* k, const void* v, void* o,
+                               int B, int H, int T, int p, int dv, int C,
+                               kata_dtype_t dtype,
+                               const float* S0, const float* z0,
+                               float* S_out, float* z_out,
+                               void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * One recurrent decode step for B*H independent streams (constant-time
+ * recurrent inference on the fixed-size state; arXiv abstract on aiqbench):
+ *   S <- S + psi(k) v^T,  z <- z + psi(k),  o = psi(q)^T S / psi(q)^T z
+ * The update comes first, so the current token is included (the same causal
+ * convention as the forward entry points).
+ *
+ * q, k: [B,H,p]; v, o: [B,H,dv] (dtype); S: [B,H,p*p,dv] and z: [B,H,p*p]
+ * fp32, read and updated in place.
+ */
+kata_status_t kata_decode_step(const void* q, const void* k, const void* v, void* o,
+                               float* S, float* z, int B, int H, int p, int dv,
+                               kata_dtype_t dtype, void* stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the device-side status word
+ * of the current device (KATA_ERR_TIMEOUT if a bounded wait in a kernel ran
+ * out since the last call), or KATA_ERR_CUDA if the stream reports an error.
+ */
+kata_status_t kata_get_status(void* stream);
+
+/* Static, human-readable name of a status code. */
+const char* kata_status_string(kata_status_t status);
+
+/*
+ * Upper bound, in SM clock cycles, on every wait inside the library's
+ * kernels (default about 2^31, i.e. on the order of a second).  Affects
+ * launches made after the call.  Passing 0 makes any wait that is not
+ * already satisfied give up at once, which tests use to exercise the timeout
+ * path; a negative value restores the default.
+ */
+void kata_set_wait_limit(long long cycles);
+
+/* ABI version of this header: major * 10000 + minor * 100 + patch. */
+int kata_abi_version(void);
+
+#define KATA_ABI_VERSION 10000
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KATA_H_ */

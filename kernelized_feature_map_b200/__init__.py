@@ -1,0 +1,16 @@
+"""KATA forward pass on B200 (sm_100a).
+
+Causal normalized linear attention with the rank-one PSD feature map
+psi(u) = vec(u u^T): o_t = sum_{s<=t} (q_t.k_s)^2 v_s / sum_{s<=t} (q_t.k_s)^2.
+
+The computation lives in ``libkata.so`` (hand-written CUDA behind the C ABI of
+``include/kata.h``); this package is its Python binding.  Entry points:
+
+* :func:`kata_fwd_quadratic` -- flash-style O(T^2) forward;
+* :func:`kata_fwd_chunked`   -- exact O(T) chunked-state forward with an
+  associative scan across chunks;
+* :func:`kata_decode_step`   -- one recurrent step on the fixed-size state.
+"""
+from ._abi import (KataError, kata_abi_version, kata_decode_step, kata_fwd_chunked,  # noqa: F401
+                   kata_fwd_chunked_workspace_size, kata_fwd_quadratic, kata_get_status,
+                   kata_set_wait_limit, lib, status_string)

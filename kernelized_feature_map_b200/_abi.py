@@ -1,0 +1,163 @@
+"""Thin ctypes binding of libkata's C ABI (include/kata.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI.  Functions carry the C names and take torch tensors
+(device memory and the current CUDA stream are PyTorch's; nothing else is).
+If the library is missing, every call raises: there is no other path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libkata.so")
+
+KATA_OK, KATA_ERR_INVALID_ARG, KATA_ERR_UNSUPPORTED, KATA_ERR_MISALIGNED = 0, 1, 2, 3
+KATA_ERR_WORKSPACE, KATA_ERR_CUDA, KATA_ERR_TIMEOUT = 4, 5, 6
+KATA_F32, KATA_BF16 = 0, 1
+
+# name -> (restype, argtypes), mirroring include/kata.h
+_c_int, _c_size, _vp, _fp = ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p
+SIGNATURES = {
+    "kata_fwd_quadratic": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp]),
+    "kata_fwd_chunked_workspace_size": (_c_size, [_c_int] * 7),
+    "kata_fwd_chunked": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                  _fp, _fp, _fp, _fp, _vp, _c_size, _vp]),
+    "kata_decode_step": (_c_int, [_vp, _vp, _vp, _vp, _fp, _fp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp]),
+    "kata_get_status": (_c_int, [_vp]),
+    "kata_status_string": (ctypes.c_char_p, [_c_int]),
+    "kata_set_wait_limit": (None, [ctypes.c_longlong]),
+    "kata_abi_version": (_c_int, []),
+}
+
+_lib = None
+
+
+class KataError(RuntimeError):
+    """A libkata call returned a status other than KATA_OK."""
+
+    def __init__(self, fn, status):
+        self.status = status
+        super().__init__("%s failed: %s (%d)" % (fn, status_string(status), status))
+
+
+def lib():
+    """The loaded libkata (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError("libkata.so is not built (run: python -m kernelized_feature_map_b200.build); "
+                               "there is no fallback path")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().kata_status_string(int(status)).decode()
+
+
+def _check(fn, status):
+    if status != KATA_OK:
+        raise KataError(fn, status)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return KATA_BF16
+    if t.dtype == torch.float32:
+        return KATA_F32
+    raise TypeError("q, k, v must be torch.bfloat16 or torch.float32, got %s" % t.dtype)
+
+
+def _stream_ptr(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dev(t, name):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError("%s must be a CUDA tensor" % name)
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _opt(t, name):
+    return None if t is None else _dev(t, name)
+
+
+def kata_fwd_quadratic(q, k, v, o=None, stream=None):
+    """Flash-style O(T^2) forward.  q,k [B,H,T,p], v [B,H,T,dv] -> o [B,H,T,dv]."""
+    B, H, T, p = q.shape
+    dv = v.shape[-1]
+    if o is None:
+        o = torch.empty((B, H, T, dv), dtype=q.dtype, device=q.device)
+    _check("kata_fwd_quadratic", lib().kata_fwd_quadratic(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), B, H, T, p, dv, _dtype_code(q), _stream_ptr(stream)))
+    return o
+
+
+def kata_fwd_chunked_workspace_size(B, H, T, p, dv, C, dtype=torch.bfloat16) -> int:
+    code = KATA_BF16 if dtype == torch.bfloat16 else KATA_F32
+    return int(lib().kata_fwd_chunked_workspace_size(B, H, T, p, dv, C, code))
+
+
+def kata_fwd_chunked(q, k, v, C=64, S0=None, z0=None, return_state=False, o=None, workspace=None,
+                     S_out=None, z_out=None, stream=None):
+    """Exact O(T) chunked-state forward.
+
+    Returns o, or (o, S_T, z_T) when return_state is True.  S0/z0 give an
+    initial state ([B,H,p*p,dv], [B,H,p*p] fp32).  ``workspace`` may be a
+    preallocated uint8 CUDA tensor of at least the queried size.
+    """
+    B, H, T, p = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    if o is None:
+        o = torch.empty((B, H, T, dv), dtype=q.dtype, device=dev)
+    if return_state and S_out is None:
+        S_out = torch.empty((B, H, p * p, dv), dtype=torch.float32, device=dev)
+        z_out = torch.empty((B, H, p * p), dtype=torch.float32, device=dev)
+    need = kata_fwd_chunked_workspace_size(B, H, T, p, dv, C, q.dtype)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    _check("kata_fwd_chunked", lib().kata_fwd_chunked(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), B, H, T, p, dv, C, _dtype_code(q),
+        _opt(S0, "S0"), _opt(z0, "z0"), _opt(S_out, "S_out"), _opt(z_out, "z_out"),
+        _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(), _stream_ptr(stream)))
+    if return_state:
+        return o, S_out, z_out
+    return o
+
+
+def kata_decode_step(q, k, v, S, z, o=None, stream=None):
+    """One decode step; S [B,H,p*p,dv] and z [B,H,p*p] (fp32) are updated in place."""
+    B, H, p = q.shape
+    dv = v.shape[-1]
+    if o is None:
+        o = torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
+    _check("kata_decode_step", lib().kata_decode_step(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), _dev(S, "S"), _dev(z, "z"), B, H, p, dv,
+        _dtype_code(q), _stream_ptr(stream)))
+    return o
+
+
+def kata_get_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device status word."""
+    return int(lib().kata_get_status(_stream_ptr(stream)))
+
+
+def kata_set_wait_limit(cycles: int) -> None:
+    lib().kata_set_wait_limit(int(cycles))
+
+
+def kata_abi_version() -> int:
+    return int(lib().kata_abi_version())

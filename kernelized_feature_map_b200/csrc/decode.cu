@@ -1,0 +1,128 @@
+// decode.cu -- one recurrent decode step on the fixed-size state.
+//
+//   S <- S + psi(k) v^T,  z <- z + psi(k),  o = psi(q)^T S / psi(q)^T z
+//
+// (constant-time recurrent inference on the state, arXiv abstract; the
+// state recurrence of the ai.info summary, Methodology in Plain English.)
+//
+// The step is bound by HBM: every (b,h) streams its p^2 x dv fp32 state in
+// and out once (2 * 64 KiB at p = 16, dv = 64).  One CTA of 256 threads per
+// (b,h).  Thread layout: DV/4 consecutive threads cover one state row with
+// 16-byte vectors, so each pass of the CTA reads 256 x 16 B contiguous
+// bytes; all of a batch's loads are issued before any use so that enough
+// bytes are in flight per SM.  Loads and stores carry the streaming hint
+// (the state is touched once per step).  psi(k)_r and psi(q)_r for the row
+// r = i*p + j are formed on the fly from the p values staged in shared
+// memory.  The numerator is reduced over rows through shared memory.
+#include "kata_common.cuh"
+#include "kata_internal.h"
+
+namespace kata {
+
+template <typename Tin, int p, int DV>
+__global__ void __launch_bounds__(256) decode_step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
+                                                          const Tin* __restrict__ v, Tin* __restrict__ o,
+                                                          float* __restrict__ S, float* __restrict__ z) {
+  constexpr int P = p * p;
+  constexpr int CG = DV / 4;        // 16-byte column groups per state row
+  constexpr int RPP = 256 / CG;     // rows covered by one pass of the CTA
+  constexpr int PASSES = P / RPP;   // passes over the state
+  constexpr int BATCH = PASSES < 16 ? PASSES : 16;
+  static_assert(PASSES % BATCH == 0, "pass batching");
+
+  __shared__ float sq[p], sk[p], sv[DV];
+  __shared__ float4 red[256];
+  __shared__ float sden[8];
+
+  const int tid = threadIdx.x;
+  const long long bh = blockIdx.x;
+  if (tid < p) {
+    sq[tid] = Elem<Tin>::load(q + bh * p + tid);
+    sk[tid] = Elem<Tin>::load(k + bh * p + tid);
+  }
+  if (tid < DV) sv[tid] = Elem<Tin>::load(v + bh * DV + tid);
+  __syncthreads();
+
+  const int cg = tid % CG;
+  const int r0 = tid / CG;
+  const float4 vv = make_float4(sv[4 * cg], sv[4 * cg + 1], sv[4 * cg + 2], sv[4 * cg + 3]);
+  float4* Sb = reinterpret_cast<float4*>(S + bh * (long long)P * DV);
+
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
+  for (int b0 = 0; b0 < PASSES; b0 += BATCH) {
+    float4 s[BATCH];
+#pragma unroll
+    for (int i = 0; i < BATCH; ++i) s[i] = __ldcs(Sb + (r0 + (b0 + i) * RPP) * CG + cg);
+#pragma unroll
+    for (int i = 0; i < BATCH; ++i) {
+      const int r = r0 + (b0 + i) * RPP;
+      const int ii = r / p, jj = r % p;
+      const float pk = sk[ii] * sk[jj];
+      const float pq = sq[ii] * sq[jj];
+      s[i].x = fmaf(pk, vv.x, s[i].x);
+      s[i].y = fmaf(pk, vv.y, s[i].y);
+      s[i].z = fmaf(pk, vv.z, s[i].z);
+      s[i].w = fmaf(pk, vv.w, s[i].w);
+      __stcs(Sb + r * CG + cg, s[i]);
+      acc.x = fmaf(pq, s[i].x, acc.x);
+      acc.y = fmaf(pq, s[i].y, acc.y);
+      acc.z = fmaf(pq, s[i].z, acc.z);
+      acc.w = fmaf(pq, s[i].w, acc.w);
+    }
+  }
+
+  // normaliser z and the denominator psi(q)^T z
+  float den = 0.f;
+  float* zb = z + bh * P;
+  for (int r = tid; r < P; r += 256) {
+    const int ii = r / p, jj = r % p;
+    const float zz = __ldcs(zb + r) + sk[ii] * sk[jj];
+    __stcs(zb + r, zz);
+    den = fmaf(sq[ii] * sq[jj], zz, den);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
+  if ((tid & 31) == 0) sden[tid >> 5] = den;
+  red[tid] = acc;
+  __syncthreads();
+
+  if (tid < DV) {
+    float D = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) D += sden[w];
+    const int c4 = tid / 4, comp = tid % 4;
+    float num = 0.f;
+#pragma unroll 4
+    for (int j = 0; j < RPP; ++j) {
+      const float4 x = red[j * CG + c4];
+      num += comp == 0 ? x.x : comp == 1 ? x.y : comp == 2 ? x.z : x.w;
+    }
+    Elem<Tin>::store(o + bh * DV + tid, D > 0.f ? num / D : 0.f);
+  }
+}
+
+template <typename Tin, int p, int DV>
+static cudaError_t launch_decode_t(const void* q, const void* k, const void* v, void* o, float* S, float* z,
+                                   int BH, cudaStream_t st) {
+  decode_step_kernel<Tin, p, DV><<<BH, 256, 0, st>>>((const Tin*)q, (const Tin*)k, (const Tin*)v, (Tin*)o, S, z);
+  return cudaGetLastError();
+}
+
+template <typename Tin>
+static cudaError_t launch_decode_dt(const void* q, const void* k, const void* v, void* o, float* S, float* z,
+                                    int BH, int p, int dv, cudaStream_t st) {
+  if (p == 16 && dv == 64) return launch_decode_t<Tin, 16, 64>(q, k, v, o, S, z, BH, st);
+  if (p == 16 && dv == 16) return launch_decode_t<Tin, 16, 16>(q, k, v, o, S, z, BH, st);
+  if (p == 32 && dv == 64) return launch_decode_t<Tin, 32, 64>(q, k, v, o, S, z, BH, st);
+  if (p == 32 && dv == 16) return launch_decode_t<Tin, 32, 16>(q, k, v, o, S, z, BH, st);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_decode(const void* q, const void* k, const void* v, void* o, float* S, float* z, int BH,
+                          int p, int dv, kata_dtype_t dt, cudaStream_t st) {
+  if (dt == KATA_BF16) return launch_decode_dt<__nv_bfloat16>(q, k, v, o, S, z, BH, p, dv, st);
+  return launch_decode_dt<float>(q, k, v, o, S, z, BH, p, dv, st);
+}
+
+}  // namespace kata

@@ -1,0 +1,356 @@
+// flash_sm100.cu -- quadratic (flash-style) KATA forward on tcgen05 / TMEM.
+//
+// o_t = sum_{s<=t} (q_t.k_s)^2 v_s / sum_{s<=t} (q_t.k_s)^2 evaluated tile by
+// tile without materialising any state: the first operating point of the
+// gist.science technical summary, sec. 2.3 (a FlashAttention-style O(T^2)
+// forward), for bf16 inputs with fp32 accumulation.
+//
+// Per CTA: two 128-row query tiles of one (b,h); key/value tiles of 128 rows
+// stream through a 4-stage TMA ring.  Warp roles (320 threads):
+//   warp 0      TMA producer (one lane): Q tiles once, then K/V tiles;
+//   warp 1      TMEM allocator and MMA issuer (one lane);
+//   warps 2-9   two "weight" warpgroups, one per query tile; thread = row.
+// Per key tile j and query tile i:
+//   S_i   = Q_i K_j^T                    tcgen05.mma, A,B from shared memory,
+//                                         fp32 accumulator in TMEM (128 cols)
+//   W_i   = (S_i)^2, causal mask          tcgen05.ld -> registers -> bf16 ->
+//                                         tcgen05.st back over S_i in TMEM
+//   O_i  += W_i V_j                       tcgen05.mma with A = W_i from TMEM
+//   D_i  += W_i 1                         same A against a block of ones, so
+//                                         numerator and denominator use the
+//                                         identical bf16 weights
+// and at the end o = O_i / D_i (D = 0 gives 0), rounded to bf16.
+// Causal masking touches only the diagonal tile; tiles above it are skipped.
+//
+// TMEM columns: S_0 [0,128) S_1 [128,256) O_0, O_1 (DV each) from 256,
+// D_0, D_1 (16 each) after them; 512 columns are allocated.
+//
+// Every wait is bounded (sm100.cuh): a wait that runs out records
+// KATA_ERR_TIMEOUT, the CTA drains its own TMA copies and MMAs, frees TMEM
+// and exits.
+#include <cuda.h>
+
+#include "kata_internal.h"
+#include "sm100.cuh"
+
+namespace kata {
+namespace {
+
+using namespace sm100;
+
+constexpr int kBM = 128;       // query rows per tile
+constexpr int kBN = 128;       // keys per tile
+constexpr int kNQ = 2;         // query tiles per CTA
+constexpr int kStages = 4;     // K/V ring depth
+constexpr int kThreads = 320;  // 10 warps
+constexpr uint32_t kTmemCols = 512;
+
+template <int p, int DV>
+struct FlashCfg {
+  static constexpr int kQKBytes = kBM * p * 2;          // one Q or K tile
+  static constexpr int kVBytes = kBN * DV * 2;          // one V tile
+  static constexpr int kOnesBytes = 512;
+  // K-major Q/K rows are p*2 bytes: 32 B (p=16, 32B swizzle) or 64 B (p=32)
+  static constexpr Swizzle kQKSw = (p == 16) ? kSw32 : kSw64;
+  static constexpr uint32_t kQKSbo = 8 * p * 2;         // 8-row group stride
+  // MN-major V rows are DV*2 bytes: 128 B (DV=64, 128B swizzle) or 32 B
+  static constexpr Swizzle kVSw = (DV == 64) ? kSw128 : kSw32;
+  static constexpr uint32_t kVSbo = 8 * DV * 2;         // 8-key group stride
+  static constexpr uint32_t kVKStep = 16 * DV * 2;      // 16 keys
+  // TMEM column map
+  static constexpr uint32_t colS(int i) { return (uint32_t)i * 128; }
+  static constexpr uint32_t colO(int i) { return 256u + (uint32_t)i * DV; }
+  static constexpr uint32_t colD(int i) { return 256u + 2u * DV + (uint32_t)i * 16; }
+  // shared memory map (offsets from a 1024-aligned base)
+  static constexpr int offQ = 0;
+  static constexpr int offK = offQ + kNQ * kQKBytes;
+  static constexpr int offV = ((offK + kStages * kQKBytes) + 1023) / 1024 * 1024;
+  static constexpr int offOnes = offV + kStages * kVBytes;
+  static constexpr int offBar = offOnes + kOnesBytes;
+  static constexpr int kNumBars = 1 + 2 * kStages + 3 * kNQ + 1;
+  static constexpr int offMisc = offBar + kNumBars * 8;
+  static constexpr int kSmemBytes = offMisc + 16 + 1024;  // + alignment slack
+};
+
+template <int p, int DV>
+__global__ void __launch_bounds__(kThreads, 1)
+    flash_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ o, int T, WaitCtl wc) {
+  using Cfg = FlashCfg<p, DV>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::offBar);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = bars + 1;
+  uint64_t* kv_empty = kv_full + kStages;
+  uint64_t* s_full = kv_empty + kStages;
+  uint64_t* p_full = s_full + kNQ;
+  uint64_t* o_full = p_full + kNQ;
+  uint64_t* mma_done = o_full + kNQ;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Cfg::offMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::offMisc + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.y;
+  const int ct = gridDim.x - 1 - blockIdx.x;  // heaviest CTAs first
+  const int n_tiles = (T + kBM - 1) / kBM;
+  int nkv[kNQ];
+#pragma unroll
+  for (int i = 0; i < kNQ; ++i) {
+    const int qtile = ct * kNQ + i;
+    nkv[i] = qtile < n_tiles ? qtile + 1 : 0;
+  }
+  const int nkv_max = nkv[0] > nkv[1] ? nkv[0] : nkv[1];
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(kv_full + s, 1);
+      mbar_init(kv_empty + s, 1);
+    }
+    for (int i = 0; i < kNQ; ++i) {
+      mbar_init(s_full + i, 1);
+      mbar_init(p_full + i, kBM);
+      mbar_init(o_full + i, 1);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  {  // block of bf16 ones for the denominator MMA
+    uint32_t* ones = reinterpret_cast<uint32_t*>(smem + Cfg::offOnes);
+    for (int x = threadIdx.x; x < Cfg::kOnesBytes / 4; x += kThreads) ones[x] = 0x3F803F80u;
+    fence_proxy_async_smem();
+  }
+  if (warp == 1) tmem_alloc(tmem_holder, kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const WaitEnv env{wc.status, abort_flag, wc.limit};
+
+  if (warp == 0) {
+    // ------------------------------------------------------------- producer
+    if (lane == 0) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      mbar_arrive_expect_tx(q_full, kNQ * Cfg::kQKBytes);
+      for (int i = 0; i < kNQ; ++i)
+        tma_load_3d(smem + Cfg::offQ + i * Cfg::kQKBytes, &tm_q, q_full, 0, (ct * kNQ + i) * kBM, bh);
+      int issued = 0;
+      for (int j = 0; j < nkv_max; ++j) {
+        const int st = j % kStages;
+        if (!mbar_wait(kv_empty + st, ((j / kStages) & 1) ^ 1, env)) break;
+        mbar_arrive_expect_tx(kv_full + st, Cfg::kQKBytes + Cfg::kVBytes);
+        tma_load_3d(smem + Cfg::offK + st * Cfg::kQKBytes, &tm_k, kv_full + st, 0, j * kBN, bh);
+        tma_load_3d(smem + Cfg::offV + st * Cfg::kVBytes, &tm_v, kv_full + st, 0, j * kBN, bh);
+        ++issued;
+      }
+      // drain: every copy this CTA started must land before it exits
+      mbar_wait_drain(q_full, 0, wc.limit);
+      for (int j = issued - kStages < 0 ? 0 : issued - kStages; j < issued; ++j)
+        mbar_wait_drain(kv_full + j % kStages, (j / kStages) & 1, wc.limit);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t id_qk = idesc_bf16(kBM, kBN, false);
+      constexpr uint32_t id_pv = idesc_bf16(kBM, DV, true);
+      constexpr uint32_t id_d = idesc_bf16(kBM, 16, false);
+      const uint32_t sQ = smem_u32(smem + Cfg::offQ), sK = smem_u32(smem + Cfg::offK);
+      const uint32_t sV = smem_u32(smem + Cfg::offV), sOnes = smem_u32(smem + Cfg::offOnes);
+      const uint64_t ones_desc = smem_desc(sOnes, 256, 128, kSwNone);
+      if (mbar_wait(q_full, 0, env)) {
+        for (int j = 0; j < nkv_max; ++j) {
+          const int st = j % kStages;
+          if (!mbar_wait(kv_full + st, (j / kStages) & 1, env)) break;
+          tc_fence_after();
+          for (int i = 0; i < kNQ; ++i) {
+            if (j >= nkv[i]) continue;
+#pragma unroll
+            for (int ks = 0; ks < p / 16; ++ks) {
+              const uint64_t a = smem_desc(sQ + i * Cfg::kQKBytes + ks * 32, 16, Cfg::kQKSbo, Cfg::kQKSw);
+              const uint64_t b = smem_desc(sK + st * Cfg::kQKBytes + ks * 32, 16, Cfg::kQKSbo, Cfg::kQKSw);
+              mma_ss(tmem + Cfg::colS(i), a, b, id_qk, ks > 0);
+            }
+            mma_commit(s_full + i);
+          }
+          bool ok = true;
+          for (int i = 0; i < kNQ && ok; ++i) {
+            if (j >= nkv[i]) continue;
+            if (!mbar_wait(p_full + i, j & 1, env)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < kBN / 16; ++ks) {
+              const uint32_t a = tmem + Cfg::colS(i) + ks * 8;  // 16 bf16 weights = 8 columns
+              const uint64_t b = smem_desc(sV + st * Cfg::kVBytes + ks * Cfg::kVKStep, Cfg::kVBytes, Cfg::kVSbo,
+                                           Cfg::kVSw);
+              const uint32_t acc = (j > 0 || ks > 0) ? 1u : 0u;
+              mma_ts(tmem + Cfg::colO(i), a, b, id_pv, acc);
+              mma_ts(tmem + Cfg::colD(i), a, ones_desc, id_d, acc);
+            }
+            if (j == nkv[i] - 1) mma_commit(o_full + i);
+          }
+          if (!ok) break;
+          mma_commit(kv_empty + st);
+        }
+      }
+      mma_commit(mma_done);
+      mbar_wait_drain(mma_done, 0, wc.limit);
+    }
+  } else {
+    // ------------------------------------------------------------- weights + epilogue
+    const int i = (warp - 2) / 4;          // query tile of this warpgroup
+    const int quarter = warp % 4;          // TMEM lane quarter this warp may access
+    const int m = quarter * 32 + lane;     // row within the tile
+    const int qtile = ct * kNQ + i;
+    const int t = qtile * kBM + m;
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    bool ok = nkv[i] > 0;
+    for (int j = 0; ok && j < nkv[i]; ++j) {
+      if (!mbar_wait(s_full + i, j & 1, env)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const bool diag = (j == nkv[i] - 1);
+      const uint32_t sa = lane_base + Cfg::colS(i);
+#pragma unroll
+      for (int b = 0; b < kBN / 32; ++b) {
+        uint32_t r[32];
+        tmem_ld32(sa + 32 * b, r);
+        tmem_wait_ld();
+        uint32_t w[16];
+#pragma unroll
+        for (int x = 0; x < 16; ++x) {
+          const float s0 = __uint_as_float(r[2 * x]), s1 = __uint_as_float(r[2 * x + 1]);
+          float w0 = s0 * s0, w1 = s1 * s1;
+          if (diag) {
+            const int c = 32 * b + 2 * x;
+            if (c > m) w0 = 0.f;
+            if (c + 1 > m) w1 = 0.f;
+          }
+          w[x] = pack_bf16x2(w0, w1);
+        }
+        tmem_st16(sa + 16 * b, w);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(p_full + i);
+    }
+    if (ok && mbar_wait(o_full + i, 0, env)) {
+      tc_fence_after();
+      uint32_t dbits;
+      tmem_ld1(lane_base + Cfg::colD(i), dbits);
+      float ov[DV];
+      if constexpr (DV == 64) {
+        uint32_t r0[32], r1[32];
+        tmem_ld32(lane_base + Cfg::colO(i), r0);
+        tmem_ld32(lane_base + Cfg::colO(i) + 32, r1);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          ov[e] = __uint_as_float(r0[e]);
+          ov[32 + e] = __uint_as_float(r1[e]);
+        }
+      } else {
+        uint32_t r0[16];
+        tmem_ld16(lane_base + Cfg::colO(i), r0);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) ov[e] = __uint_as_float(r0[e]);
+      }
+      const float D = __uint_as_float(dbits);
+      const float inv = D > 0.f ? 1.f / D : 0.f;
+      if (t < T) {
+        uint4* dst = reinterpret_cast<uint4*>(o + ((size_t)bh * T + t) * DV);
+#pragma unroll
+        for (int e = 0; e < DV / 8; ++e) {
+          uint4 u;
+          u.x = pack_bf16x2(ov[8 * e + 0] * inv, ov[8 * e + 1] * inv);
+          u.y = pack_bf16x2(ov[8 * e + 2] * inv, ov[8 * e + 3] * inv);
+          u.z = pack_bf16x2(ov[8 * e + 4] * inv, ov[8 * e + 5] * inv);
+          u.w = pack_bf16x2(ov[8 * e + 6] * inv, ov[8 * e + 7] * inv);
+          dst[e] = u;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+}  // namespace
+
+EncodeTiledFn get_encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 3-D bf16 tensor map over [BH][T][inner] with a box of {inner, rows, 1}.
+bool make_tmap_bf16(CUtensorMap* map, const void* base, int inner, int T, int BH, int rows) {
+  EncodeTiledFn enc = get_encode_tiled();
+  if (!enc) return false;
+  const int row_bytes = inner * 2;
+  CUtensorMapSwizzle sw = row_bytes == 32    ? CU_TENSOR_MAP_SWIZZLE_32B
+                          : row_bytes == 64  ? CU_TENSOR_MAP_SWIZZLE_64B
+                          : row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                             : CU_TENSOR_MAP_SWIZZLE_NONE;
+  cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)T, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)row_bytes, (cuuint64_t)row_bytes * (cuuint64_t)T};
+  cuuint32_t box[3] = {(cuuint32_t)inner, (cuuint32_t)rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int p, int DV>
+static cudaError_t launch_flash_t(const void* q, const void* k, const void* v, void* o, int BH, int T,
+                                  const WaitCtl& wc, cudaStream_t st) {
+  using Cfg = FlashCfg<p, DV>;
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap_bf16(&tq, q, p, T, BH, kBM) || !make_tmap_bf16(&tk, k, p, T, BH, kBN) ||
+      !make_tmap_bf16(&tv, v, DV, T, BH, kBN))
+    return cudaErrorInvalidValue;
+  auto kern = flash_fwd_kernel<p, DV>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  dim3 grid((T + kBM * kNQ - 1) / (kBM * kNQ), BH);
+  kern<<<grid, kThreads, Cfg::kSmemBytes, st>>>(tq, tk, tv, static_cast<__nv_bfloat16*>(o), T, wc);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_flash_sm100(const void* q, const void* k, const void* v, void* o, int BH, int T, int p, int dv,
+                               const WaitCtl& wc, cudaStream_t st) {
+  if (p == 16 && dv == 64) return launch_flash_t<16, 64>(q, k, v, o, BH, T, wc, st);
+  if (p == 16 && dv == 16) return launch_flash_t<16, 16>(q, k, v, o, BH, T, wc, st);
+  if (p == 32 && dv == 64) return launch_flash_t<32, 64>(q, k, v, o, BH, T, wc, st);
+  if (p == 32 && dv == 16) return launch_flash_t<32, 16>(q, k, v, o, BH, T, wc, st);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace kata

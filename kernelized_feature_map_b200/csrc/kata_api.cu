@@ -1,0 +1,189 @@
+// kata_api.cu -- the C ABI of libkata (declared in include/kata.h).
+//
+// Validates every argument before anything is launched, plans the chunked
+// path, and enqueues the kernels on the caller's stream.  Owns the
+// device-side status word that kernels use to report a bounded wait that ran
+// out.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "kata_internal.h"
+
+#define KATA_API extern "C" __attribute__((visibility("default")))
+
+namespace kata {
+
+__device__ int g_kata_status;
+
+static std::atomic<long long> g_wait_limit{-1};
+constexpr long long kDefaultWaitLimit = 1ll << 31;  // SM cycles (about a second)
+
+long long wait_limit() {
+  long long v = g_wait_limit.load();
+  return v < 0 ? kDefaultWaitLimit : v;
+}
+
+static int* status_word() {
+  static std::mutex mu;
+  static int* addr[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_kata_status) != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<int*>(p);
+  }
+  return addr[dev];
+}
+
+WaitCtl wait_ctl() { return WaitCtl{status_word(), wait_limit()}; }
+
+// Super-chunk length: the largest of 4096 ... 128 tokens that still gives at
+// least kTargetUnits independent (b,h, super-chunk) work units, so that the
+// state records stay few (each costs a P x ld fp32 round trip through HBM)
+// while every SM gets work.  A pure function of the sizes, so that the
+// workspace query and the call agree.
+constexpr int kTargetUnits = 2 * 148;
+
+ChunkPlan make_chunk_plan(int B, int H, int T, int p, int dv, int C, int /*num_sms*/) {
+  ChunkPlan pl{};
+  pl.BH = B * H;
+  pl.T = T;
+  pl.p = p;
+  pl.P = p * p;
+  pl.dv = dv;
+  pl.ld = dv + 16;
+  pl.C = C;
+  pl.Ls = 128;
+  const int cands[] = {4096, 2048, 1024, 512, 256, 128};
+  for (int c : cands) {
+    const long long units = (long long)pl.BH * ((T + c - 1) / c);
+    if (units >= kTargetUnits) {
+      pl.Ls = c;
+      break;
+    }
+  }
+  if (pl.Ls < C) pl.Ls = C;
+  pl.G = T > 0 ? (T + pl.Ls - 1) / pl.Ls : 0;
+  pl.record_floats = (size_t)pl.P * pl.ld;
+  pl.workspace_bytes = (size_t)pl.BH * pl.G * pl.record_floats * sizeof(float);
+  return pl;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static kata_status_t check_common(int B, int H, int T, int p, int dv, kata_dtype_t dt) {
+  if (B < 1 || H < 1 || T < 0) return KATA_ERR_INVALID_ARG;
+  if (dt != KATA_F32 && dt != KATA_BF16) return KATA_ERR_INVALID_ARG;
+  if (!((p == 16 || p == 32) && (dv == 16 || dv == 64))) return KATA_ERR_UNSUPPORTED;
+  // per-(b,h) offsets are kept in 32-bit integers inside the kernels
+  if ((long long)T * (dv > p ? dv : p) >= (1ll << 31)) return KATA_ERR_UNSUPPORTED;
+  if ((long long)B * H >= (1ll << 31) / 1) return KATA_ERR_UNSUPPORTED;
+  return KATA_OK;
+}
+
+static kata_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? KATA_OK : KATA_ERR_CUDA; }
+
+}  // namespace kata
+
+using namespace kata;
+
+KATA_API int kata_abi_version(void) { return KATA_ABI_VERSION; }
+
+KATA_API const char* kata_status_string(kata_status_t s) {
+  switch (s) {
+    case KATA_OK: return "KATA_OK";
+    case KATA_ERR_INVALID_ARG: return "KATA_ERR_INVALID_ARG";
+    case KATA_ERR_UNSUPPORTED: return "KATA_ERR_UNSUPPORTED";
+    case KATA_ERR_MISALIGNED: return "KATA_ERR_MISALIGNED";
+    case KATA_ERR_WORKSPACE: return "KATA_ERR_WORKSPACE";
+    case KATA_ERR_CUDA: return "KATA_ERR_CUDA";
+    case KATA_ERR_TIMEOUT: return "KATA_ERR_TIMEOUT";
+  }
+  return "KATA_ERR_UNKNOWN";
+}
+
+KATA_API void kata_set_wait_limit(long long cycles) { g_wait_limit.store(cycles < 0 ? -1 : cycles); }
+
+KATA_API kata_status_t kata_get_status(void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return KATA_ERR_CUDA;
+  int* addr = status_word();
+  if (!addr) return KATA_ERR_CUDA;
+  int h = 0;
+  if (cudaMemcpy(&h, addr, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return KATA_ERR_CUDA;
+  if (h != 0) {
+    const int zero = 0;
+    if (cudaMemcpy(addr, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return KATA_ERR_CUDA;
+  }
+  return static_cast<kata_status_t>(h);
+}
+
+KATA_API kata_status_t kata_fwd_quadratic(const void* q, const void* k, const void* v, void* o, int B, int H, int T,
+                                          int p, int dv, kata_dtype_t dtype, void* stream) {
+  kata_status_t s = check_common(B, H, T, p, dv, dtype);
+  if (s != KATA_OK) return s;
+  if (T == 0) return KATA_OK;
+  if (!q || !k || !v || !o) return KATA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return KATA_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == KATA_BF16) return from_cuda(launch_flash_sm100(q, k, v, o, B * H, T, p, dv, wait_ctl(), st));
+  return from_cuda(launch_quadratic_simt(q, k, v, o, B * H, T, p, dv, dtype, st));
+}
+
+KATA_API size_t kata_fwd_chunked_workspace_size(int B, int H, int T, int p, int dv, int C, kata_dtype_t dtype) {
+  if (check_common(B, H, T, p, dv, dtype) != KATA_OK || !(C == 64 || C == 128) || T == 0) return 0;
+  return make_chunk_plan(B, H, T, p, dv, C, 0).workspace_bytes;
+}
+
+KATA_API kata_status_t kata_fwd_chunked(const void* q, const void* k, const void* v, void* o, int B, int H, int T,
+                                        int p, int dv, int C, kata_dtype_t dtype, const float* S0, const float* z0,
+                                        float* S_out, float* z_out, void* workspace, size_t workspace_bytes,
+                                        void* stream) {
+  kata_status_t s = check_common(B, H, T, p, dv, dtype);
+  if (s != KATA_OK) return s;
+  if (!(C == 64 || C == 128)) return KATA_ERR_UNSUPPORTED;
+  if ((S0 == nullptr) != (z0 == nullptr)) return KATA_ERR_INVALID_ARG;
+  if ((S_out == nullptr) != (z_out == nullptr)) return KATA_ERR_INVALID_ARG;
+  for (const void* ptr : {(const void*)S0, (const void*)z0, (const void*)S_out, (const void*)z_out})
+    if (ptr && !aligned16(ptr)) return KATA_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t P = (size_t)p * p, BH = (size_t)B * H;
+  if (T == 0) {
+    if (!S_out) return KATA_OK;
+    if (S0) {
+      cudaError_t e = cudaMemcpyAsync(S_out, S0, BH * P * dv * sizeof(float), cudaMemcpyDeviceToDevice, st);
+      if (e == cudaSuccess) e = cudaMemcpyAsync(z_out, z0, BH * P * sizeof(float), cudaMemcpyDeviceToDevice, st);
+      return from_cuda(e);
+    }
+    cudaError_t e = cudaMemsetAsync(S_out, 0, BH * P * dv * sizeof(float), st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(z_out, 0, BH * P * sizeof(float), st);
+    return from_cuda(e);
+  }
+  if (!q || !k || !v || !o) return KATA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return KATA_ERR_MISALIGNED;
+  const ChunkPlan plan = make_chunk_plan(B, H, T, p, dv, C, 0);
+  if (!workspace || workspace_bytes < plan.workspace_bytes) return KATA_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KATA_ERR_MISALIGNED;
+  float* ws = static_cast<float*>(workspace);
+  cudaError_t e = launch_chunk_aggregate_simt(k, v, ws, plan, dtype, st);
+  if (e == cudaSuccess) e = launch_state_scan(ws, plan, S0, z0, S_out, z_out, st);
+  if (e == cudaSuccess) e = launch_chunk_readout_simt(q, k, v, o, ws, plan, dtype, st);
+  return from_cuda(e);
+}
+
+KATA_API kata_status_t kata_decode_step(const void* q, const void* k, const void* v, void* o, float* S, float* z,
+                                        int B, int H, int p, int dv, kata_dtype_t dtype, void* stream) {
+  kata_status_t s = check_common(B, H, 1, p, dv, dtype);
+  if (s != KATA_OK) return s;
+  if (!q || !k || !v || !o || !S || !z) return KATA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(S) || !aligned16(z))
+    return KATA_ERR_MISALIGNED;
+  return from_cuda(launch_decode(q, k, v, o, S, z, B * H, p, dv, dtype, static_cast<cudaStream_t>(stream)));
+}

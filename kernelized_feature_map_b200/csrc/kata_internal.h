@@ -1,0 +1,59 @@
+// kata_internal.h -- host-side interface between the C ABI (kata_api.cu) and
+// the kernel translation units.  Not part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/kata.h"
+
+namespace kata {
+
+// Everything a kernel needs to report a bounded wait that ran out.
+struct WaitCtl {
+  int* status;           // device address of the library's status word
+  long long limit;       // cycles before a wait gives up
+};
+
+// Chunked-path plan: how the sequence is grouped for the state scan.
+struct ChunkPlan {
+  int BH;        // B * H
+  int T;
+  int p, P;      // psi input width, P = p * p
+  int dv;
+  int ld;        // row stride (floats) of a state record: dv + 16
+  int C;         // chunk length requested by the caller
+  int Ls;        // super-chunk length (tokens per state record), multiple of 128 and C
+  int G;         // number of super-chunks per (b,h): ceil(T / Ls)
+  size_t record_floats;  // P * ld
+  size_t workspace_bytes;
+};
+
+ChunkPlan make_chunk_plan(int B, int H, int T, int p, int dv, int C, int num_sms);
+
+// decode.cu
+cudaError_t launch_decode(const void* q, const void* k, const void* v, void* o, float* S, float* z,
+                          int BH, int p, int dv, kata_dtype_t dt, cudaStream_t st);
+
+// scan.cu -- exclusive prefix over the G records of every (b,h), in place,
+// plus S0 and the final state.
+cudaError_t launch_state_scan(float* ws, const ChunkPlan& plan, const float* S0, const float* z0,
+                              float* S_out, float* z_out, cudaStream_t st);
+
+// simt.cu -- CUDA-core kernels (fp32 inputs; exact fp32 arithmetic).
+cudaError_t launch_quadratic_simt(const void* q, const void* k, const void* v, void* o, int BH, int T,
+                                  int p, int dv, kata_dtype_t dt, cudaStream_t st);
+cudaError_t launch_chunk_aggregate_simt(const void* k, const void* v, float* ws, const ChunkPlan& plan,
+                                        kata_dtype_t dt, cudaStream_t st);
+cudaError_t launch_chunk_readout_simt(const void* q, const void* k, const void* v, void* o, float* ws,
+                                      const ChunkPlan& plan, kata_dtype_t dt, cudaStream_t st);
+
+// flash_sm100.cu -- tcgen05 flash-style forward (bf16 inputs).
+cudaError_t launch_flash_sm100(const void* q, const void* k, const void* v, void* o, int BH, int T, int p, int dv,
+                               const WaitCtl& wc, cudaStream_t st);
+
+// Current bound on in-kernel waits and the status word (kata_api.cu).
+WaitCtl wait_ctl();
+
+}  // namespace kata

@@ -1,0 +1,106 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every entry point include/kata.h declares, and rejects bad arguments before
+anything is launched."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from kernelized_feature_map_b200 import _abi, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names.update(re.findall(r"\b(kata_\w+)\s*\(", text))
+    return sorted(names)
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return _abi.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    declared = _declared_functions()
+    assert len(declared) >= 8
+    for name in declared:
+        assert hasattr(L, name), name
+        assert name in _abi.SIGNATURES, "binding lacks " + name
+
+
+def test_only_abi_symbols_are_exported():
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", _abi.LIB_PATH], capture_output=True, text=True).stdout
+    exported = {l.split()[-1] for l in out.splitlines() if " T " in l}
+    assert exported == set(_declared_functions())
+
+
+def test_status_strings_and_version(L):
+    assert _abi.kata_abi_version() == 10000
+    for code, name in [(0, "KATA_OK"), (2, "KATA_ERR_UNSUPPORTED"), (6, "KATA_ERR_TIMEOUT")]:
+        assert _abi.status_string(code) == name
+    assert _abi.status_string(99) == "KATA_ERR_UNKNOWN"
+
+
+def test_workspace_size_query(L):
+    ws = _abi.kata_fwd_chunked_workspace_size
+    # zero for T == 0 and for unsupported shapes
+    assert ws(1, 1, 0, 16, 64, 64) == 0
+    assert ws(1, 1, 100, 8, 64, 64) == 0
+    assert ws(1, 1, 100, 16, 64, 96) == 0
+    # one fp32 record of P x (dv + 16) per (b,h) per super-chunk
+    n = ws(1, 1, 256, 16, 16, 64, dtype=None)
+    assert n > 0 and n % (256 * 32 * 4) == 0
+    assert ws(8, 16, 2048, 16, 64, 64) % (256 * 80 * 4) == 0
+    # grows with T (more super-chunks) and never shrinks
+    sizes = [ws(1, 16, t, 16, 64, 64) for t in (1024, 4096, 16384, 65536, 131072)]
+    assert sizes == sorted(sizes)
+
+
+VP = ctypes.c_void_p
+
+
+def _fake(addr):
+    return VP(addr)
+
+
+def test_argument_errors_before_launch(L):
+    a, b, c, d = _fake(0x10000), _fake(0x20000), _fake(0x30000), _fake(0x40000)
+    st = VP(0)
+    f = L.kata_fwd_quadratic
+    assert f(a, b, c, d, 1, 1, 16, 8, 64, 1, st) == _abi.KATA_ERR_UNSUPPORTED      # p
+    assert f(a, b, c, d, 1, 1, 16, 16, 32, 1, st) == _abi.KATA_ERR_UNSUPPORTED     # dv
+    assert f(a, b, c, d, 0, 1, 16, 16, 64, 1, st) == _abi.KATA_ERR_INVALID_ARG     # B
+    assert f(a, b, c, d, 1, 1, -1, 16, 64, 1, st) == _abi.KATA_ERR_INVALID_ARG     # T
+    assert f(a, b, c, d, 1, 1, 16, 16, 64, 7, st) == _abi.KATA_ERR_INVALID_ARG     # dtype
+    assert f(None, b, c, d, 1, 1, 16, 16, 64, 1, st) == _abi.KATA_ERR_INVALID_ARG  # null
+    assert f(_fake(0x10008), b, c, d, 1, 1, 16, 16, 64, 1, st) == _abi.KATA_ERR_MISALIGNED
+    assert f(a, b, c, d, 1, 1, 0, 16, 64, 1, st) == _abi.KATA_OK                   # T = 0: no-op
+    g = L.kata_fwd_chunked
+    ws = _fake(0x50000)
+    assert g(a, b, c, d, 1, 1, 16, 16, 64, 96, 1, None, None, None, None, ws, 1 << 20, st) == _abi.KATA_ERR_UNSUPPORTED
+    assert g(a, b, c, d, 1, 1, 16, 16, 64, 64, 1, _fake(0x60000), None, None, None, ws, 1 << 20, st) == _abi.KATA_ERR_INVALID_ARG
+    assert g(a, b, c, d, 1, 1, 16, 16, 64, 64, 1, None, None, None, _fake(0x60000), ws, 1 << 20, st) == _abi.KATA_ERR_INVALID_ARG
+    assert g(a, b, c, d, 1, 1, 16, 16, 64, 64, 1, None, None, None, None, ws, 16, st) == _abi.KATA_ERR_WORKSPACE
+    assert g(a, b, c, d, 1, 1, 16, 16, 64, 64, 1, None, None, None, None, None, 1 << 20, st) == _abi.KATA_ERR_WORKSPACE
+    assert g(a, b, c, d, 1, 1, 16, 16, 64, 64, 1, None, None, None, None, _fake(0x50010), 1 << 20, st) == _abi.KATA_ERR_MISALIGNED
+    assert g(a, b, c, d, 1, 1, 0, 16, 64, 64, 1, None, None, None, None, None, 0, st) == _abi.KATA_OK
+    h = L.kata_decode_step
+    assert h(a, b, c, d, _fake(0x70000), None, 1, 1, 16, 64, 1, st) == _abi.KATA_ERR_INVALID_ARG
+    assert h(a, b, c, d, _fake(0x70000), _fake(0x80000), 1, 1, 24, 64, 1, st) == _abi.KATA_ERR_UNSUPPORTED
+    assert h(a, b, c, d, _fake(0x70004), _fake(0x80000), 1, 1, 16, 64, 1, st) == _abi.KATA_ERR_MISALIGNED
+
+
+def test_binding_requires_cuda_tensors():
+    import torch
+    q = torch.zeros(1, 1, 4, 16)
+    with pytest.raises(TypeError):
+        _abi.kata_fwd_quadratic(q, q, torch.zeros(1, 1, 4, 64))
