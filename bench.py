@@ -1,0 +1,449 @@
+#!/usr/bin/env python
+"""Benchmark of the KATA forward hot path on B200.
+
+One step = one pass of every hot-path operation over one batch of synthetic
+input resident in HBM:
+  1. kata_fwd_quadratic  -- flash-style O(T^2) forward (tcgen05 / TMEM),
+  2. kata_fwd_chunked    -- exact O(T) chunked-state forward (state build,
+                            associative scan, readout), returning the final
+                            state,
+  3. kata_decode_step    -- one recurrent decode token per sequence, continuing
+                            from that final state.
+Tokens per step = B*T (the batch's tokens; the decode token is not counted).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (launched with torchrun): the (batch, head) pairs are independent,
+so each rank runs its own batch with no collective on the data path (weak
+scaling); the step time is the max over ranks and `value` counts all ranks'
+tokens.  `--impl reference` times the fp64 CPU oracle on the host cores on a
+bounded sample of the same workload (rank 0 only).
+
+Timing: CUDA events on the launching stream around each step, after W
+warm-up steps; L2 is flushed (a 512 MiB write) between timed steps, outside
+the events.  Clocks are sampled with nvidia-smi during the timed steps.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+METRIC = "KATA-Mg fwd tokens/sec at T=2k and 131k (1 B200); % of roofline"
+UNIT = "tokens/s"
+LAUNCHES_PER_STEP = 5  # flash 1 + chunked 3 (state build, scan, readout) + decode 1
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in PEAKS_FALLBACK if k in d}, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work per launch (the per-unit figures are stated in the design doc)
+# ---------------------------------------------------------------------------
+def flash_flops(BH, T, p, dv):
+    """Causal-useful tensor flops: 2 (p + dv) per (query, key<=query) pair."""
+    return BH * T * (T + 1) * (p + dv)
+
+
+def chunked_bytes(BH, T, p, dv, elem=2):
+    """q, k, v read and o written once: (2p + 2dv) elements per token-head."""
+    return BH * T * (2 * p + 2 * dv) * elem
+
+
+def decode_bytes(BH, p, dv, elem=2):
+    """State S (P x dv fp32) and z (P fp32) read and written; q,k,v read, o written."""
+    P = p * p
+    return BH * (2 * (P * dv + P) * 4 + (2 * p + 2 * dv) * elem)
+
+
+# ---------------------------------------------------------------------------
+# clocks
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.QUERY,
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import kernelized_feature_map_b200 as K
+    from kernelized_feature_map_b200 import _abi
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    cfg = workloads.CONFIGS[args.workload]
+    B, H, T, p, dv, C = cfg["B"], cfg["H"], cfg["T"], cfg["p"], cfg["dv"], cfg["C"]
+    BH = B * H
+    # each rank draws its own batch (weak scaling: per-GPU work fixed)
+    cfg_r = dict(cfg, seed=cfg["seed"] + 1000 * rank)
+    qn, kn, vn = workloads.make_inputs(cfg_r)
+    dq, dk, dvv, dS, dz = workloads.decode_inputs(B, H, p, dv, seed=cfg["seed"] + 7 + 1000 * rank)
+    bf = torch.bfloat16
+
+    def pinned(x, dt=bf):
+        return torch.from_numpy(x).to(dt).pin_memory()
+
+    hq, hk, hv = pinned(qn), pinned(kn), pinned(vn)
+    hdq, hdk, hdv = pinned(dq), pinned(dk), pinned(dvv)
+    q, k, v = hq.to(dev), hk.to(dev), hv.to(dev)
+    qd, kd, vd = hdq.to(dev), hdk.to(dev), hdv.to(dev)
+    o_quad = torch.empty((B, H, T, dv), dtype=bf, device=dev)
+    o_chunk = torch.empty_like(o_quad)
+    o_dec = torch.empty((B, H, dv), dtype=bf, device=dev)
+    S = torch.empty((B, H, p * p, dv), dtype=torch.float32, device=dev)
+    z = torch.empty((B, H, p * p), dtype=torch.float32, device=dev)
+    ws = torch.empty(max(256, K.kata_fwd_chunked_workspace_size(B, H, T, p, dv, C, bf)), dtype=torch.uint8,
+                     device=dev)
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+
+    def step(times=None):
+        e = [ev() for _ in range(4)] if times is not None else None
+        if e: e[0].record(stream)
+        K.kata_fwd_quadratic(q, k, v, o=o_quad)
+        if e: e[1].record(stream)
+        K.kata_fwd_chunked(q, k, v, C=C, o=o_chunk, workspace=ws, S_out=S, z_out=z, return_state=True)
+        if e: e[2].record(stream)
+        K.kata_decode_step(qd, kd, vd, S, z, o=o_dec)
+        if e: e[3].record(stream)
+        if times is not None:
+            times.append(e)
+
+    for _ in range(args.warmup):
+        step()
+        flush.fill_(1)
+    torch.cuda.synchronize()
+    if K.kata_get_status() != 0:
+        raise RuntimeError("kernel reported a wait timeout during warm-up")
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    recs = []
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        for _ in range(args.steps):
+            step(recs)
+            flush.fill_(1)
+        torch.cuda.synchronize()
+    barrier()
+    per = np.array([[r[0].elapsed_time(r[1]), r[1].elapsed_time(r[2]), r[2].elapsed_time(r[3])] for r in recs])
+    step_ms = float(per.sum(axis=1).mean())
+    path_ms = per.mean(axis=0)
+
+    # end to end through the public API with host buffers: H2D of the step's
+    # inputs from pinned memory, the three calls, D2H of the three outputs
+    ho_quad = torch.empty(o_quad.shape, dtype=bf).pin_memory()
+    ho_chunk = torch.empty(o_chunk.shape, dtype=bf).pin_memory()
+    ho_dec = torch.empty(o_dec.shape, dtype=bf).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdq, hdk, hdv))
+    d2h = sum(t.numel() * t.element_size() for t in (ho_quad, ho_chunk, ho_dec))
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True); k.copy_(hk, non_blocking=True); v.copy_(hv, non_blocking=True)
+        qd.copy_(hdq, non_blocking=True); kd.copy_(hdk, non_blocking=True); vd.copy_(hdv, non_blocking=True)
+        step()
+        ho_quad.copy_(o_quad, non_blocking=True); ho_chunk.copy_(o_chunk, non_blocking=True)
+        ho_dec.copy_(o_dec, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    e2e_ms = []
+    for _ in range(max(3, args.steps // 2)):
+        a, b = ev(), ev()
+        flush.fill_(1)
+        a.record(stream)
+        e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms.append(a.elapsed_time(b))
+    e2e_ms = float(np.mean(e2e_ms))
+
+    # long context: chunked (and quadratic) at T = 131072
+    long = None
+    if args.long and world == 1:
+        long = run_long(args, K, torch, dev, stream, flush)
+
+    status = K.kata_get_status()
+    return dict(step_ms=step_ms, path_ms=path_ms.tolist(), e2e_ms=e2e_ms, h2d=h2d, d2h=d2h,
+                clocks=clk.summary(), long=long, status=status, tokens=B * T, BH=BH, T=T, p=p, dv=dv, C=C)
+
+
+def run_long(args, K, torch, dev, stream, flush):
+    cfg = workloads.CONFIGS["long_ctx131k"]
+    B, H, T, p, dv = cfg["B"], cfg["H"], cfg["T"], cfg["p"], cfg["dv"]
+    qn, kn, vn = workloads.make_inputs(cfg)
+    bf = torch.bfloat16
+    q = torch.from_numpy(qn).to(dev, bf)
+    k = torch.from_numpy(kn).to(dev, bf)
+    v = torch.from_numpy(vn).to(dev, bf)
+    o = torch.empty((B, H, T, dv), dtype=bf, device=dev)
+    out = {}
+    for C in (64, 128):
+        ws = torch.empty(max(256, K.kata_fwd_chunked_workspace_size(B, H, T, p, dv, C, bf)), dtype=torch.uint8,
+                         device=dev)
+        ms = []
+        for i in range(3 + args.long_steps):
+            flush.fill_(1)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            K.kata_fwd_chunked(q, k, v, C=C, o=o, workspace=ws)
+            b.record(stream)
+            torch.cuda.synchronize()
+            if i >= 3:
+                ms.append(a.elapsed_time(b))
+        out["chunked_C%d_ms" % C] = float(np.mean(ms))
+    ms = []
+    for i in range(2 + max(1, args.long_steps // 4)):
+        flush.fill_(1)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        K.kata_fwd_quadratic(q, k, v, o=o)
+        b.record(stream)
+        torch.cuda.synchronize()
+        if i >= 2:
+            ms.append(a.elapsed_time(b))
+    out["quadratic_ms"] = float(np.mean(ms))
+    out.update(B=B, H=H, T=T, p=p, dv=dv)
+    return out
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the fp64 CPU oracle on the host cores
+# ---------------------------------------------------------------------------
+def time_oracle(cfg, budget_s=15.0):
+    """Oracle (psi recurrence, all host threads) on whole (b,h) sequences of the
+    workload until about budget_s of CPU time; returns tokens/s and the sample."""
+    import oracle
+    B, H, T, p, dv = cfg["B"], cfg["H"], cfg["T"], cfg["p"], cfg["dv"]
+    threads = oracle.default_threads()
+    q, k, v = workloads.make_inputs(dict(cfg, B=1))
+    # probe one head to size the sample
+    t0 = time.perf_counter()
+    oracle.recurrent(q[:, :1], k[:, :1], v[:, :1], nthreads=1)
+    one = max(time.perf_counter() - t0, 1e-3)
+    n_heads = int(max(1, min(B * H, budget_s / one * threads * 0.8)))
+    n_heads = max(threads, (n_heads // threads) * threads) if n_heads >= threads else n_heads
+    reps = (n_heads + H - 1) // H
+    qs = np.concatenate([q] * reps, axis=0).reshape(-1, 1, T, p)[:n_heads]
+    ks = np.concatenate([k] * reps, axis=0).reshape(-1, 1, T, p)[:n_heads]
+    vs = np.concatenate([v] * reps, axis=0).reshape(-1, 1, T, dv)[:n_heads]
+    t0 = time.perf_counter()
+    oracle.recurrent(qs, ks, vs, nthreads=0)
+    dt = time.perf_counter() - t0
+    tokens = n_heads * T / H  # token-heads -> tokens of an H-head batch
+    return dict(value=tokens / dt, cores=threads, seconds=dt,
+                sample="oracle psi recurrence (fp64) over %d whole (b,h) sequences of T=%d" % (n_heads, T))
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    cfg = workloads.CONFIGS[args.workload]
+    vals = []
+    for _ in range(args.warmup):
+        time_oracle(cfg, budget_s=2.0)
+    for _ in range(args.steps):
+        vals.append(time_oracle(cfg, budget_s=args.ref_budget))
+    value = float(np.mean([x["value"] for x in vals]))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": float(np.mean([x["seconds"] for x in vals]) * 1e3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(cfg, world),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": vals[0]["cores"], "kind": "oracle",
+                         "sample": vals[0]["sample"]},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_dict(cfg, world):
+    return {"workload": "%s: B=%d H=%d T=%d p=%d dv=%d C=%d bf16" % (
+        "340M-layer shape" if cfg["T"] == 2048 else cfg.get("kind", ""), cfg["B"], cfg["H"], cfg["T"], cfg["p"],
+        cfg["dv"], cfg["C"]),
+        "B": cfg["B"], "H": cfg["H"], "T": cfg["T"], "p": cfg["p"], "dv": cfg["dv"], "C": cfg["C"],
+        "step": "kata_fwd_quadratic + kata_fwd_chunked(final state) + kata_decode_step",
+        "l2": "flushed between timed steps (512 MiB write outside the timed events)",
+        "parallelism": "independent (b,h) batches per rank, no collective" if world > 1 else "1 GPU"}
+
+
+def main():
+    ap = argparse.ArgumentParser(description="KATA forward hot-path benchmark")
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="layer340m_ctx2k", choices=sorted(workloads.CONFIGS))
+    ap.add_argument("--long", type=int, default=1, help="also time the T=131072 workload (1 GPU)")
+    ap.add_argument("--long-steps", type=int, default=8)
+    ap.add_argument("--cpu-baseline", type=int, default=1)
+    ap.add_argument("--ref-budget", type=float, default=15.0, help="seconds of oracle work per reference step")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        if args.impl == "ours":
+            torch.cuda.set_device(local_rank)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local_rank))
+        else:
+            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=600))
+
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+            return
+        res = run_ours(args, rank, world, local_rank)
+        step_ms = res["step_ms"]
+        e2e_ms = res["e2e_ms"]
+        if world > 1:
+            import torch
+            import torch.distributed as dist
+            t = torch.tensor([step_ms, e2e_ms], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            step_ms, e2e_ms = t.tolist()
+        if rank != 0:
+            return
+        report(args, res, step_ms, e2e_ms, world)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+def report(args, res, step_ms, e2e_ms, world):
+    peaks, peak_src = load_peaks()
+    cfg = workloads.CONFIGS[args.workload]
+    BH, T, p, dv = res["BH"], res["T"], res["p"], res["dv"]
+    tokens_all = res["tokens"] * world
+    value = tokens_all / (step_ms * 1e-3)
+    quad_ms, chunk_ms, dec_ms = res["path_ms"]
+    fl = flash_flops(BH, T, p, dv)
+    achieved = fl / (quad_ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(cfg, world),
+        "paths": {
+            "quadratic": {"ms": quad_ms, "tokens_per_s": res["tokens"] / (quad_ms * 1e-3)},
+            "chunked": {"ms": chunk_ms, "tokens_per_s": res["tokens"] / (chunk_ms * 1e-3),
+                        "hbm_frac": chunked_bytes(BH, T, p, dv) / (chunk_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+            "decode": {"ms": dec_ms, "tokens_per_s": (BH / cfg["H"]) / (dec_ms * 1e-3),
+                       "hbm_frac": decode_bytes(BH, p, dv) / (dec_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+        },
+        "roofline": {"kernel": "flash_fwd_kernel (kata_fwd_quadratic)", "bound": "tensor", "achieved": achieved,
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                     "traffic": None, "peak_source": peak_src + " (bf16 burst)",
+                     "algorithmic": "%.4g causal-useful flops per launch" % fl},
+        "e2e": {"value": tokens_all / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": res["h2d"],
+                "d2h_bytes_per_step": res["d2h"]},
+        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "clocks": res["clocks"],
+        "kernel_status": res["status"],
+    }
+    if res["long"]:
+        lg = res["long"]
+        lb = chunked_bytes(lg["B"] * lg["H"], lg["T"], lg["p"], lg["dv"])
+        ltok = lg["B"] * lg["T"]
+        lf = flash_flops(lg["B"] * lg["H"], lg["T"], lg["p"], lg["dv"])
+        line["long_ctx"] = {
+            "workload": "B=%d H=%d T=%d p=%d dv=%d bf16" % (lg["B"], lg["H"], lg["T"], lg["p"], lg["dv"]),
+            "chunked_C64": {"ms": lg["chunked_C64_ms"], "tokens_per_s": ltok / (lg["chunked_C64_ms"] * 1e-3),
+                            "hbm_frac": lb / (lg["chunked_C64_ms"] * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+            "chunked_C128": {"ms": lg["chunked_C128_ms"], "tokens_per_s": ltok / (lg["chunked_C128_ms"] * 1e-3),
+                             "hbm_frac": lb / (lg["chunked_C128_ms"] * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+            "quadratic": {"ms": lg["quadratic_ms"], "tokens_per_s": ltok / (lg["quadratic_ms"] * 1e-3),
+                          "tensor_frac": lf / (lg["quadratic_ms"] * 1e-3) / 1e12 / peaks["bf16_tflops"]},
+        }
+    if args.cpu_baseline and world == 1:
+        cb = time_oracle(cfg)
+        line["cpu_baseline"] = {"value": cb["value"], "unit": UNIT, "cores": cb["cores"], "kind": "oracle",
+                                "sample": cb["sample"]}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()
