@@ -155,9 +155,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t id_qk = idesc_bf16(kBM, kBN, false);
-      constexpr uint32_t id_pv = idesc_bf16(kBM, DV, true);
-      constexpr uint32_t id_d = idesc_bf16(kBM, 16, false);
+      constexpr uint32_t id_qk = idesc_bf16(kBM, kBN, false, false);
+      constexpr uint32_t id_pv = idesc_bf16(kBM, DV, false, true);
+      constexpr uint32_t id_d = idesc_bf16(kBM, 16, false, false);
       const uint32_t sQ = smem_u32(smem + Cfg::offQ), sK = smem_u32(smem + Cfg::offK);
       const uint32_t sV = smem_u32(smem + Cfg::offV), sOnes = smem_u32(smem + Cfg::offOnes);
       const uint64_t ones_desc = smem_desc(sOnes, 256, 128, kSwNone);

@@ -172,9 +172,16 @@ KATA_API kata_status_t kata_fwd_chunked(const void* q, const void* k, const void
   if (!workspace || workspace_bytes < plan.workspace_bytes) return KATA_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KATA_ERR_MISALIGNED;
   float* ws = static_cast<float*>(workspace);
-  cudaError_t e = launch_chunk_aggregate_simt(k, v, ws, plan, dtype, st);
+  // bf16 with p = 16 runs on the tensor cores; fp32 inputs (and p = 32) run
+  // the same three steps on the CUDA cores
+  const bool tc = dtype == KATA_BF16 && p == 16;
+  const WaitCtl wc = wait_ctl();
+  cudaError_t e = tc ? launch_chunk_state_sm100(k, v, ws, plan, wc, st)
+                     : launch_chunk_aggregate_simt(k, v, ws, plan, dtype, st);
   if (e == cudaSuccess) e = launch_state_scan(ws, plan, S0, z0, S_out, z_out, st);
-  if (e == cudaSuccess) e = launch_chunk_readout_simt(q, k, v, o, ws, plan, dtype, st);
+  if (e == cudaSuccess)
+    e = tc ? launch_chunk_readout_sm100(q, k, v, o, ws, plan, wc, st)
+           : launch_chunk_readout_simt(q, k, v, o, ws, plan, dtype, st);
   return from_cuda(e);
 }
 

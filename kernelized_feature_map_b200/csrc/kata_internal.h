@@ -53,6 +53,12 @@ cudaError_t launch_chunk_readout_simt(const void* q, const void* k, const void* 
 cudaError_t launch_flash_sm100(const void* q, const void* k, const void* v, void* o, int BH, int T, int p, int dv,
                                const WaitCtl& wc, cudaStream_t st);
 
+// chunk_sm100.cu -- tcgen05 chunked-state forward (bf16 inputs, p = 16).
+cudaError_t launch_chunk_state_sm100(const void* k, const void* v, float* ws, const ChunkPlan& pl, const WaitCtl& wc,
+                                     cudaStream_t st);
+cudaError_t launch_chunk_readout_sm100(const void* q, const void* k, const void* v, void* o, const float* ws,
+                                       const ChunkPlan& pl, const WaitCtl& wc, cudaStream_t st);
+
 // Current bound on in-kernel waits and the status word (kata_api.cu).
 WaitCtl wait_ctl();
 

@@ -178,12 +178,13 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint
   return d;
 }
 
-// Instruction descriptor: D fp32, A and B bf16, A K-major, B K- or MN-major.
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major) {
+// Instruction descriptor: D fp32, A and B bf16; each operand K-major or
+// MN-major (an A operand read from TMEM must be K-major).
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major, bool b_mn_major) {
   return (1u << 4)                 // D format: f32
          | (1u << 7)               // A format: bf16
          | (1u << 10)              // B format: bf16
-         | (0u << 15)              // A K-major
+         | ((a_mn_major ? 1u : 0u) << 15)
          | ((b_mn_major ? 1u : 0u) << 16)
          | ((uint32_t)(N >> 3) << 17)
          | ((uint32_t)(M >> 4) << 24);

@@ -135,13 +135,23 @@ def test_chunked_state_in_and_out(kata, dtype):
     o_ref, S_ref, z_ref = oracle.recurrent(q, k, v, return_state=True)
     _, S1, z1 = oracle.recurrent(q[:, :, :t0], k[:, :, :t0], v[:, :, :t0], return_state=True)
     qd, kd, vd = to_dev(q, dtype), to_dev(k, dtype), to_dev(v, dtype)
+    # elementwise bound on the final state from the arithmetic: every term
+    # psi(k_t)_r v_t is rounded once to the operand type (bf16: 2^-9 relative
+    # for the psi entry, then exact products into fp32) and T terms are summed
+    # in fp32; the bound is  eps * sum_t |psi(k_t)_r| |v_t|  with
+    # eps = 2^-8 + (T + 4) 2^-24 for bf16 and (T + 4) 2^-24 for fp32.
+    _, S_abs, z_abs = oracle.recurrent(np.abs(q), np.abs(k), np.abs(v), return_state=True, need_output=False)
+    eps = (2.0 ** -8 if dtype == "bf16" else 0.0) + (T + 4) * 2.0 ** -24
+
+    def state_ok(S_dev, z_dev):
+        return (np.all(np.abs(S_dev.cpu().numpy() - S_ref) <= eps * S_abs + 1e-6)
+                and np.all(np.abs(z_dev.cpu().numpy() - z_ref) <= eps * z_abs + 1e-6))
+
     # whole sequence with final state
     o, S, z = kata.kata_fwd_chunked(qd, kd, vd, return_state=True)
     torch.cuda.synchronize()
     assert row_rel_err(to_np(o), o_ref, v) <= TOL[dtype]
-    scale = np.abs(S_ref).max()
-    assert np.abs(S.cpu().numpy() - S_ref).max() <= 1e-4 * scale
-    assert np.abs(z.cpu().numpy() - z_ref).max() <= 1e-4 * np.abs(z_ref).max()
+    assert state_ok(S, z)
     # split: first part on the device, resume from the device state
     oa, Sa, za = kata.kata_fwd_chunked(qd[:, :, :t0].contiguous(), kd[:, :, :t0].contiguous(),
                                        vd[:, :, :t0].contiguous(), return_state=True)
@@ -150,7 +160,7 @@ def test_chunked_state_in_and_out(kata, dtype):
     torch.cuda.synchronize()
     o_split = np.concatenate([to_np(oa), to_np(ob)], axis=2)
     assert row_rel_err(o_split, o_ref, v) <= TOL[dtype]
-    assert np.abs(Sb.cpu().numpy() - S_ref).max() <= 1e-4 * scale
+    assert state_ok(Sb, zb)
     # resume from the oracle's state
     o2 = kata.kata_fwd_chunked(qd[:, :, t0:].contiguous(), kd[:, :, t0:].contiguous(), vd[:, :, t0:].contiguous(),
                                S0=torch.from_numpy(S1.astype(np.float32)).cuda(),
