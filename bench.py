@@ -76,22 +76,48 @@ def decode_bytes(BH, p, dv, elem=2):
 
 
 # ---------------------------------------------------------------------------
+# ranks: independent batches, max-over-ranks timing
+# ---------------------------------------------------------------------------
+def rank_config(cfg, rank):
+    """Each rank draws its own batch of the same shape (weak scaling): the seed
+    is offset by the rank; shapes are unchanged."""
+    return dict(cfg, seed=cfg["seed"] + 1000 * rank)
+
+
+def reduce_max(values, world, device="cpu"):
+    """Element-wise max of a list of floats over all ranks (identity at world 1)."""
+    if world <= 1:
+        return list(values)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def aggregate_value(tokens_per_rank, world, step_ms):
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's step time."""
+    return tokens_per_rank * world / (step_ms * 1e-3)
+
+
+# ---------------------------------------------------------------------------
 # clocks
 # ---------------------------------------------------------------------------
 class ClockSampler:
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    QUERY = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, index):
         self.index = index
         self.proc = None
-        self.lines = []
+        self.lines = []          # (host time, line)
+        self.window = None       # (t_start, t_end) of the timed region
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.QUERY,
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", "25"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
@@ -101,7 +127,12 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.time(), line.strip()))
+
+    def wait_first_sample(self, timeout=5.0):
+        t0 = time.time()
+        while self.proc and not self.lines and time.time() - t0 < timeout:
+            time.sleep(0.01)
 
     def __exit__(self, *a):
         if self.proc:
@@ -114,7 +145,11 @@ class ClockSampler:
     def summary(self):
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
+        lo, hi = self.window if self.window else (0.0, float("inf"))
+        for ts, line in self.lines:
+            # a sample describes the interval before it was printed
+            if ts < lo or ts > hi + 0.1:
+                continue
             parts = [x.strip() for x in line.split(",")]
             if len(parts) < 9:
                 continue
@@ -144,7 +179,7 @@ def run_ours(args, rank, world, local_rank):
     B, H, T, p, dv, C = cfg["B"], cfg["H"], cfg["T"], cfg["p"], cfg["dv"], cfg["C"]
     BH = B * H
     # each rank draws its own batch (weak scaling: per-GPU work fixed)
-    cfg_r = dict(cfg, seed=cfg["seed"] + 1000 * rank)
+    cfg_r = rank_config(cfg, rank)
     qn, kn, vn = workloads.make_inputs(cfg_r)
     dq, dk, dvv, dS, dz = workloads.decode_inputs(B, H, p, dv, seed=cfg["seed"] + 7 + 1000 * rank)
     bf = torch.bfloat16
@@ -193,14 +228,18 @@ def run_ours(args, rank, world, local_rank):
             dist.barrier()
 
     recs = []
-    barrier()
-    torch.cuda.synchronize()
     with ClockSampler(local_rank) as clk:
+        clk.wait_first_sample()
+        barrier()
+        torch.cuda.synchronize()
+        t_start = time.time()
         for _ in range(args.steps):
             step(recs)
             flush.fill_(1)
         torch.cuda.synchronize()
-    barrier()
+        clk.window = (t_start, time.time())
+        barrier()
+        time.sleep(0.15)
     per = np.array([[r[0].elapsed_time(r[1]), r[1].elapsed_time(r[2]), r[2].elapsed_time(r[3])] for r in recs])
     step_ms = float(per.sum(axis=1).mean())
     path_ms = per.mean(axis=0)
@@ -224,7 +263,7 @@ def run_ours(args, rank, world, local_rank):
         e2e_step()
     torch.cuda.synchronize()
     e2e_ms = []
-    for _ in range(max(3, args.steps // 2)):
+    for _ in range(min(20, max(3, args.steps // 2))):
         a, b = ev(), ev()
         flush.fill_(1)
         a.record(stream)
@@ -241,7 +280,7 @@ def run_ours(args, rank, world, local_rank):
 
     status = K.kata_get_status()
     return dict(step_ms=step_ms, path_ms=path_ms.tolist(), e2e_ms=e2e_ms, h2d=h2d, d2h=d2h,
-                clocks=clk.summary(), long=long, status=status, tokens=B * T, BH=BH, T=T, p=p, dv=dv, C=C)
+                clocks=clk.summary(), timed_s=clk.window[1] - clk.window[0], long=long, status=status, tokens=B * T, BH=BH, T=T, p=p, dv=dv, C=C)
 
 
 def run_long(args, K, torch, dev, stream, flush):
@@ -346,8 +385,8 @@ def config_dict(cfg, world):
 def main():
     ap = argparse.ArgumentParser(description="KATA forward hot-path benchmark")
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="layer340m_ctx2k", choices=sorted(workloads.CONFIGS))
     ap.add_argument("--long", type=int, default=1, help="also time the T=131072 workload (1 GPU)")
@@ -379,12 +418,7 @@ def main():
         res = run_ours(args, rank, world, local_rank)
         step_ms = res["step_ms"]
         e2e_ms = res["e2e_ms"]
-        if world > 1:
-            import torch
-            import torch.distributed as dist
-            t = torch.tensor([step_ms, e2e_ms], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            step_ms, e2e_ms = t.tolist()
+        step_ms, e2e_ms = reduce_max([step_ms, e2e_ms], world, device="cuda")
         if rank != 0:
             return
         report(args, res, step_ms, e2e_ms, world)
@@ -399,7 +433,7 @@ def report(args, res, step_ms, e2e_ms, world):
     cfg = workloads.CONFIGS[args.workload]
     BH, T, p, dv = res["BH"], res["T"], res["p"], res["dv"]
     tokens_all = res["tokens"] * world
-    value = tokens_all / (step_ms * 1e-3)
+    value = aggregate_value(res["tokens"], world, step_ms)
     quad_ms, chunk_ms, dec_ms = res["path_ms"]
     fl = flash_flops(BH, T, p, dv)
     achieved = fl / (quad_ms * 1e-3) / 1e12
@@ -422,6 +456,7 @@ def report(args, res, step_ms, e2e_ms, world):
                 "d2h_bytes_per_step": res["d2h"]},
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "clocks": res["clocks"],
+        "timed_region_s": res["timed_s"],
         "kernel_status": res["status"],
     }
     if res["long"]:

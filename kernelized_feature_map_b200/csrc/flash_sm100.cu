@@ -11,19 +11,27 @@
 //   warp 1      TMEM allocator and MMA issuer (one lane);
 //   warps 2-9   two "weight" warpgroups, one per query tile; thread = row.
 // Per key tile j and query tile i:
-//   S_i   = Q_i K_j^T                    tcgen05.mma, A,B from shared memory,
+//   S_i      = Q_i K_j^T                 tcgen05.mma, A,B from shared memory,
 //                                         fp32 accumulator in TMEM (128 cols)
-//   W_i   = (S_i)^2, causal mask          tcgen05.ld -> registers -> bf16 ->
+//   W_i      = (S_i)^2, causal mask       tcgen05.ld -> registers -> bf16 ->
 //                                         tcgen05.st back over S_i in TMEM
-//   O_i  += W_i V_j                       tcgen05.mma with A = W_i from TMEM
-//   D_i  += W_i 1                         same A against a block of ones, so
-//                                         numerator and denominator use the
-//                                         identical bf16 weights
+//   [O|D]_i += W_i [V_j | 1]              one tcgen05.mma per 16 keys with
+//                                         A = W_i from TMEM; the B operand is
+//                                         the V tile followed (one swizzle atom
+//                                         further) by a block of ones, so the
+//                                         denominator D comes out of the same
+//                                         MMA, from the identical bf16 weights
 // and at the end o = O_i / D_i (D = 0 gives 0), rounded to bf16.
 // Causal masking touches only the diagonal tile; tiles above it are skipped.
 //
-// TMEM columns: S_0 [0,128) S_1 [128,256) O_0, O_1 (DV each) from 256,
-// D_0, D_1 (16 each) after them; 512 columns are allocated.
+// The MMA issue order alternates between the two query tiles
+//   ... [O|D]_0 += W_0 V_j, S_0 = Q_0 K_{j+1}^T, [O|D]_1 += W_1 V_j,
+//       S_1 = Q_1 K_{j+1}^T, ...
+// so that one warpgroup squares its next tile while the tensor core works
+// for the other.
+//
+// TMEM columns: S_0 [0,128) S_1 [128,256) [O|D]_0, [O|D]_1 (DV + 16 each)
+// from 256; 512 columns are allocated.
 //
 // Every wait is bounded (sm100.cuh): a wait that runs out records
 // KATA_ERR_TIMEOUT, the CTA drains its own TMA copies and MMAs, frees TMEM
@@ -49,7 +57,8 @@ template <int p, int DV>
 struct FlashCfg {
   static constexpr int kQKBytes = kBM * p * 2;          // one Q or K tile
   static constexpr int kVBytes = kBN * DV * 2;          // one V tile
-  static constexpr int kOnesBytes = 512;
+  // block of ones read as the second N-atom of the [V | 1] operand
+  static constexpr int kOnesBytes = kBN * DV * 2;
   // K-major Q/K rows are p*2 bytes: 32 B (p=16, 32B swizzle) or 64 B (p=32)
   static constexpr Swizzle kQKSw = (p == 16) ? kSw32 : kSw64;
   static constexpr uint32_t kQKSbo = 8 * p * 2;         // 8-row group stride
@@ -59,13 +68,13 @@ struct FlashCfg {
   static constexpr uint32_t kVKStep = 16 * DV * 2;      // 16 keys
   // TMEM column map
   static constexpr uint32_t colS(int i) { return (uint32_t)i * 128; }
-  static constexpr uint32_t colO(int i) { return 256u + (uint32_t)i * DV; }
-  static constexpr uint32_t colD(int i) { return 256u + 2u * DV + (uint32_t)i * 16; }
+  static constexpr uint32_t colO(int i) { return 256u + (uint32_t)i * (DV + 16); }
+  static constexpr uint32_t colD(int i) { return colO(i) + DV; }
   // shared memory map (offsets from a 1024-aligned base)
   static constexpr int offQ = 0;
   static constexpr int offK = offQ + kNQ * kQKBytes;
   static constexpr int offV = ((offK + kStages * kQKBytes) + 1023) / 1024 * 1024;
-  static constexpr int offOnes = offV + kStages * kVBytes;
+  static constexpr int offOnes = offV + kStages * kVBytes;  // 1024-aligned
   static constexpr int offBar = offOnes + kOnesBytes;
   static constexpr int kNumBars = 1 + 2 * kStages + 3 * kNQ + 1;
   static constexpr int offMisc = offBar + kNumBars * 8;
@@ -156,48 +165,59 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t id_qk = idesc_bf16(kBM, kBN, false, false);
-      constexpr uint32_t id_pv = idesc_bf16(kBM, DV, false, true);
-      constexpr uint32_t id_d = idesc_bf16(kBM, 16, false, false);
+      constexpr uint32_t id_pv = idesc_bf16(kBM, DV + 16, false, true);  // [V | 1]
       const uint32_t sQ = smem_u32(smem + Cfg::offQ), sK = smem_u32(smem + Cfg::offK);
       const uint32_t sV = smem_u32(smem + Cfg::offV), sOnes = smem_u32(smem + Cfg::offOnes);
-      const uint64_t ones_desc = smem_desc(sOnes, 256, 128, kSwNone);
-      if (mbar_wait(q_full, 0, env)) {
-        for (int j = 0; j < nkv_max; ++j) {
-          const int st = j % kStages;
-          if (!mbar_wait(kv_full + st, (j / kStages) & 1, env)) break;
-          tc_fence_after();
-          for (int i = 0; i < kNQ; ++i) {
-            if (j >= nkv[i]) continue;
+      auto issue_qk = [&](int i, int st) {
 #pragma unroll
-            for (int ks = 0; ks < p / 16; ++ks) {
-              const uint64_t a = smem_desc(sQ + i * Cfg::kQKBytes + ks * 32, 16, Cfg::kQKSbo, Cfg::kQKSw);
-              const uint64_t b = smem_desc(sK + st * Cfg::kQKBytes + ks * 32, 16, Cfg::kQKSbo, Cfg::kQKSw);
-              mma_ss(tmem + Cfg::colS(i), a, b, id_qk, ks > 0);
-            }
-            mma_commit(s_full + i);
-          }
-          bool ok = true;
-          for (int i = 0; i < kNQ && ok; ++i) {
-            if (j >= nkv[i]) continue;
-            if (!mbar_wait(p_full + i, j & 1, env)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-#pragma unroll
-            for (int ks = 0; ks < kBN / 16; ++ks) {
-              const uint32_t a = tmem + Cfg::colS(i) + ks * 8;  // 16 bf16 weights = 8 columns
-              const uint64_t b = smem_desc(sV + st * Cfg::kVBytes + ks * Cfg::kVKStep, Cfg::kVBytes, Cfg::kVSbo,
-                                           Cfg::kVSw);
-              const uint32_t acc = (j > 0 || ks > 0) ? 1u : 0u;
-              mma_ts(tmem + Cfg::colO(i), a, b, id_pv, acc);
-              mma_ts(tmem + Cfg::colD(i), a, ones_desc, id_d, acc);
-            }
-            if (j == nkv[i] - 1) mma_commit(o_full + i);
-          }
-          if (!ok) break;
-          mma_commit(kv_empty + st);
+        for (int ks = 0; ks < p / 16; ++ks) {
+          const uint64_t a = smem_desc(sQ + i * Cfg::kQKBytes + ks * 32, 16, Cfg::kQKSbo, Cfg::kQKSw);
+          const uint64_t b = smem_desc(sK + st * Cfg::kQKBytes + ks * 32, 16, Cfg::kQKSbo, Cfg::kQKSw);
+          mma_ss(tmem + Cfg::colS(i), a, b, id_qk, ks > 0);
         }
+        mma_commit(s_full + i);
+      };
+      int kv_ready = -1;  // highest key tile whose K/V landed
+      bool ok = mbar_wait(q_full, 0, env) && (nkv_max == 0 || mbar_wait(kv_full, 0, env));
+      if (ok && nkv_max > 0) {
+        kv_ready = 0;
+        tc_fence_after();
+        for (int i = 0; i < kNQ; ++i)
+          if (nkv[i] > 0) issue_qk(i, 0);
+      }
+      for (int j = 0; ok && j < nkv_max; ++j) {
+        const int st = j % kStages;
+        const uint32_t sVst = sV + st * Cfg::kVBytes;
+        const uint32_t lbo = sOnes - sVst;  // V atom -> ones atom
+        for (int i = 0; i < kNQ; ++i) {
+          if (j >= nkv[i]) continue;
+          if (!mbar_wait(p_full + i, j & 1, env)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int ks = 0; ks < kBN / 16; ++ks) {
+            const uint32_t a = tmem + Cfg::colS(i) + ks * 8;  // 16 bf16 weights = 8 columns
+            const uint64_t b = smem_desc(sVst + ks * Cfg::kVKStep, lbo, Cfg::kVSbo, Cfg::kVSw);
+            mma_ts(tmem + Cfg::colO(i), a, b, id_pv, (j > 0 || ks > 0) ? 1u : 0u);
+          }
+          if (j == nkv[i] - 1) mma_commit(o_full + i);
+          if (j + 1 < nkv[i]) {
+            const int st1 = (j + 1) % kStages;
+            if (kv_ready < j + 1) {
+              if (!mbar_wait(kv_full + st1, ((j + 1) / kStages) & 1, env)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              kv_ready = j + 1;
+            }
+            issue_qk(i, st1);
+          }
+        }
+        if (!ok) break;
+        mma_commit(kv_empty + st);
       }
       mma_commit(mma_done);
       mbar_wait_drain(mma_done, 0, wc.limit);
@@ -220,23 +240,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool diag = (j == nkv[i] - 1);
       const uint32_t sa = lane_base + Cfg::colS(i);
 #pragma unroll
-      for (int b = 0; b < kBN / 32; ++b) {
-        uint32_t r[32];
-        tmem_ld32(sa + 32 * b, r);
+      for (int b2 = 0; b2 < kBN / 64; ++b2) {
+        uint32_t r[2][32];
+        tmem_ld32(sa + 64 * b2, r[0]);
+        tmem_ld32(sa + 64 * b2 + 32, r[1]);
         tmem_wait_ld();
-        uint32_t w[16];
 #pragma unroll
-        for (int x = 0; x < 16; ++x) {
-          const float s0 = __uint_as_float(r[2 * x]), s1 = __uint_as_float(r[2 * x + 1]);
-          float w0 = s0 * s0, w1 = s1 * s1;
-          if (diag) {
-            const int c = 32 * b + 2 * x;
-            if (c > m) w0 = 0.f;
-            if (c + 1 > m) w1 = 0.f;
+        for (int h = 0; h < 2; ++h) {
+          uint32_t w[16];
+#pragma unroll
+          for (int x = 0; x < 16; ++x) {
+            const float s0 = __uint_as_float(r[h][2 * x]), s1 = __uint_as_float(r[h][2 * x + 1]);
+            float w0 = s0 * s0, w1 = s1 * s1;
+            if (diag) {
+              const int c = 64 * b2 + 32 * h + 2 * x;
+              if (c > m) w0 = 0.f;
+              if (c + 1 > m) w1 = 0.f;
+            }
+            w[x] = pack_bf16x2(w0, w1);
           }
-          w[x] = pack_bf16x2(w0, w1);
+          tmem_st16(sa + 32 * b2 + 16 * h, w);
         }
-        tmem_st16(sa + 16 * b, w);
       }
       tmem_wait_st();
       tc_fence_before();

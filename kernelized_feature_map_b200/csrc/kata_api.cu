@@ -51,14 +51,14 @@ WaitCtl wait_ctl() { return WaitCtl{status_word(), wait_limit()}; }
 // workspace query and the call agree.
 constexpr int kTargetUnits = 2 * 148;
 
-ChunkPlan make_chunk_plan(int B, int H, int T, int p, int dv, int C, int /*num_sms*/) {
+ChunkPlan make_chunk_plan(int B, int H, int T, int p, int dv, int C, kata_dtype_t dt) {
   ChunkPlan pl{};
   pl.BH = B * H;
   pl.T = T;
   pl.p = p;
   pl.P = p * p;
   pl.dv = dv;
-  pl.ld = dv + 16;
+  pl.ld = dv + 4;
   pl.C = C;
   pl.Ls = 128;
   const int cands[] = {4096, 2048, 1024, 512, 256, 128};
@@ -71,7 +71,8 @@ ChunkPlan make_chunk_plan(int B, int H, int T, int p, int dv, int C, int /*num_s
   }
   if (pl.Ls < C) pl.Ls = C;
   pl.G = T > 0 ? (T + pl.Ls - 1) / pl.Ls : 0;
-  pl.record_floats = (size_t)pl.P * pl.ld;
+  pl.layout = chunked_on_tensor_cores(p, dv, dt) ? kRecPackedT : kRecUnpacked;
+  pl.record_floats = pl.layout == kRecPackedT ? (size_t)(dv + 1) * 144 : (size_t)pl.P * pl.ld;
   pl.workspace_bytes = (size_t)pl.BH * pl.G * pl.record_floats * sizeof(float);
   return pl;
 }
@@ -139,7 +140,7 @@ KATA_API kata_status_t kata_fwd_quadratic(const void* q, const void* k, const vo
 
 KATA_API size_t kata_fwd_chunked_workspace_size(int B, int H, int T, int p, int dv, int C, kata_dtype_t dtype) {
   if (check_common(B, H, T, p, dv, dtype) != KATA_OK || !(C == 64 || C == 128) || T == 0) return 0;
-  return make_chunk_plan(B, H, T, p, dv, C, 0).workspace_bytes;
+  return make_chunk_plan(B, H, T, p, dv, C, dtype).workspace_bytes;
 }
 
 KATA_API kata_status_t kata_fwd_chunked(const void* q, const void* k, const void* v, void* o, int B, int H, int T,
@@ -168,13 +169,13 @@ KATA_API kata_status_t kata_fwd_chunked(const void* q, const void* k, const void
   }
   if (!q || !k || !v || !o) return KATA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return KATA_ERR_MISALIGNED;
-  const ChunkPlan plan = make_chunk_plan(B, H, T, p, dv, C, 0);
+  const ChunkPlan plan = make_chunk_plan(B, H, T, p, dv, C, dtype);
   if (!workspace || workspace_bytes < plan.workspace_bytes) return KATA_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KATA_ERR_MISALIGNED;
   float* ws = static_cast<float*>(workspace);
-  // bf16 with p = 16 runs on the tensor cores; fp32 inputs (and p = 32) run
-  // the same three steps on the CUDA cores
-  const bool tc = dtype == KATA_BF16 && p == 16;
+  // bf16 with p = 16, dv = 64 runs on the tensor cores; other sizes and fp32
+  // inputs run the same three steps on the CUDA cores
+  const bool tc = plan.layout == kRecPackedT;
   const WaitCtl wc = wait_ctl();
   cudaError_t e = tc ? launch_chunk_state_sm100(k, v, ws, plan, wc, st)
                      : launch_chunk_aggregate_simt(k, v, ws, plan, dtype, st);

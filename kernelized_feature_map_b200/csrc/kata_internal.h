@@ -16,21 +16,33 @@ struct WaitCtl {
   long long limit;       // cycles before a wait gives up
 };
 
+// Layout of a workspace state record (one per (b,h) per super-chunk).
+enum RecordLayout {
+  kRecUnpacked = 0,  // P rows x ld floats: [sum psi(k) v^T | sum psi(k) | pad]
+  kRecPackedT = 1,   // 65 rows x 144 floats: transposed, packed psi (p=16, dv=64)
+};
+
 // Chunked-path plan: how the sequence is grouped for the state scan.
 struct ChunkPlan {
   int BH;        // B * H
   int T;
   int p, P;      // psi input width, P = p * p
   int dv;
-  int ld;        // row stride (floats) of a state record: dv + 16
+  int ld;        // row stride (floats) of an unpacked record: dv + 4
   int C;         // chunk length requested by the caller
   int Ls;        // super-chunk length (tokens per state record), multiple of 128 and C
   int G;         // number of super-chunks per (b,h): ceil(T / Ls)
-  size_t record_floats;  // P * ld
+  int layout;    // RecordLayout
+  size_t record_floats;
   size_t workspace_bytes;
 };
 
-ChunkPlan make_chunk_plan(int B, int H, int T, int p, int dv, int C, int num_sms);
+// True when the tensor-core chunked kernels serve these sizes (bf16, p = 16, dv = 64).
+inline bool chunked_on_tensor_cores(int p, int dv, kata_dtype_t dt) {
+  return dt == KATA_BF16 && p == 16 && dv == 64;
+}
+
+ChunkPlan make_chunk_plan(int B, int H, int T, int p, int dv, int C, kata_dtype_t dt);
 
 // decode.cu
 cudaError_t launch_decode(const void* q, const void* k, const void* v, void* o, float* S, float* z,

@@ -10,15 +10,22 @@
 // O(log G) (gist.science technical summary, sec. 2.3 "Chunked Parallelism" /
 // "Complexiteitsreductie": recurrence depth O(N_C) -> O(log N_C)).
 //
-// Work decomposition: one CTA per (b,h) and strip of 32 state entries; lane
-// = entry, the 8 warps share the tree levels.  The [G x 32] strip sits in
-// shared memory (at most 1024 records per pass; longer sequences are scanned
-// in blocks of 1024 with a running carry).  The kernel streams each record
-// once in and once out, so it is bound by HBM.
+// Work decomposition: one CTA per (b,h) and column block of NC record
+// entries; the [G x NC] tile sits in shared memory (at most 1024 records per
+// pass; longer sequences are scanned in blocks of 1024 with a running carry)
+// and the 256 threads share every tree level.  NC is chosen so that a tile is
+// about 32 KiB: the kernel streams every record once in and once out and is
+// bound by HBM.
 //
-// Record layout (per (b,h), per super-chunk g): P rows x ld floats; columns
-// 0..dv-1 hold the sum of psi(k) v^T, column dv the sum of psi(k) (the
-// normaliser), columns dv+1..ld-1 are padding and are not touched here.
+// Record layouts (per (b,h), per super-chunk g), see kata_internal.h:
+//   kRecUnpacked  P rows x ld floats: columns 0..dv-1 = sum psi(k) v^T,
+//                 column dv = sum psi(k), the rest padding;
+//   kRecPackedT   65 rows x 144 floats: row d < 64 = value column d, row 64 =
+//                 normaliser; column = packed psi coordinate (runs i = 0..15
+//                 of (i, j >= i), each padded to even length), off-diagonal
+//                 coordinates carry the sum of the (i,j) and (j,i) entries.
+// S0/z0 (optional initial state) and S_out/z_out (optional final state) use
+// the ABI layout [P, dv] / [P] and are converted here.
 #include "kata_common.cuh"
 #include "kata_internal.h"
 
@@ -27,85 +34,195 @@ namespace kata {
 constexpr int kScanBlock = 1024;  // records per shared-memory pass
 constexpr int kScanThreads = 256;
 
-__global__ void __launch_bounds__(kScanThreads) state_scan_kernel(float* __restrict__ ws, int G, int P, int dv,
-                                                                   int ld, long long record_floats,
-                                                                   const float* __restrict__ S0,
-                                                                   const float* __restrict__ z0,
-                                                                   float* __restrict__ S_out,
-                                                                   float* __restrict__ z_out) {
-  extern __shared__ float tile[];  // [Gp][32]
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int nwarps = kScanThreads / 32;
+// packed coordinate -> (i, j), -1 for a pad (p = 16)
+__constant__ signed char c_pack_i[144];
+__constant__ signed char c_pack_j[144];
+
+struct PackTable {
+  signed char i[144], j[144];
+  PackTable() {
+    int w = 0;
+    for (int a = 0; a < 16; ++a) {
+      for (int b = a; b < 16; ++b) {
+        i[w] = (signed char)a;
+        j[w] = (signed char)b;
+        ++w;
+      }
+      if ((16 - a) & 1) {
+        i[w] = -1;
+        j[w] = -1;
+        ++w;
+      }
+    }
+  }
+};
+
+static cudaError_t upload_pack_table() {
+  static int done_mask = 0;  // per device bit
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 31 && (done_mask >> dev) & 1) return cudaSuccess;
+  static const PackTable tab;
+  e = cudaMemcpyToSymbol(c_pack_i, tab.i, sizeof(tab.i));
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(c_pack_j, tab.j, sizeof(tab.j));
+  if (e == cudaSuccess && dev < 31) done_mask |= 1 << dev;
+  return e;
+}
+
+struct ScanArgs {
+  float* ws;
+  int G;
+  int E;          // floats per record
+  int NC;         // columns per CTA (power of two)
+  int Gp;         // records per shared-memory pass (power of two)
+  int layout;     // kRecUnpacked / kRecPackedT
+  int p, P, dv, ld;
+  const float* S0;
+  const float* z0;
+  float* S_out;
+  float* z_out;
+};
+
+// Initial value of record entry e for (b,h) from the ABI-layout S0/z0.
+__device__ __forceinline__ float initial_entry(const ScanArgs& a, long long bh, int e) {
+  if (a.layout == kRecUnpacked) {
+    const int r = e / a.ld, c = e % a.ld;
+    if (c < a.dv) return a.S0[(bh * a.P + r) * a.dv + c];
+    if (c == a.dv) return a.z0[bh * a.P + r];
+    return 0.f;
+  }
+  const int d = e / 144, w = e % 144;
+  const int i = c_pack_i[w], j = c_pack_j[w];
+  if (i < 0) return 0.f;
+  const int r1 = i * 16 + j, r2 = j * 16 + i;
+  if (d < 64) {
+    const float* S = a.S0 + bh * a.P * a.dv;
+    return i == j ? S[r1 * a.dv + d] : S[r1 * a.dv + d] + S[r2 * a.dv + d];
+  }
+  const float* z = a.z0 + bh * a.P;
+  return i == j ? z[r1] : z[r1] + z[r2];
+}
+
+// Write the final value of record entry e into the ABI-layout S_out/z_out.
+__device__ __forceinline__ void final_entry(const ScanArgs& a, long long bh, int e, float val) {
+  if (a.layout == kRecUnpacked) {
+    const int r = e / a.ld, c = e % a.ld;
+    if (c < a.dv) a.S_out[(bh * a.P + r) * a.dv + c] = val;
+    else if (c == a.dv) a.z_out[bh * a.P + r] = val;
+    return;
+  }
+  const int d = e / 144, w = e % 144;
+  const int i = c_pack_i[w], j = c_pack_j[w];
+  if (i < 0) return;
+  const float h = i == j ? val : 0.5f * val;  // symmetric halves (exact)
+  const int r1 = i * 16 + j, r2 = j * 16 + i;
+  if (d < 64) {
+    float* S = a.S_out + bh * a.P * a.dv;
+    S[r1 * a.dv + d] = h;
+    if (i != j) S[r2 * a.dv + d] = h;
+  } else {
+    float* z = a.z_out + bh * a.P;
+    z[r1] = h;
+    if (i != j) z[r2] = h;
+  }
+}
+
+__global__ void __launch_bounds__(kScanThreads) state_scan_kernel(ScanArgs a) {
+  extern __shared__ float sm[];
+  const int NC = a.NC, Gp_max = a.Gp;
+  float* tile = sm;                       // [Gp_max][NC]
+  float* carry = tile + Gp_max * NC;      // [NC]
+  float* total = carry + NC;              // [NC]
+  const int tid = threadIdx.x;
   const long long bh = blockIdx.y;
-  const int E = P * (dv + 1);
-  const int e = blockIdx.x * 32 + lane;
-  const bool active = e < E;
-  const int r = active ? e / (dv + 1) : 0;
-  const int c = active ? e % (dv + 1) : 0;
-  const long long off = (long long)r * ld + c;
-  float* base = ws + bh * (long long)G * record_floats + off;
+  const int col0 = blockIdx.x * NC;
+  float* base = a.ws + bh * (long long)a.G * a.E + col0;
+  int lognc = 0;
+  while ((1 << lognc) < NC) ++lognc;
 
-  float carry = 0.f;
-  if (active && S0) carry = (c < dv) ? S0[(bh * P + r) * dv + c] : z0[bh * P + r];
-
-  for (int g0 = 0; g0 < G; g0 += kScanBlock) {
-    const int n = min(kScanBlock, G - g0);
+  for (int c = tid; c < NC; c += kScanThreads) {
+    const int e = col0 + c;
+    carry[c] = (a.S0 && e < a.E) ? initial_entry(a, bh, e) : 0.f;
+  }
+  for (int g0 = 0; g0 < a.G; g0 += kScanBlock) {
+    const int n = min(kScanBlock, a.G - g0);
     int Gp = 1;
     while (Gp < n) Gp <<= 1;
-    for (int g = warp; g < Gp; g += nwarps)
-      tile[g * 32 + lane] = (active && g < n) ? base[(long long)(g0 + g) * record_floats] : 0.f;
+    for (int idx = tid; idx < Gp * NC; idx += kScanThreads) {
+      const int g = idx >> lognc, c = idx & (NC - 1);
+      tile[idx] = (g < n && col0 + c < a.E) ? base[(long long)(g0 + g) * a.E + c] : 0.f;
+    }
     __syncthreads();
-    // up-sweep: tile[k*2d + 2d - 1] += tile[k*2d + d - 1]
+    // up-sweep: tile[(2i+2)d - 1] += tile[(2i+1)d - 1]
     for (int d = 1; d < Gp; d <<= 1) {
       const int pairs = Gp / (2 * d);
-      for (int i = warp; i < pairs; i += nwarps) {
-        const int hi = (2 * i + 2) * d - 1, lo = (2 * i + 1) * d - 1;
-        tile[hi * 32 + lane] += tile[lo * 32 + lane];
+      for (int idx = tid; idx < pairs * NC; idx += kScanThreads) {
+        const int i = idx >> lognc, c = idx & (NC - 1);
+        tile[((2 * i + 2) * d - 1) * NC + c] += tile[((2 * i + 1) * d - 1) * NC + c];
       }
       __syncthreads();
     }
-    const float total = tile[(Gp - 1) * 32 + lane];
-    __syncthreads();
-    if (warp == 0) tile[(Gp - 1) * 32 + lane] = 0.f;
+    for (int c = tid; c < NC; c += kScanThreads) {
+      total[c] = tile[(Gp - 1) * NC + c];
+      tile[(Gp - 1) * NC + c] = 0.f;
+    }
     __syncthreads();
     // down-sweep
     for (int d = Gp >> 1; d >= 1; d >>= 1) {
       const int pairs = Gp / (2 * d);
-      for (int i = warp; i < pairs; i += nwarps) {
-        const int hi = (2 * i + 2) * d - 1, lo = (2 * i + 1) * d - 1;
-        const float t = tile[lo * 32 + lane];
-        tile[lo * 32 + lane] = tile[hi * 32 + lane];
-        tile[hi * 32 + lane] += t;
+      for (int idx = tid; idx < pairs * NC; idx += kScanThreads) {
+        const int i = idx >> lognc, c = idx & (NC - 1);
+        float* lo = tile + ((2 * i + 1) * d - 1) * NC + c;
+        float* hi = tile + ((2 * i + 2) * d - 1) * NC + c;
+        const float t = *lo;
+        *lo = *hi;
+        *hi += t;
       }
       __syncthreads();
     }
-    if (active)
-      for (int g = warp; g < n; g += nwarps) base[(long long)(g0 + g) * record_floats] = carry + tile[g * 32 + lane];
-    carry += total;
+    for (int idx = tid; idx < n * NC; idx += kScanThreads) {
+      const int g = idx >> lognc, c = idx & (NC - 1);
+      if (col0 + c < a.E) base[(long long)(g0 + g) * a.E + c] = carry[c] + tile[idx];
+    }
+    __syncthreads();
+    for (int c = tid; c < NC; c += kScanThreads) carry[c] += total[c];
     __syncthreads();
   }
-  if (active && warp == 0) {
-    if (c < dv) {
-      if (S_out) S_out[(bh * P + r) * dv + c] = carry;
-    } else {
-      if (z_out) z_out[bh * P + r] = carry;
-    }
-  }
+  if (a.S_out)
+    for (int c = tid; c < NC; c += kScanThreads)
+      if (col0 + c < a.E) final_entry(a, bh, col0 + c, carry[c]);
 }
 
 cudaError_t launch_state_scan(float* ws, const ChunkPlan& plan, const float* S0, const float* z0, float* S_out,
                               float* z_out, cudaStream_t st) {
-  int Gp = 1;
-  while (Gp < plan.G && Gp < kScanBlock) Gp <<= 1;
-  const size_t smem = (size_t)Gp * 32 * sizeof(float);
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(state_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (plan.layout == kRecPackedT) {
+    cudaError_t e = upload_pack_table();
     if (e != cudaSuccess) return e;
   }
-  const int E = plan.P * (plan.dv + 1);
-  dim3 grid(ceil_div(E, 32), plan.BH);
-  state_scan_kernel<<<grid, kScanThreads, smem, st>>>(ws, plan.G, plan.P, plan.dv, plan.ld,
-                                                      (long long)plan.record_floats, S0, z0, S_out, z_out);
+  ScanArgs a;
+  a.ws = ws;
+  a.G = plan.G;
+  a.E = (int)plan.record_floats;
+  a.Gp = 1;
+  while (a.Gp < plan.G && a.Gp < kScanBlock) a.Gp <<= 1;
+  a.NC = 8192 / a.Gp;
+  if (a.NC < 32) a.NC = 32;
+  if (a.NC > 2048) a.NC = 2048;
+  a.layout = plan.layout;
+  a.p = plan.p;
+  a.P = plan.P;
+  a.dv = plan.dv;
+  a.ld = plan.ld;
+  a.S0 = S0;
+  a.z0 = z0;
+  a.S_out = S_out;
+  a.z_out = z_out;
+  const size_t smem = ((size_t)a.Gp * a.NC + 2 * (size_t)a.NC) * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(state_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(ceil_div(a.E, a.NC), plan.BH);
+  state_scan_kernel<<<grid, kScanThreads, smem, st>>>(a);
   return cudaGetLastError();
 }
 
