@@ -24,6 +24,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD_DIR = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libkata.so")
+TRACE_LIB = os.path.join(PKG, "libkata_trace.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
@@ -53,15 +54,25 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(d) <= t for d in _deps())
 
 
-def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
-    """Compile and link libkata.so if any source is newer than it; returns its path."""
-    if not force and up_to_date():
+def build(force: bool = False, verbose: bool = False, extra_flags=(), trace: bool = False) -> str:
+    """Compile and link libkata.so if any source is newer than it; returns its path.
+
+    trace=True builds libkata_trace.so instead: the same sources with
+    KATA_ENABLE_TRACE defined (per-CTA pipeline timestamps, see
+    csrc/kata_trace.cuh).  It is a diagnostic build, never loaded by the
+    package.
+    """
+    lib_path = TRACE_LIB if trace else LIB
+    if not force and not trace and up_to_date():
         return LIB
-    os.makedirs(BUILD_DIR, exist_ok=True)
+    build_dir = BUILD_DIR + ("_trace" if trace else "")
+    if trace:
+        extra_flags = tuple(extra_flags) + ("-DKATA_ENABLE_TRACE",)
+    os.makedirs(build_dir, exist_ok=True)
     cc = nvcc()
 
     def compile_one(src):
-        obj = os.path.join(BUILD_DIR, os.path.basename(src) + ".o")
+        obj = os.path.join(build_dir, os.path.basename(src) + ".o")
         cmd = [cc, *NVCC_FLAGS, *extra_flags, "-c", src, "-o", obj]
         if verbose:
             print(" ".join(cmd), flush=True)
@@ -74,7 +85,7 @@ def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
 
     with ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
         objs = list(ex.map(compile_one, _sources()))
-    tmp = LIB + ".tmp.%d" % os.getpid()
+    tmp = lib_path + ".tmp.%d" % os.getpid()
     cmd = [cc, *ARCH, "-shared", "-cudart", "static", "-Xcompiler", "-fvisibility=hidden", "-o", tmp, *objs,
            "-lpthread", "-ldl", "-lrt"]
     if verbose:
@@ -82,8 +93,8 @@ def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError("link failed:\n%s%s" % (r.stdout, r.stderr))
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib_path)
+    return lib_path
 
 
 def main(argv=None):
@@ -91,9 +102,10 @@ def main(argv=None):
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true")
     ap.add_argument("--ptxas-info", action="store_true", help="print registers/spills/shared memory per kernel")
+    ap.add_argument("--trace", action="store_true", help="build the diagnostic libkata_trace.so")
     a = ap.parse_args(argv)
     extra = ["-Xptxas", "-v"] if a.ptxas_info else []
-    print(build(force=a.force or a.ptxas_info, verbose=a.verbose or a.ptxas_info, extra_flags=extra))
+    print(build(force=a.force or a.ptxas_info, verbose=a.verbose or a.ptxas_info, extra_flags=extra, trace=a.trace))
 
 
 if __name__ == "__main__":

@@ -36,7 +36,11 @@
 #include <cuda.h>
 
 #include "kata_internal.h"
+#include "kata_trace.cuh"
 #include "sm100.cuh"
+
+KATA_TRACE_DECLARE(chunk)
+KATA_TRACE_DECLARE(chunkstate)
 
 namespace kata {
 
@@ -214,29 +218,94 @@ __device__ __forceinline__ void global_to_state_lane(const float* row, uint32_t 
   }
 }
 
+// One 8-coordinate chunk (c = 0 or 1) of atom `atom` of row n of the bf16 copy.
+__device__ __forceinline__ void store_state_bf16_chunk(uint8_t* sb, int n, int atom, int c, const uint32_t* e) {
+  const int sw = (n >> 2) & 1;
+  *reinterpret_cast<uint4*>(sb + atom * kSBAtom + n * 32 + ((c ^ sw) << 4)) = make_uint4(
+      pack_bf16x2(__uint_as_float(e[0]), __uint_as_float(e[1])), pack_bf16x2(__uint_as_float(e[2]), __uint_as_float(e[3])),
+      pack_bf16x2(__uint_as_float(e[4]), __uint_as_float(e[5])), pack_bf16x2(__uint_as_float(e[6]), __uint_as_float(e[7])));
+}
+
+// Half `half` of a TMEM lane of S~^T (half 0: packed coordinates 0..71,
+// half 1: 72..143) -> bf16 copy row n (when `active`).  All loads of the half
+// are in flight before a single wait.  Warp-collective.
+__device__ __forceinline__ void state_half_to_bf16(uint32_t taddr, uint8_t* sb, int n, bool active, int half) {
+  uint32_t a[32], b[32], c[8];
+  if (half == 0) {
+    tmem_ld32(taddr, a);
+    tmem_ld32(taddr + 32, b);
+    tmem_ld8(taddr + 64, c);
+    tmem_wait_ld();
+    if (active) {
+      store_state_bf16_atom(sb, n, 0, a);
+      store_state_bf16_atom(sb, n, 1, a + 16);
+      store_state_bf16_atom(sb, n, 2, b);
+      store_state_bf16_atom(sb, n, 3, b + 16);
+      store_state_bf16_chunk(sb, n, 4, 0, c);
+    }
+  } else {
+    tmem_ld8(taddr + 72, c);
+    tmem_ld32(taddr + 80, a);
+    tmem_ld32(taddr + 112, b);
+    tmem_wait_ld();
+    if (active) {
+      store_state_bf16_chunk(sb, n, 4, 1, c);
+      store_state_bf16_atom(sb, n, 5, a);
+      store_state_bf16_atom(sb, n, 6, a + 16);
+      store_state_bf16_atom(sb, n, 7, b);
+      store_state_bf16_atom(sb, n, 8, b + 16);
+    }
+  }
+}
+
+// Half of an fp32 record row (or zeros) -> TMEM lane and bf16 copy row n.
+// Warp-collective.
+__device__ __forceinline__ void global_half_to_state(const float* row, uint32_t taddr, uint8_t* sb, int n,
+                                                     bool active, int half) {
+  auto ld4 = [&](int col, uint32_t* r) {
+    float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (active) v4 = *reinterpret_cast<const float4*>(row + col);
+    r[0] = __float_as_uint(v4.x);
+    r[1] = __float_as_uint(v4.y);
+    r[2] = __float_as_uint(v4.z);
+    r[3] = __float_as_uint(v4.w);
+  };
+  const int a0 = half == 0 ? 0 : 5;  // first whole atom of the half
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    uint32_t r[16];
+#pragma unroll
+    for (int e = 0; e < 16; e += 4) ld4(16 * (a0 + a) + e, r + e);
+    tmem_st16(taddr + 16 * (a0 + a), r);
+    if (active) store_state_bf16_atom(sb, n, a0 + a, r);
+  }
+  uint32_t r[8];
+  const int col = half == 0 ? 64 : 72;
+  ld4(col, r);
+  ld4(col + 4, r + 4);
+  tmem_st8(taddr + col, r);
+  if (active) store_state_bf16_chunk(sb, n, 4, half, r);
+}
+
 __device__ __forceinline__ void fill_ones(uint8_t* ones, int tid, int nthreads) {
   uint32_t* w = reinterpret_cast<uint32_t*>(ones);
   for (int x = tid; x < kOnesBytes / 4; x += nthreads) w[x] = 0x3F803F80u;
 }
 
-// A operand [V_c | 1]^T (M = 128: value columns then ones), K step ks.
-__device__ __forceinline__ uint64_t desc_vones_A(uint32_t sV, uint32_t sOnes, int ks) {
-  return smem_desc(sV + ks * 2048, sOnes - sV, 1024, kSw128);
-}
-// B operand [V_c | 1] (N = 80), K step ks.
-__device__ __forceinline__ uint64_t desc_vones_B(uint32_t sV, uint32_t sOnes, int ks) {
-  return smem_desc(sV + ks * 2048, sOnes - sV, 1024, kSw128);
-}
-// B operand psi~(K_c) [K = tokens x N = 144], K step ks.
-__device__ __forceinline__ uint64_t desc_psi_B(uint32_t sPsi, int ks) {
-  return smem_desc(sPsi + ks * 512, kPsiAtom, 256, kSw32);
+// [V_c | 1] as an MN-major operand with 128-byte swizzle: the V tile is the
+// first atom (columns / rows 0..63), the block of ones the second (64..127).
+// Used as the A operand [V_c | 1]^T (M = 128) of the state update and as the
+// B operand [V_c | 1] (N = 80) of the intra-chunk product.  K steps of 16
+// tokens are +2048 bytes.
+__device__ __forceinline__ uint64_t desc_vones(uint32_t sV, uint32_t sOnes) {
+  return smem_desc(sV, sOnes - sV, 1024, kSw128);
 }
 
 // ===========================================================================
 // 1. per-super-chunk state sums
 // ===========================================================================
 constexpr int kStateThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 psi~(k) + record
-constexpr int kStateStages = 3;
+constexpr int kStateStages = 6;
 
 struct StateSmem {
   static constexpr int kStage = kVBytes + kQKBytes;  // [V | K]
@@ -300,6 +369,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
         const int st = c % kStateStages;
         if (!mbar_wait(kv_empty + st, ((c / kStateStages) & 1) ^ 1, env)) break;
         uint8_t* base = smem + L::offStage + st * L::kStage;
+        KATA_TRACE(chunkstate, c, 5);
         mbar_arrive_expect_tx(kv_full + st, L::kStage);
         tma_load_3d(base, &tm_v, kv_full + st, 0, t0 + c * kTile, bh);
         tma_load_3d(base + kVBytes, &tm_k, kv_full + st, 0, t0 + c * kTile, bh);
@@ -313,16 +383,19 @@ __global__ void __launch_bounds__(kStateThreads, 1)
       constexpr uint32_t id_u = idesc_bf16(128, kNP, true, true);
       const uint32_t sStage = smem_u32(smem + L::offStage), sOnes = smem_u32(smem + L::offOnes);
       const uint32_t sPsi = smem_u32(smem + L::offPsi);
+      const uint64_t dpsi = smem_desc(sPsi, kPsiAtom, 256, kSw32);
       for (int c = 0; c < n_chunks; ++c) {
         const int st = c % kStateStages, pb = c & 1;
         if (!mbar_wait(kv_full + st, (c / kStateStages) & 1, env)) break;
         if (!mbar_wait(psi_full + pb, (c >> 1) & 1, env)) break;
+        KATA_TRACE(chunkstate, c, 0);
         tc_fence_after();
         const uint32_t sV = sStage + st * L::kStage;
+        const uint64_t da = desc_vones(sV, sOnes), db = desc_add(dpsi, pb * kPsiBytes);
 #pragma unroll
         for (int ks = 0; ks < kTile / 16; ++ks)
-          mma_ss(tmem, desc_vones_A(sV, sOnes, ks), desc_psi_B(sPsi + pb * kPsiBytes, ks), id_u,
-                 (c > 0 || ks > 0) ? 1u : 0u);
+          mma_ss(tmem, desc_add(da, ks * 2048), desc_add(db, ks * 512), id_u, (c > 0 || ks > 0) ? 1u : 0u);
+        KATA_TRACE(chunkstate, c, 1);
         mma_commit(psi_empty + pb);
         mma_commit(kv_empty + st);
       }
@@ -340,10 +413,12 @@ __global__ void __launch_bounds__(kStateThreads, 1)
         ok = false;
         break;
       }
+      if (tid == 0) KATA_TRACE(chunkstate, c, 2);
       if (c >= 2 && !mbar_wait(psi_empty + pb, ((c >> 1) - 1) & 1, env)) {
         ok = false;
         break;
       }
+      if (tid == 0) KATA_TRACE(chunkstate, c, 3);
       __nv_bfloat162 u[8];
       load_row_sw32(smem + L::offStage + st * L::kStage + kVBytes, tid, u);
       uint32_t w[kNPW];
@@ -351,6 +426,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
       store_psi_k(smem + L::offPsi + pb * kPsiBytes, tid, w);
       fence_proxy_async_smem();
       mbar_arrive(psi_full + pb);
+      if (tid == 0) KATA_TRACE(chunkstate, c, 4);
     }
     // record rows 0..64 live in TMEM lanes 0..64: warps of lane quarters 0-2
     // load (the load is warp-collective), lanes below 65 store
@@ -372,24 +448,38 @@ __global__ void __launch_bounds__(kStateThreads, 1)
 // ===========================================================================
 // 3. readout
 // ===========================================================================
-constexpr int kReadThreads = 448;  // warps: 0 TMA, 1 MMA, 2-5 weights+output, 6-9 psi~, 10-13 state
-constexpr int kReadStages = 3;
+// Warp roles (448 threads):
+//   warp 0       TMA: [V | Q | K] tiles of each chunk into a 6-stage ring
+//   warp 1       TMEM allocator, MMA issuer (one lane)
+//   warps 2-5    weights W = (Q K^T)^2 (causal) into TMEM; output o = O / D
+//   warps 6-9    psi~(q) into TMEM, psi~(k) into shared memory; bf16 copy of
+//                packed coordinates 0..71 of the state after each chunk
+//   warps 10-13  prefix state in; bf16 copy of coordinates 72..143
+// MMA order per chunk c: advance S~ by chunk c, readout of chunk c against
+// the bf16 copy of S~ made before chunk c, intra-chunk weights, then the
+// scores of chunk c+1.  The readout reads only the bf16 copy, so the state
+// can advance first; the copy for chunk c+1 is then refreshed while the
+// readout and intra-chunk MMAs of chunk c run (the copy is double-buffered).
+// The [O | D] accumulator is double-buffered so the readout of chunk c+1
+// does not wait for the output of chunk c to be read.
+constexpr int kReadThreads = 448;
+constexpr int kReadStages = 5;
 
 struct ReadSmem {
   static constexpr int kStage = kVBytes + 2 * kQKBytes;  // [V | Q | K]
   static constexpr int offStage = 0;
   static constexpr int offOnes = offStage + kReadStages * kStage;  // 1024-aligned
   static constexpr int offPsi = offOnes + kOnesBytes;
-  static constexpr int offSB = offPsi + kPsiBytes;
-  static constexpr int offBar = offSB + kSBBytes;
-  static constexpr int kBars = 2 * kReadStages + 10;
+  static constexpr int offSB = offPsi + kPsiBytes;     // 2 buffers
+  static constexpr int offBar = offSB + 2 * kSBBytes;
+  static constexpr int kBars = 2 * kReadStages + 12;
   static constexpr int offMisc = offBar + kBars * 8;
   static constexpr int kBytes = offMisc + 16 + 1024;
-  // TMEM columns (all multiples of 16)
-  static constexpr uint32_t colRun = 0;    // S~^T, 144 columns
-  static constexpr uint32_t colO = 144;    // [O | D], 80 columns
-  static constexpr uint32_t colPQ = 224;   // psi~(Q_c), 72 columns
-  static constexpr uint32_t colS = 304;    // Q K^T scores, then the bf16 weights
+  // TMEM columns (multiples of 16, 512 in total)
+  static constexpr uint32_t colRun = 0;                                    // S~^T, 144
+  static constexpr uint32_t colO(int b) { return 144u + 80u * (uint32_t)b; }  // [O | D] x 2
+  static constexpr uint32_t colPQ = 304;                                   // psi~(Q_c), 72
+  static constexpr uint32_t colS = 384;                                    // scores / weights, 128
 };
 
 __global__ void __launch_bounds__(kReadThreads, 1)
@@ -406,12 +496,12 @@ __global__ void __launch_bounds__(kReadThreads, 1)
   uint64_t* p_full = s_full + 1;              // weights written (128)
   uint64_t* fq_full = p_full + 1;             // psi~(Q_c) in TMEM (128)
   uint64_t* fk_full = fq_full + 1;            // psi~(K_c) in shared memory (128)
-  uint64_t* state_full = fk_full + 1;         // bf16 state copy ready (128)
+  uint64_t* state_full = fk_full + 1;         // bf16 state copy ready (256)
   uint64_t* rd_done = state_full + 1;         // readout of the chunk done
   uint64_t* upd_done = rd_done + 1;           // state advanced by the chunk
-  uint64_t* o_full = upd_done + 1;            // [O | D] complete
-  uint64_t* o_free = o_full + 1;              // [O | D] read (128)
-  uint64_t* mma_done = o_free + 1;
+  uint64_t* o_full = upd_done + 1;            // [2] [O | D] complete
+  uint64_t* o_free = o_full + 2;              // [2] [O | D] read (128)
+  uint64_t* mma_done = o_free + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::offMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::offMisc + 4);
 
@@ -432,11 +522,13 @@ __global__ void __launch_bounds__(kReadThreads, 1)
     mbar_init(p_full, 128);
     mbar_init(fq_full, 128);
     mbar_init(fk_full, 128);
-    mbar_init(state_full, 128);
+    mbar_init(state_full, 256);
     mbar_init(rd_done, 1);
     mbar_init(upd_done, 1);
-    mbar_init(o_full, 1);
-    mbar_init(o_free, 128);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(o_full + b, 1);
+      mbar_init(o_free + b, 128);
+    }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -480,9 +572,13 @@ __global__ void __launch_bounds__(kReadThreads, 1)
       constexpr uint32_t id_u = idesc_bf16(128, kNP, true, true);    // A = [V | 1]^T, B = psi~(K)
       const uint32_t sStage = smem_u32(smem + L::offStage), sOnes = smem_u32(smem + L::offOnes);
       const uint32_t sPsi = smem_u32(smem + L::offPsi), sSB = smem_u32(smem + L::offSB);
+      // descriptors built once; stages and K steps are constant offsets
+      const uint64_t dq0 = smem_desc(sStage + kVBytes, 16, 256, kSw32);
+      const uint64_t dk0 = smem_desc(sStage + kVBytes + kQKBytes, 16, 256, kSw32);
+      const uint64_t dpsi = smem_desc(sPsi, kPsiAtom, 256, kSw32);
+      const uint64_t dsb0 = smem_desc(sSB, 16, 256, kSw32);
       auto issue_qk = [&](int st) {
-        const uint32_t sQ = sStage + st * L::kStage + kVBytes;
-        mma_ss(tmem + L::colS, smem_desc(sQ, 16, 256, kSw32), smem_desc(sQ + kQKBytes, 16, 256, kSw32), id_qk, 0);
+        mma_ss(tmem + L::colS, desc_add(dq0, st * L::kStage), desc_add(dk0, st * L::kStage), id_qk, 0);
         mma_commit(s_full);
       };
       bool ok = n_chunks > 0 && mbar_wait(kv_full, 0, env);
@@ -491,47 +587,58 @@ __global__ void __launch_bounds__(kReadThreads, 1)
         issue_qk(0);
       }
       for (int c = 0; ok && c < n_chunks; ++c) {
-        const int st = c % kReadStages;
+        const int st = c % kReadStages, ob = c & 1;
         const uint32_t sV = sStage + st * L::kStage;
-        // readout against the state entering the chunk
-        if (!mbar_wait(fq_full, c & 1, env) || !mbar_wait(state_full, c & 1, env) ||
-            (c > 0 && !mbar_wait(o_free, (c - 1) & 1, env))) {
+        // advance the state by the chunk, once the bf16 copy of the state
+        // entering it has been read out of TMEM (state_full) and psi~(K_c)
+        // is in shared memory
+        KATA_TRACE(chunk, c, 0);
+        if (!mbar_wait(state_full, c & 1, env) || !mbar_wait(fk_full, c & 1, env)) {
           ok = false;
           break;
         }
+        KATA_TRACE(chunk, c, 1);
         tc_fence_after();
-#pragma unroll
-        for (int ks = 0; ks < kNP / 16; ++ks)
-          mma_ts(tmem + L::colO, tmem + L::colPQ + ks * 8, smem_desc(sSB + ks * kSBAtom, 16, 256, kSw32), id_rd,
-                 ks > 0);
-        mma_commit(rd_done);
-        // advance the state by the chunk
-        if (!mbar_wait(fk_full, c & 1, env)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
+        const uint64_t dvo = desc_vones(sV, sOnes);
 #pragma unroll
         for (int ks = 0; ks < kTile / 16; ++ks)
-          mma_ss(tmem + L::colRun, desc_vones_A(sV, sOnes, ks), desc_psi_B(sPsi, ks), id_u, 1);
+          mma_ss(tmem + L::colRun, desc_add(dvo, ks * 2048), desc_add(dpsi, ks * 512), id_u, 1);
         mma_commit(upd_done);
+        // readout against the bf16 copy of the state entering the chunk
+        KATA_TRACE(chunk, c, 2);
+        if (!mbar_wait(fq_full, c & 1, env) || (c >= 2 && !mbar_wait(o_free + ob, ((c - 2) >> 1) & 1, env))) {
+          ok = false;
+          break;
+        }
+        KATA_TRACE(chunk, c, 3);
+        tc_fence_after();
+        const uint64_t dsb = desc_add(dsb0, ob * kSBBytes);
+        const uint32_t dO = tmem + L::colO(ob);
+#pragma unroll
+        for (int ks = 0; ks < kNP / 16; ++ks)
+          mma_ts(dO, tmem + L::colPQ + ks * 8, desc_add(dsb, ks * kSBAtom), id_rd, ks > 0);
+        mma_commit(rd_done);
         // intra-chunk weights against [V_c | 1]
+        KATA_TRACE(chunk, c, 4);
         if (!mbar_wait(p_full, c & 1, env)) {
           ok = false;
           break;
         }
+        KATA_TRACE(chunk, c, 5);
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < kTile / 16; ++ks)
-          mma_ts(tmem + L::colO, tmem + L::colS + ks * 8, desc_vones_B(sV, sOnes, ks), id_wv, 1);
-        mma_commit(o_full);
+          mma_ts(dO, tmem + L::colS + ks * 8, desc_add(dvo, ks * 2048), id_wv, 1);
+        mma_commit(o_full + ob);
         mma_commit(kv_empty + st);
         if (c + 1 < n_chunks) {
           const int st1 = (c + 1) % kReadStages;
+          KATA_TRACE(chunk, c, 6);
           if (!mbar_wait(kv_full + st1, ((c + 1) / kReadStages) & 1, env)) {
             ok = false;
             break;
           }
+          KATA_TRACE(chunk, c, 7);
           tc_fence_after();
           issue_qk(st1);
         }
@@ -546,38 +653,52 @@ __global__ void __launch_bounds__(kReadThreads, 1)
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
     for (int c = 0; c < n_chunks; ++c) {
       if (!mbar_wait(s_full, c & 1, env)) break;
+      if (m == 0) KATA_TRACE(chunk, c, 8);
       tc_fence_after();
+      // causal within the chunk: 32-column block bb of row m is fully kept
+      // for bb < quarter, diagonal for bb == quarter, zero for bb > quarter
 #pragma unroll
-      for (int b2 = 0; b2 < 2; ++b2) {
-        uint32_t r[2][32];
-        tmem_ld32(lane_base + L::colS + 64 * b2, r[0]);
-        tmem_ld32(lane_base + L::colS + 64 * b2 + 32, r[1]);
-        tmem_wait_ld();
+      for (int bb = 0; bb < 4; ++bb) {
+        uint32_t w[16];
+        if (bb > quarter) {
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t w[16];
+          for (int x = 0; x < 16; ++x) w[x] = 0u;
+        } else {
+          uint32_t r[32];
+          tmem_ld32(lane_base + L::colS + 32 * bb, r);
+          tmem_wait_ld();
+          if (bb < quarter) {
 #pragma unroll
-          for (int x = 0; x < 16; ++x) {
-            const float s0 = __uint_as_float(r[h][2 * x]), s1 = __uint_as_float(r[h][2 * x + 1]);
-            const int col = 64 * b2 + 32 * h + 2 * x;
-            w[x] = pack_bf16x2(col > m ? 0.f : s0 * s0, col + 1 > m ? 0.f : s1 * s1);
+            for (int x = 0; x < 16; ++x) {
+              const float s0 = __uint_as_float(r[2 * x]), s1 = __uint_as_float(r[2 * x + 1]);
+              w[x] = pack_bf16x2(s0 * s0, s1 * s1);
+            }
+          } else {
+#pragma unroll
+            for (int x = 0; x < 16; ++x) {
+              const float s0 = __uint_as_float(r[2 * x]), s1 = __uint_as_float(r[2 * x + 1]);
+              w[x] = pack_bf16x2(2 * x > lane ? 0.f : s0 * s0, 2 * x + 1 > lane ? 0.f : s1 * s1);
+            }
           }
-          tmem_st16(lane_base + L::colS + 32 * b2 + 16 * h, w);
         }
+        tmem_st16(lane_base + L::colS + 16 * bb, w);
       }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(p_full);
+      if (m == 0) KATA_TRACE(chunk, c, 9);
       // output of the chunk
-      if (!mbar_wait(o_full, c & 1, env)) break;
+      const int ob = c & 1;
+      if (!mbar_wait(o_full + ob, (c >> 1) & 1, env)) break;
       tc_fence_after();
       uint32_t r0[32], r1[32], db;
-      tmem_ld32(lane_base + L::colO, r0);
-      tmem_ld32(lane_base + L::colO + 32, r1);
-      tmem_ld1(lane_base + L::colO + 64, db);
+      tmem_ld32(lane_base + L::colO(ob), r0);
+      tmem_ld32(lane_base + L::colO(ob) + 32, r1);
+      tmem_ld1(lane_base + L::colO(ob) + 64, db);
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(o_free);
+      mbar_arrive(o_free + ob);
+      if (m == 0) KATA_TRACE(chunk, c, 14);
       const int t = t0 + c * kTile + m;
       if (t < t1) {
         const float D = __uint_as_float(db);
@@ -595,54 +716,78 @@ __global__ void __launch_bounds__(kReadThreads, 1)
         }
       }
     }
-  } else if (warp < 10) {
-    // ------------------------------------------------------------- packed psi of q and k
-    const int quarter = warp % 4;
-    const int m = quarter * 32 + lane;  // token of the chunk = TMEM lane of its psi~(q)
-    const uint32_t pq_addr = tmem + ((uint32_t)(quarter * 32) << 16) + L::colPQ;
-    for (int c = 0; c < n_chunks; ++c) {
-      const int st = c % kReadStages;
-      if (!mbar_wait(kv_full + st, (c / kReadStages) & 1, env)) break;
-      const uint8_t* stage = smem + L::offStage + st * L::kStage;
-      __nv_bfloat162 uq[8], uk[8];
-      load_row_sw32(stage + kVBytes, m, uq);
-      load_row_sw32(stage + kVBytes + kQKBytes, m, uk);
-      uint32_t w[kNPW];
-      packed_psi<false>(uq, w);
-      if (c > 0 && !mbar_wait(rd_done, (c - 1) & 1, env)) break;
-      tc_fence_after();
-      store_psi_q_tmem(pq_addr, w);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(fq_full);
-      packed_psi<true>(uk, w);
-      if (c > 0 && !mbar_wait(upd_done, (c - 1) & 1, env)) break;
-      store_psi_k(smem + L::offPsi, m, w);
-      fence_proxy_async_smem();
-      mbar_arrive(fk_full);
-    }
   } else {
-    // ------------------------------------------------------------- state: prefix in, bf16 copies
+    // ------------------------------------------------------------- psi~ and state copies
+    const bool psi_group = warp < 10;   // warps 6-9: psi~ + half 0; warps 10-13: half 1
+    const int half = psi_group ? 0 : 1;
     const int quarter = warp % 4;
-    const int d = quarter * 32 + lane;  // TMEM lane = row of S~^T
-    const uint32_t run_addr = tmem + ((uint32_t)(quarter * 32) << 16) + L::colRun;
+    const int m = quarter * 32 + lane;  // token of the chunk / TMEM lane
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
     uint8_t* sb = smem + L::offSB;
-    const bool active = d < kSBRows;  // rows 0..63 values, 64..79 copies of z
+    const bool active = m < kSBRows;    // rows 0..63 values, 64..79 copies of z
+    // running state <- scanned prefix (fp32 into TMEM, bf16 into shared memory)
     if (quarter < 3) {
-      const float* row = ws + ((size_t)bh * G + g) * record_floats + (size_t)min(d, kRecRows - 1) * kNP;
-      global_to_state_lane(row, run_addr, sb, d, active);
+      const float* row = ws + ((size_t)bh * G + g) * record_floats + (size_t)min(m, kRecRows - 1) * kNP;
+      global_half_to_state(row, lane_base + L::colRun, sb, m, active, half);
     }
     tmem_wait_st();
     fence_proxy_async_smem();
     tc_fence_before();
     mbar_arrive(state_full);
-    for (int c = 0; c + 1 < n_chunks; ++c) {
-      if (!mbar_wait(upd_done, c & 1, env)) break;
-      tc_fence_after();
-      if (quarter < 3) state_lane_to_bf16(run_addr, sb, d, active);
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(state_full);
+    // chunk 0: psi~(k_0) needs nothing but the stage
+    bool ok = true;
+    if (psi_group && n_chunks > 0) {
+      if (!mbar_wait(kv_full, 0, env)) ok = false;
+      else {
+        __nv_bfloat162 uk[8];
+        uint32_t w[kNPW];
+        load_row_sw32(smem + L::offStage + kVBytes + kQKBytes, m, uk);
+        packed_psi<true>(uk, w);
+        store_psi_k(smem + L::offPsi, m, w);
+        fence_proxy_async_smem();
+        mbar_arrive(fk_full);
+      }
+    }
+    for (int c = 0; ok && c < n_chunks; ++c) {
+      if (psi_group) {
+        // psi~(q_c) into TMEM once the readout of chunk c-1 has consumed it
+        const int st = c % kReadStages;
+        if (!mbar_wait(kv_full + st, (c / kReadStages) & 1, env)) break;
+        __nv_bfloat162 uq[8];
+        uint32_t w[kNPW];
+        load_row_sw32(smem + L::offStage + st * L::kStage + kVBytes, m, uq);
+        packed_psi<false>(uq, w);
+        if (c > 0 && !mbar_wait(rd_done, (c - 1) & 1, env)) break;
+        tc_fence_after();
+        store_psi_q_tmem(lane_base + L::colPQ, w);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(fq_full);
+        if (m == 0) KATA_TRACE(chunk, c, 10);
+      }
+      if (c + 1 < n_chunks) {
+        // the state after chunk c is complete: this group's half of the bf16
+        // copy for the readout of chunk c+1, then psi~(k_{c+1})
+        if (!mbar_wait(upd_done, c & 1, env)) break;
+        tc_fence_after();
+        if (quarter < 3) state_half_to_bf16(lane_base + L::colRun, sb + ((c + 1) & 1) * kSBBytes, m, active, half);
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(state_full);
+        if (m == 0) KATA_TRACE(chunk, c, psi_group ? 12 : 13);
+        if (psi_group) {
+          const int st1 = (c + 1) % kReadStages;
+          if (!mbar_wait(kv_full + st1, ((c + 1) / kReadStages) & 1, env)) break;
+          __nv_bfloat162 uk[8];
+          uint32_t w[kNPW];
+          load_row_sw32(smem + L::offStage + st1 * L::kStage + kVBytes + kQKBytes, m, uk);
+          packed_psi<true>(uk, w);
+          store_psi_k(smem + L::offPsi, m, w);
+          fence_proxy_async_smem();
+          mbar_arrive(fk_full);
+          if (m == 0) KATA_TRACE(chunk, c, 11);
+        }
+      }
     }
   }
 

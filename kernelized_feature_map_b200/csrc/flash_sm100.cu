@@ -168,13 +168,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t id_pv = idesc_bf16(kBM, DV + 16, false, true);  // [V | 1]
       const uint32_t sQ = smem_u32(smem + Cfg::offQ), sK = smem_u32(smem + Cfg::offK);
       const uint32_t sV = smem_u32(smem + Cfg::offV), sOnes = smem_u32(smem + Cfg::offOnes);
+      // descriptors built once; K steps and stages are constant offsets
+      const uint64_t dq0 = smem_desc(sQ, 16, Cfg::kQKSbo, Cfg::kQKSw);
+      const uint64_t dk0 = smem_desc(sK, 16, Cfg::kQKSbo, Cfg::kQKSw);
       auto issue_qk = [&](int i, int st) {
+        const uint64_t a = desc_add(dq0, i * Cfg::kQKBytes), b = desc_add(dk0, st * Cfg::kQKBytes);
 #pragma unroll
-        for (int ks = 0; ks < p / 16; ++ks) {
-          const uint64_t a = smem_desc(sQ + i * Cfg::kQKBytes + ks * 32, 16, Cfg::kQKSbo, Cfg::kQKSw);
-          const uint64_t b = smem_desc(sK + st * Cfg::kQKBytes + ks * 32, 16, Cfg::kQKSbo, Cfg::kQKSw);
-          mma_ss(tmem + Cfg::colS(i), a, b, id_qk, ks > 0);
-        }
+        for (int ks = 0; ks < p / 16; ++ks) mma_ss(tmem + Cfg::colS(i), desc_add(a, ks * 32), desc_add(b, ks * 32), id_qk, ks > 0);
         mma_commit(s_full + i);
       };
       int kv_ready = -1;  // highest key tile whose K/V landed
@@ -188,7 +188,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; ok && j < nkv_max; ++j) {
         const int st = j % kStages;
         const uint32_t sVst = sV + st * Cfg::kVBytes;
-        const uint32_t lbo = sOnes - sVst;  // V atom -> ones atom
+        const uint64_t dv = smem_desc(sVst, sOnes - sVst, Cfg::kVSbo, Cfg::kVSw);  // V atom, then ones atom
         for (int i = 0; i < kNQ; ++i) {
           if (j >= nkv[i]) continue;
           if (!mbar_wait(p_full + i, j & 1, env)) {
@@ -196,12 +196,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
+          const uint32_t aw = tmem + Cfg::colS(i), dO = tmem + Cfg::colO(i);
 #pragma unroll
-          for (int ks = 0; ks < kBN / 16; ++ks) {
-            const uint32_t a = tmem + Cfg::colS(i) + ks * 8;  // 16 bf16 weights = 8 columns
-            const uint64_t b = smem_desc(sVst + ks * Cfg::kVKStep, lbo, Cfg::kVSbo, Cfg::kVSw);
-            mma_ts(tmem + Cfg::colO(i), a, b, id_pv, (j > 0 || ks > 0) ? 1u : 0u);
-          }
+          for (int ks = 0; ks < kBN / 16; ++ks)  // 16 bf16 weights = 8 TMEM columns per K step
+            mma_ts(dO, aw + ks * 8, desc_add(dv, ks * Cfg::kVKStep), id_pv, (j > 0 || ks > 0) ? 1u : 0u);
           if (j == nkv[i] - 1) mma_commit(o_full + i);
           if (j + 1 < nkv[i]) {
             const int st1 = (j + 1) % kStages;

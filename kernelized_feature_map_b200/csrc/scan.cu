@@ -149,9 +149,20 @@ __global__ void __launch_bounds__(kScanThreads) state_scan_kernel(ScanArgs a) {
     const int n = min(kScanBlock, a.G - g0);
     int Gp = 1;
     while (Gp < n) Gp <<= 1;
-    for (int idx = tid; idx < Gp * NC; idx += kScanThreads) {
-      const int g = idx >> lognc, c = idx & (NC - 1);
-      tile[idx] = (g < n && col0 + c < a.E) ? base[(long long)(g0 + g) * a.E + c] : 0.f;
+    // loads are batched 8 deep so that many are in flight per thread
+    for (int idx0 = 0; idx0 < Gp * NC; idx0 += 8 * kScanThreads) {
+      float r[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int idx = idx0 + u * kScanThreads + tid;
+        const int g = idx >> lognc, c = idx & (NC - 1);
+        r[u] = (idx < Gp * NC && g < n && col0 + c < a.E) ? __ldcs(base + (long long)(g0 + g) * a.E + c) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int idx = idx0 + u * kScanThreads + tid;
+        if (idx < Gp * NC) tile[idx] = r[u];
+      }
     }
     __syncthreads();
     // up-sweep: tile[(2i+2)d - 1] += tile[(2i+1)d - 1]
