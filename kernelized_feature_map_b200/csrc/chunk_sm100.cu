@@ -110,6 +110,44 @@ __device__ __forceinline__ void packed_psi(const __nv_bfloat162 (&u)[8], uint32_
   }
 }
 
+// Half of the packed psi words of one token: half 0 = runs i = 0..4 (words
+// 0..35), half 1 = runs i = 5..15 (words 36..71); used when two threads
+// share a token.
+template <bool key, int half>
+__device__ __forceinline__ void packed_psi_half(const __nv_bfloat162 (&u)[8], uint32_t (&out)[kNPW / 2]) {
+  __nv_bfloat162 s[8];
+#pragma unroll
+  for (int y = 0; y < 7; ++y) s[y] = __halves2bfloat162(u[y].y, u[y + 1].x);
+  s[7] = __halves2bfloat162(u[7].y, __float2bfloat16_rn(0.f));
+  int w = 0;
+#pragma unroll
+  for (int i = (half == 0 ? 0 : 5); i < (half == 0 ? 5 : 16); ++i) {
+    const __nv_bfloat16 ui = (i & 1) ? u[i >> 1].y : u[i >> 1].x;
+    const __nv_bfloat16 ui2 = key ? __hmul(ui, __float2bfloat16_rn(2.f)) : ui;
+    const int npairs = (16 - i + 1) / 2;
+#pragma unroll
+    for (int x = 0; x < npairs; ++x) {
+      const int j0 = i + 2 * x;
+      const __nv_bfloat162 pr = (j0 & 1) ? s[j0 >> 1] : u[j0 >> 1];
+      const __nv_bfloat162 f = (x == 0) ? __halves2bfloat162(ui, ui2) : __halves2bfloat162(ui2, ui2);
+      out[w++] = as_u32(__hmul2(f, pr));
+    }
+  }
+}
+
+// Half `half` (36 words) of psi~(k) of token t into the B tile: word groups
+// of 4 are 16-byte chunks, group g -> atom g / 2, chunk g % 2.
+template <int half>
+__device__ __forceinline__ void store_psi_k_half(uint8_t* psi, int t, const uint32_t (&w)[kNPW / 2]) {
+  const int x = (t >> 2) & 1;
+#pragma unroll
+  for (int q = 0; q < 9; ++q) {
+    const int g = half * 9 + q, a = g >> 1, c = g & 1;
+    *reinterpret_cast<uint4*>(psi + a * kPsiAtom + t * 32 + ((c ^ x) << 4)) =
+        make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+  }
+}
+
 // psi~(k) of token t into the N-major 32B-swizzled B tile.
 __device__ __forceinline__ void store_psi_k(uint8_t* psi, int t, const uint32_t (&w)[kNPW]) {
   const int x = (t >> 2) & 1;
@@ -304,7 +342,7 @@ __device__ __forceinline__ uint64_t desc_vones(uint32_t sV, uint32_t sOnes) {
 // ===========================================================================
 // 1. per-super-chunk state sums
 // ===========================================================================
-constexpr int kStateThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 psi~(k) + record
+constexpr int kStateThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2-9 psi~(k), warps 2-5 record
 constexpr int kStateStages = 6;
 
 struct StateSmem {
@@ -344,7 +382,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
       mbar_init(kv_empty + s, 1);
     }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(psi_full + s, 128);
+      mbar_init(psi_full + s, 256);
       mbar_init(psi_empty + s, 1);
     }
     mbar_init(acc_done, 1);
@@ -403,7 +441,9 @@ __global__ void __launch_bounds__(kStateThreads, 1)
       mbar_wait_drain(acc_done, 0, wc.limit);
     }
   } else {
-    const int tid = threadIdx.x - 64;  // token of the chunk
+    // warps 2-9: token (warp - 2) % 4 * 32 + lane, half (warp - 2) / 4 of its packed psi
+    const int tid = ((warp - 2) & 3) * 32 + lane;
+    const int half = (warp - 2) >> 2;
     const int quarter = warp % 4;
     const int d = quarter * 32 + lane;  // TMEM lane = record row
     bool ok = true;
@@ -421,16 +461,21 @@ __global__ void __launch_bounds__(kStateThreads, 1)
       if (tid == 0) KATA_TRACE(chunkstate, c, 3);
       __nv_bfloat162 u[8];
       load_row_sw32(smem + L::offStage + st * L::kStage + kVBytes, tid, u);
-      uint32_t w[kNPW];
-      packed_psi<true>(u, w);
-      store_psi_k(smem + L::offPsi + pb * kPsiBytes, tid, w);
+      uint32_t w[kNPW / 2];
+      if (half == 0) {
+        packed_psi_half<true, 0>(u, w);
+        store_psi_k_half<0>(smem + L::offPsi + pb * kPsiBytes, tid, w);
+      } else {
+        packed_psi_half<true, 1>(u, w);
+        store_psi_k_half<1>(smem + L::offPsi + pb * kPsiBytes, tid, w);
+      }
       fence_proxy_async_smem();
       mbar_arrive(psi_full + pb);
       if (tid == 0) KATA_TRACE(chunkstate, c, 4);
     }
     // record rows 0..64 live in TMEM lanes 0..64: warps of lane quarters 0-2
     // load (the load is warp-collective), lanes below 65 store
-    if (ok && quarter < 3 && mbar_wait(acc_done, 0, env)) {
+    if (ok && warp < 6 && quarter < 3 && mbar_wait(acc_done, 0, env)) {
       tc_fence_after();
       float* row = ws + ((size_t)bh * G + g) * record_floats + (size_t)min(d, kRecRows - 1) * kNP;
       state_lane_to_global(tmem + ((uint32_t)(quarter * 32) << 16), row, d < kRecRows);

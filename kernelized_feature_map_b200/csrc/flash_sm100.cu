@@ -6,10 +6,11 @@
 // forward), for bf16 inputs with fp32 accumulation.
 //
 // Per CTA: two 128-row query tiles of one (b,h); key/value tiles of 128 rows
-// stream through a 4-stage TMA ring.  Warp roles (320 threads):
+// stream through a 4-stage TMA ring.  Warp roles (576 threads):
 //   warp 0      TMA producer (one lane): Q tiles once, then K/V tiles;
 //   warp 1      TMEM allocator and MMA issuer (one lane);
-//   warps 2-9   two "weight" warpgroups, one per query tile; thread = row.
+//   warps 2-17  two "weight" groups of 8 warps, one per query tile; a
+//               thread owns one row and one half of the key columns.
 // Per key tile j and query tile i:
 //   S_i      = Q_i K_j^T                 tcgen05.mma, A,B from shared memory,
 //                                         fp32 accumulator in TMEM (128 cols)
@@ -50,7 +51,7 @@ constexpr int kBM = 128;       // query rows per tile
 constexpr int kBN = 128;       // keys per tile
 constexpr int kNQ = 2;         // query tiles per CTA
 constexpr int kStages = 4;     // K/V ring depth
-constexpr int kThreads = 320;  // 10 warps
+constexpr int kThreads = 576;  // 18 warps
 constexpr uint32_t kTmemCols = 512;
 
 template <int p, int DV>
@@ -119,7 +120,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < kNQ; ++i) {
       mbar_init(s_full + i, 1);
-      mbar_init(p_full + i, kBM);
+      mbar_init(p_full + i, 2 * kBM);
       mbar_init(o_full + i, 1);
     }
     mbar_init(mma_done, 1);
@@ -198,8 +199,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const uint32_t aw = tmem + Cfg::colS(i), dO = tmem + Cfg::colO(i);
 #pragma unroll
-          for (int ks = 0; ks < kBN / 16; ++ks)  // 16 bf16 weights = 8 TMEM columns per K step
-            mma_ts(dO, aw + ks * 8, desc_add(dv, ks * Cfg::kVKStep), id_pv, (j > 0 || ks > 0) ? 1u : 0u);
+          for (int ks = 0; ks < kBN / 16; ++ks)  // keys 16ks..: W columns 64*(ks/4) + 8*(ks%4)
+            mma_ts(dO, aw + (ks >> 2) * 64 + (ks & 3) * 8, desc_add(dv, ks * Cfg::kVKStep), id_pv,
+                   (j > 0 || ks > 0) ? 1u : 0u);
           if (j == nkv[i] - 1) mma_commit(o_full + i);
           if (j + 1 < nkv[i]) {
             const int st1 = (j + 1) % kStages;
@@ -222,7 +224,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------- weights + epilogue
-    const int i = (warp - 2) / 4;          // query tile of this warpgroup
+    // warps 2-9 serve query tile 0, warps 10-17 query tile 1; within a tile
+    // two warps share each TMEM lane quarter and split the 128 key columns:
+    // half h squares keys 64h .. 64h+63 and writes their bf16 weights over
+    // its own score columns [64h, 64h+32), so no warp overwrites scores
+    // another warp has yet to read.
+    const int idx = warp - 2;
+    const int i = idx / 8;                 // query tile of this warpgroup
+    const int h = (idx & 7) / 4;           // key-column half
     const int quarter = warp % 4;          // TMEM lane quarter this warp may access
     const int m = quarter * 32 + lane;     // row within the tile
     const int qtile = ct * kNQ + i;
@@ -236,29 +245,36 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       const bool diag = (j == nkv[i] - 1);
-      const uint32_t sa = lane_base + Cfg::colS(i);
+      const uint32_t sa = lane_base + Cfg::colS(i) + 64 * h;
+      // on the diagonal tile, 32-column block bb of row m is kept for
+      // bb < quarter, masked for bb == quarter and zero for bb > quarter
+      const int bb0 = 2 * h;
+      const bool zero0 = diag && bb0 > quarter, zero1 = diag && bb0 + 1 > quarter;
+      uint32_t r[2][32];
+      if (!zero0) tmem_ld32(sa, r[0]);
+      if (!zero1) tmem_ld32(sa + 32, r[1]);
+      tmem_wait_ld();
 #pragma unroll
-      for (int b2 = 0; b2 < kBN / 64; ++b2) {
-        uint32_t r[2][32];
-        tmem_ld32(sa + 64 * b2, r[0]);
-        tmem_ld32(sa + 64 * b2 + 32, r[1]);
-        tmem_wait_ld();
+      for (int hh = 0; hh < 2; ++hh) {
+        const int bb = bb0 + hh;
+        uint32_t w[16];
+        if (diag && bb > quarter) {
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t w[16];
+          for (int x = 0; x < 16; ++x) w[x] = 0u;
+        } else if (diag && bb == quarter) {
 #pragma unroll
           for (int x = 0; x < 16; ++x) {
-            const float s0 = __uint_as_float(r[h][2 * x]), s1 = __uint_as_float(r[h][2 * x + 1]);
-            float w0 = s0 * s0, w1 = s1 * s1;
-            if (diag) {
-              const int c = 64 * b2 + 32 * h + 2 * x;
-              if (c > m) w0 = 0.f;
-              if (c + 1 > m) w1 = 0.f;
-            }
-            w[x] = pack_bf16x2(w0, w1);
+            const float s0 = __uint_as_float(r[hh][2 * x]), s1 = __uint_as_float(r[hh][2 * x + 1]);
+            w[x] = pack_bf16x2(2 * x > lane ? 0.f : s0 * s0, 2 * x + 1 > lane ? 0.f : s1 * s1);
           }
-          tmem_st16(sa + 32 * b2 + 16 * h, w);
+        } else {
+#pragma unroll
+          for (int x = 0; x < 16; ++x) {
+            const float s0 = __uint_as_float(r[hh][2 * x]), s1 = __uint_as_float(r[hh][2 * x + 1]);
+            w[x] = pack_bf16x2(s0 * s0, s1 * s1);
+          }
         }
+        tmem_st16(sa + 16 * hh, w);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -266,37 +282,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok && mbar_wait(o_full + i, 0, env)) {
       tc_fence_after();
+      constexpr int kHalf = DV / 2;        // output columns per thread
       uint32_t dbits;
+      uint32_t ov[kHalf];
       tmem_ld1(lane_base + Cfg::colD(i), dbits);
-      float ov[DV];
       if constexpr (DV == 64) {
-        uint32_t r0[32], r1[32];
-        tmem_ld32(lane_base + Cfg::colO(i), r0);
-        tmem_ld32(lane_base + Cfg::colO(i) + 32, r1);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          ov[e] = __uint_as_float(r0[e]);
-          ov[32 + e] = __uint_as_float(r1[e]);
-        }
+        tmem_ld32(lane_base + Cfg::colO(i) + kHalf * h, ov);
       } else {
-        uint32_t r0[16];
-        tmem_ld16(lane_base + Cfg::colO(i), r0);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 16; ++e) ov[e] = __uint_as_float(r0[e]);
+        tmem_ld8(lane_base + Cfg::colO(i) + kHalf * h, ov);
       }
+      tmem_wait_ld();
       const float D = __uint_as_float(dbits);
       const float inv = D > 0.f ? 1.f / D : 0.f;
       if (t < T) {
-        uint4* dst = reinterpret_cast<uint4*>(o + ((size_t)bh * T + t) * DV);
+        uint4* dst = reinterpret_cast<uint4*>(o + ((size_t)bh * T + t) * DV + kHalf * h);
 #pragma unroll
-        for (int e = 0; e < DV / 8; ++e) {
+        for (int e = 0; e < kHalf / 8; ++e) {
           uint4 u;
-          u.x = pack_bf16x2(ov[8 * e + 0] * inv, ov[8 * e + 1] * inv);
-          u.y = pack_bf16x2(ov[8 * e + 2] * inv, ov[8 * e + 3] * inv);
-          u.z = pack_bf16x2(ov[8 * e + 4] * inv, ov[8 * e + 5] * inv);
-          u.w = pack_bf16x2(ov[8 * e + 6] * inv, ov[8 * e + 7] * inv);
+          u.x = pack_bf16x2(__uint_as_float(ov[8 * e + 0]) * inv, __uint_as_float(ov[8 * e + 1]) * inv);
+          u.y = pack_bf16x2(__uint_as_float(ov[8 * e + 2]) * inv, __uint_as_float(ov[8 * e + 3]) * inv);
+          u.z = pack_bf16x2(__uint_as_float(ov[8 * e + 4]) * inv, __uint_as_float(ov[8 * e + 5]) * inv);
+          u.w = pack_bf16x2(__uint_as_float(ov[8 * e + 6]) * inv, __uint_as_float(ov[8 * e + 7]) * inv);
           dst[e] = u;
         }
       }

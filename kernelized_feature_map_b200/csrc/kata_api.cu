@@ -44,12 +44,15 @@ static int* status_word() {
 
 WaitCtl wait_ctl() { return WaitCtl{status_word(), wait_limit()}; }
 
-// Super-chunk length: the largest of 4096 ... 128 tokens that still gives at
-// least kTargetUnits independent (b,h, super-chunk) work units, so that the
-// state records stay few (each costs a P x ld fp32 round trip through HBM)
-// while every SM gets work.  A pure function of the sizes, so that the
-// workspace query and the call agree.
-constexpr int kTargetUnits = 2 * 148;
+// Super-chunk length.  One CTA handles one (b,h, super-chunk) unit, 148 SMs
+// run one unit each per wave, and every unit costs its chunks plus a fixed
+// overhead (prologue, state record written, scanned and read back), counted
+// as kUnitOverhead chunks.  The plan takes the multiple of 128 tokens that
+// minimises  waves * (chunks per unit + kUnitOverhead),  preferring longer
+// super-chunks (fewer records) on ties.  A pure function of the sizes, so
+// that the workspace query and the call agree.
+constexpr int kSMs = 148;
+constexpr int kUnitOverhead = 2;
 
 ChunkPlan make_chunk_plan(int B, int H, int T, int p, int dv, int C, kata_dtype_t dt) {
   ChunkPlan pl{};
@@ -61,12 +64,16 @@ ChunkPlan make_chunk_plan(int B, int H, int T, int p, int dv, int C, kata_dtype_
   pl.ld = dv + 4;
   pl.C = C;
   pl.Ls = 128;
-  const int cands[] = {4096, 2048, 1024, 512, 256, 128};
-  for (int c : cands) {
-    const long long units = (long long)pl.BH * ((T + c - 1) / c);
-    if (units >= kTargetUnits) {
-      pl.Ls = c;
-      break;
+  const long long tiles = (T + 127) / 128;
+  long long best = -1;
+  const long long kmax = tiles < 1 ? 1 : (tiles < 512 ? tiles : 512);  // super-chunks up to 64K tokens
+  for (long long k = kmax; k >= 1; --k) {
+    const long long units = (long long)pl.BH * ((tiles + k - 1) / k);
+    const long long waves = (units + kSMs - 1) / kSMs;
+    const long long cost = waves * (k + kUnitOverhead);
+    if (best < 0 || cost < best) {
+      best = cost;
+      pl.Ls = (int)(k * 128);
     }
   }
   if (pl.Ls < C) pl.Ls = C;

@@ -149,17 +149,17 @@ __global__ void __launch_bounds__(kScanThreads) state_scan_kernel(ScanArgs a) {
     const int n = min(kScanBlock, a.G - g0);
     int Gp = 1;
     while (Gp < n) Gp <<= 1;
-    // loads are batched 8 deep so that many are in flight per thread
-    for (int idx0 = 0; idx0 < Gp * NC; idx0 += 8 * kScanThreads) {
-      float r[8];
+    // loads are batched 32 deep so that many are in flight per thread
+    for (int idx0 = 0; idx0 < Gp * NC; idx0 += 32 * kScanThreads) {
+      float r[32];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
+      for (int u = 0; u < 32; ++u) {
         const int idx = idx0 + u * kScanThreads + tid;
         const int g = idx >> lognc, c = idx & (NC - 1);
         r[u] = (idx < Gp * NC && g < n && col0 + c < a.E) ? __ldcs(base + (long long)(g0 + g) * a.E + c) : 0.f;
       }
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
+      for (int u = 0; u < 32; ++u) {
         const int idx = idx0 + u * kScanThreads + tid;
         if (idx < Gp * NC) tile[idx] = r[u];
       }

@@ -56,10 +56,11 @@ def test_workspace_size_query(L):
     assert ws(1, 1, 0, 16, 64, 64) == 0
     assert ws(1, 1, 100, 8, 64, 64) == 0
     assert ws(1, 1, 100, 16, 64, 96) == 0
-    # one fp32 record of P x (dv + 16) per (b,h) per super-chunk
+    # CUDA-core layout: one fp32 record of P x (dv + 4) per (b,h) per super-chunk
     n = ws(1, 1, 256, 16, 16, 64, dtype=None)
-    assert n > 0 and n % (256 * 32 * 4) == 0
-    assert ws(8, 16, 2048, 16, 64, 64) % (256 * 80 * 4) == 0
+    assert n > 0 and n % (256 * 20 * 4) == 0
+    # tensor-core layout (bf16, p = 16, dv = 64): 65 rows x 144 packed coordinates
+    assert ws(8, 16, 2048, 16, 64, 64) % (65 * 144 * 4) == 0
     # grows with T (more super-chunks) and never shrinks
     sizes = [ws(1, 16, t, 16, 64, 64) for t in (1024, 4096, 16384, 65536, 131072)]
     assert sizes == sorted(sizes)
