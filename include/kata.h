@@ -115,6 +115,29 @@ kata_status_t kata_fwd_chunked(const void* q, const void* k, const void* v, void
                                void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * kata_fwd_chunked without a caller-provided workspace.  The pages have no
+ * counterpart of this call; it exists for callers that cannot allocate
+ * device memory themselves (for example a C host program with no allocator
+ * of its own, or a loop whose rules forbid cudaMalloc because it can block
+ * and synchronise the device).
+ *
+ * Arguments, layouts, results and errors are those of kata_fwd_chunked.
+ * The scratch space lives in one library-owned device array of 16 MiB
+ * (16 * 2^20 bytes) that every GPU which loads the library holds until the
+ * process exits; sizes whose kata_fwd_chunked_workspace_size() exceeds it
+ * return KATA_ERR_WORKSPACE.  The call allocates nothing.
+ * All calls share that array: calls that overlap on the GPU race on it and
+ * must be serialised by the caller.  The first call on a device looks up the
+ * array's device address (once per device, with that device current); make
+ * that first call before any stream capture.
+ */
+kata_status_t kata_fwd_chunked_noalloc(const void* q, const void* k, const void* v, void* o,
+                                       int B, int H, int T, int p, int dv, int C,
+                                       kata_dtype_t dtype,
+                                       const float* S0, const float* z0,
+                                       float* S_out, float* z_out, void* stream);
+
+/*
  * One recurrent decode step for B*H independent streams (constant-time
  * recurrent inference on the fixed-size state; arXiv abstract on aiqbench):
  *   S <- S + psi(k) v^T,  z <- z + psi(k),  o = psi(q)^T S / psi(q)^T z
