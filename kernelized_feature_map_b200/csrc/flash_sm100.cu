@@ -5,8 +5,10 @@
 // gist.science technical summary, sec. 2.3 (a FlashAttention-style O(T^2)
 // forward), for bf16 inputs with fp32 accumulation.
 //
-// Per CTA: two 128-row query tiles of one (b,h); key/value tiles of 128 rows
-// stream through a 4-stage TMA ring.  Warp roles (576 threads):
+// Persistent CTAs (one per SM) walk work items of two 128-row query tiles of
+// one (b,h), heaviest first; key/value tiles of 128 rows stream through a
+// 4-stage TMA ring that continues across items, and the Q tiles of the next
+// item are prefetched into a second buffer.  Warp roles (576 threads):
 //   warp 0      TMA producer (one lane): Q tiles once, then K/V tiles;
 //   warp 1      TMEM allocator and MMA issuer (one lane);
 //   warps 2-17  two "weight" groups of 8 warps, one per query tile; a
@@ -72,12 +74,12 @@ struct FlashCfg {
   static constexpr uint32_t colO(int i) { return 256u + (uint32_t)i * (DV + 16); }
   static constexpr uint32_t colD(int i) { return colO(i) + DV; }
   // shared memory map (offsets from a 1024-aligned base)
-  static constexpr int offQ = 0;
-  static constexpr int offK = offQ + kNQ * kQKBytes;
+  static constexpr int offQ = 0;                        // 2 buffers x kNQ tiles
+  static constexpr int offK = offQ + 2 * kNQ * kQKBytes;
   static constexpr int offV = ((offK + kStages * kQKBytes) + 1023) / 1024 * 1024;
   static constexpr int offOnes = offV + kStages * kVBytes;  // 1024-aligned
   static constexpr int offBar = offOnes + kOnesBytes;
-  static constexpr int kNumBars = 1 + 2 * kStages + 3 * kNQ + 1;
+  static constexpr int kNumBars = 4 + 2 * kStages + 4 * kNQ + 1;
   static constexpr int offMisc = offBar + kNumBars * 8;
   static constexpr int kSmemBytes = offMisc + 16 + 1024;  // + alignment slack
 };
@@ -85,35 +87,42 @@ struct FlashCfg {
 template <int p, int DV>
 __global__ void __launch_bounds__(kThreads, 1)
     flash_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                     const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ o, int T, WaitCtl wc) {
+                     const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ o, int T, int BH,
+                     WaitCtl wc) {
   using Cfg = FlashCfg<p, DV>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::offBar);
-  uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;
-  uint64_t* kv_empty = kv_full + kStages;
-  uint64_t* s_full = kv_empty + kStages;
-  uint64_t* p_full = s_full + kNQ;
-  uint64_t* o_full = p_full + kNQ;
-  uint64_t* mma_done = o_full + kNQ;
+  uint64_t* q_full = bars;                 // [2] Q buffers
+  uint64_t* q_empty = q_full + 2;          // [2]
+  uint64_t* kv_full = q_empty + 2;         // [kStages]
+  uint64_t* kv_empty = kv_full + kStages;  // [kStages]
+  uint64_t* s_full = kv_empty + kStages;   // [kNQ] scores of tile i in TMEM
+  uint64_t* p_full = s_full + kNQ;         // [kNQ] weights of tile i written
+  uint64_t* o_full = p_full + kNQ;         // [kNQ] [O|D] of tile i complete
+  uint64_t* o_free = o_full + kNQ;         // [kNQ] [O|D] of tile i read by the epilogue
+  uint64_t* mma_done = o_free + kNQ;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Cfg::offMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::offMisc + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = blockIdx.y;
-  const int ct = gridDim.x - 1 - blockIdx.x;  // heaviest CTAs first
+  // Persistent CTAs.  A work item is (pair of query tiles ct, head bh); items
+  // are ordered heaviest first (largest ct) and dealt round-robin over CTAs.
   const int n_tiles = (T + kBM - 1) / kBM;
-  int nkv[kNQ];
-#pragma unroll
-  for (int i = 0; i < kNQ; ++i) {
-    const int qtile = ct * kNQ + i;
-    nkv[i] = qtile < n_tiles ? qtile + 1 : 0;
-  }
-  const int nkv_max = nkv[0] > nkv[1] ? nkv[0] : nkv[1];
+  const int n_ct = (n_tiles + kNQ - 1) / kNQ;
+  const int n_items = n_ct * BH;
+  auto item_ct = [&](int it) { return n_ct - 1 - it / BH; };
+  auto item_bh = [&](int it) { return it % BH; };
+  auto item_nkv = [&](int it, int i) {
+    const int qtile = item_ct(it) * kNQ + i;
+    return qtile < n_tiles ? qtile + 1 : 0;
+  };
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(q_full + b, 1);
+      mbar_init(q_empty + b, 1);
+    }
     for (int s = 0; s < kStages; ++s) {
       mbar_init(kv_full + s, 1);
       mbar_init(kv_empty + s, 1);
@@ -122,6 +131,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(s_full + i, 1);
       mbar_init(p_full + i, 2 * kBM);
       mbar_init(o_full + i, 1);
+      mbar_init(o_free + i, 2 * kBM);
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -145,22 +155,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
-      mbar_arrive_expect_tx(q_full, kNQ * Cfg::kQKBytes);
-      for (int i = 0; i < kNQ; ++i)
-        tma_load_3d(smem + Cfg::offQ + i * Cfg::kQKBytes, &tm_q, q_full, 0, (ct * kNQ + i) * kBM, bh);
-      int issued = 0;
-      for (int j = 0; j < nkv_max; ++j) {
-        const int st = j % kStages;
-        if (!mbar_wait(kv_empty + st, ((j / kStages) & 1) ^ 1, env)) break;
-        mbar_arrive_expect_tx(kv_full + st, Cfg::kQKBytes + Cfg::kVBytes);
-        tma_load_3d(smem + Cfg::offK + st * Cfg::kQKBytes, &tm_k, kv_full + st, 0, j * kBN, bh);
-        tma_load_3d(smem + Cfg::offV + st * Cfg::kVBytes, &tm_v, kv_full + st, 0, j * kBN, bh);
-        ++issued;
+      int nq = 0;    // items whose Q was loaded
+      long g = 0;    // key/value tiles loaded so far (ring position)
+      bool ok = true;
+      for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x, ++nq) {
+        const int qb = nq & 1, ct = item_ct(it), bh = item_bh(it);
+        if (!mbar_wait(q_empty + qb, ((nq >> 1) & 1) ^ 1, env)) break;
+        mbar_arrive_expect_tx(q_full + qb, kNQ * Cfg::kQKBytes);
+        for (int i = 0; i < kNQ; ++i)
+          tma_load_3d(smem + Cfg::offQ + (qb * kNQ + i) * Cfg::kQKBytes, &tm_q, q_full + qb, 0, (ct * kNQ + i) * kBM,
+                      bh);
+        const int nkv_max = max(item_nkv(it, 0), item_nkv(it, 1));
+        for (int j = 0; j < nkv_max; ++j, ++g) {
+          const int st = (int)(g % kStages);
+          if (!mbar_wait(kv_empty + st, (int)((g / kStages) & 1) ^ 1, env)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(kv_full + st, Cfg::kQKBytes + Cfg::kVBytes);
+          tma_load_3d(smem + Cfg::offK + st * Cfg::kQKBytes, &tm_k, kv_full + st, 0, j * kBN, bh);
+          tma_load_3d(smem + Cfg::offV + st * Cfg::kVBytes, &tm_v, kv_full + st, 0, j * kBN, bh);
+        }
       }
       // drain: every copy this CTA started must land before it exits
-      mbar_wait_drain(q_full, 0, wc.limit);
-      for (int j = issued - kStages < 0 ? 0 : issued - kStages; j < issued; ++j)
-        mbar_wait_drain(kv_full + j % kStages, (j / kStages) & 1, wc.limit);
+      for (int n = nq - 2 < 0 ? 0 : nq - 2; n < nq; ++n) mbar_wait_drain(q_full + (n & 1), (n >> 1) & 1, wc.limit);
+      for (long n = g - kStages < 0 ? 0 : g - kStages; n < g; ++n)
+        mbar_wait_drain(kv_full + n % kStages, (int)((n / kStages) & 1), wc.limit);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
@@ -169,55 +189,79 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t id_pv = idesc_bf16(kBM, DV + 16, false, true);  // [V | 1]
       const uint32_t sQ = smem_u32(smem + Cfg::offQ), sK = smem_u32(smem + Cfg::offK);
       const uint32_t sV = smem_u32(smem + Cfg::offV), sOnes = smem_u32(smem + Cfg::offOnes);
-      // descriptors built once; K steps and stages are constant offsets
+      // descriptors built once; K steps, Q buffers and stages are constant offsets
       const uint64_t dq0 = smem_desc(sQ, 16, Cfg::kQKSbo, Cfg::kQKSw);
       const uint64_t dk0 = smem_desc(sK, 16, Cfg::kQKSbo, Cfg::kQKSw);
-      auto issue_qk = [&](int i, int st) {
-        const uint64_t a = desc_add(dq0, i * Cfg::kQKBytes), b = desc_add(dk0, st * Cfg::kQKBytes);
+      auto issue_qk = [&](int i, int qb, int st) {
+        const uint64_t a = desc_add(dq0, (qb * kNQ + i) * Cfg::kQKBytes), b = desc_add(dk0, st * Cfg::kQKBytes);
 #pragma unroll
         for (int ks = 0; ks < p / 16; ++ks) mma_ss(tmem + Cfg::colS(i), desc_add(a, ks * 32), desc_add(b, ks * 32), id_qk, ks > 0);
         mma_commit(s_full + i);
       };
-      int kv_ready = -1;  // highest key tile whose K/V landed
-      bool ok = mbar_wait(q_full, 0, env) && (nkv_max == 0 || mbar_wait(kv_full, 0, env));
-      if (ok && nkv_max > 0) {
-        kv_ready = 0;
+      int nq = 0;
+      long g = 0;                   // ring position of the item's first key tile
+      int p_cnt[kNQ] = {0, 0};      // p_full phases consumed per tile
+      int o_cnt[kNQ] = {0, 0};      // o_full phases committed per tile
+      bool ok = true;
+      for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x, ++nq) {
+        const int qb = nq & 1;
+        int nkv[kNQ];
+        for (int i = 0; i < kNQ; ++i) nkv[i] = item_nkv(it, i);
+        const int nkv_max = max(nkv[0], nkv[1]);
+        if (!mbar_wait(q_full + qb, (nq >> 1) & 1, env) || !mbar_wait(kv_full + g % kStages, (int)((g / kStages) & 1), env)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         for (int i = 0; i < kNQ; ++i)
-          if (nkv[i] > 0) issue_qk(i, 0);
-      }
-      for (int j = 0; ok && j < nkv_max; ++j) {
-        const int st = j % kStages;
-        const uint32_t sVst = sV + st * Cfg::kVBytes;
-        const uint64_t dv = smem_desc(sVst, sOnes - sVst, Cfg::kVSbo, Cfg::kVSw);  // V atom, then ones atom
-        for (int i = 0; i < kNQ; ++i) {
-          if (j >= nkv[i]) continue;
-          if (!mbar_wait(p_full + i, j & 1, env)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t aw = tmem + Cfg::colS(i), dO = tmem + Cfg::colO(i);
-#pragma unroll
-          for (int ks = 0; ks < kBN / 16; ++ks)  // keys 16ks..: W columns 64*(ks/4) + 8*(ks%4)
-            mma_ts(dO, aw + (ks >> 2) * 64 + (ks & 3) * 8, desc_add(dv, ks * Cfg::kVKStep), id_pv,
-                   (j > 0 || ks > 0) ? 1u : 0u);
-          if (j == nkv[i] - 1) mma_commit(o_full + i);
-          if (j + 1 < nkv[i]) {
-            const int st1 = (j + 1) % kStages;
-            if (kv_ready < j + 1) {
-              if (!mbar_wait(kv_full + st1, ((j + 1) / kStages) & 1, env)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
-              kv_ready = j + 1;
+          if (nkv[i] > 0) issue_qk(i, qb, (int)(g % kStages));
+        long kv_ready = g;  // highest ring position whose K/V landed
+        for (int j = 0; ok && j < nkv_max; ++j) {
+          const long gj = g + j;
+          const int st = (int)(gj % kStages);
+          const uint32_t sVst = sV + st * Cfg::kVBytes;
+          const uint64_t dv = smem_desc(sVst, sOnes - sVst, Cfg::kVSbo, Cfg::kVSw);  // V atom, then ones atom
+          for (int i = 0; i < kNQ; ++i) {
+            if (j >= nkv[i]) continue;
+            if (!mbar_wait(p_full + i, p_cnt[i] & 1, env)) {
+              ok = false;
+              break;
             }
-            issue_qk(i, st1);
+            ++p_cnt[i];
+            // the first P.V of this tile overwrites [O|D]_i: the previous
+            // item's epilogue must have read it
+            if (j == 0 && o_cnt[i] > 0 && !mbar_wait(o_free + i, (o_cnt[i] - 1) & 1, env)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t aw = tmem + Cfg::colS(i), dO = tmem + Cfg::colO(i);
+#pragma unroll
+            for (int ks = 0; ks < kBN / 16; ++ks)  // keys 16ks..: W columns 64*(ks/4) + 8*(ks%4)
+              mma_ts(dO, aw + (ks >> 2) * 64 + (ks & 3) * 8, desc_add(dv, ks * Cfg::kVKStep), id_pv,
+                     (j > 0 || ks > 0) ? 1u : 0u);
+            if (j == nkv[i] - 1) {
+              mma_commit(o_full + i);
+              ++o_cnt[i];
+            }
+            if (j + 1 < nkv[i]) {
+              const long gn = gj + 1;
+              if (kv_ready < gn) {
+                if (!mbar_wait(kv_full + gn % kStages, (int)((gn / kStages) & 1), env)) {
+                  ok = false;
+                  break;
+                }
+                tc_fence_after();
+                kv_ready = gn;
+              }
+              issue_qk(i, qb, (int)(gn % kStages));
+            }
           }
+          if (!ok) break;
+          mma_commit(kv_empty + st);
         }
-        if (!ok) break;
-        mma_commit(kv_empty + st);
+        mma_commit(q_empty + qb);  // the item's Q tiles are free once its MMAs complete
+        g += nkv_max;
       }
       mma_commit(mma_done);
       mbar_wait_drain(mma_done, 0, wc.limit);
@@ -234,53 +278,59 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int h = (idx & 7) / 4;           // key-column half
     const int quarter = warp % 4;          // TMEM lane quarter this warp may access
     const int m = quarter * 32 + lane;     // row within the tile
-    const int qtile = ct * kNQ + i;
-    const int t = qtile * kBM + m;
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-    bool ok = nkv[i] > 0;
-    for (int j = 0; ok && j < nkv[i]; ++j) {
-      if (!mbar_wait(s_full + i, j & 1, env)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const bool diag = (j == nkv[i] - 1);
-      const uint32_t sa = lane_base + Cfg::colS(i) + 64 * h;
-      // on the diagonal tile, 32-column block bb of row m is kept for
-      // bb < quarter, masked for bb == quarter and zero for bb > quarter
-      const int bb0 = 2 * h;
-      const bool zero0 = diag && bb0 > quarter, zero1 = diag && bb0 + 1 > quarter;
-      uint32_t r[2][32];
-      if (!zero0) tmem_ld32(sa, r[0]);
-      if (!zero1) tmem_ld32(sa + 32, r[1]);
-      tmem_wait_ld();
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const int bb = bb0 + hh;
-        uint32_t w[16];
-        if (diag && bb > quarter) {
-#pragma unroll
-          for (int x = 0; x < 16; ++x) w[x] = 0u;
-        } else if (diag && bb == quarter) {
-#pragma unroll
-          for (int x = 0; x < 16; ++x) {
-            const float s0 = __uint_as_float(r[hh][2 * x]), s1 = __uint_as_float(r[hh][2 * x + 1]);
-            w[x] = pack_bf16x2(2 * x > lane ? 0.f : s0 * s0, 2 * x + 1 > lane ? 0.f : s1 * s1);
-          }
-        } else {
-#pragma unroll
-          for (int x = 0; x < 16; ++x) {
-            const float s0 = __uint_as_float(r[hh][2 * x]), s1 = __uint_as_float(r[hh][2 * x + 1]);
-            w[x] = pack_bf16x2(s0 * s0, s1 * s1);
-          }
+    int s_cnt = 0, o_cnt = 0;
+    bool ok = true;
+    for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
+      const int nkv = item_nkv(it, i);
+      if (nkv == 0) continue;
+      const int bh = item_bh(it);
+      const int t = (item_ct(it) * kNQ + i) * kBM + m;
+      for (int j = 0; j < nkv; ++j) {
+        if (!mbar_wait(s_full + i, s_cnt & 1, env)) {
+          ok = false;
+          break;
         }
-        tmem_st16(sa + 16 * hh, w);
+        ++s_cnt;
+        tc_fence_after();
+        const bool diag = (j == nkv - 1);
+        const uint32_t sa = lane_base + Cfg::colS(i) + 64 * h;
+        // on the diagonal tile, 32-column block bb of row m is kept for
+        // bb < quarter, masked for bb == quarter and zero for bb > quarter
+        const int bb0 = 2 * h;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int bb = bb0 + hh;
+          uint32_t w[16];
+          if (diag && bb > quarter) {
+#pragma unroll
+            for (int x = 0; x < 16; ++x) w[x] = 0u;
+          } else {
+            uint32_t r[32];
+            tmem_ld32(sa + 32 * hh, r);
+            tmem_wait_ld();
+            if (diag && bb == quarter) {
+#pragma unroll
+              for (int x = 0; x < 16; ++x) {
+                const float s0 = __uint_as_float(r[2 * x]), s1 = __uint_as_float(r[2 * x + 1]);
+                w[x] = pack_bf16x2(2 * x > lane ? 0.f : s0 * s0, 2 * x + 1 > lane ? 0.f : s1 * s1);
+              }
+            } else {
+#pragma unroll
+              for (int x = 0; x < 16; ++x) {
+                const float s0 = __uint_as_float(r[2 * x]), s1 = __uint_as_float(r[2 * x + 1]);
+                w[x] = pack_bf16x2(s0 * s0, s1 * s1);
+              }
+            }
+          }
+          tmem_st16(sa + 16 * hh, w);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(p_full + i);
       }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(p_full + i);
-    }
-    if (ok && mbar_wait(o_full + i, 0, env)) {
+      if (!ok || !mbar_wait(o_full + i, o_cnt & 1, env)) break;
+      ++o_cnt;
       tc_fence_after();
       constexpr int kHalf = DV / 2;        // output columns per thread
       uint32_t dbits;
@@ -292,6 +342,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld8(lane_base + Cfg::colO(i) + kHalf * h, ov);
       }
       tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(o_free + i);
       const float D = __uint_as_float(dbits);
       const float inv = D > 0.f ? 1.f / D : 0.f;
       if (t < T) {
@@ -367,8 +419,17 @@ static cudaError_t launch_flash_t(const void* q, const void* k, const void* v, v
   auto kern = flash_fwd_kernel<p, DV>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
   if (e != cudaSuccess) return e;
-  dim3 grid((T + kBM * kNQ - 1) / (kBM * kNQ), BH);
-  kern<<<grid, kThreads, Cfg::kSmemBytes, st>>>(tq, tk, tv, static_cast<__nv_bfloat16*>(o), T, wc);
+  // persistent: one CTA per SM (or fewer when there are fewer work items)
+  static int num_sms = 0;
+  if (num_sms == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || num_sms <= 0)
+      num_sms = 148;
+  }
+  const long items = (long)((T + kBM * kNQ - 1) / (kBM * kNQ)) * BH;
+  const int grid = (int)(items < num_sms ? items : num_sms);
+  kern<<<grid, kThreads, Cfg::kSmemBytes, st>>>(tq, tk, tv, static_cast<__nv_bfloat16*>(o), T, BH, wc);
   return cudaGetLastError();
 }
 
