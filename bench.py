@@ -277,10 +277,32 @@ def run_ours(args, rank, world, local_rank):
     long = None
     if args.long and world == 1:
         long = run_long(args, K, torch, dev, stream, flush)
+        long["decode_b64"] = run_decode_b64(args, K, torch, dev, stream, flush)
 
     status = K.kata_get_status()
     return dict(step_ms=step_ms, path_ms=path_ms.tolist(), e2e_ms=e2e_ms, h2d=h2d, d2h=d2h,
                 clocks=clk.summary(), timed_s=clk.window[1] - clk.window[0], long=long, status=status, tokens=B * T, BH=BH, T=T, p=p, dv=dv, C=C)
+
+
+def run_decode_b64(args, K, torch, dev, stream, flush):
+    """The decode step alone at the batched-serving size (B=64, H=16, state [256 x 64] fp32)."""
+    c = workloads.DECODE
+    q, k, v, S, z = workloads.decode_inputs(c["B"], c["H"], c["p"], c["dv"], seed=c["seed"], dtype=c["dtype"])
+    bf = torch.bfloat16
+    qd, kd, vd = (torch.from_numpy(x).to(dev, bf) for x in (q, k, v))
+    Sd, zd = torch.from_numpy(S).to(dev), torch.from_numpy(z).to(dev)
+    o = torch.empty((c["B"], c["H"], c["dv"]), dtype=bf, device=dev)
+    ms = []
+    for i in range(5 + args.long_steps * 4):
+        flush.fill_(1)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        K.kata_decode_step(qd, kd, vd, Sd, zd, o=o)
+        b.record(stream)
+        torch.cuda.synchronize()
+        if i >= 5:
+            ms.append(a.elapsed_time(b))
+    return dict(ms=float(np.mean(ms)), B=c["B"], H=c["H"], p=c["p"], dv=c["dv"])
 
 
 def run_long(args, K, torch, dev, stream, flush):
@@ -473,6 +495,12 @@ def report(args, res, step_ms, e2e_ms, world):
             "quadratic": {"ms": lg["quadratic_ms"], "tokens_per_s": ltok / (lg["quadratic_ms"] * 1e-3),
                           "tensor_frac": lf / (lg["quadratic_ms"] * 1e-3) / 1e12 / peaks["bf16_tflops"]},
         }
+        dc = lg["decode_b64"]
+        db = decode_bytes(dc["B"] * dc["H"], dc["p"], dc["dv"])
+        line["decode_b64"] = {
+            "workload": "decode step B=%d H=%d state [%d x %d] fp32" % (dc["B"], dc["H"], dc["p"] ** 2, dc["dv"]),
+            "ms": dc["ms"], "tokens_per_s": dc["B"] / (dc["ms"] * 1e-3),
+            "hbm_gbs": db / (dc["ms"] * 1e-3) / 1e9, "hbm_frac": db / (dc["ms"] * 1e-3) / 1e9 / peaks["hbm_gbs"]}
     if args.cpu_baseline and world == 1:
         cb = time_oracle(cfg)
         line["cpu_baseline"] = {"value": cb["value"], "unit": UNIT, "cores": cb["cores"], "kind": "oracle",

@@ -42,7 +42,10 @@
 #include <cuda.h>
 
 #include "kata_internal.h"
+#include "kata_trace.cuh"
 #include "sm100.cuh"
+
+KATA_TRACE_DECLARE(flash)
 
 namespace kata {
 namespace {
@@ -172,6 +175,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
+          KATA_TRACE(flash, (int)g, 9);
           mbar_arrive_expect_tx(kv_full + st, Cfg::kQKBytes + Cfg::kVBytes);
           tma_load_3d(smem + Cfg::offK + st * Cfg::kQKBytes, &tm_k, kv_full + st, 0, j * kBN, bh);
           tma_load_3d(smem + Cfg::offV + st * Cfg::kVBytes, &tm_v, kv_full + st, 0, j * kBN, bh);
@@ -223,10 +227,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t dv = smem_desc(sVst, sOnes - sVst, Cfg::kVSbo, Cfg::kVSw);  // V atom, then ones atom
           for (int i = 0; i < kNQ; ++i) {
             if (j >= nkv[i]) continue;
+            KATA_TRACE(flash, (int)gj, 2 * i);
             if (!mbar_wait(p_full + i, p_cnt[i] & 1, env)) {
               ok = false;
               break;
             }
+            KATA_TRACE(flash, (int)gj, 2 * i + 1);
             ++p_cnt[i];
             // the first P.V of this tile overwrites [O|D]_i: the previous
             // item's epilogue must have read it
@@ -258,6 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           if (!ok) break;
+          KATA_TRACE(flash, (int)gj, 4);
           mma_commit(kv_empty + st);
         }
         mma_commit(q_empty + qb);  // the item's Q tiles are free once its MMAs complete
@@ -291,6 +298,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = false;
           break;
         }
+        if (m == 0 && h == 0) KATA_TRACE(flash, s_cnt, 5 + 2 * i);
         ++s_cnt;
         tc_fence_after();
         const bool diag = (j == nkv - 1);
@@ -328,6 +336,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(p_full + i);
+        if (m == 0 && h == 0) KATA_TRACE(flash, s_cnt - 1, 6 + 2 * i);
       }
       if (!ok || !mbar_wait(o_full + i, o_cnt & 1, env)) break;
       ++o_cnt;
