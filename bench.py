@@ -44,7 +44,16 @@ import workloads  # noqa: E402
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 METRIC = "KATA-Mg fwd tokens/sec at T=2k and 131k (1 B200); % of roofline"
 UNIT = "tokens/s"
-LAUNCHES_PER_STEP = 5  # flash 1 + chunked 3 (state build, scan, readout) + decode 1
+
+
+def launches_per_step(B, H, T, p, dv, C):
+    """Kernels one step launches: flash 1, decode 1, and the chunked call's
+    readout plus, when the sequence spans several super-chunks (it then needs
+    a workspace), the state build and the scan."""
+    import kernelized_feature_map_b200 as K
+    import torch
+    chunked = 3 if K.kata_fwd_chunked_workspace_size(B, H, T, p, dv, C, torch.bfloat16) > 0 else 1
+    return 2 + chunked
 
 
 def load_peaks():
@@ -476,7 +485,7 @@ def report(args, res, step_ms, e2e_ms, world):
                      "algorithmic": "%.4g causal-useful flops per launch" % fl},
         "e2e": {"value": tokens_all / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": res["h2d"],
                 "d2h_bytes_per_step": res["d2h"]},
-        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "gpu_launches": launches_per_step(BH // cfg["H"], cfg["H"], T, p, dv, cfg["C"]) * args.steps,
         "clocks": res["clocks"],
         "timed_region_s": res["timed_s"],
         "kernel_status": res["status"],

@@ -129,12 +129,13 @@ def kata_fwd_chunked(q, k, v, C=64, S0=None, z0=None, return_state=False, o=None
         S_out = torch.empty((B, H, p * p, dv), dtype=torch.float32, device=dev)
         z_out = torch.empty((B, H, p * p), dtype=torch.float32, device=dev)
     need = kata_fwd_chunked_workspace_size(B, H, T, p, dv, C, q.dtype)
-    if workspace is None:
-        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check("kata_fwd_chunked", lib().kata_fwd_chunked(
         _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), B, H, T, p, dv, C, _dtype_code(q),
         _opt(S0, "S0"), _opt(z0, "z0"), _opt(S_out, "S_out"), _opt(z_out, "z_out"),
-        _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(), _stream_ptr(stream)))
+        _opt(workspace, "workspace"), ws_bytes, _stream_ptr(stream)))
     if return_state:
         return o, S_out, z_out
     return o

@@ -325,6 +325,104 @@ __device__ __forceinline__ void global_half_to_state(const float* row, uint32_t 
   if (active) store_state_bf16_chunk(sb, n, 4, half, r);
 }
 
+// Packed coordinate w -> (i, j) of psi, or i = j = -1 for a pad (runs
+// i = 0..15 of (i, j >= i), each padded to even length).  Evaluated at compile
+// time inside fully unrolled loops.
+__host__ __device__ constexpr int packed_i(int w) {
+  int base = 0;
+  for (int i = 0; i < 16; ++i) {
+    const int len = (16 - i) + ((16 - i) & 1);
+    if (w < base + len) return w - base < 16 - i ? i : -1;
+    base += len;
+  }
+  return -1;
+}
+__host__ __device__ constexpr int packed_j(int w) {
+  int base = 0;
+  for (int i = 0; i < 16; ++i) {
+    const int len = (16 - i) + ((16 - i) & 1);
+    if (w < base + len) return w - base < 16 - i ? i + (w - base) : -1;
+    base += len;
+  }
+  return -1;
+}
+static_assert(packed_i(0) == 0 && packed_j(0) == 0 && packed_j(15) == 15 && packed_i(16) == 1 && packed_j(16) == 1 &&
+                  packed_i(31) == -1 && packed_i(32) == 2 && packed_i(143) == -1 && packed_j(142) == 15,
+              "packed psi coordinate layout");
+
+// Value of packed coordinate w of row d of the state in the ABI layout
+// (S [p*p, dv], z [p*p], psi index r = i*p + j): the sum of the (i, j) and
+// (j, i) entries off the diagonal (the packed key side carries the factor 2).
+// Called with w known at compile time after unrolling.
+__device__ __forceinline__ float abi_packed_entry(const float* S, const float* z, int d, int w) {
+  const int i = packed_i(w), j = packed_j(w);
+  if (i < 0) return 0.f;
+  if (d < kDV) return i == j ? S[(i * 16 + j) * kDV + d] : S[(i * 16 + j) * kDV + d] + S[(j * 16 + i) * kDV + d];
+  return i == j ? z[i * 16 + j] : z[i * 16 + j] + z[j * 16 + i];
+}
+
+// Half `half` of row d (<= 64) of the state, packed, from the ABI-layout
+// initial state (zeros when S is null) -> TMEM lane and bf16 copy row n.
+// Warp-collective.
+template <int half>
+__device__ __forceinline__ void abi_half_to_state(const float* S, const float* z, int d, uint32_t taddr, uint8_t* sb,
+                                                  int n, bool active) {
+  uint32_t r[72];
+#pragma unroll
+  for (int e = 0; e < 72; ++e) r[e] = __float_as_uint(S && active ? abi_packed_entry(S, z, d, 72 * half + e) : 0.f);
+  if (half == 0) {
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      tmem_st16(taddr + 16 * a, *reinterpret_cast<const uint32_t(*)[16]>(r + 16 * a));
+      if (active) store_state_bf16_atom(sb, n, a, r + 16 * a);
+    }
+    tmem_st8(taddr + 64, *reinterpret_cast<const uint32_t(*)[8]>(r + 64));
+    if (active) store_state_bf16_chunk(sb, n, 4, 0, r + 64);
+  } else {
+    tmem_st8(taddr + 72, *reinterpret_cast<const uint32_t(*)[8]>(r));
+    if (active) store_state_bf16_chunk(sb, n, 4, 1, r);
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      tmem_st16(taddr + 80 + 16 * a, *reinterpret_cast<const uint32_t(*)[16]>(r + 8 + 16 * a));
+      if (active) store_state_bf16_atom(sb, n, 5 + a, r + 8 + 16 * a);
+    }
+  }
+}
+
+// Half `half` of TMEM lane d (<= 64) of the final state -> the ABI layout
+// (an off-diagonal packed entry is halved into (i, j) and (j, i), exactly).
+// Warp-collective.
+template <int half>
+__device__ __forceinline__ void state_half_to_abi(uint32_t taddr, float* S, float* z, int d, bool active) {
+  uint32_t r[72];
+  if (half == 0) {
+    tmem_ld32(taddr, *reinterpret_cast<uint32_t(*)[32]>(r));
+    tmem_ld32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
+    tmem_ld8(taddr + 64, *reinterpret_cast<uint32_t(*)[8]>(r + 64));
+  } else {
+    tmem_ld8(taddr + 72, *reinterpret_cast<uint32_t(*)[8]>(r));
+    tmem_ld32(taddr + 80, *reinterpret_cast<uint32_t(*)[32]>(r + 8));
+    tmem_ld32(taddr + 112, *reinterpret_cast<uint32_t(*)[32]>(r + 40));
+  }
+  tmem_wait_ld();
+  if (!active) return;
+#pragma unroll
+  for (int e = 0; e < 72; ++e) {
+    const int w = 72 * half + e;
+    const int i = packed_i(w), j = packed_j(w);
+    if (i < 0) continue;
+    const float val = __uint_as_float(r[e]);
+    const float hv = i == j ? val : 0.5f * val;
+    if (d < kDV) {
+      S[(i * 16 + j) * kDV + d] = hv;
+      if (i != j) S[(j * 16 + i) * kDV + d] = hv;
+    } else {
+      z[i * 16 + j] = hv;
+      if (i != j) z[j * 16 + i] = hv;
+    }
+  }
+}
+
 __device__ __forceinline__ void fill_ones(uint8_t* ones, int tid, int nthreads) {
   uint32_t* w = reinterpret_cast<uint32_t*>(ones);
   for (int x = tid; x < kOnesBytes / 4; x += nthreads) w[x] = 0x3F803F80u;
@@ -372,6 +470,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::offMisc + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  KATA_TRACE_BEGIN(chunkstate);
   const int g = blockIdx.x, bh = blockIdx.y;
   const int t0 = g * Ls;
   const int n_chunks = (min(T, t0 + Ls) - t0 + kTile - 1) / kTile;
@@ -530,7 +629,9 @@ struct ReadSmem {
 __global__ void __launch_bounds__(kReadThreads, 1)
     chunk_readout_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ o,
-                         const float* __restrict__ ws, int T, int Ls, int G, long long record_floats, WaitCtl wc) {
+                         const float* __restrict__ ws, const float* __restrict__ S0, const float* __restrict__ z0,
+                         float* __restrict__ S_out, float* __restrict__ z_out, int T, int Ls, int G,
+                         long long record_floats, WaitCtl wc) {
   using L = ReadSmem;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -551,6 +652,7 @@ __global__ void __launch_bounds__(kReadThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::offMisc + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  KATA_TRACE_BEGIN(chunk);
   // super-chunks in reverse order of the state kernel, so the key/value tiles
   // it touched last are still in L2 when they are read here first
   const int g = gridDim.x - 1 - blockIdx.x, bh = blockIdx.y;
@@ -770,10 +872,20 @@ __global__ void __launch_bounds__(kReadThreads, 1)
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
     uint8_t* sb = smem + L::offSB;
     const bool active = m < kSBRows;    // rows 0..63 values, 64..79 copies of z
-    // running state <- scanned prefix (fp32 into TMEM, bf16 into shared memory)
+    // running state <- scanned prefix (fp32 into TMEM, bf16 into shared
+    // memory); with a single super-chunk there is no workspace and the
+    // prefix is the caller's initial state (or zero)
+    const int d = min(m, kRecRows - 1);  // record row of this lane
     if (quarter < 3) {
-      const float* row = ws + ((size_t)bh * G + g) * record_floats + (size_t)min(m, kRecRows - 1) * kNP;
-      global_half_to_state(row, lane_base + L::colRun, sb, m, active, half);
+      if (ws) {
+        const float* row = ws + ((size_t)bh * G + g) * record_floats + (size_t)d * kNP;
+        global_half_to_state(row, lane_base + L::colRun, sb, m, active, half);
+      } else {
+        const float* S = S0 ? S0 + (size_t)bh * 256 * kDV : nullptr;
+        const float* z = z0 ? z0 + (size_t)bh * 256 : nullptr;
+        if (half == 0) abi_half_to_state<0>(S, z, d, lane_base + L::colRun, sb, m, active);
+        else abi_half_to_state<1>(S, z, d, lane_base + L::colRun, sb, m, active);
+      }
     }
     tmem_wait_st();
     fence_proxy_async_smem();
@@ -834,6 +946,16 @@ __global__ void __launch_bounds__(kReadThreads, 1)
         }
       }
     }
+    // the last super-chunk ends at token T: its running state, once the
+    // advance by its last chunk has landed, is the final state
+    if (S_out && g == G - 1 && n_chunks > 0 && !*abort_flag && mbar_wait(upd_done, (n_chunks - 1) & 1, env) &&
+        quarter < 3) {
+      tc_fence_after();
+      float* S = S_out + (size_t)bh * 256 * kDV;
+      float* z = z_out + (size_t)bh * 256;
+      if (half == 0) state_half_to_abi<0>(lane_base + L::colRun, S, z, m, m < kRecRows);
+      else state_half_to_abi<1>(lane_base + L::colRun, S, z, m, m < kRecRows);
+    }
   }
 
   tc_fence_before();
@@ -857,15 +979,18 @@ cudaError_t launch_chunk_state_sm100(const void* k, const void* v, float* ws, co
   cudaError_t e =
       cudaFuncSetAttribute(chunk_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, StateSmem::kBytes);
   if (e != cudaSuccess) return e;
-  dim3 grid(pl.G, pl.BH);
+  if (pl.G < 2) return cudaSuccess;  // the last super-chunk's sum is never needed
+  dim3 grid(pl.G - 1, pl.BH);
   chunk_state_kernel<<<grid, kStateThreads, StateSmem::kBytes, st>>>(tk, tv, ws, pl.T, pl.Ls, pl.G,
                                                                       (long long)pl.record_floats, wc);
   return cudaGetLastError();
 }
 
 cudaError_t launch_chunk_readout_sm100(const void* q, const void* k, const void* v, void* o, const float* ws,
+                                       const float* S0, const float* z0, float* S_out, float* z_out,
                                        const ChunkPlan& pl, const WaitCtl& wc, cudaStream_t st) {
   if (pl.p != 16 || pl.dv != kDV) return cudaErrorInvalidValue;
+  if (!ws && pl.G != 1) return cudaErrorInvalidValue;
   CUtensorMap tq, tk, tv;
   if (!make_tmap_bf16(&tq, q, 16, pl.T, pl.BH, kTile) || !make_tmap_bf16(&tk, k, 16, pl.T, pl.BH, kTile) ||
       !make_tmap_bf16(&tv, v, kDV, pl.T, pl.BH, kTile))
@@ -874,9 +999,9 @@ cudaError_t launch_chunk_readout_sm100(const void* q, const void* k, const void*
       cudaFuncSetAttribute(chunk_readout_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ReadSmem::kBytes);
   if (e != cudaSuccess) return e;
   dim3 grid(pl.G, pl.BH);
-  chunk_readout_kernel<<<grid, kReadThreads, ReadSmem::kBytes, st>>>(tq, tk, tv, static_cast<__nv_bfloat16*>(o),
-                                                                      ws, pl.T, pl.Ls, pl.G,
-                                                                      (long long)pl.record_floats, wc);
+  chunk_readout_kernel<<<grid, kReadThreads, ReadSmem::kBytes, st>>>(
+      tq, tk, tv, static_cast<__nv_bfloat16*>(o), ws, S0, z0, S_out, z_out, pl.T, pl.Ls, pl.G,
+      (long long)pl.record_floats, wc);
   return cudaGetLastError();
 }
 

@@ -109,6 +109,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::offMisc + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  KATA_TRACE_BEGIN(flash);
   // Persistent CTAs.  A work item is (pair of query tiles ct, head bh); items
   // are ordered heaviest first (largest ct) and dealt round-robin over CTAs.
   const int n_tiles = (T + kBM - 1) / kBM;

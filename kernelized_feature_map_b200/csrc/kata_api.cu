@@ -80,7 +80,9 @@ ChunkPlan make_chunk_plan(int B, int H, int T, int p, int dv, int C, kata_dtype_
   pl.G = T > 0 ? (T + pl.Ls - 1) / pl.Ls : 0;
   pl.layout = chunked_on_tensor_cores(p, dv, dt) ? kRecPackedT : kRecUnpacked;
   pl.record_floats = pl.layout == kRecPackedT ? (size_t)(dv + 1) * 144 : (size_t)pl.P * pl.ld;
-  pl.workspace_bytes = (size_t)pl.BH * pl.G * pl.record_floats * sizeof(float);
+  // the tensor-core path needs no records for a single super-chunk
+  const bool no_records = pl.layout == kRecPackedT && pl.G <= 1;
+  pl.workspace_bytes = no_records ? 0 : (size_t)pl.BH * pl.G * pl.record_floats * sizeof(float);
   return pl;
 }
 
@@ -177,19 +179,30 @@ KATA_API kata_status_t kata_fwd_chunked(const void* q, const void* k, const void
   if (!q || !k || !v || !o) return KATA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return KATA_ERR_MISALIGNED;
   const ChunkPlan plan = make_chunk_plan(B, H, T, p, dv, C, dtype);
-  if (!workspace || workspace_bytes < plan.workspace_bytes) return KATA_ERR_WORKSPACE;
-  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KATA_ERR_MISALIGNED;
-  float* ws = static_cast<float*>(workspace);
-  // bf16 with p = 16, dv = 64 runs on the tensor cores; other sizes and fp32
-  // inputs run the same three steps on the CUDA cores
-  const bool tc = plan.layout == kRecPackedT;
+  if (plan.workspace_bytes > 0) {
+    if (!workspace || workspace_bytes < plan.workspace_bytes) return KATA_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KATA_ERR_MISALIGNED;
+  }
+  float* ws = plan.workspace_bytes > 0 ? static_cast<float*>(workspace) : nullptr;
   const WaitCtl wc = wait_ctl();
-  cudaError_t e = tc ? launch_chunk_state_sm100(k, v, ws, plan, wc, st)
-                     : launch_chunk_aggregate_simt(k, v, ws, plan, dtype, st);
-  if (e == cudaSuccess) e = launch_state_scan(ws, plan, S0, z0, S_out, z_out, st);
-  if (e == cudaSuccess)
-    e = tc ? launch_chunk_readout_sm100(q, k, v, o, ws, plan, wc, st)
-           : launch_chunk_readout_simt(q, k, v, o, ws, plan, dtype, st);
+  if (plan.layout == kRecPackedT) {
+    // bf16 with p = 16, dv = 64 on the tensor cores: the sums of super-chunks
+    // 0..G-2 and their scan exist only when G > 1; the readout takes the
+    // prefix (or S0 when G == 1) and writes the final state itself
+    cudaError_t e = cudaSuccess;
+    if (plan.G > 1) {
+      e = launch_chunk_state_sm100(k, v, ws, plan, wc, st);
+      if (e == cudaSuccess) e = launch_state_scan(ws, plan, plan.G - 1, S0, z0, nullptr, nullptr, st);
+    }
+    if (e == cudaSuccess)
+      e = launch_chunk_readout_sm100(q, k, v, o, ws, plan.G > 1 ? nullptr : S0, plan.G > 1 ? nullptr : z0, S_out,
+                                     z_out, plan, wc, st);
+    return from_cuda(e);
+  }
+  // other sizes and fp32 inputs: the same three steps on the CUDA cores
+  cudaError_t e = launch_chunk_aggregate_simt(k, v, ws, plan, dtype, st);
+  if (e == cudaSuccess) e = launch_state_scan(ws, plan, plan.G, S0, z0, S_out, z_out, st);
+  if (e == cudaSuccess) e = launch_chunk_readout_simt(q, k, v, o, ws, plan, dtype, st);
   return from_cuda(e);
 }
 

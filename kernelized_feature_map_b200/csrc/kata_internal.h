@@ -49,8 +49,10 @@ cudaError_t launch_decode(const void* q, const void* k, const void* v, void* o, 
                           int BH, int p, int dv, kata_dtype_t dt, cudaStream_t st);
 
 // scan.cu -- exclusive prefix over the G records of every (b,h), in place,
-// plus S0 and the final state.
-cudaError_t launch_state_scan(float* ws, const ChunkPlan& plan, const float* S0, const float* z0,
+// plus S0 and the final state.  Records g >= G_in hold no data (treated as
+// zero), so the tensor-core path, whose state kernel skips the last
+// super-chunk, passes G_in = G - 1.
+cudaError_t launch_state_scan(float* ws, const ChunkPlan& plan, int G_in, const float* S0, const float* z0,
                               float* S_out, float* z_out, cudaStream_t st);
 
 // simt.cu -- CUDA-core kernels (fp32 inputs; exact fp32 arithmetic).
@@ -66,9 +68,14 @@ cudaError_t launch_flash_sm100(const void* q, const void* k, const void* v, void
                                const WaitCtl& wc, cudaStream_t st);
 
 // chunk_sm100.cu -- tcgen05 chunked-state forward (bf16 inputs, p = 16).
+// The state kernel sums super-chunks 0..G-2 (the last one's sum is never
+// needed); the readout of super-chunk g starts from workspace record g, or,
+// when G == 1 (ws == nullptr), from S0/z0 (zero when null), and the readout
+// of the last super-chunk writes the final state S_out/z_out when non-null.
 cudaError_t launch_chunk_state_sm100(const void* k, const void* v, float* ws, const ChunkPlan& pl, const WaitCtl& wc,
                                      cudaStream_t st);
 cudaError_t launch_chunk_readout_sm100(const void* q, const void* k, const void* v, void* o, const float* ws,
+                                       const float* S0, const float* z0, float* S_out, float* z_out,
                                        const ChunkPlan& pl, const WaitCtl& wc, cudaStream_t st);
 
 // Current bound on in-kernel waits and the status word (kata_api.cu).

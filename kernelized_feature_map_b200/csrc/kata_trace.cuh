@@ -15,7 +15,7 @@
 namespace kata {
 constexpr int kTraceCtas = 8;
 constexpr int kTraceTiles = 64;
-constexpr int kTraceSlots = 16;
+constexpr int kTraceSlots = 32;
 }  // namespace kata
 
 #ifdef KATA_ENABLE_TRACE
@@ -24,14 +24,26 @@ constexpr int kTraceSlots = 16;
   extern "C" __attribute__((visibility("default"))) int kata_trace_attach_##name(void* p) { \
     return (int)cudaMemcpyToSymbol(g_trace_buf_##name, &p, sizeof(p));                    \
   }
-#define KATA_TRACE(name, tile, slot)                                                                 \
-  do {                                                                                             \
-    const unsigned cta_ = blockIdx.y * gridDim.x + blockIdx.x;                                     \
-    if (g_trace_buf_##name && cta_ < (unsigned)::kata::kTraceCtas && (tile) < ::kata::kTraceTiles) \
-      g_trace_buf_##name[(cta_ * ::kata::kTraceTiles + (tile)) * ::kata::kTraceSlots + (slot)] = clock64(); \
+// Once per kernel, before any KATA_TRACE of `name`: this CTA's slice of the
+// buffer (null when the buffer is not attached or the CTA is not traced),
+// held in a register so that recording an event is a single store.
+#define KATA_TRACE_BEGIN(name)                                                            \
+  unsigned long long* const kata_trace_ptr_##name = [] {                                 \
+    const unsigned cta_ = blockIdx.y * gridDim.x + blockIdx.x;                           \
+    return (g_trace_buf_##name && cta_ < (unsigned)::kata::kTraceCtas)                   \
+               ? g_trace_buf_##name + (size_t)cta_ * ::kata::kTraceTiles * ::kata::kTraceSlots \
+               : (unsigned long long*)nullptr;                                          \
+  }()
+#define KATA_TRACE(name, tile, slot)                                                     \
+  do {                                                                                 \
+    if (kata_trace_ptr_##name && (tile) < ::kata::kTraceTiles)                           \
+      kata_trace_ptr_##name[(tile) * ::kata::kTraceSlots + (slot)] = clock64();          \
   } while (0)
 #else
 #define KATA_TRACE_DECLARE(name)
+#define KATA_TRACE_BEGIN(name) \
+  do {                         \
+  } while (0)
 #define KATA_TRACE(name, tile, slot) \
   do {                               \
   } while (0)

@@ -73,6 +73,7 @@ static cudaError_t upload_pack_table() {
 struct ScanArgs {
   float* ws;
   int G;
+  int G_in;       // records holding data (the rest are read as zero)
   int E;          // floats per record
   int NC;         // columns per CTA (power of two)
   int Gp;         // records per shared-memory pass (power of two)
@@ -156,7 +157,9 @@ __global__ void __launch_bounds__(kScanThreads) state_scan_kernel(ScanArgs a) {
       for (int u = 0; u < 32; ++u) {
         const int idx = idx0 + u * kScanThreads + tid;
         const int g = idx >> lognc, c = idx & (NC - 1);
-        r[u] = (idx < Gp * NC && g < n && col0 + c < a.E) ? __ldcs(base + (long long)(g0 + g) * a.E + c) : 0.f;
+        r[u] = (idx < Gp * NC && g < n && g0 + g < a.G_in && col0 + c < a.E)
+                   ? __ldcs(base + (long long)(g0 + g) * a.E + c)
+                   : 0.f;
       }
 #pragma unroll
       for (int u = 0; u < 32; ++u) {
@@ -205,8 +208,8 @@ __global__ void __launch_bounds__(kScanThreads) state_scan_kernel(ScanArgs a) {
       if (col0 + c < a.E) final_entry(a, bh, col0 + c, carry[c]);
 }
 
-cudaError_t launch_state_scan(float* ws, const ChunkPlan& plan, const float* S0, const float* z0, float* S_out,
-                              float* z_out, cudaStream_t st) {
+cudaError_t launch_state_scan(float* ws, const ChunkPlan& plan, int G_in, const float* S0, const float* z0,
+                              float* S_out, float* z_out, cudaStream_t st) {
   if (plan.layout == kRecPackedT) {
     cudaError_t e = upload_pack_table();
     if (e != cudaSuccess) return e;
@@ -214,6 +217,7 @@ cudaError_t launch_state_scan(float* ws, const ChunkPlan& plan, const float* S0,
   ScanArgs a;
   a.ws = ws;
   a.G = plan.G;
+  a.G_in = G_in;
   a.E = (int)plan.record_floats;
   a.Gp = 1;
   while (a.Gp < plan.G && a.Gp < kScanBlock) a.Gp <<= 1;

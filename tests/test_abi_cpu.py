@@ -59,8 +59,13 @@ def test_workspace_size_query(L):
     # CUDA-core layout: one fp32 record of P x (dv + 4) per (b,h) per super-chunk
     n = ws(1, 1, 256, 16, 16, 64, dtype=None)
     assert n > 0 and n % (256 * 20 * 4) == 0
-    # tensor-core layout (bf16, p = 16, dv = 64): 65 rows x 144 packed coordinates
-    assert ws(8, 16, 2048, 16, 64, 64) % (65 * 144 * 4) == 0
+    # tensor-core layout (bf16, p = 16, dv = 64): 65 rows x 144 packed
+    # coordinates per (b,h) per super-chunk, and none at all when the whole
+    # sequence is one super-chunk (the readout starts from S0 and writes the
+    # final state itself)
+    assert ws(8, 16, 2048, 16, 64, 64) == 0
+    n = ws(1, 16, 131072, 16, 64, 64)
+    assert n > 0 and n % (16 * 65 * 144 * 4) == 0
     # grows with T (more super-chunks) and never shrinks
     sizes = [ws(1, 16, t, 16, 64, 64) for t in (1024, 4096, 16384, 65536, 131072)]
     assert sizes == sorted(sizes)
@@ -90,9 +95,12 @@ def test_argument_errors_before_launch(L):
     assert g(a, b, c, d, 1, 1, 16, 16, 64, 96, 1, None, None, None, None, ws, 1 << 20, st) == _abi.KATA_ERR_UNSUPPORTED
     assert g(a, b, c, d, 1, 1, 16, 16, 64, 64, 1, _fake(0x60000), None, None, None, ws, 1 << 20, st) == _abi.KATA_ERR_INVALID_ARG
     assert g(a, b, c, d, 1, 1, 16, 16, 64, 64, 1, None, None, None, _fake(0x60000), ws, 1 << 20, st) == _abi.KATA_ERR_INVALID_ARG
-    assert g(a, b, c, d, 1, 1, 16, 16, 64, 64, 1, None, None, None, None, ws, 16, st) == _abi.KATA_ERR_WORKSPACE
-    assert g(a, b, c, d, 1, 1, 16, 16, 64, 64, 1, None, None, None, None, None, 1 << 20, st) == _abi.KATA_ERR_WORKSPACE
-    assert g(a, b, c, d, 1, 1, 16, 16, 64, 64, 1, None, None, None, None, _fake(0x50010), 1 << 20, st) == _abi.KATA_ERR_MISALIGNED
+    # a sequence of several super-chunks needs a workspace (one super-chunk needs none)
+    assert g(a, b, c, d, 1, 16, 131072, 16, 64, 64, 1, None, None, None, None, ws, 16, st) == _abi.KATA_ERR_WORKSPACE
+    assert g(a, b, c, d, 1, 16, 131072, 16, 64, 64, 1, None, None, None, None, None, 1 << 20,
+             st) == _abi.KATA_ERR_WORKSPACE
+    assert g(a, b, c, d, 1, 16, 131072, 16, 64, 64, 1, None, None, None, None, _fake(0x50010), 1 << 30,
+             st) == _abi.KATA_ERR_MISALIGNED
     assert g(a, b, c, d, 1, 1, 0, 16, 64, 64, 1, None, None, None, None, None, 0, st) == _abi.KATA_OK
     h = L.kata_decode_step
     assert h(a, b, c, d, _fake(0x70000), None, 1, 1, 16, 64, 1, st) == _abi.KATA_ERR_INVALID_ARG

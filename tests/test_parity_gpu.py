@@ -126,12 +126,16 @@ def test_empty_sequence_is_a_noop(kata):
 # state: initial / final state, split-and-resume, decode
 # ---------------------------------------------------------------------------
 
+# With 128 (b,h) pairs and T = 700 every pair is one super-chunk (no
+# workspace: the readout starts from S0 and writes the final state); with 2
+# pairs and T = 20000 each spans many, with the state build, the scan and
+# the prefix records in between.
+@pytest.mark.parametrize("B,H,T,t0", [(8, 16, 700, 300), (1, 2, 20000, 7000)])
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-def test_chunked_state_in_and_out(kata, dtype):
+def test_chunked_state_in_and_out(kata, dtype, B, H, T, t0):
     import torch
-    B, H, T, p, dv = 1, 2, 700, 16, 64
+    p, dv = 16, 64
     q, k, v = workloads.normal_qkv(B, H, T, p, dv, seed=7, dtype=dtype)
-    t0 = 300
     o_ref, S_ref, z_ref = oracle.recurrent(q, k, v, return_state=True)
     _, S1, z1 = oracle.recurrent(q[:, :, :t0], k[:, :, :t0], v[:, :, :t0], return_state=True)
     qd, kd, vd = to_dev(q, dtype), to_dev(k, dtype), to_dev(v, dtype)
