@@ -111,7 +111,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   KATA_TRACE_BEGIN(flash);
   // Persistent CTAs.  A work item is (pair of query tiles ct, head bh); items
-  // are ordered heaviest first (largest ct) and dealt round-robin over CTAs.
+  // are ordered heaviest first (largest ct) and dealt over CTAs in snake order.
   const int n_tiles = (T + kBM - 1) / kBM;
   const int n_ct = (n_tiles + kNQ - 1) / kNQ;
   const int n_items = n_ct * BH;
@@ -120,6 +120,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto item_nkv = [&](int it, int i) {
     const int qtile = item_ct(it) * kNQ + i;
     return qtile < n_tiles ? qtile + 1 : 0;
+  };
+  // the r-th item of this CTA: rounds of gridDim.x items, dealt in a snake
+  // order (odd rounds reversed) so that heavy and light items pair up; -1
+  // once the items run out
+  auto my_item = [&](int r) {
+    const int it = r * (int)gridDim.x + ((r & 1) ? (int)gridDim.x - 1 - (int)blockIdx.x : (int)blockIdx.x);
+    return it < n_items ? it : -1;
   };
 
   if (threadIdx.x == 0) {
@@ -162,7 +169,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int nq = 0;    // items whose Q was loaded
       long g = 0;    // key/value tiles loaded so far (ring position)
       bool ok = true;
-      for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x, ++nq) {
+      for (int it = my_item(nq); ok && it >= 0; it = my_item(++nq)) {
         const int qb = nq & 1, ct = item_ct(it), bh = item_bh(it);
         if (!mbar_wait(q_empty + qb, ((nq >> 1) & 1) ^ 1, env)) break;
         mbar_arrive_expect_tx(q_full + qb, kNQ * Cfg::kQKBytes);
@@ -208,7 +215,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int p_cnt[kNQ] = {0, 0};      // p_full phases consumed per tile
       int o_cnt[kNQ] = {0, 0};      // o_full phases committed per tile
       bool ok = true;
-      for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x, ++nq) {
+      for (int it = my_item(nq); ok && it >= 0; it = my_item(++nq)) {
         const int qb = nq & 1;
         int nkv[kNQ];
         for (int i = 0; i < kNQ; ++i) nkv[i] = item_nkv(it, i);
@@ -289,7 +296,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
     int s_cnt = 0, o_cnt = 0;
     bool ok = true;
-    for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
+    int rr = 0;
+    for (int it = my_item(rr); ok && it >= 0; it = my_item(++rr)) {
       const int nkv = item_nkv(it, i);
       if (nkv == 0) continue;
       const int bh = item_bh(it);
@@ -318,17 +326,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t r[32];
             tmem_ld32(sa + 32 * hh, r);
             tmem_wait_ld();
+            // squares on fp32 pairs (each rounded as a scalar multiply)
             if (diag && bb == quarter) {
 #pragma unroll
               for (int x = 0; x < 16; ++x) {
-                const float s0 = __uint_as_float(r[2 * x]), s1 = __uint_as_float(r[2 * x + 1]);
-                w[x] = pack_bf16x2(2 * x > lane ? 0.f : s0 * s0, 2 * x + 1 > lane ? 0.f : s1 * s1);
+                const uint32_t a = 2 * x > lane ? 0u : r[2 * x], b = 2 * x + 1 > lane ? 0u : r[2 * x + 1];
+                const uint64_t sq = f32x2_mul(f32x2(a, b), f32x2(a, b));
+                w[x] = pack_bf16x2(f32x2_lo(sq), f32x2_hi(sq));
               }
             } else {
 #pragma unroll
               for (int x = 0; x < 16; ++x) {
-                const float s0 = __uint_as_float(r[2 * x]), s1 = __uint_as_float(r[2 * x + 1]);
-                w[x] = pack_bf16x2(s0 * s0, s1 * s1);
+                const uint64_t sq = f32x2_mul(f32x2(r[2 * x], r[2 * x + 1]), f32x2(r[2 * x], r[2 * x + 1]));
+                w[x] = pack_bf16x2(f32x2_lo(sq), f32x2_hi(sq));
               }
             }
           }

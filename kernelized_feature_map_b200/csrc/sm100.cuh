@@ -197,6 +197,24 @@ __device__ __forceinline__ void tmem_st4(uint32_t taddr, const uint32_t (&r)[4])
 }
 
 // ---------------------------------------------------------------------------
+// packed fp32 pairs (two IEEE fp32 operations per instruction, each rounded
+// to nearest as the scalar ones)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint64_t f32x2(uint32_t lo, uint32_t hi) { return ((uint64_t)hi << 32) | lo; }
+__device__ __forceinline__ uint64_t f32x2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f32x2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float f32x2_lo(uint64_t a) { return __uint_as_float((uint32_t)a); }
+__device__ __forceinline__ float f32x2_hi(uint64_t a) { return __uint_as_float((uint32_t)(a >> 32)); }
+
+// ---------------------------------------------------------------------------
 // tcgen05.mma (single CTA), kind::f16 with bf16 operands and fp32 accumulate
 // ---------------------------------------------------------------------------
 enum Swizzle : uint32_t { kSwNone = 0, kSw128 = 2, kSw64 = 4, kSw32 = 6 };
