@@ -287,6 +287,8 @@ def run_ours(args, rank, world, local_rank):
     if args.long and world == 1:
         long = run_long(args, K, torch, dev, stream, flush)
         long["decode_b64"] = run_decode_b64(args, K, torch, dev, stream, flush)
+        if args.sweep:
+            long["sweep"], long["recall"] = run_sweep(args, K, torch, dev, stream, flush)
 
     status = K.kata_get_status()
     return dict(step_ms=step_ms, path_ms=path_ms.tolist(), e2e_ms=e2e_ms, h2d=h2d, d2h=d2h,
@@ -351,6 +353,62 @@ def run_long(args, K, torch, dev, stream, flush):
     out["quadratic_ms"] = float(np.mean(ms))
     out.update(B=B, H=H, T=T, p=p, dv=dv)
     return out
+
+
+def _time_call(fn, flush, stream, reps, warm):
+    import torch
+    ms = []
+    for i in range(warm + reps):
+        flush.fill_(1)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        if i >= warm:
+            ms.append(a.elapsed_time(b))
+    return float(np.mean(ms))
+
+
+def run_sweep(args, K, torch, dev, stream, flush):
+    """Throughput grid B x T (H=16, p=16, dv=64, bf16) for both paths, and the
+    recall-shaped p=32 workload.  Sweep inputs are drawn on the device from a
+    seeded generator (q, k L2-normalised N(0,1), v N(0,1)): the times do not
+    depend on the values, and the largest point would take minutes to draw on
+    the host."""
+    bf = torch.bfloat16
+    H, p, dv, C = 16, 16, 64, 64
+    gen = torch.Generator(device=dev)
+    grid = []
+    for B in (1, 4, 16):
+        for T in (1024, 4096, 16384, 65536, 131072):
+            gen.manual_seed(1000 * B + T % 997)
+            q = torch.randn((B, H, T, p), generator=gen, device=dev)
+            k = torch.randn((B, H, T, p), generator=gen, device=dev)
+            q = (q / q.norm(dim=-1, keepdim=True)).to(bf)
+            k = (k / k.norm(dim=-1, keepdim=True)).to(bf)
+            v = torch.randn((B, H, T, dv), generator=gen, device=dev).to(bf)
+            o = torch.empty((B, H, T, dv), dtype=bf, device=dev)
+            need = K.kata_fwd_chunked_workspace_size(B, H, T, p, dv, C, bf)
+            ws = torch.empty(max(256, need), dtype=torch.uint8, device=dev)
+            c_ms = _time_call(lambda: K.kata_fwd_chunked(q, k, v, C=C, o=o, workspace=ws), flush, stream, 3, 2)
+            heavy = B * T * T > 4 * 131072 * 131072
+            q_ms = _time_call(lambda: K.kata_fwd_quadratic(q, k, v, o=o), flush, stream, 1 if heavy else 3, 1)
+            grid.append(dict(B=B, T=T, chunked_ms=c_ms, quadratic_ms=q_ms))
+            del q, k, v, o, ws
+    torch.cuda.empty_cache()
+    cfg = workloads.CONFIGS["recall_p32"]
+    B, H, T, p, dv = cfg["B"], cfg["H"], cfg["T"], cfg["p"], cfg["dv"]
+    qn, kn, vn = workloads.make_inputs(cfg)
+    q, k, v = (torch.from_numpy(x).to(dev, bf) for x in (qn, kn, vn))
+    o = torch.empty((B, H, T, dv), dtype=bf, device=dev)
+    ws = torch.empty(max(256, K.kata_fwd_chunked_workspace_size(B, H, T, p, dv, cfg["C"], bf)), dtype=torch.uint8,
+                     device=dev)
+    recall = dict(B=B, H=H, T=T, p=p, dv=dv,
+                  chunked_ms=_time_call(lambda: K.kata_fwd_chunked(q, k, v, C=cfg["C"], o=o, workspace=ws), flush,
+                                        stream, 3, 1),
+                  quadratic_ms=_time_call(lambda: K.kata_fwd_quadratic(q, k, v, o=o), flush, stream, 3, 1))
+    return grid, recall
 
 
 # ---------------------------------------------------------------------------
@@ -422,6 +480,7 @@ def main():
     ap.add_argument("--workload", default="layer340m_ctx2k", choices=sorted(workloads.CONFIGS))
     ap.add_argument("--long", type=int, default=1, help="also time the T=131072 workload (1 GPU)")
     ap.add_argument("--long-steps", type=int, default=8)
+    ap.add_argument("--sweep", type=int, default=1, help="also time the B x T grid and the p=32 recall workload")
     ap.add_argument("--cpu-baseline", type=int, default=1)
     ap.add_argument("--ref-budget", type=float, default=15.0, help="seconds of oracle work per reference step")
     args = ap.parse_args()
@@ -510,6 +569,25 @@ def report(args, res, step_ms, e2e_ms, world):
             "workload": "decode step B=%d H=%d state [%d x %d] fp32" % (dc["B"], dc["H"], dc["p"] ** 2, dc["dv"]),
             "ms": dc["ms"], "tokens_per_s": dc["B"] / (dc["ms"] * 1e-3),
             "hbm_gbs": db / (dc["ms"] * 1e-3) / 1e9, "hbm_frac": db / (dc["ms"] * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+        if "sweep" in lg:
+            hb = peaks["hbm_gbs"]
+            tf = peaks["bf16_tflops"]
+            line["sweep"] = [
+                {"B": g["B"], "T": g["T"], "chunked_ms": g["chunked_ms"], "quadratic_ms": g["quadratic_ms"],
+                 "chunked_tokens_per_s": g["B"] * g["T"] / (g["chunked_ms"] * 1e-3),
+                 "quadratic_tokens_per_s": g["B"] * g["T"] / (g["quadratic_ms"] * 1e-3),
+                 "chunked_hbm_frac": chunked_bytes(g["B"] * 16, g["T"], 16, 64) / (g["chunked_ms"] * 1e-3) / 1e9 / hb,
+                 "quadratic_tensor_frac": flash_flops(g["B"] * 16, g["T"], 16, 64) / (g["quadratic_ms"] * 1e-3) / 1e12
+                 / tf} for g in lg["sweep"]]
+            rc = lg["recall"]
+            rtok = rc["B"] * rc["T"]
+            line["recall_p32"] = {
+                "workload": "recall-shaped keys B=%d H=%d T=%d p=%d dv=%d bf16" % (rc["B"], rc["H"], rc["T"], rc["p"],
+                                                                                 rc["dv"]),
+                "chunked": {"ms": rc["chunked_ms"], "tokens_per_s": rtok / (rc["chunked_ms"] * 1e-3)},
+                "quadratic": {"ms": rc["quadratic_ms"], "tokens_per_s": rtok / (rc["quadratic_ms"] * 1e-3),
+                              "tensor_frac": flash_flops(rc["B"] * rc["H"], rc["T"], rc["p"], rc["dv"])
+                              / (rc["quadratic_ms"] * 1e-3) / 1e12 / tf}}
     if args.cpu_baseline and world == 1:
         cb = time_oracle(cfg)
         line["cpu_baseline"] = {"value": cb["value"], "unit": UNIT, "cores": cb["cores"], "kind": "oracle",

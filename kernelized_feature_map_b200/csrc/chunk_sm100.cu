@@ -814,17 +814,19 @@ __global__ void __launch_bounds__(kReadThreads, 1)
           uint32_t r[32];
           tmem_ld32(lane_base + L::colS + 32 * bb, r);
           tmem_wait_ld();
+          // squares on fp32 pairs (each rounded as a scalar multiply)
           if (bb < quarter) {
 #pragma unroll
             for (int x = 0; x < 16; ++x) {
-              const float s0 = __uint_as_float(r[2 * x]), s1 = __uint_as_float(r[2 * x + 1]);
-              w[x] = pack_bf16x2(s0 * s0, s1 * s1);
+              const uint64_t sq = f32x2_mul(f32x2(r[2 * x], r[2 * x + 1]), f32x2(r[2 * x], r[2 * x + 1]));
+              w[x] = pack_bf16x2(f32x2_lo(sq), f32x2_hi(sq));
             }
           } else {
 #pragma unroll
             for (int x = 0; x < 16; ++x) {
-              const float s0 = __uint_as_float(r[2 * x]), s1 = __uint_as_float(r[2 * x + 1]);
-              w[x] = pack_bf16x2(2 * x > lane ? 0.f : s0 * s0, 2 * x + 1 > lane ? 0.f : s1 * s1);
+              const uint32_t a = 2 * x > lane ? 0u : r[2 * x], b = 2 * x + 1 > lane ? 0u : r[2 * x + 1];
+              const uint64_t sq = f32x2_mul(f32x2(a, b), f32x2(a, b));
+              w[x] = pack_bf16x2(f32x2_lo(sq), f32x2_hi(sq));
             }
           }
         }
@@ -850,16 +852,16 @@ __global__ void __launch_bounds__(kReadThreads, 1)
       if (t < t1) {
         const float D = __uint_as_float(db);
         const float inv = D > 0.f ? 1.f / D : 0.f;
+        const uint64_t inv2 = f32x2(__float_as_uint(inv), __float_as_uint(inv));
         uint4* dst = reinterpret_cast<uint4*>(o + ((size_t)bh * T + t) * kDV);
+        auto scaled = [&](const uint32_t* src, int k) {
+          const uint64_t v = f32x2_mul(f32x2(src[k], src[k + 1]), inv2);
+          return pack_bf16x2(f32x2_lo(v), f32x2_hi(v));
+        };
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const uint32_t* src = (e < 4) ? r0 + 8 * e : r1 + 8 * (e - 4);
-          uint4 u;
-          u.x = pack_bf16x2(__uint_as_float(src[0]) * inv, __uint_as_float(src[1]) * inv);
-          u.y = pack_bf16x2(__uint_as_float(src[2]) * inv, __uint_as_float(src[3]) * inv);
-          u.z = pack_bf16x2(__uint_as_float(src[4]) * inv, __uint_as_float(src[5]) * inv);
-          u.w = pack_bf16x2(__uint_as_float(src[6]) * inv, __uint_as_float(src[7]) * inv);
-          dst[e] = u;
+          dst[e] = make_uint4(scaled(src, 0), scaled(src, 2), scaled(src, 4), scaled(src, 6));
         }
       }
     }

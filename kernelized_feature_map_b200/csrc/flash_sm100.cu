@@ -368,15 +368,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float inv = D > 0.f ? 1.f / D : 0.f;
       if (t < T) {
         uint4* dst = reinterpret_cast<uint4*>(o + ((size_t)bh * T + t) * DV + kHalf * h);
+        const uint64_t inv2 = f32x2(__float_as_uint(inv), __float_as_uint(inv));
+        auto scaled = [&](int k) {
+          const uint64_t v = f32x2_mul(f32x2(ov[k], ov[k + 1]), inv2);
+          return pack_bf16x2(f32x2_lo(v), f32x2_hi(v));
+        };
 #pragma unroll
-        for (int e = 0; e < kHalf / 8; ++e) {
-          uint4 u;
-          u.x = pack_bf16x2(__uint_as_float(ov[8 * e + 0]) * inv, __uint_as_float(ov[8 * e + 1]) * inv);
-          u.y = pack_bf16x2(__uint_as_float(ov[8 * e + 2]) * inv, __uint_as_float(ov[8 * e + 3]) * inv);
-          u.z = pack_bf16x2(__uint_as_float(ov[8 * e + 4]) * inv, __uint_as_float(ov[8 * e + 5]) * inv);
-          u.w = pack_bf16x2(__uint_as_float(ov[8 * e + 6]) * inv, __uint_as_float(ov[8 * e + 7]) * inv);
-          dst[e] = u;
-        }
+        for (int e = 0; e < kHalf / 8; ++e)
+          dst[e] = make_uint4(scaled(8 * e), scaled(8 * e + 2), scaled(8 * e + 4), scaled(8 * e + 6));
       }
     }
   }
