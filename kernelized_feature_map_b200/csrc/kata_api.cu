@@ -47,12 +47,16 @@ WaitCtl wait_ctl() { return WaitCtl{status_word(), wait_limit()}; }
 // Super-chunk length.  One CTA handles one (b,h, super-chunk) unit, 148 SMs
 // run one unit each per wave, and every unit costs its chunks plus a fixed
 // overhead (prologue, state record written, scanned and read back), counted
-// as kUnitOverhead chunks.  The plan takes the multiple of 128 tokens that
-// minimises  waves * (chunks per unit + kUnitOverhead),  preferring longer
-// super-chunks (fewer records) on ties.  A pure function of the sizes, so
-// that the workspace query and the call agree.
+// as kUnitOverhead chunks.  On the tensor-core path a single super-chunk per
+// (b,h) needs one launch instead of three (no state build, no scan), so
+// splitting costs a further kSplitOverhead chunks (two launches with their
+// prologues, measured at about that much).  The plan takes the multiple of 128
+// tokens that minimises  waves * (chunks per unit + kUnitOverhead) [+ split],
+// preferring longer super-chunks (fewer records) on ties.  A pure function of
+// the sizes, so that the workspace query and the call agree.
 constexpr int kSMs = 148;
 constexpr int kUnitOverhead = 2;
+constexpr int kSplitOverhead = 8;
 
 ChunkPlan make_chunk_plan(int B, int H, int T, int p, int dv, int C, kata_dtype_t dt) {
   ChunkPlan pl{};
@@ -64,13 +68,16 @@ ChunkPlan make_chunk_plan(int B, int H, int T, int p, int dv, int C, kata_dtype_
   pl.ld = dv + 4;
   pl.C = C;
   pl.Ls = 128;
+  pl.layout = chunked_on_tensor_cores(p, dv, dt) ? kRecPackedT : kRecUnpacked;
   const long long tiles = (T + 127) / 128;
   long long best = -1;
   const long long kmax = tiles < 1 ? 1 : (tiles < 512 ? tiles : 512);  // super-chunks up to 64K tokens
   for (long long k = kmax; k >= 1; --k) {
-    const long long units = (long long)pl.BH * ((tiles + k - 1) / k);
+    const long long per_bh = (tiles + k - 1) / k;
+    const long long units = (long long)pl.BH * per_bh;
     const long long waves = (units + kSMs - 1) / kSMs;
-    const long long cost = waves * (k + kUnitOverhead);
+    const long long split = (pl.layout == kRecPackedT && per_bh > 1) ? kSplitOverhead : 0;
+    const long long cost = waves * (k + kUnitOverhead) + split;
     if (best < 0 || cost < best) {
       best = cost;
       pl.Ls = (int)(k * 128);
@@ -78,7 +85,6 @@ ChunkPlan make_chunk_plan(int B, int H, int T, int p, int dv, int C, kata_dtype_
   }
   if (pl.Ls < C) pl.Ls = C;
   pl.G = T > 0 ? (T + pl.Ls - 1) / pl.Ls : 0;
-  pl.layout = chunked_on_tensor_cores(p, dv, dt) ? kRecPackedT : kRecUnpacked;
   pl.record_floats = pl.layout == kRecPackedT ? (size_t)(dv + 1) * 144 : (size_t)pl.P * pl.ld;
   // the tensor-core path needs no records for a single super-chunk
   const bool no_records = pl.layout == kRecPackedT && pl.G <= 1;
