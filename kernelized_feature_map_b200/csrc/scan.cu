@@ -10,12 +10,13 @@
 // O(log G) (gist.science technical summary, sec. 2.3 "Chunked Parallelism" /
 // "Complexiteitsreductie": recurrence depth O(N_C) -> O(log N_C)).
 //
-// Work decomposition: one CTA per (b,h) and column block of NC record
-// entries; the [G x NC] tile sits in shared memory (at most 1024 records per
-// pass; longer sequences are scanned in blocks of 1024 with a running carry)
-// and the 256 threads share every tree level.  NC is chosen so that a tile is
-// about 32 KiB: the kernel streams every record once in and once out and is
-// bound by HBM.
+// Work decomposition.  Up to 32 records per (b,h): one thread per record
+// column runs the tree over that column's records in registers.  More
+// records: one CTA per (b,h) and column block of NC record entries; the
+// [G x NC] tile sits in shared memory (at most 1024 records per pass; longer
+// sequences are scanned in blocks of 1024 with a running carry) and the 256
+// threads share every tree level.  NC is chosen so that a tile is about
+// 32 KiB.  Either way every record is streamed once in and once out.
 //
 // Record layouts (per (b,h), per super-chunk g), see kata_internal.h:
 //   kRecUnpacked  P rows x ld floats: columns 0..dv-1 = sum psi(k) v^T,
@@ -208,6 +209,44 @@ __global__ void __launch_bounds__(kScanThreads) state_scan_kernel(ScanArgs a) {
       if (col0 + c < a.E) final_entry(a, bh, col0 + c, carry[c]);
 }
 
+// Few records per (b,h): the same up-sweep / down-sweep tree (depth log2 GP),
+// over one record column per thread held in registers.  Consecutive threads
+// take consecutive columns, so every record row is read and written
+// coalesced, and no shared memory or block barrier is needed.
+constexpr int kScanRegThreads = 256;
+
+template <int GP>
+__global__ void __launch_bounds__(kScanRegThreads) state_scan_reg_kernel(ScanArgs a) {
+  const int col = blockIdx.x * kScanRegThreads + threadIdx.x;
+  const long long bh = blockIdx.y;
+  if (col >= a.E) return;
+  float* base = a.ws + bh * (long long)a.G * a.E + col;
+  float x[GP];
+#pragma unroll
+  for (int g = 0; g < GP; ++g) x[g] = (g < a.G_in) ? __ldcs(base + (long long)g * a.E) : 0.f;
+  const float carry = a.S0 ? initial_entry(a, bh, col) : 0.f;
+  // up-sweep: x[(2i+2)d - 1] += x[(2i+1)d - 1]
+#pragma unroll
+  for (int d = 1; d < GP; d <<= 1)
+#pragma unroll
+    for (int i = 2 * d - 1; i < GP; i += 2 * d) x[i] += x[i - d];
+  const float total = x[GP - 1];
+  x[GP - 1] = 0.f;
+  // down-sweep
+#pragma unroll
+  for (int d = GP >> 1; d >= 1; d >>= 1)
+#pragma unroll
+    for (int i = 2 * d - 1; i < GP; i += 2 * d) {
+      const float t = x[i - d];
+      x[i - d] = x[i];
+      x[i] += t;
+    }
+#pragma unroll
+  for (int g = 0; g < GP; ++g)
+    if (g < a.G) base[(long long)g * a.E] = carry + x[g];
+  if (a.S_out) final_entry(a, bh, col, carry + total);
+}
+
 cudaError_t launch_state_scan(float* ws, const ChunkPlan& plan, int G_in, const float* S0, const float* z0,
                               float* S_out, float* z_out, cudaStream_t st) {
   if (plan.layout == kRecPackedT) {
@@ -233,6 +272,15 @@ cudaError_t launch_state_scan(float* ws, const ChunkPlan& plan, int G_in, const 
   a.z0 = z0;
   a.S_out = S_out;
   a.z_out = z_out;
+  if (plan.G <= 32) {
+    dim3 grid(ceil_div(a.E, kScanRegThreads), plan.BH);
+    if (plan.G <= 2) state_scan_reg_kernel<2><<<grid, kScanRegThreads, 0, st>>>(a);
+    else if (plan.G <= 4) state_scan_reg_kernel<4><<<grid, kScanRegThreads, 0, st>>>(a);
+    else if (plan.G <= 8) state_scan_reg_kernel<8><<<grid, kScanRegThreads, 0, st>>>(a);
+    else if (plan.G <= 16) state_scan_reg_kernel<16><<<grid, kScanRegThreads, 0, st>>>(a);
+    else state_scan_reg_kernel<32><<<grid, kScanRegThreads, 0, st>>>(a);
+    return cudaGetLastError();
+  }
   const size_t smem = ((size_t)a.Gp * a.NC + 2 * (size_t)a.NC) * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(state_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
