@@ -253,34 +253,70 @@ def run_ours(args, rank, world, local_rank):
     step_ms = float(per.sum(axis=1).mean())
     path_ms = per.mean(axis=0)
 
-    # end to end through the public API with host buffers: H2D of the step's
-    # inputs from pinned memory, the three calls, D2H of the three outputs
-    ho_quad = torch.empty(o_quad.shape, dtype=bf).pin_memory()
-    ho_chunk = torch.empty(o_chunk.shape, dtype=bf).pin_memory()
-    ho_dec = torch.empty(o_dec.shape, dtype=bf).pin_memory()
+    # end to end through the public API with host buffers.  Every step copies
+    # its inputs host -> device from pinned memory, runs the three calls and
+    # copies its three outputs device -> host.  Steps are pipelined over three
+    # streams with two sets of device buffers: the H2D copy of step i, the
+    # compute of step i-1 and the D2H copy of step i-2 overlap (PCIe is full
+    # duplex and the copy engines run beside the SMs).  The L2 is flushed on
+    # the compute stream before every step.
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdq, hdk, hdv))
-    d2h = sum(t.numel() * t.element_size() for t in (ho_quad, ho_chunk, ho_dec))
+    d2h = sum(t.numel() * t.element_size() for t in (o_quad, o_chunk, o_dec))
+    sets = []
+    for _b in range(2):
+        sets.append(dict(
+            q=torch.empty_like(q), k=torch.empty_like(k), v=torch.empty_like(v),
+            qd=torch.empty_like(qd), kd=torch.empty_like(kd), vd=torch.empty_like(vd),
+            oq=torch.empty_like(o_quad), oc=torch.empty_like(o_chunk), od=torch.empty_like(o_dec),
+            S=torch.empty_like(S), z=torch.empty_like(z), ws=torch.empty_like(ws),
+            hoq=torch.empty(o_quad.shape, dtype=bf).pin_memory(), hoc=torch.empty(o_chunk.shape, dtype=bf).pin_memory(),
+            hod=torch.empty(o_dec.shape, dtype=bf).pin_memory()))
+    s_h2d, s_cmp, s_d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_cmp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
 
-    def e2e_step():
-        q.copy_(hq, non_blocking=True); k.copy_(hk, non_blocking=True); v.copy_(hv, non_blocking=True)
-        qd.copy_(hdq, non_blocking=True); kd.copy_(hdk, non_blocking=True); vd.copy_(hdv, non_blocking=True)
-        step()
-        ho_quad.copy_(o_quad, non_blocking=True); ho_chunk.copy_(o_chunk, non_blocking=True)
-        ho_dec.copy_(o_dec, non_blocking=True)
+    def e2e_run(nsteps):
+        for i in range(nsteps):
+            bi = i % 2
+            st_ = sets[bi]
+            with torch.cuda.stream(s_h2d):
+                if i >= 2:
+                    s_h2d.wait_event(ev_cmp[bi])  # step i-2 has finished reading this set's inputs
+                for dst, src in ((st_["q"], hq), (st_["k"], hk), (st_["v"], hv), (st_["qd"], hdq), (st_["kd"], hdk),
+                                 (st_["vd"], hdv)):
+                    dst.copy_(src, non_blocking=True)
+                ev_in[bi].record(s_h2d)
+            with torch.cuda.stream(s_cmp):
+                s_cmp.wait_event(ev_in[bi])
+                if i >= 2:
+                    s_cmp.wait_event(ev_out[bi])  # step i-2's outputs have been copied out
+                flush.fill_(1)
+                K.kata_fwd_quadratic(st_["q"], st_["k"], st_["v"], o=st_["oq"])
+                K.kata_fwd_chunked(st_["q"], st_["k"], st_["v"], C=C, o=st_["oc"], workspace=st_["ws"],
+                                   S_out=st_["S"], z_out=st_["z"], return_state=True)
+                K.kata_decode_step(st_["qd"], st_["kd"], st_["vd"], st_["S"], st_["z"], o=st_["od"])
+                ev_cmp[bi].record(s_cmp)
+            with torch.cuda.stream(s_d2h):
+                s_d2h.wait_event(ev_cmp[bi])
+                st_["hoq"].copy_(st_["oq"], non_blocking=True)
+                st_["hoc"].copy_(st_["oc"], non_blocking=True)
+                st_["hod"].copy_(st_["od"], non_blocking=True)
+                ev_out[bi].record(s_d2h)
 
-    for _ in range(2):
-        e2e_step()
+    e2e_run(4)
     torch.cuda.synchronize()
-    e2e_ms = []
-    for _ in range(min(20, max(3, args.steps // 2))):
-        a, b = ev(), ev()
-        flush.fill_(1)
-        a.record(stream)
-        e2e_step()
-        b.record(stream)
-        torch.cuda.synchronize()
-        e2e_ms.append(a.elapsed_time(b))
-    e2e_ms = float(np.mean(e2e_ms))
+    n_e2e = min(40, max(8, args.steps // 2))
+    e_start, e_end = ev(), ev()
+    e_start.record(s_h2d)
+    s_cmp.wait_stream(s_h2d)
+    s_d2h.wait_stream(s_h2d)
+    e2e_run(n_e2e)
+    s_d2h.wait_stream(s_cmp)
+    s_d2h.wait_stream(s_h2d)
+    e_end.record(s_d2h)
+    torch.cuda.synchronize()
+    e2e_ms = e_start.elapsed_time(e_end) / n_e2e
 
     # long context: chunked (and quadratic) at T = 131072
     long = None
