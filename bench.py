@@ -45,6 +45,27 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 METRIC = "KATA-Mg fwd tokens/sec at T=2k and 131k (1 B200); % of roofline"
 UNIT = "tokens/s"
 
+# DRAM bytes (read + write) of one flash_fwd_kernel launch at B8 H16 T2048,
+# from the ncu capture summarised in profiles/flash_fwd_kernel_ctx2k.md.  It
+# is reported only while the kernel's sources are the ones that capture ran.
+FLASH_TRAFFIC_BYTES = 50441728 + 3565824
+FLASH_TRAFFIC_SOURCES = ("kernelized_feature_map_b200/csrc/flash_sm100.cu", "kernelized_feature_map_b200/csrc/sm100.cuh",
+                         "kernelized_feature_map_b200/csrc/kata_trace.cuh")
+FLASH_TRAFFIC_SHA256 = "20a25228a5551f3834785d483e0ef1f6d2070859812d2c208674fef43ab3fafb"
+
+
+def flash_traffic(workload):
+    """Measured per-launch DRAM traffic of the flash kernel, or None when the
+    workload or the kernel sources differ from those of the capture."""
+    import hashlib
+    if workload != "layer340m_ctx2k":
+        return None
+    h = hashlib.sha256()
+    for rel in FLASH_TRAFFIC_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as fh:
+            h.update(fh.read())
+    return FLASH_TRAFFIC_BYTES if h.hexdigest() == FLASH_TRAFFIC_SHA256 else None
+
 
 def launches_per_step(B, H, T, p, dv, C):
     """Kernels one step launches: flash 1, decode 1, and the chunked call's
@@ -576,7 +597,7 @@ def report(args, res, step_ms, e2e_ms, world):
         },
         "roofline": {"kernel": "flash_fwd_kernel (kata_fwd_quadratic)", "bound": "tensor", "achieved": achieved,
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
-                     "traffic": None, "peak_source": peak_src + " (bf16 burst)",
+                     "traffic": flash_traffic(args.workload), "peak_source": peak_src + " (bf16 burst)",
                      "algorithmic": "%.4g causal-useful flops per launch" % fl},
         "e2e": {"value": tokens_all / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": res["h2d"],
                 "d2h_bytes_per_step": res["d2h"]},
