@@ -81,8 +81,11 @@ kata_status_t kata_fwd_quadratic(const void* q, const void* k, const void* v, vo
                                  kata_dtype_t dtype, void* stream);
 
 /*
- * Bytes of device workspace kata_fwd_chunked needs for these sizes (0 when
- * T == 0).  The same arguments must be passed to kata_fwd_chunked.
+ * Bytes of device workspace kata_fwd_chunked needs for these sizes: 0 when
+ * T == 0, and on the tensor-core path (bf16, p = 16, dv = 64) whenever each
+ * (b,h) sequence is handled as a single super-chunk; otherwise one fp32
+ * state record per (b,h) per super-chunk.  A pure function of the arguments;
+ * the same arguments must be passed to kata_fwd_chunked.
  */
 size_t kata_fwd_chunked_workspace_size(int B, int H, int T, int p, int dv, int C,
                                        kata_dtype_t dtype);
@@ -105,7 +108,10 @@ size_t kata_fwd_chunked_workspace_size(int B, int H, int T, int p, int dv, int C
  *            both NULL means a zero state; exactly one NULL is an error.
  * S_out,z_out optional state after token T (same layouts); both or neither.
  * workspace  device buffer of at least kata_fwd_chunked_workspace_size()
- *            bytes, 256-byte aligned; contents on entry are ignored.
+ *            bytes, 256-byte aligned; contents on entry are ignored.  When
+ *            that size is 0 (every sequence fits one super-chunk of the
+ *            plan, the normal case for short sequences on the tensor-core
+ *            path) workspace may be NULL and workspace_bytes 0.
  */
 kata_status_t kata_fwd_chunked(const void* q, const void* k, const void* v, void* o,
                                int B, int H, int T, int p, int dv, int C,

@@ -24,15 +24,18 @@
 // shared memory.  The workspace record of a super-chunk is rows 0..64 of it
 // (65 x 144 fp32).
 //
-// Three launches per call:
-//  1. chunk_state_kernel    per super-chunk g: A_g = sum over its chunks;
-//  2. state_scan_kernel     (scan.cu) exclusive prefix over g, depth O(log G);
+// Launches per call, with G super-chunks per (b,h):
+//  1. chunk_state_kernel    (G > 1) per super-chunk g < G-1: A_g = sum over
+//                           its chunks (nothing reads the last one's sum);
+//  2. state_scan            (G > 1, scan.cu) exclusive prefix over g, depth
+//                           O(log G);
 //  3. chunk_readout_kernel  per super-chunk, per 128-token chunk c:
 //        [O | D] = psi~(Q_c) S~          readout, K = 144, B = bf16 copy of S~
 //                + W_c [V_c | 1]         W = (Q_c K_c^T)^2, causal
 //        S~^T   += [V_c | 1]^T psi~(K_c) advance
 //        o_c     = O / D
-//     with S~ starting at the scanned prefix.
+//     with S~ starting at the scanned prefix (G = 1: at the caller's initial
+//     state, or zero); the CTA of the last super-chunk writes the final state.
 #include <cuda.h>
 
 #include "kata_internal.h"
