@@ -397,6 +397,9 @@ def run_long(args, K, torch, dev, stream, flush):
             if i >= 3:
                 ms.append(a.elapsed_time(b))
         out["chunked_C%d_ms" % C] = float(np.mean(ms))
+    # sequential inter-chunk baseline: one CTA per (b,h) walks all chunks
+    out["sequential_C64_ms"] = _time_call(lambda: K.kata_fwd_chunked_sequential(q, k, v, C=64, o=o), flush, stream,
+                                          3, 1)
     ms = []
     for i in range(2 + max(1, args.long_steps // 4)):
         flush.fill_(1)
@@ -619,6 +622,9 @@ def report(args, res, step_ms, e2e_ms, world):
                              "hbm_frac": lb / (lg["chunked_C128_ms"] * 1e-3) / 1e9 / peaks["hbm_gbs"]},
             "quadratic": {"ms": lg["quadratic_ms"], "tokens_per_s": ltok / (lg["quadratic_ms"] * 1e-3),
                           "tensor_frac": lf / (lg["quadratic_ms"] * 1e-3) / 1e12 / peaks["bf16_tflops"]},
+            "sequential_C64": {"ms": lg["sequential_C64_ms"],
+                               "tokens_per_s": ltok / (lg["sequential_C64_ms"] * 1e-3),
+                               "scan_speedup": lg["sequential_C64_ms"] / lg["chunked_C64_ms"]},
         }
         dc = lg["decode_b64"]
         db = decode_bytes(dc["B"] * dc["H"], dc["p"], dc["dv"])

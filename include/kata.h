@@ -144,6 +144,26 @@ kata_status_t kata_fwd_chunked_noalloc(const void* q, const void* k, const void*
                                        float* S_out, float* z_out, void* stream);
 
 /*
+ * Sequential inter-chunk baseline: the chunked forward with every (b,h)
+ * sequence handled by one CTA that walks all of its chunks in order,
+ * carrying the state from chunk to chunk (a depth-O(T/C) recurrence), with
+ * no super-chunk sums and no associative scan.  It exists to measure what
+ * the scan of kata_fwd_chunked buys (the pages compare their scan against a
+ * sequential linear-attention baseline: gist.science sec. 2.3; KATA
+ * repository README, Figure 3).  Results equal kata_fwd_chunked's up to
+ * rounding.
+ *
+ * Arguments, layouts and errors as kata_fwd_chunked, without a workspace.
+ * Only the tensor-core configuration (bf16, p = 16, dv = 64) is supported;
+ * other sizes return KATA_ERR_UNSUPPORTED.
+ */
+kata_status_t kata_fwd_chunked_sequential(const void* q, const void* k, const void* v, void* o,
+                                          int B, int H, int T, int p, int dv, int C,
+                                          kata_dtype_t dtype,
+                                          const float* S0, const float* z0,
+                                          float* S_out, float* z_out, void* stream);
+
+/*
  * One recurrent decode step for B*H independent streams (constant-time
  * recurrent inference on the fixed-size state; arXiv abstract on aiqbench):
  *   S <- S + psi(k) v^T,  z <- z + psi(k),  o = psi(q)^T S / psi(q)^T z

@@ -11,8 +11,11 @@ The computation lives in ``libkata.so`` (hand-written CUDA behind the C ABI of
   associative scan across chunks;
 * :func:`kata_decode_step`   -- one recurrent step on the fixed-size state;
 * :func:`kata_fwd_chunked_noalloc` -- the chunked forward using a fixed
-  library-owned scratch array, for callers that cannot allocate.
+  library-owned scratch array, for callers that cannot allocate;
+* :func:`kata_fwd_chunked_sequential` -- the sequential inter-chunk baseline
+  (one CTA per sequence walks its chunks in order, no scan).
 """
 from ._abi import (KataError, kata_abi_version, kata_decode_step, kata_fwd_chunked,  # noqa: F401
-                   kata_fwd_chunked_noalloc, kata_fwd_chunked_workspace_size, kata_fwd_quadratic,
+                   kata_fwd_chunked_noalloc, kata_fwd_chunked_sequential, kata_fwd_chunked_workspace_size,
+                   kata_fwd_quadratic,
                    kata_get_status, kata_set_wait_limit, lib, status_string)

@@ -28,6 +28,8 @@ SIGNATURES = {
                                   _fp, _fp, _fp, _fp, _vp, _c_size, _vp]),
     "kata_fwd_chunked_noalloc": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                           _c_int, _fp, _fp, _fp, _fp, _vp]),
+    "kata_fwd_chunked_sequential": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                             _c_int, _fp, _fp, _fp, _fp, _vp]),
     "kata_decode_step": (_c_int, [_vp, _vp, _vp, _vp, _fp, _fp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp]),
     "kata_get_status": (_c_int, [_vp]),
     "kata_status_string": (ctypes.c_char_p, [_c_int]),
@@ -164,6 +166,26 @@ def kata_fwd_chunked_noalloc(q, k, v, C=64, S0=None, z0=None, return_state=False
         S_out = torch.empty((B, H, p * p, dv), dtype=torch.float32, device=dev)
         z_out = torch.empty((B, H, p * p), dtype=torch.float32, device=dev)
     _check("kata_fwd_chunked_noalloc", lib().kata_fwd_chunked_noalloc(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), B, H, T, p, dv, C, _dtype_code(q),
+        _opt(S0, "S0"), _opt(z0, "z0"), _opt(S_out, "S_out"), _opt(z_out, "z_out"), _stream_ptr(stream)))
+    if return_state:
+        return o, S_out, z_out
+    return o
+
+
+def kata_fwd_chunked_sequential(q, k, v, C=64, S0=None, z0=None, return_state=False, o=None, S_out=None,
+                                z_out=None, stream=None):
+    """Sequential inter-chunk baseline: one CTA per (b,h) walks all of its
+    chunks in order (no super-chunk sums, no scan).  bf16, p=16, dv=64 only."""
+    B, H, T, p = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    if o is None:
+        o = torch.empty((B, H, T, dv), dtype=q.dtype, device=dev)
+    if return_state and S_out is None:
+        S_out = torch.empty((B, H, p * p, dv), dtype=torch.float32, device=dev)
+        z_out = torch.empty((B, H, p * p), dtype=torch.float32, device=dev)
+    _check("kata_fwd_chunked_sequential", lib().kata_fwd_chunked_sequential(
         _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), B, H, T, p, dv, C, _dtype_code(q),
         _opt(S0, "S0"), _opt(z0, "z0"), _opt(S_out, "S_out"), _opt(z_out, "z_out"), _stream_ptr(stream)))
     if return_state:

@@ -212,6 +212,31 @@ KATA_API kata_status_t kata_fwd_chunked(const void* q, const void* k, const void
   return from_cuda(e);
 }
 
+KATA_API kata_status_t kata_fwd_chunked_sequential(const void* q, const void* k, const void* v, void* o, int B,
+                                                   int H, int T, int p, int dv, int C, kata_dtype_t dtype,
+                                                   const float* S0, const float* z0, float* S_out, float* z_out,
+                                                   void* stream) {
+  kata_status_t s = check_common(B, H, T, p, dv, dtype);
+  if (s != KATA_OK) return s;
+  if (!(C == 64 || C == 128)) return KATA_ERR_UNSUPPORTED;
+  if (!chunked_on_tensor_cores(p, dv, dtype)) return KATA_ERR_UNSUPPORTED;
+  if ((S0 == nullptr) != (z0 == nullptr)) return KATA_ERR_INVALID_ARG;
+  if ((S_out == nullptr) != (z_out == nullptr)) return KATA_ERR_INVALID_ARG;
+  for (const void* ptr : {(const void*)S0, (const void*)z0, (const void*)S_out, (const void*)z_out})
+    if (ptr && !aligned16(ptr)) return KATA_ERR_MISALIGNED;
+  if (T == 0) return kata_fwd_chunked(q, k, v, o, B, H, T, p, dv, C, dtype, S0, z0, S_out, z_out, nullptr, 0, stream);
+  if (!q || !k || !v || !o) return KATA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return KATA_ERR_MISALIGNED;
+  // one super-chunk per (b,h): one CTA walks every chunk of its sequence in
+  // order, carrying the state; no state build, no scan, no workspace
+  ChunkPlan plan = make_chunk_plan(B, H, T, p, dv, C, dtype);
+  plan.Ls = ((T + 127) / 128) * 128;
+  plan.G = 1;
+  plan.workspace_bytes = 0;
+  return from_cuda(launch_chunk_readout_sm100(q, k, v, o, nullptr, S0, z0, S_out, z_out, plan, wait_ctl(),
+                                              static_cast<cudaStream_t>(stream)));
+}
+
 KATA_API kata_status_t kata_decode_step(const void* q, const void* k, const void* v, void* o, float* S, float* z,
                                         int B, int H, int p, int dv, kata_dtype_t dtype, void* stream) {
   kata_status_t s = check_common(B, H, 1, p, dv, dtype);

@@ -102,6 +102,11 @@ def test_argument_errors_before_launch(L):
     assert g(a, b, c, d, 1, 16, 131072, 16, 64, 64, 1, None, None, None, None, _fake(0x50010), 1 << 30,
              st) == _abi.KATA_ERR_MISALIGNED
     assert g(a, b, c, d, 1, 1, 0, 16, 64, 64, 1, None, None, None, None, None, 0, st) == _abi.KATA_OK
+    sq = L.kata_fwd_chunked_sequential
+    assert sq(a, b, c, d, 1, 1, 16, 16, 64, 64, 0, None, None, None, None, st) == _abi.KATA_ERR_UNSUPPORTED  # fp32
+    assert sq(a, b, c, d, 1, 1, 16, 32, 64, 64, 1, None, None, None, None, st) == _abi.KATA_ERR_UNSUPPORTED  # p=32
+    assert sq(a, b, c, d, 1, 1, 16, 16, 64, 96, 1, None, None, None, None, st) == _abi.KATA_ERR_UNSUPPORTED  # C
+    assert sq(a, b, c, d, 1, 1, 16, 16, 64, 64, 1, _fake(0x60000), None, None, None, st) == _abi.KATA_ERR_INVALID_ARG
     h = L.kata_decode_step
     assert h(a, b, c, d, _fake(0x70000), None, 1, 1, 16, 64, 1, st) == _abi.KATA_ERR_INVALID_ARG
     assert h(a, b, c, d, _fake(0x70000), _fake(0x80000), 1, 1, 24, 64, 1, st) == _abi.KATA_ERR_UNSUPPORTED

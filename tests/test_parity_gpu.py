@@ -172,6 +172,24 @@ def test_chunked_state_in_and_out(kata, dtype, B, H, T, t0):
     assert row_rel_err(to_np(o2), o_ref[:, :, t0:], v) <= TOL[dtype]
 
 
+# the sequential inter-chunk baseline: one CTA walks each sequence's chunks
+@pytest.mark.parametrize("B,H,T", [(1, 2, 1000), (2, 3, 2500)])
+def test_sequential_baseline_matches_oracle(kata, B, H, T):
+    import torch
+    p, dv = 16, 64
+    q, k, v = workloads.normal_qkv(B, H, T, p, dv, seed=31, dtype="bf16")
+    o_ref, S_ref, z_ref = oracle.recurrent(q, k, v, return_state=True)
+    _, S_abs, z_abs = oracle.recurrent(np.abs(q), np.abs(k), np.abs(v), return_state=True, need_output=False)
+    eps = 2.0 ** -8 + (T + 4) * 2.0 ** -24  # as in test_chunked_state_in_and_out
+    o, S, z = kata.kata_fwd_chunked_sequential(to_dev(q, "bf16"), to_dev(k, "bf16"), to_dev(v, "bf16"),
+                                               return_state=True)
+    torch.cuda.synchronize()
+    assert kata.kata_get_status() == 0
+    assert row_rel_err(to_np(o), o_ref, v) <= TOL["bf16"]
+    assert np.all(np.abs(S.cpu().numpy() - S_ref) <= eps * S_abs + 1e-6)
+    assert np.all(np.abs(z.cpu().numpy() - z_ref) <= eps * z_abs + 1e-6)
+
+
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("p,dv", [(16, 64), (16, 16), (32, 64), (32, 16)])
 def test_decode_step(kata, dtype, p, dv):
