@@ -519,27 +519,27 @@ __global__ void __launch_bounds__(kStateThreads, 1)
         mbar_wait_drain(kv_full + c % kStateStages, (c / kStateStages) & 1, wc.limit);
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    {  // whole warp; one elected lane issues
       constexpr uint32_t id_u = idesc_bf16(128, kNP, true, true);
       const uint32_t sStage = smem_u32(smem + L::offStage), sOnes = smem_u32(smem + L::offOnes);
       const uint32_t sPsi = smem_u32(smem + L::offPsi);
       const uint64_t dpsi = smem_desc(sPsi, kPsiAtom, 256, kSw32);
       for (int c = 0; c < n_chunks; ++c) {
         const int st = c % kStateStages, pb = c & 1;
-        if (!mbar_wait(kv_full + st, (c / kStateStages) & 1, env)) break;
-        if (!mbar_wait(psi_full + pb, (c >> 1) & 1, env)) break;
+        if (!mbar_wait_w(kv_full + st, (c / kStateStages) & 1, env)) break;
+        if (!mbar_wait_w(psi_full + pb, (c >> 1) & 1, env)) break;
         KATA_TRACE(chunkstate, c, 0);
         tc_fence_after();
         const uint32_t sV = sStage + st * L::kStage;
         const uint64_t da = desc_vones(sV, sOnes), db = desc_add(dpsi, pb * kPsiBytes);
 #pragma unroll
         for (int ks = 0; ks < kTile / 16; ++ks)
-          mma_ss(tmem, desc_add(da, ks * 2048), desc_add(db, ks * 512), id_u, (c > 0 || ks > 0) ? 1u : 0u);
+          mma_ss_w(tmem, desc_add(da, ks * 2048), desc_add(db, ks * 512), id_u, (c > 0 || ks > 0) ? 1u : 0u);
         KATA_TRACE(chunkstate, c, 1);
-        mma_commit(psi_empty + pb);
-        mma_commit(kv_empty + st);
+        mma_commit_w(psi_empty + pb);
+        mma_commit_w(kv_empty + st);
       }
-      mma_commit(acc_done);
+      mma_commit_w(acc_done);
       mbar_wait_drain(acc_done, 0, wc.limit);
     }
   } else {
@@ -596,30 +596,34 @@ __global__ void __launch_bounds__(kStateThreads, 1)
 // 3. readout
 // ===========================================================================
 // Warp roles (448 threads):
-//   warp 0       TMA: [V | Q | K] tiles of each chunk into a 6-stage ring
-//   warp 1       TMEM allocator, MMA issuer (one lane)
+//   warp 0       TMA: [V | Q | K] tiles of each chunk into a 3-stage ring
+//   warp 1       TMEM allocator; MMA issue (the whole warp, one elected lane)
 //   warps 2-5    weights W = (Q K^T)^2 (causal) into TMEM; output o = O / D
-//   warps 6-9    psi~(q) into TMEM, psi~(k) into shared memory; bf16 copy of
-//                packed coordinates 0..71 of the state after each chunk
+//   warps 6-9    psi~(q_c) into TMEM, psi~(k_{c+1}) into shared memory (two
+//                buffers); bf16 copy of packed coordinates 0..71 of the state
+//                after each chunk
 //   warps 10-13  prefix state in; bf16 copy of coordinates 72..143
 // MMA order per chunk c: advance S~ by chunk c, readout of chunk c against
 // the bf16 copy of S~ made before chunk c, intra-chunk weights, then the
 // scores of chunk c+1.  The readout reads only the bf16 copy, so the state
 // can advance first; the copy for chunk c+1 is then refreshed while the
 // readout and intra-chunk MMAs of chunk c run (the copy is double-buffered).
-// The [O | D] accumulator is double-buffered so the readout of chunk c+1
-// does not wait for the output of chunk c to be read.
+// The loop-carried path is advance(c) -> refresh -> advance(c+1); psi~(k_{c+1})
+// is formed into the second buffer while the advance by chunk c runs, so it
+// stays off that path.  The [O | D] accumulator is double-buffered so the
+// readout of chunk c+1 does not wait for the output of chunk c to be read.
 constexpr int kReadThreads = 448;
-constexpr int kReadStages = 5;
+constexpr int kReadStages = 3;
 
 struct ReadSmem {
   static constexpr int kStage = kVBytes + 2 * kQKBytes;  // [V | Q | K]
   static constexpr int offStage = 0;
   static constexpr int offOnes = offStage + kReadStages * kStage;  // 1024-aligned
-  static constexpr int offPsi = offOnes + kOnesBytes;
-  static constexpr int offSB = offPsi + kPsiBytes;     // 2 buffers
-  static constexpr int offBar = offSB + 2 * kSBBytes;
-  static constexpr int kBars = 2 * kReadStages + 12;
+  static constexpr int offPsi = offOnes + kOnesBytes;  // 2 buffers
+  static constexpr int offSB = offPsi + 2 * kPsiBytes;  // 2 buffers
+  static constexpr int offOut = offSB + 2 * kSBBytes;   // output tile staging, 128B swizzle (1024-aligned)
+  static constexpr int offBar = offOut + kVBytes;
+  static constexpr int kBars = 2 * kReadStages + 13;
   static constexpr int offMisc = offBar + kBars * 8;
   static constexpr int kBytes = offMisc + 16 + 1024;
   // TMEM columns (multiples of 16, 512 in total)
@@ -631,7 +635,7 @@ struct ReadSmem {
 
 __global__ void __launch_bounds__(kReadThreads, 1)
     chunk_readout_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                         const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ o,
+                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                          const float* __restrict__ ws, const float* __restrict__ S0, const float* __restrict__ z0,
                          float* __restrict__ S_out, float* __restrict__ z_out, int T, int Ls, int G,
                          long long record_floats, WaitCtl wc) {
@@ -644,8 +648,8 @@ __global__ void __launch_bounds__(kReadThreads, 1)
   uint64_t* s_full = kv_empty + kReadStages;  // scores in TMEM
   uint64_t* p_full = s_full + 1;              // weights written (128)
   uint64_t* fq_full = p_full + 1;             // psi~(Q_c) in TMEM (128)
-  uint64_t* fk_full = fq_full + 1;            // psi~(K_c) in shared memory (128)
-  uint64_t* state_full = fk_full + 1;         // bf16 state copy ready (256)
+  uint64_t* fk_full = fq_full + 1;            // [2] psi~(K_c) in shared memory buffer c % 2 (128)
+  uint64_t* state_full = fk_full + 2;         // bf16 state copy ready (256)
   uint64_t* rd_done = state_full + 1;         // readout of the chunk done
   uint64_t* upd_done = rd_done + 1;           // state advanced by the chunk
   uint64_t* o_full = upd_done + 1;            // [2] [O | D] complete
@@ -672,6 +676,7 @@ __global__ void __launch_bounds__(kReadThreads, 1)
     mbar_init(p_full, 128);
     mbar_init(fq_full, 128);
     mbar_init(fk_full, 128);
+    mbar_init(fk_full + 1, 128);
     mbar_init(state_full, 256);
     mbar_init(rd_done, 1);
     mbar_init(upd_done, 1);
@@ -715,7 +720,8 @@ __global__ void __launch_bounds__(kReadThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA
-    if (lane == 0) {
+    // the whole warp runs this loop; one elected lane issues (see mma_ts_w)
+    {
       constexpr uint32_t id_qk = idesc_bf16(128, 128, false, false);
       constexpr uint32_t id_rd = idesc_bf16(128, 80, false, false);  // A = psi~(Q) (TMEM), B = S~ K-major
       constexpr uint32_t id_wv = idesc_bf16(128, 80, false, true);   // A = W (TMEM), B = [V | 1]
@@ -728,10 +734,10 @@ __global__ void __launch_bounds__(kReadThreads, 1)
       const uint64_t dpsi = smem_desc(sPsi, kPsiAtom, 256, kSw32);
       const uint64_t dsb0 = smem_desc(sSB, 16, 256, kSw32);
       auto issue_qk = [&](int st) {
-        mma_ss(tmem + L::colS, desc_add(dq0, st * L::kStage), desc_add(dk0, st * L::kStage), id_qk, 0);
-        mma_commit(s_full);
+        mma_ss_w(tmem + L::colS, desc_add(dq0, st * L::kStage), desc_add(dk0, st * L::kStage), id_qk, 0);
+        mma_commit_w(s_full);
       };
-      bool ok = n_chunks > 0 && mbar_wait(kv_full, 0, env);
+      bool ok = n_chunks > 0 && mbar_wait_w(kv_full, 0, env);
       if (ok) {
         tc_fence_after();
         issue_qk(0);
@@ -743,7 +749,7 @@ __global__ void __launch_bounds__(kReadThreads, 1)
         // entering it has been read out of TMEM (state_full) and psi~(K_c)
         // is in shared memory
         KATA_TRACE(chunk, c, 0);
-        if (!mbar_wait(state_full, c & 1, env) || !mbar_wait(fk_full, c & 1, env)) {
+        if (!mbar_wait_w(state_full, c & 1, env) || !mbar_wait_w(fk_full + (c & 1), (c >> 1) & 1, env)) {
           ok = false;
           break;
         }
@@ -752,11 +758,11 @@ __global__ void __launch_bounds__(kReadThreads, 1)
         const uint64_t dvo = desc_vones(sV, sOnes);
 #pragma unroll
         for (int ks = 0; ks < kTile / 16; ++ks)
-          mma_ss(tmem + L::colRun, desc_add(dvo, ks * 2048), desc_add(dpsi, ks * 512), id_u, 1);
-        mma_commit(upd_done);
+          mma_ss_w(tmem + L::colRun, desc_add(dvo, ks * 2048), desc_add(dpsi, (c & 1) * kPsiBytes + ks * 512), id_u, 1);
+        mma_commit_w(upd_done);
         // readout against the bf16 copy of the state entering the chunk
         KATA_TRACE(chunk, c, 2);
-        if (!mbar_wait(fq_full, c & 1, env) || (c >= 2 && !mbar_wait(o_free + ob, ((c - 2) >> 1) & 1, env))) {
+        if (!mbar_wait_w(fq_full, c & 1, env) || (c >= 2 && !mbar_wait_w(o_free + ob, ((c - 2) >> 1) & 1, env))) {
           ok = false;
           break;
         }
@@ -766,11 +772,11 @@ __global__ void __launch_bounds__(kReadThreads, 1)
         const uint32_t dO = tmem + L::colO(ob);
 #pragma unroll
         for (int ks = 0; ks < kNP / 16; ++ks)
-          mma_ts(dO, tmem + L::colPQ + ks * 8, desc_add(dsb, ks * kSBAtom), id_rd, ks > 0);
-        mma_commit(rd_done);
+          mma_ts_w(dO, tmem + L::colPQ + ks * 8, desc_add(dsb, ks * kSBAtom), id_rd, ks > 0);
+        mma_commit_w(rd_done);
         // intra-chunk weights against [V_c | 1]
         KATA_TRACE(chunk, c, 4);
-        if (!mbar_wait(p_full, c & 1, env)) {
+        if (!mbar_wait_w(p_full, c & 1, env)) {
           ok = false;
           break;
         }
@@ -778,13 +784,13 @@ __global__ void __launch_bounds__(kReadThreads, 1)
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < kTile / 16; ++ks)
-          mma_ts(dO, tmem + L::colS + ks * 8, desc_add(dvo, ks * 2048), id_wv, 1);
-        mma_commit(o_full + ob);
-        mma_commit(kv_empty + st);
+          mma_ts_w(dO, tmem + L::colS + ks * 8, desc_add(dvo, ks * 2048), id_wv, 1);
+        mma_commit_w(o_full + ob);
+        mma_commit_w(kv_empty + st);
         if (c + 1 < n_chunks) {
           const int st1 = (c + 1) % kReadStages;
           KATA_TRACE(chunk, c, 6);
-          if (!mbar_wait(kv_full + st1, ((c + 1) / kReadStages) & 1, env)) {
+          if (!mbar_wait_w(kv_full + st1, ((c + 1) / kReadStages) & 1, env)) {
             ok = false;
             break;
           }
@@ -793,7 +799,7 @@ __global__ void __launch_bounds__(kReadThreads, 1)
           issue_qk(st1);
         }
       }
-      mma_commit(mma_done);
+      mma_commit_w(mma_done);
       mbar_wait_drain(mma_done, 0, wc.limit);
     }
   } else if (warp < 6) {
@@ -840,8 +846,8 @@ __global__ void __launch_bounds__(kReadThreads, 1)
       mbar_arrive(p_full);
       if (m == 0) KATA_TRACE(chunk, c, 9);
       // output of the chunk
-      const int ob = c & 1;
-      if (!mbar_wait(o_full + ob, (c >> 1) & 1, env)) break;
+      const int co = c, ob = co & 1;
+      if (!mbar_wait(o_full + ob, (co >> 1) & 1, env)) break;
       tc_fence_after();
       uint32_t r0[32], r1[32], db;
       tmem_ld32(lane_base + L::colO(ob), r0);
@@ -850,24 +856,36 @@ __global__ void __launch_bounds__(kReadThreads, 1)
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(o_free + ob);
-      if (m == 0) KATA_TRACE(chunk, c, 14);
-      const int t = t0 + c * kTile + m;
-      if (t < t1) {
-        const float D = __uint_as_float(db);
-        const float inv = D > 0.f ? 1.f / D : 0.f;
-        const uint64_t inv2 = f32x2(__float_as_uint(inv), __float_as_uint(inv));
-        uint4* dst = reinterpret_cast<uint4*>(o + ((size_t)bh * T + t) * kDV);
-        auto scaled = [&](const uint32_t* src, int k) {
-          const uint64_t v = f32x2_mul(f32x2(src[k], src[k + 1]), inv2);
-          return pack_bf16x2(f32x2_lo(v), f32x2_hi(v));
-        };
+      if (m == 0) KATA_TRACE(chunk, co, 14);
+      // o = O / D rounded to bf16; each warp stages its 32 rows as the
+      // 128B-swizzled [32 x 64] box of the o tensor map and writes them with
+      // one TMA store (rows past T are not written)
+      const float D = __uint_as_float(db);
+      const float inv = D > 0.f ? 1.f / D : 0.f;
+      const uint64_t inv2 = f32x2(__float_as_uint(inv), __float_as_uint(inv));
+      auto scaled = [&](const uint32_t* src, int k) {
+        const uint64_t v = f32x2_mul(f32x2(src[k], src[k + 1]), inv2);
+        return pack_bf16x2(f32x2_lo(v), f32x2_hi(v));
+      };
+      // the warp's staging slab is free once its previous store has read it
+      if (lane == 0) bulk_wait_read_all();
+      __syncwarp();
+      uint8_t* slab = smem + L::offOut + quarter * (32 * 128);
+      uint8_t* orow = slab + lane * 128;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const uint32_t* src = (e < 4) ? r0 + 8 * e : r1 + 8 * (e - 4);
-          dst[e] = make_uint4(scaled(src, 0), scaled(src, 2), scaled(src, 4), scaled(src, 6));
-        }
+      for (int e = 0; e < 8; ++e) {
+        const uint32_t* src = (e < 4) ? r0 + 8 * e : r1 + 8 * (e - 4);
+        *reinterpret_cast<uint4*>(orow + ((e ^ (m & 7)) << 4)) =
+            make_uint4(scaled(src, 0), scaled(src, 2), scaled(src, 4), scaled(src, 6));
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_3d(&tm_o, slab, 0, t0 + co * kTile + quarter * 32, bh);
+        bulk_commit_group();
       }
     }
+    if (lane == 0) bulk_wait_all();
   } else {
     // ------------------------------------------------------------- psi~ and state copies
     const bool psi_group = warp < 10;   // warps 6-9: psi~ + half 0; warps 10-13: half 1
@@ -926,10 +944,23 @@ __global__ void __launch_bounds__(kReadThreads, 1)
         tc_fence_before();
         mbar_arrive(fq_full);
         if (m == 0) KATA_TRACE(chunk, c, 10);
+        if (c + 1 < n_chunks) {
+          // psi~(k_{c+1}) into the other buffer, last read by the advance by
+          // chunk c-1, which this group saw complete before its refresh
+          const int st1 = (c + 1) % kReadStages;
+          if (!mbar_wait(kv_full + st1, ((c + 1) / kReadStages) & 1, env)) break;
+          __nv_bfloat162 uk[8];
+          load_row_sw32(smem + L::offStage + st1 * L::kStage + kVBytes + kQKBytes, m, uk);
+          packed_psi<true>(uk, w);
+          store_psi_k(smem + L::offPsi + ((c + 1) & 1) * kPsiBytes, m, w);
+          fence_proxy_async_smem();
+          mbar_arrive(fk_full + ((c + 1) & 1));
+          if (m == 0) KATA_TRACE(chunk, c, 11);
+        }
       }
       if (c + 1 < n_chunks) {
         // the state after chunk c is complete: this group's half of the bf16
-        // copy for the readout of chunk c+1, then psi~(k_{c+1})
+        // copy for the readout of chunk c+1
         if (!mbar_wait(upd_done, c & 1, env)) break;
         tc_fence_after();
         if (quarter < 3) state_half_to_bf16(lane_base + L::colRun, sb + ((c + 1) & 1) * kSBBytes, m, active, half);
@@ -937,18 +968,6 @@ __global__ void __launch_bounds__(kReadThreads, 1)
         tc_fence_before();
         mbar_arrive(state_full);
         if (m == 0) KATA_TRACE(chunk, c, psi_group ? 12 : 13);
-        if (psi_group) {
-          const int st1 = (c + 1) % kReadStages;
-          if (!mbar_wait(kv_full + st1, ((c + 1) / kReadStages) & 1, env)) break;
-          __nv_bfloat162 uk[8];
-          uint32_t w[kNPW];
-          load_row_sw32(smem + L::offStage + st1 * L::kStage + kVBytes + kQKBytes, m, uk);
-          packed_psi<true>(uk, w);
-          store_psi_k(smem + L::offPsi, m, w);
-          fence_proxy_async_smem();
-          mbar_arrive(fk_full);
-          if (m == 0) KATA_TRACE(chunk, c, 11);
-        }
       }
     }
     // the last super-chunk ends at token T: its running state, once the
@@ -996,16 +1015,16 @@ cudaError_t launch_chunk_readout_sm100(const void* q, const void* k, const void*
                                        const ChunkPlan& pl, const WaitCtl& wc, cudaStream_t st) {
   if (pl.p != 16 || pl.dv != kDV) return cudaErrorInvalidValue;
   if (!ws && pl.G != 1) return cudaErrorInvalidValue;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   if (!make_tmap_bf16(&tq, q, 16, pl.T, pl.BH, kTile) || !make_tmap_bf16(&tk, k, 16, pl.T, pl.BH, kTile) ||
-      !make_tmap_bf16(&tv, v, kDV, pl.T, pl.BH, kTile))
+      !make_tmap_bf16(&tv, v, kDV, pl.T, pl.BH, kTile) || !make_tmap_bf16(&to, o, kDV, pl.T, pl.BH, 32))
     return cudaErrorInvalidValue;
   cudaError_t e =
       cudaFuncSetAttribute(chunk_readout_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ReadSmem::kBytes);
   if (e != cudaSuccess) return e;
   dim3 grid(pl.G, pl.BH);
   chunk_readout_kernel<<<grid, kReadThreads, ReadSmem::kBytes, st>>>(
-      tq, tk, tv, static_cast<__nv_bfloat16*>(o), ws, S0, z0, S_out, z_out, pl.T, pl.Ls, pl.G,
+      tq, tk, tv, to, ws, S0, z0, S_out, z_out, pl.T, pl.Ls, pl.G,
       (long long)pl.record_floats, wc);
   return cudaGetLastError();
 }

@@ -196,7 +196,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    // the whole warp runs this loop; one elected lane issues (see mma_ts_w)
+    {
       constexpr uint32_t id_qk = idesc_bf16(kBM, kBN, false, false);
       constexpr uint32_t id_pv = idesc_bf16(kBM, DV + 16, false, true);  // [V | 1]
       const uint32_t sQ = smem_u32(smem + Cfg::offQ), sK = smem_u32(smem + Cfg::offK);
@@ -207,8 +208,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto issue_qk = [&](int i, int qb, int st) {
         const uint64_t a = desc_add(dq0, (qb * kNQ + i) * Cfg::kQKBytes), b = desc_add(dk0, st * Cfg::kQKBytes);
 #pragma unroll
-        for (int ks = 0; ks < p / 16; ++ks) mma_ss(tmem + Cfg::colS(i), desc_add(a, ks * 32), desc_add(b, ks * 32), id_qk, ks > 0);
-        mma_commit(s_full + i);
+        for (int ks = 0; ks < p / 16; ++ks) mma_ss_w(tmem + Cfg::colS(i), desc_add(a, ks * 32), desc_add(b, ks * 32), id_qk, ks > 0);
+        mma_commit_w(s_full + i);
       };
       int nq = 0;
       long g = 0;                   // ring position of the item's first key tile
@@ -220,7 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int nkv[kNQ];
         for (int i = 0; i < kNQ; ++i) nkv[i] = item_nkv(it, i);
         const int nkv_max = max(nkv[0], nkv[1]);
-        if (!mbar_wait(q_full + qb, (nq >> 1) & 1, env) || !mbar_wait(kv_full + g % kStages, (int)((g / kStages) & 1), env)) {
+        if (!mbar_wait_w(q_full + qb, (nq >> 1) & 1, env) || !mbar_wait_w(kv_full + g % kStages, (int)((g / kStages) & 1), env)) {
           ok = false;
           break;
         }
@@ -236,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < kNQ; ++i) {
             if (j >= nkv[i]) continue;
             KATA_TRACE(flash, (int)gj, 2 * i);
-            if (!mbar_wait(p_full + i, p_cnt[i] & 1, env)) {
+            if (!mbar_wait_w(p_full + i, p_cnt[i] & 1, env)) {
               ok = false;
               break;
             }
@@ -244,7 +245,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++p_cnt[i];
             // the first P.V of this tile overwrites [O|D]_i: the previous
             // item's epilogue must have read it
-            if (j == 0 && o_cnt[i] > 0 && !mbar_wait(o_free + i, (o_cnt[i] - 1) & 1, env)) {
+            if (j == 0 && o_cnt[i] > 0 && !mbar_wait_w(o_free + i, (o_cnt[i] - 1) & 1, env)) {
               ok = false;
               break;
             }
@@ -252,16 +253,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t aw = tmem + Cfg::colS(i), dO = tmem + Cfg::colO(i);
 #pragma unroll
             for (int ks = 0; ks < kBN / 16; ++ks)  // keys 16ks..: W columns 64*(ks/4) + 8*(ks%4)
-              mma_ts(dO, aw + (ks >> 2) * 64 + (ks & 3) * 8, desc_add(dv, ks * Cfg::kVKStep), id_pv,
+              mma_ts_w(dO, aw + (ks >> 2) * 64 + (ks & 3) * 8, desc_add(dv, ks * Cfg::kVKStep), id_pv,
                      (j > 0 || ks > 0) ? 1u : 0u);
             if (j == nkv[i] - 1) {
-              mma_commit(o_full + i);
+              mma_commit_w(o_full + i);
               ++o_cnt[i];
             }
             if (j + 1 < nkv[i]) {
               const long gn = gj + 1;
               if (kv_ready < gn) {
-                if (!mbar_wait(kv_full + gn % kStages, (int)((gn / kStages) & 1), env)) {
+                if (!mbar_wait_w(kv_full + gn % kStages, (int)((gn / kStages) & 1), env)) {
                   ok = false;
                   break;
                 }
@@ -273,12 +274,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (!ok) break;
           KATA_TRACE(flash, (int)gj, 4);
-          mma_commit(kv_empty + st);
+          mma_commit_w(kv_empty + st);
         }
-        mma_commit(q_empty + qb);  // the item's Q tiles are free once its MMAs complete
+        mma_commit_w(q_empty + qb);  // the item's Q tiles are free once its MMAs complete
         g += nkv_max;
       }
-      mma_commit(mma_done);
+      mma_commit_w(mma_done);
       mbar_wait_drain(mma_done, 0, wc.limit);
     }
   } else {
