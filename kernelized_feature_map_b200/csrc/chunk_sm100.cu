@@ -48,6 +48,7 @@ KATA_TRACE_DECLARE(chunkstate)
 namespace kata {
 
 bool make_tmap_bf16(CUtensorMap* map, const void* base, int inner, int T, int BH, int rows);
+bool make_tmap_bf16_box(CUtensorMap* map, const void* base, int inner, int T, int BH, int box_inner, int rows);
 
 namespace {
 
@@ -196,25 +197,6 @@ __device__ __forceinline__ void store_state_bf16_atom(uint8_t* sb, int n, int at
   }
 }
 
-// TMEM lane (this thread's row of S~^T) -> bf16 copy row n (when `active`).
-// Warp-collective: every lane of the warp must call it.
-__device__ __forceinline__ void state_lane_to_bf16(uint32_t taddr, uint8_t* sb, int n, bool active) {
-#pragma unroll
-  for (int b = 0; b < 4; ++b) {
-    uint32_t r[32];
-    tmem_ld32(taddr + 32 * b, r);
-    tmem_wait_ld();
-    if (active) {
-      store_state_bf16_atom(sb, n, 2 * b, r);
-      store_state_bf16_atom(sb, n, 2 * b + 1, r + 16);
-    }
-  }
-  uint32_t r[16];
-  tmem_ld16(taddr + 128, r);
-  tmem_wait_ld();
-  if (active) store_state_bf16_atom(sb, n, 8, r);
-}
-
 // TMEM lane -> fp32 record row in global memory (when `active`).
 // Warp-collective.
 __device__ __forceinline__ void state_lane_to_global(uint32_t taddr, float* row, bool active) {
@@ -237,26 +219,6 @@ __device__ __forceinline__ void state_lane_to_global(uint32_t taddr, float* row,
     for (int e = 0; e < 16; e += 4)
       *reinterpret_cast<float4*>(row + 128 + e) = make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]),
                                                               __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
-}
-
-// fp32 record row (or zeros) -> TMEM lane and bf16 copy row n.  Warp-collective.
-__device__ __forceinline__ void global_to_state_lane(const float* row, uint32_t taddr, uint8_t* sb, int n,
-                                                     bool active) {
-#pragma unroll 3
-  for (int a = 0; a < 9; ++a) {
-    uint32_t r[16];
-#pragma unroll
-    for (int e = 0; e < 16; e += 4) {
-      float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (active) v4 = *reinterpret_cast<const float4*>(row + 16 * a + e);
-      r[e] = __float_as_uint(v4.x);
-      r[e + 1] = __float_as_uint(v4.y);
-      r[e + 2] = __float_as_uint(v4.z);
-      r[e + 3] = __float_as_uint(v4.w);
-    }
-    tmem_st16(taddr + 16 * a, r);
-    if (active) store_state_bf16_atom(sb, n, a, r);
-  }
 }
 
 // One 8-coordinate chunk (c = 0 or 1) of atom `atom` of row n of the bf16 copy.
@@ -595,24 +557,29 @@ __global__ void __launch_bounds__(kStateThreads, 1)
 // ===========================================================================
 // 3. readout
 // ===========================================================================
-// Warp roles (448 threads):
+// Warp roles (576 threads):
 //   warp 0       TMA: [V | Q | K] tiles of each chunk into a 3-stage ring
 //   warp 1       TMEM allocator; MMA issue (the whole warp, one elected lane)
-//   warps 2-5    weights W = (Q K^T)^2 (causal) into TMEM; output o = O / D
-//   warps 6-9    psi~(q_c) into TMEM, psi~(k_{c+1}) into shared memory (two
-//                buffers); bf16 copy of packed coordinates 0..71 of the state
-//                after each chunk
-//   warps 10-13  prefix state in; bf16 copy of coordinates 72..143
-// MMA order per chunk c: advance S~ by chunk c, readout of chunk c against
-// the bf16 copy of S~ made before chunk c, intra-chunk weights, then the
-// scores of chunk c+1.  The readout reads only the bf16 copy, so the state
-// can advance first; the copy for chunk c+1 is then refreshed while the
-// readout and intra-chunk MMAs of chunk c run (the copy is double-buffered).
-// The loop-carried path is advance(c) -> refresh -> advance(c+1); psi~(k_{c+1})
-// is formed into the second buffer while the advance by chunk c runs, so it
-// stays off that path.  The [O | D] accumulator is double-buffered so the
-// readout of chunk c+1 does not wait for the output of chunk c to be read.
-constexpr int kReadThreads = 448;
+//   warps 2-5,   weights W = (Q K^T)^2 (causal) into TMEM; output o = O / D;
+//   14-17        each pair of warps on a TMEM lane quarter splits the columns
+//   warps 6-9    psi~(k_{c+1}) into shared memory (two buffers); bf16 copy of
+//                packed coordinates 0..71 of the state after chunk c
+//   warps 10-13  prefix state in; bf16 copy of coordinates 72..143; then
+//                psi~(q_{c+1}) into TMEM
+// MMA order per chunk c: scores of chunk c, advance S~ by chunk c, readout of
+// chunk c against the bf16 copy of S~ made before chunk c, intra-chunk
+// weights.  The readout reads only the bf16 copy, so the state can advance
+// first; the copy for chunk c+1 is refreshed while the readout and
+// intra-chunk MMAs of chunk c run (the copy is double-buffered).
+// The MMA warp waits on two barriers per chunk.  state_full(c) is arrived on
+// by warps 6-13 after everything chunk c needs from them (its psi~(k), its
+// psi~(q), the bf16 copy; each of them waited for chunk c's tiles to land
+// first) and by warps 2-5 and 14-17 once they have read the output of chunk
+// c-2 out of the [O | D] buffer the readout of chunk c reuses; p_full(c) by
+// warps 2-5 and 14-17 after the weights of chunk c.  Each wait in the
+// issuing warp costs ~100 cycles in which the tensor pipe drains, so the
+// implied ones are not waited for separately.
+constexpr int kReadThreads = 576;
 constexpr int kReadStages = 3;
 
 struct ReadSmem {
@@ -621,9 +588,9 @@ struct ReadSmem {
   static constexpr int offOnes = offStage + kReadStages * kStage;  // 1024-aligned
   static constexpr int offPsi = offOnes + kOnesBytes;  // 2 buffers
   static constexpr int offSB = offPsi + 2 * kPsiBytes;  // 2 buffers
-  static constexpr int offOut = offSB + 2 * kSBBytes;   // output tile staging, 128B swizzle (1024-aligned)
+  static constexpr int offOut = offSB + 2 * kSBBytes;   // output staging: 8 boxes [32 x 32], 64B swizzle
   static constexpr int offBar = offOut + kVBytes;
-  static constexpr int kBars = 2 * kReadStages + 13;
+  static constexpr int kBars = 2 * kReadStages + 8;
   static constexpr int offMisc = offBar + kBars * 8;
   static constexpr int kBytes = offMisc + 16 + 1024;
   // TMEM columns (multiples of 16, 512 in total)
@@ -646,15 +613,12 @@ __global__ void __launch_bounds__(kReadThreads, 1)
   uint64_t* kv_full = bars;
   uint64_t* kv_empty = kv_full + kReadStages;
   uint64_t* s_full = kv_empty + kReadStages;  // scores in TMEM
-  uint64_t* p_full = s_full + 1;              // weights written (128)
-  uint64_t* fq_full = p_full + 1;             // psi~(Q_c) in TMEM (128)
-  uint64_t* fk_full = fq_full + 1;            // [2] psi~(K_c) in shared memory buffer c % 2 (128)
-  uint64_t* state_full = fk_full + 2;         // bf16 state copy ready (256)
+  uint64_t* p_full = s_full + 1;              // weights written (256)
+  uint64_t* state_full = p_full + 1;          // chunk c's operands ready and its [O | D] buffer free (512)
   uint64_t* rd_done = state_full + 1;         // readout of the chunk done
   uint64_t* upd_done = rd_done + 1;           // state advanced by the chunk
   uint64_t* o_full = upd_done + 1;            // [2] [O | D] complete
-  uint64_t* o_free = o_full + 2;              // [2] [O | D] read (128)
-  uint64_t* mma_done = o_free + 2;
+  uint64_t* mma_done = o_full + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::offMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::offMisc + 4);
 
@@ -673,17 +637,11 @@ __global__ void __launch_bounds__(kReadThreads, 1)
       mbar_init(kv_empty + s, 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(p_full, 128);
-    mbar_init(fq_full, 128);
-    mbar_init(fk_full, 128);
-    mbar_init(fk_full + 1, 128);
-    mbar_init(state_full, 256);
+    mbar_init(p_full, 256);
+    mbar_init(state_full, 512);
     mbar_init(rd_done, 1);
     mbar_init(upd_done, 1);
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(o_full + b, 1);
-      mbar_init(o_free + b, 128);
-    }
+    for (int b = 0; b < 2; ++b) mbar_init(o_full + b, 1);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -733,41 +691,27 @@ __global__ void __launch_bounds__(kReadThreads, 1)
       const uint64_t dk0 = smem_desc(sStage + kVBytes + kQKBytes, 16, 256, kSw32);
       const uint64_t dpsi = smem_desc(sPsi, kPsiAtom, 256, kSw32);
       const uint64_t dsb0 = smem_desc(sSB, 16, 256, kSw32);
-      auto issue_qk = [&](int st) {
-        mma_ss_w(tmem + L::colS, desc_add(dq0, st * L::kStage), desc_add(dk0, st * L::kStage), id_qk, 0);
-        mma_commit_w(s_full);
-      };
-      bool ok = n_chunks > 0 && mbar_wait_w(kv_full, 0, env);
-      if (ok) {
-        tc_fence_after();
-        issue_qk(0);
-      }
-      for (int c = 0; ok && c < n_chunks; ++c) {
+      for (int c = 0; c < n_chunks; ++c) {
         const int st = c % kReadStages, ob = c & 1;
         const uint32_t sV = sStage + st * L::kStage;
-        // advance the state by the chunk, once the bf16 copy of the state
-        // entering it has been read out of TMEM (state_full) and psi~(K_c)
-        // is in shared memory
+        // everything chunk c needs from warps 6-13; its tiles have landed
         KATA_TRACE(chunk, c, 0);
-        if (!mbar_wait_w(state_full, c & 1, env) || !mbar_wait_w(fk_full + (c & 1), (c >> 1) & 1, env)) {
-          ok = false;
-          break;
-        }
+        if (!mbar_wait_w(state_full, c & 1, env)) break;
         KATA_TRACE(chunk, c, 1);
         tc_fence_after();
+        // scores of chunk c (overwrite the weights of chunk c-1 only after
+        // the intra-chunk MMAs of c-1 issued before them)
+        mma_ss_w(tmem + L::colS, desc_add(dq0, st * L::kStage), desc_add(dk0, st * L::kStage), id_qk, 0);
+        mma_commit_w(s_full);
+        // advance the state by the chunk
         const uint64_t dvo = desc_vones(sV, sOnes);
 #pragma unroll
         for (int ks = 0; ks < kTile / 16; ++ks)
           mma_ss_w(tmem + L::colRun, desc_add(dvo, ks * 2048), desc_add(dpsi, (c & 1) * kPsiBytes + ks * 512), id_u, 1);
         mma_commit_w(upd_done);
-        // readout against the bf16 copy of the state entering the chunk
         KATA_TRACE(chunk, c, 2);
-        if (!mbar_wait_w(fq_full, c & 1, env) || (c >= 2 && !mbar_wait_w(o_free + ob, ((c - 2) >> 1) & 1, env))) {
-          ok = false;
-          break;
-        }
-        KATA_TRACE(chunk, c, 3);
-        tc_fence_after();
+        // readout against the bf16 copy of the state entering the chunk (the
+        // [O | D] buffer is free: see state_full)
         const uint64_t dsb = desc_add(dsb0, ob * kSBBytes);
         const uint32_t dO = tmem + L::colO(ob);
 #pragma unroll
@@ -776,45 +720,86 @@ __global__ void __launch_bounds__(kReadThreads, 1)
         mma_commit_w(rd_done);
         // intra-chunk weights against [V_c | 1]
         KATA_TRACE(chunk, c, 4);
-        if (!mbar_wait_w(p_full, c & 1, env)) {
-          ok = false;
-          break;
-        }
+        if (!mbar_wait_w(p_full, c & 1, env)) break;
         KATA_TRACE(chunk, c, 5);
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < kTile / 16; ++ks)
-          mma_ts_w(dO, tmem + L::colS + ks * 8, desc_add(dvo, ks * 2048), id_wv, 1);
+          mma_ts_w(dO, tmem + L::colS + (ks >> 2) * 64 + (ks & 3) * 8, desc_add(dvo, ks * 2048), id_wv, 1);
         mma_commit_w(o_full + ob);
         mma_commit_w(kv_empty + st);
-        if (c + 1 < n_chunks) {
-          const int st1 = (c + 1) % kReadStages;
-          KATA_TRACE(chunk, c, 6);
-          if (!mbar_wait_w(kv_full + st1, ((c + 1) / kReadStages) & 1, env)) {
-            ok = false;
-            break;
-          }
-          KATA_TRACE(chunk, c, 7);
-          tc_fence_after();
-          issue_qk(st1);
-        }
+        KATA_TRACE(chunk, c, 6);
       }
       mma_commit_w(mma_done);
       mbar_wait_drain(mma_done, 0, wc.limit);
     }
-  } else if (warp < 6) {
+  } else if (warp < 6 || warp >= 14) {
     // ------------------------------------------------------------- weights + output
+    // warps 2-5 take key columns 0..63 of the weights and value columns
+    // 0..31 of the output, warps 14-17 the other halves; both warps of a
+    // pair read the same TMEM lane quarter (rows 32 * quarter ..)
     const int quarter = warp % 4;
+    const int h = warp >= 14 ? 1 : 0;
     const int m = quarter * 32 + lane;
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-    for (int c = 0; c < n_chunks; ++c) {
+    uint8_t* slab = smem + L::offOut + (quarter * 2 + h) * (32 * 64);  // this warp's [32 x 32] output box
+    // output of chunk co: read [O | D] out of TMEM, then (once the read is
+    // done) arrive on state_full(co + 2) when that chunk exists, since the
+    // readout of chunk co + 2 reuses this [O | D] buffer; then o = O / D
+    // rounded to bf16, staged as this warp's 64B-swizzled [32 x 32] box of
+    // the o tensor map (16-byte chunk j of row r at chunk j ^ ((r / 2) % 4))
+    // and written by one TMA store (rows past T are not written)
+    auto output = [&](int co) -> bool {
+      const int ob = co & 1;
+      if (!mbar_wait(o_full + ob, (co >> 1) & 1, env)) return false;
+      tc_fence_after();
+      uint32_t r[32], db;
+      tmem_ld32(lane_base + L::colO(ob) + 32 * h, r);
+      tmem_ld1(lane_base + L::colO(ob) + 64, db);
+      tmem_wait_ld();
+      tc_fence_before();
+      if (co + 2 < n_chunks) mbar_arrive(state_full);
+      if (m == 0) KATA_TRACE(chunk, co, 14);
+      const float D = __uint_as_float(db);
+      const float inv = D > 0.f ? 1.f / D : 0.f;
+      const uint64_t inv2 = f32x2(__float_as_uint(inv), __float_as_uint(inv));
+      auto scaled = [&](int k) {
+        const uint64_t v = f32x2_mul(f32x2(r[k], r[k + 1]), inv2);
+        return pack_bf16x2(f32x2_lo(v), f32x2_hi(v));
+      };
+      // the warp's staging slab is free once its previous store has read it
+      if (lane == 0) bulk_wait_read_all();
+      __syncwarp();
+      uint8_t* orow = slab + lane * 64;
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        *reinterpret_cast<uint4*>(orow + ((e ^ ((lane >> 1) & 3)) << 4)) =
+            make_uint4(scaled(8 * e), scaled(8 * e + 2), scaled(8 * e + 4), scaled(8 * e + 6));
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_3d(&tm_o, slab, 32 * h, t0 + co * kTile + quarter * 32, bh);
+        bulk_commit_group();
+      }
+      return true;
+    };
+    // the readouts of chunks 0 and 1 write fresh [O | D] buffers; an arrival
+    // for state_full(c) is made only once state_full(c-1) has completed
+    // (for c = 1: once the scores of chunk 0, issued after it, are in)
+    if (n_chunks > 0) mbar_arrive(state_full);
+    bool ok = true;
+    for (int c = 0; ok && c < n_chunks; ++c) {
       if (!mbar_wait(s_full, c & 1, env)) break;
+      if (c == 0 && n_chunks > 1) mbar_arrive(state_full);
       if (m == 0) KATA_TRACE(chunk, c, 8);
       tc_fence_after();
       // causal within the chunk: 32-column block bb of row m is fully kept
-      // for bb < quarter, diagonal for bb == quarter, zero for bb > quarter
+      // for bb < quarter, diagonal for bb == quarter, zero for bb > quarter.
+      // Block bb's 16 bf16x2 words go to columns 64 (bb / 2) + 16 (bb % 2),
+      // inside the half's own score columns and over scores already read.
 #pragma unroll
-      for (int bb = 0; bb < 4; ++bb) {
+      for (int b2 = 0; b2 < 2; ++b2) {
+        const int bb = 2 * h + b2;
         uint32_t w[16];
         if (bb > quarter) {
 #pragma unroll
@@ -839,62 +824,41 @@ __global__ void __launch_bounds__(kReadThreads, 1)
             }
           }
         }
-        tmem_st16(lane_base + L::colS + 16 * bb, w);
+        tmem_st16(lane_base + L::colS + 64 * h + 16 * b2, w);
       }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(p_full);
       if (m == 0) KATA_TRACE(chunk, c, 9);
-      // output of the chunk
-      const int co = c, ob = co & 1;
-      if (!mbar_wait(o_full + ob, (co >> 1) & 1, env)) break;
-      tc_fence_after();
-      uint32_t r0[32], r1[32], db;
-      tmem_ld32(lane_base + L::colO(ob), r0);
-      tmem_ld32(lane_base + L::colO(ob) + 32, r1);
-      tmem_ld1(lane_base + L::colO(ob) + 64, db);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(o_free + ob);
-      if (m == 0) KATA_TRACE(chunk, co, 14);
-      // o = O / D rounded to bf16; each warp stages its 32 rows as the
-      // 128B-swizzled [32 x 64] box of the o tensor map and writes them with
-      // one TMA store (rows past T are not written)
-      const float D = __uint_as_float(db);
-      const float inv = D > 0.f ? 1.f / D : 0.f;
-      const uint64_t inv2 = f32x2(__float_as_uint(inv), __float_as_uint(inv));
-      auto scaled = [&](const uint32_t* src, int k) {
-        const uint64_t v = f32x2_mul(f32x2(src[k], src[k + 1]), inv2);
-        return pack_bf16x2(f32x2_lo(v), f32x2_hi(v));
-      };
-      // the warp's staging slab is free once its previous store has read it
-      if (lane == 0) bulk_wait_read_all();
-      __syncwarp();
-      uint8_t* slab = smem + L::offOut + quarter * (32 * 128);
-      uint8_t* orow = slab + lane * 128;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const uint32_t* src = (e < 4) ? r0 + 8 * e : r1 + 8 * (e - 4);
-        *reinterpret_cast<uint4*>(orow + ((e ^ (m & 7)) << 4)) =
-            make_uint4(scaled(src, 0), scaled(src, 2), scaled(src, 4), scaled(src, 6));
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        tma_store_3d(&tm_o, slab, 0, t0 + co * kTile + quarter * 32, bh);
-        bulk_commit_group();
-      }
+      // the output of the previous chunk, after these weights so that the
+      // weights are never held up by it
+      if (c > 0) ok = output(c - 1);
     }
+    if (ok && n_chunks > 0) output(n_chunks - 1);
     if (lane == 0) bulk_wait_all();
   } else {
     // ------------------------------------------------------------- psi~ and state copies
-    const bool psi_group = warp < 10;   // warps 6-9: psi~ + half 0; warps 10-13: half 1
+    const bool psi_group = warp < 10;   // warps 6-9: psi~(k) + half 0; warps 10-13: half 1 + psi~(q)
     const int half = psi_group ? 0 : 1;
     const int quarter = warp % 4;
     const int m = quarter * 32 + lane;  // token of the chunk / TMEM lane
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
     uint8_t* sb = smem + L::offSB;
     const bool active = m < kSBRows;    // rows 0..63 values, 64..79 copies of z
+    // psi~(k) of chunk cc into shared-memory buffer cc % 2, or psi~(q) of
+    // chunk cc into TMEM, from the chunk's landed stage
+    auto psi_k = [&](int cc) {
+      __nv_bfloat162 u[8];
+      uint32_t w[kNPW];
+      load_row_sw32(smem + L::offStage + (cc % kReadStages) * L::kStage + kVBytes + kQKBytes, m, u);
+      packed_psi<true>(u, w);
+      store_psi_k(smem + L::offPsi + (cc & 1) * kPsiBytes, m, w);
+    };
+    auto psi_q_formed = [&](int cc, uint32_t (&w)[kNPW]) {
+      __nv_bfloat162 u[8];
+      load_row_sw32(smem + L::offStage + (cc % kReadStages) * L::kStage + kVBytes, m, u);
+      packed_psi<false>(u, w);
+    };
     // running state <- scanned prefix (fp32 into TMEM, bf16 into shared
     // memory); with a single super-chunk there is no workspace and the
     // prefix is the caller's initial state (or zero)
@@ -910,65 +874,53 @@ __global__ void __launch_bounds__(kReadThreads, 1)
         else abi_half_to_state<1>(S, z, d, lane_base + L::colRun, sb, m, active);
       }
     }
+    // chunk 0's psi~(k) or psi~(q): they need nothing but its stage
+    bool ok = n_chunks > 0 && mbar_wait(kv_full, 0, env);
+    if (ok) {
+      if (psi_group) {
+        psi_k(0);
+      } else {
+        uint32_t w[kNPW];
+        psi_q_formed(0, w);
+        store_psi_q_tmem(lane_base + L::colPQ, w);
+      }
+    }
     tmem_wait_st();
     fence_proxy_async_smem();
     tc_fence_before();
-    mbar_arrive(state_full);
-    // chunk 0: psi~(k_0) needs nothing but the stage
-    bool ok = true;
-    if (psi_group && n_chunks > 0) {
-      if (!mbar_wait(kv_full, 0, env)) ok = false;
-      else {
-        __nv_bfloat162 uk[8];
-        uint32_t w[kNPW];
-        load_row_sw32(smem + L::offStage + kVBytes + kQKBytes, m, uk);
-        packed_psi<true>(uk, w);
-        store_psi_k(smem + L::offPsi, m, w);
-        fence_proxy_async_smem();
-        mbar_arrive(fk_full);
-      }
-    }
-    for (int c = 0; ok && c < n_chunks; ++c) {
+    if (ok) mbar_arrive(state_full);
+    for (int c = 0; ok && c + 1 < n_chunks; ++c) {
+      // operands of chunk c+1, whose tiles land in stage (c+1) % kReadStages
+      const int st1 = (c + 1) % kReadStages;
+      if (!mbar_wait(kv_full + st1, ((c + 1) / kReadStages) & 1, env)) break;
       if (psi_group) {
-        // psi~(q_c) into TMEM once the readout of chunk c-1 has consumed it
-        const int st = c % kReadStages;
-        if (!mbar_wait(kv_full + st, (c / kReadStages) & 1, env)) break;
-        __nv_bfloat162 uq[8];
-        uint32_t w[kNPW];
-        load_row_sw32(smem + L::offStage + st * L::kStage + kVBytes, m, uq);
-        packed_psi<false>(uq, w);
-        if (c > 0 && !mbar_wait(rd_done, (c - 1) & 1, env)) break;
+        // psi~(k_{c+1}) into the buffer last read by the advance by chunk
+        // c-1, which this group saw complete in the previous iteration
+        psi_k(c + 1);
+        if (m == 0) KATA_TRACE(chunk, c, 11);
+      }
+      // the state after chunk c is complete: this group's half of the bf16
+      // copy for the readout of chunk c+1 (its buffer was last read by the
+      // readout of chunk c-1, which completed before this advance did)
+      if (!mbar_wait(upd_done, c & 1, env)) break;
+      if (m == 0) KATA_TRACE(chunk, c, psi_group ? 15 : 16);
+      tc_fence_after();
+      if (quarter < 3) state_half_to_bf16(lane_base + L::colRun, sb + ((c + 1) & 1) * kSBBytes, m, active, half);
+      if (m == 0) KATA_TRACE(chunk, c, psi_group ? 17 : 18);
+      if (!psi_group) {
+        // psi~(q_{c+1}) into TMEM once the readout of chunk c has read psi~(q_c)
+        uint32_t wq[kNPW];
+        psi_q_formed(c + 1, wq);
+        if (!mbar_wait(rd_done, c & 1, env)) break;
+        if (m == 0) KATA_TRACE(chunk, c, 19);
         tc_fence_after();
-        store_psi_q_tmem(lane_base + L::colPQ, w);
+        store_psi_q_tmem(lane_base + L::colPQ, wq);
         tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(fq_full);
-        if (m == 0) KATA_TRACE(chunk, c, 10);
-        if (c + 1 < n_chunks) {
-          // psi~(k_{c+1}) into the other buffer, last read by the advance by
-          // chunk c-1, which this group saw complete before its refresh
-          const int st1 = (c + 1) % kReadStages;
-          if (!mbar_wait(kv_full + st1, ((c + 1) / kReadStages) & 1, env)) break;
-          __nv_bfloat162 uk[8];
-          load_row_sw32(smem + L::offStage + st1 * L::kStage + kVBytes + kQKBytes, m, uk);
-          packed_psi<true>(uk, w);
-          store_psi_k(smem + L::offPsi + ((c + 1) & 1) * kPsiBytes, m, w);
-          fence_proxy_async_smem();
-          mbar_arrive(fk_full + ((c + 1) & 1));
-          if (m == 0) KATA_TRACE(chunk, c, 11);
-        }
       }
-      if (c + 1 < n_chunks) {
-        // the state after chunk c is complete: this group's half of the bf16
-        // copy for the readout of chunk c+1
-        if (!mbar_wait(upd_done, c & 1, env)) break;
-        tc_fence_after();
-        if (quarter < 3) state_half_to_bf16(lane_base + L::colRun, sb + ((c + 1) & 1) * kSBBytes, m, active, half);
-        fence_proxy_async_smem();
-        tc_fence_before();
-        mbar_arrive(state_full);
-        if (m == 0) KATA_TRACE(chunk, c, psi_group ? 12 : 13);
-      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(state_full);
+      if (m == 0) KATA_TRACE(chunk, c, psi_group ? 12 : 13);
     }
     // the last super-chunk ends at token T: its running state, once the
     // advance by its last chunk has landed, is the final state
@@ -1017,7 +969,7 @@ cudaError_t launch_chunk_readout_sm100(const void* q, const void* k, const void*
   if (!ws && pl.G != 1) return cudaErrorInvalidValue;
   CUtensorMap tq, tk, tv, to;
   if (!make_tmap_bf16(&tq, q, 16, pl.T, pl.BH, kTile) || !make_tmap_bf16(&tk, k, 16, pl.T, pl.BH, kTile) ||
-      !make_tmap_bf16(&tv, v, kDV, pl.T, pl.BH, kTile) || !make_tmap_bf16(&to, o, kDV, pl.T, pl.BH, 32))
+      !make_tmap_bf16(&tv, v, kDV, pl.T, pl.BH, kTile) || !make_tmap_bf16_box(&to, o, kDV, pl.T, pl.BH, 32, 32))
     return cudaErrorInvalidValue;
   cudaError_t e =
       cudaFuncSetAttribute(chunk_readout_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ReadSmem::kBytes);

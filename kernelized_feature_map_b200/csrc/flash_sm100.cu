@@ -410,22 +410,28 @@ EncodeTiledFn get_encode_tiled() {
   return fn;
 }
 
-// 3-D bf16 tensor map over [BH][T][inner] with a box of {inner, rows, 1}.
-bool make_tmap_bf16(CUtensorMap* map, const void* base, int inner, int T, int BH, int rows) {
+// 3-D bf16 tensor map over [BH][T][inner] with a box of {box_inner, rows, 1};
+// the swizzle is the one whose span equals the box row (32, 64 or 128 bytes).
+bool make_tmap_bf16_box(CUtensorMap* map, const void* base, int inner, int T, int BH, int box_inner, int rows) {
   EncodeTiledFn enc = get_encode_tiled();
   if (!enc) return false;
-  const int row_bytes = inner * 2;
-  CUtensorMapSwizzle sw = row_bytes == 32    ? CU_TENSOR_MAP_SWIZZLE_32B
-                          : row_bytes == 64  ? CU_TENSOR_MAP_SWIZZLE_64B
-                          : row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+  const int row_bytes = inner * 2, box_bytes = box_inner * 2;
+  CUtensorMapSwizzle sw = box_bytes == 32    ? CU_TENSOR_MAP_SWIZZLE_32B
+                          : box_bytes == 64  ? CU_TENSOR_MAP_SWIZZLE_64B
+                          : box_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
                                              : CU_TENSOR_MAP_SWIZZLE_NONE;
   cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)T, (cuuint64_t)BH};
   cuuint64_t strides[2] = {(cuuint64_t)row_bytes, (cuuint64_t)row_bytes * (cuuint64_t)T};
-  cuuint32_t box[3] = {(cuuint32_t)inner, (cuuint32_t)rows, 1};
+  cuuint32_t box[3] = {(cuuint32_t)box_inner, (cuuint32_t)rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3-D bf16 tensor map over [BH][T][inner] with a box of {inner, rows, 1}.
+bool make_tmap_bf16(CUtensorMap* map, const void* base, int inner, int T, int BH, int rows) {
+  return make_tmap_bf16_box(map, base, inner, T, BH, inner, rows);
 }
 
 template <int p, int DV>
