@@ -81,7 +81,10 @@ struct FlashCfg {
   static constexpr int offK = offQ + 2 * kNQ * kQKBytes;
   static constexpr int offV = ((offK + kStages * kQKBytes) + 1023) / 1024 * 1024;
   static constexpr int offOnes = offV + kStages * kVBytes;  // 1024-aligned
-  static constexpr int offBar = offOnes + kOnesBytes;
+  // output staging: one [32 rows x DV/2] box per weight warp (row = DV bytes)
+  static constexpr int kOutSlab = 32 * DV;
+  static constexpr int offOut = offOnes + kOnesBytes;  // 1024-aligned
+  static constexpr int offBar = offOut + 16 * kOutSlab;
   static constexpr int kNumBars = 4 + 2 * kStages + 4 * kNQ + 1;
   static constexpr int offMisc = offBar + kNumBars * 8;
   static constexpr int kSmemBytes = offMisc + 16 + 1024;  // + alignment slack
@@ -90,7 +93,7 @@ struct FlashCfg {
 template <int p, int DV>
 __global__ void __launch_bounds__(kThreads, 1)
     flash_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                     const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ o, int T, int BH,
+                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o, int T, int BH,
                      WaitCtl wc) {
   using Cfg = FlashCfg<p, DV>;
   extern __shared__ uint8_t smem_raw[];
@@ -295,14 +298,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quarter = warp % 4;          // TMEM lane quarter this warp may access
     const int m = quarter * 32 + lane;     // row within the tile
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    // the output of a pair is read out of TMEM, scaled and staged in this
+    // warp's shared-memory box right after the pair's last weights (which
+    // frees the [O|D] buffer for the next pair); its TMA store is issued
+    // after the next pair's first weights, so that the weights of the next
+    // item never wait for the store
+    constexpr int kHalf = DV / 2;          // output columns per thread
+    uint8_t* slab = smem + Cfg::offOut + idx * Cfg::kOutSlab;
+    bool pend = false;
+    int pend_row0 = 0, pend_bh = 0;
+    auto flush_out = [&]() {
+      if (pend && lane == 0) {
+        tma_store_3d(&tm_o, slab, kHalf * h, pend_row0, pend_bh);
+        bulk_commit_group();
+      }
+      pend = false;
+    };
     int s_cnt = 0, o_cnt = 0;
     bool ok = true;
     int rr = 0;
     for (int it = my_item(rr); ok && it >= 0; it = my_item(++rr)) {
       const int nkv = item_nkv(it, i);
-      if (nkv == 0) continue;
+      if (nkv == 0) {
+        flush_out();
+        continue;
+      }
       const int bh = item_bh(it);
-      const int t = (item_ct(it) * kNQ + i) * kBM + m;
+      const int row0 = (item_ct(it) * kNQ + i) * kBM + quarter * 32;  // this warp's first row
       for (int j = 0; j < nkv; ++j) {
         if (!mbar_wait(s_full + i, s_cnt & 1, env)) {
           ok = false;
@@ -349,11 +371,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         mbar_arrive(p_full + i);
         if (m == 0 && h == 0) KATA_TRACE(flash, s_cnt - 1, 6 + 2 * i);
+        if (j == 0) flush_out();
       }
       if (!ok || !mbar_wait(o_full + i, o_cnt & 1, env)) break;
       ++o_cnt;
       tc_fence_after();
-      constexpr int kHalf = DV / 2;        // output columns per thread
       uint32_t dbits;
       uint32_t ov[kHalf];
       tmem_ld1(lane_base + Cfg::colD(i), dbits);
@@ -365,20 +387,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(o_free + i);
+      // o = O / D (D = 0 gives 0) rounded to bf16, staged as row `lane` of
+      // the box: for DV = 64 the 64-byte rows are 64B-swizzled (16-byte chunk
+      // e at e ^ ((lane / 2) % 4)), for DV = 16 the 16-byte rows are plain
       const float D = __uint_as_float(dbits);
       const float inv = D > 0.f ? 1.f / D : 0.f;
-      if (t < T) {
-        uint4* dst = reinterpret_cast<uint4*>(o + ((size_t)bh * T + t) * DV + kHalf * h);
-        const uint64_t inv2 = f32x2(__float_as_uint(inv), __float_as_uint(inv));
-        auto scaled = [&](int k) {
-          const uint64_t v = f32x2_mul(f32x2(ov[k], ov[k + 1]), inv2);
-          return pack_bf16x2(f32x2_lo(v), f32x2_hi(v));
-        };
+      const uint64_t inv2 = f32x2(__float_as_uint(inv), __float_as_uint(inv));
+      auto scaled = [&](int k) {
+        const uint64_t v = f32x2_mul(f32x2(ov[k], ov[k + 1]), inv2);
+        return pack_bf16x2(f32x2_lo(v), f32x2_hi(v));
+      };
+      if (lane == 0) bulk_wait_read_all();  // the previous store has read the box
+      __syncwarp();
+      uint8_t* orow = slab + lane * DV;
 #pragma unroll
-        for (int e = 0; e < kHalf / 8; ++e)
-          dst[e] = make_uint4(scaled(8 * e), scaled(8 * e + 2), scaled(8 * e + 4), scaled(8 * e + 6));
+      for (int e = 0; e < kHalf / 8; ++e) {
+        const int chunk = DV == 64 ? (e ^ ((lane >> 1) & 3)) : e;
+        *reinterpret_cast<uint4*>(orow + chunk * 16) =
+            make_uint4(scaled(8 * e), scaled(8 * e + 2), scaled(8 * e + 4), scaled(8 * e + 6));
       }
+      fence_proxy_async_smem();
+      __syncwarp();
+      pend = true;
+      pend_row0 = row0;
+      pend_bh = bh;
     }
+    if (ok) flush_out();
+    if (lane == 0) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -438,9 +473,9 @@ template <int p, int DV>
 static cudaError_t launch_flash_t(const void* q, const void* k, const void* v, void* o, int BH, int T,
                                   const WaitCtl& wc, cudaStream_t st) {
   using Cfg = FlashCfg<p, DV>;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   if (!make_tmap_bf16(&tq, q, p, T, BH, kBM) || !make_tmap_bf16(&tk, k, p, T, BH, kBN) ||
-      !make_tmap_bf16(&tv, v, DV, T, BH, kBN))
+      !make_tmap_bf16(&tv, v, DV, T, BH, kBN) || !make_tmap_bf16_box(&to, o, DV, T, BH, DV / 2, 32))
     return cudaErrorInvalidValue;
   auto kern = flash_fwd_kernel<p, DV>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
@@ -455,7 +490,7 @@ static cudaError_t launch_flash_t(const void* q, const void* k, const void* v, v
   }
   const long items = (long)((T + kBM * kNQ - 1) / (kBM * kNQ)) * BH;
   const int grid = (int)(items < num_sms ? items : num_sms);
-  kern<<<grid, kThreads, Cfg::kSmemBytes, st>>>(tq, tk, tv, static_cast<__nv_bfloat16*>(o), T, BH, wc);
+  kern<<<grid, kThreads, Cfg::kSmemBytes, st>>>(tq, tk, tv, to, T, BH, wc);
   return cudaGetLastError();
 }
 
