@@ -861,8 +861,10 @@ __global__ void __launch_bounds__(kReadThreads, 1)
     };
     // running state <- scanned prefix (fp32 into TMEM, bf16 into shared
     // memory); with a single super-chunk there is no workspace and the
-    // prefix is the caller's initial state (or zero)
+    // prefix is the caller's initial state (or zero).  After a scan this
+    // kernel is its programmatic dependent: wait for the scanned records.
     const int d = min(m, kRecRows - 1);  // record row of this lane
+    griddep_wait();
     if (quarter < 3) {
       if (ws) {
         const float* row = ws + ((size_t)bh * G + g) * record_floats + (size_t)d * kNP;
@@ -974,10 +976,12 @@ cudaError_t launch_chunk_readout_sm100(const void* q, const void* k, const void*
   cudaError_t e =
       cudaFuncSetAttribute(chunk_readout_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ReadSmem::kBytes);
   if (e != cudaSuccess) return e;
-  dim3 grid(pl.G, pl.BH);
-  chunk_readout_kernel<<<grid, kReadThreads, ReadSmem::kBytes, st>>>(
-      tq, tk, tv, to, ws, S0, z0, S_out, z_out, pl.T, pl.Ls, pl.G,
-      (long long)pl.record_floats, wc);
+  const dim3 grid(pl.G, pl.BH), block(kReadThreads);
+  if (ws)  // after the state build and scan of this call: launched as the scan's programmatic dependent
+    return launch_pdl(chunk_readout_kernel, grid, block, (size_t)ReadSmem::kBytes, st, tq, tk, tv, to,
+                      (const float*)ws, S0, z0, S_out, z_out, pl.T, pl.Ls, pl.G, (long long)pl.record_floats, wc);
+  chunk_readout_kernel<<<grid, block, ReadSmem::kBytes, st>>>(tq, tk, tv, to, ws, S0, z0, S_out, z_out, pl.T, pl.Ls,
+                                                              pl.G, (long long)pl.record_floats, wc);
   return cudaGetLastError();
 }
 

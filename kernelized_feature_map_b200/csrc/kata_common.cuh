@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace kata {
 
 // Element access for the two input dtypes; arithmetic is always fp32.
@@ -24,5 +26,34 @@ __device__ __forceinline__ void report_status(int* status, int code) {
 }
 
 __host__ __device__ constexpr int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// Programmatic dependent launch.  A kernel launched by launch_pdl() may start
+// while the previous kernel in the stream is still running; griddep_wait()
+// blocks the calling thread until that kernel has completed and its memory
+// operations are visible (it returns at once when there is no such
+// dependency), and griddep_launch_dependents() lets the next kernel start
+// launching before this one finishes.  Used only between the kernels of one
+// library call, whose data dependencies are known; the first kernel of a
+// call is launched normally, so it depends fully on earlier stream work.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 }  // namespace kata

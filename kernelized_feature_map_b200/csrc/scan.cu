@@ -131,6 +131,10 @@ __device__ __forceinline__ void final_entry(const ScanArgs& a, long long bh, int
 }
 
 __global__ void __launch_bounds__(kScanThreads) state_scan_kernel(ScanArgs a) {
+  // launched while the kernel that wrote the records may still run: let the
+  // readout after it start launching, then wait for the records
+  griddep_launch_dependents();
+  griddep_wait();
   extern __shared__ float sm[];
   const int NC = a.NC, Gp_max = a.Gp;
   float* tile = sm;                       // [Gp_max][NC]
@@ -217,6 +221,8 @@ constexpr int kScanRegThreads = 256;
 
 template <int GP>
 __global__ void __launch_bounds__(kScanRegThreads) state_scan_reg_kernel(ScanArgs a) {
+  griddep_launch_dependents();
+  griddep_wait();
   const int col = blockIdx.x * kScanRegThreads + threadIdx.x;
   const long long bh = blockIdx.y;
   if (col >= a.E) return;
@@ -273,20 +279,19 @@ cudaError_t launch_state_scan(float* ws, const ChunkPlan& plan, int G_in, const 
   a.S_out = S_out;
   a.z_out = z_out;
   if (plan.G <= 32) {
-    dim3 grid(ceil_div(a.E, kScanRegThreads), plan.BH);
-    if (plan.G <= 2) state_scan_reg_kernel<2><<<grid, kScanRegThreads, 0, st>>>(a);
-    else if (plan.G <= 4) state_scan_reg_kernel<4><<<grid, kScanRegThreads, 0, st>>>(a);
-    else if (plan.G <= 8) state_scan_reg_kernel<8><<<grid, kScanRegThreads, 0, st>>>(a);
-    else if (plan.G <= 16) state_scan_reg_kernel<16><<<grid, kScanRegThreads, 0, st>>>(a);
-    else state_scan_reg_kernel<32><<<grid, kScanRegThreads, 0, st>>>(a);
-    return cudaGetLastError();
+    // the scan always follows the kernel of the same call that wrote the
+    // records: launched as its programmatic dependent
+    const dim3 grid(ceil_div(a.E, kScanRegThreads), plan.BH), block(kScanRegThreads);
+    if (plan.G <= 2) return launch_pdl(state_scan_reg_kernel<2>, grid, block, 0, st, a);
+    if (plan.G <= 4) return launch_pdl(state_scan_reg_kernel<4>, grid, block, 0, st, a);
+    if (plan.G <= 8) return launch_pdl(state_scan_reg_kernel<8>, grid, block, 0, st, a);
+    if (plan.G <= 16) return launch_pdl(state_scan_reg_kernel<16>, grid, block, 0, st, a);
+    return launch_pdl(state_scan_reg_kernel<32>, grid, block, 0, st, a);
   }
   const size_t smem = ((size_t)a.Gp * a.NC + 2 * (size_t)a.NC) * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(state_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(ceil_div(a.E, a.NC), plan.BH);
-  state_scan_kernel<<<grid, kScanThreads, smem, st>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(state_scan_kernel, dim3(ceil_div(a.E, a.NC), plan.BH), dim3(kScanThreads), smem, st, a);
 }
 
 }  // namespace kata
