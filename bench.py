@@ -51,10 +51,10 @@ UNIT = "tokens/s"
 # DRAM bytes (read + write) of one flash_fwd_kernel launch at B8 H16 T2048,
 # from the ncu capture summarised in profiles/flash_fwd_kernel_ctx2k.md.  It
 # is reported only while the kernel's sources are the ones that capture ran.
-FLASH_TRAFFIC_BYTES = 50441728 + 3565824
+FLASH_TRAFFIC_BYTES = 50633984 + 5805824
 FLASH_TRAFFIC_SOURCES = ("kernelized_feature_map_b200/csrc/flash_sm100.cu", "kernelized_feature_map_b200/csrc/sm100.cuh",
-                         "kernelized_feature_map_b200/csrc/kata_trace.cuh")
-FLASH_TRAFFIC_SHA256 = "20a25228a5551f3834785d483e0ef1f6d2070859812d2c208674fef43ab3fafb"
+                         "kernelized_feature_map_b200/csrc/kata_trace.cuh", "kernelized_feature_map_b200/csrc/kata_common.cuh")
+FLASH_TRAFFIC_SHA256 = "172325a6a08b5de78f41e033a4a6ffeaa5a2b477c0942680287c298cf2438c53"
 
 
 def flash_traffic(workload):
