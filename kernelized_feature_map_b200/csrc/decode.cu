@@ -10,8 +10,10 @@
 // (b,h).  Thread layout: DV/4 consecutive threads cover one state row with
 // 16-byte vectors, so each pass of the CTA reads 256 x 16 B contiguous
 // bytes; all of a batch's loads are issued before any use so that enough
-// bytes are in flight per SM.  Loads and stores carry the streaming hint
-// (the state is touched once per step).  psi(k)_r and psi(q)_r for the row
+// bytes are in flight per SM.  The first batch of state rows and the
+// normaliser entries are requested before q, k and v are staged, since they
+// do not depend on them, so their latency overlaps.  Loads and stores carry
+// the streaming hint (the state is touched once per step).  psi(k)_r and psi(q)_r for the row
 // r = i*p + j are formed on the fly from the p values staged in shared
 // memory.  The numerator is reduced over rows through shared memory.
 #include "kata_common.cuh"
@@ -34,8 +36,19 @@ __global__ void __launch_bounds__(256) decode_step_kernel(const Tin* __restrict_
   __shared__ float4 red[256];
   __shared__ float sden[8];
 
+  constexpr int ZPT = (P + 255) / 256;  // normaliser entries per thread
   const int tid = threadIdx.x;
   const long long bh = blockIdx.x;
+  const int cg = tid % CG;
+  const int r0 = tid / CG;
+  float4* Sb = reinterpret_cast<float4*>(S + bh * (long long)P * DV);
+  float* zb = z + bh * P;
+  float4 s[BATCH];
+#pragma unroll
+  for (int i = 0; i < BATCH; ++i) s[i] = __ldcs(Sb + (r0 + i * RPP) * CG + cg);
+  float zz[ZPT];
+#pragma unroll
+  for (int u = 0; u < ZPT; ++u) zz[u] = (tid + 256 * u < P) ? __ldcs(zb + tid + 256 * u) : 0.f;
   if (tid < p) {
     sq[tid] = Elem<Tin>::load(q + bh * p + tid);
     sk[tid] = Elem<Tin>::load(k + bh * p + tid);
@@ -43,17 +56,15 @@ __global__ void __launch_bounds__(256) decode_step_kernel(const Tin* __restrict_
   if (tid < DV) sv[tid] = Elem<Tin>::load(v + bh * DV + tid);
   __syncthreads();
 
-  const int cg = tid % CG;
-  const int r0 = tid / CG;
   const float4 vv = make_float4(sv[4 * cg], sv[4 * cg + 1], sv[4 * cg + 2], sv[4 * cg + 3]);
-  float4* Sb = reinterpret_cast<float4*>(S + bh * (long long)P * DV);
 
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 1
   for (int b0 = 0; b0 < PASSES; b0 += BATCH) {
-    float4 s[BATCH];
+    if (b0 > 0) {
 #pragma unroll
-    for (int i = 0; i < BATCH; ++i) s[i] = __ldcs(Sb + (r0 + (b0 + i) * RPP) * CG + cg);
+      for (int i = 0; i < BATCH; ++i) s[i] = __ldcs(Sb + (r0 + (b0 + i) * RPP) * CG + cg);
+    }
 #pragma unroll
     for (int i = 0; i < BATCH; ++i) {
       const int r = r0 + (b0 + i) * RPP;
@@ -74,12 +85,15 @@ __global__ void __launch_bounds__(256) decode_step_kernel(const Tin* __restrict_
 
   // normaliser z and the denominator psi(q)^T z
   float den = 0.f;
-  float* zb = z + bh * P;
-  for (int r = tid; r < P; r += 256) {
-    const int ii = r / p, jj = r % p;
-    const float zz = __ldcs(zb + r) + sk[ii] * sk[jj];
-    __stcs(zb + r, zz);
-    den = fmaf(sq[ii] * sq[jj], zz, den);
+#pragma unroll
+  for (int u = 0; u < ZPT; ++u) {
+    const int r = tid + 256 * u;
+    if (r < P) {
+      const int ii = r / p, jj = r % p;
+      const float zn = zz[u] + sk[ii] * sk[jj];
+      __stcs(zb + r, zn);
+      den = fmaf(sq[ii] * sq[jj], zn, den);
+    }
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
