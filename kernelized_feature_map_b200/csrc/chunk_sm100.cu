@@ -564,13 +564,15 @@ __global__ void __launch_bounds__(kStateThreads, 1)
 //   14-17        each pair of warps on a TMEM lane quarter splits the columns
 //   warps 6-9    psi~(k_{c+1}) into shared memory (two buffers); bf16 copy of
 //                packed coordinates 0..71 of the state after chunk c
-//   warps 10-13  prefix state in; bf16 copy of coordinates 72..143; then
-//                psi~(q_{c+1}) into TMEM
-// MMA order per chunk c: scores of chunk c, advance S~ by chunk c, readout of
-// chunk c against the bf16 copy of S~ made before chunk c, intra-chunk
-// weights.  The readout reads only the bf16 copy, so the state can advance
-// first; the copy for chunk c+1 is refreshed while the readout and
-// intra-chunk MMAs of chunk c run (the copy is double-buffered).
+//   warps 10-13  prefix state in; psi~(q_{c+1}) into TMEM once the readout of
+//                chunk c has read psi~(q_c); then the bf16 copy of coordinates
+//                72..143
+// MMA order per chunk c: scores of chunk c, readout of chunk c against the
+// bf16 copy of S~ made before chunk c, advance S~ by chunk c, intra-chunk
+// weights.  The readout reads only the bf16 copy, and comes first so that
+// psi~(q_c) is released early; the copy for chunk c+1 is refreshed once the
+// advance lands, while the intra-chunk MMAs of chunk c run (the copy is
+// double-buffered).
 // The MMA warp waits on two barriers per chunk.  state_full(c) is arrived on
 // by warps 6-13 after everything chunk c needs from them (its psi~(k), its
 // psi~(q), the bf16 copy; each of them waited for chunk c's tiles to land
@@ -703,21 +705,22 @@ __global__ void __launch_bounds__(kReadThreads, 1)
         // the intra-chunk MMAs of c-1 issued before them)
         mma_ss_w(tmem + L::colS, desc_add(dq0, st * L::kStage), desc_add(dk0, st * L::kStage), id_qk, 0);
         mma_commit_w(s_full);
-        // advance the state by the chunk
-        const uint64_t dvo = desc_vones(sV, sOnes);
-#pragma unroll
-        for (int ks = 0; ks < kTile / 16; ++ks)
-          mma_ss_w(tmem + L::colRun, desc_add(dvo, ks * 2048), desc_add(dpsi, (c & 1) * kPsiBytes + ks * 512), id_u, 1);
-        mma_commit_w(upd_done);
-        KATA_TRACE(chunk, c, 2);
         // readout against the bf16 copy of the state entering the chunk (the
-        // [O | D] buffer is free: see state_full)
+        // [O | D] buffer is free: see state_full); first, so that psi~(q_c)
+        // is released early for psi~(q_{c+1})
         const uint64_t dsb = desc_add(dsb0, ob * kSBBytes);
         const uint32_t dO = tmem + L::colO(ob);
 #pragma unroll
         for (int ks = 0; ks < kNP / 16; ++ks)
           mma_ts_w(dO, tmem + L::colPQ + ks * 8, desc_add(dsb, ks * kSBAtom), id_rd, ks > 0);
         mma_commit_w(rd_done);
+        KATA_TRACE(chunk, c, 2);
+        // advance the state by the chunk
+        const uint64_t dvo = desc_vones(sV, sOnes);
+#pragma unroll
+        for (int ks = 0; ks < kTile / 16; ++ks)
+          mma_ss_w(tmem + L::colRun, desc_add(dvo, ks * 2048), desc_add(dpsi, (c & 1) * kPsiBytes + ks * 512), id_u, 1);
+        mma_commit_w(upd_done);
         // intra-chunk weights against [V_c | 1]
         KATA_TRACE(chunk, c, 4);
         if (!mbar_wait_w(p_full, c & 1, env)) break;
@@ -900,6 +903,16 @@ __global__ void __launch_bounds__(kReadThreads, 1)
         // c-1, which this group saw complete in the previous iteration
         psi_k(c + 1);
         if (m == 0) KATA_TRACE(chunk, c, 11);
+      } else {
+        // psi~(q_{c+1}) into TMEM once the readout of chunk c (the first MMAs
+        // of the chunk) has read psi~(q_c)
+        uint32_t wq[kNPW];
+        psi_q_formed(c + 1, wq);
+        if (!mbar_wait(rd_done, c & 1, env)) break;
+        if (m == 0) KATA_TRACE(chunk, c, 19);
+        tc_fence_after();
+        store_psi_q_tmem(lane_base + L::colPQ, wq);
+        tmem_wait_st();
       }
       // the state after chunk c is complete: this group's half of the bf16
       // copy for the readout of chunk c+1 (its buffer was last read by the
@@ -909,16 +922,6 @@ __global__ void __launch_bounds__(kReadThreads, 1)
       tc_fence_after();
       if (quarter < 3) state_half_to_bf16(lane_base + L::colRun, sb + ((c + 1) & 1) * kSBBytes, m, active, half);
       if (m == 0) KATA_TRACE(chunk, c, psi_group ? 17 : 18);
-      if (!psi_group) {
-        // psi~(q_{c+1}) into TMEM once the readout of chunk c has read psi~(q_c)
-        uint32_t wq[kNPW];
-        psi_q_formed(c + 1, wq);
-        if (!mbar_wait(rd_done, c & 1, env)) break;
-        if (m == 0) KATA_TRACE(chunk, c, 19);
-        tc_fence_after();
-        store_psi_q_tmem(lane_base + L::colPQ, wq);
-        tmem_wait_st();
-      }
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(state_full);
