@@ -18,6 +18,12 @@ marshals numpy arrays through ctypes.  Functions:
   o_t = psi(q_t)^T S_t / psi(q_t)^T z_t, with optional initial and final
   state (ai.info summary, Methodology in Plain English).
 * :func:`decode_step` -- one step of that recurrence from a given state.
+* :func:`direct_mg`, :func:`direct_mg_rows`, :func:`recurrent_mg`,
+  :func:`decode_step_mg` -- the same for KATA-Mg: the head's d coordinates
+  split into g groups of width d/g, weight sum_j (q_t^j . k_s^j)^2, one
+  shared value vector and denominator, state [g*(d/g)^2, dv] (arXiv
+  abstract; gist.science sec. 2.3 "Varianten"; ai.info Main Findings, the
+  KATA-Mg state size d(d/g+1)/2 * dv).
 
 Readings (the pages leave these open): inclusive causal sum (s <= t);
 D_t = 0 gives o_t = 0; no score scaling; q, k used as given.
@@ -67,8 +73,18 @@ def _load():
             lib.kata_oracle_recurrent.argtypes = [_dp, _dp, _dp, _dp, ctypes.c_int64, ctypes.c_int64,
                                                   ctypes.c_int64, ctypes.c_int, ctypes.c_int,
                                                   _dp, _dp, _dp, _dp, ctypes.c_int]
+            lib.kata_oracle_direct_mg.argtypes = [_dp, _dp, _dp, _dp, ctypes.c_int64, ctypes.c_int64,
+                                                  ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                  ctypes.c_int]
+            lib.kata_oracle_direct_mg_rows.argtypes = [_dp, _dp, _dp, ctypes.c_int64, ctypes.c_int64,
+                                                       ctypes.c_int, ctypes.c_int, ctypes.c_int, _ip, _ip,
+                                                       ctypes.c_int64, _dp, _dp]
+            lib.kata_oracle_recurrent_mg.argtypes = [_dp, _dp, _dp, _dp, ctypes.c_int64, ctypes.c_int64,
+                                                     ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                     _dp, _dp, _dp, _dp, ctypes.c_int]
             lib.kata_oracle_default_threads.argtypes = []
             for f in (lib.kata_oracle_direct, lib.kata_oracle_direct_rows, lib.kata_oracle_recurrent,
+                      lib.kata_oracle_direct_mg, lib.kata_oracle_direct_mg_rows, lib.kata_oracle_recurrent_mg,
                       lib.kata_oracle_default_threads):
                 f.restype = ctypes.c_int
             _lib = lib
@@ -161,4 +177,80 @@ def decode_step(q, k, v, S, z, nthreads: int = 0):
     q, k, v = _f64(q), _f64(k), _f64(v)
     o, S1, z1 = recurrent(q[:, :, None, :], k[:, :, None, :], v[:, :, None, :], S, z,
                           return_state=True, nthreads=nthreads)
+    return o[:, :, 0, :], S1, z1
+
+
+# ---------------------------------------------------------------------------
+# KATA-Mg: g PSD factors over a head of width d
+# ---------------------------------------------------------------------------
+
+def _shape_mg(q, k, v, groups):
+    B, H, T, d, dv = _shape(q, k, v)
+    if groups < 1 or d % groups != 0:
+        raise ValueError("groups must divide the head width d")
+    return B, H, T, d, dv
+
+
+def direct_mg(q, k, v, groups: int, nthreads: int = 0) -> np.ndarray:
+    """o [B,H,T,dv] from the defining sum with w_ts = sum_j (q_t^j . k_s^j)^2 (fp64).
+
+    q, k are [B,H,T,d]; group j is coordinates j*d/g .. (j+1)*d/g - 1.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, T, d, dv = _shape_mg(q, k, v, groups)
+    o = np.empty((B, H, T, dv), np.float64)
+    _check(_load().kata_oracle_direct_mg(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, T, d, groups, dv, nthreads))
+    return o
+
+
+def direct_mg_rows(q, k, v, groups: int, bh_idx, t_idx, return_d: bool = False):
+    """:func:`direct_mg` on rows (bh_idx[r], t_idx[r]).  Returns o_rows [R,dv] (and D [R])."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, T, d, dv = _shape_mg(q, k, v, groups)
+    bh_idx = np.ascontiguousarray(bh_idx, dtype=np.int64)
+    t_idx = np.ascontiguousarray(t_idx, dtype=np.int64)
+    if bh_idx.shape != t_idx.shape or bh_idx.ndim != 1:
+        raise ValueError("bh_idx and t_idx must be 1-D of equal length")
+    R = bh_idx.shape[0]
+    o = np.empty((R, dv), np.float64)
+    dd = np.empty((R,), np.float64) if return_d else None
+    _check(_load().kata_oracle_direct_mg_rows(_ptr(q), _ptr(k), _ptr(v), B * H, T, d, groups, dv,
+                                              bh_idx.ctypes.data_as(_ip), t_idx.ctypes.data_as(_ip), R,
+                                              _ptr(o), _ptr(dd)))
+    return (o, dd) if return_d else o
+
+
+def recurrent_mg(q, k, v, groups: int, S0=None, z0=None, return_state: bool = False, nthreads: int = 0):
+    """Explicit psi_Mg recurrence (fp64) on the state [B,H,g*p*p,dv], p = d/g.
+
+    Row r = j*p*p + a*p + b of the state belongs to group j and holds the
+    products of its coordinates a and b.  Returns o, or (o, S_T, z_T).
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, T, d, dv = _shape_mg(q, k, v, groups)
+    p = d // groups
+    P = groups * p * p
+    if (S0 is None) != (z0 is None):
+        raise ValueError("give both S0 and z0 or neither")
+    if S0 is not None:
+        S0 = _f64(S0).reshape(B, H, P, dv)
+        z0 = _f64(z0).reshape(B, H, P)
+    o = np.empty((B, H, T, dv), np.float64)
+    S_out = np.empty((B, H, P, dv), np.float64) if return_state else None
+    z_out = np.empty((B, H, P), np.float64) if return_state else None
+    _check(_load().kata_oracle_recurrent_mg(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, T, d, groups, dv,
+                                            _ptr(S0), _ptr(z0), _ptr(S_out), _ptr(z_out), nthreads))
+    if return_state:
+        return o, S_out, z_out
+    return o
+
+
+def decode_step_mg(q, k, v, S, z, groups: int, nthreads: int = 0):
+    """One Mg recurrent step: q,k [B,H,d], v [B,H,dv], S [B,H,g*p*p,dv], z [B,H,g*p*p].
+
+    Update with (k, v) first, then read with q.  Returns (o [B,H,dv], S_new, z_new).
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    o, S1, z1 = recurrent_mg(q[:, :, None, :], k[:, :, None, :], v[:, :, None, :], groups, S, z,
+                             return_state=True, nthreads=nthreads)
     return o[:, :, 0, :], S1, z1

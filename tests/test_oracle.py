@@ -305,3 +305,128 @@ def test_pins_catch_planted_mistakes(tmp_path, name):
     lo, hi = np.minimum.accumulate(vr, axis=2), np.maximum.accumulate(vr, axis=2)
     caught = caught or not (np.all(o >= lo - 1e-12) and np.all(o <= hi + 1e-12))
     assert caught, "pin set failed to catch: " + name
+
+
+# ---------------------------------------------------------------------------
+# KATA-Mg (g PSD factors over a head of width d): pins of the grouped oracle
+# ---------------------------------------------------------------------------
+
+def _rand_mg(B=1, H=2, T=30, d=8, dv=3, seed=40):
+    rng = np.random.default_rng(seed)
+    return (rng.standard_normal((B, H, T, d)), rng.standard_normal((B, H, T, d)),
+            rng.standard_normal((B, H, T, dv)))
+
+
+def test_mg_one_group_is_the_full_map():
+    """g = 1 is the full rank-one map (ai.info, Main Findings: both reduced
+    families recover the full map at g = 1)."""
+    q, k, v = _rand_mg(d=6, seed=41)
+    np.testing.assert_allclose(oracle.direct_mg(q, k, v, 1), oracle.direct(q, k, v), rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("d,g", [(8, 2), (8, 4), (12, 3), (6, 6)])
+def test_mg_direct_equals_recurrent(d, g):
+    q, k, v = _rand_mg(d=d, seed=42 + d + g)
+    np.testing.assert_allclose(oracle.recurrent_mg(q, k, v, g), oracle.direct_mg(q, k, v, g),
+                               rtol=1e-10, atol=1e-12)
+
+
+@pytest.mark.parametrize("j0", [0, 2])
+def test_mg_single_active_group_reduces_to_one_factor(j0):
+    """With every query group but j0 zero, only (q^j0 . k^j0)^2 is left: the
+    single-factor oracle on the j0 slices, whatever the other key groups hold."""
+    d, g = 12, 3
+    p = d // g
+    q, k, v = _rand_mg(d=d, seed=50 + j0)
+    qz = np.zeros_like(q)
+    qz[..., j0 * p:(j0 + 1) * p] = q[..., j0 * p:(j0 + 1) * p]
+    want = oracle.direct(qz[..., j0 * p:(j0 + 1) * p], k[..., j0 * p:(j0 + 1) * p], v)
+    np.testing.assert_allclose(oracle.direct_mg(qz, k, v, g), want, rtol=1e-11, atol=1e-12)
+
+
+def test_mg_width_one_groups_closed_form():
+    """g = d (groups of width 1): w_ts = sum_i q_i^2 k_i^2, i.e. first-order
+    linear attention with the feature u -> u*u, evaluated by cumulative sums."""
+    rng = np.random.default_rng(60)
+    T, d, dv = 30, 5, 3
+    q = rng.standard_normal((1, 1, T, d))
+    k = rng.standard_normal((1, 1, T, d))
+    v = rng.standard_normal((1, 1, T, dv))
+    fq, fk = q[0, 0] ** 2, k[0, 0] ** 2
+    S = np.cumsum(fk[:, :, None] * v[0, 0][:, None, :], axis=0)  # [T, d, dv]
+    z = np.cumsum(fk, axis=0)
+    want = np.einsum("ti,tie->te", fq, S) / np.einsum("ti,ti->t", fq, z)[:, None]
+    np.testing.assert_allclose(oracle.direct_mg(q, k, v, d)[0, 0], want, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(oracle.recurrent_mg(q, k, v, d)[0, 0], want, rtol=1e-11, atol=1e-12)
+
+
+@pytest.mark.parametrize("d,g", [(8, 1), (8, 2), (8, 4), (12, 3)])
+def test_mg_feature_dimension_matches_state_size_formula(d, g):
+    """The psi_Mg features of random vectors span exactly d(d/g+1)/2
+    dimensions, the packed KATA-Mg state width per value column (ai.info,
+    Main Findings).  A cross-group product or a dropped group changes it."""
+    rng = np.random.default_rng(70 + d + g)
+    p = d // g
+    P = g * p * p
+    n = 3 * P
+    u = rng.standard_normal((1, n, d))
+    # from the zero state one step leaves z = psi_Mg(k)
+    _, _, z = oracle.decode_step_mg(u, u, np.ones((1, n, 1)), np.zeros((1, n, P, 1)), np.zeros((1, n, P)), g)
+    assert np.linalg.matrix_rank(z[0]) == d * (d // g + 1) // 2
+
+
+def test_mg_gate_properties_and_group_permutation():
+    d, g = 8, 4
+    p = d // g
+    q, k, v = _rand_mg(T=25, d=d, seed=80)
+    o = oracle.direct_mg(q, k, v, g)
+    np.testing.assert_allclose(o[:, :, 0], v[:, :, 0], rtol=1e-12, atol=1e-12)   # o_1 = v_1
+    lo, hi = np.minimum.accumulate(v, axis=2), np.maximum.accumulate(v, axis=2)
+    assert np.all(o >= lo - 1e-12) and np.all(o <= hi + 1e-12)                  # convex gate
+    kk = np.broadcast_to(k[:, :, :1], k.shape)                                    # identical keys
+    want = np.cumsum(v, axis=2) / np.arange(1, v.shape[2] + 1)[None, None, :, None]
+    np.testing.assert_allclose(oracle.direct_mg(q, kk, v, g), want, rtol=1e-11, atol=1e-12)
+    perm = np.concatenate([np.arange(j * p, (j + 1) * p) for j in (2, 0, 3, 1)])
+    np.testing.assert_allclose(oracle.direct_mg(q[..., perm], k[..., perm], v, g), o, rtol=1e-11, atol=1e-12)
+
+
+MUTATIONS_MG = {
+    "cross-group products": ("dot += q_t[j * p + i] * k_s[j * p + i];",
+                             "dot += q_t[j * p + i] * k_s[((j + 1) % g) * p + i];"),
+    "last group dropped": ("for (int j = 0; j < g; ++j) {\n    double dot", "for (int j = 0; j < g - 1; ++j) {\n    double dot"),
+    "squared sum instead of sum of squares": ("    w += dot * dot;\n  }\n  return w;", "    w += dot;\n  }\n  return w * w;"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS_MG))
+def test_mg_pins_catch_planted_mistakes(tmp_path, name):
+    old, new = MUTATIONS_MG[name]
+    lib = _build_mutant(tmp_path, name, old, new)
+    dp = ctypes.POINTER(ctypes.c_double)
+    lib.kata_oracle_direct_mg.argtypes = [dp, dp, dp, dp, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                          ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]
+
+    def mutant(q, k, v, g):
+        q, k, v = (np.ascontiguousarray(x, np.float64) for x in (q, k, v))
+        B, H, T, d = q.shape
+        o = np.empty((B, H, T, v.shape[3]))
+        lib.kata_oracle_direct_mg(q.ctypes.data_as(dp), k.ctypes.data_as(dp), v.ctypes.data_as(dp),
+                                  o.ctypes.data_as(dp), B, H, T, d, g, v.shape[3], 1)
+        return o
+
+    d, g, p = 12, 3, 4
+    q, k, v = _rand_mg(d=d, seed=90)
+    caught = False
+    # the single-active-group reduction, for the first and the last group
+    for j0 in (0, g - 1):
+        qz = np.zeros_like(q)
+        qz[..., j0 * p:(j0 + 1) * p] = q[..., j0 * p:(j0 + 1) * p]
+        want = oracle.direct(qz[..., j0 * p:(j0 + 1) * p], k[..., j0 * p:(j0 + 1) * p], v)
+        caught = caught or not np.allclose(mutant(qz, k, v, g), want, atol=1e-10)
+    # the width-one closed form
+    q1, k1, v1 = _rand_mg(B=1, H=1, T=20, d=5, seed=91)
+    fq, fk = q1[0, 0] ** 2, k1[0, 0] ** 2
+    S = np.cumsum(fk[:, :, None] * v1[0, 0][:, None, :], axis=0)
+    want = np.einsum("ti,tie->te", fq, S) / np.einsum("ti,ti->t", fq, np.cumsum(fk, axis=0))[:, None]
+    caught = caught or not np.allclose(mutant(q1, k1, v1, 5)[0, 0], want, atol=1e-10)
+    assert caught, "Mg pin set failed to catch: " + name
