@@ -277,3 +277,48 @@ def test_full_size_sampled_rows(kata, name, path):
     vmax = np.abs(v.reshape(B * H, -1)).max(axis=1)[bh_idx]
     err = rows_rel_err(o[bh_idx, t_idx], ref, vmax)
     assert err <= TOL["bf16"], err
+
+
+# ---------------------------------------------------------------------------
+# CUDA graph capture: the calls only enqueue work on the caller's stream (the
+# chunked call with several super-chunks launches state build, scan and
+# readout, the last two as programmatic dependents), so a captured step
+# replays to the same bits as the eager calls
+# ---------------------------------------------------------------------------
+
+def test_graph_replay_matches_eager(kata):
+    import torch
+    B, H, T, p, dv = 1, 2, 20000, 16, 64  # several super-chunks per head
+    q, k, v = workloads.normal_qkv(B, H, T, p, dv, seed=11, dtype="bf16")
+    qd, kd, vd = to_dev(q, "bf16"), to_dev(k, "bf16"), to_dev(v, "bf16")
+    ws = torch.empty(max(256, kata.kata_fwd_chunked_workspace_size(B, H, T, p, dv, 64)), dtype=torch.uint8,
+                     device="cuda")
+    oq, oc = torch.empty_like(vd), torch.empty_like(vd)
+    S = torch.empty((B, H, p * p, dv), dtype=torch.float32, device="cuda")
+    z = torch.empty((B, H, p * p), dtype=torch.float32, device="cuda")
+    qt, kt, vt = qd[:, :, :1].contiguous(), kd[:, :, :1].contiguous(), vd[:, :, :1].contiguous()
+    od = torch.empty((B, H, dv), dtype=torch.bfloat16, device="cuda")
+
+    def step():
+        kata.kata_fwd_quadratic(qd, kd, vd, o=oq)
+        kata.kata_fwd_chunked(qd, kd, vd, C=64, o=oc, workspace=ws, S_out=S, z_out=z, return_state=True)
+        kata.kata_decode_step(qt[:, :, 0], kt[:, :, 0], vt[:, :, 0], S, z, o=od)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    ref = [t.clone() for t in (oq, oc, S, z, od)]
+    for t in (oq, oc, S, z, od):
+        t.zero_()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    g.replay()
+    torch.cuda.synchronize()
+    assert kata.kata_get_status() == 0
+    for got, want in zip((oq, oc, S, z, od), ref):
+        assert torch.equal(got, want)
+    del g
