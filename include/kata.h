@@ -178,6 +178,50 @@ kata_status_t kata_decode_step(const void* q, const void* k, const void* v, void
                                kata_dtype_t dtype, void* stream);
 
 /*
+ * KATA-Mg: g PSD factors per head (arXiv abstract and gist.science sec. 2.3
+ * "Varianten": several PSD factors; ai.info summary, Main Findings: state
+ * d(d/g+1)/2 * dv packed, the full map at g = 1).  The head's d coordinates
+ * split into `groups` consecutive groups of width p = d / groups,
+ * u = [u^1 | ... | u^g], and the feature is the concatenation of the group
+ * maps, psi_Mg(u) = [psi(u^1) | ... | psi(u^g)], so that
+ *
+ *   w_{t,s} = sum_j (q_t^j . k_s^j)^2,   o_t = sum_{s<=t} w_{t,s} v_s / sum_{s<=t} w_{t,s}
+ *
+ * with one value vector and one denominator shared by all groups.
+ *
+ * Layouts of q, k ([.., d]) and v, o ([.., dv]) for the forward call:
+ *   KATA_LAYOUT_BHTD  [B, H, T, *] as in the entry points above;
+ *   KATA_LAYOUT_BTHD  [B, T, H, *], the layout of the pages' attention call
+ *                     (KATA repository README: (B,T,H,D) in and out),
+ *                     read and written in place through strided tile copies.
+ */
+typedef enum { KATA_LAYOUT_BHTD = 0, KATA_LAYOUT_BTHD = 1 } kata_layout_t;
+
+/*
+ * Quadratic (flash-style) KATA-Mg forward.  bf16 only; supported
+ * (p = d/groups, groups, dv): groups = 1 with p in {16, 32} and dv in
+ * {16, 64} (the single-factor kernel of kata_fwd_quadratic), and dv = 64 with
+ * (16, 2), (16, 4) or (32, 2).  Other shapes or fp32: KATA_ERR_UNSUPPORTED;
+ * groups < 1 or d not a multiple of groups: KATA_ERR_INVALID_ARG.  Pointers,
+ * streams, errors and the zero gate as above.
+ */
+kata_status_t kata_fwd_mg_quadratic(const void* q, const void* k, const void* v, void* o,
+                                    int B, int H, int T, int d, int groups, int dv,
+                                    kata_layout_t layout, kata_dtype_t dtype, void* stream);
+
+/*
+ * One KATA-Mg decode step (update with (k, v), then read with q):
+ * q, k: [B,H,d]; v, o: [B,H,dv] (fp32 or bf16); S: [B,H,groups*p*p,dv] and
+ * z: [B,H,groups*p*p] fp32, read and updated in place, with row
+ * r = j*p*p + a*p + b holding the products of coordinates j*p + a and
+ * j*p + b (group j).  Supported (p, groups, dv) as for
+ * kata_fwd_mg_quadratic, in either dtype.
+ */
+kata_status_t kata_decode_step_mg(const void* q, const void* k, const void* v, void* o,
+                                  float* S, float* z, int B, int H, int d, int groups, int dv,
+                                  kata_dtype_t dtype, void* stream);
+
+/*
  * Synchronises `stream`, then returns and clears the device-side status word
  * of the current device (KATA_ERR_TIMEOUT if a bounded wait in a kernel ran
  * out since the last call), or KATA_ERR_CUDA if the stream reports an error.
@@ -199,7 +243,7 @@ void kata_set_wait_limit(long long cycles);
 /* ABI version of this header: major * 10000 + minor * 100 + patch. */
 int kata_abi_version(void);
 
-#define KATA_ABI_VERSION 10000
+#define KATA_ABI_VERSION 10100
 
 #ifdef __cplusplus
 }

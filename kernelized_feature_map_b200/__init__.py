@@ -13,9 +13,13 @@ The computation lives in ``libkata.so`` (hand-written CUDA behind the C ABI of
 * :func:`kata_fwd_chunked_noalloc` -- the chunked forward using a fixed
   library-owned scratch array, for callers that cannot allocate;
 * :func:`kata_fwd_chunked_sequential` -- the sequential inter-chunk baseline
-  (one CTA per sequence walks its chunks in order, no scan).
+  (one CTA per sequence walks its chunks in order, no scan);
+* :func:`kata_fwd_mg_quadratic`, :func:`kata_decode_step_mg` -- KATA-Mg, with
+  several PSD factors per head (score sum_j (q^j . k^j)^2), the forward in
+  the [B,H,T,d] or [B,T,H,d] layout;
+* :func:`parallel_kata_attn` -- the pages' call shape, [B,T,H,D] in and out.
 """
 from ._abi import (KataError, kata_abi_version, kata_decode_step, kata_fwd_chunked,  # noqa: F401
                    kata_fwd_chunked_noalloc, kata_fwd_chunked_sequential, kata_fwd_chunked_workspace_size,
-                   kata_fwd_quadratic,
+                   kata_fwd_quadratic, kata_fwd_mg_quadratic, kata_decode_step_mg, parallel_kata_attn,
                    kata_get_status, kata_set_wait_limit, lib, status_string)

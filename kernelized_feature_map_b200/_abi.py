@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(_PKG, "libkata.so")
 KATA_OK, KATA_ERR_INVALID_ARG, KATA_ERR_UNSUPPORTED, KATA_ERR_MISALIGNED = 0, 1, 2, 3
 KATA_ERR_WORKSPACE, KATA_ERR_CUDA, KATA_ERR_TIMEOUT = 4, 5, 6
 KATA_F32, KATA_BF16 = 0, 1
+KATA_LAYOUT_BHTD, KATA_LAYOUT_BTHD = 0, 1
 
 # name -> (restype, argtypes), mirroring include/kata.h
 _c_int, _c_size, _vp, _fp = ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p
@@ -31,6 +32,8 @@ SIGNATURES = {
     "kata_fwd_chunked_sequential": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                              _c_int, _fp, _fp, _fp, _fp, _vp]),
     "kata_decode_step": (_c_int, [_vp, _vp, _vp, _vp, _fp, _fp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp]),
+    "kata_fwd_mg_quadratic": (_c_int, [_vp, _vp, _vp, _vp] + [_c_int] * 8 + [_vp]),
+    "kata_decode_step_mg": (_c_int, [_vp, _vp, _vp, _vp, _fp, _fp] + [_c_int] * 6 + [_vp]),
     "kata_get_status": (_c_int, [_vp]),
     "kata_status_string": (ctypes.c_char_p, [_c_int]),
     "kata_set_wait_limit": (None, [ctypes.c_longlong]),
@@ -202,6 +205,50 @@ def kata_decode_step(q, k, v, S, z, o=None, stream=None):
     _check("kata_decode_step", lib().kata_decode_step(
         _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), _dev(S, "S"), _dev(z, "z"), B, H, p, dv,
         _dtype_code(q), _stream_ptr(stream)))
+    return o
+
+
+def kata_fwd_mg_quadratic(q, k, v, groups, layout="bhtd", o=None, stream=None):
+    """Flash-style KATA-Mg forward with `groups` PSD factors per head.
+
+    layout "bhtd": q,k [B,H,T,d], v,o [B,H,T,dv]; layout "bthd": q,k
+    [B,T,H,d], v,o [B,T,H,dv].  The score of a pair is the sum over the
+    groups (consecutive blocks of d/groups coordinates) of the squared group
+    dot products.
+    """
+    if layout == "bhtd":
+        B, H, T, d = q.shape
+        code = KATA_LAYOUT_BHTD
+    elif layout == "bthd":
+        B, T, H, d = q.shape
+        code = KATA_LAYOUT_BTHD
+    else:
+        raise ValueError("layout must be 'bhtd' or 'bthd'")
+    dv = v.shape[-1]
+    if o is None:
+        o = torch.empty(v.shape, dtype=q.dtype, device=q.device)
+    _check("kata_fwd_mg_quadratic", lib().kata_fwd_mg_quadratic(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), B, H, T, d, int(groups), dv, code,
+        _dtype_code(q), _stream_ptr(stream)))
+    return o
+
+
+def parallel_kata_attn(q, k, v, num_groups=2, stream=None):
+    """The pages' attention call shape: q,k,v [B,T,H,D] -> o [B,T,H,D], with
+    num_groups PSD factors per head (KATA-Mg, forward only)."""
+    return kata_fwd_mg_quadratic(q, k, v, num_groups, layout="bthd", stream=stream)
+
+
+def kata_decode_step_mg(q, k, v, S, z, groups, o=None, stream=None):
+    """One KATA-Mg decode step: q,k [B,H,d], v [B,H,dv]; S [B,H,groups*p*p,dv]
+    and z [B,H,groups*p*p] (fp32, p = d/groups) are updated in place."""
+    B, H, d = q.shape
+    dv = v.shape[-1]
+    if o is None:
+        o = torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
+    _check("kata_decode_step_mg", lib().kata_decode_step_mg(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), _dev(S, "S"), _dev(z, "z"), B, H, d, int(groups),
+        dv, _dtype_code(q), _stream_ptr(stream)))
     return o
 
 

@@ -16,23 +16,29 @@
 // the streaming hint (the state is touched once per step).  psi(k)_r and psi(q)_r for the row
 // r = i*p + j are formed on the fly from the p values staged in shared
 // memory.  The numerator is reduced over rows through shared memory.
+//
+// KATA-Mg (G factors of width p per head, q and k rows of d = G*p values):
+// the feature is the concatenation of the G group maps, so the state has
+// G*p*p rows and row r = g*p*p + i*p + j holds the products of coordinates
+// g*p + i and g*p + j; G = 1 is the single-factor step above.
 #include "kata_common.cuh"
 #include "kata_internal.h"
 
 namespace kata {
 
-template <typename Tin, int p, int DV>
+template <typename Tin, int p, int DV, int G>
 __global__ void __launch_bounds__(256) decode_step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
                                                           const Tin* __restrict__ v, Tin* __restrict__ o,
                                                           float* __restrict__ S, float* __restrict__ z) {
-  constexpr int P = p * p;
+  constexpr int D = G * p;          // q/k row width
+  constexpr int P = G * p * p;      // state rows
   constexpr int CG = DV / 4;        // 16-byte column groups per state row
   constexpr int RPP = 256 / CG;     // rows covered by one pass of the CTA
   constexpr int PASSES = P / RPP;   // passes over the state
   constexpr int BATCH = PASSES < 16 ? PASSES : 16;
   static_assert(PASSES % BATCH == 0, "pass batching");
 
-  __shared__ float sq[p], sk[p], sv[DV];
+  __shared__ float sq[D], sk[D], sv[DV];
   __shared__ float4 red[256];
   __shared__ float sden[8];
 
@@ -49,9 +55,9 @@ __global__ void __launch_bounds__(256) decode_step_kernel(const Tin* __restrict_
   float zz[ZPT];
 #pragma unroll
   for (int u = 0; u < ZPT; ++u) zz[u] = (tid + 256 * u < P) ? __ldcs(zb + tid + 256 * u) : 0.f;
-  if (tid < p) {
-    sq[tid] = Elem<Tin>::load(q + bh * p + tid);
-    sk[tid] = Elem<Tin>::load(k + bh * p + tid);
+  if (tid < D) {
+    sq[tid] = Elem<Tin>::load(q + bh * D + tid);
+    sk[tid] = Elem<Tin>::load(k + bh * D + tid);
   }
   if (tid < DV) sv[tid] = Elem<Tin>::load(v + bh * DV + tid);
   __syncthreads();
@@ -68,7 +74,7 @@ __global__ void __launch_bounds__(256) decode_step_kernel(const Tin* __restrict_
 #pragma unroll
     for (int i = 0; i < BATCH; ++i) {
       const int r = r0 + (b0 + i) * RPP;
-      const int ii = r / p, jj = r % p;
+      const int gp = (r / (p * p)) * p, ii = gp + (r % (p * p)) / p, jj = gp + r % p;
       const float pk = sk[ii] * sk[jj];
       const float pq = sq[ii] * sq[jj];
       s[i].x = fmaf(pk, vv.x, s[i].x);
@@ -89,7 +95,7 @@ __global__ void __launch_bounds__(256) decode_step_kernel(const Tin* __restrict_
   for (int u = 0; u < ZPT; ++u) {
     const int r = tid + 256 * u;
     if (r < P) {
-      const int ii = r / p, jj = r % p;
+      const int gp = (r / (p * p)) * p, ii = gp + (r % (p * p)) / p, jj = gp + r % p;
       const float zn = zz[u] + sk[ii] * sk[jj];
       __stcs(zb + r, zn);
       den = fmaf(sq[ii] * sq[jj], zn, den);
@@ -116,27 +122,33 @@ __global__ void __launch_bounds__(256) decode_step_kernel(const Tin* __restrict_
   }
 }
 
-template <typename Tin, int p, int DV>
+template <typename Tin, int p, int DV, int G>
 static cudaError_t launch_decode_t(const void* q, const void* k, const void* v, void* o, float* S, float* z,
                                    int BH, cudaStream_t st) {
-  decode_step_kernel<Tin, p, DV><<<BH, 256, 0, st>>>((const Tin*)q, (const Tin*)k, (const Tin*)v, (Tin*)o, S, z);
+  decode_step_kernel<Tin, p, DV, G><<<BH, 256, 0, st>>>((const Tin*)q, (const Tin*)k, (const Tin*)v, (Tin*)o, S, z);
   return cudaGetLastError();
 }
 
 template <typename Tin>
 static cudaError_t launch_decode_dt(const void* q, const void* k, const void* v, void* o, float* S, float* z,
-                                    int BH, int p, int dv, cudaStream_t st) {
-  if (p == 16 && dv == 64) return launch_decode_t<Tin, 16, 64>(q, k, v, o, S, z, BH, st);
-  if (p == 16 && dv == 16) return launch_decode_t<Tin, 16, 16>(q, k, v, o, S, z, BH, st);
-  if (p == 32 && dv == 64) return launch_decode_t<Tin, 32, 64>(q, k, v, o, S, z, BH, st);
-  if (p == 32 && dv == 16) return launch_decode_t<Tin, 32, 16>(q, k, v, o, S, z, BH, st);
+                                    int BH, int p, int groups, int dv, cudaStream_t st) {
+  if (groups == 1) {
+    if (p == 16 && dv == 64) return launch_decode_t<Tin, 16, 64, 1>(q, k, v, o, S, z, BH, st);
+    if (p == 16 && dv == 16) return launch_decode_t<Tin, 16, 16, 1>(q, k, v, o, S, z, BH, st);
+    if (p == 32 && dv == 64) return launch_decode_t<Tin, 32, 64, 1>(q, k, v, o, S, z, BH, st);
+    if (p == 32 && dv == 16) return launch_decode_t<Tin, 32, 16, 1>(q, k, v, o, S, z, BH, st);
+  } else if (dv == 64) {
+    if (p == 16 && groups == 2) return launch_decode_t<Tin, 16, 64, 2>(q, k, v, o, S, z, BH, st);
+    if (p == 16 && groups == 4) return launch_decode_t<Tin, 16, 64, 4>(q, k, v, o, S, z, BH, st);
+    if (p == 32 && groups == 2) return launch_decode_t<Tin, 32, 64, 2>(q, k, v, o, S, z, BH, st);
+  }
   return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_decode(const void* q, const void* k, const void* v, void* o, float* S, float* z, int BH,
-                          int p, int dv, kata_dtype_t dt, cudaStream_t st) {
-  if (dt == KATA_BF16) return launch_decode_dt<__nv_bfloat16>(q, k, v, o, S, z, BH, p, dv, st);
-  return launch_decode_dt<float>(q, k, v, o, S, z, BH, p, dv, st);
+                          int p, int groups, int dv, kata_dtype_t dt, cudaStream_t st) {
+  if (dt == KATA_BF16) return launch_decode_dt<__nv_bfloat16>(q, k, v, o, S, z, BH, p, groups, dv, st);
+  return launch_decode_dt<float>(q, k, v, o, S, z, BH, p, groups, dv, st);
 }
 
 }  // namespace kata

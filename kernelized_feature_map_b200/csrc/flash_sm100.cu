@@ -55,19 +55,24 @@ using namespace sm100;
 constexpr int kBM = 128;       // query rows per tile
 constexpr int kBN = 128;       // keys per tile
 constexpr int kNQ = 2;         // query tiles per CTA
-constexpr int kStages = 4;     // K/V ring depth
 constexpr int kThreads = 576;  // 18 warps
 constexpr uint32_t kTmemCols = 512;
 
-template <int p, int DV>
+// p: width of one PSD factor; G: factors per head (KATA-Mg), so q and k rows
+// hold d = G * p values and the score of a (query, key) pair is the sum over
+// the groups of the squared group dot products.
+template <int p, int DV, int G>
 struct FlashCfg {
-  static constexpr int kQKBytes = kBM * p * 2;          // one Q or K tile
+  static constexpr int kD = G * p;                      // q/k row width
+  static constexpr int kQKBytes = kBM * kD * 2;         // one Q or K tile
   static constexpr int kVBytes = kBN * DV * 2;          // one V tile
   // block of ones read as the second N-atom of the [V | 1] operand
   static constexpr int kOnesBytes = kBN * DV * 2;
-  // K-major Q/K rows are p*2 bytes: 32 B (p=16, 32B swizzle) or 64 B (p=32)
-  static constexpr Swizzle kQKSw = (p == 16) ? kSw32 : kSw64;
-  static constexpr uint32_t kQKSbo = 8 * p * 2;         // 8-row group stride
+  // K/V ring depth (3 when 128-byte q/k rows would overflow shared memory)
+  static constexpr int kStages = kD >= 64 ? 3 : 4;
+  // K-major Q/K rows are d*2 bytes: 32, 64 or 128 B, swizzled over that span
+  static constexpr Swizzle kQKSw = kD == 16 ? kSw32 : kD == 32 ? kSw64 : kSw128;
+  static constexpr uint32_t kQKSbo = 8 * kD * 2;        // 8-row group stride
   // MN-major V rows are DV*2 bytes: 128 B (DV=64, 128B swizzle) or 32 B
   static constexpr Swizzle kVSw = (DV == 64) ? kSw128 : kSw32;
   static constexpr uint32_t kVSbo = 8 * DV * 2;         // 8-key group stride
@@ -85,17 +90,18 @@ struct FlashCfg {
   static constexpr int kOutSlab = 32 * DV;
   static constexpr int offOut = offOnes + kOnesBytes;  // 1024-aligned
   static constexpr int offBar = offOut + 16 * kOutSlab;
-  static constexpr int kNumBars = 4 + 2 * kStages + 4 * kNQ + 1;
+  static constexpr int kNumBars = 4 + 2 * kStages + 5 * kNQ + 1;
   static constexpr int offMisc = offBar + kNumBars * 8;
   static constexpr int kSmemBytes = offMisc + 16 + 1024;  // + alignment slack
 };
 
-template <int p, int DV>
+template <int p, int DV, int G>
 __global__ void __launch_bounds__(kThreads, 1)
     flash_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o, int T, int BH,
-                     WaitCtl wc) {
-  using Cfg = FlashCfg<p, DV>;
+                     int H, int bthd, WaitCtl wc) {
+  using Cfg = FlashCfg<p, DV, G>;
+  constexpr int kStages = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::offBar);
@@ -107,7 +113,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* p_full = s_full + kNQ;         // [kNQ] weights of tile i written
   uint64_t* o_full = p_full + kNQ;         // [kNQ] [O|D] of tile i complete
   uint64_t* o_free = o_full + kNQ;         // [kNQ] [O|D] of tile i read by the epilogue
-  uint64_t* mma_done = o_free + kNQ;
+  uint64_t* s_read = o_free + kNQ;         // [kNQ] scores of one group of tile i read (G > 1)
+  uint64_t* mma_done = s_read + kNQ;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Cfg::offMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::offMisc + 4);
 
@@ -146,6 +153,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(p_full + i, 2 * kBM);
       mbar_init(o_full + i, 1);
       mbar_init(o_free + i, 2 * kBM);
+      mbar_init(s_read + i, 2 * kBM);
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -162,6 +170,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   const WaitEnv env{wc.status, abort_flag, wc.limit};
+  // rows [row, row + box) of head bh: the tensor maps are 4-D, {inner, T, H, B}
+  // for the [B,H,T,inner] layout and {inner, H, T, B} for [B,T,H,inner]
+  auto load_rows = [&](void* dst, const CUtensorMap* map, uint64_t* bar, int row, int bh) {
+    const int b = bh / H, hd = bh - b * H;
+    if (bthd)
+      tma_load_4d(dst, map, bar, 0, hd, row, b);
+    else
+      tma_load_4d(dst, map, bar, 0, row, hd, b);
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------------- producer
@@ -177,8 +194,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(q_empty + qb, ((nq >> 1) & 1) ^ 1, env)) break;
         mbar_arrive_expect_tx(q_full + qb, kNQ * Cfg::kQKBytes);
         for (int i = 0; i < kNQ; ++i)
-          tma_load_3d(smem + Cfg::offQ + (qb * kNQ + i) * Cfg::kQKBytes, &tm_q, q_full + qb, 0, (ct * kNQ + i) * kBM,
-                      bh);
+          load_rows(smem + Cfg::offQ + (qb * kNQ + i) * Cfg::kQKBytes, &tm_q, q_full + qb, (ct * kNQ + i) * kBM, bh);
         const int nkv_max = max(item_nkv(it, 0), item_nkv(it, 1));
         for (int j = 0; j < nkv_max; ++j, ++g) {
           const int st = (int)(g % kStages);
@@ -188,8 +204,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           KATA_TRACE(flash, (int)g, 9);
           mbar_arrive_expect_tx(kv_full + st, Cfg::kQKBytes + Cfg::kVBytes);
-          tma_load_3d(smem + Cfg::offK + st * Cfg::kQKBytes, &tm_k, kv_full + st, 0, j * kBN, bh);
-          tma_load_3d(smem + Cfg::offV + st * Cfg::kVBytes, &tm_v, kv_full + st, 0, j * kBN, bh);
+          load_rows(smem + Cfg::offK + st * Cfg::kQKBytes, &tm_k, kv_full + st, j * kBN, bh);
+          load_rows(smem + Cfg::offV + st * Cfg::kVBytes, &tm_v, kv_full + st, j * kBN, bh);
         }
       }
       // drain: every copy this CTA started must land before it exits
@@ -208,8 +224,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       // descriptors built once; K steps, Q buffers and stages are constant offsets
       const uint64_t dq0 = smem_desc(sQ, 16, Cfg::kQKSbo, Cfg::kQKSw);
       const uint64_t dk0 = smem_desc(sK, 16, Cfg::kQKSbo, Cfg::kQKSw);
-      auto issue_qk = [&](int i, int qb, int st) {
-        const uint64_t a = desc_add(dq0, (qb * kNQ + i) * Cfg::kQKBytes), b = desc_add(dk0, st * Cfg::kQKBytes);
+      // scores of group grp: columns grp*p .. of the Q and K rows
+      auto issue_qk = [&](int i, int qb, int st, int grp) {
+        const uint64_t a = desc_add(dq0, (qb * kNQ + i) * Cfg::kQKBytes + grp * p * 2),
+                       b = desc_add(dk0, st * Cfg::kQKBytes + grp * p * 2);
 #pragma unroll
         for (int ks = 0; ks < p / 16; ++ks) mma_ss_w(tmem + Cfg::colS(i), desc_add(a, ks * 32), desc_add(b, ks * 32), id_qk, ks > 0);
         mma_commit_w(s_full + i);
@@ -218,7 +236,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       long g = 0;                   // ring position of the item's first key tile
       int p_cnt[kNQ] = {0, 0};      // p_full phases consumed per tile
       int o_cnt[kNQ] = {0, 0};      // o_full phases committed per tile
+      int r_cnt[kNQ] = {0, 0};      // s_read phases consumed per tile
       bool ok = true;
+      // groups 1..G-1 of the scores of key tile at ring stage st, for the
+      // tiles i with has(i): each overwrites the previous group's scores, so
+      // it waits until the weight warps of tile i have read them
+      auto issue_groups = [&](int qb, int st, bool has0, bool has1) -> bool {
+        for (int grp = 1; grp < G; ++grp)
+          for (int i = 0; i < kNQ; ++i) {
+            if (!(i == 0 ? has0 : has1)) continue;
+            if (!mbar_wait_w(s_read + i, r_cnt[i] & 1, env)) return false;
+            ++r_cnt[i];
+            tc_fence_after();
+            issue_qk(i, qb, st, grp);
+          }
+        return true;
+      };
       for (int it = my_item(nq); ok && it >= 0; it = my_item(++nq)) {
         const int qb = nq & 1;
         int nkv[kNQ];
@@ -230,7 +263,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         for (int i = 0; i < kNQ; ++i)
-          if (nkv[i] > 0) issue_qk(i, qb, (int)(g % kStages));
+          if (nkv[i] > 0) issue_qk(i, qb, (int)(g % kStages), 0);
+        if (!issue_groups(qb, (int)(g % kStages), nkv[0] > 0, nkv[1] > 0)) {
+          ok = false;
+          break;
+        }
         long kv_ready = g;  // highest ring position whose K/V landed
         for (int j = 0; ok && j < nkv_max; ++j) {
           const long gj = g + j;
@@ -272,10 +309,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 kv_ready = gn;
               }
-              issue_qk(i, qb, (int)(gn % kStages));
+              issue_qk(i, qb, (int)(gn % kStages), 0);
             }
           }
           if (!ok) break;
+          if (!issue_groups(qb, (int)((gj + 1) % kStages), j + 1 < nkv[0], j + 1 < nkv[1])) {
+            ok = false;
+            break;
+          }
           KATA_TRACE(flash, (int)gj, 4);
           mma_commit_w(kv_empty + st);
         }
@@ -309,7 +350,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     int pend_row0 = 0, pend_bh = 0;
     auto flush_out = [&]() {
       if (pend && lane == 0) {
-        tma_store_3d(&tm_o, slab, kHalf * h, pend_row0, pend_bh);
+        const int b = pend_bh / H, hd = pend_bh - b * H;
+        if (bthd)
+          tma_store_4d(&tm_o, slab, kHalf * h, hd, pend_row0, b);
+        else
+          tma_store_4d(&tm_o, slab, kHalf * h, pend_row0, hd, b);
         bulk_commit_group();
       }
       pend = false;
@@ -338,34 +383,93 @@ __global__ void __launch_bounds__(kThreads, 1)
         // on the diagonal tile, 32-column block bb of row m is kept for
         // bb < quarter, masked for bb == quarter and zero for bb > quarter
         const int bb0 = 2 * h;
+        if constexpr (G == 1) {
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const int bb = bb0 + hh;
-          uint32_t w[16];
-          if (diag && bb > quarter) {
+          for (int hh = 0; hh < 2; ++hh) {
+            const int bb = bb0 + hh;
+            uint32_t w[16];
+            if (diag && bb > quarter) {
 #pragma unroll
-            for (int x = 0; x < 16; ++x) w[x] = 0u;
-          } else {
-            uint32_t r[32];
-            tmem_ld32(sa + 32 * hh, r);
-            tmem_wait_ld();
-            // squares on fp32 pairs (each rounded as a scalar multiply)
-            if (diag && bb == quarter) {
+              for (int x = 0; x < 16; ++x) w[x] = 0u;
+            } else {
+              uint32_t r[32];
+              tmem_ld32(sa + 32 * hh, r);
+              tmem_wait_ld();
+              // squares on fp32 pairs (each rounded as a scalar multiply)
+              if (diag && bb == quarter) {
 #pragma unroll
-              for (int x = 0; x < 16; ++x) {
-                const uint32_t a = 2 * x > lane ? 0u : r[2 * x], b = 2 * x + 1 > lane ? 0u : r[2 * x + 1];
-                const uint64_t sq = f32x2_mul(f32x2(a, b), f32x2(a, b));
-                w[x] = pack_bf16x2(f32x2_lo(sq), f32x2_hi(sq));
+                for (int x = 0; x < 16; ++x) {
+                  const uint32_t a = 2 * x > lane ? 0u : r[2 * x], b = 2 * x + 1 > lane ? 0u : r[2 * x + 1];
+                  const uint64_t sq = f32x2_mul(f32x2(a, b), f32x2(a, b));
+                  w[x] = pack_bf16x2(f32x2_lo(sq), f32x2_hi(sq));
+                }
+              } else {
+#pragma unroll
+                for (int x = 0; x < 16; ++x) {
+                  const uint64_t sq = f32x2_mul(f32x2(r[2 * x], r[2 * x + 1]), f32x2(r[2 * x], r[2 * x + 1]));
+                  w[x] = pack_bf16x2(f32x2_lo(sq), f32x2_hi(sq));
+                }
+              }
+            }
+            tmem_st16(sa + 16 * hh, w);
+          }
+        } else {
+          // KATA-Mg: W = sum over the groups of the squared group scores.
+          // The groups' scores arrive one after another in the same columns;
+          // the sum is kept in fp32 pairs, acc[16 hh + y] holding keys
+          // 32 (bb0 + hh) + 2y and + 2y + 1 (blocks above the diagonal are
+          // never read)
+          uint64_t acc[32];
+          for (int grp = 0; grp < G; ++grp) {
+            if (grp > 0) {
+              if (!mbar_wait(s_full + i, s_cnt & 1, env)) {
+                ok = false;
+                break;
+              }
+              ++s_cnt;
+              tc_fence_after();
+            }
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              if (diag && bb0 + hh > quarter) continue;
+#pragma unroll
+              for (int hf = 0; hf < 4; ++hf) {
+                uint32_t r[8];
+                tmem_ld8(sa + 32 * hh + 8 * hf, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                  const uint64_t sc = f32x2(r[2 * x], r[2 * x + 1]);
+                  uint64_t& ac = acc[16 * hh + 4 * hf + x];
+                  ac = grp == 0 ? f32x2_mul(sc, sc) : f32x2_fma(sc, sc, ac);
+                }
+              }
+            }
+            if (grp + 1 < G) {
+              tc_fence_before();
+              mbar_arrive(s_read + i);
+            }
+          }
+          if (!ok) break;
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const int bb = bb0 + hh;
+            uint32_t w[16];
+            if (diag && bb > quarter) {
+#pragma unroll
+              for (int y = 0; y < 16; ++y) w[y] = 0u;
+            } else if (diag && bb == quarter) {
+#pragma unroll
+              for (int y = 0; y < 16; ++y) {
+                const uint64_t ac = acc[16 * hh + y];
+                w[y] = pack_bf16x2(2 * y > lane ? 0.f : f32x2_lo(ac), 2 * y + 1 > lane ? 0.f : f32x2_hi(ac));
               }
             } else {
 #pragma unroll
-              for (int x = 0; x < 16; ++x) {
-                const uint64_t sq = f32x2_mul(f32x2(r[2 * x], r[2 * x + 1]), f32x2(r[2 * x], r[2 * x + 1]));
-                w[x] = pack_bf16x2(f32x2_lo(sq), f32x2_hi(sq));
-              }
+              for (int y = 0; y < 16; ++y) w[y] = pack_bf16x2(f32x2_lo(acc[16 * hh + y]), f32x2_hi(acc[16 * hh + y]));
             }
+            tmem_st16(sa + 16 * hh, w);
           }
-          tmem_st16(sa + 16 * hh, w);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -469,15 +573,60 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, int inner, int T, int BH
   return make_tmap_bf16_box(map, base, inner, T, BH, inner, rows);
 }
 
-template <int p, int DV>
-static cudaError_t launch_flash_t(const void* q, const void* k, const void* v, void* o, int BH, int T,
+// 4-D bf16 tensor map over a [B,H,T,inner] tensor (dims {inner, T, H, B}) or,
+// with bthd, a [B,T,H,inner] tensor (dims {inner, H, T, B}), so that the
+// strides grow with the dimension either way; the box covers box_inner
+// values of `rows` consecutive tokens of one head, swizzled over the box row.
+bool make_tmap_bf16_4d(CUtensorMap* map, const void* base, int inner, int T, int H, int B, bool bthd, int box_inner,
+                       int rows) {
+  EncodeTiledFn enc = get_encode_tiled();
+  if (!enc) return false;
+  const cuuint64_t row_bytes = (cuuint64_t)inner * 2;
+  const int box_bytes = box_inner * 2;
+  CUtensorMapSwizzle sw = box_bytes == 32    ? CU_TENSOR_MAP_SWIZZLE_32B
+                          : box_bytes == 64  ? CU_TENSOR_MAP_SWIZZLE_64B
+                          : box_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                             : CU_TENSOR_MAP_SWIZZLE_NONE;
+  cuuint64_t dims[4], strides[3];
+  cuuint32_t box[4];
+  dims[0] = (cuuint64_t)inner;
+  dims[3] = (cuuint64_t)B;
+  box[0] = (cuuint32_t)box_inner;
+  box[3] = 1;
+  if (bthd) {
+    dims[1] = (cuuint64_t)H;
+    dims[2] = (cuuint64_t)T;
+    strides[0] = row_bytes;       // next head
+    strides[1] = row_bytes * H;   // next token
+    box[1] = 1;
+    box[2] = (cuuint32_t)rows;
+  } else {
+    dims[1] = (cuuint64_t)T;
+    dims[2] = (cuuint64_t)H;
+    strides[0] = row_bytes;       // next token
+    strides[1] = row_bytes * T;   // next head
+    box[1] = (cuuint32_t)rows;
+    box[2] = 1;
+  }
+  strides[2] = row_bytes * (cuuint64_t)T * (cuuint64_t)H;  // next batch entry
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int p, int DV, int G>
+static cudaError_t launch_flash_t(const void* q, const void* k, const void* v, void* o, int B, int H, int T, bool bthd,
                                   const WaitCtl& wc, cudaStream_t st) {
-  using Cfg = FlashCfg<p, DV>;
+  using Cfg = FlashCfg<p, DV, G>;
+  const int BH = B * H;
   CUtensorMap tq, tk, tv, to;
-  if (!make_tmap_bf16(&tq, q, p, T, BH, kBM) || !make_tmap_bf16(&tk, k, p, T, BH, kBN) ||
-      !make_tmap_bf16(&tv, v, DV, T, BH, kBN) || !make_tmap_bf16_box(&to, o, DV, T, BH, DV / 2, 32))
+  if (!make_tmap_bf16_4d(&tq, q, Cfg::kD, T, H, B, bthd, Cfg::kD, kBM) ||
+      !make_tmap_bf16_4d(&tk, k, Cfg::kD, T, H, B, bthd, Cfg::kD, kBN) ||
+      !make_tmap_bf16_4d(&tv, v, DV, T, H, B, bthd, DV, kBN) ||
+      !make_tmap_bf16_4d(&to, o, DV, T, H, B, bthd, DV / 2, 32))
     return cudaErrorInvalidValue;
-  auto kern = flash_fwd_kernel<p, DV>;
+  auto kern = flash_fwd_kernel<p, DV, G>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
   if (e != cudaSuccess) return e;
   // persistent: one CTA per SM (or fewer when there are fewer work items)
@@ -490,16 +639,27 @@ static cudaError_t launch_flash_t(const void* q, const void* k, const void* v, v
   }
   const long items = (long)((T + kBM * kNQ - 1) / (kBM * kNQ)) * BH;
   const int grid = (int)(items < num_sms ? items : num_sms);
-  kern<<<grid, kThreads, Cfg::kSmemBytes, st>>>(tq, tk, tv, to, T, BH, wc);
+  kern<<<grid, kThreads, Cfg::kSmemBytes, st>>>(tq, tk, tv, to, T, BH, H, bthd ? 1 : 0, wc);
   return cudaGetLastError();
 }
 
-cudaError_t launch_flash_sm100(const void* q, const void* k, const void* v, void* o, int BH, int T, int p, int dv,
-                               const WaitCtl& wc, cudaStream_t st) {
-  if (p == 16 && dv == 64) return launch_flash_t<16, 64>(q, k, v, o, BH, T, wc, st);
-  if (p == 16 && dv == 16) return launch_flash_t<16, 16>(q, k, v, o, BH, T, wc, st);
-  if (p == 32 && dv == 64) return launch_flash_t<32, 64>(q, k, v, o, BH, T, wc, st);
-  if (p == 32 && dv == 16) return launch_flash_t<32, 16>(q, k, v, o, BH, T, wc, st);
+bool flash_sm100_supports(int p, int groups, int dv) {
+  if (groups == 1) return (p == 16 || p == 32) && (dv == 16 || dv == 64);
+  return dv == 64 && ((p == 16 && (groups == 2 || groups == 4)) || (p == 32 && groups == 2));
+}
+
+cudaError_t launch_flash_sm100(const void* q, const void* k, const void* v, void* o, int B, int H, int T, int p,
+                               int groups, int dv, bool bthd, const WaitCtl& wc, cudaStream_t st) {
+  if (groups == 1) {
+    if (p == 16 && dv == 64) return launch_flash_t<16, 64, 1>(q, k, v, o, B, H, T, bthd, wc, st);
+    if (p == 16 && dv == 16) return launch_flash_t<16, 16, 1>(q, k, v, o, B, H, T, bthd, wc, st);
+    if (p == 32 && dv == 64) return launch_flash_t<32, 64, 1>(q, k, v, o, B, H, T, bthd, wc, st);
+    if (p == 32 && dv == 16) return launch_flash_t<32, 16, 1>(q, k, v, o, B, H, T, bthd, wc, st);
+  } else if (dv == 64) {
+    if (p == 16 && groups == 2) return launch_flash_t<16, 64, 2>(q, k, v, o, B, H, T, bthd, wc, st);
+    if (p == 16 && groups == 4) return launch_flash_t<16, 64, 4>(q, k, v, o, B, H, T, bthd, wc, st);
+    if (p == 32 && groups == 2) return launch_flash_t<32, 64, 2>(q, k, v, o, B, H, T, bthd, wc, st);
+  }
   return cudaErrorInvalidValue;
 }
 

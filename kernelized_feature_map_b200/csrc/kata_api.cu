@@ -149,7 +149,7 @@ KATA_API kata_status_t kata_fwd_quadratic(const void* q, const void* k, const vo
   if (!q || !k || !v || !o) return KATA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return KATA_ERR_MISALIGNED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (dtype == KATA_BF16) return from_cuda(launch_flash_sm100(q, k, v, o, B * H, T, p, dv, wait_ctl(), st));
+  if (dtype == KATA_BF16) return from_cuda(launch_flash_sm100(q, k, v, o, B, H, T, p, 1, dv, false, wait_ctl(), st));
   return from_cuda(launch_quadratic_simt(q, k, v, o, B * H, T, p, dv, dtype, st));
 }
 
@@ -244,5 +244,44 @@ KATA_API kata_status_t kata_decode_step(const void* q, const void* k, const void
   if (!q || !k || !v || !o || !S || !z) return KATA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(S) || !aligned16(z))
     return KATA_ERR_MISALIGNED;
-  return from_cuda(launch_decode(q, k, v, o, S, z, B * H, p, dv, dtype, static_cast<cudaStream_t>(stream)));
+  return from_cuda(launch_decode(q, k, v, o, S, z, B * H, p, 1, dv, dtype, static_cast<cudaStream_t>(stream)));
+}
+
+// Shape checks shared by the KATA-Mg entry points: p = d / groups.
+static kata_status_t check_mg(int B, int H, int T, int d, int groups, int dv, kata_dtype_t dt, int* p_out) {
+  if (groups < 1 || d < 1 || d % groups != 0) return KATA_ERR_INVALID_ARG;
+  const int p = d / groups;
+  kata_status_t s = check_common(B, H, T, p, dv, dt);
+  if (s != KATA_OK) return s;
+  if ((long long)T * d >= (1ll << 31)) return KATA_ERR_UNSUPPORTED;
+  if (!flash_sm100_supports(p, groups, dv)) return KATA_ERR_UNSUPPORTED;
+  *p_out = p;
+  return KATA_OK;
+}
+
+KATA_API kata_status_t kata_fwd_mg_quadratic(const void* q, const void* k, const void* v, void* o, int B, int H,
+                                             int T, int d, int groups, int dv, kata_layout_t layout,
+                                             kata_dtype_t dtype, void* stream) {
+  int p = 0;
+  kata_status_t s = check_mg(B, H, T, d, groups, dv, dtype, &p);
+  if (s != KATA_OK) return s;
+  if (layout != KATA_LAYOUT_BHTD && layout != KATA_LAYOUT_BTHD) return KATA_ERR_INVALID_ARG;
+  if (dtype != KATA_BF16) return KATA_ERR_UNSUPPORTED;
+  if (T == 0) return KATA_OK;
+  if (!q || !k || !v || !o) return KATA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return KATA_ERR_MISALIGNED;
+  return from_cuda(launch_flash_sm100(q, k, v, o, B, H, T, p, groups, dv, layout == KATA_LAYOUT_BTHD, wait_ctl(),
+                                      static_cast<cudaStream_t>(stream)));
+}
+
+KATA_API kata_status_t kata_decode_step_mg(const void* q, const void* k, const void* v, void* o, float* S, float* z,
+                                           int B, int H, int d, int groups, int dv, kata_dtype_t dtype,
+                                           void* stream) {
+  int p = 0;
+  kata_status_t s = check_mg(B, H, 1, d, groups, dv, dtype, &p);
+  if (s != KATA_OK) return s;
+  if (!q || !k || !v || !o || !S || !z) return KATA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(S) || !aligned16(z))
+    return KATA_ERR_MISALIGNED;
+  return from_cuda(launch_decode(q, k, v, o, S, z, B * H, p, groups, dv, dtype, static_cast<cudaStream_t>(stream)));
 }

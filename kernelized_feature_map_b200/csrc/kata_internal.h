@@ -44,9 +44,9 @@ inline bool chunked_on_tensor_cores(int p, int dv, kata_dtype_t dt) {
 
 ChunkPlan make_chunk_plan(int B, int H, int T, int p, int dv, int C, kata_dtype_t dt);
 
-// decode.cu
+// decode.cu -- `groups` PSD factors of width p per head (1: the single-factor step)
 cudaError_t launch_decode(const void* q, const void* k, const void* v, void* o, float* S, float* z,
-                          int BH, int p, int dv, kata_dtype_t dt, cudaStream_t st);
+                          int BH, int p, int groups, int dv, kata_dtype_t dt, cudaStream_t st);
 
 // scan.cu -- exclusive prefix over the G records of every (b,h), in place,
 // plus S0 and the final state.  Records g >= G_in hold no data (treated as
@@ -63,9 +63,12 @@ cudaError_t launch_chunk_aggregate_simt(const void* k, const void* v, float* ws,
 cudaError_t launch_chunk_readout_simt(const void* q, const void* k, const void* v, void* o, float* ws,
                                       const ChunkPlan& plan, kata_dtype_t dt, cudaStream_t st);
 
-// flash_sm100.cu -- tcgen05 flash-style forward (bf16 inputs).
-cudaError_t launch_flash_sm100(const void* q, const void* k, const void* v, void* o, int BH, int T, int p, int dv,
-                               const WaitCtl& wc, cudaStream_t st);
+// flash_sm100.cu -- tcgen05 flash-style forward (bf16 inputs) with `groups`
+// PSD factors of width p per head; bthd selects the [B,T,H,*] layout of
+// q, k, v and o instead of [B,H,T,*].
+bool flash_sm100_supports(int p, int groups, int dv);
+cudaError_t launch_flash_sm100(const void* q, const void* k, const void* v, void* o, int B, int H, int T, int p,
+                               int groups, int dv, bool bthd, const WaitCtl& wc, cudaStream_t st);
 
 // chunk_sm100.cu -- tcgen05 chunked-state forward (bf16 inputs, p = 16).
 // The state kernel sums super-chunks 0..G-2 (the last one's sum is never

@@ -44,7 +44,7 @@ def test_only_abi_symbols_are_exported():
 
 
 def test_status_strings_and_version(L):
-    assert _abi.kata_abi_version() == 10000
+    assert _abi.kata_abi_version() == 10100
     for code, name in [(0, "KATA_OK"), (2, "KATA_ERR_UNSUPPORTED"), (6, "KATA_ERR_TIMEOUT")]:
         assert _abi.status_string(code) == name
     assert _abi.status_string(99) == "KATA_ERR_UNKNOWN"
@@ -118,3 +118,27 @@ def test_binding_requires_cuda_tensors():
     q = torch.zeros(1, 1, 4, 16)
     with pytest.raises(TypeError):
         _abi.kata_fwd_quadratic(q, q, torch.zeros(1, 1, 4, 64))
+
+
+def test_mg_argument_errors_before_launch(L):
+    a, b, c, d = _fake(0x10000), _fake(0x20000), _fake(0x30000), _fake(0x40000)
+    S, z = _fake(0x70000), _fake(0x80000)
+    st = VP(0)
+    m = L.kata_fwd_mg_quadratic  # q k v o B H T d groups dv layout dtype stream
+    BHTD, BTHD = _abi.KATA_LAYOUT_BHTD, _abi.KATA_LAYOUT_BTHD
+    assert m(a, b, c, d, 1, 1, 16, 64, 3, 64, BHTD, 1, st) == _abi.KATA_ERR_INVALID_ARG   # d % groups
+    assert m(a, b, c, d, 1, 1, 16, 64, 0, 64, BHTD, 1, st) == _abi.KATA_ERR_INVALID_ARG   # groups
+    assert m(a, b, c, d, 1, 1, 16, 64, 8, 64, BHTD, 1, st) == _abi.KATA_ERR_UNSUPPORTED   # p = 8
+    assert m(a, b, c, d, 1, 1, 16, 64, 4, 16, BHTD, 1, st) == _abi.KATA_ERR_UNSUPPORTED   # dv 16 with groups
+    assert m(a, b, c, d, 1, 1, 16, 128, 4, 64, BHTD, 1, st) == _abi.KATA_ERR_UNSUPPORTED  # p 32 x 4 groups
+    assert m(a, b, c, d, 1, 1, 16, 64, 4, 64, 2, 1, st) == _abi.KATA_ERR_INVALID_ARG      # layout
+    assert m(a, b, c, d, 1, 1, 16, 64, 4, 64, BHTD, 0, st) == _abi.KATA_ERR_UNSUPPORTED   # fp32
+    assert m(None, b, c, d, 1, 1, 16, 64, 4, 64, BTHD, 1, st) == _abi.KATA_ERR_INVALID_ARG
+    assert m(_fake(0x10008), b, c, d, 1, 1, 16, 64, 4, 64, BTHD, 1, st) == _abi.KATA_ERR_MISALIGNED
+    assert m(a, b, c, d, 1, 1, 0, 64, 4, 64, BTHD, 1, st) == _abi.KATA_OK                 # T = 0: no-op
+    md = L.kata_decode_step_mg  # q k v o S z B H d groups dv dtype stream
+    assert md(a, b, c, d, S, None, 1, 1, 64, 4, 64, 1, st) == _abi.KATA_ERR_INVALID_ARG
+    assert md(a, b, c, d, S, z, 1, 1, 64, 4, 16, 1, st) == _abi.KATA_ERR_UNSUPPORTED
+    assert md(a, b, c, d, S, z, 1, 1, 48, 4, 64, 1, st) == _abi.KATA_ERR_UNSUPPORTED      # p = 12
+    assert md(a, b, c, d, S, z, 1, 1, 64, 5, 64, 1, st) == _abi.KATA_ERR_INVALID_ARG
+    assert md(a, b, c, d, _fake(0x70004), z, 1, 1, 64, 2, 64, 1, st) == _abi.KATA_ERR_MISALIGNED

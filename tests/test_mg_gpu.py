@@ -1,0 +1,151 @@
+"""GPU parity of the KATA-Mg entry points (g PSD factors per head) against
+the fp64 Mg oracle on the same seeded inputs: the flash-style forward in both
+layouts and the decode step.  Gate as for the single-factor paths: per-row
+relative error 2e-2 for bf16 inputs, 1e-4 for fp32 (tests/helpers.py)."""
+import numpy as np
+import pytest
+
+import oracle
+import workloads
+from helpers import TOL, row_rel_err, rows_rel_err, to_dev, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def kata():
+    import torch
+    import kernelized_feature_map_b200 as K
+    from kernelized_feature_map_b200 import build
+    build.build()
+    assert torch.cuda.is_available()
+    return K
+
+
+def _bthd(x):
+    return np.ascontiguousarray(np.asarray(x).transpose(0, 2, 1, 3))
+
+
+def _run_mg(K, q, k, v, groups, layout):
+    import torch
+    if layout == "bthd":
+        o = K.kata_fwd_mg_quadratic(to_dev(_bthd(q), "bf16"), to_dev(_bthd(k), "bf16"), to_dev(_bthd(v), "bf16"),
+                                    groups, layout="bthd")
+        out = _bthd(to_np(o))
+    else:
+        o = K.kata_fwd_mg_quadratic(to_dev(q, "bf16"), to_dev(k, "bf16"), to_dev(v, "bf16"), groups)
+        out = to_np(o)
+    torch.cuda.synchronize()
+    assert K.kata_get_status() == 0
+    return out
+
+
+MG_SHAPES = [
+    # B, H, T, d, groups, dv -- T spans several 128-row tiles and ends ragged
+    (2, 2, 1000, 64, 4, 64),
+    (1, 3, 777, 64, 2, 64),
+    (2, 2, 600, 32, 2, 64),
+    (1, 2, 385, 16, 1, 16),
+    (1, 1, 129, 32, 1, 64),
+]
+
+
+@pytest.mark.parametrize("layout", ["bhtd", "bthd"])
+@pytest.mark.parametrize("shape", MG_SHAPES)
+def test_mg_flash_matches_oracle(kata, shape, layout):
+    B, H, T, d, g, dv = shape
+    q, k, v = workloads.normal_qkv(B, H, T, d, dv, seed=200 + T + g, dtype="bf16")
+    ref = oracle.direct_mg(q, k, v, g)
+    err = row_rel_err(_run_mg(kata, q, k, v, g, layout), ref, v)
+    assert err <= TOL["bf16"], (shape, layout, err)
+
+
+def test_mg_layouts_agree_bitwise_and_one_group_is_the_flash_kernel(kata):
+    import torch
+    B, H, T, d, g, dv = 2, 3, 700, 64, 4, 64
+    q, k, v = workloads.normal_qkv(B, H, T, d, dv, seed=310, dtype="bf16")
+    assert np.array_equal(_run_mg(kata, q, k, v, g, "bhtd"), _run_mg(kata, q, k, v, g, "bthd"))
+    q1, k1, v1 = workloads.normal_qkv(B, H, T, 16, dv, seed=311, dtype="bf16")
+    qd, kd, vd = to_dev(q1, "bf16"), to_dev(k1, "bf16"), to_dev(v1, "bf16")
+    a = kata.kata_fwd_quadratic(qd, kd, vd)
+    b = kata.kata_fwd_mg_quadratic(qd, kd, vd, 1)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
+def test_mg_edge_cases(kata):
+    # a single token, a tile plus one, and rows whose query is zero (zero
+    # denominator: the output row is 0 on both sides)
+    for (T, g) in [(1, 4), (129, 2)]:
+        q, k, v = workloads.normal_qkv(1, 2, T, 64, 64, seed=320 + T, dtype="bf16")
+        q[:, :, T // 2] = 0.0
+        ref = oracle.direct_mg(q, k, v, g)
+        for layout in ("bhtd", "bthd"):
+            got = _run_mg(kata, q, k, v, g, layout)
+            assert np.all(got[:, :, T // 2] == 0.0)
+            assert row_rel_err(got, ref, v) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("name", sorted(workloads.MG_CONFIGS))
+def test_mg_full_size_sampled_rows(kata, name):
+    """The benchmark's Mg workloads at full size, in the launch configuration
+    bench.py times, compared on sampled rows the oracle computes one by one."""
+    cfg = workloads.MG_CONFIGS[name]
+    B, H, T, d, g, dv = cfg["B"], cfg["H"], cfg["T"], cfg["d"], cfg["groups"], cfg["dv"]
+    q, k, v = workloads.normal_qkv(B, H, T, d, dv, seed=cfg["seed"], dtype=cfg["dtype"])
+    got = _run_mg(kata, q, k, v, g, cfg["layout"])
+    rng = np.random.default_rng(cfg["seed"])
+    bh = rng.integers(0, B * H, size=96)
+    t = np.concatenate([rng.integers(0, T, size=80), [0, 1, 127, 128, 129, T - 2, T - 1, T // 2] * 2])[:96]
+    ref = oracle.direct_mg_rows(q, k, v, g, bh, t)
+    vmax = np.abs(v.reshape(B * H, -1)).max(axis=1)[bh]
+    rows = got.reshape(B * H, T, dv)[bh, t]
+    assert rows_rel_err(rows, ref, vmax) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("d,g", [(64, 4), (64, 2), (32, 2)])
+def test_mg_decode_step(kata, dtype, d, g):
+    import torch
+    B, H, dv = 5, 3, 64
+    q, k, v, S, z = workloads.decode_inputs_mg(B, H, d, g, dv, seed=d + g, dtype=dtype)
+    o_ref, S_ref, z_ref = oracle.decode_step_mg(q, k, v, S, z, g)
+    Sd = torch.from_numpy(S).cuda()
+    zd = torch.from_numpy(z).cuda()
+    o = kata.kata_decode_step_mg(to_dev(q, dtype), to_dev(k, dtype), to_dev(v, dtype), Sd, zd, g)
+    torch.cuda.synchronize()
+    assert kata.kata_get_status() == 0
+    np.testing.assert_allclose(Sd.cpu().numpy(), S_ref, rtol=1e-6, atol=1e-5)
+    np.testing.assert_allclose(zd.cpu().numpy(), z_ref, rtol=1e-6, atol=1e-5)
+    err = np.abs(to_np(o) - o_ref).max() / np.abs(o_ref).max()
+    assert err <= TOL[dtype], err
+
+
+def test_mg_decode_continues_the_forward(kata):
+    """Decode steps from the oracle's Mg state after T tokens reproduce the
+    flash Mg forward's outputs for the next tokens."""
+    import torch
+    B, H, T, d, g, dv = 2, 2, 200, 64, 4, 64
+    q, k, v = workloads.normal_qkv(B, H, T + 3, d, dv, seed=330, dtype="bf16")
+    o_fwd = _run_mg(kata, q, k, v, g, "bhtd")
+    _, S, z = oracle.recurrent_mg(q[:, :, :T], k[:, :, :T], v[:, :, :T], g, return_state=True)
+    Sd = torch.from_numpy(S.astype(np.float32)).cuda()
+    zd = torch.from_numpy(z.astype(np.float32)).cuda()
+    outs = []
+    for t in range(T, T + 3):
+        outs.append(to_np(kata.kata_decode_step_mg(to_dev(q[:, :, t], "bf16"), to_dev(k[:, :, t], "bf16"),
+                                                   to_dev(v[:, :, t], "bf16"), Sd, zd, g)))
+    torch.cuda.synchronize()
+    assert row_rel_err(np.stack(outs, axis=2), o_fwd[:, :, T:], v) <= TOL["bf16"]
+
+
+def test_mg_pages_call_shape(kata):
+    """parallel_kata_attn: [B,T,H,D] in and out, num_groups factors per head."""
+    import torch
+    B, T, H, D = 2, 300, 4, 64
+    q, k, v = workloads.normal_qkv(B, H, T, D, D, seed=340, dtype="bf16")
+    o = kata.parallel_kata_attn(to_dev(_bthd(q), "bf16"), to_dev(_bthd(k), "bf16"), to_dev(_bthd(v), "bf16"),
+                                num_groups=2)
+    torch.cuda.synchronize()
+    assert tuple(o.shape) == (B, T, H, D)
+    assert row_rel_err(_bthd(to_np(o)), oracle.direct_mg(q, k, v, 2), v) <= TOL["bf16"]

@@ -33,6 +33,16 @@ CONFIGS = {
     "long_ctx131k": dict(B=1, H=16, T=131072, p=16, dv=64, C=64, dtype="bf16", kind="normal", seed=2),
     "recall_p32": dict(B=4, H=16, T=8192, p=32, dv=64, C=64, dtype="bf16", kind="recall", seed=3),
 }
+
+# KATA-Mg configurations: the 340M model's heads (hidden size 1024 over 16
+# heads, d = 64) split into `groups` PSD factors -- 2 as in the README's model
+# config (spd_num_groups=2, p = 32) and 4 (p = 16) -- at context 2048, in the
+# README attention call's [B, T, H, d] layout.  q, k are L2-normalised over
+# the whole head row.
+MG_CONFIGS = {
+    "mg2_ctx2k": dict(B=8, H=16, T=2048, d=64, groups=2, dv=64, dtype="bf16", layout="bthd", seed=5),
+    "mg4_ctx2k": dict(B=8, H=16, T=2048, d=64, groups=4, dv=64, dtype="bf16", layout="bthd", seed=6),
+}
 SWEEP_B = (1, 4, 16)
 SWEEP_T = (1024, 4096, 16384, 65536, 131072)
 DECODE = dict(B=64, H=16, p=16, dv=64, dtype="bf16", seed=4)
@@ -128,4 +138,26 @@ def decode_inputs(B, H, p, dv, seed=4, dtype="bf16"):
     G = rng.standard_normal((B, H, p, p)).astype(np.float64)
     Z = np.matmul(G, G.transpose(0, 1, 3, 2)) / p + 0.1 * np.eye(p)
     z = Z.reshape(B, H, p * p).astype(np.float32)
+    return q, k, v, S, z
+
+
+def decode_inputs_mg(B, H, d, groups, dv, seed=7, dtype="bf16"):
+    """One KATA-Mg decode step's q, k [B,H,d], v [B,H,dv] and a random
+    starting state S [B,H,groups*p*p,dv], z [B,H,groups*p*p] (p = d/groups):
+    one block per group, each built as in :func:`decode_inputs` (symmetric in
+    the two indices, positive-definite normaliser)."""
+    rng = np.random.default_rng(seed)
+    p = d // groups
+    q = _cast(_l2n(rng.standard_normal((B, H, d), dtype=np.float32)), dtype)
+    k = _cast(_l2n(rng.standard_normal((B, H, d), dtype=np.float32)), dtype)
+    v = _cast(rng.standard_normal((B, H, dv), dtype=np.float32), dtype)
+    Ss, zs = [], []
+    for _ in range(groups):
+        A = rng.standard_normal((B, H, p, p, dv), dtype=np.float32)
+        Ss.append((0.5 * (A + A.transpose(0, 1, 3, 2, 4))).reshape(B, H, p * p, dv))
+        Gm = rng.standard_normal((B, H, p, p)).astype(np.float64)
+        Z = np.matmul(Gm, Gm.transpose(0, 1, 3, 2)) / p + 0.1 * np.eye(p)
+        zs.append(Z.reshape(B, H, p * p))
+    S = np.concatenate(Ss, axis=2).astype(np.float32)
+    z = np.concatenate(zs, axis=2).astype(np.float32)
     return q, k, v, S, z
