@@ -58,21 +58,16 @@ constexpr int kNQ = 2;         // query tiles per CTA
 constexpr int kThreads = 576;  // 18 warps
 constexpr uint32_t kTmemCols = 512;
 
-// p: width of one PSD factor; G: factors per head (KATA-Mg), so q and k rows
-// hold d = G * p values and the score of a (query, key) pair is the sum over
-// the groups of the squared group dot products.
-template <int p, int DV, int G>
+template <int p, int DV>
 struct FlashCfg {
-  static constexpr int kD = G * p;                      // q/k row width
-  static constexpr int kQKBytes = kBM * kD * 2;         // one Q or K tile
+  static constexpr int kQKBytes = kBM * p * 2;          // one Q or K tile
   static constexpr int kVBytes = kBN * DV * 2;          // one V tile
   // block of ones read as the second N-atom of the [V | 1] operand
   static constexpr int kOnesBytes = kBN * DV * 2;
-  // K/V ring depth (3 when 128-byte q/k rows would overflow shared memory)
-  static constexpr int kStages = kD >= 64 ? 3 : 4;
-  // K-major Q/K rows are d*2 bytes: 32, 64 or 128 B, swizzled over that span
-  static constexpr Swizzle kQKSw = kD == 16 ? kSw32 : kD == 32 ? kSw64 : kSw128;
-  static constexpr uint32_t kQKSbo = 8 * kD * 2;        // 8-row group stride
+  static constexpr int kStages = 4;                     // K/V ring depth
+  // K-major Q/K rows are p*2 bytes: 32 B (p=16, 32B swizzle) or 64 B (p=32)
+  static constexpr Swizzle kQKSw = (p == 16) ? kSw32 : kSw64;
+  static constexpr uint32_t kQKSbo = 8 * p * 2;         // 8-row group stride
   // MN-major V rows are DV*2 bytes: 128 B (DV=64, 128B swizzle) or 32 B
   static constexpr Swizzle kVSw = (DV == 64) ? kSw128 : kSw32;
   static constexpr uint32_t kVSbo = 8 * DV * 2;         // 8-key group stride
@@ -90,17 +85,17 @@ struct FlashCfg {
   static constexpr int kOutSlab = 32 * DV;
   static constexpr int offOut = offOnes + kOnesBytes;  // 1024-aligned
   static constexpr int offBar = offOut + 16 * kOutSlab;
-  static constexpr int kNumBars = 4 + 2 * kStages + 5 * kNQ + 1;
+  static constexpr int kNumBars = 4 + 2 * kStages + 4 * kNQ + 1;
   static constexpr int offMisc = offBar + kNumBars * 8;
   static constexpr int kSmemBytes = offMisc + 16 + 1024;  // + alignment slack
 };
 
-template <int p, int DV, int G>
+template <int p, int DV>
 __global__ void __launch_bounds__(kThreads, 1)
     flash_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o, int T, int BH,
                      int H, int bthd, WaitCtl wc) {
-  using Cfg = FlashCfg<p, DV, G>;
+  using Cfg = FlashCfg<p, DV>;
   constexpr int kStages = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -113,8 +108,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* p_full = s_full + kNQ;         // [kNQ] weights of tile i written
   uint64_t* o_full = p_full + kNQ;         // [kNQ] [O|D] of tile i complete
   uint64_t* o_free = o_full + kNQ;         // [kNQ] [O|D] of tile i read by the epilogue
-  uint64_t* s_read = o_free + kNQ;         // [kNQ] scores of one group of tile i read (G > 1)
-  uint64_t* mma_done = s_read + kNQ;
+  uint64_t* mma_done = o_free + kNQ;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Cfg::offMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::offMisc + 4);
 
@@ -153,7 +147,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(p_full + i, 2 * kBM);
       mbar_init(o_full + i, 1);
       mbar_init(o_free + i, 2 * kBM);
-      mbar_init(s_read + i, 2 * kBM);
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -224,10 +217,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // descriptors built once; K steps, Q buffers and stages are constant offsets
       const uint64_t dq0 = smem_desc(sQ, 16, Cfg::kQKSbo, Cfg::kQKSw);
       const uint64_t dk0 = smem_desc(sK, 16, Cfg::kQKSbo, Cfg::kQKSw);
-      // scores of group grp: columns grp*p .. of the Q and K rows
-      auto issue_qk = [&](int i, int qb, int st, int grp) {
-        const uint64_t a = desc_add(dq0, (qb * kNQ + i) * Cfg::kQKBytes + grp * p * 2),
-                       b = desc_add(dk0, st * Cfg::kQKBytes + grp * p * 2);
+      auto issue_qk = [&](int i, int qb, int st) {
+        const uint64_t a = desc_add(dq0, (qb * kNQ + i) * Cfg::kQKBytes), b = desc_add(dk0, st * Cfg::kQKBytes);
 #pragma unroll
         for (int ks = 0; ks < p / 16; ++ks) mma_ss_w(tmem + Cfg::colS(i), desc_add(a, ks * 32), desc_add(b, ks * 32), id_qk, ks > 0);
         mma_commit_w(s_full + i);
@@ -236,22 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       long g = 0;                   // ring position of the item's first key tile
       int p_cnt[kNQ] = {0, 0};      // p_full phases consumed per tile
       int o_cnt[kNQ] = {0, 0};      // o_full phases committed per tile
-      int r_cnt[kNQ] = {0, 0};      // s_read phases consumed per tile
       bool ok = true;
-      // groups 1..G-1 of the scores of key tile at ring stage st, for the
-      // tiles i with has(i): each overwrites the previous group's scores, so
-      // it waits until the weight warps of tile i have read them
-      auto issue_groups = [&](int qb, int st, bool has0, bool has1) -> bool {
-        for (int grp = 1; grp < G; ++grp)
-          for (int i = 0; i < kNQ; ++i) {
-            if (!(i == 0 ? has0 : has1)) continue;
-            if (!mbar_wait_w(s_read + i, r_cnt[i] & 1, env)) return false;
-            ++r_cnt[i];
-            tc_fence_after();
-            issue_qk(i, qb, st, grp);
-          }
-        return true;
-      };
       for (int it = my_item(nq); ok && it >= 0; it = my_item(++nq)) {
         const int qb = nq & 1;
         int nkv[kNQ];
@@ -263,11 +239,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         for (int i = 0; i < kNQ; ++i)
-          if (nkv[i] > 0) issue_qk(i, qb, (int)(g % kStages), 0);
-        if (!issue_groups(qb, (int)(g % kStages), nkv[0] > 0, nkv[1] > 0)) {
-          ok = false;
-          break;
-        }
+          if (nkv[i] > 0) issue_qk(i, qb, (int)(g % kStages));
         long kv_ready = g;  // highest ring position whose K/V landed
         for (int j = 0; ok && j < nkv_max; ++j) {
           const long gj = g + j;
@@ -309,14 +281,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 kv_ready = gn;
               }
-              issue_qk(i, qb, (int)(gn % kStages), 0);
+              issue_qk(i, qb, (int)(gn % kStages));
             }
           }
           if (!ok) break;
-          if (!issue_groups(qb, (int)((gj + 1) % kStages), j + 1 < nkv[0], j + 1 < nkv[1])) {
-            ok = false;
-            break;
-          }
           KATA_TRACE(flash, (int)gj, 4);
           mma_commit_w(kv_empty + st);
         }
@@ -383,93 +351,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         // on the diagonal tile, 32-column block bb of row m is kept for
         // bb < quarter, masked for bb == quarter and zero for bb > quarter
         const int bb0 = 2 * h;
-        if constexpr (G == 1) {
 #pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const int bb = bb0 + hh;
-            uint32_t w[16];
-            if (diag && bb > quarter) {
+        for (int hh = 0; hh < 2; ++hh) {
+          const int bb = bb0 + hh;
+          uint32_t w[16];
+          if (diag && bb > quarter) {
 #pragma unroll
-              for (int x = 0; x < 16; ++x) w[x] = 0u;
-            } else {
-              uint32_t r[32];
-              tmem_ld32(sa + 32 * hh, r);
-              tmem_wait_ld();
-              // squares on fp32 pairs (each rounded as a scalar multiply)
-              if (diag && bb == quarter) {
+            for (int x = 0; x < 16; ++x) w[x] = 0u;
+          } else {
+            uint32_t r[32];
+            tmem_ld32(sa + 32 * hh, r);
+            tmem_wait_ld();
+            // squares on fp32 pairs (each rounded as a scalar multiply)
+            if (diag && bb == quarter) {
 #pragma unroll
-                for (int x = 0; x < 16; ++x) {
-                  const uint32_t a = 2 * x > lane ? 0u : r[2 * x], b = 2 * x + 1 > lane ? 0u : r[2 * x + 1];
-                  const uint64_t sq = f32x2_mul(f32x2(a, b), f32x2(a, b));
-                  w[x] = pack_bf16x2(f32x2_lo(sq), f32x2_hi(sq));
-                }
-              } else {
-#pragma unroll
-                for (int x = 0; x < 16; ++x) {
-                  const uint64_t sq = f32x2_mul(f32x2(r[2 * x], r[2 * x + 1]), f32x2(r[2 * x], r[2 * x + 1]));
-                  w[x] = pack_bf16x2(f32x2_lo(sq), f32x2_hi(sq));
-                }
-              }
-            }
-            tmem_st16(sa + 16 * hh, w);
-          }
-        } else {
-          // KATA-Mg: W = sum over the groups of the squared group scores.
-          // The groups' scores arrive one after another in the same columns;
-          // the sum is kept in fp32 pairs, acc[16 hh + y] holding keys
-          // 32 (bb0 + hh) + 2y and + 2y + 1 (blocks above the diagonal are
-          // never read)
-          uint64_t acc[32];
-          for (int grp = 0; grp < G; ++grp) {
-            if (grp > 0) {
-              if (!mbar_wait(s_full + i, s_cnt & 1, env)) {
-                ok = false;
-                break;
-              }
-              ++s_cnt;
-              tc_fence_after();
-            }
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-              if (diag && bb0 + hh > quarter) continue;
-#pragma unroll
-              for (int hf = 0; hf < 4; ++hf) {
-                uint32_t r[8];
-                tmem_ld8(sa + 32 * hh + 8 * hf, r);
-                tmem_wait_ld();
-#pragma unroll
-                for (int x = 0; x < 4; ++x) {
-                  const uint64_t sc = f32x2(r[2 * x], r[2 * x + 1]);
-                  uint64_t& ac = acc[16 * hh + 4 * hf + x];
-                  ac = grp == 0 ? f32x2_mul(sc, sc) : f32x2_fma(sc, sc, ac);
-                }
-              }
-            }
-            if (grp + 1 < G) {
-              tc_fence_before();
-              mbar_arrive(s_read + i);
-            }
-          }
-          if (!ok) break;
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const int bb = bb0 + hh;
-            uint32_t w[16];
-            if (diag && bb > quarter) {
-#pragma unroll
-              for (int y = 0; y < 16; ++y) w[y] = 0u;
-            } else if (diag && bb == quarter) {
-#pragma unroll
-              for (int y = 0; y < 16; ++y) {
-                const uint64_t ac = acc[16 * hh + y];
-                w[y] = pack_bf16x2(2 * y > lane ? 0.f : f32x2_lo(ac), 2 * y + 1 > lane ? 0.f : f32x2_hi(ac));
+              for (int x = 0; x < 16; ++x) {
+                const uint32_t a = 2 * x > lane ? 0u : r[2 * x], b = 2 * x + 1 > lane ? 0u : r[2 * x + 1];
+                const uint64_t sq = f32x2_mul(f32x2(a, b), f32x2(a, b));
+                w[x] = pack_bf16x2(f32x2_lo(sq), f32x2_hi(sq));
               }
             } else {
 #pragma unroll
-              for (int y = 0; y < 16; ++y) w[y] = pack_bf16x2(f32x2_lo(acc[16 * hh + y]), f32x2_hi(acc[16 * hh + y]));
+              for (int x = 0; x < 16; ++x) {
+                const uint64_t sq = f32x2_mul(f32x2(r[2 * x], r[2 * x + 1]), f32x2(r[2 * x], r[2 * x + 1]));
+                w[x] = pack_bf16x2(f32x2_lo(sq), f32x2_hi(sq));
+              }
             }
-            tmem_st16(sa + 16 * hh, w);
           }
+          tmem_st16(sa + 16 * hh, w);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -615,18 +524,17 @@ bool make_tmap_bf16_4d(CUtensorMap* map, const void* base, int inner, int T, int
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int p, int DV, int G>
+template <int p, int DV>
 static cudaError_t launch_flash_t(const void* q, const void* k, const void* v, void* o, int B, int H, int T, bool bthd,
                                   const WaitCtl& wc, cudaStream_t st) {
-  using Cfg = FlashCfg<p, DV, G>;
+  using Cfg = FlashCfg<p, DV>;
   const int BH = B * H;
   CUtensorMap tq, tk, tv, to;
-  if (!make_tmap_bf16_4d(&tq, q, Cfg::kD, T, H, B, bthd, Cfg::kD, kBM) ||
-      !make_tmap_bf16_4d(&tk, k, Cfg::kD, T, H, B, bthd, Cfg::kD, kBN) ||
+  if (!make_tmap_bf16_4d(&tq, q, p, T, H, B, bthd, p, kBM) || !make_tmap_bf16_4d(&tk, k, p, T, H, B, bthd, p, kBN) ||
       !make_tmap_bf16_4d(&tv, v, DV, T, H, B, bthd, DV, kBN) ||
       !make_tmap_bf16_4d(&to, o, DV, T, H, B, bthd, DV / 2, 32))
     return cudaErrorInvalidValue;
-  auto kern = flash_fwd_kernel<p, DV, G>;
+  auto kern = flash_fwd_kernel<p, DV>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
   if (e != cudaSuccess) return e;
   // persistent: one CTA per SM (or fewer when there are fewer work items)
@@ -643,23 +551,12 @@ static cudaError_t launch_flash_t(const void* q, const void* k, const void* v, v
   return cudaGetLastError();
 }
 
-bool flash_sm100_supports(int p, int groups, int dv) {
-  if (groups == 1) return (p == 16 || p == 32) && (dv == 16 || dv == 64);
-  return dv == 64 && ((p == 16 && (groups == 2 || groups == 4)) || (p == 32 && groups == 2));
-}
-
-cudaError_t launch_flash_sm100(const void* q, const void* k, const void* v, void* o, int B, int H, int T, int p,
-                               int groups, int dv, bool bthd, const WaitCtl& wc, cudaStream_t st) {
-  if (groups == 1) {
-    if (p == 16 && dv == 64) return launch_flash_t<16, 64, 1>(q, k, v, o, B, H, T, bthd, wc, st);
-    if (p == 16 && dv == 16) return launch_flash_t<16, 16, 1>(q, k, v, o, B, H, T, bthd, wc, st);
-    if (p == 32 && dv == 64) return launch_flash_t<32, 64, 1>(q, k, v, o, B, H, T, bthd, wc, st);
-    if (p == 32 && dv == 16) return launch_flash_t<32, 16, 1>(q, k, v, o, B, H, T, bthd, wc, st);
-  } else if (dv == 64) {
-    if (p == 16 && groups == 2) return launch_flash_t<16, 64, 2>(q, k, v, o, B, H, T, bthd, wc, st);
-    if (p == 16 && groups == 4) return launch_flash_t<16, 64, 4>(q, k, v, o, B, H, T, bthd, wc, st);
-    if (p == 32 && groups == 2) return launch_flash_t<32, 64, 2>(q, k, v, o, B, H, T, bthd, wc, st);
-  }
+cudaError_t launch_flash_sm100(const void* q, const void* k, const void* v, void* o, int B, int H, int T, int p, int dv,
+                               bool bthd, const WaitCtl& wc, cudaStream_t st) {
+  if (p == 16 && dv == 64) return launch_flash_t<16, 64>(q, k, v, o, B, H, T, bthd, wc, st);
+  if (p == 16 && dv == 16) return launch_flash_t<16, 16>(q, k, v, o, B, H, T, bthd, wc, st);
+  if (p == 32 && dv == 64) return launch_flash_t<32, 64>(q, k, v, o, B, H, T, bthd, wc, st);
+  if (p == 32 && dv == 16) return launch_flash_t<32, 16>(q, k, v, o, B, H, T, bthd, wc, st);
   return cudaErrorInvalidValue;
 }
 

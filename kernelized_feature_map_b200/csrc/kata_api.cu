@@ -149,7 +149,7 @@ KATA_API kata_status_t kata_fwd_quadratic(const void* q, const void* k, const vo
   if (!q || !k || !v || !o) return KATA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return KATA_ERR_MISALIGNED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (dtype == KATA_BF16) return from_cuda(launch_flash_sm100(q, k, v, o, B, H, T, p, 1, dv, false, wait_ctl(), st));
+  if (dtype == KATA_BF16) return from_cuda(launch_flash_sm100(q, k, v, o, B, H, T, p, dv, false, wait_ctl(), st));
   return from_cuda(launch_quadratic_simt(q, k, v, o, B * H, T, p, dv, dtype, st));
 }
 
@@ -254,7 +254,7 @@ static kata_status_t check_mg(int B, int H, int T, int d, int groups, int dv, ka
   kata_status_t s = check_common(B, H, T, p, dv, dt);
   if (s != KATA_OK) return s;
   if ((long long)T * d >= (1ll << 31)) return KATA_ERR_UNSUPPORTED;
-  if (!flash_sm100_supports(p, groups, dv)) return KATA_ERR_UNSUPPORTED;
+  if (groups > 1 && !flash_mg_sm100_supports(p, groups, dv)) return KATA_ERR_UNSUPPORTED;
   *p_out = p;
   return KATA_OK;
 }
@@ -270,8 +270,10 @@ KATA_API kata_status_t kata_fwd_mg_quadratic(const void* q, const void* k, const
   if (T == 0) return KATA_OK;
   if (!q || !k || !v || !o) return KATA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return KATA_ERR_MISALIGNED;
-  return from_cuda(launch_flash_sm100(q, k, v, o, B, H, T, p, groups, dv, layout == KATA_LAYOUT_BTHD, wait_ctl(),
-                                      static_cast<cudaStream_t>(stream)));
+  const bool bthd = layout == KATA_LAYOUT_BTHD;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (groups == 1) return from_cuda(launch_flash_sm100(q, k, v, o, B, H, T, p, dv, bthd, wait_ctl(), st));
+  return from_cuda(launch_flash_mg_sm100(q, k, v, o, B, H, T, p, groups, bthd, wait_ctl(), st));
 }
 
 KATA_API kata_status_t kata_decode_step_mg(const void* q, const void* k, const void* v, void* o, float* S, float* z,

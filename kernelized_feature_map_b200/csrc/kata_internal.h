@@ -63,12 +63,17 @@ cudaError_t launch_chunk_aggregate_simt(const void* k, const void* v, float* ws,
 cudaError_t launch_chunk_readout_simt(const void* q, const void* k, const void* v, void* o, float* ws,
                                       const ChunkPlan& plan, kata_dtype_t dt, cudaStream_t st);
 
-// flash_sm100.cu -- tcgen05 flash-style forward (bf16 inputs) with `groups`
-// PSD factors of width p per head; bthd selects the [B,T,H,*] layout of
-// q, k, v and o instead of [B,H,T,*].
-bool flash_sm100_supports(int p, int groups, int dv);
-cudaError_t launch_flash_sm100(const void* q, const void* k, const void* v, void* o, int B, int H, int T, int p,
-                               int groups, int dv, bool bthd, const WaitCtl& wc, cudaStream_t st);
+// flash_sm100.cu -- tcgen05 flash-style forward (bf16 inputs), one PSD
+// factor of width p per head; bthd selects the [B,T,H,*] layout of q, k, v
+// and o instead of [B,H,T,*].
+cudaError_t launch_flash_sm100(const void* q, const void* k, const void* v, void* o, int B, int H, int T, int p, int dv,
+                               bool bthd, const WaitCtl& wc, cudaStream_t st);
+
+// flash_mg_sm100.cu -- tcgen05 flash-style KATA-Mg forward (bf16 inputs,
+// dv = 64) with `groups` PSD factors of width p per head.
+bool flash_mg_sm100_supports(int p, int groups, int dv);
+cudaError_t launch_flash_mg_sm100(const void* q, const void* k, const void* v, void* o, int B, int H, int T, int p,
+                                  int groups, bool bthd, const WaitCtl& wc, cudaStream_t st);
 
 // chunk_sm100.cu -- tcgen05 chunked-state forward (bf16 inputs, p = 16).
 // The state kernel sums super-chunks 0..G-2 (the last one's sum is never
