@@ -51,10 +51,10 @@ UNIT = "tokens/s"
 # DRAM bytes (read + write) of one flash_fwd_kernel launch at B8 H16 T2048,
 # from the ncu capture summarised in profiles/flash_fwd_kernel_ctx2k.md.  It
 # is reported only while the kernel's sources are the ones that capture ran.
-FLASH_TRAFFIC_BYTES = 50633984 + 5805824
+FLASH_TRAFFIC_BYTES = 50535424 + 6024448
 FLASH_TRAFFIC_SOURCES = ("kernelized_feature_map_b200/csrc/flash_sm100.cu", "kernelized_feature_map_b200/csrc/sm100.cuh",
                          "kernelized_feature_map_b200/csrc/kata_trace.cuh", "kernelized_feature_map_b200/csrc/kata_common.cuh")
-FLASH_TRAFFIC_SHA256 = "172325a6a08b5de78f41e033a4a6ffeaa5a2b477c0942680287c298cf2438c53"
+FLASH_TRAFFIC_SHA256 = "7e106fad3b63565fcfa6bbfca7c8a6597349ff0803f6c324d62cf9c30866e1aa"
 
 
 def flash_traffic(workload):
@@ -382,6 +382,7 @@ def run_ours(args, rank, world, local_rank):
         long["decode_b64"] = run_decode_b64(args, K, torch, dev, stream, flush)
         if args.sweep:
             long["sweep"], long["recall"] = run_sweep(args, K, torch, dev, stream, flush)
+            long["mg"] = run_mg(args, K, torch, dev, stream, flush)
 
     status = K.kata_get_status()
     return dict(step_ms=step_ms, eager_step_ms=eager_step_ms, graph=bool(args.graph), path_ms=path_ms.tolist(),
@@ -506,6 +507,39 @@ def run_sweep(args, K, torch, dev, stream, flush):
                                         stream, 3, 1),
                   quadratic_ms=_time_call(lambda: K.kata_fwd_quadratic(q, k, v, o=o), flush, stream, 3, 1))
     return grid, recall
+
+
+def run_mg(args, K, torch, dev, stream, flush):
+    """KATA-Mg forward (several PSD factors per head) on the workloads of
+    workloads.MG_CONFIGS: the 340M model's d = 64 heads in 2 or 4 groups at
+    T = 2048, in the [B,T,H,d] layout of the pages' attention call."""
+    bf = torch.bfloat16
+    out = {}
+    for name, cfg in sorted(workloads.MG_CONFIGS.items()):
+        B, H, T, d, g, dv = cfg["B"], cfg["H"], cfg["T"], cfg["d"], cfg["groups"], cfg["dv"]
+        qn, kn, vn = workloads.normal_qkv(B, H, T, d, dv, seed=cfg["seed"], dtype=cfg["dtype"])
+        q, k, v = (torch.from_numpy(np.ascontiguousarray(x.transpose(0, 2, 1, 3))).to(dev, bf) for x in (qn, kn, vn))
+        o = torch.empty_like(v)
+        ms = _time_call(lambda: K.kata_fwd_mg_quadratic(q, k, v, g, layout=cfg["layout"], o=o), flush, stream, 10, 3)
+        out[name] = dict(B=B, H=H, T=T, d=d, groups=g, dv=dv, layout=cfg["layout"], ms=ms)
+        del q, k, v, o
+    # decode step on the concatenated per-group state (B = 64, as for the
+    # single-factor decode line): HBM-bound, the state is read and written once
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(77)
+    for g in (2, 4):
+        B, H, d, dv = 64, 16, 64, 64
+        P = g * (d // g) ** 2
+        q = torch.randn((B, H, d), generator=gen, device=dev).to(bf)
+        k = torch.randn((B, H, d), generator=gen, device=dev).to(bf)
+        v = torch.randn((B, H, dv), generator=gen, device=dev).to(bf)
+        S = torch.randn((B, H, P, dv), generator=gen, device=dev)
+        z = torch.rand((B, H, P), generator=gen, device=dev) + 0.5
+        o = torch.empty((B, H, dv), dtype=bf, device=dev)
+        ms = _time_call(lambda: K.kata_decode_step_mg(q, k, v, S, z, g, o=o), flush, stream, 20, 3)
+        out["decode_mg%d_b64" % g] = dict(B=B, H=H, d=d, groups=g, dv=dv, P=P, ms=ms)
+        del q, k, v, S, z, o
+    return out
 
 
 # ---------------------------------------------------------------------------
@@ -691,6 +725,23 @@ def report(args, res, step_ms, e2e_ms, world):
                 "quadratic": {"ms": rc["quadratic_ms"], "tokens_per_s": rtok / (rc["quadratic_ms"] * 1e-3),
                               "tensor_frac": flash_flops(rc["B"] * rc["H"], rc["T"], rc["p"], rc["dv"])
                               / (rc["quadratic_ms"] * 1e-3) / 1e12 / tf}}
+        if "mg" in lg:
+            line["mg"] = {}
+            for name, m in lg["mg"].items():
+                if "P" in m:  # decode step
+                    mb = 2 * m["B"] * m["H"] * (m["P"] * m["dv"] + m["P"]) * 4
+                    line["mg"][name] = {
+                        "workload": "KATA-Mg decode step B=%d H=%d d=%d groups=%d state [%d x %d] fp32" % (
+                            m["B"], m["H"], m["d"], m["groups"], m["P"], m["dv"]),
+                        "ms": m["ms"], "tokens_per_s": m["B"] / (m["ms"] * 1e-3),
+                        "hbm_frac": mb / (m["ms"] * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+                else:
+                    line["mg"][name] = {
+                        "workload": "KATA-Mg B=%d H=%d T=%d d=%d groups=%d dv=%d bf16 [%s]" % (
+                            m["B"], m["H"], m["T"], m["d"], m["groups"], m["dv"], m["layout"]),
+                        "ms": m["ms"], "tokens_per_s": m["B"] * m["T"] / (m["ms"] * 1e-3),
+                        "tensor_frac": flash_flops(m["B"] * m["H"], m["T"], m["d"], m["dv"]) / (m["ms"] * 1e-3)
+                        / 1e12 / peaks["bf16_tflops"]}
     if args.cpu_baseline and world == 1:
         cb = time_oracle(cfg)
         line["cpu_baseline"] = {"value": cb["value"], "unit": UNIT, "cores": cb["cores"], "kind": "oracle",

@@ -13,20 +13,25 @@
 //     of 128 rows stream through a 4-stage TMA ring that continues across
 //     items; the next item's Q tile is prefetched into a second buffer.
 //   * The scores of two groups fit TMEM side by side (S_0 and S_1, 128 fp32
-//     columns each, beside the [O|D] accumulator), so one hand-off between
-//     the MMA warp and the weight warps covers two groups: G = 2 needs one
-//     round per key tile, G = 4 two rounds whose squares are summed in
-//     registers.
+//     columns each), so one hand-off between the MMA warp and the weight
+//     warps covers two groups: G = 2 needs one round per key tile, G = 4
+//     two rounds whose squares are summed in registers.
 //   * Sixteen weight warps share the tile: the warp of TMEM lane quarter qr
 //     and key quarter kq owns rows 32qr.. and keys 32kq..32kq+31, reads
 //     those 32 columns of every group's scores, sums the squares in fp32
 //     pairs, applies the causal mask on the diagonal tile, and writes its 32
-//     bf16 weights over the first 16 of its own S_0 columns (no warp writes
-//     columns another warp reads).
+//     bf16 weights to its 16 columns of a weight buffer.
+//   * The weights live apart from the scores, in two alternating TMEM
+//     buffers, so the scores of key tile j+1 are computed as soon as the
+//     weight warps have loaded those of tile j (barrier s_read), while they
+//     square and convert; [O|D] += W_j [V_j | 1] follows once W_j is written
+//     (B8 H16 T2048 d64, two groups: 132 -> 115 us against weights written
+//     over the scores).  What remains is mostly the tensor pipe: the P.V
+//     MMAs, which read their A operand from TMEM, run at about half rate
+//     while sixteen warps load scores from TMEM beside them.
 //   * [O|D] += W [V | 1] by one tcgen05.mma per 16 keys (A = W from TMEM),
 //     the denominator coming out of the same MMA from the identical bf16
-//     weights.  The MMA for the next key tile's scores follows in issue
-//     order, so it overwrites the weights only after they were read.
+//     weights.
 //   * Epilogue: each weight warp reads its 32 rows x 16 value columns of
 //     [O|D], frees the accumulator, scales by 1/D (D = 0 gives 0), rounds to
 //     bf16 and stages them as its own 32B-swizzled box; one TMA store per
@@ -39,7 +44,10 @@
 #include <cuda.h>
 
 #include "kata_internal.h"
+#include "kata_trace.cuh"
 #include "sm100.cuh"
+
+KATA_TRACE_DECLARE(mg)
 
 namespace kata {
 
@@ -69,9 +77,10 @@ struct MgCfg {
   static constexpr uint32_t kQKSbo = 8 * kD * 2;
   static constexpr uint32_t kVSbo = 8 * kMgDV * 2;
   static constexpr uint32_t kVKStep = 16 * kMgDV * 2;
-  // TMEM columns: scores of the round's two groups, then [O | D]
+  // TMEM columns: scores of the round's groups, two weight buffers, [O | D]
   static constexpr uint32_t colS(int gg) { return (uint32_t)gg * 128; }
-  static constexpr uint32_t colO = 256;
+  static constexpr uint32_t colW(int b) { return 256u + 64u * (uint32_t)b; }
+  static constexpr uint32_t colO = 384;
   static constexpr uint32_t colD = colO + kMgDV;
   // shared memory (offsets from a 1024-aligned base)
   static constexpr int offQ = 0;                                   // 2 buffers
@@ -81,7 +90,7 @@ struct MgCfg {
   static constexpr int kOutSlab = 32 * 16 * 2;                     // [32 rows x 16 values] per warp
   static constexpr int offOut = offOnes + kOnesBytes;
   static constexpr int offBar = offOut + 16 * kOutSlab;
-  static constexpr int kNumBars = 4 + 2 * kMgStages + 6;
+  static constexpr int kNumBars = 4 + 2 * kMgStages + 7;
   static constexpr int offMisc = offBar + kNumBars * 8;
   static constexpr int kSmemBytes = offMisc + 16 + 1024;
   static_assert(G % kGR == 0, "groups per round");
@@ -103,14 +112,15 @@ __global__ void __launch_bounds__(kMgThreads, 1)
   uint64_t* kv_empty = kv_full + kMgStages;   // [kMgStages]
   uint64_t* s_full = kv_empty + kMgStages;    // a round's scores in TMEM
   uint64_t* s_read = s_full + 1;              // a round's scores read (512)
-  uint64_t* p_full = s_read + 1;              // weights written (512)
-  uint64_t* o_full = p_full + 1;              // [O|D] of the item complete
+  uint64_t* p_full = s_read + 1;              // [2] weight buffer written (512)
+  uint64_t* o_full = p_full + 2;              // [O|D] of the item complete
   uint64_t* o_free = o_full + 1;              // [O|D] read by the epilogue (512)
   uint64_t* mma_done = o_free + 1;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Cfg::offMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::offMisc + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  KATA_TRACE_BEGIN(mg);
   const int n_tiles = (T + kMgBM - 1) / kMgBM;
   const int n_items = n_tiles * BH;
   auto item_tile = [&](int it) { return n_tiles - 1 - it / BH; };  // heaviest first
@@ -132,6 +142,7 @@ __global__ void __launch_bounds__(kMgThreads, 1)
     mbar_init(s_full, 1);
     mbar_init(s_read, 512);
     mbar_init(p_full, 512);
+    mbar_init(p_full + 1, 512);
     mbar_init(o_full, 1);
     mbar_init(o_free, 512);
     mbar_init(mma_done, 1);
@@ -208,19 +219,21 @@ __global__ void __launch_bounds__(kMgThreads, 1)
         }
         mma_commit_w(s_full);
       };
-      int r_cnt = 0, p_cnt = 0, o_cnt = 0;
-      // all rounds of one key tile; rounds after the first overwrite the
-      // previous round's scores, so each waits until they were read
+      // rounds issued so far; round k + 1 overwrites the scores of round k,
+      // so it first waits until the weight warps have loaded them (s_read)
+      int r_cnt = 0;
       auto issue_tile = [&](int qb, int st) -> bool {
-        issue_round(qb, st, 0);
-        for (int r = 1; r < Cfg::kRounds; ++r) {
-          if (!mbar_wait_w(s_read, r_cnt & 1, env)) return false;
+        for (int r = 0; r < Cfg::kRounds; ++r) {
+          if (r_cnt > 0) {
+            if (!mbar_wait_w(s_read, (r_cnt - 1) & 1, env)) return false;
+            tc_fence_after();
+          }
           ++r_cnt;
-          tc_fence_after();
           issue_round(qb, st, r);
         }
         return true;
       };
+      int n_step = 0, o_cnt = 0;  // key steps done (weight buffer n_step % 2); items finished
       int nq = 0;
       long g = 0;
       bool ok = true;
@@ -232,36 +245,20 @@ __global__ void __launch_bounds__(kMgThreads, 1)
           break;
         }
         tc_fence_after();
+        KATA_TRACE(mg, n_step, 0);
         if (!issue_tile(qb, (int)(g % kMgStages))) {
           ok = false;
           break;
         }
+        KATA_TRACE(mg, n_step, 1);
         for (int j = 0; j < nkv; ++j) {
           const long gj = g + j;
           const int st = (int)(gj % kMgStages);
-          const uint32_t sVst = sV + st * Cfg::kVBytes;
-          const uint64_t dv = smem_desc(sVst, sOnes - sVst, Cfg::kVSbo, kSw128);  // V atom, then ones atom
-          if (!mbar_wait_w(p_full, p_cnt & 1, env)) {
-            ok = false;
-            break;
-          }
-          ++p_cnt;
-          // the first P.V of the item overwrites [O|D]: the previous item's
-          // epilogue must have read it
-          if (j == 0 && o_cnt > 0 && !mbar_wait_w(o_free, (o_cnt - 1) & 1, env)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-#pragma unroll
-          for (int ks = 0; ks < kMgBN / 16; ++ks)  // keys 16ks..: weights at S_0 column 32(ks/2) + 8(ks%2)
-            mma_ts_w(tmem + Cfg::colO, tmem + Cfg::colS(0) + (ks >> 1) * 32 + (ks & 1) * 8,
-                     desc_add(dv, ks * Cfg::kVKStep), id_pv, (j > 0 || ks > 0) ? 1u : 0u);
-          if (j == nkv - 1) {
-            mma_commit_w(o_full);
-            ++o_cnt;
-          } else {
+          // scores of key tile j + 1 first: they run while the weight warps
+          // square tile j
+          if (j + 1 < nkv) {
             const long gn = gj + 1;
+            KATA_TRACE(mg, n_step + 1, 0);
             if (!mbar_wait_w(kv_full + gn % kMgStages, (int)((gn / kMgStages) & 1), env)) {
               ok = false;
               break;
@@ -271,6 +268,32 @@ __global__ void __launch_bounds__(kMgThreads, 1)
               ok = false;
               break;
             }
+            KATA_TRACE(mg, n_step + 1, 1);
+          }
+          const int wb = n_step & 1;
+          if (!mbar_wait_w(p_full + wb, (n_step >> 1) & 1, env)) {
+            ok = false;
+            break;
+          }
+          KATA_TRACE(mg, n_step, 2);
+          ++n_step;
+          // the first P.V of the item overwrites [O|D]: the previous item's
+          // epilogue must have read it
+          if (j == 0 && o_cnt > 0 && !mbar_wait_w(o_free, (o_cnt - 1) & 1, env)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sVst = sV + st * Cfg::kVBytes;
+          const uint64_t dv = smem_desc(sVst, sOnes - sVst, Cfg::kVSbo, kSw128);  // V atom, then ones atom
+#pragma unroll
+          for (int ks = 0; ks < kMgBN / 16; ++ks)  // keys 16ks..: weight buffer columns 8ks..
+            mma_ts_w(tmem + Cfg::colO, tmem + Cfg::colW(wb) + 8 * ks, desc_add(dv, ks * Cfg::kVKStep), id_pv,
+                     (j > 0 || ks > 0) ? 1u : 0u);
+          KATA_TRACE(mg, n_step - 1, 3);
+          if (j == nkv - 1) {
+            mma_commit_w(o_full);
+            ++o_cnt;
           }
           mma_commit_w(kv_empty + st);
         }
@@ -299,7 +322,8 @@ __global__ void __launch_bounds__(kMgThreads, 1)
       }
       pend = false;
     };
-    int s_cnt = 0, o_cnt = 0;
+    int s_cnt = 0, o_cnt = 0, n_step = 0;
+    const int tslot = (warp == 2 && lane == 0) ? 5 : (warp == 17 && lane == 0) ? 8 : -1;  // traced warps
     bool ok = true;
     int rr = 0;
     for (int it = my_item(rr); ok && it >= 0; it = my_item(++rr)) {
@@ -318,28 +342,30 @@ __global__ void __launch_bounds__(kMgThreads, 1)
             break;
           }
           ++s_cnt;
+          if (tslot >= 0 && r == 0) KATA_TRACE(mg, n_step, tslot);
           tc_fence_after();
           if (!skip) {
 #pragma unroll
             for (int gg = 0; gg < Cfg::kGR; ++gg) {
 #pragma unroll
               for (int hf = 0; hf < 2; ++hf) {
-                uint32_t s[16];
-                tmem_ld16(lane_base + Cfg::colS(gg) + 32 * kq + 16 * hf, s);
+                uint32_t sc16[16];
+                tmem_ld16(lane_base + Cfg::colS(gg) + 32 * kq + 16 * hf, sc16);
                 tmem_wait_ld();
 #pragma unroll
                 for (int x = 0; x < 8; ++x) {
-                  const uint64_t sc = f32x2(s[2 * x], s[2 * x + 1]);
+                  const uint64_t sc = f32x2(sc16[2 * x], sc16[2 * x + 1]);
                   uint64_t& a = acc[8 * hf + x];
                   a = (r == 0 && gg == 0) ? f32x2_mul(sc, sc) : f32x2_fma(sc, sc, a);
                 }
               }
             }
           }
-          if (r + 1 < Cfg::kRounds) {
-            tc_fence_before();
-            mbar_arrive(s_read);
-          }
+          // the scores are in registers: the next round or key tile may
+          // overwrite them
+          tc_fence_before();
+          mbar_arrive(s_read);
+          if (tslot >= 0 && r == Cfg::kRounds - 1) KATA_TRACE(mg, n_step, tslot + 1);
         }
         if (!ok) break;
         uint32_t w[16];
@@ -354,10 +380,15 @@ __global__ void __launch_bounds__(kMgThreads, 1)
 #pragma unroll
           for (int y = 0; y < 16; ++y) w[y] = pack_bf16x2(f32x2_lo(acc[y]), f32x2_hi(acc[y]));
         }
-        tmem_st16(lane_base + Cfg::colS(0) + 32 * kq, w);
+        // weight buffer n_step % 2: the P.V that last read it (two key steps
+        // ago) completed before the scores just read were computed
+        const int wb = n_step & 1;
+        ++n_step;
+        tmem_st16(lane_base + Cfg::colW(wb) + 16 * kq, w);
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(p_full);
+        mbar_arrive(p_full + wb);
+        if (tslot >= 0) KATA_TRACE(mg, n_step - 1, tslot + 2);
         if (j == 0) flush_out();
       }
       if (!ok || !mbar_wait(o_full, o_cnt & 1, env)) break;
@@ -433,6 +464,10 @@ static cudaError_t launch_flash_mg_t(const void* q, const void* k, const void* v
 
 }  // namespace
 
+// One group per head stays on the single-factor kernel (flash_sm100.cu): its
+// two query tiles per CTA interleave one tile's weights with the other's
+// MMAs, which this kernel's single tile cannot (82 against 104 us at
+// B8 H16 T2048 p16, with bitwise identical outputs).
 bool flash_mg_sm100_supports(int p, int groups, int dv) {
   return dv == kMgDV && ((p == 16 && (groups == 2 || groups == 4)) || (p == 32 && groups == 2));
 }

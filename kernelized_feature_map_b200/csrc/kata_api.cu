@@ -272,8 +272,9 @@ KATA_API kata_status_t kata_fwd_mg_quadratic(const void* q, const void* k, const
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return KATA_ERR_MISALIGNED;
   const bool bthd = layout == KATA_LAYOUT_BTHD;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (groups == 1) return from_cuda(launch_flash_sm100(q, k, v, o, B, H, T, p, dv, bthd, wait_ctl(), st));
-  return from_cuda(launch_flash_mg_sm100(q, k, v, o, B, H, T, p, groups, bthd, wait_ctl(), st));
+  if (flash_mg_sm100_supports(p, groups, dv))
+    return from_cuda(launch_flash_mg_sm100(q, k, v, o, B, H, T, p, groups, bthd, wait_ctl(), st));
+  return from_cuda(launch_flash_sm100(q, k, v, o, B, H, T, p, dv, bthd, wait_ctl(), st));
 }
 
 KATA_API kata_status_t kata_decode_step_mg(const void* q, const void* k, const void* v, void* o, float* S, float* z,
