@@ -1,0 +1,59 @@
+"""fp64 gradients of the KATA forward pass (test infrastructure only).
+
+Only the test suite and the benchmark's CPU leg may import this module; it
+shares nothing with the CUDA path.
+
+For one (batch, head) pair, with S_ts = q_t . k_s, w_ts = S_ts^2 (s <= t),
+N_t = sum_s w_ts v_s, D_t = sum_s w_ts and o_t = N_t / D_t (o_t = 0 when
+D_t = 0) -- the operation of the gist.science technical summary, sec. 2.1
+"Output Gating" and sec. 2.2 "PSD Kegel (Rank-One)" -- the gradients of a
+loss with upstream gradient dO follow by the chain rule:
+
+    dN_t  = dO_t / D_t                   dD_t = -(dO_t . o_t) / D_t
+    dw_ts = dN_t . v_s + dD_t            (s <= t)
+    dv_s  = sum_{t >= s} w_ts dN_t
+    dS_ts = 2 S_ts dw_ts
+    dq_t  = sum_{s <= t} dS_ts k_s       dk_s = sum_{t >= s} dS_ts q_t
+
+and a row with D_t = 0 (its output is the constant 0) passes no gradient.
+The pages print no backward pass; this is the derivative of the forward
+they define, written out step by step (the pages claim the kernels are
+competitive on the training step: arXiv abstract).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+def forward_with_d(q, k, v):
+    """o [B,H,T,dv] and D [B,H,T] in fp64 by the defining sums (T x T matrices)."""
+    q, k, v = (np.asarray(x, np.float64) for x in (q, k, v))
+    S = np.einsum("bhtp,bhsp->bhts", q, k)
+    T = q.shape[2]
+    mask = np.tril(np.ones((T, T), dtype=bool))
+    W = np.where(mask, S * S, 0.0)
+    N = np.einsum("bhts,bhse->bhte", W, v)
+    D = W.sum(axis=-1)
+    safe = np.where(D > 0, D, 1.0)
+    o = np.where((D > 0)[..., None], N / safe[..., None], 0.0)
+    return o, D
+
+
+def backward(q, k, v, dO):
+    """(dq, dk, dv) in fp64 for the upstream gradient dO [B,H,T,dv]."""
+    q, k, v, dO = (np.asarray(x, np.float64) for x in (q, k, v, dO))
+    o, D = forward_with_d(q, k, v)
+    live = D > 0
+    safe = np.where(live, D, 1.0)
+    dN = np.where(live[..., None], dO / safe[..., None], 0.0)
+    dD = np.where(live, -np.einsum("bhte,bhte->bht", dO, o) / safe, 0.0)
+    S = np.einsum("bhtp,bhsp->bhts", q, k)
+    T = q.shape[2]
+    mask = np.tril(np.ones((T, T), dtype=bool))
+    W = np.where(mask, S * S, 0.0)
+    dW = np.where(mask, np.einsum("bhte,bhse->bhts", dN, v) + dD[..., None], 0.0)
+    dv = np.einsum("bhts,bhte->bhse", W, dN)
+    dS = 2.0 * S * dW
+    dq = np.einsum("bhts,bhsp->bhtp", dS, k)
+    dk = np.einsum("bhts,bhtp->bhsp", dS, q)
+    return dq, dk, dv

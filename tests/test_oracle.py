@@ -430,3 +430,60 @@ def test_mg_pins_catch_planted_mistakes(tmp_path, name):
     want = np.einsum("ti,tie->te", fq, S) / np.einsum("ti,ti->t", fq, np.cumsum(fk, axis=0))[:, None]
     caught = caught or not np.allclose(mutant(q1, k1, v1, 5)[0, 0], want, atol=1e-10)
     assert caught, "Mg pin set failed to catch: " + name
+
+
+# ---------------------------------------------------------------------------
+# backward pass: pins of the fp64 gradient oracle
+# ---------------------------------------------------------------------------
+
+from oracle import backward as obw  # noqa: E402
+
+
+def _loss(q, k, v, dO):
+    return float((oracle.direct(q, k, v) * dO).sum())
+
+
+def test_backward_forward_matches_direct():
+    q, k, v = _rand(B=1, H=2, T=30, p=5, dv=3, seed=101)
+    o, D = obw.forward_with_d(q, k, v)
+    np.testing.assert_allclose(o, oracle.direct(q, k, v), rtol=1e-11, atol=1e-12)
+    _, d_rows = oracle.direct_rows(q, k, v, np.zeros(30, np.int64), np.arange(30), return_d=True)
+    np.testing.assert_allclose(D[0, 0], d_rows, rtol=1e-12)
+
+
+def test_backward_matches_finite_differences():
+    """Central differences of the (independently pinned) C direct-sum oracle."""
+    rng = np.random.default_rng(102)
+    q, k, v = _rand(B=1, H=1, T=7, p=3, dv=2, seed=103)
+    dO = rng.standard_normal(v.shape)
+    dq, dk, dv = obw.backward(q, k, v, dO)
+    h = 1e-6
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        num = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args_p = {"q": q, "k": k, "v": v}
+            args_m = dict(args_p)
+            args_p[name], args_m[name] = xp, xm
+            num[idx] = (_loss(args_p["q"], args_p["k"], args_p["v"], dO)
+                        - _loss(args_m["q"], args_m["k"], args_m["v"], dO)) / (2 * h)
+        np.testing.assert_allclose(g, num, rtol=1e-6, atol=1e-7, err_msg=name)
+
+
+def test_backward_identities():
+    """o_t is invariant to scaling q_t, to scaling all keys, and shifts with
+    v: so q_t . dq_t = 0, sum_s k_s . dk_s = 0 and sum_s dv_s = sum_t dO_t."""
+    rng = np.random.default_rng(104)
+    q, k, v = _rand(B=2, H=2, T=40, p=6, dv=4, seed=105)
+    dO = rng.standard_normal(v.shape)
+    dq, dk, dv = obw.backward(q, k, v, dO)
+    np.testing.assert_allclose(np.einsum("bhtp,bhtp->bht", q, dq), 0.0, atol=1e-9)
+    np.testing.assert_allclose(np.einsum("bhsp,bhsp->bh", k, dk), 0.0, atol=1e-9)
+    np.testing.assert_allclose(dv.sum(axis=2), dO.sum(axis=2), rtol=1e-10, atol=1e-10)
+    # a row whose query is zero has D_t = 0: its output is the constant 0
+    q0 = q.copy()
+    q0[:, :, 7] = 0.0
+    dq0, _, _ = obw.backward(q0, k, v, dO)
+    assert np.all(dq0[:, :, 7] == 0.0)
