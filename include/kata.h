@@ -178,6 +178,29 @@ kata_status_t kata_decode_step(const void* q, const void* k, const void* v, void
                                kata_dtype_t dtype, void* stream);
 
 /*
+ * Training: the forward that also saves each row's denominator, and the
+ * backward pass (the chain rule through o = N / D with w = (q.k)^2; the
+ * pages print no backward pass).  bf16 only, p in {16, 32}, dv = 64, the
+ * [B,H,T,*] layouts above; other shapes or fp32: KATA_ERR_UNSUPPORTED.
+ *
+ * kata_fwd_quadratic_train: as kata_fwd_quadratic, and D: [B,H,T] fp32 out,
+ *   D_t = sum_{s<=t} (q_t . k_s)^2.
+ * kata_bwd_quadratic: given q, k, v, the forward's o and D, and the upstream
+ *   gradient dO ([B,H,T,dv]), writes dq, dk ([B,H,T,p]) and dv ([B,H,T,dv]),
+ *   all bf16 (fp32 accumulation).  A row with D_t = 0 (output constant 0)
+ *   passes no gradient.  `workspace` (16-byte aligned, at least
+ *   kata_bwd_quadratic_workspace_size bytes) holds dO/D and (dO.o)/D per row.
+ */
+kata_status_t kata_fwd_quadratic_train(const void* q, const void* k, const void* v, void* o, float* D,
+                                       int B, int H, int T, int p, int dv,
+                                       kata_dtype_t dtype, void* stream);
+size_t kata_bwd_quadratic_workspace_size(int B, int H, int T, int p, int dv, kata_dtype_t dtype);
+kata_status_t kata_bwd_quadratic(const void* q, const void* k, const void* v, const void* o,
+                                 const float* D, const void* dO, void* dq, void* dk, void* dv,
+                                 int B, int H, int T, int p, int dv_width, kata_dtype_t dtype,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * KATA-Mg: g PSD factors per head (arXiv abstract and gist.science sec. 2.3
  * "Varianten": several PSD factors; ai.info summary, Main Findings: state
  * d(d/g+1)/2 * dv packed, the full map at g = 1).  The head's d coordinates
@@ -243,7 +266,7 @@ void kata_set_wait_limit(long long cycles);
 /* ABI version of this header: major * 10000 + minor * 100 + patch. */
 int kata_abi_version(void);
 
-#define KATA_ABI_VERSION 10100
+#define KATA_ABI_VERSION 10200
 
 #ifdef __cplusplus
 }

@@ -17,9 +17,13 @@ The computation lives in ``libkata.so`` (hand-written CUDA behind the C ABI of
 * :func:`kata_fwd_mg_quadratic`, :func:`kata_decode_step_mg` -- KATA-Mg, with
   several PSD factors per head (score sum_j (q^j . k^j)^2), the forward in
   the [B,H,T,d] or [B,T,H,d] layout;
-* :func:`parallel_kata_attn` -- the pages' call shape, [B,T,H,D] in and out.
+* :func:`parallel_kata_attn` -- the pages' call shape, [B,T,H,D] in and out;
+* :func:`kata_fwd_quadratic_train`, :func:`kata_bwd_quadratic` -- the forward
+  that also returns the denominators, and the backward pass;
+  :func:`kata_attention` wraps them as an autograd function.
 """
 from ._abi import (KataError, kata_abi_version, kata_decode_step, kata_fwd_chunked,  # noqa: F401
                    kata_fwd_chunked_noalloc, kata_fwd_chunked_sequential, kata_fwd_chunked_workspace_size,
                    kata_fwd_quadratic, kata_fwd_mg_quadratic, kata_decode_step_mg, parallel_kata_attn,
+                   kata_fwd_quadratic_train, kata_bwd_quadratic, kata_attention, KataAttention,
                    kata_get_status, kata_set_wait_limit, lib, status_string)

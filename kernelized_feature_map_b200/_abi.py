@@ -32,6 +32,9 @@ SIGNATURES = {
     "kata_fwd_chunked_sequential": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                              _c_int, _fp, _fp, _fp, _fp, _vp]),
     "kata_decode_step": (_c_int, [_vp, _vp, _vp, _vp, _fp, _fp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp]),
+    "kata_fwd_quadratic_train": (_c_int, [_vp, _vp, _vp, _vp, _fp] + [_c_int] * 6 + [_vp]),
+    "kata_bwd_quadratic_workspace_size": (_c_size, [_c_int] * 6),
+    "kata_bwd_quadratic": (_c_int, [_vp] * 9 + [_c_int] * 6 + [_vp, _c_size, _vp]),
     "kata_fwd_mg_quadratic": (_c_int, [_vp, _vp, _vp, _vp] + [_c_int] * 8 + [_vp]),
     "kata_decode_step_mg": (_c_int, [_vp, _vp, _vp, _vp, _fp, _fp] + [_c_int] * 6 + [_vp]),
     "kata_get_status": (_c_int, [_vp]),
@@ -206,6 +209,63 @@ def kata_decode_step(q, k, v, S, z, o=None, stream=None):
         _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), _dev(S, "S"), _dev(z, "z"), B, H, p, dv,
         _dtype_code(q), _stream_ptr(stream)))
     return o
+
+
+def kata_fwd_quadratic_train(q, k, v, o=None, D=None, stream=None):
+    """Flash-style forward that also returns each row's denominator.
+
+    q,k [B,H,T,p], v [B,H,T,dv] (bf16) -> (o [B,H,T,dv], D [B,H,T] fp32).
+    """
+    B, H, T, p = q.shape
+    dv = v.shape[-1]
+    if o is None:
+        o = torch.empty((B, H, T, dv), dtype=q.dtype, device=q.device)
+    if D is None:
+        D = torch.empty((B, H, T), dtype=torch.float32, device=q.device)
+    _check("kata_fwd_quadratic_train", lib().kata_fwd_quadratic_train(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), _dev(D, "D"), B, H, T, p, dv, _dtype_code(q),
+        _stream_ptr(stream)))
+    return o, D
+
+
+def kata_bwd_quadratic(q, k, v, o, D, dO, workspace=None, stream=None):
+    """Gradients (dq, dk, dv) of the flash-style forward for the upstream
+    gradient dO, from the forward's o and D (kata_fwd_quadratic_train)."""
+    B, H, T, p = q.shape
+    dvw = v.shape[-1]
+    dq = torch.empty_like(q)
+    dk = torch.empty_like(k)
+    dv = torch.empty_like(v)
+    need = int(lib().kata_bwd_quadratic_workspace_size(B, H, T, p, dvw, _dtype_code(q)))
+    if workspace is None:
+        workspace = torch.empty(max(256, need), dtype=torch.uint8, device=q.device)
+    _check("kata_bwd_quadratic", lib().kata_bwd_quadratic(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), _dev(D, "D"), _dev(dO, "dO"), _dev(dq, "dq"),
+        _dev(dk, "dk"), _dev(dv, "dv"), B, H, T, p, dvw, _dtype_code(q), _dev(workspace, "workspace"),
+        workspace.numel(), _stream_ptr(stream)))
+    return dq, dk, dv
+
+
+class KataAttention(torch.autograd.Function):
+    """Autograd wrapper: forward by kata_fwd_quadratic_train, backward by
+    kata_bwd_quadratic (argument marshalling only)."""
+
+    @staticmethod
+    def forward(ctx, q, k, v):
+        q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+        o, D = kata_fwd_quadratic_train(q, k, v)
+        ctx.save_for_backward(q, k, v, o, D)
+        return o
+
+    @staticmethod
+    def backward(ctx, dO):
+        q, k, v, o, D = ctx.saved_tensors
+        return kata_bwd_quadratic(q, k, v, o, D, dO.contiguous())
+
+
+def kata_attention(q, k, v):
+    """Differentiable flash-style KATA attention, q,k [B,H,T,p], v [B,H,T,dv]."""
+    return KataAttention.apply(q, k, v)
 
 
 def kata_fwd_mg_quadratic(q, k, v, groups, layout="bhtd", o=None, stream=None):

@@ -1,0 +1,591 @@
+// flash_bwd_sm100.cu -- backward pass of the quadratic (flash-style) KATA
+// forward on tcgen05 / TMEM (bf16 inputs, fp32 accumulation, dv = 64).
+//
+// For one (b,h): S_ts = q_t . k_s, w_ts = S_ts^2 (s <= t), o_t = N_t / D_t
+// with N_t = sum_s w_ts v_s and D_t = sum_s w_ts (gist.science technical
+// summary, sec. 2.1 "Output Gating" and sec. 2.2 "PSD Kegel (Rank-One)").
+// Given dO, the chain rule through o = N / D gives
+//   dN_t  = dO_t / D_t,   dD_t = -(dO_t . o_t) / D_t    (0 where D_t = 0)
+//   dS_ts = 2 S_ts (dN_t . v_s + dD_t)                    (s <= t)
+//   dv_s  = sum_{t>=s} w_ts dN_t
+//   dq_t  = sum_{s<=t} dS_ts k_s,   dk_s = sum_{t>=s} dS_ts q_t
+// (the pages print no backward pass; they say the kernels are competitive
+// on the training step, arXiv abstract).  D comes from the forward
+// (kata_fwd_quadratic_train).  Three launches:
+//   1. bwd_prep_kernel   dN (bf16) and dD (fp32) per row, one warp per row;
+//   2. bwd_dq_kernel     one CTA per 128-row query tile: per key tile j,
+//                        S = Q K_j^T and dP = dN V_j^T on the tensor core,
+//                        dS = 2 S (dP + dD) in the weight warps, then
+//                        dQ += dS K_j with dS read from TMEM;
+//   3. bwd_dkdv_kernel   one CTA per 128-row key tile: per query tile i,
+//                        S^T = K Q_i^T and dP^T = V dN_i^T, W^T = (S^T)^2 and
+//                        dS^T in the weight warps, then dV += W^T dN_i and
+//                        dK += dS^T Q_i.
+// Both main kernels keep the products in TMEM with keys (dQ) or queries
+// (dK, dV) along the reduction dimension, so every MMA's A operand comes
+// from TMEM in the K-major form tcgen05 requires and every B operand is a
+// TMA tile read K-major or MN-major as loaded.  The next tile's S and dP are
+// issued as soon as the weight warps have loaded the current ones.
+// Warps: 0 TMA, 1 MMA (converged, elected lane), 2-17 sixteen weight warps
+// (TMEM lane quarter x 32-column quarter).  Every wait is bounded.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "kata_internal.h"
+#include "sm100.cuh"
+
+namespace kata {
+
+bool make_tmap_bf16(CUtensorMap* map, const void* base, int inner, int T, int BH, int rows);
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kBw = 128;          // rows per tile (queries or keys)
+constexpr int kBwDV = 64;
+constexpr int kBwThreads = 576;
+constexpr int kBwStages = 4;
+constexpr uint32_t kBwTmemCols = 512;
+
+// ---------------------------------------------------------------------------
+// 1. dN = dO / D rounded to bf16 and dD = -(dO . o) / D per row; a row with
+//    D = 0 (output constant 0) gets dN = 0 and dD = 0.  One warp per row of
+//    64 values, two per lane.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __restrict__ dO,
+                                                       const __nv_bfloat16* __restrict__ o,
+                                                       const float* __restrict__ D, __nv_bfloat16* __restrict__ dN,
+                                                       float* __restrict__ dD, long long rows) {
+  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const float2 a = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(dO + row * kBwDV)[lane]);
+  const float2 b = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(o + row * kBwDV)[lane]);
+  float dot = fmaf(a.x, b.x, a.y * b.y);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+  const float d = D[row];
+  const float inv = d > 0.f ? 1.f / d : 0.f;
+  reinterpret_cast<__nv_bfloat162*>(dN + row * kBwDV)[lane] = __floats2bfloat162_rn(a.x * inv, a.y * inv);
+  if (lane == 0) dD[row] = -dot * inv;
+}
+
+template <int p>
+struct BwCfg {
+  static constexpr int kQKBytes = kBw * p * 2;         // a Q or K tile
+  static constexpr int kVBytes = kBw * kBwDV * 2;      // a V or dN tile
+  static constexpr Swizzle kQKSw = p == 16 ? kSw32 : kSw64;
+  // 8-row group stride: K-major rows of the Q/K tile, or 8 reduction rows
+  // when the same tile is read MN-major
+  static constexpr uint32_t kQKSbo = 8 * p * 2;
+  static constexpr uint32_t kVSbo = 8 * kBwDV * 2;
+  static constexpr uint32_t kQKKStep = 16 * p * 2;     // 16 rows of a Q/K tile read MN-major
+  static constexpr uint32_t kVKStep = 16 * kBwDV * 2;  // 16 rows of a V/dN tile read MN-major
+  // TMEM columns
+  static constexpr uint32_t colS = 0;                  // S or S^T, fp32
+  static constexpr uint32_t colP = 128;                // dP or dP^T, fp32
+  static constexpr uint32_t colA(int b) { return 256u + 64u * (uint32_t)b; }  // bf16 operands (2 x 64)
+  static constexpr uint32_t colAcc = 384;              // dQ (p) or dV (64) then dK (p)
+};
+
+// Gradient weights (and, with kW, squares) of 16 columns of one row, half
+// HF of the row's 32: s, d are the 16 fp32 scores and dP values, dd(c) the
+// dD term of column c.  g[8 HF + x] receives the bf16 pair of dS = 2 s (d + dd)
+// for columns 2x, 2x + 1, w[8 HF + x] that of s^2; columns with keep(c) false
+// become 0.
+template <int HF, bool kW, typename DD, typename Keep>
+__device__ __forceinline__ void grad_block(const uint32_t (&s)[16], const uint32_t (&d)[16], DD dd, Keep keep,
+                                           uint32_t (&g)[16], uint32_t (&w)[16]) {
+#pragma unroll
+  for (int x = 0; x < 8; ++x) {
+    const float s0 = __uint_as_float(s[2 * x]), s1 = __uint_as_float(s[2 * x + 1]);
+    const float g0 = 2.f * s0 * (__uint_as_float(d[2 * x]) + dd(2 * x));
+    const float g1 = 2.f * s1 * (__uint_as_float(d[2 * x + 1]) + dd(2 * x + 1));
+    const bool k0 = keep(2 * x), k1 = keep(2 * x + 1);
+    g[8 * HF + x] = pack_bf16x2(k0 ? g0 : 0.f, k1 ? g1 : 0.f);
+    if (kW) w[8 * HF + x] = pack_bf16x2(k0 ? s0 * s0 : 0.f, k1 ? s1 * s1 : 0.f);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// 2. dQ: CTA (query tile i, head bh), key tiles j = 0..i
+// ---------------------------------------------------------------------------
+template <int p>
+struct DqSmem {
+  using C = BwCfg<p>;
+  static constexpr int offDN = 0;                                       // dN_i (SW128)
+  static constexpr int offQ = offDN + C::kVBytes;                       // Q_i
+  static constexpr int offK = (offQ + C::kQKBytes + 1023) / 1024 * 1024;  // ring of K_j
+  static constexpr int offV = (offK + kBwStages * C::kQKBytes + 1023) / 1024 * 1024;  // ring of V_j
+  static constexpr int offBar = offV + kBwStages * C::kVBytes;
+  static constexpr int kBars = 1 + 2 * kBwStages + 5;
+  static constexpr int offMisc = offBar + kBars * 8;
+  static constexpr int kBytes = offMisc + 16 + 1024;
+};
+
+template <int p>
+__global__ void __launch_bounds__(kBwThreads, 1)
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_dn,
+                  const float* __restrict__ dD, __nv_bfloat16* __restrict__ dq, int T, WaitCtl wc) {
+  using C = BwCfg<p>;
+  using L = DqSmem<p>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::offBar);
+  uint64_t* q_full = bars;                      // Q_i and dN_i landed
+  uint64_t* kv_full = q_full + 1;               // [kBwStages]
+  uint64_t* kv_empty = kv_full + kBwStages;     // [kBwStages]
+  uint64_t* s_full = kv_empty + kBwStages;      // S and dP of a key tile in TMEM
+  uint64_t* s_read = s_full + 1;                // ... loaded by the weight warps (512)
+  uint64_t* p_full = s_read + 1;                // [2] dS buffer written (512)
+  uint64_t* done = p_full + 2;                  // every MMA of the CTA complete
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::offMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::offMisc + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_tiles = (T + kBw - 1) / kBw;
+  const int tile = n_tiles - 1 - (int)blockIdx.x;  // heaviest first
+  const int bh = blockIdx.y;
+  const int nkv = tile + 1;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < kBwStages; ++s) {
+      mbar_init(kv_full + s, 1);
+      mbar_init(kv_empty + s, 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(s_read, 512);
+    mbar_init(p_full, 512);
+    mbar_init(p_full + 1, 512);
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_holder, kBwTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const WaitEnv env{wc.status, abort_flag, wc.limit};
+
+  if (warp == 0) {
+    // ------------------------------------------------------------- producer
+    if (lane == 0) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      prefetch_tmap(&tm_dn);
+      mbar_arrive_expect_tx(q_full, C::kVBytes + C::kQKBytes);
+      tma_load_3d(smem + L::offDN, &tm_dn, q_full, 0, tile * kBw, bh);
+      tma_load_3d(smem + L::offQ, &tm_q, q_full, 0, tile * kBw, bh);
+      int issued = 0;
+      for (int j = 0; j < nkv; ++j) {
+        const int st = j % kBwStages;
+        if (!mbar_wait(kv_empty + st, ((j / kBwStages) & 1) ^ 1, env)) break;
+        mbar_arrive_expect_tx(kv_full + st, C::kQKBytes + C::kVBytes);
+        tma_load_3d(smem + L::offK + st * C::kQKBytes, &tm_k, kv_full + st, 0, j * kBw, bh);
+        tma_load_3d(smem + L::offV + st * C::kVBytes, &tm_v, kv_full + st, 0, j * kBw, bh);
+        ++issued;
+      }
+      mbar_wait_drain(q_full, 0, wc.limit);
+      for (int j = issued - kBwStages < 0 ? 0 : issued - kBwStages; j < issued; ++j)
+        mbar_wait_drain(kv_full + j % kBwStages, (j / kBwStages) & 1, wc.limit);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------- MMA issuer
+    constexpr uint32_t id_s = idesc_bf16(kBw, kBw, false, false);  // both operands K-major
+    constexpr uint32_t id_dq = idesc_bf16(kBw, p, false, true);    // A = dS (TMEM), B = K_j MN-major
+    const uint64_t dq0 = smem_desc(smem_u32(smem + L::offQ), 16, C::kQKSbo, C::kQKSw);
+    const uint64_t ddn0 = smem_desc(smem_u32(smem + L::offDN), 16, C::kVSbo, kSw128);
+    const uint64_t dk0 = smem_desc(smem_u32(smem + L::offK), 16, C::kQKSbo, C::kQKSw);
+    const uint64_t dv0 = smem_desc(smem_u32(smem + L::offV), 16, C::kVSbo, kSw128);
+    // S = Q K_j^T (K = p) and dP = dN V_j^T (K = dv) of the key tile at stage st
+    auto issue_sdp = [&](int st) {
+#pragma unroll
+      for (int ks = 0; ks < p / 16; ++ks)
+        mma_ss_w(tmem + C::colS, desc_add(dq0, ks * 32), desc_add(dk0, st * C::kQKBytes + ks * 32), id_s, ks > 0);
+#pragma unroll
+      for (int ks = 0; ks < kBwDV / 16; ++ks)
+        mma_ss_w(tmem + C::colP, desc_add(ddn0, ks * 32), desc_add(dv0, st * C::kVBytes + ks * 32), id_s, ks > 0);
+      mma_commit_w(s_full);
+    };
+    bool ok = mbar_wait_w(q_full, 0, env) && mbar_wait_w(kv_full, 0, env);
+    if (ok) {
+      tc_fence_after();
+      issue_sdp(0);
+    }
+    for (int j = 0; ok && j < nkv; ++j) {
+      const int st = j % kBwStages;
+      if (j + 1 < nkv) {
+        const int sn = (j + 1) % kBwStages;
+        // the next tile's S and dP overwrite the current ones: wait until loaded
+        if (!mbar_wait_w(kv_full + sn, ((j + 1) / kBwStages) & 1, env) || !mbar_wait_w(s_read, j & 1, env)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        issue_sdp(sn);
+      }
+      if (!mbar_wait_w(p_full + (j & 1), (j >> 1) & 1, env)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int ks = 0; ks < kBw / 16; ++ks)  // keys 16ks..: dS columns 8ks.. of the buffer
+        mma_ts_w(tmem + C::colAcc, tmem + C::colA(j & 1) + 8 * ks, desc_add(dk0, st * C::kQKBytes + ks * C::kQKKStep),
+                 id_dq, (j > 0 || ks > 0) ? 1u : 0u);
+      mma_commit_w(kv_empty + st);
+    }
+    mma_commit_w(done);
+    mbar_wait_drain(done, 0, wc.limit);
+  } else {
+    // ------------------------------------------------------------- weight warps
+    const int quarter = warp % 4;                 // rows (queries) 32 quarter ..
+    const int kq = (warp - 2) / 4;                // keys 32 kq .. of the key tile
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    const int row = tile * kBw + quarter * 32 + lane;
+    const float dDr = row < T ? dD[(size_t)bh * T + row] : 0.f;
+    bool ok = true;
+    for (int j = 0; j < nkv; ++j) {
+      if (!mbar_wait(s_full, j & 1, env)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      // causal mask on the diagonal tile: key 32 kq + c <= query 32 quarter + lane
+      const bool diag = (j == nkv - 1);
+      const bool skip = diag && kq > quarter;
+      const bool part = diag && kq == quarter;
+      uint32_t g[16], unused[16];
+      if (skip) {
+#pragma unroll
+        for (int x = 0; x < 16; ++x) g[x] = 0u;
+      } else {
+        uint32_t s[16], d[16];
+        auto dd = [&](int) { return dDr; };
+        tmem_ld16(lane_base + C::colS + 32 * kq, s);
+        tmem_ld16(lane_base + C::colP + 32 * kq, d);
+        tmem_wait_ld();
+        grad_block<0, false>(s, d, dd, [&](int c) { return !part || c <= lane; }, g, unused);
+        tmem_ld16(lane_base + C::colS + 32 * kq + 16, s);
+        tmem_ld16(lane_base + C::colP + 32 * kq + 16, d);
+        tmem_wait_ld();
+        grad_block<1, false>(s, d, dd, [&](int c) { return !part || 16 + c <= lane; }, g, unused);
+      }
+      // S and dP are in registers: the next key tile's may overwrite them
+      tc_fence_before();
+      mbar_arrive(s_read);
+      // dS buffer j % 2 was last read by the dQ MMAs of key tile j - 2, which
+      // completed before S(j) did
+      tmem_st16(lane_base + C::colA(j & 1) + 16 * kq, g);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(p_full + (j & 1));
+    }
+    // epilogue: dQ (fp32, p columns) -> bf16, rows < T; warps of key quarter 0
+    if (ok && kq == 0 && mbar_wait(done, 0, env)) {
+      tc_fence_after();
+#pragma unroll
+      for (int c0 = 0; c0 < p; c0 += 16) {
+        uint32_t r[16];
+        tmem_ld16(lane_base + C::colAcc + c0, r);
+        tmem_wait_ld();
+        if (row < T) {
+          uint4* dst = reinterpret_cast<uint4*>(dq + ((size_t)bh * T + row) * p + c0);
+          dst[0] = make_uint4(pack_bf16x2(__uint_as_float(r[0]), __uint_as_float(r[1])),
+                              pack_bf16x2(__uint_as_float(r[2]), __uint_as_float(r[3])),
+                              pack_bf16x2(__uint_as_float(r[4]), __uint_as_float(r[5])),
+                              pack_bf16x2(__uint_as_float(r[6]), __uint_as_float(r[7])));
+          dst[1] = make_uint4(pack_bf16x2(__uint_as_float(r[8]), __uint_as_float(r[9])),
+                              pack_bf16x2(__uint_as_float(r[10]), __uint_as_float(r[11])),
+                              pack_bf16x2(__uint_as_float(r[12]), __uint_as_float(r[13])),
+                              pack_bf16x2(__uint_as_float(r[14]), __uint_as_float(r[15])));
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kBwTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// 3. dK, dV: CTA (key tile j, head bh), query tiles i = j..n_tiles-1
+// ---------------------------------------------------------------------------
+template <int p>
+struct DkvSmem {
+  using C = BwCfg<p>;
+  static constexpr int offV = 0;                                        // V_j (SW128)
+  static constexpr int offK = offV + C::kVBytes;                        // K_j
+  static constexpr int offDN = (offK + C::kQKBytes + 1023) / 1024 * 1024;  // ring of dN_i
+  static constexpr int offQ = offDN + kBwStages * C::kVBytes;           // ring of Q_i
+  static constexpr int offBar = (offQ + kBwStages * C::kQKBytes + 1023) / 1024 * 1024;
+  static constexpr int kBars = 1 + 2 * kBwStages + 5;
+  static constexpr int offMisc = offBar + kBars * 8;
+  static constexpr int kBytes = offMisc + 16 + 1024;
+};
+
+template <int p>
+__global__ void __launch_bounds__(kBwThreads, 1)
+    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_dn,
+                    const float* __restrict__ dD, __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
+                    int T, WaitCtl wc) {
+  using C = BwCfg<p>;
+  using L = DkvSmem<p>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::offBar);
+  uint64_t* kv_full = bars;                     // K_j and V_j landed
+  uint64_t* q_full = kv_full + 1;               // [kBwStages] Q_i and dN_i
+  uint64_t* q_empty = q_full + kBwStages;       // [kBwStages]
+  uint64_t* s_full = q_empty + kBwStages;       // S^T and dP^T of a query tile in TMEM
+  uint64_t* s_read = s_full + 1;                // ... loaded by the weight warps (512)
+  uint64_t* p_full = s_read + 1;                // W^T and dS^T written (512)
+  uint64_t* w_free = p_full + 1;                // ... read by the dV / dK MMAs
+  uint64_t* done = w_free + 1;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::offMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::offMisc + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_tiles = (T + kBw - 1) / kBw;
+  const int tile = (int)blockIdx.x;             // key tile; tile 0 has the most query tiles
+  const int bh = blockIdx.y;
+  const int cnt = n_tiles - tile;               // query tiles tile .. n_tiles - 1
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int s = 0; s < kBwStages; ++s) {
+      mbar_init(q_full + s, 1);
+      mbar_init(q_empty + s, 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(s_read, 512);
+    mbar_init(p_full, 512);
+    mbar_init(w_free, 1);
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_holder, kBwTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const WaitEnv env{wc.status, abort_flag, wc.limit};
+
+  if (warp == 0) {
+    // ------------------------------------------------------------- producer
+    if (lane == 0) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      prefetch_tmap(&tm_dn);
+      mbar_arrive_expect_tx(kv_full, C::kVBytes + C::kQKBytes);
+      tma_load_3d(smem + L::offV, &tm_v, kv_full, 0, tile * kBw, bh);
+      tma_load_3d(smem + L::offK, &tm_k, kv_full, 0, tile * kBw, bh);
+      int issued = 0;
+      for (int n = 0; n < cnt; ++n) {
+        const int st = n % kBwStages, i = tile + n;
+        if (!mbar_wait(q_empty + st, ((n / kBwStages) & 1) ^ 1, env)) break;
+        mbar_arrive_expect_tx(q_full + st, C::kVBytes + C::kQKBytes);
+        tma_load_3d(smem + L::offDN + st * C::kVBytes, &tm_dn, q_full + st, 0, i * kBw, bh);
+        tma_load_3d(smem + L::offQ + st * C::kQKBytes, &tm_q, q_full + st, 0, i * kBw, bh);
+        ++issued;
+      }
+      mbar_wait_drain(kv_full, 0, wc.limit);
+      for (int n = issued - kBwStages < 0 ? 0 : issued - kBwStages; n < issued; ++n)
+        mbar_wait_drain(q_full + n % kBwStages, (n / kBwStages) & 1, wc.limit);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------- MMA issuer
+    constexpr uint32_t id_s = idesc_bf16(kBw, kBw, false, false);
+    constexpr uint32_t id_dv = idesc_bf16(kBw, kBwDV, false, true);  // A = W^T (TMEM), B = dN_i MN-major
+    constexpr uint32_t id_dk = idesc_bf16(kBw, p, false, true);      // A = dS^T (TMEM), B = Q_i MN-major
+    const uint64_t dk0 = smem_desc(smem_u32(smem + L::offK), 16, C::kQKSbo, C::kQKSw);
+    const uint64_t dv0 = smem_desc(smem_u32(smem + L::offV), 16, C::kVSbo, kSw128);
+    const uint64_t dq0 = smem_desc(smem_u32(smem + L::offQ), 16, C::kQKSbo, C::kQKSw);
+    const uint64_t ddn0 = smem_desc(smem_u32(smem + L::offDN), 16, C::kVSbo, kSw128);
+    // S^T = K Q_i^T (K = p) and dP^T = V dN_i^T (K = dv) of the query tile at stage st
+    auto issue_sdp = [&](int st) {
+#pragma unroll
+      for (int ks = 0; ks < p / 16; ++ks)
+        mma_ss_w(tmem + C::colS, desc_add(dk0, ks * 32), desc_add(dq0, st * C::kQKBytes + ks * 32), id_s, ks > 0);
+#pragma unroll
+      for (int ks = 0; ks < kBwDV / 16; ++ks)
+        mma_ss_w(tmem + C::colP, desc_add(dv0, ks * 32), desc_add(ddn0, st * C::kVBytes + ks * 32), id_s, ks > 0);
+      mma_commit_w(s_full);
+    };
+    bool ok = mbar_wait_w(kv_full, 0, env) && mbar_wait_w(q_full, 0, env);
+    if (ok) {
+      tc_fence_after();
+      issue_sdp(0);
+    }
+    for (int n = 0; ok && n < cnt; ++n) {
+      const int st = n % kBwStages;
+      if (n + 1 < cnt) {
+        const int sn = (n + 1) % kBwStages;
+        if (!mbar_wait_w(q_full + sn, ((n + 1) / kBwStages) & 1, env) || !mbar_wait_w(s_read, n & 1, env)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        issue_sdp(sn);
+      }
+      if (!mbar_wait_w(p_full, n & 1, env)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int ks = 0; ks < kBw / 16; ++ks)  // queries 16ks..: operand columns 8ks..
+        mma_ts_w(tmem + C::colAcc, tmem + C::colA(0) + 8 * ks, desc_add(ddn0, st * C::kVBytes + ks * C::kVKStep),
+                 id_dv, (n > 0 || ks > 0) ? 1u : 0u);
+#pragma unroll
+      for (int ks = 0; ks < kBw / 16; ++ks)
+        mma_ts_w(tmem + C::colAcc + kBwDV, tmem + C::colA(1) + 8 * ks,
+                 desc_add(dq0, st * C::kQKBytes + ks * C::kQKKStep), id_dk, (n > 0 || ks > 0) ? 1u : 0u);
+      mma_commit_w(w_free);
+      mma_commit_w(q_empty + st);
+    }
+    mma_commit_w(done);
+    mbar_wait_drain(done, 0, wc.limit);
+  } else {
+    // ------------------------------------------------------------- weight warps
+    const int quarter = warp % 4;                 // rows (keys) 32 quarter ..
+    const int kq = (warp - 2) / 4;                // queries 32 kq .. of the query tile
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    const int row = tile * kBw + quarter * 32 + lane;  // this thread's key
+    bool ok = true;
+    for (int n = 0; n < cnt; ++n) {
+      // dD of this warp's 32 queries, one per lane (0 past T)
+      const int qrow = (tile + n) * kBw + 32 * kq + lane;
+      const float dDl = qrow < T ? dD[(size_t)bh * T + qrow] : 0.f;
+      if (!mbar_wait(s_full, n & 1, env)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      // causal mask on the diagonal tile: query 32 kq + c >= key 32 quarter + lane
+      const bool diag = (n == 0);
+      const bool skip = diag && kq < quarter;
+      const bool part = diag && kq == quarter;
+      uint32_t g[16], w[16];
+      if (skip) {
+#pragma unroll
+        for (int x = 0; x < 16; ++x) g[x] = w[x] = 0u;
+      } else {
+        uint32_t s[16], d[16];
+        tmem_ld16(lane_base + C::colS + 32 * kq, s);
+        tmem_ld16(lane_base + C::colP + 32 * kq, d);
+        tmem_wait_ld();
+        grad_block<0, true>(s, d, [&](int c) { return __shfl_sync(0xffffffffu, dDl, c); },
+                            [&](int c) { return !part || c >= lane; }, g, w);
+        tmem_ld16(lane_base + C::colS + 32 * kq + 16, s);
+        tmem_ld16(lane_base + C::colP + 32 * kq + 16, d);
+        tmem_wait_ld();
+        grad_block<1, true>(s, d, [&](int c) { return __shfl_sync(0xffffffffu, dDl, 16 + c); },
+                            [&](int c) { return !part || 16 + c >= lane; }, g, w);
+      }
+      tc_fence_before();
+      mbar_arrive(s_read);
+      // the operand buffers are read by the previous query tile's MMAs
+      if (n > 0 && !mbar_wait(w_free, (n - 1) & 1, env)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      tmem_st16(lane_base + C::colA(0) + 16 * kq, w);
+      tmem_st16(lane_base + C::colA(1) + 16 * kq, g);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(p_full);
+    }
+    // epilogue: dV (64 columns: 16 per key quarter warp) and dK (p columns,
+    // warps of key quarter 0) -> bf16, rows < T
+    if (ok && mbar_wait(done, 0, env)) {
+      tc_fence_after();
+      auto store16 = [&](__nv_bfloat16* dst_row, uint32_t col) {
+        uint32_t r[16];
+        tmem_ld16(lane_base + col, r);
+        tmem_wait_ld();
+        if (row < T) {
+          uint4* dst = reinterpret_cast<uint4*>(dst_row);
+          dst[0] = make_uint4(pack_bf16x2(__uint_as_float(r[0]), __uint_as_float(r[1])),
+                              pack_bf16x2(__uint_as_float(r[2]), __uint_as_float(r[3])),
+                              pack_bf16x2(__uint_as_float(r[4]), __uint_as_float(r[5])),
+                              pack_bf16x2(__uint_as_float(r[6]), __uint_as_float(r[7])));
+          dst[1] = make_uint4(pack_bf16x2(__uint_as_float(r[8]), __uint_as_float(r[9])),
+                              pack_bf16x2(__uint_as_float(r[10]), __uint_as_float(r[11])),
+                              pack_bf16x2(__uint_as_float(r[12]), __uint_as_float(r[13])),
+                              pack_bf16x2(__uint_as_float(r[14]), __uint_as_float(r[15])));
+        }
+      };
+      const size_t r0 = (size_t)bh * T + (row < T ? row : 0);
+      store16(dv + r0 * kBwDV + 16 * kq, C::colAcc + 16 * kq);
+      if (kq == 0) {
+#pragma unroll
+        for (int c0 = 0; c0 < p; c0 += 16) store16(dk + r0 * p + c0, C::colAcc + kBwDV + c0);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kBwTmemCols);
+  }
+}
+
+template <int p>
+static cudaError_t launch_bwd_t(const void* q, const void* k, const void* v, const void* o, const float* D,
+                                const void* dO, void* dq, void* dk, void* dv, int BH, int T, void* ws,
+                                const WaitCtl& wc, cudaStream_t st) {
+  __nv_bfloat16* dN = static_cast<__nv_bfloat16*>(ws);
+  float* dD = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + (size_t)BH * T * kBwDV * 2);
+  const long long rows = (long long)BH * T;
+  bwd_prep_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(dO),
+                                                                 static_cast<const __nv_bfloat16*>(o), D, dN, dD, rows);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  CUtensorMap tq, tk, tv, tdn;
+  if (!make_tmap_bf16(&tq, q, p, T, BH, kBw) || !make_tmap_bf16(&tk, k, p, T, BH, kBw) ||
+      !make_tmap_bf16(&tv, v, kBwDV, T, BH, kBw) || !make_tmap_bf16(&tdn, dN, kBwDV, T, BH, kBw))
+    return cudaErrorInvalidValue;
+  const dim3 grid((T + kBw - 1) / kBw, BH);
+  auto kq = bwd_dq_kernel<p>;
+  auto kkv = bwd_dkdv_kernel<p>;
+  if ((e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, DqSmem<p>::kBytes)) != cudaSuccess ||
+      (e = cudaFuncSetAttribute(kkv, cudaFuncAttributeMaxDynamicSharedMemorySize, DkvSmem<p>::kBytes)) != cudaSuccess)
+    return e;
+  kq<<<grid, kBwThreads, DqSmem<p>::kBytes, st>>>(tq, tk, tv, tdn, dD, static_cast<__nv_bfloat16*>(dq), T, wc);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  kkv<<<grid, kBwThreads, DkvSmem<p>::kBytes, st>>>(tq, tk, tv, tdn, dD, static_cast<__nv_bfloat16*>(dk),
+                                                     static_cast<__nv_bfloat16*>(dv), T, wc);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t flash_bwd_workspace_bytes(int BH, int T, int dv) {
+  return (size_t)BH * T * dv * 2 + (size_t)BH * T * 4;
+}
+
+cudaError_t launch_flash_bwd_sm100(const void* q, const void* k, const void* v, const void* o, const float* D,
+                                  const void* dO, void* dq, void* dk, void* dv, int BH, int T, int p, void* ws,
+                                  const WaitCtl& wc, cudaStream_t st) {
+  if (p == 16) return launch_bwd_t<16>(q, k, v, o, D, dO, dq, dk, dv, BH, T, ws, wc, st);
+  if (p == 32) return launch_bwd_t<32>(q, k, v, o, D, dO, dq, dk, dv, BH, T, ws, wc, st);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace kata

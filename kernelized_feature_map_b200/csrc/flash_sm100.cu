@@ -94,7 +94,7 @@ template <int p, int DV>
 __global__ void __launch_bounds__(kThreads, 1)
     flash_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o, int T, int BH,
-                     int H, int bthd, WaitCtl wc) {
+                     int H, int bthd, float* __restrict__ D_out, WaitCtl wc) {
   using Cfg = FlashCfg<p, DV>;
   constexpr int kStages = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -404,6 +404,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the box: for DV = 64 the 64-byte rows are 64B-swizzled (16-byte chunk
       // e at e ^ ((lane / 2) % 4)), for DV = 16 the 16-byte rows are plain
       const float D = __uint_as_float(dbits);
+      // the denominator of each row, for the backward pass (optional)
+      if (D_out != nullptr && h == 0 && row0 + lane < T) D_out[(size_t)bh * T + row0 + lane] = D;
       const float inv = D > 0.f ? 1.f / D : 0.f;
       const uint64_t inv2 = f32x2(__float_as_uint(inv), __float_as_uint(inv));
       auto scaled = [&](int k) {
@@ -526,7 +528,7 @@ bool make_tmap_bf16_4d(CUtensorMap* map, const void* base, int inner, int T, int
 
 template <int p, int DV>
 static cudaError_t launch_flash_t(const void* q, const void* k, const void* v, void* o, int B, int H, int T, bool bthd,
-                                  const WaitCtl& wc, cudaStream_t st) {
+                                  float* D_out, const WaitCtl& wc, cudaStream_t st) {
   using Cfg = FlashCfg<p, DV>;
   const int BH = B * H;
   CUtensorMap tq, tk, tv, to;
@@ -547,16 +549,16 @@ static cudaError_t launch_flash_t(const void* q, const void* k, const void* v, v
   }
   const long items = (long)((T + kBM * kNQ - 1) / (kBM * kNQ)) * BH;
   const int grid = (int)(items < num_sms ? items : num_sms);
-  kern<<<grid, kThreads, Cfg::kSmemBytes, st>>>(tq, tk, tv, to, T, BH, H, bthd ? 1 : 0, wc);
+  kern<<<grid, kThreads, Cfg::kSmemBytes, st>>>(tq, tk, tv, to, T, BH, H, bthd ? 1 : 0, D_out, wc);
   return cudaGetLastError();
 }
 
 cudaError_t launch_flash_sm100(const void* q, const void* k, const void* v, void* o, int B, int H, int T, int p, int dv,
-                               bool bthd, const WaitCtl& wc, cudaStream_t st) {
-  if (p == 16 && dv == 64) return launch_flash_t<16, 64>(q, k, v, o, B, H, T, bthd, wc, st);
-  if (p == 16 && dv == 16) return launch_flash_t<16, 16>(q, k, v, o, B, H, T, bthd, wc, st);
-  if (p == 32 && dv == 64) return launch_flash_t<32, 64>(q, k, v, o, B, H, T, bthd, wc, st);
-  if (p == 32 && dv == 16) return launch_flash_t<32, 16>(q, k, v, o, B, H, T, bthd, wc, st);
+                               bool bthd, float* D_out, const WaitCtl& wc, cudaStream_t st) {
+  if (p == 16 && dv == 64) return launch_flash_t<16, 64>(q, k, v, o, B, H, T, bthd, D_out, wc, st);
+  if (p == 16 && dv == 16) return launch_flash_t<16, 16>(q, k, v, o, B, H, T, bthd, D_out, wc, st);
+  if (p == 32 && dv == 64) return launch_flash_t<32, 64>(q, k, v, o, B, H, T, bthd, D_out, wc, st);
+  if (p == 32 && dv == 16) return launch_flash_t<32, 16>(q, k, v, o, B, H, T, bthd, D_out, wc, st);
   return cudaErrorInvalidValue;
 }
 

@@ -149,7 +149,7 @@ KATA_API kata_status_t kata_fwd_quadratic(const void* q, const void* k, const vo
   if (!q || !k || !v || !o) return KATA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return KATA_ERR_MISALIGNED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (dtype == KATA_BF16) return from_cuda(launch_flash_sm100(q, k, v, o, B, H, T, p, dv, false, wait_ctl(), st));
+  if (dtype == KATA_BF16) return from_cuda(launch_flash_sm100(q, k, v, o, B, H, T, p, dv, false, nullptr, wait_ctl(), st));
   return from_cuda(launch_quadratic_simt(q, k, v, o, B * H, T, p, dv, dtype, st));
 }
 
@@ -247,6 +247,47 @@ KATA_API kata_status_t kata_decode_step(const void* q, const void* k, const void
   return from_cuda(launch_decode(q, k, v, o, S, z, B * H, p, 1, dv, dtype, static_cast<cudaStream_t>(stream)));
 }
 
+static kata_status_t check_train(int B, int H, int T, int p, int dv, kata_dtype_t dt) {
+  kata_status_t s = check_common(B, H, T, p, dv, dt);
+  if (s != KATA_OK) return s;
+  if (dt != KATA_BF16 || dv != 64) return KATA_ERR_UNSUPPORTED;
+  return KATA_OK;
+}
+
+KATA_API kata_status_t kata_fwd_quadratic_train(const void* q, const void* k, const void* v, void* o, float* D,
+                                                int B, int H, int T, int p, int dv, kata_dtype_t dtype,
+                                                void* stream) {
+  kata_status_t s = check_train(B, H, T, p, dv, dtype);
+  if (s != KATA_OK) return s;
+  if (T == 0) return KATA_OK;
+  if (!q || !k || !v || !o || !D) return KATA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(D)) return KATA_ERR_MISALIGNED;
+  return from_cuda(
+      launch_flash_sm100(q, k, v, o, B, H, T, p, dv, false, D, wait_ctl(), static_cast<cudaStream_t>(stream)));
+}
+
+KATA_API size_t kata_bwd_quadratic_workspace_size(int B, int H, int T, int p, int dv, kata_dtype_t dtype) {
+  if (check_train(B, H, T, p, dv, dtype) != KATA_OK || T == 0) return 0;
+  return flash_bwd_workspace_bytes(B * H, T, dv);
+}
+
+KATA_API kata_status_t kata_bwd_quadratic(const void* q, const void* k, const void* v, const void* o, const float* D,
+                                          const void* dO, void* dq, void* dk, void* dv, int B, int H, int T, int p,
+                                          int dv_width, kata_dtype_t dtype, void* workspace, size_t workspace_bytes,
+                                          void* stream) {
+  kata_status_t s = check_train(B, H, T, p, dv_width, dtype);
+  if (s != KATA_OK) return s;
+  if (T == 0) return KATA_OK;
+  for (const void* ptr : {q, k, v, o, (const void*)D, dO, (const void*)dq, (const void*)dk, (const void*)dv})
+    if (!ptr) return KATA_ERR_INVALID_ARG;
+  for (const void* ptr : {q, k, v, o, (const void*)D, dO, (const void*)dq, (const void*)dk, (const void*)dv})
+    if (!aligned16(ptr)) return KATA_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < flash_bwd_workspace_bytes(B * H, T, dv_width)) return KATA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return KATA_ERR_MISALIGNED;
+  return from_cuda(launch_flash_bwd_sm100(q, k, v, o, D, dO, dq, dk, dv, B * H, T, p, workspace, wait_ctl(),
+                                          static_cast<cudaStream_t>(stream)));
+}
+
 // Shape checks shared by the KATA-Mg entry points: p = d / groups.
 static kata_status_t check_mg(int B, int H, int T, int d, int groups, int dv, kata_dtype_t dt, int* p_out) {
   if (groups < 1 || d < 1 || d % groups != 0) return KATA_ERR_INVALID_ARG;
@@ -274,7 +315,7 @@ KATA_API kata_status_t kata_fwd_mg_quadratic(const void* q, const void* k, const
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (flash_mg_sm100_supports(p, groups, dv))
     return from_cuda(launch_flash_mg_sm100(q, k, v, o, B, H, T, p, groups, bthd, wait_ctl(), st));
-  return from_cuda(launch_flash_sm100(q, k, v, o, B, H, T, p, dv, bthd, wait_ctl(), st));
+  return from_cuda(launch_flash_sm100(q, k, v, o, B, H, T, p, dv, bthd, nullptr, wait_ctl(), st));
 }
 
 KATA_API kata_status_t kata_decode_step_mg(const void* q, const void* k, const void* v, void* o, float* S, float* z,

@@ -65,9 +65,18 @@ cudaError_t launch_chunk_readout_simt(const void* q, const void* k, const void* 
 
 // flash_sm100.cu -- tcgen05 flash-style forward (bf16 inputs), one PSD
 // factor of width p per head; bthd selects the [B,T,H,*] layout of q, k, v
-// and o instead of [B,H,T,*].
+// and o instead of [B,H,T,*].  D_out (nullable, fp32 [B*H, T]) receives each
+// row's denominator.
 cudaError_t launch_flash_sm100(const void* q, const void* k, const void* v, void* o, int B, int H, int T, int p, int dv,
-                               bool bthd, const WaitCtl& wc, cudaStream_t st);
+                               bool bthd, float* D_out, const WaitCtl& wc, cudaStream_t st);
+
+// flash_bwd_sm100.cu -- backward pass of the flash-style forward (bf16,
+// p in {16, 32}, dv = 64, [B*H, T, *] layouts); D is the forward's
+// denominator [B*H, T] fp32; ws holds flash_bwd_workspace_bytes().
+size_t flash_bwd_workspace_bytes(int BH, int T, int dv);
+cudaError_t launch_flash_bwd_sm100(const void* q, const void* k, const void* v, const void* o, const float* D,
+                                   const void* dO, void* dq, void* dk, void* dv, int BH, int T, int p, void* ws,
+                                   const WaitCtl& wc, cudaStream_t st);
 
 // flash_mg_sm100.cu -- tcgen05 flash-style KATA-Mg forward (bf16 inputs,
 // dv = 64) with `groups` PSD factors of width p per head.

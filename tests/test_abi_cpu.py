@@ -44,7 +44,7 @@ def test_only_abi_symbols_are_exported():
 
 
 def test_status_strings_and_version(L):
-    assert _abi.kata_abi_version() == 10100
+    assert _abi.kata_abi_version() == 10200
     for code, name in [(0, "KATA_OK"), (2, "KATA_ERR_UNSUPPORTED"), (6, "KATA_ERR_TIMEOUT")]:
         assert _abi.status_string(code) == name
     assert _abi.status_string(99) == "KATA_ERR_UNKNOWN"
@@ -142,3 +142,26 @@ def test_mg_argument_errors_before_launch(L):
     assert md(a, b, c, d, S, z, 1, 1, 48, 4, 64, 1, st) == _abi.KATA_ERR_UNSUPPORTED      # p = 12
     assert md(a, b, c, d, S, z, 1, 1, 64, 5, 64, 1, st) == _abi.KATA_ERR_INVALID_ARG
     assert md(a, b, c, d, _fake(0x70004), z, 1, 1, 64, 2, 64, 1, st) == _abi.KATA_ERR_MISALIGNED
+
+
+def test_training_entry_points_reject_bad_arguments(L):
+    a, b, c, d = _fake(0x10000), _fake(0x20000), _fake(0x30000), _fake(0x40000)
+    D, dO, gq, gk, gv, ws = (_fake(0x50000 + 0x10000 * i) for i in range(6))
+    st = VP(0)
+    f = L.kata_fwd_quadratic_train  # q k v o D B H T p dv dtype stream
+    assert f(a, b, c, d, D, 1, 1, 16, 16, 64, 0, st) == _abi.KATA_ERR_UNSUPPORTED   # fp32
+    assert f(a, b, c, d, D, 1, 1, 16, 16, 16, 1, st) == _abi.KATA_ERR_UNSUPPORTED   # dv 16
+    assert f(a, b, c, d, None, 1, 1, 16, 16, 64, 1, st) == _abi.KATA_ERR_INVALID_ARG
+    assert f(a, b, c, d, _fake(0x50004), 1, 1, 16, 16, 64, 1, st) == _abi.KATA_ERR_MISALIGNED
+    assert f(a, b, c, d, D, 1, 1, 0, 16, 64, 1, st) == _abi.KATA_OK
+    ws_size = _abi.lib().kata_bwd_quadratic_workspace_size
+    assert ws_size(2, 3, 100, 16, 64, 1) == 2 * 3 * 100 * (64 * 2 + 4)
+    assert ws_size(2, 3, 100, 16, 64, 0) == 0 and ws_size(1, 1, 0, 16, 64, 1) == 0
+    g = L.kata_bwd_quadratic  # q k v o D dO dq dk dv B H T p dv dtype ws bytes stream
+    n = 1 * 1 * 16 * (64 * 2 + 4)
+    assert g(a, b, c, d, D, dO, gq, gk, gv, 1, 1, 16, 24, 64, 1, ws, n, st) == _abi.KATA_ERR_UNSUPPORTED
+    assert g(a, b, c, d, D, None, gq, gk, gv, 1, 1, 16, 16, 64, 1, ws, n, st) == _abi.KATA_ERR_INVALID_ARG
+    assert g(a, b, c, d, D, dO, gq, gk, gv, 1, 1, 16, 16, 64, 1, ws, n - 1, st) == _abi.KATA_ERR_WORKSPACE
+    assert g(a, b, c, d, D, dO, gq, gk, gv, 1, 1, 16, 16, 64, 1, None, n, st) == _abi.KATA_ERR_WORKSPACE
+    assert g(a, b, c, d, D, dO, gq, gk, _fake(0x90008), 1, 1, 16, 16, 64, 1, ws, n, st) == _abi.KATA_ERR_MISALIGNED
+    assert g(a, b, c, d, D, dO, gq, gk, gv, 1, 1, 0, 16, 64, 1, None, 0, st) == _abi.KATA_OK

@@ -1,0 +1,125 @@
+"""GPU parity of the training entry points against the fp64 gradient oracle
+(oracle/backward.py, pinned by finite differences): the forward that saves
+the denominators, and the backward pass.
+
+Gate for the gradients (bf16 inputs, fp32 accumulation): per (b,h) and per
+tensor, ||g - g_ref||_F / ||g_ref||_F <= 2e-2.  The bf16 operands of the
+backward MMAs (q, k, v, dO/D, the squares and dS) each carry one rounding of
+relative size 2^-9; summed over a row with mixed signs, the resulting error
+stays a small multiple of that, and a norm-relative gate (rather than an
+elementwise one) is used because dq and dk are sums whose terms cancel
+(sum_s w_ts dw_ts = 0 for every t), so single entries can be small.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import workloads
+from helpers import TOL, to_dev, to_np
+from oracle import backward as obw
+
+pytestmark = pytest.mark.gpu
+GRAD_TOL = 2e-2
+
+
+@pytest.fixture(scope="module")
+def kata():
+    import torch
+    import kernelized_feature_map_b200 as K
+    from kernelized_feature_map_b200 import build
+    build.build()
+    assert torch.cuda.is_available()
+    return K
+
+
+def _grad_err(got, ref):
+    got = np.asarray(got, np.float64).reshape(ref.shape[0] * ref.shape[1], -1)
+    ref = np.asarray(ref, np.float64).reshape(got.shape)
+    num = np.linalg.norm(got - ref, axis=1)
+    den = np.maximum(np.linalg.norm(ref, axis=1), 1e-30)
+    return float((num / den).max())
+
+
+def _dO(shape, seed):
+    return workloads.round_bf16(np.random.default_rng(seed).standard_normal(shape).astype(np.float32))
+
+
+def _run(K, q, k, v, dO):
+    import torch
+    qd, kd, vd = to_dev(q, "bf16"), to_dev(k, "bf16"), to_dev(v, "bf16")
+    o, D = K.kata_fwd_quadratic_train(qd, kd, vd)
+    dq, dk, dv = K.kata_bwd_quadratic(qd, kd, vd, o, D, to_dev(dO, "bf16"))
+    torch.cuda.synchronize()
+    assert K.kata_get_status() == 0
+    return to_np(o), D.cpu().numpy(), to_np(dq), to_np(dk), to_np(dv)
+
+
+SHAPES = [
+    # B, H, T, p -- several 128-row tiles with a ragged tail, a single tile,
+    # an exact tile, and p = 32
+    (2, 2, 1000, 16),
+    (1, 1, 129, 16),
+    (1, 2, 128, 16),
+    (1, 3, 777, 32),
+]
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+def test_backward_matches_oracle(kata, shape):
+    B, H, T, p = shape
+    q, k, v = workloads.normal_qkv(B, H, T, p, 64, seed=400 + T + p, dtype="bf16")
+    dO = _dO(v.shape, 401 + T)
+    o, D, dq, dk, dv = _run(kata, q, k, v, dO)
+    o_ref, D_ref = obw.forward_with_d(q, k, v)
+    np.testing.assert_allclose(D, D_ref, rtol=1e-2, atol=1e-30)
+    gq, gk, gv = obw.backward(q, k, v, dO)
+    errs = {n: _grad_err(g, r) for n, g, r in (("dq", dq, gq), ("dk", dk, gk), ("dv", dv, gv))}
+    assert max(errs.values()) <= GRAD_TOL, errs
+
+
+def test_train_forward_is_the_flash_forward(kata):
+    import torch
+    q, k, v = workloads.normal_qkv(2, 3, 600, 16, 64, seed=410, dtype="bf16")
+    qd, kd, vd = to_dev(q, "bf16"), to_dev(k, "bf16"), to_dev(v, "bf16")
+    o1 = kata.kata_fwd_quadratic(qd, kd, vd)
+    o2, _ = kata.kata_fwd_quadratic_train(qd, kd, vd)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2)
+
+
+def test_zero_denominator_rows_pass_no_gradient(kata):
+    q, k, v = workloads.normal_qkv(1, 2, 300, 16, 64, seed=420, dtype="bf16")
+    q[:, :, [0, 150, 299]] = 0.0
+    dO = _dO(v.shape, 421)
+    o, D, dq, dk, dv = _run(kata, q, k, v, dO)
+    assert np.all(D[:, :, [0, 150, 299]] == 0.0)
+    assert np.all(dq[:, :, [0, 150, 299]] == 0.0)
+    gq, gk, gv = obw.backward(q, k, v, dO)
+    assert max(_grad_err(dq, gq), _grad_err(dk, gk), _grad_err(dv, gv)) <= GRAD_TOL
+
+
+def test_autograd_wrapper(kata):
+    import torch
+    q, k, v = workloads.normal_qkv(1, 2, 256, 16, 64, seed=430, dtype="bf16")
+    dO = _dO(v.shape, 431)
+    qd, kd, vd = (to_dev(x, "bf16").requires_grad_(True) for x in (q, k, v))
+    o = kata.kata_attention(qd, kd, vd)
+    o.backward(to_dev(dO, "bf16"))
+    torch.cuda.synchronize()
+    _, _, dq, dk, dv = _run(kata, q, k, v, dO)
+    assert np.array_equal(to_np(qd.grad), dq) and np.array_equal(to_np(kd.grad), dk)
+    assert np.array_equal(to_np(vd.grad), dv)
+
+
+def test_backward_full_size_sampled_heads(kata):
+    """The training workload at full size (B8 H16 T2048 p16 dv64); the
+    oracle's T x T gradient is computed for a few heads and compared whole."""
+    cfg = workloads.CONFIGS["layer340m_ctx2k"]
+    q, k, v = workloads.make_inputs(cfg)
+    dO = _dO(v.shape, 440)
+    _, _, dq, dk, dv = _run(kata, q, k, v, dO)
+    for (b, h) in [(0, 0), (3, 7), (7, 15)]:
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        gq, gk, gv = obw.backward(q[sl], k[sl], v[sl], dO[sl])
+        errs = (_grad_err(dq[sl], gq), _grad_err(dk[sl], gk), _grad_err(dv[sl], gv))
+        assert max(errs) <= GRAD_TOL, (b, h, errs)
