@@ -383,6 +383,7 @@ def run_ours(args, rank, world, local_rank):
         if args.sweep:
             long["sweep"], long["recall"] = run_sweep(args, K, torch, dev, stream, flush)
             long["mg"] = run_mg(args, K, torch, dev, stream, flush)
+            long["train"] = run_train(args, K, torch, dev, stream, flush)
 
     status = K.kata_get_status()
     return dict(step_ms=step_ms, eager_step_ms=eager_step_ms, graph=bool(args.graph), path_ms=path_ms.tolist(),
@@ -540,6 +541,33 @@ def run_mg(args, K, torch, dev, stream, flush):
         out["decode_mg%d_b64" % g] = dict(B=B, H=H, d=d, groups=g, dv=dv, P=P, ms=ms)
         del q, k, v, S, z, o
     return out
+
+
+def run_train(args, K, torch, dev, stream, flush):
+    """Training step of the flash path on the bench workload's shape (B8 H16
+    T2048 p16 dv64, bf16): the forward that saves the denominators, then the
+    backward pass for an upstream gradient; device-drawn inputs."""
+    bf = torch.bfloat16
+    B, H, T, p, dv = 8, 16, 2048, 16, 64
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(99)
+    q = torch.randn((B, H, T, p), generator=gen, device=dev)
+    k = torch.randn((B, H, T, p), generator=gen, device=dev)
+    q = (q / q.norm(dim=-1, keepdim=True)).to(bf)
+    k = (k / k.norm(dim=-1, keepdim=True)).to(bf)
+    v = torch.randn((B, H, T, dv), generator=gen, device=dev).to(bf)
+    dO = torch.randn((B, H, T, dv), generator=gen, device=dev).to(bf)
+    o, D = K.kata_fwd_quadratic_train(q, k, v)
+    ws = torch.empty(max(256, int(K.lib().kata_bwd_quadratic_workspace_size(B, H, T, p, dv, 1))), dtype=torch.uint8,
+                     device=dev)
+    fwd_ms = _time_call(lambda: K.kata_fwd_quadratic_train(q, k, v, o=o, D=D), flush, stream, 10, 3)
+    bwd_ms = _time_call(lambda: K.kata_bwd_quadratic(q, k, v, o, D, dO, workspace=ws), flush, stream, 10, 3)
+
+    def step():
+        K.kata_fwd_quadratic_train(q, k, v, o=o, D=D)
+        K.kata_bwd_quadratic(q, k, v, o, D, dO, workspace=ws)
+    step_ms = _time_call(step, flush, stream, 10, 3)
+    return dict(B=B, H=H, T=T, p=p, dv=dv, fwd_ms=fwd_ms, bwd_ms=bwd_ms, step_ms=step_ms)
 
 
 # ---------------------------------------------------------------------------
@@ -742,6 +770,17 @@ def report(args, res, step_ms, e2e_ms, world):
                         "ms": m["ms"], "tokens_per_s": m["B"] * m["T"] / (m["ms"] * 1e-3),
                         "tensor_frac": flash_flops(m["B"] * m["H"], m["T"], m["d"], m["dv"]) / (m["ms"] * 1e-3)
                         / 1e12 / peaks["bf16_tflops"]}
+        if "train" in lg:
+            tr = lg["train"]
+            pairs = tr["B"] * tr["H"] * tr["T"] * (tr["T"] + 1) / 2
+            bwd_flops = pairs * 2 * (3 * tr["p"] + 2 * tr["dv"])
+            line["train"] = {
+                "workload": "training step of the flash path B=%d H=%d T=%d p=%d dv=%d bf16 (forward saving D, then "
+                            "backward)" % (tr["B"], tr["H"], tr["T"], tr["p"], tr["dv"]),
+                "step_ms": tr["step_ms"], "tokens_per_s": tr["B"] * tr["T"] / (tr["step_ms"] * 1e-3),
+                "fwd_ms": tr["fwd_ms"], "bwd_ms": tr["bwd_ms"],
+                "bwd_tensor_frac": bwd_flops / (tr["bwd_ms"] * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                "bwd_algorithmic": "2(3p+2dv) flops per causal pair: S, dP, dV, dQ, dK"}
     if args.cpu_baseline and world == 1:
         cb = time_oracle(cfg)
         line["cpu_baseline"] = {"value": cb["value"], "unit": UNIT, "cores": cb["cores"], "kind": "oracle",

@@ -8,8 +8,9 @@ that launches the kernel of interest a known number of times:
 Inputs are drawn on the device (q, k L2-normalised N(0, 1) per token, v
 N(0, 1), bf16); the program prints the call's status and nothing is timed.
 Paths: ``quadratic`` (kata_fwd_quadratic, q/k width d), ``chunked``
-(kata_fwd_chunked), ``mg`` (kata_fwd_mg_quadratic with --groups) and
-``decode`` (kata_decode_step_mg on a zero state, T ignored).
+(kata_fwd_chunked), ``mg`` (kata_fwd_mg_quadratic with --groups),
+``decode`` (kata_decode_step_mg on a zero state, T ignored) and ``train``
+(kata_fwd_quadratic_train then kata_bwd_quadratic for a random dO).
 """
 from __future__ import annotations
 
@@ -22,7 +23,7 @@ def main(argv=None):
     import kernelized_feature_map_b200 as K
 
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
-    ap.add_argument("--path", choices=["quadratic", "chunked", "mg", "decode"], required=True)
+    ap.add_argument("--path", choices=["quadratic", "chunked", "mg", "decode", "train"], required=True)
     ap.add_argument("--B", type=int, default=8)
     ap.add_argument("--H", type=int, default=16)
     ap.add_argument("--T", type=int, default=2048)
@@ -62,6 +63,13 @@ def main(argv=None):
             ap.error("--layout bthd is for --path mg")
         elif a.path == "quadratic":
             call = lambda: K.kata_fwd_quadratic(q, k, v, o=o)  # noqa: E731
+        elif a.path == "train":
+            dO = torch.randn(v.shape, generator=gen, device=dev).to(bf)
+            D = torch.empty((a.B, a.H, a.T), dtype=torch.float32, device=dev)
+
+            def call():
+                K.kata_fwd_quadratic_train(q, k, v, o=o, D=D)
+                K.kata_bwd_quadratic(q, k, v, o, D, dO)
         else:
             ws = torch.empty(max(256, K.kata_fwd_chunked_workspace_size(a.B, a.H, a.T, a.d, a.dv, a.C, bf)),
                              dtype=torch.uint8, device=dev)
