@@ -17,7 +17,7 @@
 //                        S = Q K_j^T and dP = dN V_j^T on the tensor core,
 //                        dS = 2 S (dP + dD) in the weight warps, then
 //                        dQ += dS K_j with dS read from TMEM;
-//   3. bwd_dkdv_kernel   one CTA per 128-row key tile: per query tile i,
+//   3. bwd_dkdv_kernel   persistent, items of one 128-row key tile: per query tile i,
 //                        S^T = K Q_i^T and dP^T = V dN_i^T, W^T = (S^T)^2 and
 //                        dS^T in the weight warps, then dV += W^T dN_i and
 //                        dK += dS^T Q_i.
@@ -318,17 +318,31 @@ __global__ void __launch_bounds__(kBwThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// 3. dK, dV: CTA (key tile j, head bh), query tiles i = j..n_tiles-1
+// 3. dK, dV: persistent CTAs over items (key tile j, head bh), heaviest
+//    (j = 0) first; per item, query tiles i = j..n_tiles-1
 // ---------------------------------------------------------------------------
+// 16 fp32 values -> 16 bf16 at dst (32 bytes, 16-byte aligned)
+__device__ __forceinline__ void store_row16(__nv_bfloat16* dst_row, const uint32_t (&r)[16]) {
+  uint4* dst = reinterpret_cast<uint4*>(dst_row);
+  dst[0] = make_uint4(pack_bf16x2(__uint_as_float(r[0]), __uint_as_float(r[1])),
+                      pack_bf16x2(__uint_as_float(r[2]), __uint_as_float(r[3])),
+                      pack_bf16x2(__uint_as_float(r[4]), __uint_as_float(r[5])),
+                      pack_bf16x2(__uint_as_float(r[6]), __uint_as_float(r[7])));
+  dst[1] = make_uint4(pack_bf16x2(__uint_as_float(r[8]), __uint_as_float(r[9])),
+                      pack_bf16x2(__uint_as_float(r[10]), __uint_as_float(r[11])),
+                      pack_bf16x2(__uint_as_float(r[12]), __uint_as_float(r[13])),
+                      pack_bf16x2(__uint_as_float(r[14]), __uint_as_float(r[15])));
+}
+
 template <int p>
 struct DkvSmem {
   using C = BwCfg<p>;
-  static constexpr int offV = 0;                                        // V_j (SW128)
-  static constexpr int offK = offV + C::kVBytes;                        // K_j
-  static constexpr int offDN = (offK + C::kQKBytes + 1023) / 1024 * 1024;  // ring of dN_i
+  static constexpr int offV = 0;                                        // 2 buffers of V_j (SW128)
+  static constexpr int offK = offV + 2 * C::kVBytes;                    // 2 buffers of K_j
+  static constexpr int offDN = (offK + 2 * C::kQKBytes + 1023) / 1024 * 1024;  // ring of dN_i
   static constexpr int offQ = offDN + kBwStages * C::kVBytes;           // ring of Q_i
   static constexpr int offBar = (offQ + kBwStages * C::kQKBytes + 1023) / 1024 * 1024;
-  static constexpr int kBars = 1 + 2 * kBwStages + 5;
+  static constexpr int kBars = 4 + 2 * kBwStages + 7;
   static constexpr int offMisc = offBar + kBars * 8;
   static constexpr int kBytes = offMisc + 16 + 1024;
 };
@@ -338,31 +352,41 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_dn,
                     const float* __restrict__ dD, __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
-                    int T, WaitCtl wc) {
+                    int T, int BH, WaitCtl wc) {
   using C = BwCfg<p>;
   using L = DkvSmem<p>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::offBar);
-  uint64_t* kv_full = bars;                     // K_j and V_j landed
-  uint64_t* q_full = kv_full + 1;               // [kBwStages] Q_i and dN_i
+  uint64_t* kv_full = bars;                     // [2] K_j and V_j landed
+  uint64_t* kv_empty = kv_full + 2;             // [2]
+  uint64_t* q_full = kv_empty + 2;              // [kBwStages] Q_i and dN_i
   uint64_t* q_empty = q_full + kBwStages;       // [kBwStages]
   uint64_t* s_full = q_empty + kBwStages;       // S^T and dP^T of a query tile in TMEM
   uint64_t* s_read = s_full + 1;                // ... loaded by the weight warps (512)
   uint64_t* p_full = s_read + 1;                // W^T and dS^T written (512)
   uint64_t* w_free = p_full + 1;                // ... read by the dV / dK MMAs
-  uint64_t* done = w_free + 1;
+  uint64_t* acc_full = w_free + 1;              // an item's dV, dK complete
+  uint64_t* acc_free = acc_full + 1;            // ... read by the epilogue (512)
+  uint64_t* done = acc_free + 1;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::offMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::offMisc + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_tiles = (T + kBw - 1) / kBw;
-  const int tile = (int)blockIdx.x;             // key tile; tile 0 has the most query tiles
-  const int bh = blockIdx.y;
-  const int cnt = n_tiles - tile;               // query tiles tile .. n_tiles - 1
+  const int n_items = n_tiles * BH;
+  // item it: key tile it / BH (tile 0 has the most query tiles), head it % BH;
+  // the r-th item of this CTA in snake order over the CTAs
+  auto my_item = [&](int r) {
+    const int it = r * (int)gridDim.x + ((r & 1) ? (int)gridDim.x - 1 - (int)blockIdx.x : (int)blockIdx.x);
+    return it < n_items ? it : -1;
+  };
 
   if (threadIdx.x == 0) {
-    mbar_init(kv_full, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(kv_full + b, 1);
+      mbar_init(kv_empty + b, 1);
+    }
     for (int s = 0; s < kBwStages; ++s) {
       mbar_init(q_full + s, 1);
       mbar_init(q_empty + s, 1);
@@ -371,6 +395,8 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     mbar_init(s_read, 512);
     mbar_init(p_full, 512);
     mbar_init(w_free, 1);
+    mbar_init(acc_full, 1);
+    mbar_init(acc_free, 512);
     mbar_init(done, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -389,21 +415,29 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
       prefetch_tmap(&tm_dn);
-      mbar_arrive_expect_tx(kv_full, C::kVBytes + C::kQKBytes);
-      tma_load_3d(smem + L::offV, &tm_v, kv_full, 0, tile * kBw, bh);
-      tma_load_3d(smem + L::offK, &tm_k, kv_full, 0, tile * kBw, bh);
-      int issued = 0;
-      for (int n = 0; n < cnt; ++n) {
-        const int st = n % kBwStages, i = tile + n;
-        if (!mbar_wait(q_empty + st, ((n / kBwStages) & 1) ^ 1, env)) break;
-        mbar_arrive_expect_tx(q_full + st, C::kVBytes + C::kQKBytes);
-        tma_load_3d(smem + L::offDN + st * C::kVBytes, &tm_dn, q_full + st, 0, i * kBw, bh);
-        tma_load_3d(smem + L::offQ + st * C::kQKBytes, &tm_q, q_full + st, 0, i * kBw, bh);
-        ++issued;
+      int nq = 0;
+      long rg = 0;  // query tiles loaded (ring position)
+      bool ok = true;
+      for (int it = my_item(nq); ok && it >= 0; it = my_item(++nq)) {
+        const int tile = it / BH, bh = it % BH, kb = nq & 1;
+        if (!mbar_wait(kv_empty + kb, ((nq >> 1) & 1) ^ 1, env)) break;
+        mbar_arrive_expect_tx(kv_full + kb, C::kVBytes + C::kQKBytes);
+        tma_load_3d(smem + L::offV + kb * C::kVBytes, &tm_v, kv_full + kb, 0, tile * kBw, bh);
+        tma_load_3d(smem + L::offK + kb * C::kQKBytes, &tm_k, kv_full + kb, 0, tile * kBw, bh);
+        for (int i = tile; i < n_tiles; ++i, ++rg) {
+          const int st = (int)(rg % kBwStages);
+          if (!mbar_wait(q_empty + st, (int)((rg / kBwStages) & 1) ^ 1, env)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(q_full + st, C::kVBytes + C::kQKBytes);
+          tma_load_3d(smem + L::offDN + st * C::kVBytes, &tm_dn, q_full + st, 0, i * kBw, bh);
+          tma_load_3d(smem + L::offQ + st * C::kQKBytes, &tm_q, q_full + st, 0, i * kBw, bh);
+        }
       }
-      mbar_wait_drain(kv_full, 0, wc.limit);
-      for (int n = issued - kBwStages < 0 ? 0 : issued - kBwStages; n < issued; ++n)
-        mbar_wait_drain(q_full + n % kBwStages, (n / kBwStages) & 1, wc.limit);
+      for (int n = nq - 2 < 0 ? 0 : nq - 2; n < nq; ++n) mbar_wait_drain(kv_full + (n & 1), (n >> 1) & 1, wc.limit);
+      for (long n = rg - kBwStages < 0 ? 0 : rg - kBwStages; n < rg; ++n)
+        mbar_wait_drain(q_full + n % kBwStages, (int)((n / kBwStages) & 1), wc.limit);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
@@ -414,127 +448,153 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     const uint64_t dv0 = smem_desc(smem_u32(smem + L::offV), 16, C::kVSbo, kSw128);
     const uint64_t dq0 = smem_desc(smem_u32(smem + L::offQ), 16, C::kQKSbo, C::kQKSw);
     const uint64_t ddn0 = smem_desc(smem_u32(smem + L::offDN), 16, C::kVSbo, kSw128);
-    // S^T = K Q_i^T (K = p) and dP^T = V dN_i^T (K = dv) of the query tile at stage st
-    auto issue_sdp = [&](int st) {
+    // S^T = K Q_i^T (K = p) and dP^T = V dN_i^T (K = dv): key buffer kb, query stage st
+    auto issue_sdp = [&](int kb, int st) {
 #pragma unroll
       for (int ks = 0; ks < p / 16; ++ks)
-        mma_ss_w(tmem + C::colS, desc_add(dk0, ks * 32), desc_add(dq0, st * C::kQKBytes + ks * 32), id_s, ks > 0);
+        mma_ss_w(tmem + C::colS, desc_add(dk0, kb * C::kQKBytes + ks * 32), desc_add(dq0, st * C::kQKBytes + ks * 32),
+                 id_s, ks > 0);
 #pragma unroll
       for (int ks = 0; ks < kBwDV / 16; ++ks)
-        mma_ss_w(tmem + C::colP, desc_add(dv0, ks * 32), desc_add(ddn0, st * C::kVBytes + ks * 32), id_s, ks > 0);
+        mma_ss_w(tmem + C::colP, desc_add(dv0, kb * C::kVBytes + ks * 32), desc_add(ddn0, st * C::kVBytes + ks * 32),
+                 id_s, ks > 0);
       mma_commit_w(s_full);
     };
-    bool ok = mbar_wait_w(kv_full, 0, env) && mbar_wait_w(q_full, 0, env);
-    if (ok) {
+    int gs = 0;       // query tiles processed by this CTA (global step)
+    int nq = 0, acc_cnt = 0;
+    bool ok = true;
+    for (int it = my_item(nq); ok && it >= 0; it = my_item(++nq)) {
+      const int tile = it / BH, kb = nq & 1, cnt = n_tiles - tile;
+      if (!mbar_wait_w(kv_full + kb, (nq >> 1) & 1, env) ||
+          !mbar_wait_w(q_full + gs % kBwStages, (int)((gs / kBwStages) & 1), env) ||
+          (gs > 0 && !mbar_wait_w(s_read, (int)((gs - 1) & 1), env))) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
-      issue_sdp(0);
-    }
-    for (int n = 0; ok && n < cnt; ++n) {
-      const int st = n % kBwStages;
-      if (n + 1 < cnt) {
-        const int sn = (n + 1) % kBwStages;
-        if (!mbar_wait_w(q_full + sn, ((n + 1) / kBwStages) & 1, env) || !mbar_wait_w(s_read, n & 1, env)) {
+      issue_sdp(kb, (int)(gs % kBwStages));
+      for (int n = 0; n < cnt; ++n) {
+        const int g = gs + n;
+        const int st = g % kBwStages;
+        if (n + 1 < cnt) {
+          // the next tile's S^T and dP^T overwrite the current ones: wait until loaded
+          if (!mbar_wait_w(q_full + (g + 1) % kBwStages, (int)(((g + 1) / kBwStages) & 1), env) ||
+              !mbar_wait_w(s_read, (int)(g & 1), env)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_sdp(kb, (int)((g + 1) % kBwStages));
+        }
+        if (!mbar_wait_w(p_full, (int)(g & 1), env)) {
+          ok = false;
+          break;
+        }
+        // the item's first dV / dK overwrite the accumulators: the previous
+        // item's epilogue must have read them
+        if (n == 0 && acc_cnt > 0 && !mbar_wait_w(acc_free, (acc_cnt - 1) & 1, env)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        issue_sdp(sn);
-      }
-      if (!mbar_wait_w(p_full, n & 1, env)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
 #pragma unroll
-      for (int ks = 0; ks < kBw / 16; ++ks)  // queries 16ks..: operand columns 8ks..
-        mma_ts_w(tmem + C::colAcc, tmem + C::colA(0) + 8 * ks, desc_add(ddn0, st * C::kVBytes + ks * C::kVKStep),
-                 id_dv, (n > 0 || ks > 0) ? 1u : 0u);
+        for (int ks = 0; ks < kBw / 16; ++ks)  // queries 16ks..: operand columns 8ks..
+          mma_ts_w(tmem + C::colAcc, tmem + C::colA(0) + 8 * ks, desc_add(ddn0, st * C::kVBytes + ks * C::kVKStep),
+                   id_dv, (n > 0 || ks > 0) ? 1u : 0u);
 #pragma unroll
-      for (int ks = 0; ks < kBw / 16; ++ks)
-        mma_ts_w(tmem + C::colAcc + kBwDV, tmem + C::colA(1) + 8 * ks,
-                 desc_add(dq0, st * C::kQKBytes + ks * C::kQKKStep), id_dk, (n > 0 || ks > 0) ? 1u : 0u);
-      mma_commit_w(w_free);
-      mma_commit_w(q_empty + st);
+        for (int ks = 0; ks < kBw / 16; ++ks)
+          mma_ts_w(tmem + C::colAcc + kBwDV, tmem + C::colA(1) + 8 * ks,
+                   desc_add(dq0, st * C::kQKBytes + ks * C::kQKKStep), id_dk, (n > 0 || ks > 0) ? 1u : 0u);
+        mma_commit_w(w_free);
+        mma_commit_w(q_empty + st);
+      }
+      if (!ok) break;
+      mma_commit_w(acc_full);
+      ++acc_cnt;
+      mma_commit_w(kv_empty + kb);
+      gs += cnt;
     }
     mma_commit_w(done);
     mbar_wait_drain(done, 0, wc.limit);
   } else {
-    // ------------------------------------------------------------- weight warps
+    // ------------------------------------------------------------- weight warps + epilogue
     const int quarter = warp % 4;                 // rows (keys) 32 quarter ..
     const int kq = (warp - 2) / 4;                // queries 32 kq .. of the query tile
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-    const int row = tile * kBw + quarter * 32 + lane;  // this thread's key
+    int gs = 0;
+    int nq = 0, acc_cnt = 0;
     bool ok = true;
-    for (int n = 0; n < cnt; ++n) {
-      // dD of this warp's 32 queries, one per lane (0 past T)
-      const int qrow = (tile + n) * kBw + 32 * kq + lane;
-      const float dDl = qrow < T ? dD[(size_t)bh * T + qrow] : 0.f;
-      if (!mbar_wait(s_full, n & 1, env)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      // causal mask on the diagonal tile: query 32 kq + c >= key 32 quarter + lane
-      const bool diag = (n == 0);
-      const bool skip = diag && kq < quarter;
-      const bool part = diag && kq == quarter;
-      uint32_t g[16], w[16];
-      if (skip) {
-#pragma unroll
-        for (int x = 0; x < 16; ++x) g[x] = w[x] = 0u;
-      } else {
-        uint32_t s[16], d[16];
-        tmem_ld16(lane_base + C::colS + 32 * kq, s);
-        tmem_ld16(lane_base + C::colP + 32 * kq, d);
-        tmem_wait_ld();
-        grad_block<0, true>(s, d, [&](int c) { return __shfl_sync(0xffffffffu, dDl, c); },
-                            [&](int c) { return !part || c >= lane; }, g, w);
-        tmem_ld16(lane_base + C::colS + 32 * kq + 16, s);
-        tmem_ld16(lane_base + C::colP + 32 * kq + 16, d);
-        tmem_wait_ld();
-        grad_block<1, true>(s, d, [&](int c) { return __shfl_sync(0xffffffffu, dDl, 16 + c); },
-                            [&](int c) { return !part || 16 + c >= lane; }, g, w);
-      }
-      tc_fence_before();
-      mbar_arrive(s_read);
-      // the operand buffers are read by the previous query tile's MMAs
-      if (n > 0 && !mbar_wait(w_free, (n - 1) & 1, env)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      tmem_st16(lane_base + C::colA(0) + 16 * kq, w);
-      tmem_st16(lane_base + C::colA(1) + 16 * kq, g);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(p_full);
-    }
-    // epilogue: dV (64 columns: 16 per key quarter warp) and dK (p columns,
-    // warps of key quarter 0) -> bf16, rows < T
-    if (ok && mbar_wait(done, 0, env)) {
-      tc_fence_after();
-      auto store16 = [&](__nv_bfloat16* dst_row, uint32_t col) {
-        uint32_t r[16];
-        tmem_ld16(lane_base + col, r);
-        tmem_wait_ld();
-        if (row < T) {
-          uint4* dst = reinterpret_cast<uint4*>(dst_row);
-          dst[0] = make_uint4(pack_bf16x2(__uint_as_float(r[0]), __uint_as_float(r[1])),
-                              pack_bf16x2(__uint_as_float(r[2]), __uint_as_float(r[3])),
-                              pack_bf16x2(__uint_as_float(r[4]), __uint_as_float(r[5])),
-                              pack_bf16x2(__uint_as_float(r[6]), __uint_as_float(r[7])));
-          dst[1] = make_uint4(pack_bf16x2(__uint_as_float(r[8]), __uint_as_float(r[9])),
-                              pack_bf16x2(__uint_as_float(r[10]), __uint_as_float(r[11])),
-                              pack_bf16x2(__uint_as_float(r[12]), __uint_as_float(r[13])),
-                              pack_bf16x2(__uint_as_float(r[14]), __uint_as_float(r[15])));
+    for (int it = my_item(nq); ok && it >= 0; it = my_item(++nq)) {
+      const int tile = it / BH, bh = it % BH, cnt = n_tiles - tile;
+      for (int n = 0; n < cnt; ++n) {
+        const int g = gs + n;
+        // dD of this warp's 32 queries, one per lane (0 past T)
+        const int qrow = (tile + n) * kBw + 32 * kq + lane;
+        const float dDl = qrow < T ? dD[(size_t)bh * T + qrow] : 0.f;
+        if (!mbar_wait(s_full, (int)(g & 1), env)) {
+          ok = false;
+          break;
         }
-      };
-      const size_t r0 = (size_t)bh * T + (row < T ? row : 0);
-      store16(dv + r0 * kBwDV + 16 * kq, C::colAcc + 16 * kq);
-      if (kq == 0) {
+        tc_fence_after();
+        // causal mask on the diagonal tile: query 32 kq + c >= key 32 quarter + lane
+        const bool diag = (n == 0);
+        const bool skip = diag && kq < quarter;
+        const bool part = diag && kq == quarter;
+        uint32_t gr[16], w[16];
+        if (skip) {
 #pragma unroll
-        for (int c0 = 0; c0 < p; c0 += 16) store16(dk + r0 * p + c0, C::colAcc + kBwDV + c0);
+          for (int x = 0; x < 16; ++x) gr[x] = w[x] = 0u;
+        } else {
+          uint32_t s[16], d[16];
+          tmem_ld16(lane_base + C::colS + 32 * kq, s);
+          tmem_ld16(lane_base + C::colP + 32 * kq, d);
+          tmem_wait_ld();
+          grad_block<0, true>(s, d, [&](int c) { return __shfl_sync(0xffffffffu, dDl, c); },
+                              [&](int c) { return !part || c >= lane; }, gr, w);
+          tmem_ld16(lane_base + C::colS + 32 * kq + 16, s);
+          tmem_ld16(lane_base + C::colP + 32 * kq + 16, d);
+          tmem_wait_ld();
+          grad_block<1, true>(s, d, [&](int c) { return __shfl_sync(0xffffffffu, dDl, 16 + c); },
+                              [&](int c) { return !part || 16 + c >= lane; }, gr, w);
+        }
+        tc_fence_before();
+        mbar_arrive(s_read);
+        // the operand buffers are read by the previous query tile's MMAs
+        if (g > 0 && !mbar_wait(w_free, (int)((g - 1) & 1), env)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        tmem_st16(lane_base + C::colA(0) + 16 * kq, w);
+        tmem_st16(lane_base + C::colA(1) + 16 * kq, gr);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(p_full);
       }
+      if (!ok || !mbar_wait(acc_full, acc_cnt & 1, env)) break;
+      ++acc_cnt;
+      tc_fence_after();
+      // epilogue: dV (16 columns per key-quarter warp) and dK (p columns,
+      // warps of key quarter 0) -> registers, then free the accumulators
+      uint32_t rv[16], rk0[16], rk1[16];
+      tmem_ld16(lane_base + C::colAcc + 16 * kq, rv);
+      if (kq == 0) {
+        tmem_ld16(lane_base + C::colAcc + kBwDV, rk0);
+        if constexpr (p == 32) tmem_ld16(lane_base + C::colAcc + kBwDV + 16, rk1);
+      }
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(acc_free);
+      const int row = tile * kBw + quarter * 32 + lane;  // this thread's key
+      if (row < T) {
+        const size_t r0 = (size_t)bh * T + row;
+        store_row16(dv + r0 * kBwDV + 16 * kq, rv);
+        if (kq == 0) {
+          store_row16(dk + r0 * p, rk0);
+          if constexpr (p == 32) store_row16(dk + r0 * p + 16, rk1);
+        }
+      }
+      gs += cnt;
     }
   }
 
@@ -569,8 +629,17 @@ static cudaError_t launch_bwd_t(const void* q, const void* k, const void* v, con
     return e;
   kq<<<grid, kBwThreads, DqSmem<p>::kBytes, st>>>(tq, tk, tv, tdn, dD, static_cast<__nv_bfloat16*>(dq), T, wc);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  kkv<<<grid, kBwThreads, DkvSmem<p>::kBytes, st>>>(tq, tk, tv, tdn, dD, static_cast<__nv_bfloat16*>(dk),
-                                                     static_cast<__nv_bfloat16*>(dv), T, wc);
+  static int num_sms = 0;
+  if (num_sms == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || num_sms <= 0)
+      num_sms = 148;
+  }
+  const long items = (long)grid.x * BH;
+  const int pgrid = (int)(items < num_sms ? items : num_sms);
+  kkv<<<pgrid, kBwThreads, DkvSmem<p>::kBytes, st>>>(tq, tk, tv, tdn, dD, static_cast<__nv_bfloat16*>(dk),
+                                                      static_cast<__nv_bfloat16*>(dv), T, BH, wc);
   return cudaGetLastError();
 }
 
