@@ -49,9 +49,11 @@ constexpr int kBwStages = 4;
 constexpr uint32_t kBwTmemCols = 512;
 
 // ---------------------------------------------------------------------------
-// 1. dN = dO / D rounded to bf16 and dD = -(dO . o) / D per row; a row with
-//    D = 0 (output constant 0) gets dN = 0 and dD = 0.  One warp per row of
-//    64 values, two per lane.
+// 1. dN' = 2 dO / D rounded to bf16 and dD' = -2 (dO . o) / D per row; a row
+//    with D = 0 (output constant 0) gets 0 for both.  The factor 2 of
+//    dS = 2 S (dP + dD) is folded in here (scaling by 2 is exact), so that
+//    dS = S (dN' . v + dD'); the dV accumulator, built from dN', is halved in
+//    its epilogue.  One warp per row of 64 values, two per lane.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __restrict__ dO,
                                                        const __nv_bfloat16* __restrict__ o,
@@ -67,8 +69,9 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __re
   for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
   const float d = D[row];
   const float inv = d > 0.f ? 1.f / d : 0.f;
-  reinterpret_cast<__nv_bfloat162*>(dN + row * kBwDV)[lane] = __floats2bfloat162_rn(a.x * inv, a.y * inv);
-  if (lane == 0) dD[row] = -dot * inv;
+  reinterpret_cast<__nv_bfloat162*>(dN + row * kBwDV)[lane] =
+      __floats2bfloat162_rn(2.f * (a.x * inv), 2.f * (a.y * inv));
+  if (lane == 0) dD[row] = -2.f * (dot * inv);
 }
 
 template <int p>
@@ -90,21 +93,37 @@ struct BwCfg {
 };
 
 // Gradient weights (and, with kW, squares) of 16 columns of one row, half
-// HF of the row's 32: s, d are the 16 fp32 scores and dP values, dd(c) the
-// dD term of column c.  g[8 HF + x] receives the bf16 pair of dS = 2 s (d + dd)
-// for columns 2x, 2x + 1, w[8 HF + x] that of s^2; columns with keep(c) false
-// become 0.
-template <int HF, bool kW, typename DD, typename Keep>
-__device__ __forceinline__ void grad_block(const uint32_t (&s)[16], const uint32_t (&d)[16], DD dd, Keep keep,
-                                           uint32_t (&g)[16], uint32_t (&w)[16]) {
+// HF of the row's 32, on fp32 pairs: s, d are the 16 scores and dP' values;
+// the dD' term is ddr for every column, or, with kCol, dd[x] for columns
+// 2x, 2x + 1.  g[8 HF + x] receives the bf16 pair of dS = s (dP' + dD'),
+// w[8 HF + x] that of s^2.  With kMask, column c (0..31 in the row's 32) is
+// kept only when kGE ? c >= lane : c <= lane, and is 0 otherwise.
+template <int HF, bool kW, bool kCol, bool kMask, bool kGE>
+__device__ __forceinline__ void grad_pairs(const uint32_t (&s)[16], const uint32_t (&d)[16], const float2* dd,
+                                           float ddr, int lane, uint32_t (&g)[16], uint32_t (&w)[16]) {
 #pragma unroll
   for (int x = 0; x < 8; ++x) {
-    const float s0 = __uint_as_float(s[2 * x]), s1 = __uint_as_float(s[2 * x + 1]);
-    const float g0 = 2.f * s0 * (__uint_as_float(d[2 * x]) + dd(2 * x));
-    const float g1 = 2.f * s1 * (__uint_as_float(d[2 * x + 1]) + dd(2 * x + 1));
-    const bool k0 = keep(2 * x), k1 = keep(2 * x + 1);
-    g[8 * HF + x] = pack_bf16x2(k0 ? g0 : 0.f, k1 ? g1 : 0.f);
-    if (kW) w[8 * HF + x] = pack_bf16x2(k0 ? s0 * s0 : 0.f, k1 ? s1 * s1 : 0.f);
+    const float2 e = kCol ? dd[x] : make_float2(ddr, ddr);
+    const uint64_t s2 = f32x2(s[2 * x], s[2 * x + 1]);
+    const uint64_t gg = f32x2_mul(s2, f32x2_add(f32x2(d[2 * x], d[2 * x + 1]),
+                                                f32x2(__float_as_uint(e.x), __float_as_uint(e.y))));
+    float g0 = f32x2_lo(gg), g1 = f32x2_hi(gg);
+    if (kMask) {
+      const int c = 16 * HF + 2 * x;
+      if (kGE ? c < lane : c > lane) g0 = 0.f;
+      if (kGE ? c + 1 < lane : c + 1 > lane) g1 = 0.f;
+    }
+    g[8 * HF + x] = pack_bf16x2(g0, g1);
+    if (kW) {
+      const uint64_t ww = f32x2_mul(s2, s2);
+      float w0 = f32x2_lo(ww), w1 = f32x2_hi(ww);
+      if (kMask) {
+        const int c = 16 * HF + 2 * x;
+        if (kGE ? c < lane : c > lane) w0 = 0.f;
+        if (kGE ? c + 1 < lane : c + 1 > lane) w1 = 0.f;
+      }
+      w[8 * HF + x] = pack_bf16x2(w0, w1);
+    }
   }
 }
 
@@ -266,15 +285,20 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         for (int x = 0; x < 16; ++x) g[x] = 0u;
       } else {
         uint32_t s[16], d[16];
-        auto dd = [&](int) { return dDr; };
         tmem_ld16(lane_base + C::colS + 32 * kq, s);
         tmem_ld16(lane_base + C::colP + 32 * kq, d);
         tmem_wait_ld();
-        grad_block<0, false>(s, d, dd, [&](int c) { return !part || c <= lane; }, g, unused);
+        if (part)
+          grad_pairs<0, false, false, true, false>(s, d, nullptr, dDr, lane, g, unused);
+        else
+          grad_pairs<0, false, false, false, false>(s, d, nullptr, dDr, lane, g, unused);
         tmem_ld16(lane_base + C::colS + 32 * kq + 16, s);
         tmem_ld16(lane_base + C::colP + 32 * kq + 16, d);
         tmem_wait_ld();
-        grad_block<1, false>(s, d, dd, [&](int c) { return !part || 16 + c <= lane; }, g, unused);
+        if (part)
+          grad_pairs<1, false, false, true, false>(s, d, nullptr, dDr, lane, g, unused);
+        else
+          grad_pairs<1, false, false, false, false>(s, d, nullptr, dDr, lane, g, unused);
       }
       // S and dP are in registers: the next key tile's may overwrite them
       tc_fence_before();
@@ -341,7 +365,8 @@ struct DkvSmem {
   static constexpr int offK = offV + 2 * C::kVBytes;                    // 2 buffers of K_j
   static constexpr int offDN = (offK + 2 * C::kQKBytes + 1023) / 1024 * 1024;  // ring of dN_i
   static constexpr int offQ = offDN + kBwStages * C::kVBytes;           // ring of Q_i
-  static constexpr int offBar = (offQ + kBwStages * C::kQKBytes + 1023) / 1024 * 1024;
+  static constexpr int offDD = offQ + kBwStages * C::kQKBytes;          // dD' of 32 queries per weight warp
+  static constexpr int offBar = (offDD + 16 * 32 * 4 + 1023) / 1024 * 1024;
   static constexpr int kBars = 4 + 2 * kBwStages + 7;
   static constexpr int offMisc = offBar + kBars * 8;
   static constexpr int kBytes = offMisc + 16 + 1024;
@@ -521,6 +546,8 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     const int quarter = warp % 4;                 // rows (keys) 32 quarter ..
     const int kq = (warp - 2) / 4;                // queries 32 kq .. of the query tile
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    float* dd_slot = reinterpret_cast<float*>(smem + L::offDD) + (warp - 2) * 32;
+    const float2* dd_pairs = reinterpret_cast<const float2*>(dd_slot);
     int gs = 0;
     int nq = 0, acc_cnt = 0;
     bool ok = true;
@@ -545,17 +572,25 @@ __global__ void __launch_bounds__(kBwThreads, 1)
 #pragma unroll
           for (int x = 0; x < 16; ++x) gr[x] = w[x] = 0u;
         } else {
+          // the 32 dD' values, read back as column pairs (a broadcast per pair)
+          __syncwarp();
+          dd_slot[lane] = dDl;
+          __syncwarp();
           uint32_t s[16], d[16];
           tmem_ld16(lane_base + C::colS + 32 * kq, s);
           tmem_ld16(lane_base + C::colP + 32 * kq, d);
           tmem_wait_ld();
-          grad_block<0, true>(s, d, [&](int c) { return __shfl_sync(0xffffffffu, dDl, c); },
-                              [&](int c) { return !part || c >= lane; }, gr, w);
+          if (part)
+            grad_pairs<0, true, true, true, true>(s, d, dd_pairs, 0.f, lane, gr, w);
+          else
+            grad_pairs<0, true, true, false, true>(s, d, dd_pairs, 0.f, lane, gr, w);
           tmem_ld16(lane_base + C::colS + 32 * kq + 16, s);
           tmem_ld16(lane_base + C::colP + 32 * kq + 16, d);
           tmem_wait_ld();
-          grad_block<1, true>(s, d, [&](int c) { return __shfl_sync(0xffffffffu, dDl, 16 + c); },
-                              [&](int c) { return !part || 16 + c >= lane; }, gr, w);
+          if (part)
+            grad_pairs<1, true, true, true, true>(s, d, dd_pairs + 8, 0.f, lane, gr, w);
+          else
+            grad_pairs<1, true, true, false, true>(s, d, dd_pairs + 8, 0.f, lane, gr, w);
         }
         tc_fence_before();
         mbar_arrive(s_read);
@@ -585,6 +620,9 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(acc_free);
+      // dV was accumulated from dN' = 2 dO / D: halve it (exact)
+#pragma unroll
+      for (int x = 0; x < 16; ++x) rv[x] = __float_as_uint(0.5f * __uint_as_float(rv[x]));
       const int row = tile * kBw + quarter * 32 + lane;  // this thread's key
       if (row < T) {
         const size_t r0 = (size_t)bh * T + row;
