@@ -13,7 +13,7 @@
 // on the training step, arXiv abstract).  D comes from the forward
 // (kata_fwd_quadratic_train).  Three launches:
 //   1. bwd_prep_kernel   dN (bf16) and dD (fp32) per row, one warp per row;
-//   2. bwd_dq_kernel     one CTA per 128-row query tile: per key tile j,
+//   2. bwd_dq_kernel     persistent, items of one 128-row query tile: per key tile j,
 //                        S = Q K_j^T and dP = dN V_j^T on the tensor core,
 //                        dS = 2 S (dP + dD) in the weight warps, then
 //                        dQ += dS K_j with dS read from TMEM;
@@ -127,18 +127,32 @@ __device__ __forceinline__ void grad_pairs(const uint32_t (&s)[16], const uint32
   }
 }
 
+// 16 fp32 values -> 16 bf16 at dst (32 bytes, 16-byte aligned)
+__device__ __forceinline__ void store_row16(__nv_bfloat16* dst_row, const uint32_t (&r)[16]) {
+  uint4* dst = reinterpret_cast<uint4*>(dst_row);
+  dst[0] = make_uint4(pack_bf16x2(__uint_as_float(r[0]), __uint_as_float(r[1])),
+                      pack_bf16x2(__uint_as_float(r[2]), __uint_as_float(r[3])),
+                      pack_bf16x2(__uint_as_float(r[4]), __uint_as_float(r[5])),
+                      pack_bf16x2(__uint_as_float(r[6]), __uint_as_float(r[7])));
+  dst[1] = make_uint4(pack_bf16x2(__uint_as_float(r[8]), __uint_as_float(r[9])),
+                      pack_bf16x2(__uint_as_float(r[10]), __uint_as_float(r[11])),
+                      pack_bf16x2(__uint_as_float(r[12]), __uint_as_float(r[13])),
+                      pack_bf16x2(__uint_as_float(r[14]), __uint_as_float(r[15])));
+}
+
 // ---------------------------------------------------------------------------
-// 2. dQ: CTA (query tile i, head bh), key tiles j = 0..i
+// 2. dQ: persistent CTAs over items (query tile i, head bh), heaviest first;
+//    per item, key tiles j = 0..i
 // ---------------------------------------------------------------------------
 template <int p>
 struct DqSmem {
   using C = BwCfg<p>;
-  static constexpr int offDN = 0;                                       // dN_i (SW128)
-  static constexpr int offQ = offDN + C::kVBytes;                       // Q_i
-  static constexpr int offK = (offQ + C::kQKBytes + 1023) / 1024 * 1024;  // ring of K_j
+  static constexpr int offDN = 0;                                       // 2 buffers of dN_i (SW128)
+  static constexpr int offQ = offDN + 2 * C::kVBytes;                   // 2 buffers of Q_i
+  static constexpr int offK = (offQ + 2 * C::kQKBytes + 1023) / 1024 * 1024;  // ring of K_j
   static constexpr int offV = (offK + kBwStages * C::kQKBytes + 1023) / 1024 * 1024;  // ring of V_j
   static constexpr int offBar = offV + kBwStages * C::kVBytes;
-  static constexpr int kBars = 1 + 2 * kBwStages + 5;
+  static constexpr int kBars = 4 + 2 * kBwStages + 7;
   static constexpr int offMisc = offBar + kBars * 8;
   static constexpr int kBytes = offMisc + 16 + 1024;
 };
@@ -147,38 +161,48 @@ template <int p>
 __global__ void __launch_bounds__(kBwThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_dn,
-                  const float* __restrict__ dD, __nv_bfloat16* __restrict__ dq, int T, WaitCtl wc) {
+                  const float* __restrict__ dD, __nv_bfloat16* __restrict__ dq, int T, int BH, WaitCtl wc) {
   using C = BwCfg<p>;
   using L = DqSmem<p>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::offBar);
-  uint64_t* q_full = bars;                      // Q_i and dN_i landed
-  uint64_t* kv_full = q_full + 1;               // [kBwStages]
+  uint64_t* q_full = bars;                      // [2] Q_i and dN_i landed
+  uint64_t* q_empty = q_full + 2;               // [2]
+  uint64_t* kv_full = q_empty + 2;              // [kBwStages]
   uint64_t* kv_empty = kv_full + kBwStages;     // [kBwStages]
   uint64_t* s_full = kv_empty + kBwStages;      // S and dP of a key tile in TMEM
   uint64_t* s_read = s_full + 1;                // ... loaded by the weight warps (512)
   uint64_t* p_full = s_read + 1;                // [2] dS buffer written (512)
-  uint64_t* done = p_full + 2;                  // every MMA of the CTA complete
+  uint64_t* acc_full = p_full + 2;              // an item's dQ complete
+  uint64_t* acc_free = acc_full + 1;            // ... read by the epilogue (512)
+  uint64_t* done = acc_free + 1;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::offMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::offMisc + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_tiles = (T + kBw - 1) / kBw;
-  const int tile = n_tiles - 1 - (int)blockIdx.x;  // heaviest first
-  const int bh = blockIdx.y;
-  const int nkv = tile + 1;
+  const int n_items = n_tiles * BH;
+  auto item_tile = [&](int it) { return n_tiles - 1 - it / BH; };  // heaviest first
+  auto my_item = [&](int r) {
+    const int it = r * (int)gridDim.x + ((r & 1) ? (int)gridDim.x - 1 - (int)blockIdx.x : (int)blockIdx.x);
+    return it < n_items ? it : -1;
+  };
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(q_full + b, 1);
+      mbar_init(q_empty + b, 1);
+      mbar_init(p_full + b, 512);
+    }
     for (int s = 0; s < kBwStages; ++s) {
       mbar_init(kv_full + s, 1);
       mbar_init(kv_empty + s, 1);
     }
     mbar_init(s_full, 1);
     mbar_init(s_read, 512);
-    mbar_init(p_full, 512);
-    mbar_init(p_full + 1, 512);
+    mbar_init(acc_full, 1);
+    mbar_init(acc_free, 512);
     mbar_init(done, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -197,21 +221,29 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
       prefetch_tmap(&tm_dn);
-      mbar_arrive_expect_tx(q_full, C::kVBytes + C::kQKBytes);
-      tma_load_3d(smem + L::offDN, &tm_dn, q_full, 0, tile * kBw, bh);
-      tma_load_3d(smem + L::offQ, &tm_q, q_full, 0, tile * kBw, bh);
-      int issued = 0;
-      for (int j = 0; j < nkv; ++j) {
-        const int st = j % kBwStages;
-        if (!mbar_wait(kv_empty + st, ((j / kBwStages) & 1) ^ 1, env)) break;
-        mbar_arrive_expect_tx(kv_full + st, C::kQKBytes + C::kVBytes);
-        tma_load_3d(smem + L::offK + st * C::kQKBytes, &tm_k, kv_full + st, 0, j * kBw, bh);
-        tma_load_3d(smem + L::offV + st * C::kVBytes, &tm_v, kv_full + st, 0, j * kBw, bh);
-        ++issued;
+      int nq = 0;
+      long rg = 0;  // key tiles loaded (ring position)
+      bool ok = true;
+      for (int it = my_item(nq); ok && it >= 0; it = my_item(++nq)) {
+        const int tile = item_tile(it), bh = it % BH, qb = nq & 1;
+        if (!mbar_wait(q_empty + qb, ((nq >> 1) & 1) ^ 1, env)) break;
+        mbar_arrive_expect_tx(q_full + qb, C::kVBytes + C::kQKBytes);
+        tma_load_3d(smem + L::offDN + qb * C::kVBytes, &tm_dn, q_full + qb, 0, tile * kBw, bh);
+        tma_load_3d(smem + L::offQ + qb * C::kQKBytes, &tm_q, q_full + qb, 0, tile * kBw, bh);
+        for (int j = 0; j <= tile; ++j, ++rg) {
+          const int st = (int)(rg % kBwStages);
+          if (!mbar_wait(kv_empty + st, (int)((rg / kBwStages) & 1) ^ 1, env)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(kv_full + st, C::kQKBytes + C::kVBytes);
+          tma_load_3d(smem + L::offK + st * C::kQKBytes, &tm_k, kv_full + st, 0, j * kBw, bh);
+          tma_load_3d(smem + L::offV + st * C::kVBytes, &tm_v, kv_full + st, 0, j * kBw, bh);
+        }
       }
-      mbar_wait_drain(q_full, 0, wc.limit);
-      for (int j = issued - kBwStages < 0 ? 0 : issued - kBwStages; j < issued; ++j)
-        mbar_wait_drain(kv_full + j % kBwStages, (j / kBwStages) & 1, wc.limit);
+      for (int n = nq - 2 < 0 ? 0 : nq - 2; n < nq; ++n) mbar_wait_drain(q_full + (n & 1), (n >> 1) & 1, wc.limit);
+      for (long n = rg - kBwStages < 0 ? 0 : rg - kBwStages; n < rg; ++n)
+        mbar_wait_drain(kv_full + n % kBwStages, (int)((n / kBwStages) & 1), wc.limit);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
@@ -221,115 +253,140 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     const uint64_t ddn0 = smem_desc(smem_u32(smem + L::offDN), 16, C::kVSbo, kSw128);
     const uint64_t dk0 = smem_desc(smem_u32(smem + L::offK), 16, C::kQKSbo, C::kQKSw);
     const uint64_t dv0 = smem_desc(smem_u32(smem + L::offV), 16, C::kVSbo, kSw128);
-    // S = Q K_j^T (K = p) and dP = dN V_j^T (K = dv) of the key tile at stage st
-    auto issue_sdp = [&](int st) {
+    // S = Q K_j^T (K = p) and dP' = dN' V_j^T (K = dv): query buffer qb, key stage st
+    auto issue_sdp = [&](int qb, int st) {
 #pragma unroll
       for (int ks = 0; ks < p / 16; ++ks)
-        mma_ss_w(tmem + C::colS, desc_add(dq0, ks * 32), desc_add(dk0, st * C::kQKBytes + ks * 32), id_s, ks > 0);
+        mma_ss_w(tmem + C::colS, desc_add(dq0, qb * C::kQKBytes + ks * 32), desc_add(dk0, st * C::kQKBytes + ks * 32),
+                 id_s, ks > 0);
 #pragma unroll
       for (int ks = 0; ks < kBwDV / 16; ++ks)
-        mma_ss_w(tmem + C::colP, desc_add(ddn0, ks * 32), desc_add(dv0, st * C::kVBytes + ks * 32), id_s, ks > 0);
+        mma_ss_w(tmem + C::colP, desc_add(ddn0, qb * C::kVBytes + ks * 32), desc_add(dv0, st * C::kVBytes + ks * 32),
+                 id_s, ks > 0);
       mma_commit_w(s_full);
     };
-    bool ok = mbar_wait_w(q_full, 0, env) && mbar_wait_w(kv_full, 0, env);
-    if (ok) {
+    int gs = 0;       // key tiles processed by this CTA (global step)
+    int nq = 0, acc_cnt = 0;
+    bool ok = true;
+    for (int it = my_item(nq); ok && it >= 0; it = my_item(++nq)) {
+      const int qb = nq & 1, nkv = item_tile(it) + 1;
+      if (!mbar_wait_w(q_full + qb, (nq >> 1) & 1, env) ||
+          !mbar_wait_w(kv_full + gs % kBwStages, (gs / kBwStages) & 1, env) ||
+          (gs > 0 && !mbar_wait_w(s_read, (gs - 1) & 1, env))) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
-      issue_sdp(0);
-    }
-    for (int j = 0; ok && j < nkv; ++j) {
-      const int st = j % kBwStages;
-      if (j + 1 < nkv) {
-        const int sn = (j + 1) % kBwStages;
-        // the next tile's S and dP overwrite the current ones: wait until loaded
-        if (!mbar_wait_w(kv_full + sn, ((j + 1) / kBwStages) & 1, env) || !mbar_wait_w(s_read, j & 1, env)) {
+      issue_sdp(qb, gs % kBwStages);
+      for (int j = 0; j < nkv; ++j) {
+        const int g = gs + j, st = g % kBwStages;
+        if (j + 1 < nkv) {
+          // the next tile's S and dP' overwrite the current ones: wait until loaded
+          if (!mbar_wait_w(kv_full + (g + 1) % kBwStages, ((g + 1) / kBwStages) & 1, env) ||
+              !mbar_wait_w(s_read, g & 1, env)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_sdp(qb, (g + 1) % kBwStages);
+        }
+        if (!mbar_wait_w(p_full + (g & 1), (g >> 1) & 1, env)) {
+          ok = false;
+          break;
+        }
+        // the item's first dQ MMA overwrites the accumulator: the previous
+        // item's epilogue must have read it
+        if (j == 0 && acc_cnt > 0 && !mbar_wait_w(acc_free, (acc_cnt - 1) & 1, env)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        issue_sdp(sn);
-      }
-      if (!mbar_wait_w(p_full + (j & 1), (j >> 1) & 1, env)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
 #pragma unroll
-      for (int ks = 0; ks < kBw / 16; ++ks)  // keys 16ks..: dS columns 8ks.. of the buffer
-        mma_ts_w(tmem + C::colAcc, tmem + C::colA(j & 1) + 8 * ks, desc_add(dk0, st * C::kQKBytes + ks * C::kQKKStep),
-                 id_dq, (j > 0 || ks > 0) ? 1u : 0u);
-      mma_commit_w(kv_empty + st);
+        for (int ks = 0; ks < kBw / 16; ++ks)  // keys 16ks..: dS columns 8ks.. of the buffer
+          mma_ts_w(tmem + C::colAcc, tmem + C::colA(g & 1) + 8 * ks,
+                   desc_add(dk0, st * C::kQKBytes + ks * C::kQKKStep), id_dq, (j > 0 || ks > 0) ? 1u : 0u);
+        mma_commit_w(kv_empty + st);
+      }
+      if (!ok) break;
+      mma_commit_w(acc_full);
+      ++acc_cnt;
+      mma_commit_w(q_empty + qb);
+      gs += nkv;
     }
     mma_commit_w(done);
     mbar_wait_drain(done, 0, wc.limit);
   } else {
-    // ------------------------------------------------------------- weight warps
+    // ------------------------------------------------------------- weight warps + epilogue
     const int quarter = warp % 4;                 // rows (queries) 32 quarter ..
     const int kq = (warp - 2) / 4;                // keys 32 kq .. of the key tile
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-    const int row = tile * kBw + quarter * 32 + lane;
-    const float dDr = row < T ? dD[(size_t)bh * T + row] : 0.f;
+    int gs = 0;
+    int nq = 0, acc_cnt = 0;
     bool ok = true;
-    for (int j = 0; j < nkv; ++j) {
-      if (!mbar_wait(s_full, j & 1, env)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      // causal mask on the diagonal tile: key 32 kq + c <= query 32 quarter + lane
-      const bool diag = (j == nkv - 1);
-      const bool skip = diag && kq > quarter;
-      const bool part = diag && kq == quarter;
-      uint32_t g[16], unused[16];
-      if (skip) {
-#pragma unroll
-        for (int x = 0; x < 16; ++x) g[x] = 0u;
-      } else {
-        uint32_t s[16], d[16];
-        tmem_ld16(lane_base + C::colS + 32 * kq, s);
-        tmem_ld16(lane_base + C::colP + 32 * kq, d);
-        tmem_wait_ld();
-        if (part)
-          grad_pairs<0, false, false, true, false>(s, d, nullptr, dDr, lane, g, unused);
-        else
-          grad_pairs<0, false, false, false, false>(s, d, nullptr, dDr, lane, g, unused);
-        tmem_ld16(lane_base + C::colS + 32 * kq + 16, s);
-        tmem_ld16(lane_base + C::colP + 32 * kq + 16, d);
-        tmem_wait_ld();
-        if (part)
-          grad_pairs<1, false, false, true, false>(s, d, nullptr, dDr, lane, g, unused);
-        else
-          grad_pairs<1, false, false, false, false>(s, d, nullptr, dDr, lane, g, unused);
-      }
-      // S and dP are in registers: the next key tile's may overwrite them
-      tc_fence_before();
-      mbar_arrive(s_read);
-      // dS buffer j % 2 was last read by the dQ MMAs of key tile j - 2, which
-      // completed before S(j) did
-      tmem_st16(lane_base + C::colA(j & 1) + 16 * kq, g);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(p_full + (j & 1));
-    }
-    // epilogue: dQ (fp32, p columns) -> bf16, rows < T; warps of key quarter 0
-    if (ok && kq == 0 && mbar_wait(done, 0, env)) {
-      tc_fence_after();
-#pragma unroll
-      for (int c0 = 0; c0 < p; c0 += 16) {
-        uint32_t r[16];
-        tmem_ld16(lane_base + C::colAcc + c0, r);
-        tmem_wait_ld();
-        if (row < T) {
-          uint4* dst = reinterpret_cast<uint4*>(dq + ((size_t)bh * T + row) * p + c0);
-          dst[0] = make_uint4(pack_bf16x2(__uint_as_float(r[0]), __uint_as_float(r[1])),
-                              pack_bf16x2(__uint_as_float(r[2]), __uint_as_float(r[3])),
-                              pack_bf16x2(__uint_as_float(r[4]), __uint_as_float(r[5])),
-                              pack_bf16x2(__uint_as_float(r[6]), __uint_as_float(r[7])));
-          dst[1] = make_uint4(pack_bf16x2(__uint_as_float(r[8]), __uint_as_float(r[9])),
-                              pack_bf16x2(__uint_as_float(r[10]), __uint_as_float(r[11])),
-                              pack_bf16x2(__uint_as_float(r[12]), __uint_as_float(r[13])),
-                              pack_bf16x2(__uint_as_float(r[14]), __uint_as_float(r[15])));
+    for (int it = my_item(nq); ok && it >= 0; it = my_item(++nq)) {
+      const int tile = item_tile(it), bh = it % BH, nkv = tile + 1;
+      const int row = tile * kBw + quarter * 32 + lane;
+      const float dDr = row < T ? dD[(size_t)bh * T + row] : 0.f;
+      for (int j = 0; j < nkv; ++j) {
+        const int g = gs + j;
+        if (!mbar_wait(s_full, g & 1, env)) {
+          ok = false;
+          break;
         }
+        tc_fence_after();
+        // causal mask on the diagonal tile: key 32 kq + c <= query 32 quarter + lane
+        const bool diag = (j == nkv - 1);
+        const bool skip = diag && kq > quarter;
+        const bool part = diag && kq == quarter;
+        uint32_t gr[16], unused[16];
+        if (skip) {
+#pragma unroll
+          for (int x = 0; x < 16; ++x) gr[x] = 0u;
+        } else {
+          uint32_t s[16], d[16];
+          tmem_ld16(lane_base + C::colS + 32 * kq, s);
+          tmem_ld16(lane_base + C::colP + 32 * kq, d);
+          tmem_wait_ld();
+          if (part)
+            grad_pairs<0, false, false, true, false>(s, d, nullptr, dDr, lane, gr, unused);
+          else
+            grad_pairs<0, false, false, false, false>(s, d, nullptr, dDr, lane, gr, unused);
+          tmem_ld16(lane_base + C::colS + 32 * kq + 16, s);
+          tmem_ld16(lane_base + C::colP + 32 * kq + 16, d);
+          tmem_wait_ld();
+          if (part)
+            grad_pairs<1, false, false, true, false>(s, d, nullptr, dDr, lane, gr, unused);
+          else
+            grad_pairs<1, false, false, false, false>(s, d, nullptr, dDr, lane, gr, unused);
+        }
+        // S and dP' are in registers: the next key tile's may overwrite them
+        tc_fence_before();
+        mbar_arrive(s_read);
+        // dS buffer g % 2 was last read by the dQ MMAs of step g - 2, which
+        // completed before S(g) did
+        tmem_st16(lane_base + C::colA(g & 1) + 16 * kq, gr);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(p_full + (g & 1));
       }
+      if (!ok || !mbar_wait(acc_full, acc_cnt & 1, env)) break;
+      ++acc_cnt;
+      tc_fence_after();
+      // epilogue: dQ (p fp32 columns) -> registers (warps of key quarter 0),
+      // then free the accumulator; bf16 rows < T
+      uint32_t r0[16], r1[16];
+      if (kq == 0) {
+        tmem_ld16(lane_base + C::colAcc, r0);
+        if constexpr (p == 32) tmem_ld16(lane_base + C::colAcc + 16, r1);
+        tmem_wait_ld();
+      }
+      tc_fence_before();
+      mbar_arrive(acc_free);
+      if (kq == 0 && row < T) {
+        store_row16(dq + ((size_t)bh * T + row) * p, r0);
+        if constexpr (p == 32) store_row16(dq + ((size_t)bh * T + row) * p + 16, r1);
+      }
+      gs += nkv;
     }
   }
 
@@ -339,23 +396,6 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, kBwTmemCols);
   }
-}
-
-// ---------------------------------------------------------------------------
-// 3. dK, dV: persistent CTAs over items (key tile j, head bh), heaviest
-//    (j = 0) first; per item, query tiles i = j..n_tiles-1
-// ---------------------------------------------------------------------------
-// 16 fp32 values -> 16 bf16 at dst (32 bytes, 16-byte aligned)
-__device__ __forceinline__ void store_row16(__nv_bfloat16* dst_row, const uint32_t (&r)[16]) {
-  uint4* dst = reinterpret_cast<uint4*>(dst_row);
-  dst[0] = make_uint4(pack_bf16x2(__uint_as_float(r[0]), __uint_as_float(r[1])),
-                      pack_bf16x2(__uint_as_float(r[2]), __uint_as_float(r[3])),
-                      pack_bf16x2(__uint_as_float(r[4]), __uint_as_float(r[5])),
-                      pack_bf16x2(__uint_as_float(r[6]), __uint_as_float(r[7])));
-  dst[1] = make_uint4(pack_bf16x2(__uint_as_float(r[8]), __uint_as_float(r[9])),
-                      pack_bf16x2(__uint_as_float(r[10]), __uint_as_float(r[11])),
-                      pack_bf16x2(__uint_as_float(r[12]), __uint_as_float(r[13])),
-                      pack_bf16x2(__uint_as_float(r[14]), __uint_as_float(r[15])));
 }
 
 template <int p>
@@ -665,8 +705,6 @@ static cudaError_t launch_bwd_t(const void* q, const void* k, const void* v, con
   if ((e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, DqSmem<p>::kBytes)) != cudaSuccess ||
       (e = cudaFuncSetAttribute(kkv, cudaFuncAttributeMaxDynamicSharedMemorySize, DkvSmem<p>::kBytes)) != cudaSuccess)
     return e;
-  kq<<<grid, kBwThreads, DqSmem<p>::kBytes, st>>>(tq, tk, tv, tdn, dD, static_cast<__nv_bfloat16*>(dq), T, wc);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
   static int num_sms = 0;
   if (num_sms == 0) {
     int dev = 0;
@@ -676,6 +714,8 @@ static cudaError_t launch_bwd_t(const void* q, const void* k, const void* v, con
   }
   const long items = (long)grid.x * BH;
   const int pgrid = (int)(items < num_sms ? items : num_sms);
+  kq<<<pgrid, kBwThreads, DqSmem<p>::kBytes, st>>>(tq, tk, tv, tdn, dD, static_cast<__nv_bfloat16*>(dq), T, BH, wc);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
   kkv<<<pgrid, kBwThreads, DkvSmem<p>::kBytes, st>>>(tq, tk, tv, tdn, dD, static_cast<__nv_bfloat16*>(dk),
                                                       static_cast<__nv_bfloat16*>(dv), T, BH, wc);
   return cudaGetLastError();
