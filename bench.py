@@ -51,10 +51,10 @@ UNIT = "tokens/s"
 # DRAM bytes (read + write) of one flash_fwd_kernel launch at B8 H16 T2048,
 # from the ncu capture summarised in profiles/flash_fwd_kernel_ctx2k.md.  It
 # is reported only while the kernel's sources are the ones that capture ran.
-FLASH_TRAFFIC_BYTES = 50535424 + 6024448
+FLASH_TRAFFIC_BYTES = 50472704 + 6547712
 FLASH_TRAFFIC_SOURCES = ("kernelized_feature_map_b200/csrc/flash_sm100.cu", "kernelized_feature_map_b200/csrc/sm100.cuh",
                          "kernelized_feature_map_b200/csrc/kata_trace.cuh", "kernelized_feature_map_b200/csrc/kata_common.cuh")
-FLASH_TRAFFIC_SHA256 = "7e106fad3b63565fcfa6bbfca7c8a6597349ff0803f6c324d62cf9c30866e1aa"
+FLASH_TRAFFIC_SHA256 = "ab7f7563bcf48676323ac1b90d0185ccad44e79b9b632361233c127cf371f620"
 
 
 def flash_traffic(workload):
