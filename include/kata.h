@@ -189,7 +189,8 @@ kata_status_t kata_decode_step(const void* q, const void* k, const void* v, void
  *   gradient dO ([B,H,T,dv]), writes dq, dk ([B,H,T,p]) and dv ([B,H,T,dv]),
  *   all bf16 (fp32 accumulation).  A row with D_t = 0 (output constant 0)
  *   passes no gradient.  `workspace` (16-byte aligned, at least
- *   kata_bwd_quadratic_workspace_size bytes) holds dO/D and (dO.o)/D per row.
+ *   kata_bwd_quadratic_workspace_size bytes = 8 per row) holds dO.o and 1/D
+ *   per row.
  */
 kata_status_t kata_fwd_quadratic_train(const void* q, const void* k, const void* v, void* o, float* D,
                                        int B, int H, int T, int p, int dv,

@@ -9,17 +9,24 @@
 //   dS_ts = 2 S_ts (dN_t . v_s + dD_t)                    (s <= t)
 //   dv_s  = sum_{t>=s} w_ts dN_t
 //   dq_t  = sum_{s<=t} dS_ts k_s,   dk_s = sum_{t>=s} dS_ts q_t
+// evaluated as dS_ts = 2 (S_ts r_t) (dO_t . v_s - delta_t) and
+// dv_s = sum_t (S_ts^2 r_t) dO_t with r_t = 1 / D_t and delta_t = dO_t . o_t:
+// the tensor core multiplies dO itself (exact bf16 input), and the
+// difference dO.v - dO.o, which cancels when the row's weight sits on few
+// keys, is taken in fp32 before the 1 / D scaling.  (Rounding dN = dO / D to
+// bf16 first turns that cancellation into errors of order 2^-9 |dO||v| / D,
+// which dominate the gradient when some D_t is small.)
 // (the pages print no backward pass; they say the kernels are competitive
 // on the training step, arXiv abstract).  D comes from the forward
 // (kata_fwd_quadratic_train).  Three launches:
-//   1. bwd_prep_kernel   dN (bf16) and dD (fp32) per row, one warp per row;
+//   1. bwd_rows_kernel   (-delta_t, r_t) per row, one warp per row;
 //   2. bwd_dq_kernel     persistent, items of one 128-row query tile: per key tile j,
-//                        S = Q K_j^T and dP = dN V_j^T on the tensor core,
-//                        dS = 2 S (dP + dD) in the weight warps, then
+//                        S = Q K_j^T and dP = dO V_j^T on the tensor core,
+//                        dS in the weight warps, then
 //                        dQ += dS K_j with dS read from TMEM;
 //   3. bwd_dkdv_kernel   persistent, items of one 128-row key tile: per query tile i,
-//                        S^T = K Q_i^T and dP^T = V dN_i^T, W^T = (S^T)^2 and
-//                        dS^T in the weight warps, then dV += W^T dN_i and
+//                        S^T = K Q_i^T and dP^T = V dO_i^T, W^T = (S^T)^2 r and
+//                        dS^T in the weight warps, then dV += W^T dO_i and
 //                        dK += dS^T Q_i.
 // Both main kernels keep the products in TMEM with keys (dQ) or queries
 // (dK, dV) along the reduction dimension, so every MMA's A operand comes
@@ -32,7 +39,10 @@
 #include <cuda_bf16.h>
 
 #include "kata_internal.h"
+#include "kata_trace.cuh"
 #include "sm100.cuh"
+
+KATA_TRACE_DECLARE(bwd)
 
 namespace kata {
 
@@ -49,16 +59,14 @@ constexpr int kBwStages = 4;
 constexpr uint32_t kBwTmemCols = 512;
 
 // ---------------------------------------------------------------------------
-// 1. dN' = 2 dO / D rounded to bf16 and dD' = -2 (dO . o) / D per row; a row
-//    with D = 0 (output constant 0) gets 0 for both.  The factor 2 of
-//    dS = 2 S (dP + dD) is folded in here (scaling by 2 is exact), so that
-//    dS = S (dN' . v + dD'); the dV accumulator, built from dN', is halved in
-//    its epilogue.  One warp per row of 64 values, two per lane.
+// 1. Per row: (-delta_t, r_t) with delta_t = dO_t . o_t and r_t = 1 / D_t, both
+//    fp32; a row with D_t = 0 (output constant 0) gets r_t = 0, so it passes
+//    no gradient.  One warp per row of 64 values, two per lane.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __restrict__ dO,
+__global__ void __launch_bounds__(256) bwd_rows_kernel(const __nv_bfloat16* __restrict__ dO,
                                                        const __nv_bfloat16* __restrict__ o,
-                                                       const float* __restrict__ D, __nv_bfloat16* __restrict__ dN,
-                                                       float* __restrict__ dD, long long rows) {
+                                                       const float* __restrict__ D, float2* __restrict__ rowc,
+                                                       long long rows) {
   const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
@@ -68,23 +76,20 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __re
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
   const float d = D[row];
-  const float inv = d > 0.f ? 1.f / d : 0.f;
-  reinterpret_cast<__nv_bfloat162*>(dN + row * kBwDV)[lane] =
-      __floats2bfloat162_rn(2.f * (a.x * inv), 2.f * (a.y * inv));
-  if (lane == 0) dD[row] = -2.f * (dot * inv);
+  if (lane == 0) rowc[row] = make_float2(-dot, d > 0.f ? 1.f / d : 0.f);
 }
 
 template <int p>
 struct BwCfg {
   static constexpr int kQKBytes = kBw * p * 2;         // a Q or K tile
-  static constexpr int kVBytes = kBw * kBwDV * 2;      // a V or dN tile
+  static constexpr int kVBytes = kBw * kBwDV * 2;      // a V or dO tile
   static constexpr Swizzle kQKSw = p == 16 ? kSw32 : kSw64;
   // 8-row group stride: K-major rows of the Q/K tile, or 8 reduction rows
   // when the same tile is read MN-major
   static constexpr uint32_t kQKSbo = 8 * p * 2;
   static constexpr uint32_t kVSbo = 8 * kBwDV * 2;
   static constexpr uint32_t kQKKStep = 16 * p * 2;     // 16 rows of a Q/K tile read MN-major
-  static constexpr uint32_t kVKStep = 16 * kBwDV * 2;  // 16 rows of a V/dN tile read MN-major
+  static constexpr uint32_t kVKStep = 16 * kBwDV * 2;  // 16 rows of a V/dO tile read MN-major
   // TMEM columns
   static constexpr uint32_t colS = 0;                  // S or S^T, fp32
   static constexpr uint32_t colP = 128;                // dP or dP^T, fp32
@@ -92,21 +97,24 @@ struct BwCfg {
   static constexpr uint32_t colAcc = 384;              // dQ (p) or dV (64) then dK (p)
 };
 
-// Gradient weights (and, with kW, squares) of 16 columns of one row, half
-// HF of the row's 32, on fp32 pairs: s, d are the 16 scores and dP' values;
-// the dD' term is ddr for every column, or, with kCol, dd[x] for columns
-// 2x, 2x + 1.  g[8 HF + x] receives the bf16 pair of dS = s (dP' + dD'),
-// w[8 HF + x] that of s^2.  With kMask, column c (0..31 in the row's 32) is
-// kept only when kGE ? c >= lane : c <= lane, and is 0 otherwise.
+// Gradient weights (and, with kW, scaled squares) of 16 columns of one row,
+// half HF of the row's 32, on fp32 pairs: s, d are the 16 scores and dP
+// values; the row constants (-delta, r) of column c are rc for every column,
+// or, with kCol, cc[x] = (-delta, r of column 2x, -delta, r of column 2x + 1).
+// g[8 HF + x] receives the bf16 pair of dS = 2 (s r) (dP - delta) for
+// columns 2x, 2x + 1, w[8 HF + x] that of s (s r).  With kMask, column c
+// (0..31 in the row's 32) is kept only when kGE ? c >= lane : c <= lane.
 template <int HF, bool kW, bool kCol, bool kMask, bool kGE>
-__device__ __forceinline__ void grad_pairs(const uint32_t (&s)[16], const uint32_t (&d)[16], const float2* dd,
-                                           float ddr, int lane, uint32_t (&g)[16], uint32_t (&w)[16]) {
+__device__ __forceinline__ void grad_pairs(const uint32_t (&s)[16], const uint32_t (&d)[16], const float4* cc,
+                                           float2 rc, int lane, uint32_t (&g)[16], uint32_t (&w)[16]) {
 #pragma unroll
   for (int x = 0; x < 8; ++x) {
-    const float2 e = kCol ? dd[x] : make_float2(ddr, ddr);
+    const float4 e = kCol ? cc[x] : make_float4(rc.x, rc.y, rc.x, rc.y);
     const uint64_t s2 = f32x2(s[2 * x], s[2 * x + 1]);
-    const uint64_t gg = f32x2_mul(s2, f32x2_add(f32x2(d[2 * x], d[2 * x + 1]),
-                                                f32x2(__float_as_uint(e.x), __float_as_uint(e.y))));
+    const uint64_t t = f32x2_add(f32x2(d[2 * x], d[2 * x + 1]), f32x2(__float_as_uint(e.x), __float_as_uint(e.z)));
+    const uint64_t u = f32x2_mul(s2, f32x2(__float_as_uint(e.y), __float_as_uint(e.w)));
+    uint64_t gg = f32x2_mul(u, t);
+    gg = f32x2_add(gg, gg);
     float g0 = f32x2_lo(gg), g1 = f32x2_hi(gg);
     if (kMask) {
       const int c = 16 * HF + 2 * x;
@@ -115,7 +123,7 @@ __device__ __forceinline__ void grad_pairs(const uint32_t (&s)[16], const uint32
     }
     g[8 * HF + x] = pack_bf16x2(g0, g1);
     if (kW) {
-      const uint64_t ww = f32x2_mul(s2, s2);
+      const uint64_t ww = f32x2_mul(s2, u);
       float w0 = f32x2_lo(ww), w1 = f32x2_hi(ww);
       if (kMask) {
         const int c = 16 * HF + 2 * x;
@@ -147,8 +155,8 @@ __device__ __forceinline__ void store_row16(__nv_bfloat16* dst_row, const uint32
 template <int p>
 struct DqSmem {
   using C = BwCfg<p>;
-  static constexpr int offDN = 0;                                       // 2 buffers of dN_i (SW128)
-  static constexpr int offQ = offDN + 2 * C::kVBytes;                   // 2 buffers of Q_i
+  static constexpr int offDO = 0;                                       // 2 buffers of dO_i (SW128)
+  static constexpr int offQ = offDO + 2 * C::kVBytes;                   // 2 buffers of Q_i
   static constexpr int offK = (offQ + 2 * C::kQKBytes + 1023) / 1024 * 1024;  // ring of K_j
   static constexpr int offV = (offK + kBwStages * C::kQKBytes + 1023) / 1024 * 1024;  // ring of V_j
   static constexpr int offBar = offV + kBwStages * C::kVBytes;
@@ -160,14 +168,14 @@ struct DqSmem {
 template <int p>
 __global__ void __launch_bounds__(kBwThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_dn,
-                  const float* __restrict__ dD, __nv_bfloat16* __restrict__ dq, int T, int BH, WaitCtl wc) {
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                  const float2* __restrict__ rowc, __nv_bfloat16* __restrict__ dq, int T, int BH, WaitCtl wc) {
   using C = BwCfg<p>;
   using L = DqSmem<p>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::offBar);
-  uint64_t* q_full = bars;                      // [2] Q_i and dN_i landed
+  uint64_t* q_full = bars;                      // [2] Q_i and dO_i landed
   uint64_t* q_empty = q_full + 2;               // [2]
   uint64_t* kv_full = q_empty + 2;              // [kBwStages]
   uint64_t* kv_empty = kv_full + kBwStages;     // [kBwStages]
@@ -220,7 +228,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
-      prefetch_tmap(&tm_dn);
+      prefetch_tmap(&tm_do);
       int nq = 0;
       long rg = 0;  // key tiles loaded (ring position)
       bool ok = true;
@@ -228,7 +236,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         const int tile = item_tile(it), bh = it % BH, qb = nq & 1;
         if (!mbar_wait(q_empty + qb, ((nq >> 1) & 1) ^ 1, env)) break;
         mbar_arrive_expect_tx(q_full + qb, C::kVBytes + C::kQKBytes);
-        tma_load_3d(smem + L::offDN + qb * C::kVBytes, &tm_dn, q_full + qb, 0, tile * kBw, bh);
+        tma_load_3d(smem + L::offDO + qb * C::kVBytes, &tm_do, q_full + qb, 0, tile * kBw, bh);
         tma_load_3d(smem + L::offQ + qb * C::kQKBytes, &tm_q, q_full + qb, 0, tile * kBw, bh);
         for (int j = 0; j <= tile; ++j, ++rg) {
           const int st = (int)(rg % kBwStages);
@@ -250,10 +258,10 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     constexpr uint32_t id_s = idesc_bf16(kBw, kBw, false, false);  // both operands K-major
     constexpr uint32_t id_dq = idesc_bf16(kBw, p, false, true);    // A = dS (TMEM), B = K_j MN-major
     const uint64_t dq0 = smem_desc(smem_u32(smem + L::offQ), 16, C::kQKSbo, C::kQKSw);
-    const uint64_t ddn0 = smem_desc(smem_u32(smem + L::offDN), 16, C::kVSbo, kSw128);
+    const uint64_t ddn0 = smem_desc(smem_u32(smem + L::offDO), 16, C::kVSbo, kSw128);
     const uint64_t dk0 = smem_desc(smem_u32(smem + L::offK), 16, C::kQKSbo, C::kQKSw);
     const uint64_t dv0 = smem_desc(smem_u32(smem + L::offV), 16, C::kVSbo, kSw128);
-    // S = Q K_j^T (K = p) and dP' = dN' V_j^T (K = dv): query buffer qb, key stage st
+    // S = Q K_j^T (K = p) and dP = dO V_j^T (K = dv): query buffer qb, key stage st
     auto issue_sdp = [&](int qb, int st) {
 #pragma unroll
       for (int ks = 0; ks < p / 16; ++ks)
@@ -326,7 +334,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     for (int it = my_item(nq); ok && it >= 0; it = my_item(++nq)) {
       const int tile = item_tile(it), bh = it % BH, nkv = tile + 1;
       const int row = tile * kBw + quarter * 32 + lane;
-      const float dDr = row < T ? dD[(size_t)bh * T + row] : 0.f;
+      const float2 rc = row < T ? rowc[(size_t)bh * T + row] : make_float2(0.f, 0.f);  // (-delta, 1/D)
       for (int j = 0; j < nkv; ++j) {
         const int g = gs + j;
         if (!mbar_wait(s_full, g & 1, env)) {
@@ -348,16 +356,16 @@ __global__ void __launch_bounds__(kBwThreads, 1)
           tmem_ld16(lane_base + C::colP + 32 * kq, d);
           tmem_wait_ld();
           if (part)
-            grad_pairs<0, false, false, true, false>(s, d, nullptr, dDr, lane, gr, unused);
+            grad_pairs<0, false, false, true, false>(s, d, nullptr, rc, lane, gr, unused);
           else
-            grad_pairs<0, false, false, false, false>(s, d, nullptr, dDr, lane, gr, unused);
+            grad_pairs<0, false, false, false, false>(s, d, nullptr, rc, lane, gr, unused);
           tmem_ld16(lane_base + C::colS + 32 * kq + 16, s);
           tmem_ld16(lane_base + C::colP + 32 * kq + 16, d);
           tmem_wait_ld();
           if (part)
-            grad_pairs<1, false, false, true, false>(s, d, nullptr, dDr, lane, gr, unused);
+            grad_pairs<1, false, false, true, false>(s, d, nullptr, rc, lane, gr, unused);
           else
-            grad_pairs<1, false, false, false, false>(s, d, nullptr, dDr, lane, gr, unused);
+            grad_pairs<1, false, false, false, false>(s, d, nullptr, rc, lane, gr, unused);
         }
         // S and dP' are in registers: the next key tile's may overwrite them
         tc_fence_before();
@@ -403,10 +411,10 @@ struct DkvSmem {
   using C = BwCfg<p>;
   static constexpr int offV = 0;                                        // 2 buffers of V_j (SW128)
   static constexpr int offK = offV + 2 * C::kVBytes;                    // 2 buffers of K_j
-  static constexpr int offDN = (offK + 2 * C::kQKBytes + 1023) / 1024 * 1024;  // ring of dN_i
-  static constexpr int offQ = offDN + kBwStages * C::kVBytes;           // ring of Q_i
-  static constexpr int offDD = offQ + kBwStages * C::kQKBytes;          // dD' of 32 queries per weight warp
-  static constexpr int offBar = (offDD + 16 * 32 * 4 + 1023) / 1024 * 1024;
+  static constexpr int offDO = (offK + 2 * C::kQKBytes + 1023) / 1024 * 1024;  // ring of dO_i
+  static constexpr int offQ = offDO + kBwStages * C::kVBytes;           // ring of Q_i
+  static constexpr int offDD = offQ + kBwStages * C::kQKBytes;          // (-delta, 1/D) of 32 queries per weight warp
+  static constexpr int offBar = (offDD + 16 * 32 * 8 + 1023) / 1024 * 1024;
   static constexpr int kBars = 4 + 2 * kBwStages + 7;
   static constexpr int offMisc = offBar + kBars * 8;
   static constexpr int kBytes = offMisc + 16 + 1024;
@@ -415,8 +423,8 @@ struct DkvSmem {
 template <int p>
 __global__ void __launch_bounds__(kBwThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_dn,
-                    const float* __restrict__ dD, __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                    const float2* __restrict__ rowc, __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
                     int T, int BH, WaitCtl wc) {
   using C = BwCfg<p>;
   using L = DkvSmem<p>;
@@ -425,7 +433,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::offBar);
   uint64_t* kv_full = bars;                     // [2] K_j and V_j landed
   uint64_t* kv_empty = kv_full + 2;             // [2]
-  uint64_t* q_full = kv_empty + 2;              // [kBwStages] Q_i and dN_i
+  uint64_t* q_full = kv_empty + 2;              // [kBwStages] Q_i and dO_i
   uint64_t* q_empty = q_full + kBwStages;       // [kBwStages]
   uint64_t* s_full = q_empty + kBwStages;       // S^T and dP^T of a query tile in TMEM
   uint64_t* s_read = s_full + 1;                // ... loaded by the weight warps (512)
@@ -438,6 +446,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::offMisc + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  KATA_TRACE_BEGIN(bwd);
   const int n_tiles = (T + kBw - 1) / kBw;
   const int n_items = n_tiles * BH;
   // item it: key tile it / BH (tile 0 has the most query tiles), head it % BH;
@@ -479,7 +488,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
-      prefetch_tmap(&tm_dn);
+      prefetch_tmap(&tm_do);
       int nq = 0;
       long rg = 0;  // query tiles loaded (ring position)
       bool ok = true;
@@ -496,7 +505,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
             break;
           }
           mbar_arrive_expect_tx(q_full + st, C::kVBytes + C::kQKBytes);
-          tma_load_3d(smem + L::offDN + st * C::kVBytes, &tm_dn, q_full + st, 0, i * kBw, bh);
+          tma_load_3d(smem + L::offDO + st * C::kVBytes, &tm_do, q_full + st, 0, i * kBw, bh);
           tma_load_3d(smem + L::offQ + st * C::kQKBytes, &tm_q, q_full + st, 0, i * kBw, bh);
         }
       }
@@ -507,13 +516,13 @@ __global__ void __launch_bounds__(kBwThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
     constexpr uint32_t id_s = idesc_bf16(kBw, kBw, false, false);
-    constexpr uint32_t id_dv = idesc_bf16(kBw, kBwDV, false, true);  // A = W^T (TMEM), B = dN_i MN-major
+    constexpr uint32_t id_dv = idesc_bf16(kBw, kBwDV, false, true);  // A = W^T (TMEM), B = dO_i MN-major
     constexpr uint32_t id_dk = idesc_bf16(kBw, p, false, true);      // A = dS^T (TMEM), B = Q_i MN-major
     const uint64_t dk0 = smem_desc(smem_u32(smem + L::offK), 16, C::kQKSbo, C::kQKSw);
     const uint64_t dv0 = smem_desc(smem_u32(smem + L::offV), 16, C::kVSbo, kSw128);
     const uint64_t dq0 = smem_desc(smem_u32(smem + L::offQ), 16, C::kQKSbo, C::kQKSw);
-    const uint64_t ddn0 = smem_desc(smem_u32(smem + L::offDN), 16, C::kVSbo, kSw128);
-    // S^T = K Q_i^T (K = p) and dP^T = V dN_i^T (K = dv): key buffer kb, query stage st
+    const uint64_t ddn0 = smem_desc(smem_u32(smem + L::offDO), 16, C::kVSbo, kSw128);
+    // S^T = K Q_i^T (K = p) and dP^T = V dO_i^T (K = dv): key buffer kb, query stage st
     auto issue_sdp = [&](int kb, int st) {
 #pragma unroll
       for (int ks = 0; ks < p / 16; ++ks)
@@ -538,6 +547,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       }
       tc_fence_after();
       issue_sdp(kb, (int)(gs % kBwStages));
+      KATA_TRACE(bwd, gs, 0);
       for (int n = 0; n < cnt; ++n) {
         const int g = gs + n;
         const int st = g % kBwStages;
@@ -550,11 +560,13 @@ __global__ void __launch_bounds__(kBwThreads, 1)
           }
           tc_fence_after();
           issue_sdp(kb, (int)((g + 1) % kBwStages));
+          KATA_TRACE(bwd, g + 1, 0);
         }
         if (!mbar_wait_w(p_full, (int)(g & 1), env)) {
           ok = false;
           break;
         }
+        KATA_TRACE(bwd, g, 1);
         // the item's first dV / dK overwrite the accumulators: the previous
         // item's epilogue must have read them
         if (n == 0 && acc_cnt > 0 && !mbar_wait_w(acc_free, (acc_cnt - 1) & 1, env)) {
@@ -572,6 +584,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
                    desc_add(dq0, st * C::kQKBytes + ks * C::kQKKStep), id_dk, (n > 0 || ks > 0) ? 1u : 0u);
         mma_commit_w(w_free);
         mma_commit_w(q_empty + st);
+        KATA_TRACE(bwd, g, 2);
       }
       if (!ok) break;
       mma_commit_w(acc_full);
@@ -586,8 +599,9 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     const int quarter = warp % 4;                 // rows (keys) 32 quarter ..
     const int kq = (warp - 2) / 4;                // queries 32 kq .. of the query tile
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-    float* dd_slot = reinterpret_cast<float*>(smem + L::offDD) + (warp - 2) * 32;
-    const float2* dd_pairs = reinterpret_cast<const float2*>(dd_slot);
+    float2* dd_slot = reinterpret_cast<float2*>(smem + L::offDD) + (warp - 2) * 32;
+    const int tslot = (warp == 2 && lane == 0) ? 5 : (warp == 17 && lane == 0) ? 9 : -1;  // traced warps
+    const float4* dd_pairs = reinterpret_cast<const float4*>(dd_slot);
     int gs = 0;
     int nq = 0, acc_cnt = 0;
     bool ok = true;
@@ -595,13 +609,14 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       const int tile = it / BH, bh = it % BH, cnt = n_tiles - tile;
       for (int n = 0; n < cnt; ++n) {
         const int g = gs + n;
-        // dD of this warp's 32 queries, one per lane (0 past T)
+        // (-delta, 1/D) of this warp's 32 queries, one per lane (0 past T)
         const int qrow = (tile + n) * kBw + 32 * kq + lane;
-        const float dDl = qrow < T ? dD[(size_t)bh * T + qrow] : 0.f;
+        const float2 rcl = qrow < T ? rowc[(size_t)bh * T + qrow] : make_float2(0.f, 0.f);
         if (!mbar_wait(s_full, (int)(g & 1), env)) {
           ok = false;
           break;
         }
+        if (tslot >= 0) KATA_TRACE(bwd, g, tslot);
         tc_fence_after();
         // causal mask on the diagonal tile: query 32 kq + c >= key 32 quarter + lane
         const bool diag = (n == 0);
@@ -612,39 +627,42 @@ __global__ void __launch_bounds__(kBwThreads, 1)
 #pragma unroll
           for (int x = 0; x < 16; ++x) gr[x] = w[x] = 0u;
         } else {
-          // the 32 dD' values, read back as column pairs (a broadcast per pair)
+          // the 32 queries' constants, read back as column pairs (a broadcast per pair)
           __syncwarp();
-          dd_slot[lane] = dDl;
+          dd_slot[lane] = rcl;
           __syncwarp();
           uint32_t s[16], d[16];
           tmem_ld16(lane_base + C::colS + 32 * kq, s);
           tmem_ld16(lane_base + C::colP + 32 * kq, d);
           tmem_wait_ld();
           if (part)
-            grad_pairs<0, true, true, true, true>(s, d, dd_pairs, 0.f, lane, gr, w);
+            grad_pairs<0, true, true, true, true>(s, d, dd_pairs, make_float2(0.f, 0.f), lane, gr, w);
           else
-            grad_pairs<0, true, true, false, true>(s, d, dd_pairs, 0.f, lane, gr, w);
+            grad_pairs<0, true, true, false, true>(s, d, dd_pairs, make_float2(0.f, 0.f), lane, gr, w);
           tmem_ld16(lane_base + C::colS + 32 * kq + 16, s);
           tmem_ld16(lane_base + C::colP + 32 * kq + 16, d);
           tmem_wait_ld();
           if (part)
-            grad_pairs<1, true, true, true, true>(s, d, dd_pairs + 8, 0.f, lane, gr, w);
+            grad_pairs<1, true, true, true, true>(s, d, dd_pairs + 8, make_float2(0.f, 0.f), lane, gr, w);
           else
-            grad_pairs<1, true, true, false, true>(s, d, dd_pairs + 8, 0.f, lane, gr, w);
+            grad_pairs<1, true, true, false, true>(s, d, dd_pairs + 8, make_float2(0.f, 0.f), lane, gr, w);
         }
         tc_fence_before();
         mbar_arrive(s_read);
+        if (tslot >= 0) KATA_TRACE(bwd, g, tslot + 1);
         // the operand buffers are read by the previous query tile's MMAs
         if (g > 0 && !mbar_wait(w_free, (int)((g - 1) & 1), env)) {
           ok = false;
           break;
         }
+        if (tslot >= 0) KATA_TRACE(bwd, g, tslot + 2);
         tc_fence_after();
         tmem_st16(lane_base + C::colA(0) + 16 * kq, w);
         tmem_st16(lane_base + C::colA(1) + 16 * kq, gr);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(p_full);
+        if (tslot >= 0) KATA_TRACE(bwd, g, tslot + 3);
       }
       if (!ok || !mbar_wait(acc_full, acc_cnt & 1, env)) break;
       ++acc_cnt;
@@ -660,9 +678,6 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(acc_free);
-      // dV was accumulated from dN' = 2 dO / D: halve it (exact)
-#pragma unroll
-      for (int x = 0; x < 16; ++x) rv[x] = __float_as_uint(0.5f * __uint_as_float(rv[x]));
       const int row = tile * kBw + quarter * 32 + lane;  // this thread's key
       if (row < T) {
         const size_t r0 = (size_t)bh * T + row;
@@ -688,16 +703,15 @@ template <int p>
 static cudaError_t launch_bwd_t(const void* q, const void* k, const void* v, const void* o, const float* D,
                                 const void* dO, void* dq, void* dk, void* dv, int BH, int T, void* ws,
                                 const WaitCtl& wc, cudaStream_t st) {
-  __nv_bfloat16* dN = static_cast<__nv_bfloat16*>(ws);
-  float* dD = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + (size_t)BH * T * kBwDV * 2);
+  float2* rowc = static_cast<float2*>(ws);
   const long long rows = (long long)BH * T;
-  bwd_prep_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(dO),
-                                                                 static_cast<const __nv_bfloat16*>(o), D, dN, dD, rows);
+  bwd_rows_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(dO),
+                                                                 static_cast<const __nv_bfloat16*>(o), D, rowc, rows);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  CUtensorMap tq, tk, tv, tdn;
+  CUtensorMap tq, tk, tv, tdo;
   if (!make_tmap_bf16(&tq, q, p, T, BH, kBw) || !make_tmap_bf16(&tk, k, p, T, BH, kBw) ||
-      !make_tmap_bf16(&tv, v, kBwDV, T, BH, kBw) || !make_tmap_bf16(&tdn, dN, kBwDV, T, BH, kBw))
+      !make_tmap_bf16(&tv, v, kBwDV, T, BH, kBw) || !make_tmap_bf16(&tdo, dO, kBwDV, T, BH, kBw))
     return cudaErrorInvalidValue;
   const dim3 grid((T + kBw - 1) / kBw, BH);
   auto kq = bwd_dq_kernel<p>;
@@ -714,9 +728,9 @@ static cudaError_t launch_bwd_t(const void* q, const void* k, const void* v, con
   }
   const long items = (long)grid.x * BH;
   const int pgrid = (int)(items < num_sms ? items : num_sms);
-  kq<<<pgrid, kBwThreads, DqSmem<p>::kBytes, st>>>(tq, tk, tv, tdn, dD, static_cast<__nv_bfloat16*>(dq), T, BH, wc);
+  kq<<<pgrid, kBwThreads, DqSmem<p>::kBytes, st>>>(tq, tk, tv, tdo, rowc, static_cast<__nv_bfloat16*>(dq), T, BH, wc);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  kkv<<<pgrid, kBwThreads, DkvSmem<p>::kBytes, st>>>(tq, tk, tv, tdn, dD, static_cast<__nv_bfloat16*>(dk),
+  kkv<<<pgrid, kBwThreads, DkvSmem<p>::kBytes, st>>>(tq, tk, tv, tdo, rowc, static_cast<__nv_bfloat16*>(dk),
                                                       static_cast<__nv_bfloat16*>(dv), T, BH, wc);
   return cudaGetLastError();
 }
@@ -724,7 +738,8 @@ static cudaError_t launch_bwd_t(const void* q, const void* k, const void* v, con
 }  // namespace
 
 size_t flash_bwd_workspace_bytes(int BH, int T, int dv) {
-  return (size_t)BH * T * dv * 2 + (size_t)BH * T * 4;
+  (void)dv;
+  return (size_t)BH * T * sizeof(float2);  // (-delta, 1/D) per row
 }
 
 cudaError_t launch_flash_bwd_sm100(const void* q, const void* k, const void* v, const void* o, const float* D,

@@ -155,10 +155,10 @@ def test_training_entry_points_reject_bad_arguments(L):
     assert f(a, b, c, d, _fake(0x50004), 1, 1, 16, 16, 64, 1, st) == _abi.KATA_ERR_MISALIGNED
     assert f(a, b, c, d, D, 1, 1, 0, 16, 64, 1, st) == _abi.KATA_OK
     ws_size = _abi.lib().kata_bwd_quadratic_workspace_size
-    assert ws_size(2, 3, 100, 16, 64, 1) == 2 * 3 * 100 * (64 * 2 + 4)
+    assert ws_size(2, 3, 100, 16, 64, 1) == 2 * 3 * 100 * 8
     assert ws_size(2, 3, 100, 16, 64, 0) == 0 and ws_size(1, 1, 0, 16, 64, 1) == 0
     g = L.kata_bwd_quadratic  # q k v o D dO dq dk dv B H T p dv dtype ws bytes stream
-    n = 1 * 1 * 16 * (64 * 2 + 4)
+    n = 1 * 1 * 16 * 8
     assert g(a, b, c, d, D, dO, gq, gk, gv, 1, 1, 16, 24, 64, 1, ws, n, st) == _abi.KATA_ERR_UNSUPPORTED
     assert g(a, b, c, d, D, None, gq, gk, gv, 1, 1, 16, 16, 64, 1, ws, n, st) == _abi.KATA_ERR_INVALID_ARG
     assert g(a, b, c, d, D, dO, gq, gk, gv, 1, 1, 16, 16, 64, 1, ws, n - 1, st) == _abi.KATA_ERR_WORKSPACE

@@ -123,3 +123,26 @@ def test_backward_full_size_sampled_heads(kata):
         gq, gk, gv = obw.backward(q[sl], k[sl], v[sl], dO[sl])
         errs = (_grad_err(dq[sl], gq), _grad_err(dk[sl], gk), _grad_err(dv[sl], gv))
         assert max(errs) <= GRAD_TOL, (b, h, errs)
+
+
+def test_backward_with_tiny_denominators(kata):
+    """Rows whose query is nearly orthogonal to every key seen so far have a
+    tiny D_t; their gradient terms scale with 1/D_t and cancel (o_t is almost
+    a single value vector).  Query 0 of each head is made nearly orthogonal
+    to key 0 (D_0 ~ 1e-6), and query 5 nearly orthogonal to keys 0..5."""
+    B, H, T, p = 1, 2, 300, 16
+    q, k, v = workloads.normal_qkv(B, H, T, p, 64, seed=0, dtype="bf16")
+    rng = np.random.default_rng(450)
+    for h in range(H):
+        for t in (0, 5):
+            K0 = k[0, h, :t + 1].astype(np.float64)
+            x = rng.standard_normal(p)
+            x -= K0.T @ np.linalg.lstsq(K0.T, x, rcond=None)[0]   # orthogonal to keys 0..t
+            x = x / np.linalg.norm(x) + 1e-3 * K0[0] / np.linalg.norm(K0[0])
+            q[0, h, t] = workloads.round_bf16((x / np.linalg.norm(x)).astype(np.float32))
+    dO = _dO(v.shape, 451)
+    _, D, dq, dk, dv = _run(kata, q, k, v, dO)
+    assert D[0, :, 0].max() < 1e-4
+    gq, gk, gv = obw.backward(q, k, v, dO)
+    errs = (_grad_err(dq, gq), _grad_err(dk, gk), _grad_err(dv, gv))
+    assert max(errs) <= GRAD_TOL, errs
