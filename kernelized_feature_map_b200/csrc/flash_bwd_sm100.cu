@@ -59,9 +59,11 @@ constexpr int kBwStages = 4;
 constexpr uint32_t kBwTmemCols = 512;
 
 // ---------------------------------------------------------------------------
-// 1. Per row: (-delta_t, r_t) with delta_t = dO_t . o_t and r_t = 1 / D_t, both
-//    fp32; a row with D_t = 0 (output constant 0) gets r_t = 0, so it passes
-//    no gradient.  One warp per row of 64 values, two per lane.
+// 1. Per row: (-delta_t, r_t) with delta_t = dO_t . o_t and r_t = 2 / D_t, both
+//    fp32 (the factor 2 of dS is folded into r; the dV accumulator, which
+//    gets it too, is halved in its epilogue -- exact); a row with D_t = 0
+//    (output constant 0) gets r_t = 0, so it passes no gradient.  One warp
+//    per row of 64 values, two per lane.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) bwd_rows_kernel(const __nv_bfloat16* __restrict__ dO,
                                                        const __nv_bfloat16* __restrict__ o,
@@ -76,7 +78,7 @@ __global__ void __launch_bounds__(256) bwd_rows_kernel(const __nv_bfloat16* __re
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
   const float d = D[row];
-  if (lane == 0) rowc[row] = make_float2(-dot, d > 0.f ? 1.f / d : 0.f);
+  if (lane == 0) rowc[row] = make_float2(-dot, d > 0.f ? 2.f / d : 0.f);
 }
 
 template <int p>
@@ -101,8 +103,9 @@ struct BwCfg {
 // half HF of the row's 32, on fp32 pairs: s, d are the 16 scores and dP
 // values; the row constants (-delta, r) of column c are rc for every column,
 // or, with kCol, cc[x] = (-delta, r of column 2x, -delta, r of column 2x + 1).
-// g[8 HF + x] receives the bf16 pair of dS = 2 (s r) (dP - delta) for
-// columns 2x, 2x + 1, w[8 HF + x] that of s (s r).  With kMask, column c
+// g[8 HF + x] receives the bf16 pair of dS = (s r) (dP - delta) for
+// columns 2x, 2x + 1, w[8 HF + x] that of s (s r) (with r = 2 / D: twice the
+// weight the dV product needs).  With kMask, column c
 // (0..31 in the row's 32) is kept only when kGE ? c >= lane : c <= lane.
 template <int HF, bool kW, bool kCol, bool kMask, bool kGE>
 __device__ __forceinline__ void grad_pairs(const uint32_t (&s)[16], const uint32_t (&d)[16], const float4* cc,
@@ -113,8 +116,7 @@ __device__ __forceinline__ void grad_pairs(const uint32_t (&s)[16], const uint32
     const uint64_t s2 = f32x2(s[2 * x], s[2 * x + 1]);
     const uint64_t t = f32x2_add(f32x2(d[2 * x], d[2 * x + 1]), f32x2(__float_as_uint(e.x), __float_as_uint(e.z)));
     const uint64_t u = f32x2_mul(s2, f32x2(__float_as_uint(e.y), __float_as_uint(e.w)));
-    uint64_t gg = f32x2_mul(u, t);
-    gg = f32x2_add(gg, gg);
+    const uint64_t gg = f32x2_mul(u, t);
     float g0 = f32x2_lo(gg), g1 = f32x2_hi(gg);
     if (kMask) {
       const int c = 16 * HF + 2 * x;
@@ -678,6 +680,9 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(acc_free);
+      // dV was accumulated with r = 2 / D: halve it (exact)
+#pragma unroll
+      for (int x = 0; x < 16; ++x) rv[x] = __float_as_uint(0.5f * __uint_as_float(rv[x]));
       const int row = tile * kBw + quarter * 32 + lane;  // this thread's key
       if (row < T) {
         const size_t r0 = (size_t)bh * T + row;
