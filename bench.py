@@ -90,7 +90,7 @@ def load_peaks():
 
 
 # ---------------------------------------------------------------------------
-# algorithmic work per launch (the per-unit figures are stated in the design doc)
+# algorithmic work per launch: flops per causal pair, bytes per token-head
 # ---------------------------------------------------------------------------
 def flash_flops(BH, T, p, dv):
     """Causal-useful tensor flops: 2 (p + dv) per (query, key<=query) pair."""

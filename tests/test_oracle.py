@@ -53,7 +53,8 @@ def test_zero_denominator_reading(fn):
     np.testing.assert_array_equal(o, o_expected)
 
 
-# ---------------------------------------------------------------------------
+# four identities that follow from the definition: direct = recurrent, o_1 = v_1,
+# the convex-gate bounds, identical keys give the running mean
 # the four spec identities
 # ---------------------------------------------------------------------------
 
