@@ -146,3 +146,17 @@ def test_backward_with_tiny_denominators(kata):
     gq, gk, gv = obw.backward(q, k, v, dO)
     errs = (_grad_err(dq, gq), _grad_err(dk, gk), _grad_err(dv, gv))
     assert max(errs) <= GRAD_TOL, errs
+
+
+def test_backward_many_items_ragged(kata):
+    """More (tile, head) items than SMs, so every persistent CTA walks several
+    items, with a ragged last tile (T = 1000); whole heads compared."""
+    B, H, T, p = 4, 16, 1000, 16
+    q, k, v = workloads.normal_qkv(B, H, T, p, 64, seed=460, dtype="bf16")
+    dO = _dO(v.shape, 461)
+    _, _, dq, dk, dv = _run(kata, q, k, v, dO)
+    for (b, h) in [(0, 0), (1, 9), (3, 15)]:
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        gq, gk, gv = obw.backward(q[sl], k[sl], v[sl], dO[sl])
+        errs = (_grad_err(dq[sl], gq), _grad_err(dk[sl], gk), _grad_err(dv[sl], gv))
+        assert max(errs) <= GRAD_TOL, (b, h, errs)

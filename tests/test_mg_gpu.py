@@ -149,3 +149,18 @@ def test_mg_pages_call_shape(kata):
     torch.cuda.synchronize()
     assert tuple(o.shape) == (B, T, H, D)
     assert row_rel_err(_bthd(to_np(o)), oracle.direct_mg(q, k, v, 2), v) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("g", [2, 4])
+def test_mg_many_items_ragged(kata, g):
+    """More query-tile items than SMs with a ragged last tile (T = 1000):
+    every persistent CTA walks several items; sampled rows against the oracle."""
+    B, H, T, d, dv = 4, 16, 1000, 64, 64
+    q, k, v = workloads.normal_qkv(B, H, T, d, dv, seed=470 + g, dtype="bf16")
+    got = _run_mg(kata, q, k, v, g, "bthd")
+    rng = np.random.default_rng(471)
+    bh = rng.integers(0, B * H, size=64)
+    t = np.concatenate([rng.integers(0, T, size=56), [0, 127, 128, 895, 896, 998, 999, 500]])
+    ref = oracle.direct_mg_rows(q, k, v, g, bh, t)
+    vmax = np.abs(v.reshape(B * H, -1)).max(axis=1)[bh]
+    assert rows_rel_err(got.reshape(B * H, T, dv)[bh, t], ref, vmax) <= TOL["bf16"]
