@@ -57,3 +57,52 @@ def backward(q, k, v, dO):
     dq = np.einsum("bhts,bhsp->bhtp", dS, k)
     dk = np.einsum("bhts,bhtp->bhsp", dS, q)
     return dq, dk, dv
+
+
+def forward_mg_with_d(q, k, v, groups: int):
+    """KATA-Mg forward (g PSD factors over a head of width d, weight
+    sum_j (q_t^j . k_s^j)^2) with its denominators, fp64, T x T matrices."""
+    q, k, v = (np.asarray(x, np.float64) for x in (q, k, v))
+    d = q.shape[-1]
+    p = d // groups
+    T = q.shape[2]
+    mask = np.tril(np.ones((T, T), dtype=bool))
+    W = np.zeros(q.shape[:2] + (T, T))
+    for j in range(groups):
+        Sj = np.einsum("bhtp,bhsp->bhts", q[..., j * p:(j + 1) * p], k[..., j * p:(j + 1) * p])
+        W += Sj * Sj
+    W = np.where(mask, W, 0.0)
+    N = np.einsum("bhts,bhse->bhte", W, v)
+    D = W.sum(axis=-1)
+    safe = np.where(D > 0, D, 1.0)
+    o = np.where((D > 0)[..., None], N / safe[..., None], 0.0)
+    return o, D
+
+
+def backward_mg(q, k, v, dO, groups: int):
+    """(dq, dk, dv) of the KATA-Mg forward, fp64: the single-factor chain rule
+    with w = sum_j S_j^2, so dS_j = 2 S_j dw and each group's dq^j, dk^j come
+    from its own scores."""
+    q, k, v, dO = (np.asarray(x, np.float64) for x in (q, k, v, dO))
+    d = q.shape[-1]
+    p = d // groups
+    T = q.shape[2]
+    mask = np.tril(np.ones((T, T), dtype=bool))
+    o, D = forward_mg_with_d(q, k, v, groups)
+    live = D > 0
+    safe = np.where(live, D, 1.0)
+    dN = np.where(live[..., None], dO / safe[..., None], 0.0)
+    dD = np.where(live, -np.einsum("bhte,bhte->bht", dO, o) / safe, 0.0)
+    dW = np.where(mask, np.einsum("bhte,bhse->bhts", dN, v) + dD[..., None], 0.0)
+    W = np.zeros(q.shape[:2] + (T, T))
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    for j in range(groups):
+        sl = slice(j * p, (j + 1) * p)
+        Sj = np.einsum("bhtp,bhsp->bhts", q[..., sl], k[..., sl])
+        W += np.where(mask, Sj * Sj, 0.0)
+        dSj = 2.0 * Sj * dW
+        dq[..., sl] = np.einsum("bhts,bhsp->bhtp", dSj, k[..., sl])
+        dk[..., sl] = np.einsum("bhts,bhtp->bhsp", dSj, q[..., sl])
+    dv = np.einsum("bhts,bhte->bhse", W, dN)
+    return dq, dk, dv

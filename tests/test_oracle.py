@@ -488,3 +488,34 @@ def test_backward_identities():
     q0[:, :, 7] = 0.0
     dq0, _, _ = obw.backward(q0, k, v, dO)
     assert np.all(dq0[:, :, 7] == 0.0)
+
+
+def test_backward_mg_pins():
+    """KATA-Mg gradients: g = 1 equals the single-factor gradients, the Mg
+    forward equals the C Mg oracle, and central differences of the C Mg
+    oracle match; scaling a whole query row leaves its output unchanged, so
+    q_t . dq_t = 0 row by row."""
+    q, k, v = _rand_mg(B=1, H=1, T=6, d=4, dv=2, seed=480)
+    rng = np.random.default_rng(481)
+    dO = rng.standard_normal(v.shape)
+    for a, b in zip(obw.backward_mg(q, k, v, dO, 1), obw.backward(q, k, v, dO)):
+        np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-13)
+    o, _ = obw.forward_mg_with_d(q, k, v, 2)
+    np.testing.assert_allclose(o, oracle.direct_mg(q, k, v, 2), rtol=1e-11, atol=1e-12)
+    dq, dk, dv = obw.backward_mg(q, k, v, dO, 2)
+    h = 1e-6
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        num = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            ap = {"q": q, "k": k, "v": v}
+            am = dict(ap)
+            ap[name], am[name] = xp, xm
+            num[idx] = ((oracle.direct_mg(ap["q"], ap["k"], ap["v"], 2) * dO).sum()
+                        - (oracle.direct_mg(am["q"], am["k"], am["v"], 2) * dO).sum()) / (2 * h)
+        np.testing.assert_allclose(g, num, rtol=1e-6, atol=1e-7, err_msg=name)
+    q2, k2, v2 = _rand_mg(B=1, H=2, T=30, d=8, dv=3, seed=482)
+    dq2, _, _ = obw.backward_mg(q2, k2, v2, rng.standard_normal(v2.shape), 2)
+    np.testing.assert_allclose(np.einsum("bhtd,bhtd->bht", q2, dq2), 0.0, atol=1e-9)
