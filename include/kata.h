@@ -202,6 +202,25 @@ kata_status_t kata_bwd_quadratic(const void* q, const void* k, const void* v, co
                                  void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Training with KATA-Mg ([B,H,T,*] layout, bf16, dv = 64, the (p, groups)
+ * of kata_fwd_mg_quadratic with groups > 1): the Mg forward that also saves
+ * D [B,H,T] fp32, and its backward pass.  With w = sum_j (q^j . k^j)^2 the
+ * gradient of each group's q^j, k^j is the single-factor one taken with the
+ * group's own scores and the Mg output's o and D, and dv is the sum over the
+ * groups; the backward runs the single-factor kernels once per group on the
+ * group's columns (read and written in place) and accumulates dv.  Workspace
+ * as kata_bwd_quadratic (8 bytes per row).
+ */
+kata_status_t kata_fwd_mg_quadratic_train(const void* q, const void* k, const void* v, void* o, float* D,
+                                          int B, int H, int T, int d, int groups, int dv,
+                                          kata_dtype_t dtype, void* stream);
+kata_status_t kata_bwd_mg_quadratic(const void* q, const void* k, const void* v, const void* o,
+                                    const float* D, const void* dO, void* dq, void* dk, void* dv,
+                                    int B, int H, int T, int d, int groups, int dv_width,
+                                    kata_dtype_t dtype, void* workspace, size_t workspace_bytes,
+                                    void* stream);
+
+/*
  * KATA-Mg: g PSD factors per head (arXiv abstract and gist.science sec. 2.3
  * "Varianten": several PSD factors; ai.info summary, Main Findings: state
  * d(d/g+1)/2 * dv packed, the full map at g = 1).  The head's d coordinates
@@ -267,7 +286,7 @@ void kata_set_wait_limit(long long cycles);
 /* ABI version of this header: major * 10000 + minor * 100 + patch. */
 int kata_abi_version(void);
 
-#define KATA_ABI_VERSION 10200
+#define KATA_ABI_VERSION 10300
 
 #ifdef __cplusplus
 }

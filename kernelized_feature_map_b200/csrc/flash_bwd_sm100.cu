@@ -48,6 +48,35 @@ namespace kata {
 
 bool make_tmap_bf16(CUtensorMap* map, const void* base, int inner, int T, int BH, int rows);
 
+// 3-D bf16 tensor map over rows of `inner` values that start ld values apart
+// ([B*H][T][ld], e.g. one group's columns of a [B*H, T, d] tensor), box
+// {inner, rows, 1}, swizzled over the box row.
+static bool make_tmap_bf16_ld(CUtensorMap* map, const void* base, int inner, int ld, int T, int BH, int rows) {
+  typedef CUresult (*EncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                               const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                               CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+  static EncodeFn enc = nullptr;
+  if (!enc) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &qr) != cudaSuccess ||
+        qr != cudaDriverEntryPointSuccess)
+      return false;
+    enc = reinterpret_cast<EncodeFn>(fn);
+  }
+  const int box_bytes = inner * 2;
+  const CUtensorMapSwizzle sw = box_bytes == 32   ? CU_TENSOR_MAP_SWIZZLE_32B
+                                : box_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                  : CU_TENSOR_MAP_SWIZZLE_128B;
+  const cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)T, (cuuint64_t)BH};
+  const cuuint64_t strides[2] = {(cuuint64_t)ld * 2, (cuuint64_t)ld * 2 * (cuuint64_t)T};
+  const cuuint32_t box[3] = {(cuuint32_t)inner, (cuuint32_t)rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 namespace {
 
 using namespace sm100;
@@ -171,7 +200,7 @@ template <int p>
 __global__ void __launch_bounds__(kBwThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                  const float2* __restrict__ rowc, __nv_bfloat16* __restrict__ dq, int T, int BH, WaitCtl wc) {
+                  const float2* __restrict__ rowc, __nv_bfloat16* __restrict__ dq, int T, int BH, int ld, WaitCtl wc) {
   using C = BwCfg<p>;
   using L = DqSmem<p>;
   extern __shared__ uint8_t smem_raw[];
@@ -393,8 +422,8 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       tc_fence_before();
       mbar_arrive(acc_free);
       if (kq == 0 && row < T) {
-        store_row16(dq + ((size_t)bh * T + row) * p, r0);
-        if constexpr (p == 32) store_row16(dq + ((size_t)bh * T + row) * p + 16, r1);
+        store_row16(dq + ((size_t)bh * T + row) * ld, r0);
+        if constexpr (p == 32) store_row16(dq + ((size_t)bh * T + row) * ld + 16, r1);
       }
       gs += nkv;
     }
@@ -427,7 +456,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const float2* __restrict__ rowc, __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
-                    int T, int BH, WaitCtl wc) {
+                    int T, int BH, int ld, int dv_accumulate, WaitCtl wc) {
   using C = BwCfg<p>;
   using L = DkvSmem<p>;
   extern __shared__ uint8_t smem_raw[];
@@ -686,10 +715,21 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       const int row = tile * kBw + quarter * 32 + lane;  // this thread's key
       if (row < T) {
         const size_t r0 = (size_t)bh * T + row;
-        store_row16(dv + r0 * kBwDV + 16 * kq, rv);
+        __nv_bfloat16* dvr = dv + r0 * kBwDV + 16 * kq;
+        if (dv_accumulate) {  // another group's dV is already there
+          const uint4* old = reinterpret_cast<const uint4*>(dvr);
+          const uint4 a = old[0], b = old[1];
+          const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+          for (int x = 0; x < 8; ++x) {  // bf16 -> fp32 is a 16-bit shift (exact)
+            rv[2 * x] = __float_as_uint(__uint_as_float(rv[2 * x]) + __uint_as_float(w[x] << 16));
+            rv[2 * x + 1] = __float_as_uint(__uint_as_float(rv[2 * x + 1]) + __uint_as_float(w[x] & 0xffff0000u));
+          }
+        }
+        store_row16(dvr, rv);
         if (kq == 0) {
-          store_row16(dk + r0 * p, rk0);
-          if constexpr (p == 32) store_row16(dk + r0 * p + 16, rk1);
+          store_row16(dk + r0 * ld, rk0);
+          if constexpr (p == 32) store_row16(dk + r0 * ld + 16, rk1);
         }
       }
       gs += cnt;
@@ -706,16 +746,18 @@ __global__ void __launch_bounds__(kBwThreads, 1)
 
 template <int p>
 static cudaError_t launch_bwd_t(const void* q, const void* k, const void* v, const void* o, const float* D,
-                                const void* dO, void* dq, void* dk, void* dv, int BH, int T, void* ws,
-                                const WaitCtl& wc, cudaStream_t st) {
+                                const void* dO, void* dq, void* dk, void* dv, int BH, int T, int ld, bool rows_ready,
+                                bool dv_accumulate, void* ws, const WaitCtl& wc, cudaStream_t st) {
   float2* rowc = static_cast<float2*>(ws);
   const long long rows = (long long)BH * T;
-  bwd_rows_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(dO),
-                                                                 static_cast<const __nv_bfloat16*>(o), D, rowc, rows);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  cudaError_t e = cudaSuccess;
+  if (!rows_ready) {
+    bwd_rows_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(dO),
+                                                                   static_cast<const __nv_bfloat16*>(o), D, rowc, rows);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
   CUtensorMap tq, tk, tv, tdo;
-  if (!make_tmap_bf16(&tq, q, p, T, BH, kBw) || !make_tmap_bf16(&tk, k, p, T, BH, kBw) ||
+  if (!make_tmap_bf16_ld(&tq, q, p, ld, T, BH, kBw) || !make_tmap_bf16_ld(&tk, k, p, ld, T, BH, kBw) ||
       !make_tmap_bf16(&tv, v, kBwDV, T, BH, kBw) || !make_tmap_bf16(&tdo, dO, kBwDV, T, BH, kBw))
     return cudaErrorInvalidValue;
   const dim3 grid((T + kBw - 1) / kBw, BH);
@@ -733,10 +775,12 @@ static cudaError_t launch_bwd_t(const void* q, const void* k, const void* v, con
   }
   const long items = (long)grid.x * BH;
   const int pgrid = (int)(items < num_sms ? items : num_sms);
-  kq<<<pgrid, kBwThreads, DqSmem<p>::kBytes, st>>>(tq, tk, tv, tdo, rowc, static_cast<__nv_bfloat16*>(dq), T, BH, wc);
+  kq<<<pgrid, kBwThreads, DqSmem<p>::kBytes, st>>>(tq, tk, tv, tdo, rowc, static_cast<__nv_bfloat16*>(dq), T, BH, ld,
+                                                    wc);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   kkv<<<pgrid, kBwThreads, DkvSmem<p>::kBytes, st>>>(tq, tk, tv, tdo, rowc, static_cast<__nv_bfloat16*>(dk),
-                                                      static_cast<__nv_bfloat16*>(dv), T, BH, wc);
+                                                      static_cast<__nv_bfloat16*>(dv), T, BH, ld, dv_accumulate ? 1 : 0,
+                                                      wc);
   return cudaGetLastError();
 }
 
@@ -748,10 +792,12 @@ size_t flash_bwd_workspace_bytes(int BH, int T, int dv) {
 }
 
 cudaError_t launch_flash_bwd_sm100(const void* q, const void* k, const void* v, const void* o, const float* D,
-                                  const void* dO, void* dq, void* dk, void* dv, int BH, int T, int p, void* ws,
-                                  const WaitCtl& wc, cudaStream_t st) {
-  if (p == 16) return launch_bwd_t<16>(q, k, v, o, D, dO, dq, dk, dv, BH, T, ws, wc, st);
-  if (p == 32) return launch_bwd_t<32>(q, k, v, o, D, dO, dq, dk, dv, BH, T, ws, wc, st);
+                                   const void* dO, void* dq, void* dk, void* dv, int BH, int T, int p, int ld,
+                                   bool rows_ready, bool dv_accumulate, void* ws, const WaitCtl& wc, cudaStream_t st) {
+  if (p == 16)
+    return launch_bwd_t<16>(q, k, v, o, D, dO, dq, dk, dv, BH, T, ld, rows_ready, dv_accumulate, ws, wc, st);
+  if (p == 32)
+    return launch_bwd_t<32>(q, k, v, o, D, dO, dq, dk, dv, BH, T, ld, rows_ready, dv_accumulate, ws, wc, st);
   return cudaErrorInvalidValue;
 }
 

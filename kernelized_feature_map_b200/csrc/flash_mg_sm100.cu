@@ -101,7 +101,7 @@ template <int p, int G>
 __global__ void __launch_bounds__(kMgThreads, 1)
     flash_mg_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o, int T, int BH,
-                    int H, int bthd, WaitCtl wc) {
+                    int H, int bthd, float* __restrict__ D_out, WaitCtl wc) {
   using Cfg = MgCfg<p, G>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -401,6 +401,8 @@ __global__ void __launch_bounds__(kMgThreads, 1)
       tc_fence_before();
       mbar_arrive(o_free);
       const float D = __uint_as_float(dbits);
+      // the denominator of each row, for the backward pass (optional)
+      if (D_out != nullptr && kq == 0 && row0 + lane < T) D_out[(size_t)bh * T + row0 + lane] = D;
       const float inv = D > 0.f ? 1.f / D : 0.f;
       const uint64_t inv2 = f32x2(__float_as_uint(inv), __float_as_uint(inv));
       auto scaled = [&](int x) {
@@ -437,7 +439,8 @@ __global__ void __launch_bounds__(kMgThreads, 1)
 }
 
 template <int p, int G>
-static cudaError_t launch_flash_mg_t(const void* q, const void* k, const void* v, void* o, int B, int H, int T,
+static cudaError_t launch_flash_mg_t(const void* q, const void* k, const void* v, void* o, float* D_out, int B, int H,
+                                     int T,
                                      bool bthd, const WaitCtl& wc, cudaStream_t st) {
   using Cfg = MgCfg<p, G>;
   CUtensorMap tq, tk, tv, to;
@@ -458,7 +461,7 @@ static cudaError_t launch_flash_mg_t(const void* q, const void* k, const void* v
   }
   const long items = (long)((T + kMgBM - 1) / kMgBM) * B * H;
   const int grid = (int)(items < num_sms ? items : num_sms);
-  kern<<<grid, kMgThreads, Cfg::kSmemBytes, st>>>(tq, tk, tv, to, T, B * H, H, bthd ? 1 : 0, wc);
+  kern<<<grid, kMgThreads, Cfg::kSmemBytes, st>>>(tq, tk, tv, to, T, B * H, H, bthd ? 1 : 0, D_out, wc);
   return cudaGetLastError();
 }
 
@@ -472,11 +475,11 @@ bool flash_mg_sm100_supports(int p, int groups, int dv) {
   return dv == kMgDV && ((p == 16 && (groups == 2 || groups == 4)) || (p == 32 && groups == 2));
 }
 
-cudaError_t launch_flash_mg_sm100(const void* q, const void* k, const void* v, void* o, int B, int H, int T, int p,
-                                  int groups, bool bthd, const WaitCtl& wc, cudaStream_t st) {
-  if (p == 16 && groups == 2) return launch_flash_mg_t<16, 2>(q, k, v, o, B, H, T, bthd, wc, st);
-  if (p == 16 && groups == 4) return launch_flash_mg_t<16, 4>(q, k, v, o, B, H, T, bthd, wc, st);
-  if (p == 32 && groups == 2) return launch_flash_mg_t<32, 2>(q, k, v, o, B, H, T, bthd, wc, st);
+cudaError_t launch_flash_mg_sm100(const void* q, const void* k, const void* v, void* o, float* D_out, int B, int H, int T,
+                                  int p, int groups, bool bthd, const WaitCtl& wc, cudaStream_t st) {
+  if (p == 16 && groups == 2) return launch_flash_mg_t<16, 2>(q, k, v, o, D_out, B, H, T, bthd, wc, st);
+  if (p == 16 && groups == 4) return launch_flash_mg_t<16, 4>(q, k, v, o, D_out, B, H, T, bthd, wc, st);
+  if (p == 32 && groups == 2) return launch_flash_mg_t<32, 2>(q, k, v, o, D_out, B, H, T, bthd, wc, st);
   return cudaErrorInvalidValue;
 }
 

@@ -284,8 +284,8 @@ KATA_API kata_status_t kata_bwd_quadratic(const void* q, const void* k, const vo
     if (!aligned16(ptr)) return KATA_ERR_MISALIGNED;
   if (!workspace || workspace_bytes < flash_bwd_workspace_bytes(B * H, T, dv_width)) return KATA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return KATA_ERR_MISALIGNED;
-  return from_cuda(launch_flash_bwd_sm100(q, k, v, o, D, dO, dq, dk, dv, B * H, T, p, workspace, wait_ctl(),
-                                          static_cast<cudaStream_t>(stream)));
+  return from_cuda(launch_flash_bwd_sm100(q, k, v, o, D, dO, dq, dk, dv, B * H, T, p, p, false, false, workspace,
+                                          wait_ctl(), static_cast<cudaStream_t>(stream)));
 }
 
 // Shape checks shared by the KATA-Mg entry points: p = d / groups.
@@ -314,8 +314,50 @@ KATA_API kata_status_t kata_fwd_mg_quadratic(const void* q, const void* k, const
   const bool bthd = layout == KATA_LAYOUT_BTHD;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (flash_mg_sm100_supports(p, groups, dv))
-    return from_cuda(launch_flash_mg_sm100(q, k, v, o, B, H, T, p, groups, bthd, wait_ctl(), st));
+    return from_cuda(launch_flash_mg_sm100(q, k, v, o, nullptr, B, H, T, p, groups, bthd, wait_ctl(), st));
   return from_cuda(launch_flash_sm100(q, k, v, o, B, H, T, p, dv, bthd, nullptr, wait_ctl(), st));
+}
+
+KATA_API kata_status_t kata_fwd_mg_quadratic_train(const void* q, const void* k, const void* v, void* o, float* D,
+                                                   int B, int H, int T, int d, int groups, int dv,
+                                                   kata_dtype_t dtype, void* stream) {
+  int p = 0;
+  kata_status_t s = check_mg(B, H, T, d, groups, dv, dtype, &p);
+  if (s != KATA_OK) return s;
+  if (dtype != KATA_BF16 || groups < 2) return KATA_ERR_UNSUPPORTED;
+  if (T == 0) return KATA_OK;
+  if (!q || !k || !v || !o || !D) return KATA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(D)) return KATA_ERR_MISALIGNED;
+  return from_cuda(launch_flash_mg_sm100(q, k, v, o, D, B, H, T, p, groups, false, wait_ctl(),
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+KATA_API kata_status_t kata_bwd_mg_quadratic(const void* q, const void* k, const void* v, const void* o,
+                                             const float* D, const void* dO, void* dq, void* dk, void* dv, int B,
+                                             int H, int T, int d, int groups, int dv_width, kata_dtype_t dtype,
+                                             void* workspace, size_t workspace_bytes, void* stream) {
+  int p = 0;
+  kata_status_t s = check_mg(B, H, T, d, groups, dv_width, dtype, &p);
+  if (s != KATA_OK) return s;
+  if (dtype != KATA_BF16 || groups < 2) return KATA_ERR_UNSUPPORTED;
+  if (T == 0) return KATA_OK;
+  for (const void* ptr : {q, k, v, o, (const void*)D, dO, (const void*)dq, (const void*)dk, (const void*)dv})
+    if (!ptr) return KATA_ERR_INVALID_ARG;
+  for (const void* ptr : {q, k, v, o, (const void*)D, dO, (const void*)dq, (const void*)dk, (const void*)dv})
+    if (!aligned16(ptr)) return KATA_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < flash_bwd_workspace_bytes(B * H, T, dv_width)) return KATA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return KATA_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // one pass per group on its columns: dq^j, dk^j from the group's scores,
+  // dv summed over the groups; the per-row constants are computed once
+  for (int j = 0; j < groups; ++j) {
+    const size_t off = (size_t)j * p * 2;  // bytes
+    cudaError_t e = launch_flash_bwd_sm100(static_cast<const char*>(q) + off, static_cast<const char*>(k) + off, v, o, D,
+                                           dO, static_cast<char*>(dq) + off, static_cast<char*>(dk) + off, dv, B * H,
+                                           T, p, d, j > 0, j > 0, workspace, wait_ctl(), st);
+    if (e != cudaSuccess) return from_cuda(e);
+  }
+  return KATA_OK;
 }
 
 KATA_API kata_status_t kata_decode_step_mg(const void* q, const void* k, const void* v, void* o, float* S, float* z,

@@ -73,16 +73,20 @@ cudaError_t launch_flash_sm100(const void* q, const void* k, const void* v, void
 // flash_bwd_sm100.cu -- backward pass of the flash-style forward (bf16,
 // p in {16, 32}, dv = 64, [B*H, T, *] layouts); D is the forward's
 // denominator [B*H, T] fp32; ws holds flash_bwd_workspace_bytes().
+// q, k, dq and dk rows are ld elements apart (ld = p for [B*H, T, p]; one
+// group of a [B*H, T, d] tensor with ld = d); with rows_ready the per-row
+// constants already in ws are reused; with dv_accumulate dv is added to.
 size_t flash_bwd_workspace_bytes(int BH, int T, int dv);
 cudaError_t launch_flash_bwd_sm100(const void* q, const void* k, const void* v, const void* o, const float* D,
-                                   const void* dO, void* dq, void* dk, void* dv, int BH, int T, int p, void* ws,
-                                   const WaitCtl& wc, cudaStream_t st);
+                                   const void* dO, void* dq, void* dk, void* dv, int BH, int T, int p, int ld,
+                                   bool rows_ready, bool dv_accumulate, void* ws, const WaitCtl& wc, cudaStream_t st);
 
 // flash_mg_sm100.cu -- tcgen05 flash-style KATA-Mg forward (bf16 inputs,
-// dv = 64) with `groups` PSD factors of width p per head.
+// dv = 64) with `groups` PSD factors of width p per head; D_out (nullable,
+// fp32 [B*H, T]) receives each row's denominator.
 bool flash_mg_sm100_supports(int p, int groups, int dv);
-cudaError_t launch_flash_mg_sm100(const void* q, const void* k, const void* v, void* o, int B, int H, int T, int p,
-                                  int groups, bool bthd, const WaitCtl& wc, cudaStream_t st);
+cudaError_t launch_flash_mg_sm100(const void* q, const void* k, const void* v, void* o, float* D_out, int B, int H, int T,
+                                  int p, int groups, bool bthd, const WaitCtl& wc, cudaStream_t st);
 
 // chunk_sm100.cu -- tcgen05 chunked-state forward (bf16 inputs, p = 16).
 // The state kernel sums super-chunks 0..G-2 (the last one's sum is never

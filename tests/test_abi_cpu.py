@@ -44,7 +44,7 @@ def test_only_abi_symbols_are_exported():
 
 
 def test_status_strings_and_version(L):
-    assert _abi.kata_abi_version() == 10200
+    assert _abi.kata_abi_version() == 10300
     for code, name in [(0, "KATA_OK"), (2, "KATA_ERR_UNSUPPORTED"), (6, "KATA_ERR_TIMEOUT")]:
         assert _abi.status_string(code) == name
     assert _abi.status_string(99) == "KATA_ERR_UNKNOWN"
@@ -165,3 +165,21 @@ def test_training_entry_points_reject_bad_arguments(L):
     assert g(a, b, c, d, D, dO, gq, gk, gv, 1, 1, 16, 16, 64, 1, None, n, st) == _abi.KATA_ERR_WORKSPACE
     assert g(a, b, c, d, D, dO, gq, gk, _fake(0x90008), 1, 1, 16, 16, 64, 1, ws, n, st) == _abi.KATA_ERR_MISALIGNED
     assert g(a, b, c, d, D, dO, gq, gk, gv, 1, 1, 0, 16, 64, 1, None, 0, st) == _abi.KATA_OK
+
+
+def test_mg_training_entry_points_reject_bad_arguments(L):
+    a, b, c, d = _fake(0x10000), _fake(0x20000), _fake(0x30000), _fake(0x40000)
+    D, dO, gq, gk, gv, ws = (_fake(0x50000 + 0x10000 * i) for i in range(6))
+    st = VP(0)
+    f = L.kata_fwd_mg_quadratic_train  # q k v o D B H T d groups dv dtype stream
+    assert f(a, b, c, d, D, 1, 1, 16, 64, 1, 64, 1, st) == _abi.KATA_ERR_UNSUPPORTED   # one group: single-factor call
+    assert f(a, b, c, d, D, 1, 1, 16, 64, 2, 64, 0, st) == _abi.KATA_ERR_UNSUPPORTED   # fp32
+    assert f(a, b, c, d, None, 1, 1, 16, 64, 2, 64, 1, st) == _abi.KATA_ERR_INVALID_ARG
+    assert f(a, b, c, d, D, 1, 1, 16, 64, 3, 64, 1, st) == _abi.KATA_ERR_INVALID_ARG   # 64 % 3
+    assert f(a, b, c, d, D, 1, 1, 0, 64, 2, 64, 1, st) == _abi.KATA_OK
+    g = L.kata_bwd_mg_quadratic  # q k v o D dO dq dk dv B H T d groups dv dtype ws bytes stream
+    n = 16 * 8
+    assert g(a, b, c, d, D, dO, gq, gk, gv, 1, 1, 16, 64, 2, 16, 1, ws, n, st) == _abi.KATA_ERR_UNSUPPORTED
+    assert g(a, b, c, d, D, dO, gq, gk, gv, 1, 1, 16, 64, 2, 64, 1, ws, n - 1, st) == _abi.KATA_ERR_WORKSPACE
+    assert g(a, b, c, d, D, None, gq, gk, gv, 1, 1, 16, 64, 2, 64, 1, ws, n, st) == _abi.KATA_ERR_INVALID_ARG
+    assert g(a, b, c, d, D, dO, gq, gk, gv, 1, 1, 0, 64, 4, 64, 1, None, 0, st) == _abi.KATA_OK
