@@ -519,3 +519,40 @@ def test_backward_mg_pins():
     q2, k2, v2 = _rand_mg(B=1, H=2, T=30, d=8, dv=3, seed=482)
     dq2, _, _ = obw.backward_mg(q2, k2, v2, rng.standard_normal(v2.shape), 2)
     np.testing.assert_allclose(np.einsum("bhtd,bhtd->bht", q2, dq2), 0.0, atol=1e-9)
+
+
+# ---------------------------------------------------------------------------
+# KATA-Sigma-g (summed factors): pins of the numpy oracle
+# ---------------------------------------------------------------------------
+
+from oracle import sigma_g as osg  # noqa: E402
+
+
+def test_sigma_g_pins():
+    q, k, v = _rand_mg(B=1, H=2, T=20, d=8, dv=3, seed=500)
+    # g = 1 is the full rank-one map
+    np.testing.assert_allclose(osg.direct_sg(q, k, v, 1), oracle.direct(q, k, v), rtol=1e-11, atol=1e-12)
+    # the two forms agree
+    for g in (2, 4):
+        np.testing.assert_allclose(osg.recurrent_sg(q, k, v, g), osg.direct_sg(q, k, v, g), rtol=1e-10, atol=1e-12)
+    # the weight pairs every query group with every key group: permuting the
+    # query's groups alone changes nothing (it would for KATA-Mg)
+    perm = np.concatenate([np.arange(4, 8), np.arange(0, 4)])
+    np.testing.assert_allclose(osg.direct_sg(q[..., perm], k, v, 2), osg.direct_sg(q, k, v, 2), rtol=1e-11, atol=1e-12)
+    assert np.abs(oracle.direct_mg(q[..., perm], k, v, 2) - oracle.direct_mg(q, k, v, 2)).max() > 1e-3
+    # width-one groups: w = |q|^2 |k|^2, so o_t is the |k|^2-weighted running
+    # mean of v whatever q_t (!= 0) is
+    q1, k1, v1 = _rand_mg(B=1, H=1, T=15, d=3, dv=2, seed=501)
+    kk = (k1[0, 0] ** 2).sum(-1)
+    want = np.cumsum(kk[:, None] * v1[0, 0], axis=0) / np.cumsum(kk)[:, None]
+    np.testing.assert_allclose(osg.direct_sg(q1, k1, v1, 3)[0, 0], want, rtol=1e-11, atol=1e-12)
+
+
+@pytest.mark.parametrize("d,g", [(8, 2), (8, 4), (12, 3)])
+def test_sigma_g_feature_dimension_matches_state_size_formula(d, g):
+    """The summed features span (d/g)(d/g+1)/2 dimensions: the KATA-Sigma-g
+    state width per value column (ai.info, Main Findings)."""
+    rng = np.random.default_rng(510 + d + g)
+    p = d // g
+    f = osg.features_sg(rng.standard_normal((3 * p * p, d)), g)
+    assert np.linalg.matrix_rank(f) == p * (p + 1) // 2
