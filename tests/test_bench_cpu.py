@@ -1,0 +1,41 @@
+"""bench.py's JSON line, built from fabricated timings on the CPU: every key
+the benchmark contract names is present, and the derived fractions follow
+from the times (no GPU involved)."""
+import argparse
+import io
+import json
+from contextlib import redirect_stdout
+
+import bench
+
+
+def _fake_result():
+    mg = {"mg2_ctx2k": dict(B=8, H=16, T=2048, d=64, groups=2, dv=64, layout="bthd", ms=0.115),
+          "decode_mg4_b64": dict(B=64, H=16, d=64, groups=4, dv=64, P=1024, ms=0.094)}
+    grid = [dict(B=1, T=1024, chunked_ms=0.02, quadratic_ms=0.02)]
+    long = dict(B=1, H=16, T=131072, p=16, dv=64, chunked_C64_ms=0.235, chunked_C128_ms=0.234, quadratic_ms=29.0,
+                sequential_C64_ms=1.25, decode_b64=dict(B=64, H=16, p=16, dv=64, ms=0.03), sweep=grid,
+                recall=dict(B=4, H=16, T=8192, p=32, dv=64, chunked_ms=13.8, quadratic_ms=0.51), mg=mg,
+                train=dict(B=8, H=16, T=2048, p=16, dv=64, fwd_ms=0.08, bwd_ms=0.36, step_ms=0.43))
+    return dict(step_ms=0.116, eager_step_ms=0.125, graph=True, path_ms=[0.081, 0.035, 0.0088], e2e_ms=11.0,
+                h2d=50356224, d2h=67125248, clocks={"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []},
+                timed_s=0.5, long=long, status=0, tokens=8 * 2048, BH=128, T=2048, p=16, dv=64, C=64)
+
+
+def test_report_line_has_the_contract_keys():
+    args = argparse.Namespace(workload="layer340m_ctx2k", steps=1000, warmup=10, cpu_baseline=0)
+    buf = io.StringIO()
+    with redirect_stdout(buf):
+        bench.report(args, _fake_result(), 0.116, 11.0, 1)
+    line = json.loads(buf.getvalue().strip().splitlines()[-1])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+                "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches", "clocks"):
+        assert key in line, key
+    assert line["value"] == 8 * 2048 / 0.116e-3
+    rf = line["roofline"]
+    assert abs(rf["frac"] - rf["achieved"] / rf["peak"]) < 1e-12
+    assert rf["achieved"] == bench.flash_flops(128, 2048, 16, 64) / 0.081e-3 / 1e12
+    assert set(line["mg"]) == {"mg2_ctx2k", "decode_mg4_b64"}
+    assert "tensor_frac" in line["mg"]["mg2_ctx2k"] and "hbm_frac" in line["mg"]["decode_mg4_b64"]
+    tr = line["train"]
+    assert tr["tokens_per_s"] == 8 * 2048 / 0.43e-3 and 0 < tr["bwd_tensor_frac"] < 1
