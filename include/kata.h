@@ -253,6 +253,21 @@ kata_status_t kata_fwd_mg_quadratic(const void* q, const void* k, const void* v,
                                     kata_layout_t layout, kata_dtype_t dtype, void* stream);
 
 /*
+ * Quadratic (flash-style) KATA-Sigma-g forward: summed PSD factors
+ * (gist.science sec. 2.3 "Varianten"; ai.info Main Findings: state
+ * (d/g)(d/g+1)/2 * dv).  The feature is the sum of the groups' rank-one maps,
+ * psi_S(u) = sum_j vec(u^j u^j^T), so that
+ *   w_{t,s} = sum_{j,l} (q_t^j . k_s^l)^2
+ * over every pair of a query group and a key group, with one value vector and
+ * one denominator.  Arguments, layouts, supported (p, groups, dv) and errors
+ * as for kata_fwd_mg_quadratic with groups > 1 (groups = 1 is the single
+ * factor: use kata_fwd_mg_quadratic).
+ */
+kata_status_t kata_fwd_sg_quadratic(const void* q, const void* k, const void* v, void* o,
+                                    int B, int H, int T, int d, int groups, int dv,
+                                    kata_layout_t layout, kata_dtype_t dtype, void* stream);
+
+/*
  * One KATA-Mg decode step (update with (k, v), then read with q):
  * q, k: [B,H,d]; v, o: [B,H,dv] (fp32 or bf16); S: [B,H,groups*p*p,dv] and
  * z: [B,H,groups*p*p] fp32, read and updated in place, with row
@@ -286,7 +301,7 @@ void kata_set_wait_limit(long long cycles);
 /* ABI version of this header: major * 10000 + minor * 100 + patch. */
 int kata_abi_version(void);
 
-#define KATA_ABI_VERSION 10300
+#define KATA_ABI_VERSION 10400
 
 #ifdef __cplusplus
 }

@@ -37,6 +37,7 @@ SIGNATURES = {
     "kata_bwd_quadratic": (_c_int, [_vp] * 9 + [_c_int] * 6 + [_vp, _c_size, _vp]),
     "kata_fwd_mg_quadratic": (_c_int, [_vp, _vp, _vp, _vp] + [_c_int] * 8 + [_vp]),
     "kata_fwd_mg_quadratic_train": (_c_int, [_vp, _vp, _vp, _vp, _fp] + [_c_int] * 7 + [_vp]),
+    "kata_fwd_sg_quadratic": (_c_int, [_vp, _vp, _vp, _vp] + [_c_int] * 8 + [_vp]),
     "kata_bwd_mg_quadratic": (_c_int, [_vp] * 9 + [_c_int] * 7 + [_vp, _c_size, _vp]),
     "kata_decode_step_mg": (_c_int, [_vp, _vp, _vp, _vp, _fp, _fp] + [_c_int] * 6 + [_vp]),
     "kata_get_status": (_c_int, [_vp]),
@@ -268,6 +269,27 @@ class KataAttention(torch.autograd.Function):
 def kata_attention(q, k, v):
     """Differentiable flash-style KATA attention, q,k [B,H,T,p], v [B,H,T,dv]."""
     return KataAttention.apply(q, k, v)
+
+
+def kata_fwd_sg_quadratic(q, k, v, groups, layout="bhtd", o=None, stream=None):
+    """Flash-style KATA-Sigma-g forward: weight sum_{j,l} (q^j . k^l)^2 over
+    every pair of a query group and a key group.  Layouts as for
+    kata_fwd_mg_quadratic; groups > 1."""
+    if layout == "bhtd":
+        B, H, T, d = q.shape
+        code = KATA_LAYOUT_BHTD
+    elif layout == "bthd":
+        B, T, H, d = q.shape
+        code = KATA_LAYOUT_BTHD
+    else:
+        raise ValueError("layout must be 'bhtd' or 'bthd'")
+    dv = v.shape[-1]
+    if o is None:
+        o = torch.empty(v.shape, dtype=q.dtype, device=q.device)
+    _check("kata_fwd_sg_quadratic", lib().kata_fwd_sg_quadratic(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), B, H, T, d, int(groups), dv, code,
+        _dtype_code(q), _stream_ptr(stream)))
+    return o
 
 
 def kata_fwd_mg_quadratic_train(q, k, v, groups, o=None, D=None, stream=None):

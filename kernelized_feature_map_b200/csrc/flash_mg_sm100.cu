@@ -65,11 +65,19 @@ constexpr int kMgThreads = 576;   // warp 0 TMA, warp 1 MMA, warps 2-17 weights 
 constexpr int kMgStages = 4;      // K/V ring depth
 constexpr uint32_t kMgTmemCols = 512;
 
-template <int p, int G>
+// kSum selects KATA-Sigma-g (summed factors, gist.science sec. 2.3
+// "Varianten"): the weight is sum_{j,l} (q^j . k^l)^2 over every pair of a
+// query group and a key group, so the kernel's score "groups" are the G^2
+// pairs (j, l) -- the same pipeline with G^2 instead of G score blocks.
+template <int p, int G, bool kSum = false>
 struct MgCfg {
   static constexpr int kD = G * p;                      // q/k row width (32 or 64)
-  static constexpr int kGR = 2;                         // groups per round
-  static constexpr int kRounds = G / kGR;
+  static constexpr int kGR = 2;                         // score blocks per round
+  static constexpr int kBlocks = kSum ? G * G : G;      // score blocks per key tile
+  static constexpr int kRounds = kBlocks / kGR;
+  // column group of the query (key) side of score block v
+  static constexpr int q_group(int v) { return kSum ? v / G : v; }
+  static constexpr int k_group(int v) { return kSum ? v % G : v; }
   static constexpr int kQKBytes = kMgBM * kD * 2;       // one Q or K tile
   static constexpr int kVBytes = kMgBN * kMgDV * 2;     // one V tile
   static constexpr int kOnesBytes = kMgBN * kMgDV * 2;  // ones block of the [V | 1] operand
@@ -93,16 +101,16 @@ struct MgCfg {
   static constexpr int kNumBars = 4 + 2 * kMgStages + 7;
   static constexpr int offMisc = offBar + kNumBars * 8;
   static constexpr int kSmemBytes = offMisc + 16 + 1024;
-  static_assert(G % kGR == 0, "groups per round");
+  static_assert(kBlocks % kGR == 0, "score blocks per round");
   static_assert(offV % 1024 == 0 && offOnes % 1024 == 0 && offOut % 1024 == 0, "alignment");
 };
 
-template <int p, int G>
+template <int p, int G, bool kSum>
 __global__ void __launch_bounds__(kMgThreads, 1)
     flash_mg_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o, int T, int BH,
                     int H, int bthd, float* __restrict__ D_out, WaitCtl wc) {
-  using Cfg = MgCfg<p, G>;
+  using Cfg = MgCfg<p, G, kSum>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::offBar);
@@ -211,8 +219,9 @@ __global__ void __launch_bounds__(kMgThreads, 1)
       auto issue_round = [&](int qb, int st, int r) {
 #pragma unroll
         for (int gg = 0; gg < Cfg::kGR; ++gg) {
-          const uint32_t off = (uint32_t)((r * Cfg::kGR + gg) * p * 2);
-          const uint64_t a = desc_add(dq0, qb * Cfg::kQKBytes + off), b = desc_add(dk0, st * Cfg::kQKBytes + off);
+          const int blk = r * Cfg::kGR + gg;
+          const uint32_t qoff = (uint32_t)(Cfg::q_group(blk) * p * 2), koff = (uint32_t)(Cfg::k_group(blk) * p * 2);
+          const uint64_t a = desc_add(dq0, qb * Cfg::kQKBytes + qoff), b = desc_add(dk0, st * Cfg::kQKBytes + koff);
 #pragma unroll
           for (int ks = 0; ks < p / 16; ++ks)
             mma_ss_w(tmem + Cfg::colS(gg), desc_add(a, ks * 32), desc_add(b, ks * 32), id_qk, ks > 0);
@@ -438,18 +447,17 @@ __global__ void __launch_bounds__(kMgThreads, 1)
   }
 }
 
-template <int p, int G>
+template <int p, int G, bool kSum = false>
 static cudaError_t launch_flash_mg_t(const void* q, const void* k, const void* v, void* o, float* D_out, int B, int H,
-                                     int T,
-                                     bool bthd, const WaitCtl& wc, cudaStream_t st) {
-  using Cfg = MgCfg<p, G>;
+                                     int T, bool bthd, const WaitCtl& wc, cudaStream_t st) {
+  using Cfg = MgCfg<p, G, kSum>;
   CUtensorMap tq, tk, tv, to;
   if (!make_tmap_bf16_4d(&tq, q, Cfg::kD, T, H, B, bthd, Cfg::kD, kMgBM) ||
       !make_tmap_bf16_4d(&tk, k, Cfg::kD, T, H, B, bthd, Cfg::kD, kMgBN) ||
       !make_tmap_bf16_4d(&tv, v, kMgDV, T, H, B, bthd, kMgDV, kMgBN) ||
       !make_tmap_bf16_4d(&to, o, kMgDV, T, H, B, bthd, 16, 32))
     return cudaErrorInvalidValue;
-  auto kern = flash_mg_kernel<p, G>;
+  auto kern = flash_mg_kernel<p, G, kSum>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
   if (e != cudaSuccess) return e;
   static int num_sms = 0;
@@ -480,6 +488,14 @@ cudaError_t launch_flash_mg_sm100(const void* q, const void* k, const void* v, v
   if (p == 16 && groups == 2) return launch_flash_mg_t<16, 2>(q, k, v, o, D_out, B, H, T, bthd, wc, st);
   if (p == 16 && groups == 4) return launch_flash_mg_t<16, 4>(q, k, v, o, D_out, B, H, T, bthd, wc, st);
   if (p == 32 && groups == 2) return launch_flash_mg_t<32, 2>(q, k, v, o, D_out, B, H, T, bthd, wc, st);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_flash_sg_sm100(const void* q, const void* k, const void* v, void* o, int B, int H, int T, int p,
+                                  int groups, bool bthd, const WaitCtl& wc, cudaStream_t st) {
+  if (p == 16 && groups == 2) return launch_flash_mg_t<16, 2, true>(q, k, v, o, nullptr, B, H, T, bthd, wc, st);
+  if (p == 16 && groups == 4) return launch_flash_mg_t<16, 4, true>(q, k, v, o, nullptr, B, H, T, bthd, wc, st);
+  if (p == 32 && groups == 2) return launch_flash_mg_t<32, 2, true>(q, k, v, o, nullptr, B, H, T, bthd, wc, st);
   return cudaErrorInvalidValue;
 }
 

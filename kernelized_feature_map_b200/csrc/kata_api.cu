@@ -318,6 +318,21 @@ KATA_API kata_status_t kata_fwd_mg_quadratic(const void* q, const void* k, const
   return from_cuda(launch_flash_sm100(q, k, v, o, B, H, T, p, dv, bthd, nullptr, wait_ctl(), st));
 }
 
+KATA_API kata_status_t kata_fwd_sg_quadratic(const void* q, const void* k, const void* v, void* o, int B, int H,
+                                             int T, int d, int groups, int dv, kata_layout_t layout,
+                                             kata_dtype_t dtype, void* stream) {
+  int p = 0;
+  kata_status_t s = check_mg(B, H, T, d, groups, dv, dtype, &p);
+  if (s != KATA_OK) return s;
+  if (layout != KATA_LAYOUT_BHTD && layout != KATA_LAYOUT_BTHD) return KATA_ERR_INVALID_ARG;
+  if (dtype != KATA_BF16 || groups < 2) return KATA_ERR_UNSUPPORTED;
+  if (T == 0) return KATA_OK;
+  if (!q || !k || !v || !o) return KATA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return KATA_ERR_MISALIGNED;
+  return from_cuda(launch_flash_sg_sm100(q, k, v, o, B, H, T, p, groups, layout == KATA_LAYOUT_BTHD, wait_ctl(),
+                                         static_cast<cudaStream_t>(stream)));
+}
+
 KATA_API kata_status_t kata_fwd_mg_quadratic_train(const void* q, const void* k, const void* v, void* o, float* D,
                                                    int B, int H, int T, int d, int groups, int dv,
                                                    kata_dtype_t dtype, void* stream) {

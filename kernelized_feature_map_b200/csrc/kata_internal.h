@@ -85,6 +85,10 @@ cudaError_t launch_flash_bwd_sm100(const void* q, const void* k, const void* v, 
 // dv = 64) with `groups` PSD factors of width p per head; D_out (nullable,
 // fp32 [B*H, T]) receives each row's denominator.
 bool flash_mg_sm100_supports(int p, int groups, int dv);
+// KATA-Sigma-g (summed factors): the same kernel over all (query group, key
+// group) score pairs; the (p, groups, dv) of flash_mg_sm100_supports.
+cudaError_t launch_flash_sg_sm100(const void* q, const void* k, const void* v, void* o, int B, int H, int T, int p,
+                                  int groups, bool bthd, const WaitCtl& wc, cudaStream_t st);
 cudaError_t launch_flash_mg_sm100(const void* q, const void* k, const void* v, void* o, float* D_out, int B, int H, int T,
                                   int p, int groups, bool bthd, const WaitCtl& wc, cudaStream_t st);
 

@@ -44,7 +44,7 @@ def test_only_abi_symbols_are_exported():
 
 
 def test_status_strings_and_version(L):
-    assert _abi.kata_abi_version() == 10300
+    assert _abi.kata_abi_version() == 10400
     for code, name in [(0, "KATA_OK"), (2, "KATA_ERR_UNSUPPORTED"), (6, "KATA_ERR_TIMEOUT")]:
         assert _abi.status_string(code) == name
     assert _abi.status_string(99) == "KATA_ERR_UNKNOWN"
@@ -183,3 +183,14 @@ def test_mg_training_entry_points_reject_bad_arguments(L):
     assert g(a, b, c, d, D, dO, gq, gk, gv, 1, 1, 16, 64, 2, 64, 1, ws, n - 1, st) == _abi.KATA_ERR_WORKSPACE
     assert g(a, b, c, d, D, None, gq, gk, gv, 1, 1, 16, 64, 2, 64, 1, ws, n, st) == _abi.KATA_ERR_INVALID_ARG
     assert g(a, b, c, d, D, dO, gq, gk, gv, 1, 1, 0, 64, 4, 64, 1, None, 0, st) == _abi.KATA_OK
+
+
+def test_sg_argument_errors_before_launch(L):
+    a, b, c, d = _fake(0x10000), _fake(0x20000), _fake(0x30000), _fake(0x40000)
+    st = VP(0)
+    f = L.kata_fwd_sg_quadratic  # q k v o B H T d groups dv layout dtype stream
+    assert f(a, b, c, d, 1, 1, 16, 64, 1, 64, 0, 1, st) == _abi.KATA_ERR_UNSUPPORTED   # one group
+    assert f(a, b, c, d, 1, 1, 16, 64, 3, 64, 0, 1, st) == _abi.KATA_ERR_INVALID_ARG   # 64 % 3
+    assert f(a, b, c, d, 1, 1, 16, 64, 2, 64, 5, 1, st) == _abi.KATA_ERR_INVALID_ARG   # layout
+    assert f(a, b, c, d, 1, 1, 16, 64, 2, 64, 0, 0, st) == _abi.KATA_ERR_UNSUPPORTED   # fp32
+    assert f(a, b, c, d, 1, 1, 0, 64, 2, 64, 1, 1, st) == _abi.KATA_OK

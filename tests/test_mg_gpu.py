@@ -164,3 +164,26 @@ def test_mg_many_items_ragged(kata, g):
     ref = oracle.direct_mg_rows(q, k, v, g, bh, t)
     vmax = np.abs(v.reshape(B * H, -1)).max(axis=1)[bh]
     assert rows_rel_err(got.reshape(B * H, T, dv)[bh, t], ref, vmax) <= TOL["bf16"]
+
+
+# ---------------------------------------------------------------------------
+# KATA-Sigma-g (summed factors) through the same kernel
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("layout", ["bhtd", "bthd"])
+@pytest.mark.parametrize("shape", [(2, 2, 600, 64, 2), (1, 2, 385, 64, 4), (1, 3, 300, 32, 2)])
+def test_sg_flash_matches_oracle(kata, shape, layout):
+    import torch
+    from oracle import sigma_g as osg
+    B, H, T, d, g, dv = shape + (64,)
+    q, k, v = workloads.normal_qkv(B, H, T, d, dv, seed=520 + T + g, dtype="bf16")
+    ref = osg.direct_sg(q, k, v, g)
+    if layout == "bthd":
+        o = kata.kata_fwd_sg_quadratic(to_dev(_bthd(q), "bf16"), to_dev(_bthd(k), "bf16"), to_dev(_bthd(v), "bf16"),
+                                       g, layout="bthd")
+        got = _bthd(to_np(o))
+    else:
+        got = to_np(kata.kata_fwd_sg_quadratic(to_dev(q, "bf16"), to_dev(k, "bf16"), to_dev(v, "bf16"), g))
+    torch.cuda.synchronize()
+    assert kata.kata_get_status() == 0
+    assert row_rel_err(got, ref, v) <= TOL["bf16"]
