@@ -523,6 +523,10 @@ def run_mg(args, K, torch, dev, stream, flush):
         o = torch.empty_like(v)
         ms = _time_call(lambda: K.kata_fwd_mg_quadratic(q, k, v, g, layout=cfg["layout"], o=o), flush, stream, 10, 3)
         out[name] = dict(B=B, H=H, T=T, d=d, groups=g, dv=dv, layout=cfg["layout"], ms=ms)
+        # KATA-Sigma-g (summed factors) on the same inputs: g^2 score blocks
+        ms_sg = _time_call(lambda: K.kata_fwd_sg_quadratic(q, k, v, g, layout=cfg["layout"], o=o), flush, stream, 10,
+                           3)
+        out["sg" + name[2:]] = dict(B=B, H=H, T=T, d=d, groups=g, dv=dv, layout=cfg["layout"], ms=ms_sg, summed=True)
         del q, k, v, o
     # decode step on the concatenated per-group state (B = 64, as for the
     # single-factor decode line): HBM-bound, the state is read and written once
@@ -764,11 +768,16 @@ def report(args, res, step_ms, e2e_ms, world):
                         "ms": m["ms"], "tokens_per_s": m["B"] / (m["ms"] * 1e-3),
                         "hbm_frac": mb / (m["ms"] * 1e-3) / 1e9 / peaks["hbm_gbs"]}
                 else:
+                    # score flops: d per pair for KATA-Mg, g*d for KATA-Sigma-g
+                    # (every query group against every key group)
+                    summed = m.get("summed", False)
+                    width = m["groups"] * m["d"] if summed else m["d"]
                     line["mg"][name] = {
-                        "workload": "KATA-Mg B=%d H=%d T=%d d=%d groups=%d dv=%d bf16 [%s]" % (
-                            m["B"], m["H"], m["T"], m["d"], m["groups"], m["dv"], m["layout"]),
+                        "workload": "%s B=%d H=%d T=%d d=%d groups=%d dv=%d bf16 [%s]" % (
+                            "KATA-Sigma-g" if summed else "KATA-Mg", m["B"], m["H"], m["T"], m["d"], m["groups"],
+                            m["dv"], m["layout"]),
                         "ms": m["ms"], "tokens_per_s": m["B"] * m["T"] / (m["ms"] * 1e-3),
-                        "tensor_frac": flash_flops(m["B"] * m["H"], m["T"], m["d"], m["dv"]) / (m["ms"] * 1e-3)
+                        "tensor_frac": flash_flops(m["B"] * m["H"], m["T"], width, m["dv"]) / (m["ms"] * 1e-3)
                         / 1e12 / peaks["bf16_tflops"]}
         if "train" in lg:
             tr = lg["train"]

@@ -11,6 +11,7 @@ import bench
 
 def _fake_result():
     mg = {"mg2_ctx2k": dict(B=8, H=16, T=2048, d=64, groups=2, dv=64, layout="bthd", ms=0.115),
+          "sg2_ctx2k": dict(B=8, H=16, T=2048, d=64, groups=2, dv=64, layout="bthd", ms=0.19, summed=True),
           "decode_mg4_b64": dict(B=64, H=16, d=64, groups=4, dv=64, P=1024, ms=0.094)}
     grid = [dict(B=1, T=1024, chunked_ms=0.02, quadratic_ms=0.02)]
     long = dict(B=1, H=16, T=131072, p=16, dv=64, chunked_C64_ms=0.235, chunked_C128_ms=0.234, quadratic_ms=29.0,
@@ -35,7 +36,9 @@ def test_report_line_has_the_contract_keys():
     rf = line["roofline"]
     assert abs(rf["frac"] - rf["achieved"] / rf["peak"]) < 1e-12
     assert rf["achieved"] == bench.flash_flops(128, 2048, 16, 64) / 0.081e-3 / 1e12
-    assert set(line["mg"]) == {"mg2_ctx2k", "decode_mg4_b64"}
+    assert set(line["mg"]) == {"mg2_ctx2k", "sg2_ctx2k", "decode_mg4_b64"}
+    assert line["mg"]["sg2_ctx2k"]["workload"].startswith("KATA-Sigma-g")
+    assert line["mg"]["sg2_ctx2k"]["tensor_frac"] == bench.flash_flops(128, 2048, 128, 64) / 0.19e-3 / 1e12 / 1617.3
     assert "tensor_frac" in line["mg"]["mg2_ctx2k"] and "hbm_frac" in line["mg"]["decode_mg4_b64"]
     tr = line["train"]
     assert tr["tokens_per_s"] == 8 * 2048 / 0.43e-3 and 0 < tr["bwd_tensor_frac"] < 1
