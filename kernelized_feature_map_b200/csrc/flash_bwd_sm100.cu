@@ -9,8 +9,8 @@
 //   dS_ts = 2 S_ts (dN_t . v_s + dD_t)                    (s <= t)
 //   dv_s  = sum_{t>=s} w_ts dN_t
 //   dq_t  = sum_{s<=t} dS_ts k_s,   dk_s = sum_{t>=s} dS_ts q_t
-// evaluated as dS_ts = 2 (S_ts r_t) (dO_t . v_s - delta_t) and
-// dv_s = sum_t (S_ts^2 r_t) dO_t with r_t = 1 / D_t and delta_t = dO_t . o_t:
+// evaluated as dS_ts = (S_ts r_t) (dO_t . v_s - delta_t) and
+// dv_s = 1/2 sum_t (S_ts^2 r_t) dO_t with r_t = 2 / D_t and delta_t = dO_t . o_t:
 // the tensor core multiplies dO itself (exact bf16 input), and the
 // difference dO.v - dO.o, which cancels when the row's weight sits on few
 // keys, is taken in fp32 before the 1 / D scaling.  (Rounding dN = dO / D to
@@ -25,7 +25,7 @@
 //                        dS in the weight warps, then
 //                        dQ += dS K_j with dS read from TMEM;
 //   3. bwd_dkdv_kernel   persistent, items of one 128-row key tile: per query tile i,
-//                        S^T = K Q_i^T and dP^T = V dO_i^T, W^T = (S^T)^2 r and
+//                        S^T = K Q_i^T and dP^T = V dO_i^T, W^T = (S^T)^2 r / 2 and
 //                        dS^T in the weight warps, then dV += W^T dO_i and
 //                        dK += dS^T Q_i.
 // Both main kernels keep the products in TMEM with keys (dQ) or queries
@@ -320,7 +320,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       for (int j = 0; j < nkv; ++j) {
         const int g = gs + j, st = g % kBwStages;
         if (j + 1 < nkv) {
-          // the next tile's S and dP' overwrite the current ones: wait until loaded
+          // the next tile's S and dP overwrite the current ones: wait until loaded
           if (!mbar_wait_w(kv_full + (g + 1) % kBwStages, ((g + 1) / kBwStages) & 1, env) ||
               !mbar_wait_w(s_read, g & 1, env)) {
             ok = false;
@@ -398,7 +398,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
           else
             grad_pairs<1, false, false, false, false>(s, d, nullptr, rc, lane, gr, unused);
         }
-        // S and dP' are in registers: the next key tile's may overwrite them
+        // S and dP are in registers: the next key tile's may overwrite them
         tc_fence_before();
         mbar_arrive(s_read);
         // dS buffer g % 2 was last read by the dQ MMAs of step g - 2, which
