@@ -128,15 +128,18 @@ kata_status_t kata_fwd_chunked(const void* q, const void* k, const void* v, void
  * and synchronise the device).
  *
  * Arguments, layouts, results and errors are those of kata_fwd_chunked.
- * The scratch space lives in one library-owned device array of 16 MiB
- * (16 * 2^20 bytes) that every GPU which loads the library holds until the
- * process exits; sizes whose kata_fwd_chunked_workspace_size() exceeds it
- * return KATA_ERR_WORKSPACE.  The call allocates nothing.
+ * The scratch space lives in one library-owned device array of
+ * KATA_NOALLOC_SCRATCH_BYTES (16 MiB) that every GPU which loads the library
+ * holds until the process exits; sizes whose
+ * kata_fwd_chunked_workspace_size() exceeds it return KATA_ERR_WORKSPACE,
+ * after the argument checks of kata_fwd_chunked.  The call allocates nothing.
  * All calls share that array: calls that overlap on the GPU race on it and
  * must be serialised by the caller.  The first call on a device looks up the
- * array's device address (once per device, with that device current); make
- * that first call before any stream capture.
+ * array's device address (with that device current), and looks it up again
+ * when the calling thread's CUDA context has changed since (a device reset);
+ * make that first call before any stream capture.
  */
+#define KATA_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
 kata_status_t kata_fwd_chunked_noalloc(const void* q, const void* k, const void* v, void* o,
                                        int B, int H, int T, int p, int dv, int C,
                                        kata_dtype_t dtype,

@@ -478,7 +478,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
         ++issued;
       }
       for (int c = issued - kStateStages < 0 ? 0 : issued - kStateStages; c < issued; ++c)
-        mbar_wait_drain(kv_full + c % kStateStages, (c / kStateStages) & 1, wc.limit);
+        mbar_wait_drain(kv_full + c % kStateStages, (c / kStateStages) & 1);
     }
   } else if (warp == 1) {
     {  // whole warp; one elected lane issues
@@ -502,7 +502,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
         mma_commit_w(kv_empty + st);
       }
       mma_commit_w(acc_done);
-      mbar_wait_drain(acc_done, 0, wc.limit);
+      mbar_wait_drain(acc_done, 0);
     }
   } else {
     // warps 2-9: token (warp - 2) % 4 * 32 + lane, half (warp - 2) / 4 of its packed psi
@@ -513,12 +513,12 @@ __global__ void __launch_bounds__(kStateThreads, 1)
     bool ok = true;
     for (int c = 0; c < n_chunks; ++c) {
       const int st = c % kStateStages, pb = c & 1;
-      if (!mbar_wait(kv_full + st, (c / kStateStages) & 1, env)) {
+      if (!mbar_wait_w(kv_full + st, (c / kStateStages) & 1, env)) {
         ok = false;
         break;
       }
       if (tid == 0) KATA_TRACE(chunkstate, c, 2);
-      if (c >= 2 && !mbar_wait(psi_empty + pb, ((c >> 1) - 1) & 1, env)) {
+      if (c >= 2 && !mbar_wait_w(psi_empty + pb, ((c >> 1) - 1) & 1, env)) {
         ok = false;
         break;
       }
@@ -539,7 +539,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
     }
     // record rows 0..64 live in TMEM lanes 0..64: warps of lane quarters 0-2
     // load (the load is warp-collective), lanes below 65 store
-    if (ok && warp < 6 && quarter < 3 && mbar_wait(acc_done, 0, env)) {
+    if (ok && warp < 6 && quarter < 3 && mbar_wait_w(acc_done, 0, env)) {
       tc_fence_after();
       float* row = ws + ((size_t)bh * G + g) * record_floats + (size_t)min(d, kRecRows - 1) * kNP;
       state_lane_to_global(tmem + ((uint32_t)(quarter * 32) << 16), row, d < kRecRows);
@@ -676,7 +676,7 @@ __global__ void __launch_bounds__(kReadThreads, 1)
         ++issued;
       }
       for (int c = issued - kReadStages < 0 ? 0 : issued - kReadStages; c < issued; ++c)
-        mbar_wait_drain(kv_full + c % kReadStages, (c / kReadStages) & 1, wc.limit);
+        mbar_wait_drain(kv_full + c % kReadStages, (c / kReadStages) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA
@@ -734,7 +734,7 @@ __global__ void __launch_bounds__(kReadThreads, 1)
         KATA_TRACE(chunk, c, 6);
       }
       mma_commit_w(mma_done);
-      mbar_wait_drain(mma_done, 0, wc.limit);
+      mbar_wait_drain(mma_done, 0);
     }
   } else if (warp < 6 || warp >= 14) {
     // ------------------------------------------------------------- weights + output
@@ -754,7 +754,7 @@ __global__ void __launch_bounds__(kReadThreads, 1)
     // and written by one TMA store (rows past T are not written)
     auto output = [&](int co) -> bool {
       const int ob = co & 1;
-      if (!mbar_wait(o_full + ob, (co >> 1) & 1, env)) return false;
+      if (!mbar_wait_w(o_full + ob, (co >> 1) & 1, env)) return false;
       tc_fence_after();
       uint32_t r[32], db;
       tmem_ld32(lane_base + L::colO(ob) + 32 * h, r);
@@ -792,7 +792,7 @@ __global__ void __launch_bounds__(kReadThreads, 1)
     if (n_chunks > 0) mbar_arrive(state_full);
     bool ok = true;
     for (int c = 0; ok && c < n_chunks; ++c) {
-      if (!mbar_wait(s_full, c & 1, env)) break;
+      if (!mbar_wait_w(s_full, c & 1, env)) break;
       if (c == 0 && n_chunks > 1) mbar_arrive(state_full);
       if (m == 0) KATA_TRACE(chunk, c, 8);
       tc_fence_after();
@@ -880,7 +880,7 @@ __global__ void __launch_bounds__(kReadThreads, 1)
       }
     }
     // chunk 0's psi~(k) or psi~(q): they need nothing but its stage
-    bool ok = n_chunks > 0 && mbar_wait(kv_full, 0, env);
+    bool ok = n_chunks > 0 && mbar_wait_w(kv_full, 0, env);
     if (ok) {
       if (psi_group) {
         psi_k(0);
@@ -897,7 +897,7 @@ __global__ void __launch_bounds__(kReadThreads, 1)
     for (int c = 0; ok && c + 1 < n_chunks; ++c) {
       // operands of chunk c+1, whose tiles land in stage (c+1) % kReadStages
       const int st1 = (c + 1) % kReadStages;
-      if (!mbar_wait(kv_full + st1, ((c + 1) / kReadStages) & 1, env)) break;
+      if (!mbar_wait_w(kv_full + st1, ((c + 1) / kReadStages) & 1, env)) break;
       if (psi_group) {
         // psi~(k_{c+1}) into the buffer last read by the advance by chunk
         // c-1, which this group saw complete in the previous iteration
@@ -908,7 +908,7 @@ __global__ void __launch_bounds__(kReadThreads, 1)
         // of the chunk) has read psi~(q_c)
         uint32_t wq[kNPW];
         psi_q_formed(c + 1, wq);
-        if (!mbar_wait(rd_done, c & 1, env)) break;
+        if (!mbar_wait_w(rd_done, c & 1, env)) break;
         if (m == 0) KATA_TRACE(chunk, c, 19);
         tc_fence_after();
         store_psi_q_tmem(lane_base + L::colPQ, wq);
@@ -917,7 +917,7 @@ __global__ void __launch_bounds__(kReadThreads, 1)
       // the state after chunk c is complete: this group's half of the bf16
       // copy for the readout of chunk c+1 (its buffer was last read by the
       // readout of chunk c-1, which completed before this advance did)
-      if (!mbar_wait(upd_done, c & 1, env)) break;
+      if (!mbar_wait_w(upd_done, c & 1, env)) break;
       if (m == 0) KATA_TRACE(chunk, c, psi_group ? 15 : 16);
       tc_fence_after();
       if (quarter < 3) state_half_to_bf16(lane_base + L::colRun, sb + ((c + 1) & 1) * kSBBytes, m, active, half);
@@ -929,7 +929,7 @@ __global__ void __launch_bounds__(kReadThreads, 1)
     }
     // the last super-chunk ends at token T: its running state, once the
     // advance by its last chunk has landed, is the final state
-    if (S_out && g == G - 1 && n_chunks > 0 && !*abort_flag && mbar_wait(upd_done, (n_chunks - 1) & 1, env) &&
+    if (S_out && g == G - 1 && n_chunks > 0 && mbar_wait_w(upd_done, (n_chunks - 1) & 1, env) &&
         quarter < 3) {
       tc_fence_after();
       float* S = S_out + (size_t)bh * 256 * kDV;

@@ -280,9 +280,9 @@ __global__ void __launch_bounds__(kBwThreads, 1)
           tma_load_3d(smem + L::offV + st * C::kVBytes, &tm_v, kv_full + st, 0, j * kBw, bh);
         }
       }
-      for (int n = nq - 2 < 0 ? 0 : nq - 2; n < nq; ++n) mbar_wait_drain(q_full + (n & 1), (n >> 1) & 1, wc.limit);
+      for (int n = nq - 2 < 0 ? 0 : nq - 2; n < nq; ++n) mbar_wait_drain(q_full + (n & 1), (n >> 1) & 1);
       for (long n = rg - kBwStages < 0 ? 0 : rg - kBwStages; n < rg; ++n)
-        mbar_wait_drain(kv_full + n % kBwStages, (int)((n / kBwStages) & 1), wc.limit);
+        mbar_wait_drain(kv_full + n % kBwStages, (int)((n / kBwStages) & 1));
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
@@ -353,7 +353,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       gs += nkv;
     }
     mma_commit_w(done);
-    mbar_wait_drain(done, 0, wc.limit);
+    mbar_wait_drain(done, 0);
   } else {
     // ------------------------------------------------------------- weight warps + epilogue
     const int quarter = warp % 4;                 // rows (queries) 32 quarter ..
@@ -368,7 +368,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       const float2 rc = row < T ? rowc[(size_t)bh * T + row] : make_float2(0.f, 0.f);  // (-delta, 1/D)
       for (int j = 0; j < nkv; ++j) {
         const int g = gs + j;
-        if (!mbar_wait(s_full, g & 1, env)) {
+        if (!mbar_wait_w(s_full, g & 1, env)) {
           ok = false;
           break;
         }
@@ -408,7 +408,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         tc_fence_before();
         mbar_arrive(p_full + (g & 1));
       }
-      if (!ok || !mbar_wait(acc_full, acc_cnt & 1, env)) break;
+      if (!ok || !mbar_wait_w(acc_full, acc_cnt & 1, env)) break;
       ++acc_cnt;
       tc_fence_after();
       // epilogue: dQ (p fp32 columns) -> registers (warps of key quarter 0),
@@ -540,9 +540,9 @@ __global__ void __launch_bounds__(kBwThreads, 1)
           tma_load_3d(smem + L::offQ + st * C::kQKBytes, &tm_q, q_full + st, 0, i * kBw, bh);
         }
       }
-      for (int n = nq - 2 < 0 ? 0 : nq - 2; n < nq; ++n) mbar_wait_drain(kv_full + (n & 1), (n >> 1) & 1, wc.limit);
+      for (int n = nq - 2 < 0 ? 0 : nq - 2; n < nq; ++n) mbar_wait_drain(kv_full + (n & 1), (n >> 1) & 1);
       for (long n = rg - kBwStages < 0 ? 0 : rg - kBwStages; n < rg; ++n)
-        mbar_wait_drain(q_full + n % kBwStages, (int)((n / kBwStages) & 1), wc.limit);
+        mbar_wait_drain(q_full + n % kBwStages, (int)((n / kBwStages) & 1));
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
@@ -624,7 +624,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       gs += cnt;
     }
     mma_commit_w(done);
-    mbar_wait_drain(done, 0, wc.limit);
+    mbar_wait_drain(done, 0);
   } else {
     // ------------------------------------------------------------- weight warps + epilogue
     const int quarter = warp % 4;                 // rows (keys) 32 quarter ..
@@ -643,7 +643,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         // (-delta, 1/D) of this warp's 32 queries, one per lane (0 past T)
         const int qrow = (tile + n) * kBw + 32 * kq + lane;
         const float2 rcl = qrow < T ? rowc[(size_t)bh * T + qrow] : make_float2(0.f, 0.f);
-        if (!mbar_wait(s_full, (int)(g & 1), env)) {
+        if (!mbar_wait_w(s_full, (int)(g & 1), env)) {
           ok = false;
           break;
         }
@@ -682,7 +682,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         mbar_arrive(s_read);
         if (tslot >= 0) KATA_TRACE(bwd, g, tslot + 1);
         // the operand buffers are read by the previous query tile's MMAs
-        if (g > 0 && !mbar_wait(w_free, (int)((g - 1) & 1), env)) {
+        if (g > 0 && !mbar_wait_w(w_free, (int)((g - 1) & 1), env)) {
           ok = false;
           break;
         }
@@ -695,7 +695,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         mbar_arrive(p_full);
         if (tslot >= 0) KATA_TRACE(bwd, g, tslot + 3);
       }
-      if (!ok || !mbar_wait(acc_full, acc_cnt & 1, env)) break;
+      if (!ok || !mbar_wait_w(acc_full, acc_cnt & 1, env)) break;
       ++acc_cnt;
       tc_fence_after();
       // epilogue: dV (16 columns per key-quarter warp) and dK (p columns,

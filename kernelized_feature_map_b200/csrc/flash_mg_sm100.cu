@@ -201,9 +201,9 @@ __global__ void __launch_bounds__(kMgThreads, 1)
           load_rows(smem + Cfg::offV + st * Cfg::kVBytes, &tm_v, kv_full + st, j * kMgBN, bh);
         }
       }
-      for (int n = nq - 2 < 0 ? 0 : nq - 2; n < nq; ++n) mbar_wait_drain(q_full + (n & 1), (n >> 1) & 1, wc.limit);
+      for (int n = nq - 2 < 0 ? 0 : nq - 2; n < nq; ++n) mbar_wait_drain(q_full + (n & 1), (n >> 1) & 1);
       for (long n = g - kMgStages < 0 ? 0 : g - kMgStages; n < g; ++n)
-        mbar_wait_drain(kv_full + n % kMgStages, (int)((n / kMgStages) & 1), wc.limit);
+        mbar_wait_drain(kv_full + n % kMgStages, (int)((n / kMgStages) & 1));
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
@@ -310,7 +310,7 @@ __global__ void __launch_bounds__(kMgThreads, 1)
         g += nkv;
       }
       mma_commit_w(mma_done);
-      mbar_wait_drain(mma_done, 0, wc.limit);
+      mbar_wait_drain(mma_done, 0);
     }
   } else {
     // ------------------------------------------------------------- weights + epilogue
@@ -346,7 +346,7 @@ __global__ void __launch_bounds__(kMgThreads, 1)
         const bool skip = diag && kq > quarter;
         uint64_t acc[16];  // keys 2y, 2y + 1 of this warp's 32, fp32 pairs
         for (int r = 0; r < Cfg::kRounds; ++r) {
-          if (!mbar_wait(s_full, s_cnt & 1, env)) {
+          if (!mbar_wait_w(s_full, s_cnt & 1, env)) {
             ok = false;
             break;
           }
@@ -400,7 +400,7 @@ __global__ void __launch_bounds__(kMgThreads, 1)
         if (tslot >= 0) KATA_TRACE(mg, n_step - 1, tslot + 2);
         if (j == 0) flush_out();
       }
-      if (!ok || !mbar_wait(o_full, o_cnt & 1, env)) break;
+      if (!ok || !mbar_wait_w(o_full, o_cnt & 1, env)) break;
       ++o_cnt;
       tc_fence_after();
       uint32_t dbits, ov[16];

@@ -202,9 +202,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       // drain: every copy this CTA started must land before it exits
-      for (int n = nq - 2 < 0 ? 0 : nq - 2; n < nq; ++n) mbar_wait_drain(q_full + (n & 1), (n >> 1) & 1, wc.limit);
+      for (int n = nq - 2 < 0 ? 0 : nq - 2; n < nq; ++n) mbar_wait_drain(q_full + (n & 1), (n >> 1) & 1);
       for (long n = g - kStages < 0 ? 0 : g - kStages; n < g; ++n)
-        mbar_wait_drain(kv_full + n % kStages, (int)((n / kStages) & 1), wc.limit);
+        mbar_wait_drain(kv_full + n % kStages, (int)((n / kStages) & 1));
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
@@ -292,7 +292,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         g += nkv_max;
       }
       mma_commit_w(mma_done);
-      mbar_wait_drain(mma_done, 0, wc.limit);
+      mbar_wait_drain(mma_done, 0);
     }
   } else {
     // ------------------------------------------------------------- weights + epilogue
@@ -339,7 +339,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int bh = item_bh(it);
       const int row0 = (item_ct(it) * kNQ + i) * kBM + quarter * 32;  // this warp's first row
       for (int j = 0; j < nkv; ++j) {
-        if (!mbar_wait(s_full + i, s_cnt & 1, env)) {
+        if (!mbar_wait_w(s_full + i, s_cnt & 1, env)) {
           ok = false;
           break;
         }
@@ -386,7 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (m == 0 && h == 0) KATA_TRACE(flash, s_cnt - 1, 6 + 2 * i);
         if (j == 0) flush_out();
       }
-      if (!ok || !mbar_wait(o_full + i, o_cnt & 1, env)) break;
+      if (!ok || !mbar_wait_w(o_full + i, o_cnt & 1, env)) break;
       ++o_cnt;
       tc_fence_after();
       uint32_t dbits;

@@ -28,18 +28,45 @@ long long wait_limit() {
   return v < 0 ? kDefaultWaitLimit : v;
 }
 
-static int* status_word() {
-  static std::mutex mu;
-  static int* addr[64] = {nullptr};
+// Driver handle of the calling thread's current CUDA context, or nullptr
+// when none is current (or the driver entry point is unavailable).
+void* current_context() {
+  using Fn = CUresult (*)(CUcontext*);
+  static const Fn fn = []() -> Fn {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &qr) != cudaSuccess ||
+        qr != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<Fn>(f);
+  }();
+  CUcontext ctx = nullptr;
+  if (!fn || fn(&ctx) != CUDA_SUCCESS) return nullptr;
+  return ctx;
+}
+
+// Device address of a __device__ symbol on the current device, cached per
+// device and re-queried whenever the current context differs from the one
+// the cached address was taken in (after a device reset the module, and the
+// symbol with it, can move).
+void* SymbolCache::address(const void* symbol) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_kata_status) != cudaSuccess) return nullptr;
-    addr[dev] = static_cast<int*>(p);
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return nullptr;
+  std::lock_guard<std::mutex> lock(mu_);
+  void* ctx = current_context();
+  if (dev < kMaxDevices && ctx && ctx_[dev] == ctx && addr_[dev]) return addr_[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, symbol) != cudaSuccess) return nullptr;
+  if (dev < kMaxDevices) {
+    ctx_[dev] = current_context();  // the lookup made the device's context current
+    addr_[dev] = p;
   }
-  return addr[dev];
+  return p;
+}
+
+static int* status_word() {
+  static SymbolCache cache;
+  return static_cast<int*>(cache.address(&g_kata_status));
 }
 
 WaitCtl wait_ctl() { return WaitCtl{status_word(), wait_limit()}; }
@@ -158,10 +185,12 @@ KATA_API size_t kata_fwd_chunked_workspace_size(int B, int H, int T, int p, int 
   return make_chunk_plan(B, H, T, p, dv, C, dtype).workspace_bytes;
 }
 
-KATA_API kata_status_t kata_fwd_chunked(const void* q, const void* k, const void* v, void* o, int B, int H, int T,
-                                        int p, int dv, int C, kata_dtype_t dtype, const float* S0, const float* z0,
-                                        float* S_out, float* z_out, void* workspace, size_t workspace_bytes,
-                                        void* stream) {
+namespace kata {
+// Every argument check of kata_fwd_chunked except the workspace's, in the
+// order that call makes them.
+kata_status_t check_chunked_args(const void* q, const void* k, const void* v, const void* o, int B, int H, int T,
+                                 int p, int dv, int C, kata_dtype_t dtype, const float* S0, const float* z0,
+                                 const float* S_out, const float* z_out) {
   kata_status_t s = check_common(B, H, T, p, dv, dtype);
   if (s != KATA_OK) return s;
   if (!(C == 64 || C == 128)) return KATA_ERR_UNSUPPORTED;
@@ -169,6 +198,19 @@ KATA_API kata_status_t kata_fwd_chunked(const void* q, const void* k, const void
   if ((S_out == nullptr) != (z_out == nullptr)) return KATA_ERR_INVALID_ARG;
   for (const void* ptr : {(const void*)S0, (const void*)z0, (const void*)S_out, (const void*)z_out})
     if (ptr && !aligned16(ptr)) return KATA_ERR_MISALIGNED;
+  if (T == 0) return KATA_OK;
+  if (!q || !k || !v || !o) return KATA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return KATA_ERR_MISALIGNED;
+  return KATA_OK;
+}
+}  // namespace kata
+
+KATA_API kata_status_t kata_fwd_chunked(const void* q, const void* k, const void* v, void* o, int B, int H, int T,
+                                        int p, int dv, int C, kata_dtype_t dtype, const float* S0, const float* z0,
+                                        float* S_out, float* z_out, void* workspace, size_t workspace_bytes,
+                                        void* stream) {
+  kata_status_t s = check_chunked_args(q, k, v, o, B, H, T, p, dv, C, dtype, S0, z0, S_out, z_out);
+  if (s != KATA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const size_t P = (size_t)p * p, BH = (size_t)B * H;
   if (T == 0) {
@@ -182,8 +224,6 @@ KATA_API kata_status_t kata_fwd_chunked(const void* q, const void* k, const void
     if (e == cudaSuccess) e = cudaMemsetAsync(z_out, 0, BH * P * sizeof(float), st);
     return from_cuda(e);
   }
-  if (!q || !k || !v || !o) return KATA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return KATA_ERR_MISALIGNED;
   const ChunkPlan plan = make_chunk_plan(B, H, T, p, dv, C, dtype);
   if (plan.workspace_bytes > 0) {
     if (!workspace || workspace_bytes < plan.workspace_bytes) return KATA_ERR_WORKSPACE;

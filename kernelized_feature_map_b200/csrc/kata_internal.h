@@ -6,6 +6,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "../../include/kata.h"
 
 namespace kata {
@@ -43,6 +45,11 @@ inline bool chunked_on_tensor_cores(int p, int dv, kata_dtype_t dt) {
 }
 
 ChunkPlan make_chunk_plan(int B, int H, int T, int p, int dv, int C, kata_dtype_t dt);
+
+// Every argument check of kata_fwd_chunked except the workspace's (kata_api.cu).
+kata_status_t check_chunked_args(const void* q, const void* k, const void* v, const void* o, int B, int H, int T,
+                                 int p, int dv, int C, kata_dtype_t dtype, const float* S0, const float* z0,
+                                 const float* S_out, const float* z_out);
 
 // decode.cu -- `groups` PSD factors of width p per head (1: the single-factor step)
 cudaError_t launch_decode(const void* q, const void* k, const void* v, void* o, float* S, float* z,
@@ -105,5 +112,20 @@ cudaError_t launch_chunk_readout_sm100(const void* q, const void* k, const void*
 
 // Current bound on in-kernel waits and the status word (kata_api.cu).
 WaitCtl wait_ctl();
+
+// Device addresses of file-scope __device__ arrays, for host code (kata_api.cu).
+void* current_context();
+class SymbolCache {
+ public:
+  // Address of `symbol` (the host-side name of a __device__ variable) on the
+  // current device, or nullptr on failure.  Thread-safe.
+  void* address(const void* symbol);
+
+ private:
+  static constexpr int kMaxDevices = 64;
+  std::mutex mu_;
+  void* ctx_[kMaxDevices] = {};
+  void* addr_[kMaxDevices] = {};
+};
 
 }  // namespace kata

@@ -17,38 +17,29 @@
 // in the array needs to start at zero: every record the path reads was
 // written earlier in the same call.
 //
-// The device address of the array is looked up once per device, with that
-// device current, by the first call made on it (cudaGetSymbolAddress); make
-// that first call before any stream capture.  Host code never uses the
-// array's name as an address.
+// The device address of the array is looked up with that device current by
+// the first call made on it (cudaGetSymbolAddress), and again whenever the
+// calling thread's CUDA context is no longer the one the address was taken
+// in (after a device reset the array can move); make that first call before
+// any stream capture.  Host code never uses the array's name as an address.
 #include <cuda_runtime.h>
 
-#include <mutex>
-
-#include "../../include/kata.h"
+#include "kata_internal.h"
 
 #define KATA_API extern "C" __attribute__((visibility("default")))
 
 namespace kata {
 namespace {
 
-constexpr size_t kNoallocScratchBytes = 16u << 20;
+constexpr size_t kNoallocScratchBytes = KATA_NOALLOC_SCRATCH_BYTES;
+static_assert(kNoallocScratchBytes == (size_t)16 << 20, "the scratch size stated in kata.h");
 
 static __device__ __align__(256) float g_noalloc_scratch[kNoallocScratchBytes / sizeof(float)];
 
 // Device address of g_noalloc_scratch on the current device, or nullptr.
 void* scratch_address() {
-  static std::mutex mu;
-  static void* addr[64] = {nullptr};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
-    addr[dev] = p;
-  }
-  return addr[dev];
+  static SymbolCache cache;
+  return cache.address(&g_noalloc_scratch);
 }
 
 }  // namespace
@@ -57,8 +48,9 @@ void* scratch_address() {
 KATA_API kata_status_t kata_fwd_chunked_noalloc(const void* q, const void* k, const void* v, void* o, int B, int H,
                                                 int T, int p, int dv, int C, kata_dtype_t dtype, const float* S0,
                                                 const float* z0, float* S_out, float* z_out, void* stream) {
-  // argument and shape errors are reported by the workspace query (0 bytes)
-  // and by kata_fwd_chunked itself, exactly as for the allocating call
+  // the argument errors of kata_fwd_chunked, in its order, before the size
+  kata_status_t s = kata::check_chunked_args(q, k, v, o, B, H, T, p, dv, C, dtype, S0, z0, S_out, z_out);
+  if (s != KATA_OK) return s;
   const size_t need = kata_fwd_chunked_workspace_size(B, H, T, p, dv, C, dtype);
   if (need > kata::kNoallocScratchBytes) return KATA_ERR_WORKSPACE;
   void* scratch = nullptr;

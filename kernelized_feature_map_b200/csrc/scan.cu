@@ -35,41 +35,34 @@ namespace kata {
 constexpr int kScanBlock = 1024;  // records per shared-memory pass
 constexpr int kScanThreads = 256;
 
-// packed coordinate -> (i, j), -1 for a pad (p = 16)
-__constant__ signed char c_pack_i[144];
-__constant__ signed char c_pack_j[144];
-
+// packed coordinate -> (i, j), -1 for a pad (p = 16): runs i = 0..15 of
+// (i, j >= i), each padded to even length.  Built at compile time, so no
+// upload (and no host-side state) is needed before the first launch.
 struct PackTable {
   signed char i[144], j[144];
-  PackTable() {
-    int w = 0;
-    for (int a = 0; a < 16; ++a) {
-      for (int b = a; b < 16; ++b) {
-        i[w] = (signed char)a;
-        j[w] = (signed char)b;
-        ++w;
-      }
-      if ((16 - a) & 1) {
-        i[w] = -1;
-        j[w] = -1;
-        ++w;
-      }
+};
+constexpr PackTable make_pack_table() {
+  PackTable t{};
+  int w = 0;
+  for (int a = 0; a < 16; ++a) {
+    for (int b = a; b < 16; ++b) {
+      t.i[w] = (signed char)a;
+      t.j[w] = (signed char)b;
+      ++w;
+    }
+    if ((16 - a) & 1) {
+      t.i[w] = -1;
+      t.j[w] = -1;
+      ++w;
     }
   }
-};
-
-static cudaError_t upload_pack_table() {
-  static int done_mask = 0;  // per device bit
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 31 && (done_mask >> dev) & 1) return cudaSuccess;
-  static const PackTable tab;
-  e = cudaMemcpyToSymbol(c_pack_i, tab.i, sizeof(tab.i));
-  if (e == cudaSuccess) e = cudaMemcpyToSymbol(c_pack_j, tab.j, sizeof(tab.j));
-  if (e == cudaSuccess && dev < 31) done_mask |= 1 << dev;
-  return e;
+  return t;
 }
+constexpr PackTable kPackTable = make_pack_table();
+static_assert(kPackTable.i[16] == 1 && kPackTable.j[16] == 1 && kPackTable.i[31] == -1 &&
+                  kPackTable.j[142] == 15 && kPackTable.i[143] == -1,
+              "packed psi coordinate layout");
+__constant__ PackTable c_pack = kPackTable;
 
 struct ScanArgs {
   float* ws;
@@ -95,7 +88,7 @@ __device__ __forceinline__ float initial_entry(const ScanArgs& a, long long bh, 
     return 0.f;
   }
   const int d = e / 144, w = e % 144;
-  const int i = c_pack_i[w], j = c_pack_j[w];
+  const int i = c_pack.i[w], j = c_pack.j[w];
   if (i < 0) return 0.f;
   const int r1 = i * 16 + j, r2 = j * 16 + i;
   if (d < 64) {
@@ -115,7 +108,7 @@ __device__ __forceinline__ void final_entry(const ScanArgs& a, long long bh, int
     return;
   }
   const int d = e / 144, w = e % 144;
-  const int i = c_pack_i[w], j = c_pack_j[w];
+  const int i = c_pack.i[w], j = c_pack.j[w];
   if (i < 0) return;
   const float h = i == j ? val : 0.5f * val;  // symmetric halves (exact)
   const int r1 = i * 16 + j, r2 = j * 16 + i;
@@ -255,10 +248,6 @@ __global__ void __launch_bounds__(kScanRegThreads) state_scan_reg_kernel(ScanArg
 
 cudaError_t launch_state_scan(float* ws, const ChunkPlan& plan, int G_in, const float* S0, const float* z0,
                               float* S_out, float* z_out, cudaStream_t st) {
-  if (plan.layout == kRecPackedT) {
-    cudaError_t e = upload_pack_table();
-    if (e != cudaSuccess) return e;
-  }
   ScanArgs a;
   a.ws = ws;
   a.G = plan.G;

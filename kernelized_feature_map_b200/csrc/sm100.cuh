@@ -85,17 +85,39 @@ struct WaitEnv {
   long long limit;
 };
 
+// Non-blocking test for the completion of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// A plain try_wait may itself block for a short, hardware-defined time, so
+// a limit of 0 is tested without blocking: it gives up at once when the
+// phase has not already completed.  Otherwise the abort flag and the limit
+// are checked before each sleep.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitEnv& env) {
+  if (env.limit == 0 && !mbar_test_wait(bar, parity)) {
+    *env.abort_flag = 1;
+    report_status(env.status, kErrTimeout);
+    return false;
+  }
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
-    if (mbar_try_wait_sleep(bar, parity)) return true;
     if (*env.abort_flag) return false;
-    if (clock64() - t0 > env.limit) {
+    if (clock64() - t0 >= env.limit) {
       *env.abort_flag = 1;
       report_status(env.status, kErrTimeout);
       return false;
     }
+    if (mbar_try_wait_sleep(bar, parity)) return true;
   }
 }
 
@@ -106,13 +128,17 @@ __device__ __forceinline__ bool mbar_wait_w(uint64_t* bar, uint32_t parity, cons
   return __all_sync(0xffffffffu, ok);
 }
 
-// Bounded wait used while tearing down after an abort: ignores the abort
-// flag (it is waiting for the CTA's own copies and MMAs to land).
-__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, long long limit) {
+// Bounded wait used while tearing down: ignores the abort flag, since it
+// waits for the CTA's own TMA copies and MMAs, which complete by themselves.
+// Its bound is fixed (about a second of SM cycles), independent of the
+// caller-set limit of the other waits, so that a CTA that gave up early
+// still lets everything it issued land before it frees TMEM and exits.
+constexpr long long kDrainLimit = 1ll << 31;
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try_wait_sleep(bar, parity)) {
-    if (clock64() - t0 > limit) return false;
+    if (clock64() - t0 > kDrainLimit) return false;
   }
   return true;
 }

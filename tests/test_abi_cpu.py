@@ -194,3 +194,12 @@ def test_sg_argument_errors_before_launch(L):
     assert f(a, b, c, d, 1, 1, 16, 64, 2, 64, 5, 1, st) == _abi.KATA_ERR_INVALID_ARG   # layout
     assert f(a, b, c, d, 1, 1, 16, 64, 2, 64, 0, 0, st) == _abi.KATA_ERR_UNSUPPORTED   # fp32
     assert f(a, b, c, d, 1, 1, 0, 64, 2, 64, 1, 1, st) == _abi.KATA_OK
+
+
+def test_noalloc_scratch_size_matches_header():
+    """The binding's copy of the no-allocation scratch size is the header's
+    KATA_NOALLOC_SCRATCH_BYTES (the library asserts the same at build time)."""
+    text = open(os.path.join(ROOT, "include", "kata.h")).read()
+    m = re.search(r"#define KATA_NOALLOC_SCRATCH_BYTES \(\(size_t\)(\d+) << (\d+)\)", text)
+    assert m
+    assert _abi.NOALLOC_SCRATCH_BYTES == int(m.group(1)) << int(m.group(2))
