@@ -175,10 +175,13 @@ class ClockSampler:
             except Exception:
                 self.proc.kill()
 
-    def summary(self):
+    def summary(self, window=None):
+        """Median SM clock, max clock and throttle reasons over `window`
+        (host times; default: the whole timed region)."""
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        lo, hi = self.window if self.window else (0.0, float("inf"))
+        window = window or self.window
+        lo, hi = window if window else (0.0, float("inf"))
         for ts, line in self.lines:
             # a sample describes the interval before it was printed
             if ts < lo or ts > hi + 0.1:
@@ -281,7 +284,10 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
 
     recs, grecs = [], []
-    with ClockSampler(local_rank) as clk:
+    windows = {}
+    clk = ClockSampler(local_rank)
+    clk.__enter__()
+    try:  # the clock record covers every timed part below
         clk.wait_first_sample()
         barrier()
         torch.cuda.synchronize()
@@ -300,95 +306,105 @@ def run_ours(args, rank, world, local_rank):
                 flush.fill_(1)
                 grecs.append((a, b))
         torch.cuda.synchronize()
-        clk.window = (t_start, time.time())
+        windows["step"] = (t_start, time.time())
         barrier()
+        per = np.array([[r[0].elapsed_time(r[1]), r[1].elapsed_time(r[2]), r[2].elapsed_time(r[3])] for r in recs])
+        eager_step_ms = float(per.sum(axis=1).mean())
+        step_ms = float(np.mean([a.elapsed_time(b) for a, b in grecs])) if grecs else eager_step_ms
+        path_ms = per.mean(axis=0)
+        if graph is not None:
+            del graph
+
+        # end to end through the public API with host buffers.  Every step copies
+        # its inputs host -> device from pinned memory, runs the three calls and
+        # copies its three outputs device -> host.  Steps are pipelined over three
+        # streams with two sets of device buffers: the H2D copy of step i, the
+        # compute of step i-1 and the D2H copy of step i-2 overlap (PCIe is full
+        # duplex and the copy engines run beside the SMs).  The L2 is flushed on
+        # the compute stream before every step.
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdq, hdk, hdv))
+        d2h = sum(t.numel() * t.element_size() for t in (o_quad, o_chunk, o_dec))
+        sets = []
+        for _b in range(2):
+            sets.append(dict(
+                q=torch.empty_like(q), k=torch.empty_like(k), v=torch.empty_like(v),
+                qd=torch.empty_like(qd), kd=torch.empty_like(kd), vd=torch.empty_like(vd),
+                oq=torch.empty_like(o_quad), oc=torch.empty_like(o_chunk), od=torch.empty_like(o_dec),
+                S=torch.empty_like(S), z=torch.empty_like(z), ws=torch.empty_like(ws),
+                hoq=torch.empty(o_quad.shape, dtype=bf).pin_memory(), hoc=torch.empty(o_chunk.shape, dtype=bf).pin_memory(),
+                hod=torch.empty(o_dec.shape, dtype=bf).pin_memory()))
+        s_h2d, s_cmp, s_d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_cmp = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
+
+        def e2e_run(nsteps):
+            for i in range(nsteps):
+                bi = i % 2
+                st_ = sets[bi]
+                with torch.cuda.stream(s_h2d):
+                    if i >= 2:
+                        s_h2d.wait_event(ev_cmp[bi])  # step i-2 has finished reading this set's inputs
+                    for dst, src in ((st_["q"], hq), (st_["k"], hk), (st_["v"], hv), (st_["qd"], hdq), (st_["kd"], hdk),
+                                     (st_["vd"], hdv)):
+                        dst.copy_(src, non_blocking=True)
+                    ev_in[bi].record(s_h2d)
+                with torch.cuda.stream(s_cmp):
+                    s_cmp.wait_event(ev_in[bi])
+                    if i >= 2:
+                        s_cmp.wait_event(ev_out[bi])  # step i-2's outputs have been copied out
+                    flush.fill_(1)
+                    K.kata_fwd_quadratic(st_["q"], st_["k"], st_["v"], o=st_["oq"])
+                    K.kata_fwd_chunked(st_["q"], st_["k"], st_["v"], C=C, o=st_["oc"], workspace=st_["ws"],
+                                       S_out=st_["S"], z_out=st_["z"], return_state=True)
+                    K.kata_decode_step(st_["qd"], st_["kd"], st_["vd"], st_["S"], st_["z"], o=st_["od"])
+                    ev_cmp[bi].record(s_cmp)
+                with torch.cuda.stream(s_d2h):
+                    s_d2h.wait_event(ev_cmp[bi])
+                    st_["hoq"].copy_(st_["oq"], non_blocking=True)
+                    st_["hoc"].copy_(st_["oc"], non_blocking=True)
+                    st_["hod"].copy_(st_["od"], non_blocking=True)
+                    ev_out[bi].record(s_d2h)
+
+        e2e_run(4)
+        torch.cuda.synchronize()
+        n_e2e = min(40, max(8, args.steps // 2))
+        e_start, e_end = ev(), ev()
+        e_start.record(s_h2d)
+        s_cmp.wait_stream(s_h2d)
+        s_d2h.wait_stream(s_h2d)
+        e2e_run(n_e2e)
+        s_d2h.wait_stream(s_cmp)
+        s_d2h.wait_stream(s_h2d)
+        e_end.record(s_d2h)
+        torch.cuda.synchronize()
+        e2e_ms = e_start.elapsed_time(e_end) / n_e2e
+
+        # long context: chunked (and quadratic) at T = 131072, and the decode
+        # step at the serving batch; each timed inside the clock record
+        long = None
+        if args.long and world == 1:
+            t0 = time.time()
+            long = run_long(args, K, torch, dev, stream, flush)
+            windows["long_ctx"] = (t0, time.time())
+            t0 = time.time()
+            long["decode_b64"] = run_decode_b64(args, K, torch, dev, stream, flush)
+            windows["decode_b64"] = (t0, time.time())
+            if args.sweep:
+                long["sweep"], long["recall"] = run_sweep(args, K, torch, dev, stream, flush)
+                long["mg"] = run_mg(args, K, torch, dev, stream, flush)
+                long["train"] = run_train(args, K, torch, dev, stream, flush)
+        t_end = time.time()
         time.sleep(0.15)
-    per = np.array([[r[0].elapsed_time(r[1]), r[1].elapsed_time(r[2]), r[2].elapsed_time(r[3])] for r in recs])
-    eager_step_ms = float(per.sum(axis=1).mean())
-    step_ms = float(np.mean([a.elapsed_time(b) for a, b in grecs])) if grecs else eager_step_ms
-    path_ms = per.mean(axis=0)
-    if graph is not None:
-        del graph
-
-    # end to end through the public API with host buffers.  Every step copies
-    # its inputs host -> device from pinned memory, runs the three calls and
-    # copies its three outputs device -> host.  Steps are pipelined over three
-    # streams with two sets of device buffers: the H2D copy of step i, the
-    # compute of step i-1 and the D2H copy of step i-2 overlap (PCIe is full
-    # duplex and the copy engines run beside the SMs).  The L2 is flushed on
-    # the compute stream before every step.
-    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdq, hdk, hdv))
-    d2h = sum(t.numel() * t.element_size() for t in (o_quad, o_chunk, o_dec))
-    sets = []
-    for _b in range(2):
-        sets.append(dict(
-            q=torch.empty_like(q), k=torch.empty_like(k), v=torch.empty_like(v),
-            qd=torch.empty_like(qd), kd=torch.empty_like(kd), vd=torch.empty_like(vd),
-            oq=torch.empty_like(o_quad), oc=torch.empty_like(o_chunk), od=torch.empty_like(o_dec),
-            S=torch.empty_like(S), z=torch.empty_like(z), ws=torch.empty_like(ws),
-            hoq=torch.empty(o_quad.shape, dtype=bf).pin_memory(), hoc=torch.empty(o_chunk.shape, dtype=bf).pin_memory(),
-            hod=torch.empty(o_dec.shape, dtype=bf).pin_memory()))
-    s_h2d, s_cmp, s_d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    ev_in = [torch.cuda.Event() for _ in range(2)]
-    ev_cmp = [torch.cuda.Event() for _ in range(2)]
-    ev_out = [torch.cuda.Event() for _ in range(2)]
-
-    def e2e_run(nsteps):
-        for i in range(nsteps):
-            bi = i % 2
-            st_ = sets[bi]
-            with torch.cuda.stream(s_h2d):
-                if i >= 2:
-                    s_h2d.wait_event(ev_cmp[bi])  # step i-2 has finished reading this set's inputs
-                for dst, src in ((st_["q"], hq), (st_["k"], hk), (st_["v"], hv), (st_["qd"], hdq), (st_["kd"], hdk),
-                                 (st_["vd"], hdv)):
-                    dst.copy_(src, non_blocking=True)
-                ev_in[bi].record(s_h2d)
-            with torch.cuda.stream(s_cmp):
-                s_cmp.wait_event(ev_in[bi])
-                if i >= 2:
-                    s_cmp.wait_event(ev_out[bi])  # step i-2's outputs have been copied out
-                flush.fill_(1)
-                K.kata_fwd_quadratic(st_["q"], st_["k"], st_["v"], o=st_["oq"])
-                K.kata_fwd_chunked(st_["q"], st_["k"], st_["v"], C=C, o=st_["oc"], workspace=st_["ws"],
-                                   S_out=st_["S"], z_out=st_["z"], return_state=True)
-                K.kata_decode_step(st_["qd"], st_["kd"], st_["vd"], st_["S"], st_["z"], o=st_["od"])
-                ev_cmp[bi].record(s_cmp)
-            with torch.cuda.stream(s_d2h):
-                s_d2h.wait_event(ev_cmp[bi])
-                st_["hoq"].copy_(st_["oq"], non_blocking=True)
-                st_["hoc"].copy_(st_["oc"], non_blocking=True)
-                st_["hod"].copy_(st_["od"], non_blocking=True)
-                ev_out[bi].record(s_d2h)
-
-    e2e_run(4)
-    torch.cuda.synchronize()
-    n_e2e = min(40, max(8, args.steps // 2))
-    e_start, e_end = ev(), ev()
-    e_start.record(s_h2d)
-    s_cmp.wait_stream(s_h2d)
-    s_d2h.wait_stream(s_h2d)
-    e2e_run(n_e2e)
-    s_d2h.wait_stream(s_cmp)
-    s_d2h.wait_stream(s_h2d)
-    e_end.record(s_d2h)
-    torch.cuda.synchronize()
-    e2e_ms = e_start.elapsed_time(e_end) / n_e2e
-
-    # long context: chunked (and quadratic) at T = 131072
-    long = None
-    if args.long and world == 1:
-        long = run_long(args, K, torch, dev, stream, flush)
-        long["decode_b64"] = run_decode_b64(args, K, torch, dev, stream, flush)
-        if args.sweep:
-            long["sweep"], long["recall"] = run_sweep(args, K, torch, dev, stream, flush)
-            long["mg"] = run_mg(args, K, torch, dev, stream, flush)
-            long["train"] = run_train(args, K, torch, dev, stream, flush)
-
-    status = K.kata_get_status()
-    return dict(step_ms=step_ms, eager_step_ms=eager_step_ms, graph=bool(args.graph), path_ms=path_ms.tolist(),
-                e2e_ms=e2e_ms, h2d=h2d, d2h=d2h,
-                clocks=clk.summary(), timed_s=clk.window[1] - clk.window[0], long=long, status=status, tokens=B * T, BH=BH, T=T, p=p, dv=dv, C=C)
+        clk.window = (windows["step"][0], windows.get("decode_b64", windows["step"])[1])
+        status = K.kata_get_status()
+        return dict(step_ms=step_ms, eager_step_ms=eager_step_ms, graph=bool(args.graph), path_ms=path_ms.tolist(),
+                    e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, clocks=clk.summary(),
+                    clocks_by_part={name: clk.summary(w) for name, w in windows.items()},
+                    timed_s=t_end - windows["step"][0], long=long, status=status, tokens=B * T, BH=BH, T=T, p=p, dv=dv,
+                    C=C)
+    finally:
+        clk.__exit__()
 
 
 def run_decode_b64(args, K, torch, dev, stream, flush):
@@ -624,6 +640,62 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------------------
+# --case: one call of the library a few times on device-drawn inputs, for
+# profilers (ncu wants a short program that launches the kernel of interest a
+# known number of times); nothing is timed or printed but the call's status
+# ---------------------------------------------------------------------------
+def run_case(args):
+    import torch
+    import kernelized_feature_map_b200 as K
+
+    dev = torch.device("cuda")
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(args.seed)
+    bf = torch.bfloat16
+
+    def unit(shape):
+        x = torch.randn(shape, generator=gen, device=dev)
+        return (x / x.norm(dim=-1, keepdim=True)).to(bf)
+
+    B, H, T, d, dv, g = args.B, args.H, args.T, args.d, args.dv, args.groups
+    if args.case == "decode":
+        p = d // g
+        q, k = unit((B, H, d)), unit((B, H, d))
+        v = torch.randn((B, H, dv), generator=gen, device=dev).to(bf)
+        S = torch.zeros((B, H, g * p * p, dv), dtype=torch.float32, device=dev)
+        z = torch.zeros((B, H, g * p * p), dtype=torch.float32, device=dev)
+        call = lambda: K.kata_decode_step_mg(q, k, v, S, z, g)  # noqa: E731
+    else:
+        lead = (B, T, H) if args.layout == "bthd" else (B, H, T)
+        q, k = unit(lead + (d,)), unit(lead + (d,))
+        v = torch.randn(lead + (dv,), generator=gen, device=dev).to(bf)
+        o = torch.empty_like(v)
+        if args.case == "mg":
+            call = lambda: K.kata_fwd_mg_quadratic(q, k, v, g, layout=args.layout, o=o)  # noqa: E731
+        elif args.layout != "bhtd":
+            raise SystemExit("--layout bthd is for --case mg")
+        elif args.case == "quadratic":
+            call = lambda: K.kata_fwd_quadratic(q, k, v, o=o)  # noqa: E731
+        elif args.case == "train":
+            dO = torch.randn(v.shape, generator=gen, device=dev).to(bf)
+            D = torch.empty((B, H, T), dtype=torch.float32, device=dev)
+
+            def call():
+                K.kata_fwd_quadratic_train(q, k, v, o=o, D=D)
+                K.kata_bwd_quadratic(q, k, v, o, D, dO)
+        else:
+            ws = torch.empty(max(256, K.kata_fwd_chunked_workspace_size(B, H, T, d, dv, args.C, bf)),
+                             dtype=torch.uint8, device=dev)
+            call = lambda: K.kata_fwd_chunked(q, k, v, C=args.C, o=o, workspace=ws)  # noqa: E731
+    for _ in range(args.reps):
+        call()
+    torch.cuda.synchronize()
+    status = K.kata_get_status()
+    print("%s reps=%d status=%d (%s)" % (args.case, args.reps, status, K.status_string(status)))
+    return 0 if status == 0 else 1
+
+
 def config_dict(cfg, world):
     return {"workload": "%s: B=%d H=%d T=%d p=%d dv=%d C=%d bf16" % (
         "340M-layer shape" if cfg["T"] == 2048 else cfg.get("kind", ""), cfg["B"], cfg["H"], cfg["T"], cfg["p"],
@@ -648,7 +720,21 @@ def main():
     ap.add_argument("--cpu-baseline", type=int, default=1)
     ap.add_argument("--graph", type=int, default=1, help="time the step as a CUDA graph replay (per-path times stay eager)")
     ap.add_argument("--ref-budget", type=float, default=15.0, help="seconds of oracle work per reference step")
+    pc = ap.add_argument_group("--case: launch one call a few times on device-drawn inputs (for profilers)")
+    pc.add_argument("--case", choices=["quadratic", "chunked", "mg", "decode", "train"])
+    pc.add_argument("--B", type=int, default=8)
+    pc.add_argument("--H", type=int, default=16)
+    pc.add_argument("--T", type=int, default=2048)
+    pc.add_argument("--d", type=int, default=16, help="q/k width (p for the single-factor paths)")
+    pc.add_argument("--dv", type=int, default=64)
+    pc.add_argument("--groups", type=int, default=1)
+    pc.add_argument("--layout", choices=["bhtd", "bthd"], default="bhtd")
+    pc.add_argument("--C", type=int, default=64)
+    pc.add_argument("--reps", type=int, default=3)
+    pc.add_argument("--seed", type=int, default=0)
     args = ap.parse_args()
+    if args.case:
+        sys.exit(run_case(args))
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
@@ -681,6 +767,47 @@ def main():
         if world > 1:
             import torch.distributed as dist
             dist.destroy_process_group()
+
+
+def roofline_points(res, peaks, cfg):
+    """Each path of the metric on its own: tokens/s and the fraction of its
+    binding roofline at T = 2048 (the step's batch, eager per-path times) and
+    at T = 131072 (chunked C = 64 and 128, and quadratic), plus the decode
+    step at B = 64; each with the clocks sampled while it was timed."""
+    hb, tf = peaks["hbm_gbs"], peaks["bf16_tflops"]
+    cl = res.get("clocks_by_part", {})
+    BH, T, p, dv = res["BH"], res["T"], res["p"], res["dv"]
+    tok = res["tokens"]
+    quad_ms, chunk_ms, _ = res["path_ms"]
+
+    def hbm_point(path, workload, ms, tokens, nbytes, clocks, **kw):
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        return dict(path=path, workload=workload, ms=ms, tokens_per_s=tokens / (ms * 1e-3), bound="hbm",
+                    achieved=gbs, peak=hb, unit="GB/s", frac=gbs / hb, clocks=clocks, **kw)
+
+    def tensor_point(path, workload, ms, tokens, flops, clocks, **kw):
+        tfs = flops / (ms * 1e-3) / 1e12
+        return dict(path=path, workload=workload, ms=ms, tokens_per_s=tokens / (ms * 1e-3), bound="tensor",
+                    achieved=tfs, peak=tf, unit="TFLOP/s", frac=tfs / tf, clocks=clocks, **kw)
+
+    w2k = "B=%d H=%d T=%d p=%d dv=%d bf16" % (BH // cfg["H"], cfg["H"], T, p, dv)
+    pts = [tensor_point("quadratic", w2k, quad_ms, tok, flash_flops(BH, T, p, dv), cl.get("step"), T=T),
+           hbm_point("chunked", w2k, chunk_ms, tok, chunked_bytes(BH, T, p, dv), cl.get("step"), T=T, C=res["C"])]
+    lg = res.get("long")
+    if lg:
+        lbh, ltok = lg["B"] * lg["H"], lg["B"] * lg["T"]
+        wl = "B=%d H=%d T=%d p=%d dv=%d bf16" % (lg["B"], lg["H"], lg["T"], lg["p"], lg["dv"])
+        for C in (64, 128):
+            pts.append(hbm_point("chunked", wl, lg["chunked_C%d_ms" % C], ltok,
+                                 chunked_bytes(lbh, lg["T"], lg["p"], lg["dv"]), cl.get("long_ctx"), T=lg["T"], C=C))
+        pts.append(tensor_point("quadratic", wl, lg["quadratic_ms"], ltok, flash_flops(lbh, lg["T"], lg["p"], lg["dv"]),
+                                cl.get("long_ctx"), T=lg["T"]))
+        dc = lg["decode_b64"]
+        pts.append(hbm_point("decode", "decode step B=%d H=%d state [%d x %d] fp32" % (dc["B"], dc["H"], dc["p"] ** 2,
+                                                                                     dc["dv"]),
+                             dc["ms"], dc["B"], decode_bytes(dc["B"] * dc["H"], dc["p"], dc["dv"]),
+                             cl.get("decode_b64")))
+    return pts
 
 
 def report(args, res, step_ms, e2e_ms, world):
@@ -790,6 +917,7 @@ def report(args, res, step_ms, e2e_ms, world):
                 "fwd_ms": tr["fwd_ms"], "bwd_ms": tr["bwd_ms"],
                 "bwd_tensor_frac": bwd_flops / (tr["bwd_ms"] * 1e-3) / 1e12 / peaks["bf16_tflops"],
                 "bwd_algorithmic": "2(3p+2dv) flops per causal pair: S, dP, dV, dQ, dK"}
+    line["roofline"]["points"] = roofline_points(res, peaks, cfg)
     if args.cpu_baseline and world == 1:
         cb = time_oracle(cfg)
         line["cpu_baseline"] = {"value": cb["value"], "unit": UNIT, "cores": cb["cores"], "kind": "oracle",

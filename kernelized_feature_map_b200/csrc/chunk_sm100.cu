@@ -407,14 +407,19 @@ __device__ __forceinline__ uint64_t desc_vones(uint32_t sV, uint32_t sOnes) {
 // ===========================================================================
 constexpr int kStateThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2-9 psi~(k), warps 2-5 record
 constexpr int kStateStages = 6;
+// psi~(K) buffers.  Measured at B1 H16 T131072: 6 stages with 2 buffers
+// 243 us for the whole chunked call, 4 with 3 buffers 252 us, 3 with 4
+// buffers 259 us -- the deeper TMA ring matters more than forming psi~(K)
+// further ahead
+constexpr int kStatePsiBufs = 2;
 
 struct StateSmem {
   static constexpr int kStage = kVBytes + kQKBytes;  // [V | K]
   static constexpr int offStage = 0;
   static constexpr int offOnes = offStage + kStateStages * kStage;  // 1024-aligned
-  static constexpr int offPsi = offOnes + kOnesBytes;                 // 2 buffers
-  static constexpr int offBar = offPsi + 2 * kPsiBytes;
-  static constexpr int kBars = 2 * kStateStages + 4 + 1;
+  static constexpr int offPsi = offOnes + kOnesBytes;                 // kStatePsiBufs buffers
+  static constexpr int offBar = offPsi + kStatePsiBufs * kPsiBytes;
+  static constexpr int kBars = 2 * kStateStages + 2 * kStatePsiBufs + 1;
   static constexpr int offMisc = offBar + kBars * 8;
   static constexpr int kBytes = offMisc + 16 + 1024;
 };
@@ -428,9 +433,9 @@ __global__ void __launch_bounds__(kStateThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::offBar);
   uint64_t* kv_full = bars;
   uint64_t* kv_empty = kv_full + kStateStages;
-  uint64_t* psi_full = kv_empty + kStateStages;  // [2]
-  uint64_t* psi_empty = psi_full + 2;            // [2]
-  uint64_t* acc_done = psi_empty + 2;
+  uint64_t* psi_full = kv_empty + kStateStages;  // [kStatePsiBufs]
+  uint64_t* psi_empty = psi_full + kStatePsiBufs;
+  uint64_t* acc_done = psi_empty + kStatePsiBufs;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::offMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::offMisc + 4);
 
@@ -445,7 +450,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
       mbar_init(kv_full + s, 1);
       mbar_init(kv_empty + s, 1);
     }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kStatePsiBufs; ++s) {
       mbar_init(psi_full + s, 256);
       mbar_init(psi_empty + s, 1);
     }
@@ -487,9 +492,9 @@ __global__ void __launch_bounds__(kStateThreads, 1)
       const uint32_t sPsi = smem_u32(smem + L::offPsi);
       const uint64_t dpsi = smem_desc(sPsi, kPsiAtom, 256, kSw32);
       for (int c = 0; c < n_chunks; ++c) {
-        const int st = c % kStateStages, pb = c & 1;
+        const int st = c % kStateStages, pb = c % kStatePsiBufs;
         if (!mbar_wait_w(kv_full + st, (c / kStateStages) & 1, env)) break;
-        if (!mbar_wait_w(psi_full + pb, (c >> 1) & 1, env)) break;
+        if (!mbar_wait_w(psi_full + pb, (c / kStatePsiBufs) & 1, env)) break;
         KATA_TRACE(chunkstate, c, 0);
         tc_fence_after();
         const uint32_t sV = sStage + st * L::kStage;
@@ -512,13 +517,13 @@ __global__ void __launch_bounds__(kStateThreads, 1)
     const int d = quarter * 32 + lane;  // TMEM lane = record row
     bool ok = true;
     for (int c = 0; c < n_chunks; ++c) {
-      const int st = c % kStateStages, pb = c & 1;
+      const int st = c % kStateStages, pb = c % kStatePsiBufs;
       if (!mbar_wait_w(kv_full + st, (c / kStateStages) & 1, env)) {
         ok = false;
         break;
       }
       if (tid == 0) KATA_TRACE(chunkstate, c, 2);
-      if (c >= 2 && !mbar_wait_w(psi_empty + pb, ((c >> 1) - 1) & 1, env)) {
+      if (c >= kStatePsiBufs && !mbar_wait_w(psi_empty + pb, ((c / kStatePsiBufs) - 1) & 1, env)) {
         ok = false;
         break;
       }

@@ -42,3 +42,25 @@ def test_report_line_has_the_contract_keys():
     assert "tensor_frac" in line["mg"]["mg2_ctx2k"] and "hbm_frac" in line["mg"]["decode_mg4_b64"]
     tr = line["train"]
     assert tr["tokens_per_s"] == 8 * 2048 / 0.43e-3 and 0 < tr["bwd_tensor_frac"] < 1
+
+
+def test_report_line_has_per_path_points():
+    """Every path of the metric is reported on its own inside `roofline`:
+    tokens/s and the fraction of its binding roofline at T = 2048 and at
+    T = 131072 (chunked C = 64 and 128, quadratic), and the B = 64 decode."""
+    args = argparse.Namespace(workload="layer340m_ctx2k", steps=1000, warmup=10, cpu_baseline=0)
+    res = _fake_result()
+    res["clocks_by_part"] = {"step": {"sm_mhz": 1965.0}, "long_ctx": {"sm_mhz": 1950.0}, "decode_b64": {}}
+    buf = io.StringIO()
+    with redirect_stdout(buf):
+        bench.report(args, res, 0.116, 11.0, 1)
+    pts = json.loads(buf.getvalue().strip().splitlines()[-1])["roofline"]["points"]
+    key = {(p["path"], p.get("T"), p.get("C")): p for p in pts}
+    c131 = key[("chunked", 131072, 64)]
+    assert c131["bound"] == "hbm" and c131["clocks"] == {"sm_mhz": 1950.0}
+    assert abs(c131["achieved"] - bench.chunked_bytes(16, 131072, 16, 64) / 0.235e-3 / 1e9) < 1e-6
+    assert abs(c131["frac"] - c131["achieved"] / c131["peak"]) < 1e-12
+    assert c131["tokens_per_s"] == 131072 / 0.235e-3
+    assert ("chunked", 131072, 128) in key and ("quadratic", 131072, None) in key
+    assert key[("quadratic", 2048, None)]["bound"] == "tensor" and ("chunked", 2048, 64) in key
+    assert any(p["path"] == "decode" for p in pts)
