@@ -82,10 +82,12 @@ kata_status_t kata_fwd_quadratic(const void* q, const void* k, const void* v, vo
 
 /*
  * Bytes of device workspace kata_fwd_chunked needs for these sizes: 0 when
- * T == 0, and on the tensor-core path (bf16, p = 16, dv = 64) whenever each
- * (b,h) sequence is handled as a single super-chunk; otherwise one fp32
- * state record per (b,h) per super-chunk.  A pure function of the arguments;
- * the same arguments must be passed to kata_fwd_chunked.
+ * T == 0, and on the tensor-core path (bf16, dv = 64, p = 16 or 32) whenever
+ * each (b,h) sequence is handled as a single super-chunk; otherwise one fp32
+ * state record per (b,h) per super-chunk (four for p = 32 on the tensor
+ * cores).  A pure function of the arguments; the same arguments must be
+ * passed to kata_fwd_chunked.  The dtype is an argument because it selects
+ * the path and with it the record layout.
  */
 size_t kata_fwd_chunked_workspace_size(int B, int H, int T, int p, int dv, int C,
                                        kata_dtype_t dtype);
@@ -94,13 +96,22 @@ size_t kata_fwd_chunked_workspace_size(int B, int H, int T, int p, int dv, int C
  * Exact O(T) chunked-state operating point (gist.science sec. 2.3, "Chunked
  * Parallelism" and the second operating point; ai.info Main Findings,
  * "Chunk recurrence avoids the triangular solve"):
- *   1. per-chunk states psi(K_c)^T [V_c | 1] built as tensor-core
- *      contractions and summed over groups of consecutive chunks,
- *   2. an exclusive associative (parallel prefix) scan of those sums along
- *      the sequence, depth O(log(T/C)) (gist.science sec. 2.3,
- *      "Complexiteitsreductie"),
+ *   1. per-chunk states psi(K_c)^T [V_c | 1], summed over super-chunks of
+ *      Ls consecutive tokens,
+ *   2. an exclusive associative (parallel prefix) scan of those sums over
+ *      the G = ceil(T / Ls) super-chunks of each sequence, depth O(log G)
+ *      (gist.science sec. 2.3, "Complexiteitsreductie"),
  *   3. per chunk: intra-chunk squared-score attention plus the readout
- *      psi(Q_c) . S_prefix, then o = numerator / denominator.
+ *      psi(Q_c) . S_prefix, then o = numerator / denominator; inside a
+ *      super-chunk one CTA (p = 32: one cluster of four) carries the state
+ *      from chunk to chunk, Ls/128 steps in sequence.
+ * Ls is chosen by the plan (a pure function of the sizes) to fill the GPU:
+ * for example Ls = 2048 (G = 1) at B = 8, H = 16, T = 2048 and Ls = 14592
+ * (G = 9, 114 steps per CTA) at B = 1, H = 16, T = 131072, both p = 16.
+ * Steps 1 and 3 run on the tensor cores (tcgen05) for bf16 inputs with
+ * dv = 64 and p = 16 or 32 (p = 32 splits the packed state over four CTAs);
+ * fp32 inputs, and bf16 with dv = 16, run the same three steps on the CUDA
+ * cores in exact fp32 arithmetic.
  * The result equals kata_fwd_quadratic's up to rounding; C is the chunk
  * length and changes rounding only.
  *

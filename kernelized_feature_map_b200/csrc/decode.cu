@@ -6,10 +6,10 @@
 // state recurrence of the ai.info summary, Methodology in Plain English.)
 //
 // The step is bound by HBM: every (b,h) streams its p^2 x dv fp32 state in
-// and out once (2 * 64 KiB at p = 16, dv = 64).  One CTA of 256 threads per
-// (b,h).  Thread layout: DV/4 consecutive threads cover one state row with
-// 16-byte vectors, so each pass of the CTA reads 256 x 16 B contiguous
-// bytes; all of a batch's loads are issued before any use so that enough
+// and out once (2 * 64 KiB at p = 16, dv = 64).  One CTA per (b,h) (128 or
+// 256 threads, see DecodeCfg).  Thread layout: DV/4 consecutive threads
+// cover one state row with 16-byte vectors, so each pass of the CTA reads
+// one 16-byte vector per thread, contiguous across the CTA; all of a batch's loads are issued before any use so that enough
 // bytes are in flight per SM.  The first batch of state rows and the
 // normaliser entries are requested before q, k and v are staged, since they
 // do not depend on them, so their latency overlaps.  Loads and stores carry
@@ -26,23 +26,46 @@
 
 namespace kata {
 
+// Threads per CTA, batch of state loads per thread, and CTAs per SM.  A
+// small state (64 KiB per stream for the p = 16 single factor) runs on
+// 128-thread CTAs in batches of 8 loads per thread, seven CTAs per SM: the
+// 1024 streams of a B = 64, H = 16 step are then resident in one wave, each
+// SM keeping ~110 KiB of loads in flight, instead of three and a half waves
+// of two 256-thread CTAs with a tail.  Larger states (p = 32, KATA-Mg)
+// stream long enough per CTA with 256 threads and 16-deep batches.
+// Measured at B = 64, H = 16 (p = 16, dv = 64): 33 us with 256-thread CTAs
+// and 16-deep batches, 28.8 us in this configuration; double-buffering the
+// batches (next batch's loads issued before the current one is stored)
+// measured 29.7 us and is not used.
+template <int P, int DV>
+struct DecodeCfg {
+  static constexpr bool kSmall = P * DV <= 256 * 64;
+  static constexpr int kThreads = kSmall ? 128 : 256;
+  static constexpr int kBatchMax = kSmall ? 8 : 16;
+  static constexpr bool kPipe = false;
+  static constexpr int kMinBlocks = kSmall ? 7 : 1;
+};
+
 template <typename Tin, int p, int DV, int G>
-__global__ void __launch_bounds__(256) decode_step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
-                                                          const Tin* __restrict__ v, Tin* __restrict__ o,
-                                                          float* __restrict__ S, float* __restrict__ z) {
+__global__ void __launch_bounds__((DecodeCfg<G * p * p, DV>::kThreads), (DecodeCfg<G * p * p, DV>::kMinBlocks))
+    decode_step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
+                       Tin* __restrict__ o, float* __restrict__ S, float* __restrict__ z) {
   constexpr int D = G * p;          // q/k row width
   constexpr int P = G * p * p;      // state rows
+  constexpr int NT = DecodeCfg<P, DV>::kThreads;
   constexpr int CG = DV / 4;        // 16-byte column groups per state row
-  constexpr int RPP = 256 / CG;     // rows covered by one pass of the CTA
+  constexpr int RPP = NT / CG;      // rows covered by one pass of the CTA
   constexpr int PASSES = P / RPP;   // passes over the state
-  constexpr int BATCH = PASSES < 16 ? PASSES : 16;
+  constexpr int BMAX = DecodeCfg<P, DV>::kBatchMax;
+  constexpr int BATCH = PASSES < BMAX ? PASSES : BMAX;
   static_assert(PASSES % BATCH == 0, "pass batching");
+  static_assert(D <= NT && DV <= NT, "q, k and v are staged by one thread per value");
 
   __shared__ float sq[D], sk[D], sv[DV];
-  __shared__ float4 red[256];
-  __shared__ float sden[8];
+  __shared__ float4 red[NT];
+  __shared__ float sden[NT / 32];
 
-  constexpr int ZPT = (P + 255) / 256;  // normaliser entries per thread
+  constexpr int ZPT = (P + NT - 1) / NT;  // normaliser entries per thread
   const int tid = threadIdx.x;
   const long long bh = blockIdx.x;
   const int cg = tid % CG;
@@ -54,7 +77,7 @@ __global__ void __launch_bounds__(256) decode_step_kernel(const Tin* __restrict_
   for (int i = 0; i < BATCH; ++i) s[i] = __ldcs(Sb + (r0 + i * RPP) * CG + cg);
   float zz[ZPT];
 #pragma unroll
-  for (int u = 0; u < ZPT; ++u) zz[u] = (tid + 256 * u < P) ? __ldcs(zb + tid + 256 * u) : 0.f;
+  for (int u = 0; u < ZPT; ++u) zz[u] = (tid + NT * u < P) ? __ldcs(zb + tid + NT * u) : 0.f;
   if (tid < D) {
     sq[tid] = Elem<Tin>::load(q + bh * D + tid);
     sk[tid] = Elem<Tin>::load(k + bh * D + tid);
@@ -67,7 +90,13 @@ __global__ void __launch_bounds__(256) decode_step_kernel(const Tin* __restrict_
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 1
   for (int b0 = 0; b0 < PASSES; b0 += BATCH) {
-    if (b0 > 0) {
+    float4 nx[DecodeCfg<P, DV>::kPipe ? BATCH : 1];
+    if constexpr (DecodeCfg<P, DV>::kPipe) {
+      if (b0 + BATCH < PASSES) {
+#pragma unroll
+        for (int i = 0; i < BATCH; ++i) nx[i] = __ldcs(Sb + (r0 + (b0 + BATCH + i) * RPP) * CG + cg);
+      }
+    } else if (b0 > 0) {
 #pragma unroll
       for (int i = 0; i < BATCH; ++i) s[i] = __ldcs(Sb + (r0 + (b0 + i) * RPP) * CG + cg);
     }
@@ -87,13 +116,17 @@ __global__ void __launch_bounds__(256) decode_step_kernel(const Tin* __restrict_
       acc.z = fmaf(pq, s[i].z, acc.z);
       acc.w = fmaf(pq, s[i].w, acc.w);
     }
+    if constexpr (DecodeCfg<P, DV>::kPipe) {
+#pragma unroll
+      for (int i = 0; i < BATCH; ++i) s[i] = nx[i];
+    }
   }
 
   // normaliser z and the denominator psi(q)^T z
   float den = 0.f;
 #pragma unroll
   for (int u = 0; u < ZPT; ++u) {
-    const int r = tid + 256 * u;
+    const int r = tid + NT * u;
     if (r < P) {
       const int gp = (r / (p * p)) * p, ii = gp + (r % (p * p)) / p, jj = gp + r % p;
       const float zn = zz[u] + sk[ii] * sk[jj];
@@ -110,7 +143,7 @@ __global__ void __launch_bounds__(256) decode_step_kernel(const Tin* __restrict_
   if (tid < DV) {
     float D = 0.f;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) D += sden[w];
+    for (int w = 0; w < NT / 32; ++w) D += sden[w];
     const int c4 = tid / 4, comp = tid % 4;
     float num = 0.f;
 #pragma unroll 4
@@ -125,7 +158,8 @@ __global__ void __launch_bounds__(256) decode_step_kernel(const Tin* __restrict_
 template <typename Tin, int p, int DV, int G>
 static cudaError_t launch_decode_t(const void* q, const void* k, const void* v, void* o, float* S, float* z,
                                    int BH, cudaStream_t st) {
-  decode_step_kernel<Tin, p, DV, G><<<BH, 256, 0, st>>>((const Tin*)q, (const Tin*)k, (const Tin*)v, (Tin*)o, S, z);
+  decode_step_kernel<Tin, p, DV, G><<<BH, DecodeCfg<G * p * p, DV>::kThreads, 0, st>>>(
+      (const Tin*)q, (const Tin*)k, (const Tin*)v, (Tin*)o, S, z);
   return cudaGetLastError();
 }
 

@@ -99,10 +99,14 @@ ChunkPlan make_chunk_plan(int B, int H, int T, int p, int dv, int C, kata_dtype_
   const long long tiles = (T + 127) / 128;
   long long best = -1;
   const long long kmax = tiles < 1 ? 1 : (tiles < 512 ? tiles : 512);  // super-chunks up to 64K tokens
+  // p = 32 on the tensor cores: a unit is a cluster of four CTAs (one per
+  // coordinate block), and clusters fill whole groups of four SMs
+  const int cta_per_unit = pl.layout == kRecPackedT ? chunk_blocks(p) : 1;
+  const long long slots = cta_per_unit > 1 ? (kSMs / 4) * 4 : kSMs;
   for (long long k = kmax; k >= 1; --k) {
     const long long per_bh = (tiles + k - 1) / k;
-    const long long units = (long long)pl.BH * per_bh;
-    const long long waves = (units + kSMs - 1) / kSMs;
+    const long long units = (long long)pl.BH * per_bh * cta_per_unit;
+    const long long waves = (units + slots - 1) / slots;
     const long long split = (pl.layout == kRecPackedT && per_bh > 1) ? kSplitOverhead : 0;
     const long long cost = waves * (k + kUnitOverhead) + split;
     if (best < 0 || cost < best) {
@@ -115,7 +119,7 @@ ChunkPlan make_chunk_plan(int B, int H, int T, int p, int dv, int C, kata_dtype_
   pl.record_floats = pl.layout == kRecPackedT ? (size_t)(dv + 1) * 144 : (size_t)pl.P * pl.ld;
   // the tensor-core path needs no records for a single super-chunk
   const bool no_records = pl.layout == kRecPackedT && pl.G <= 1;
-  pl.workspace_bytes = no_records ? 0 : (size_t)pl.BH * pl.G * pl.record_floats * sizeof(float);
+  pl.workspace_bytes = no_records ? 0 : (size_t)pl.BH * cta_per_unit * pl.G * pl.record_floats * sizeof(float);
   return pl;
 }
 
@@ -231,6 +235,21 @@ KATA_API kata_status_t kata_fwd_chunked(const void* q, const void* k, const void
   }
   float* ws = plan.workspace_bytes > 0 ? static_cast<float*>(workspace) : nullptr;
   const WaitCtl wc = wait_ctl();
+  if (plan.layout == kRecPackedT && p == 32) {
+    // bf16 with p = 32, dv = 64 on the tensor cores, the state in four
+    // coordinate blocks: the block sums of super-chunks 0..G-2 and their scan
+    // (4 B H sequences of records, no initial state) exist only when G > 1;
+    // the readout adds S0 to every prefix and writes the final state itself
+    cudaError_t e = cudaSuccess;
+    if (plan.G > 1) {
+      e = launch_chunk_state_p32(k, v, ws, plan, wc, st);
+      ChunkPlan blocks = plan;
+      blocks.BH = plan.BH * chunk_blocks(p);
+      if (e == cudaSuccess) e = launch_state_scan(ws, blocks, plan.G - 1, nullptr, nullptr, nullptr, nullptr, st);
+    }
+    if (e == cudaSuccess) e = launch_chunk_readout_p32(q, k, v, o, ws, S0, z0, S_out, z_out, plan, wc, st);
+    return from_cuda(e);
+  }
   if (plan.layout == kRecPackedT) {
     // bf16 with p = 16, dv = 64 on the tensor cores: the sums of super-chunks
     // 0..G-2 and their scan exist only when G > 1; the readout takes the
@@ -259,7 +278,7 @@ KATA_API kata_status_t kata_fwd_chunked_sequential(const void* q, const void* k,
   kata_status_t s = check_common(B, H, T, p, dv, dtype);
   if (s != KATA_OK) return s;
   if (!(C == 64 || C == 128)) return KATA_ERR_UNSUPPORTED;
-  if (!chunked_on_tensor_cores(p, dv, dtype)) return KATA_ERR_UNSUPPORTED;
+  if (!chunked_on_tensor_cores(p, dv, dtype) || p != 16) return KATA_ERR_UNSUPPORTED;
   if ((S0 == nullptr) != (z0 == nullptr)) return KATA_ERR_INVALID_ARG;
   if ((S_out == nullptr) != (z_out == nullptr)) return KATA_ERR_INVALID_ARG;
   for (const void* ptr : {(const void*)S0, (const void*)z0, (const void*)S_out, (const void*)z_out})

@@ -21,7 +21,7 @@ struct WaitCtl {
 // Layout of a workspace state record (one per (b,h) per super-chunk).
 enum RecordLayout {
   kRecUnpacked = 0,  // P rows x ld floats: [sum psi(k) v^T | sum psi(k) | pad]
-  kRecPackedT = 1,   // 65 rows x 144 floats: transposed, packed psi (p=16, dv=64)
+  kRecPackedT = 1,   // 65 rows x 144 floats: transposed, packed psi (p=16, dv=64; per block for p=32)
 };
 
 // Chunked-path plan: how the sequence is grouped for the state scan.
@@ -39,10 +39,16 @@ struct ChunkPlan {
   size_t workspace_bytes;
 };
 
-// True when the tensor-core chunked kernels serve these sizes (bf16, p = 16, dv = 64).
+// True when the tensor-core chunked kernels serve these sizes (bf16, dv = 64,
+// p = 16 in chunk_sm100.cu or p = 32 in chunk_p32_sm100.cu).
 inline bool chunked_on_tensor_cores(int p, int dv, kata_dtype_t dt) {
-  return dt == KATA_BF16 && p == 16 && dv == 64;
+  return dt == KATA_BF16 && (p == 16 || p == 32) && dv == 64;
 }
+
+// Coordinate blocks per (b,h) of the tensor-core chunked state: p = 32 splits
+// its packed feature over four blocks of the p = 16 size (one CTA of a
+// cluster each); p = 16 has one.
+inline int chunk_blocks(int p) { return p == 32 ? 4 : 1; }
 
 ChunkPlan make_chunk_plan(int B, int H, int T, int p, int dv, int C, kata_dtype_t dt);
 
@@ -109,6 +115,16 @@ cudaError_t launch_chunk_state_sm100(const void* k, const void* v, float* ws, co
 cudaError_t launch_chunk_readout_sm100(const void* q, const void* k, const void* v, void* o, const float* ws,
                                        const float* S0, const float* z0, float* S_out, float* z_out,
                                        const ChunkPlan& pl, const WaitCtl& wc, cudaStream_t st);
+
+// chunk_p32_sm100.cu -- the same for p = 32, the state split over four
+// coordinate blocks (records ((bh * 4 + block) * G + g)).  The readout adds
+// S0/z0 (when non-null) to the scanned prefix of every super-chunk itself,
+// so the scan runs without an initial state.
+cudaError_t launch_chunk_state_p32(const void* k, const void* v, float* ws, const ChunkPlan& pl, const WaitCtl& wc,
+                                   cudaStream_t st);
+cudaError_t launch_chunk_readout_p32(const void* q, const void* k, const void* v, void* o, const float* ws,
+                                     const float* S0, const float* z0, float* S_out, float* z_out,
+                                     const ChunkPlan& pl, const WaitCtl& wc, cudaStream_t st);
 
 // Current bound on in-kernel waits and the status word (kata_api.cu).
 WaitCtl wait_ctl();

@@ -130,11 +130,13 @@ def test_empty_sequence_is_a_noop(kata):
 # workspace: the readout starts from S0 and writes the final state); with 2
 # pairs and T = 20000 each spans many, with the state build, the scan and
 # the prefix records in between.
+# p = 32 in bf16 runs the four-block cluster kernels (the state split over
+# four coordinate blocks, one CTA each), with the same two regimes.
 @pytest.mark.parametrize("B,H,T,t0", [(8, 16, 700, 300), (1, 2, 20000, 7000)])
-@pytest.mark.parametrize("dtype", ["f32", "bf16"])
-def test_chunked_state_in_and_out(kata, dtype, B, H, T, t0):
+@pytest.mark.parametrize("dtype,p", [("f32", 16), ("bf16", 16), ("bf16", 32)])
+def test_chunked_state_in_and_out(kata, dtype, p, B, H, T, t0):
     import torch
-    p, dv = 16, 64
+    dv = 64
     q, k, v = workloads.normal_qkv(B, H, T, p, dv, seed=7, dtype=dtype)
     o_ref, S_ref, z_ref = oracle.recurrent(q, k, v, return_state=True)
     _, S1, z1 = oracle.recurrent(q[:, :, :t0], k[:, :, :t0], v[:, :, :t0], return_state=True)
