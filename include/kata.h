@@ -267,6 +267,33 @@ kata_status_t kata_fwd_mg_quadratic(const void* q, const void* k, const void* v,
                                     kata_layout_t layout, kata_dtype_t dtype, void* stream);
 
 /*
+ * Exact O(T) chunked-state KATA-Mg forward (the chunked operating point of
+ * kata_fwd_chunked with the concatenated feature psi_Mg): the same
+ * arguments as kata_fwd_mg_quadratic plus the chunk length C (64 or 128,
+ * rounding only), an optional initial and final state, and a workspace.
+ * The state is the concatenation of the groups' states:
+ * S [B,H,groups*p*p,dv] and z [B,H,groups*p*p] fp32, row
+ * r = j*p*p + a*p + b holding the products of coordinates j*p + a and
+ * j*p + b (group j), as for kata_decode_step_mg; S0/z0 and S_out/z_out are
+ * both-or-neither, as for kata_fwd_chunked.
+ *
+ * bf16, dv = 64.  (d, groups) = (64, 4) and (64, 2) run the cluster kernels:
+ * each group's packed state in its own CTAs (one for a group of 16, four
+ * for a group of 32) with each group's intra-chunk squared scores in the
+ * first of them, in either layout.  groups = 1 is kata_fwd_chunked (p = d;
+ * [B,T,H,*] only for p = 32).  Other shapes or fp32: KATA_ERR_UNSUPPORTED.
+ * workspace: at least kata_fwd_mg_chunked_workspace_size() bytes, 256-byte
+ * aligned (NULL when that size is 0).
+ */
+size_t kata_fwd_mg_chunked_workspace_size(int B, int H, int T, int d, int groups, int dv, int C,
+                                          kata_dtype_t dtype);
+kata_status_t kata_fwd_mg_chunked(const void* q, const void* k, const void* v, void* o,
+                                  int B, int H, int T, int d, int groups, int dv, int C,
+                                  kata_layout_t layout, kata_dtype_t dtype,
+                                  const float* S0, const float* z0, float* S_out, float* z_out,
+                                  void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Quadratic (flash-style) KATA-Sigma-g forward: summed PSD factors
  * (gist.science sec. 2.3 "Varianten"; ai.info Main Findings: state
  * (d/g)(d/g+1)/2 * dv).  The feature is the sum of the groups' rank-one maps,

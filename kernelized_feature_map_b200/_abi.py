@@ -38,6 +38,8 @@ SIGNATURES = {
     "kata_fwd_mg_quadratic": (_c_int, [_vp, _vp, _vp, _vp] + [_c_int] * 8 + [_vp]),
     "kata_fwd_mg_quadratic_train": (_c_int, [_vp, _vp, _vp, _vp, _fp] + [_c_int] * 7 + [_vp]),
     "kata_fwd_sg_quadratic": (_c_int, [_vp, _vp, _vp, _vp] + [_c_int] * 8 + [_vp]),
+    "kata_fwd_mg_chunked_workspace_size": (_c_size, [_c_int] * 8),
+    "kata_fwd_mg_chunked": (_c_int, [_vp, _vp, _vp, _vp] + [_c_int] * 9 + [_fp, _fp, _fp, _fp, _vp, _c_size, _vp]),
     "kata_bwd_mg_quadratic": (_c_int, [_vp] * 9 + [_c_int] * 7 + [_vp, _c_size, _vp]),
     "kata_decode_step_mg": (_c_int, [_vp, _vp, _vp, _vp, _fp, _fp] + [_c_int] * 6 + [_vp]),
     "kata_get_status": (_c_int, [_vp]),
@@ -368,6 +370,51 @@ def kata_fwd_mg_quadratic(q, k, v, groups, layout="bhtd", o=None, stream=None):
     _check("kata_fwd_mg_quadratic", lib().kata_fwd_mg_quadratic(
         _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), B, H, T, d, int(groups), dv, code,
         _dtype_code(q), _stream_ptr(stream)))
+    return o
+
+
+def kata_fwd_mg_chunked_workspace_size(B, H, T, d, groups, dv, C, dtype=torch.bfloat16) -> int:
+    code = KATA_BF16 if dtype == torch.bfloat16 else KATA_F32
+    return int(lib().kata_fwd_mg_chunked_workspace_size(B, H, T, d, int(groups), dv, C, code))
+
+
+def kata_fwd_mg_chunked(q, k, v, groups, C=64, layout="bhtd", S0=None, z0=None, return_state=False, o=None,
+                        workspace=None, S_out=None, z_out=None, stream=None):
+    """Exact O(T) chunked-state KATA-Mg forward with `groups` PSD factors per head.
+
+    Layouts as kata_fwd_mg_quadratic.  Returns o, or (o, S_T, z_T) when
+    return_state is True; the state is [B,H,groups*p*p,dv] and
+    [B,H,groups*p*p] fp32 (p = d / groups), S0/z0 an initial state of the
+    same shapes.  ``workspace`` may be a preallocated uint8 CUDA tensor of at
+    least the queried size.
+    """
+    if layout == "bhtd":
+        B, H, T, d = q.shape
+        code = KATA_LAYOUT_BHTD
+    elif layout == "bthd":
+        B, T, H, d = q.shape
+        code = KATA_LAYOUT_BTHD
+    else:
+        raise ValueError("layout must be 'bhtd' or 'bthd'")
+    dv = v.shape[-1]
+    g = int(groups)
+    p = d // g
+    dev = q.device
+    if o is None:
+        o = torch.empty(v.shape, dtype=q.dtype, device=dev)
+    if return_state and S_out is None:
+        S_out = torch.empty((B, H, g * p * p, dv), dtype=torch.float32, device=dev)
+        z_out = torch.empty((B, H, g * p * p), dtype=torch.float32, device=dev)
+    need = kata_fwd_mg_chunked_workspace_size(B, H, T, d, g, dv, C, q.dtype)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("kata_fwd_mg_chunked", lib().kata_fwd_mg_chunked(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), B, H, T, d, g, dv, C, code, _dtype_code(q),
+        _opt(S0, "S0"), _opt(z0, "z0"), _opt(S_out, "S_out"), _opt(z_out, "z_out"),
+        _opt(workspace, "workspace"), ws_bytes, _stream_ptr(stream)))
+    if return_state:
+        return o, S_out, z_out
     return o
 
 

@@ -85,7 +85,9 @@ constexpr int kSMs = 148;
 constexpr int kUnitOverhead = 2;
 constexpr int kSplitOverhead = 8;
 
-ChunkPlan make_chunk_plan(int B, int H, int T, int p, int dv, int C, kata_dtype_t dt) {
+// Shared by both plans: tensor-core layout when `tc`, `cta_per_unit` CTAs
+// per (b,h, super-chunk) unit (a cluster fills whole groups of four SMs).
+static ChunkPlan plan_units(int B, int H, int T, int p, int dv, int C, bool tc, int cta_per_unit) {
   ChunkPlan pl{};
   pl.BH = B * H;
   pl.T = T;
@@ -95,19 +97,16 @@ ChunkPlan make_chunk_plan(int B, int H, int T, int p, int dv, int C, kata_dtype_
   pl.ld = dv + 4;
   pl.C = C;
   pl.Ls = 128;
-  pl.layout = chunked_on_tensor_cores(p, dv, dt) ? kRecPackedT : kRecUnpacked;
+  pl.layout = tc ? kRecPackedT : kRecUnpacked;
   const long long tiles = (T + 127) / 128;
   long long best = -1;
   const long long kmax = tiles < 1 ? 1 : (tiles < 512 ? tiles : 512);  // super-chunks up to 64K tokens
-  // p = 32 on the tensor cores: a unit is a cluster of four CTAs (one per
-  // coordinate block), and clusters fill whole groups of four SMs
-  const int cta_per_unit = pl.layout == kRecPackedT ? chunk_blocks(p) : 1;
   const long long slots = cta_per_unit > 1 ? (kSMs / 4) * 4 : kSMs;
   for (long long k = kmax; k >= 1; --k) {
     const long long per_bh = (tiles + k - 1) / k;
     const long long units = (long long)pl.BH * per_bh * cta_per_unit;
     const long long waves = (units + slots - 1) / slots;
-    const long long split = (pl.layout == kRecPackedT && per_bh > 1) ? kSplitOverhead : 0;
+    const long long split = (tc && per_bh > 1) ? kSplitOverhead : 0;
     const long long cost = waves * (k + kUnitOverhead) + split;
     if (best < 0 || cost < best) {
       best = cost;
@@ -116,11 +115,20 @@ ChunkPlan make_chunk_plan(int B, int H, int T, int p, int dv, int C, kata_dtype_
   }
   if (pl.Ls < C) pl.Ls = C;
   pl.G = T > 0 ? (T + pl.Ls - 1) / pl.Ls : 0;
-  pl.record_floats = pl.layout == kRecPackedT ? (size_t)(dv + 1) * 144 : (size_t)pl.P * pl.ld;
+  pl.record_floats = tc ? (size_t)(dv + 1) * 144 : (size_t)pl.P * pl.ld;
   // the tensor-core path needs no records for a single super-chunk
-  const bool no_records = pl.layout == kRecPackedT && pl.G <= 1;
+  const bool no_records = tc && pl.G <= 1;
   pl.workspace_bytes = no_records ? 0 : (size_t)pl.BH * cta_per_unit * pl.G * pl.record_floats * sizeof(float);
   return pl;
+}
+
+ChunkPlan make_chunk_plan(int B, int H, int T, int p, int dv, int C, kata_dtype_t dt) {
+  const bool tc = chunked_on_tensor_cores(p, dv, dt);
+  return plan_units(B, H, T, p, dv, C, tc, tc ? cluster_blocks(p, 1) : 1);
+}
+
+ChunkPlan make_cluster_plan(int B, int H, int T, int p, int blocks, int dv, int C) {
+  return plan_units(B, H, T, p, dv, C, true, blocks);
 }
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -190,6 +198,25 @@ KATA_API size_t kata_fwd_chunked_workspace_size(int B, int H, int T, int p, int 
 }
 
 namespace kata {
+// The chunked path of the cluster kernels (p = 32, KATA-Mg): the block sums
+// of super-chunks 0..G-2 and their scan (B H x blocks sequences of records,
+// no initial state) exist only when G > 1; the readout adds S0 to every
+// prefix and writes the final state itself.
+static cudaError_t run_cluster_chunked(const void* q, const void* k, const void* v, void* o, const ChunkPlan& plan,
+                                       int H, int groups, bool bthd, const float* S0, const float* z0, float* S_out,
+                                       float* z_out, float* ws, const WaitCtl& wc, cudaStream_t st) {
+  cudaError_t e = cudaSuccess;
+  if (plan.G > 1) {
+    e = launch_chunk_state_cluster(k, v, ws, plan, H, groups, bthd, wc, st);
+    ChunkPlan blocks = plan;
+    blocks.BH = plan.BH * cluster_blocks(plan.p, groups);
+    if (e == cudaSuccess) e = launch_state_scan(ws, blocks, plan.G - 1, nullptr, nullptr, nullptr, nullptr, st);
+  }
+  if (e == cudaSuccess)
+    e = launch_chunk_readout_cluster(q, k, v, o, ws, S0, z0, S_out, z_out, plan, H, groups, bthd, wc, st);
+  return e;
+}
+
 // Every argument check of kata_fwd_chunked except the workspace's, in the
 // order that call makes them.
 kata_status_t check_chunked_args(const void* q, const void* k, const void* v, const void* o, int B, int H, int T,
@@ -235,21 +262,8 @@ KATA_API kata_status_t kata_fwd_chunked(const void* q, const void* k, const void
   }
   float* ws = plan.workspace_bytes > 0 ? static_cast<float*>(workspace) : nullptr;
   const WaitCtl wc = wait_ctl();
-  if (plan.layout == kRecPackedT && p == 32) {
-    // bf16 with p = 32, dv = 64 on the tensor cores, the state in four
-    // coordinate blocks: the block sums of super-chunks 0..G-2 and their scan
-    // (4 B H sequences of records, no initial state) exist only when G > 1;
-    // the readout adds S0 to every prefix and writes the final state itself
-    cudaError_t e = cudaSuccess;
-    if (plan.G > 1) {
-      e = launch_chunk_state_p32(k, v, ws, plan, wc, st);
-      ChunkPlan blocks = plan;
-      blocks.BH = plan.BH * chunk_blocks(p);
-      if (e == cudaSuccess) e = launch_state_scan(ws, blocks, plan.G - 1, nullptr, nullptr, nullptr, nullptr, st);
-    }
-    if (e == cudaSuccess) e = launch_chunk_readout_p32(q, k, v, o, ws, S0, z0, S_out, z_out, plan, wc, st);
-    return from_cuda(e);
-  }
+  if (plan.layout == kRecPackedT && p == 32)
+    return from_cuda(run_cluster_chunked(q, k, v, o, plan, H, 1, false, S0, z0, S_out, z_out, ws, wc, st));
   if (plan.layout == kRecPackedT) {
     // bf16 with p = 16, dv = 64 on the tensor cores: the sums of super-chunks
     // 0..G-2 and their scan exist only when G > 1; the readout takes the
@@ -375,6 +389,65 @@ KATA_API kata_status_t kata_fwd_mg_quadratic(const void* q, const void* k, const
   if (flash_mg_sm100_supports(p, groups, dv))
     return from_cuda(launch_flash_mg_sm100(q, k, v, o, nullptr, B, H, T, p, groups, bthd, wait_ctl(), st));
   return from_cuda(launch_flash_sm100(q, k, v, o, B, H, T, p, dv, bthd, nullptr, wait_ctl(), st));
+}
+
+// (d, groups) of the chunked KATA-Mg path on the cluster kernels, after the
+// shape checks of check_mg.
+static bool mg_chunked_on_clusters(int p, int groups, int dv, kata_dtype_t dt) {
+  return dt == KATA_BF16 && groups > 1 && cluster_chunked_supports(p, groups, dv);
+}
+
+KATA_API size_t kata_fwd_mg_chunked_workspace_size(int B, int H, int T, int d, int groups, int dv, int C,
+                                                   kata_dtype_t dtype) {
+  int p = 0;
+  if (check_mg(B, H, T, d, groups, dv, dtype, &p) != KATA_OK || !(C == 64 || C == 128) || T == 0) return 0;
+  if (groups == 1) return kata_fwd_chunked_workspace_size(B, H, T, p, dv, C, dtype);
+  if (!mg_chunked_on_clusters(p, groups, dv, dtype)) return 0;
+  return make_cluster_plan(B, H, T, p, cluster_blocks(p, groups), dv, C).workspace_bytes;
+}
+
+KATA_API kata_status_t kata_fwd_mg_chunked(const void* q, const void* k, const void* v, void* o, int B, int H, int T,
+                                           int d, int groups, int dv, int C, kata_layout_t layout,
+                                           kata_dtype_t dtype, const float* S0, const float* z0, float* S_out,
+                                           float* z_out, void* workspace, size_t workspace_bytes, void* stream) {
+  int p = 0;
+  kata_status_t s = check_mg(B, H, T, d, groups, dv, dtype, &p);
+  if (s != KATA_OK) return s;
+  if (layout != KATA_LAYOUT_BHTD && layout != KATA_LAYOUT_BTHD) return KATA_ERR_INVALID_ARG;
+  if (!(C == 64 || C == 128)) return KATA_ERR_UNSUPPORTED;
+  const bool bthd = layout == KATA_LAYOUT_BTHD;
+  if (groups == 1 && !bthd)
+    return kata_fwd_chunked(q, k, v, o, B, H, T, p, dv, C, dtype, S0, z0, S_out, z_out, workspace, workspace_bytes,
+                            stream);
+  const bool single32 = groups == 1 && p == 32 && dtype == KATA_BF16 && dv == 64;
+  if (!single32 && !mg_chunked_on_clusters(p, groups, dv, dtype)) return KATA_ERR_UNSUPPORTED;
+  if ((S0 == nullptr) != (z0 == nullptr)) return KATA_ERR_INVALID_ARG;
+  if ((S_out == nullptr) != (z_out == nullptr)) return KATA_ERR_INVALID_ARG;
+  for (const void* ptr : {(const void*)S0, (const void*)z0, (const void*)S_out, (const void*)z_out})
+    if (ptr && !aligned16(ptr)) return KATA_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t P = (size_t)groups * p * p, BH = (size_t)B * H;
+  if (T == 0) {
+    if (!S_out) return KATA_OK;
+    cudaError_t e;
+    if (S0) {
+      e = cudaMemcpyAsync(S_out, S0, BH * P * dv * sizeof(float), cudaMemcpyDeviceToDevice, st);
+      if (e == cudaSuccess) e = cudaMemcpyAsync(z_out, z0, BH * P * sizeof(float), cudaMemcpyDeviceToDevice, st);
+    } else {
+      e = cudaMemsetAsync(S_out, 0, BH * P * dv * sizeof(float), st);
+      if (e == cudaSuccess) e = cudaMemsetAsync(z_out, 0, BH * P * sizeof(float), st);
+    }
+    return from_cuda(e);
+  }
+  if (!q || !k || !v || !o) return KATA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return KATA_ERR_MISALIGNED;
+  const ChunkPlan plan = make_cluster_plan(B, H, T, p, cluster_blocks(p, groups), dv, C);
+  if (plan.workspace_bytes > 0) {
+    if (!workspace || workspace_bytes < plan.workspace_bytes) return KATA_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KATA_ERR_MISALIGNED;
+  }
+  float* ws = plan.workspace_bytes > 0 ? static_cast<float*>(workspace) : nullptr;
+  return from_cuda(run_cluster_chunked(q, k, v, o, plan, H, groups, bthd, S0, z0, S_out, z_out, ws, wait_ctl(), st));
 }
 
 KATA_API kata_status_t kata_fwd_sg_quadratic(const void* q, const void* k, const void* v, void* o, int B, int H,

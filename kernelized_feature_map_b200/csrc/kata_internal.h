@@ -45,12 +45,11 @@ inline bool chunked_on_tensor_cores(int p, int dv, kata_dtype_t dt) {
   return dt == KATA_BF16 && (p == 16 || p == 32) && dv == 64;
 }
 
-// Coordinate blocks per (b,h) of the tensor-core chunked state: p = 32 splits
-// its packed feature over four blocks of the p = 16 size (one CTA of a
-// cluster each); p = 16 has one.
-inline int chunk_blocks(int p) { return p == 32 ? 4 : 1; }
+
 
 ChunkPlan make_chunk_plan(int B, int H, int T, int p, int dv, int C, kata_dtype_t dt);
+// The plan of the cluster kernels: p = factor width, `blocks` CTAs per unit.
+ChunkPlan make_cluster_plan(int B, int H, int T, int p, int blocks, int dv, int C);
 
 // Every argument check of kata_fwd_chunked except the workspace's (kata_api.cu).
 kata_status_t check_chunked_args(const void* q, const void* k, const void* v, const void* o, int B, int H, int T,
@@ -116,15 +115,21 @@ cudaError_t launch_chunk_readout_sm100(const void* q, const void* k, const void*
                                        const float* S0, const float* z0, float* S_out, float* z_out,
                                        const ChunkPlan& pl, const WaitCtl& wc, cudaStream_t st);
 
-// chunk_p32_sm100.cu -- the same for p = 32, the state split over four
-// coordinate blocks (records ((bh * 4 + block) * G + g)).  The readout adds
-// S0/z0 (when non-null) to the scanned prefix of every super-chunk itself,
-// so the scan runs without an initial state.
-cudaError_t launch_chunk_state_p32(const void* k, const void* v, float* ws, const ChunkPlan& pl, const WaitCtl& wc,
-                                   cudaStream_t st);
-cudaError_t launch_chunk_readout_p32(const void* q, const void* k, const void* v, void* o, const float* ws,
-                                     const float* S0, const float* z0, float* S_out, float* z_out,
-                                     const ChunkPlan& pl, const WaitCtl& wc, cudaStream_t st);
+// chunk_cluster_sm100.cu -- the same with the packed state split over the
+// CTAs of a cluster: p = 32 (groups = 1: four blocks) and KATA-Mg over d = 64
+// (groups = 2 of p = 32: eight blocks; groups = 4 of p = 16: four blocks);
+// q, k, v, o in [B,H,T,*] or, with bthd, [B,T,H,*].  Records
+// ((bh * blocks + block) * G + g).  The readout adds S0/z0 (when non-null)
+// to the scanned prefix of every super-chunk itself, so the scan runs
+// without an initial state.  pl.p is the width of one factor.
+bool cluster_chunked_supports(int p, int groups, int dv);
+inline int cluster_blocks(int p, int groups) { return groups * (p == 32 ? 4 : 1); }
+cudaError_t launch_chunk_state_cluster(const void* k, const void* v, float* ws, const ChunkPlan& pl, int H, int groups,
+                                       bool bthd, const WaitCtl& wc, cudaStream_t st);
+cudaError_t launch_chunk_readout_cluster(const void* q, const void* k, const void* v, void* o, const float* ws,
+                                         const float* S0, const float* z0, float* S_out, float* z_out,
+                                         const ChunkPlan& pl, int H, int groups, bool bthd, const WaitCtl& wc,
+                                         cudaStream_t st);
 
 // Current bound on in-kernel waits and the status word (kata_api.cu).
 WaitCtl wait_ctl();

@@ -188,3 +188,100 @@ def test_sg_flash_matches_oracle(kata, shape, layout):
     torch.cuda.synchronize()
     assert kata.kata_get_status() == 0
     assert row_rel_err(got, ref, v) <= TOL["bf16"]
+
+
+# ---------------------------------------------------------------------------
+# KATA-Mg on the exact O(T) chunked path (cluster kernels: each group's
+# packed state in its own CTAs, each group's intra-chunk squared scores in
+# the first of them)
+# ---------------------------------------------------------------------------
+
+def _run_mg_chunked(K, q, k, v, groups, layout, C=64, S0=None, z0=None, return_state=False):
+    import torch
+    dq, dk, dv_ = ((to_dev(_bthd(x), "bf16") if layout == "bthd" else to_dev(x, "bf16")) for x in (q, k, v))
+    res = K.kata_fwd_mg_chunked(dq, dk, dv_, groups, C=C, layout=layout, S0=S0, z0=z0, return_state=return_state)
+    torch.cuda.synchronize()
+    assert K.kata_get_status() == 0
+    o = res[0] if return_state else res
+    out = _bthd(to_np(o)) if layout == "bthd" else to_np(o)
+    return (out, res[1], res[2]) if return_state else out
+
+
+MG_CHUNKED_SHAPES = [
+    # B, H, T, d, groups -- dv = 64; T ragged, one or several chunks
+    (2, 2, 1000, 64, 4),
+    (1, 3, 777, 64, 2),
+    (1, 2, 129, 64, 4),
+    (2, 1, 385, 64, 2),
+    (1, 2, 600, 32, 1),   # the single factor p = 32 through the cluster kernel ([B,T,H,*] too)
+]
+
+
+@pytest.mark.parametrize("layout", ["bhtd", "bthd"])
+@pytest.mark.parametrize("shape", MG_CHUNKED_SHAPES, ids=lambda s: "B%dH%dT%dd%dg%d" % s)
+def test_mg_chunked_matches_oracle(kata, shape, layout):
+    B, H, T, d, g = shape
+    q, k, v = workloads.normal_qkv(B, H, T, d, 64, seed=400 + T + g, dtype="bf16")
+    ref = oracle.direct_mg(q, k, v, g)
+    err = row_rel_err(_run_mg_chunked(kata, q, k, v, g, layout), ref, v)
+    assert err <= TOL["bf16"], (shape, layout, err)
+
+
+@pytest.mark.parametrize("g", [4, 2])
+@pytest.mark.parametrize("B,H,T,t0", [(4, 16, 700, 300), (1, 2, 20000, 7000)])
+def test_mg_chunked_state_in_and_out(kata, g, B, H, T, t0):
+    """Final state against the oracle's (elementwise bound from the
+    arithmetic, as for the single factor), split-and-resume through the
+    device state, and resume from the oracle's state.  With two heads and
+    T = 20000 each sequence spans many super-chunks (state build, scan and
+    prefix records); with 64 heads and T = 700 each is one super-chunk."""
+    import torch
+    d, dv = 64, 64
+    q, k, v = workloads.normal_qkv(B, H, T, d, dv, seed=17 + g, dtype="bf16")
+    o_ref, S_ref, z_ref = oracle.recurrent_mg(q, k, v, g, return_state=True)
+    _, S1, z1 = oracle.recurrent_mg(q[:, :, :t0], k[:, :, :t0], v[:, :, :t0], g, return_state=True)
+    _, S_abs, z_abs = oracle.recurrent_mg(np.abs(q), np.abs(k), np.abs(v), g, return_state=True)
+    eps = 2.0 ** -8 + (T + 4) * 2.0 ** -24
+
+    def state_ok(S_dev, z_dev):
+        return (np.all(np.abs(S_dev.cpu().numpy() - S_ref) <= eps * S_abs + 1e-6)
+                and np.all(np.abs(z_dev.cpu().numpy() - z_ref) <= eps * z_abs + 1e-6))
+
+    o, S, z = _run_mg_chunked(kata, q, k, v, g, "bhtd", return_state=True)
+    assert row_rel_err(o, o_ref, v) <= TOL["bf16"]
+    assert state_ok(S, z)
+    oa, Sa, za = _run_mg_chunked(kata, q[:, :, :t0], k[:, :, :t0], v[:, :, :t0], g, "bhtd", return_state=True)
+    ob, Sb, zb = _run_mg_chunked(kata, q[:, :, t0:], k[:, :, t0:], v[:, :, t0:], g, "bhtd", S0=Sa, z0=za,
+                                 return_state=True)
+    assert row_rel_err(np.concatenate([oa, ob], axis=2), o_ref, v) <= TOL["bf16"]
+    assert state_ok(Sb, zb)
+    o2 = _run_mg_chunked(kata, q[:, :, t0:], k[:, :, t0:], v[:, :, t0:], g, "bthd",
+                         S0=torch.from_numpy(S1.astype(np.float32)).cuda(),
+                         z0=torch.from_numpy(z1.astype(np.float32)).cuda())
+    assert row_rel_err(o2, o_ref[:, :, t0:], v) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("name", sorted(workloads.MG_CONFIGS))
+def test_mg_chunked_full_size_sampled_rows(kata, name):
+    """The benchmark's Mg workloads at full size through the chunked path, on
+    sampled rows the oracle computes one by one; and the same bits in both
+    layouts."""
+    cfg = workloads.MG_CONFIGS[name]
+    B, H, T, d, g, dv = cfg["B"], cfg["H"], cfg["T"], cfg["d"], cfg["groups"], cfg["dv"]
+    q, k, v = workloads.normal_qkv(B, H, T, d, dv, seed=cfg["seed"], dtype=cfg["dtype"])
+    got = _run_mg_chunked(kata, q, k, v, g, cfg["layout"])
+    assert np.array_equal(got, _run_mg_chunked(kata, q, k, v, g, "bhtd" if cfg["layout"] == "bthd" else "bthd"))
+    rng = np.random.default_rng(cfg["seed"])
+    bh = rng.integers(0, B * H, size=96)
+    t = np.concatenate([rng.integers(0, T, size=80), [0, 1, 127, 128, 129, T - 2, T - 1, T // 2] * 2])[:96]
+    ref = oracle.direct_mg_rows(q, k, v, g, bh, t)
+    vmax = np.abs(v.reshape(B * H, -1)).max(axis=1)[bh]
+    assert rows_rel_err(got.reshape(B * H, T, dv)[bh, t], ref, vmax) <= TOL["bf16"]
+
+
+def test_mg_chunked_agrees_with_flash(kata):
+    B, H, T, d, g, dv = 2, 4, 1500, 64, 4, 64
+    q, k, v = workloads.normal_qkv(B, H, T, d, dv, seed=333, dtype="bf16")
+    a = _run_mg_chunked(kata, q, k, v, g, "bhtd")
+    b = _run_mg(kata, q, k, v, g, "bhtd")
+    assert row_rel_err(a, b.astype(np.float64), v) <= 2 * TOL["bf16"]
