@@ -47,6 +47,9 @@
 
 #include "chunk_common.cuh"
 #include "kata_internal.h"
+#include "kata_trace.cuh"
+
+KATA_TRACE_DECLARE(cluster)
 
 namespace kata {
 
@@ -90,17 +93,24 @@ __device__ __forceinline__ uint32_t map_rank(uint32_t a, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
   return r;
 }
-__device__ __forceinline__ void st_cluster_v4(uint32_t a, float x, float y, float z, float w) {
-  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(a), "f"(x), "f"(y), "f"(z), "f"(w)
+// Asynchronous stores into another CTA's shared memory that report their
+// bytes to an mbarrier of that CTA on completion (the issuing thread does
+// not wait; the receiver's barrier counts the bytes).
+__device__ __forceinline__ void st_async_v4(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w,
+                                            uint32_t bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(a),
+               "r"(x), "r"(y), "r"(z), "r"(w), "r"(bar)
                : "memory");
 }
-__device__ __forceinline__ void st_cluster_f32(uint32_t a, float x) {
-  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(a), "f"(x) : "memory");
+__device__ __forceinline__ void st_async_b32(uint32_t a, uint32_t x, uint32_t bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(a), "r"(x), "r"(bar)
+               : "memory");
 }
-// arrive on an mbarrier of a CTA of the cluster, releasing this thread's
-// earlier writes at cluster scope
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster_addr) : "memory");
+// Arrive on an mbarrier of a CTA of the cluster without ordering this
+// thread's earlier memory accesses (a release arrival waits for them at
+// cluster scope, ~1000 cycles per arrival measured).
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t bar_cluster_addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster_addr) : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
   uint32_t ok;
@@ -483,10 +493,12 @@ __global__ void __launch_bounds__(kStateThreads, 1)
 // one buffer: it is refreshed once the advance by chunk c has landed, and
 // the readout of chunk c, issued before that advance, has then completed.
 // Cluster exchange per chunk: slot[src][row][68 floats] in the owning CTA
-// (O columns 0..63, D at 64); recv_full (256 arrivals: every CTA's 2 x rows
-// lanes) completes when all partial rows of the chunk are in; recv_empty[t]
-// in the sending CTA (one arrival per owner-side lane of CTA t) completes
-// when CTA t has read them, so its slot may be reused.
+// (O columns 0..63, D at 64), written with asynchronous remote stores that
+// count their bytes on the owner's recv_full, which completes when all
+// partial rows of the chunk are in (one arrival per phase, with the byte
+// count, from the owner); recv_empty[t] in the sending CTA (one arrival from
+// each of CTA t's two adding warps) completes when CTA t has read them, so
+// its slot may be reused.
 constexpr int kReadCThreads = 640;
 constexpr int kSlotFloats = 68;  // per row: O (64), D, pad
 
@@ -524,6 +536,9 @@ __global__ void __launch_bounds__(kReadCThreads, 1)
   using L = ReadCSmem<P, NG>;
   constexpr int kSt = C::kStages;
   constexpr int kRows = C::kRows;
+  // bytes an owner receives per chunk: from every CTA, its rows' O (64
+  // floats, two 32-column halves) and D
+  constexpr uint32_t kRecvBytes = (uint32_t)C::kCS * kRows * 65 * 4;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::offBar);
@@ -536,8 +551,8 @@ __global__ void __launch_bounds__(kReadCThreads, 1)
   uint64_t* upd_done = rd_done + 1;   // state advanced by the chunk
   uint64_t* o_full = upd_done + 1;    // [2] [O | D] complete
   uint64_t* mma_done = o_full + 2;
-  uint64_t* recv_full = mma_done + 1; // all partial rows of the chunk received (256)
-  uint64_t* recv_empty = recv_full + 1;  // [cluster size] CTA t has read this CTA's rows (2 x rows)
+  uint64_t* recv_full = mma_done + 1; // all partial rows of the chunk received (kRecvBytes)
+  uint64_t* recv_empty = recv_full + 1;  // [cluster size] CTA t has read this CTA's rows (its 2 adding warps)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::offMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::offMisc + 4);
 
@@ -545,6 +560,7 @@ __global__ void __launch_bounds__(kReadCThreads, 1)
   const int blk = (int)cluster_rank();
   const int grp = blk / C::kBPG, bb = blk % C::kBPG;
   const bool lead = bb == 0;  // computes its factor's intra-chunk part
+  KATA_TRACE_BEGIN_IDX(cluster, (blockIdx.y * gridDim.x + blockIdx.x) * gridDim.z + blk);
   const int g = blockIdx.x, bh = blockIdx.y;
   const int t0 = g * Ls;
   const int t1 = min(T, t0 + Ls);
@@ -562,8 +578,8 @@ __global__ void __launch_bounds__(kReadCThreads, 1)
     mbar_init(upd_done, 1);
     for (int b = 0; b < 2; ++b) mbar_init(o_full + b, 1);
     mbar_init(mma_done, 1);
-    mbar_init(recv_full, 256);
-    for (int b = 0; b < C::kCS; ++b) mbar_init(recv_empty + b, 2 * kRows);
+    mbar_init(recv_full, 1);
+    for (int b = 0; b < C::kCS; ++b) mbar_init(recv_empty + b, 2);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -616,7 +632,9 @@ __global__ void __launch_bounds__(kReadCThreads, 1)
     for (int c = 0; c < n_chunks; ++c) {
       const int st = c % kSt, ob = c & 1;
       const uint32_t sV = sStage + st * L::kStage;
+      KATA_TRACE(cluster, c, 0);
       if (!mbar_wait_w(state_full, c & 1, env)) break;
+      KATA_TRACE(cluster, c, 1);
       tc_fence_after();
       if (lead) {
 #pragma unroll
@@ -631,13 +649,16 @@ __global__ void __launch_bounds__(kReadCThreads, 1)
         mma_ts_w(dO, tmem + L::colPQ + ks * 8, desc_add(dsb, ks * kSBAtom), id_rd, ks > 0);
       mma_commit_w(rd_done);
       if (!lead) mma_commit_w(o_full + ob);
+      KATA_TRACE(cluster, c, 2);
       const uint64_t dvo = desc_vones(sV, sOnes);
 #pragma unroll
       for (int ks = 0; ks < kTile / 16; ++ks)
         mma_ss_w(tmem + L::colRun, desc_add(dvo, ks * 2048), desc_add(dpsi, (c & 1) * kPsiBytes + ks * 512), id_u, 1);
       mma_commit_w(upd_done);
+      KATA_TRACE(cluster, c, 3);
       if (lead) {
         if (!mbar_wait_w(p_full, c & 1, env)) break;
+        KATA_TRACE(cluster, c, 4);
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < kTile / 16; ++ks)
@@ -645,6 +666,7 @@ __global__ void __launch_bounds__(kReadCThreads, 1)
         mma_commit_w(o_full + ob);
       }
       mma_commit_w(kv_empty + st);
+      KATA_TRACE(cluster, c, 5);
     }
     mma_commit_w(mma_done);
     mbar_wait_drain(mma_done, 0);
@@ -663,6 +685,7 @@ __global__ void __launch_bounds__(kReadCThreads, 1)
     auto send = [&](int co) -> bool {
       const int ob = co & 1;
       if (!mbar_wait_w(o_full + ob, (co >> 1) & 1, env)) return false;
+      if (m == 0 && h == 0) KATA_TRACE(cluster, co, 10);
       tc_fence_after();
       uint32_t r[32], db;
       tmem_ld32(lane_base + L::colO(ob) + 32 * h, r);
@@ -680,12 +703,13 @@ __global__ void __launch_bounds__(kReadCThreads, 1)
       }
       // the owner has read what this lane sent for chunk co-1
       if (co > 0 && !mbar_wait_cluster_w(empty_local, (co - 1) & 1, env)) return false;
+      if (m == 0 && h == 0) KATA_TRACE(cluster, co, 11);
 #pragma unroll
       for (int e = 0; e < 32; e += 4)
-        st_cluster_v4(slot_remote + (32 * h + e) * 4, __uint_as_float(r[e]), __uint_as_float(r[e + 1]),
-                      __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
-      if (h == 0) st_cluster_f32(slot_remote + 64 * 4, __uint_as_float(db));
-      mbar_arrive_cluster(full_remote);
+        st_async_v4(slot_remote + (32 * h + e) * 4, r[e], r[e + 1], r[e + 2], r[e + 3], full_remote);
+      if (h == 0) st_async_b32(slot_remote + 64 * 4, db, full_remote);
+      if (m == 0 && h == 0) KATA_TRACE(cluster, co, 26);
+      if (m == 0 && h == 0) KATA_TRACE(cluster, co, 12);
       return true;
     };
     bool ok = true;
@@ -699,6 +723,7 @@ __global__ void __launch_bounds__(kReadCThreads, 1)
     for (int c = 0; ok && c < n_chunks; ++c) {
       if (lead) {
         if (!mbar_wait_w(s_full, c & 1, env)) break;
+        if (m == 0 && h == 0) KATA_TRACE(cluster, c, 8);
         tc_fence_after();
 #pragma unroll
         for (int b2 = 0; b2 < 2; ++b2) {
@@ -731,6 +756,7 @@ __global__ void __launch_bounds__(kReadCThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(p_full);
+        if (m == 0 && h == 0) KATA_TRACE(cluster, c, 9);
         if (c > 0) ok = send(c - 1);
       } else {
         ok = send(c);
@@ -745,8 +771,11 @@ __global__ void __launch_bounds__(kReadCThreads, 1)
     uint8_t* slab = smem + L::offOut + h * (kRows * 64);
     const float* slot = reinterpret_cast<const float*>(smem + L::offSlot) + lr * kSlotFloats;
     const uint32_t full_local = smem_u32(recv_full);
+    // the bytes of chunk 0 are expected (one arrival per phase, by one lane)
+    if (h == 0 && lane == 0 && n_chunks > 0) mbar_arrive_expect_tx(recv_full, kRecvBytes);
     for (int c = 0; c < n_chunks; ++c) {
       if (!mbar_wait_cluster_w(full_local, c & 1, env)) break;
+      if (lane == 0 && h == 0) KATA_TRACE(cluster, c, 14);
       float acc[32], D = 0.f;
 #pragma unroll
       for (int e = 0; e < 32; ++e) acc[e] = 0.f;
@@ -763,15 +792,25 @@ __global__ void __launch_bounds__(kReadCThreads, 1)
         }
         D += row[64];
       }
-      // every source's slot may be refilled
-      if (act) {
+      if (lane == 0 && h == 0) KATA_TRACE(cluster, c, 23);
+      // the bytes of chunk c+1 are expected before any source may send
+      // them (they wait for this warp's arrival below)
+      if (h == 0 && lane == 0 && c + 1 < n_chunks) mbar_arrive_expect_tx(recv_full, kRecvBytes);
+      // every source's slot may be refilled: one arrival per warp and
+      // source once all its lanes have read (the values are in registers,
+      // already added, so no later store into the slot can change them)
+      __syncwarp();
+      if (lane == 0) {
 #pragma unroll
-        for (int s = 0; s < C::kCS; ++s) mbar_arrive_cluster(map_rank(smem_u32(recv_empty + blk), (uint32_t)s));
+        for (int s = 0; s < C::kCS; ++s)
+          mbar_arrive_cluster_relaxed(map_rank(smem_u32(recv_empty + blk), (uint32_t)s));
       }
+      if (lane == 0 && h == 0) KATA_TRACE(cluster, c, 24);
       const float inv = D > 0.f ? 1.f / D : 0.f;
       // this warp's staging box is free once its previous store has read it
       if (lane == 0) bulk_wait_read_all();
       __syncwarp();
+      if (lane == 0 && h == 0) KATA_TRACE(cluster, c, 25);
       if (act) {
         uint8_t* orow = slab + lane * 64;
 #pragma unroll
@@ -787,6 +826,7 @@ __global__ void __launch_bounds__(kReadCThreads, 1)
       if (lane == 0) {
         store_tile(&tm_o, slab, 32 * h, t0 + c * kTile + kRows * blk, bh, H, bthd);
         bulk_commit_group();
+        if (h == 0) KATA_TRACE(cluster, c, 15);
       }
     }
     if (lane == 0) bulk_wait_all();
@@ -837,6 +877,7 @@ __global__ void __launch_bounds__(kReadCThreads, 1)
     for (int c = 0; ok && c + 1 < n_chunks; ++c) {
       const int st1 = (c + 1) % kSt;
       if (!mbar_wait_w(kv_full + st1, ((c + 1) / kSt) & 1, env)) break;
+      if (m == 0) KATA_TRACE(cluster, c, psi_group ? 16 : 21);
       if (psi_group) {
         // psi~(k_{c+1}) into the buffer last read by the advance by chunk
         // c-1, which this group saw complete in the previous iteration
@@ -845,6 +886,7 @@ __global__ void __launch_bounds__(kReadCThreads, 1)
         uint32_t wq[kNPW];
         psi_q_formed(c + 1, wq);
         if (!mbar_wait_w(rd_done, c & 1, env)) break;
+        if (m == 0) KATA_TRACE(cluster, c, 19);
         tc_fence_after();
         store_psi_q_tmem(lane_base + L::colPQ, wq);
         tmem_wait_st();
@@ -852,11 +894,13 @@ __global__ void __launch_bounds__(kReadCThreads, 1)
       // the state after chunk c is complete; the readout of chunk c, issued
       // before that advance, has read the single bf16 copy
       if (!mbar_wait_w(upd_done, c & 1, env)) break;
+      if (m == 0) KATA_TRACE(cluster, c, psi_group ? 17 : 22);
       tc_fence_after();
       if (quarter < 3) state_half_to_bf16(lane_base + L::colRun, sb, m, active, half);
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(state_full);
+      if (m == 0) KATA_TRACE(cluster, c, psi_group ? 18 : 20);
     }
     // the last super-chunk ends at token T: its running state, once the
     // advance by its last chunk has landed, is this block's part of the

@@ -34,6 +34,14 @@ constexpr int kTraceSlots = 32;
                ? g_trace_buf_##name + (size_t)cta_ * ::kata::kTraceTiles * ::kata::kTraceSlots \
                : (unsigned long long*)nullptr;                                          \
   }()
+// The same with an explicit CTA index (kernels with a 3-D grid).
+#define KATA_TRACE_BEGIN_IDX(name, idx)                                                   \
+  unsigned long long* const kata_trace_ptr_##name = [&] {                                \
+    const unsigned cta_ = (idx);                                                         \
+    return (g_trace_buf_##name && cta_ < (unsigned)::kata::kTraceCtas)                   \
+               ? g_trace_buf_##name + (size_t)cta_ * ::kata::kTraceTiles * ::kata::kTraceSlots \
+               : (unsigned long long*)nullptr;                                          \
+  }()
 #define KATA_TRACE(name, tile, slot)                                                     \
   do {                                                                                 \
     if (kata_trace_ptr_##name && (tile) < ::kata::kTraceTiles)                           \
@@ -43,6 +51,9 @@ constexpr int kTraceSlots = 32;
 #define KATA_TRACE_DECLARE(name)
 #define KATA_TRACE_BEGIN(name) \
   do {                         \
+  } while (0)
+#define KATA_TRACE_BEGIN_IDX(name, idx) \
+  do {                                  \
   } while (0)
 #define KATA_TRACE(name, tile, slot) \
   do {                               \
