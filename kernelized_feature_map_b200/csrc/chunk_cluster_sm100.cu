@@ -487,7 +487,8 @@ __global__ void __launch_bounds__(kStateThreads, 1)
 //   warps 10-13  prefix in; psi~_b(q_{c+1}) into TMEM once the readout of
 //                chunk c has read psi~_b(q_c); bf16 copy of coordinates 72..143
 //   warps 18-19  the partial rows of this CTA's own rows summed over the
-//                cluster, o = O / D, stored (columns 0..31 and 32..63)
+//                cluster, o = O / D written from registers (columns 0..31
+//                and 32..63)
 // MMA order per chunk: [first CTA of a factor: scores], readout, advance,
 // [first CTA of a factor: intra-chunk weights].  The bf16 copy of S~_b has
 // one buffer: it is refreshed once the advance by chunk c has landed, and
@@ -512,8 +513,7 @@ struct ReadCSmem {
   static constexpr int offPsi = offOnes + kOnesBytes;                      // 2 buffers
   static constexpr int offSB = offPsi + 2 * kPsiBytes;                     // 1 buffer
   static constexpr int offSlot = offSB + kSBBytes;                         // [sources]
-  static constexpr int offOut = (offSlot + C::kCS * kSlotBytes + 1023) / 1024 * 1024;  // 2 boxes [rows x 32] bf16
-  static constexpr int offBar = offOut + 2 * C::kRows * 64;
+  static constexpr int offBar = offSlot + C::kCS * kSlotBytes;
   static constexpr int kBars = 2 * C::kStages + 9 + C::kCS;
   static constexpr int offMisc = offBar + kBars * 8;
   static constexpr int kBytes = offMisc + 16 + 1024;
@@ -521,14 +521,14 @@ struct ReadCSmem {
   static constexpr uint32_t colO(int b) { return 144u + 80u * (uint32_t)b; }  // [O | D] x 2
   static constexpr uint32_t colPQ = 304;                                   // psi~_b(Q_c), 72
   static constexpr uint32_t colS = 384;                                    // scores / weights, 128
-  static_assert(offSlot % 16 == 0 && offOut % 1024 == 0 && offSB % 1024 == 0 && kBytes <= 232448,
+  static_assert(offSlot % 16 == 0 && offSB % 1024 == 0 && kBytes <= 232448,
                 "shared-memory layout");
 };
 
 template <int P, int NG>
 __global__ void __launch_bounds__(kReadCThreads, 1)
     chunk_readout_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                                 const __grid_constant__ CUtensorMap tm_v, void* __restrict__ o,
                                  const float* __restrict__ ws, const float* __restrict__ S0,
                                  const float* __restrict__ z0, float* __restrict__ S_out, float* __restrict__ z_out,
                                  int T, int H, int bthd, int Ls, int G, long long record_floats, WaitCtl wc) {
@@ -768,7 +768,12 @@ __global__ void __launch_bounds__(kReadCThreads, 1)
     const int h = warp - 18;  // output columns 32h .. 32h+31
     const bool act = lane < kRows;
     const int lr = act ? lane : 0;  // this lane's own row
-    uint8_t* slab = smem + L::offOut + h * (kRows * 64);
+    // row t of this head of o ([B,H,T,dv] or [B,T,H,dv])
+    const int ob = bh / H, oh = bh - ob * H;
+    auto out_row = [&](int t) {
+      const size_t r = bthd ? ((size_t)ob * T + t) * H + oh : ((size_t)ob * H + oh) * T + t;
+      return reinterpret_cast<__nv_bfloat16*>(o) + r * kDV;
+    };
     const float* slot = reinterpret_cast<const float*>(smem + L::offSlot) + lr * kSlotFloats;
     const uint32_t full_local = smem_u32(recv_full);
     // the bytes of chunk 0 are expected (one arrival per phase, by one lane)
@@ -807,29 +812,22 @@ __global__ void __launch_bounds__(kReadCThreads, 1)
       }
       if (lane == 0 && h == 0) KATA_TRACE(cluster, c, 24);
       const float inv = D > 0.f ? 1.f / D : 0.f;
-      // this warp's staging box is free once its previous store has read it
-      if (lane == 0) bulk_wait_read_all();
-      __syncwarp();
-      if (lane == 0 && h == 0) KATA_TRACE(cluster, c, 25);
-      if (act) {
-        uint8_t* orow = slab + lane * 64;
+      // o = O / D straight from registers: this lane's 32 values of its row
+      // (64 bytes; the other warp writes the other half of the row).  A TMA
+      // store from shared memory measured ~2300 cycles per chunk here, its
+      // proxy fence waiting behind the cluster's incoming traffic.
+      const int t = t0 + c * kTile + kRows * blk + lane;
+      if (act && t < T) {
+        uint4* dst = reinterpret_cast<uint4*>(out_row(t) + 32 * h);
 #pragma unroll
         for (int e = 0; e < 4; ++e)
-          *reinterpret_cast<uint4*>(orow + ((e ^ ((lane >> 1) & 3)) << 4)) =
-              make_uint4(pack_bf16x2(acc[8 * e] * inv, acc[8 * e + 1] * inv),
-                         pack_bf16x2(acc[8 * e + 2] * inv, acc[8 * e + 3] * inv),
-                         pack_bf16x2(acc[8 * e + 4] * inv, acc[8 * e + 5] * inv),
-                         pack_bf16x2(acc[8 * e + 6] * inv, acc[8 * e + 7] * inv));
+          dst[e] = make_uint4(pack_bf16x2(acc[8 * e] * inv, acc[8 * e + 1] * inv),
+                              pack_bf16x2(acc[8 * e + 2] * inv, acc[8 * e + 3] * inv),
+                              pack_bf16x2(acc[8 * e + 4] * inv, acc[8 * e + 5] * inv),
+                              pack_bf16x2(acc[8 * e + 6] * inv, acc[8 * e + 7] * inv));
       }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        store_tile(&tm_o, slab, 32 * h, t0 + c * kTile + kRows * blk, bh, H, bthd);
-        bulk_commit_group();
-        if (h == 0) KATA_TRACE(cluster, c, 15);
-      }
+      if (lane == 0 && h == 0) KATA_TRACE(cluster, c, 15);
     }
-    if (lane == 0) bulk_wait_all();
   } else {
     // ------------------------------------------------------------- psi~ and state copies
     const bool psi_group = warp < 10;   // warps 6-9: psi~(k) + half 0; warps 10-13: half 1 + psi~(q)
@@ -952,11 +950,10 @@ cudaError_t launch_readout_t(const void* q, const void* k, const void* v, void* 
   using L = ReadCSmem<P, NG>;
   if (!ws && pl.G != 1) return cudaErrorInvalidValue;
   const int B = pl.BH / H;
-  CUtensorMap tq, tk, tv, to;
+  CUtensorMap tq, tk, tv;
   if (!make_tmap_bf16_4d(&tq, q, C::kD, pl.T, H, B, bthd, P, kTile) ||
       !make_tmap_bf16_4d(&tk, k, C::kD, pl.T, H, B, bthd, P, kTile) ||
-      !make_tmap_bf16_4d(&tv, v, kDV, pl.T, H, B, bthd, kDV, kTile) ||
-      !make_tmap_bf16_4d(&to, o, kDV, pl.T, H, B, bthd, 32, C::kRows))
+      !make_tmap_bf16_4d(&tv, v, kDV, pl.T, H, B, bthd, kDV, kTile))
     return cudaErrorInvalidValue;
   auto kern = chunk_readout_cluster_kernel<P, NG>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
@@ -976,7 +973,7 @@ cudaError_t launch_readout_t(const void* q, const void* k, const void* v, void* 
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = ws ? 2 : 1;
-  return cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, to, ws, S0, z0, S_out, z_out, pl.T, H, bthd ? 1 : 0, pl.Ls, pl.G,
+  return cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, o, ws, S0, z0, S_out, z_out, pl.T, H, bthd ? 1 : 0, pl.Ls, pl.G,
                             (long long)pl.record_floats, wc);
 }
 
