@@ -234,7 +234,7 @@ def run_ours(args, rank, world, local_rank):
     z = torch.empty((B, H, p * p), dtype=torch.float32, device=dev)
     ws = torch.empty(max(256, K.kata_fwd_chunked_workspace_size(B, H, T, p, dv, C, bf)), dtype=torch.uint8,
                      device=dev)
-    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    flush = L2Flush(torch, dev)
     stream = torch.cuda.current_stream(dev)
 
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
@@ -253,7 +253,7 @@ def run_ours(args, rank, world, local_rank):
 
     for _ in range(args.warmup):
         step()
-        flush.fill_(1)
+        flush()
     torch.cuda.synchronize()
     if K.kata_get_status() != 0:
         raise RuntimeError("kernel reported a wait timeout during warm-up")
@@ -280,7 +280,7 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
         for _ in range(args.warmup):
             graph.replay()
-            flush.fill_(1)
+            flush()
         torch.cuda.synchronize()
 
     recs, grecs = [], []
@@ -295,7 +295,7 @@ def run_ours(args, rank, world, local_rank):
         # per-path times: the calls launched one by one, events between them
         for _ in range(args.steps):
             step(recs)
-            flush.fill_(1)
+            flush()
         # the step as a whole: graph replays
         if graph is not None:
             for _ in range(args.steps):
@@ -303,7 +303,7 @@ def run_ours(args, rank, world, local_rank):
                 a.record(stream)
                 graph.replay()
                 b.record(stream)
-                flush.fill_(1)
+                flush()
                 grecs.append((a, b))
         torch.cuda.synchronize()
         windows["step"] = (t_start, time.time())
@@ -353,7 +353,7 @@ def run_ours(args, rank, world, local_rank):
                     s_cmp.wait_event(ev_in[bi])
                     if i >= 2:
                         s_cmp.wait_event(ev_out[bi])  # step i-2's outputs have been copied out
-                    flush.fill_(1)
+                    flush()
                     K.kata_fwd_quadratic(st_["q"], st_["k"], st_["v"], o=st_["oq"])
                     K.kata_fwd_chunked(st_["q"], st_["k"], st_["v"], C=C, o=st_["oc"], workspace=st_["ws"],
                                        S_out=st_["S"], z_out=st_["z"], return_state=True)
@@ -392,7 +392,9 @@ def run_ours(args, rank, world, local_rank):
             windows["decode_b64"] = (t0, time.time())
             if args.sweep:
                 long["sweep"], long["recall"] = run_sweep(args, K, torch, dev, stream, flush)
+                t0 = time.time()
                 long["mg"] = run_mg(args, K, torch, dev, stream, flush)
+                windows["mg"] = (t0, time.time())
                 long["train"] = run_train(args, K, torch, dev, stream, flush)
         t_end = time.time()
         time.sleep(0.15)
@@ -417,7 +419,7 @@ def run_decode_b64(args, K, torch, dev, stream, flush):
     o = torch.empty((c["B"], c["H"], c["dv"]), dtype=bf, device=dev)
     ms = []
     for i in range(5 + args.long_steps * 4):
-        flush.fill_(1)
+        flush()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         K.kata_decode_step(qd, kd, vd, Sd, zd, o=o)
@@ -443,7 +445,7 @@ def run_long(args, K, torch, dev, stream, flush):
                          device=dev)
         ms = []
         for i in range(3 + args.long_steps):
-            flush.fill_(1)
+            flush()
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
             K.kata_fwd_chunked(q, k, v, C=C, o=o, workspace=ws)
@@ -457,7 +459,7 @@ def run_long(args, K, torch, dev, stream, flush):
                                           3, 1)
     ms = []
     for i in range(2 + max(1, args.long_steps // 4)):
-        flush.fill_(1)
+        flush()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         K.kata_fwd_quadratic(q, k, v, o=o)
@@ -470,11 +472,29 @@ def run_long(args, K, torch, dev, stream, flush):
     return out
 
 
+class L2Flush:
+    """Empties the 126 MB L2 between timed calls: a 512 MiB write evicts
+    whatever the last call left, then a 256 MiB read replaces the written
+    (dirty) lines with clean ones, so that the next timed kernel neither
+    finds its data in L2 nor pays for writing the flush buffer back to HBM
+    (for the decode step, ~126 MB of write-back against its 136 MB of state
+    traffic).  Runs outside the timed events."""
+
+    def __init__(self, torch, dev):
+        self.w = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
+        self.r = torch.ones(64 * 1024 * 1024, dtype=torch.float32, device=dev)
+        self.acc = torch.empty((), dtype=torch.float32, device=dev)
+
+    def __call__(self):
+        self.w.fill_(1)
+        self.acc.copy_(self.r.sum())
+
+
 def _time_call(fn, flush, stream, reps, warm):
     import torch
     ms = []
     for i in range(warm + reps):
-        flush.fill_(1)
+        flush()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         fn()
@@ -539,11 +559,37 @@ def run_mg(args, K, torch, dev, stream, flush):
         o = torch.empty_like(v)
         ms = _time_call(lambda: K.kata_fwd_mg_quadratic(q, k, v, g, layout=cfg["layout"], o=o), flush, stream, 10, 3)
         out[name] = dict(B=B, H=H, T=T, d=d, groups=g, dv=dv, layout=cfg["layout"], ms=ms)
+        # the chunked (O(T)) KATA-Mg path on the same inputs
+        ws = torch.empty(max(256, K.kata_fwd_mg_chunked_workspace_size(B, H, T, d, g, dv, 64)), dtype=torch.uint8,
+                         device=dev)
+        ms_c = _time_call(lambda: K.kata_fwd_mg_chunked(q, k, v, g, C=64, layout=cfg["layout"], o=o, workspace=ws),
+                          flush, stream, 10, 3)
+        out["chunked_" + name] = dict(B=B, H=H, T=T, d=d, groups=g, dv=dv, layout=cfg["layout"], ms=ms_c,
+                                      chunked=True)
         # KATA-Sigma-g (summed factors) on the same inputs: g^2 score blocks
         ms_sg = _time_call(lambda: K.kata_fwd_sg_quadratic(q, k, v, g, layout=cfg["layout"], o=o), flush, stream, 10,
                            3)
         out["sg" + name[2:]] = dict(B=B, H=H, T=T, d=d, groups=g, dv=dv, layout=cfg["layout"], ms=ms_sg, summed=True)
         del q, k, v, o
+    # the chunked path at the long context (B = 1, H = 16, T = 131072), where
+    # the flash-style path costs seconds; device-drawn inputs
+    gen_l = torch.Generator(device=dev)
+    for g in (2, 4):
+        B, H, T, d, dv = 1, 16, 131072, 64, 64
+        gen_l.manual_seed(500 + g)
+        q = torch.randn((B, T, H, d), generator=gen_l, device=dev)
+        k = torch.randn((B, T, H, d), generator=gen_l, device=dev)
+        q = (q / q.norm(dim=-1, keepdim=True)).to(bf)
+        k = (k / k.norm(dim=-1, keepdim=True)).to(bf)
+        v = torch.randn((B, T, H, dv), generator=gen_l, device=dev).to(bf)
+        o = torch.empty_like(v)
+        ws = torch.empty(max(256, K.kata_fwd_mg_chunked_workspace_size(B, H, T, d, g, dv, 64)), dtype=torch.uint8,
+                         device=dev)
+        ms_c = _time_call(lambda: K.kata_fwd_mg_chunked(q, k, v, g, C=64, layout="bthd", o=o, workspace=ws), flush,
+                          stream, 5, 2)
+        out["chunked_mg%d_ctx131k" % g] = dict(B=B, H=H, T=T, d=d, groups=g, dv=dv, layout="bthd", ms=ms_c,
+                                               chunked=True)
+        del q, k, v, o, ws
     # decode step on the concatenated per-group state (B = 64, as for the
     # single-factor decode line): HBM-bound, the state is read and written once
     gen = torch.Generator(device=dev)
@@ -673,6 +719,11 @@ def run_case(args):
         o = torch.empty_like(v)
         if args.case == "mg":
             call = lambda: K.kata_fwd_mg_quadratic(q, k, v, g, layout=args.layout, o=o)  # noqa: E731
+        elif args.case == "mg_chunked":
+            ws = torch.empty(max(256, K.kata_fwd_mg_chunked_workspace_size(B, H, T, d, g, dv, args.C, bf)),
+                             dtype=torch.uint8, device=dev)
+            call = lambda: K.kata_fwd_mg_chunked(q, k, v, g, C=args.C, layout=args.layout, o=o,  # noqa: E731
+                                                 workspace=ws)
         elif args.layout != "bhtd":
             raise SystemExit("--layout bthd is for --case mg")
         elif args.case == "quadratic":
@@ -703,7 +754,8 @@ def config_dict(cfg, world):
         "B": cfg["B"], "H": cfg["H"], "T": cfg["T"], "p": cfg["p"], "dv": cfg["dv"], "C": cfg["C"],
         "step": "kata_fwd_quadratic + kata_fwd_chunked(final state) + kata_decode_step",
         "launch": "step timed as a CUDA graph replay of the three calls; per-path times launched one by one",
-        "l2": "flushed between timed steps (512 MiB write outside the timed events)",
+        "l2": "flushed between timed steps outside the timed events: a 512 MiB write, then a 256 MiB read so "
+              "that the lines left in L2 are clean",
         "parallelism": "independent (b,h) batches per rank, no collective" if world > 1 else "1 GPU"}
 
 
@@ -721,7 +773,7 @@ def main():
     ap.add_argument("--graph", type=int, default=1, help="time the step as a CUDA graph replay (per-path times stay eager)")
     ap.add_argument("--ref-budget", type=float, default=15.0, help="seconds of oracle work per reference step")
     pc = ap.add_argument_group("--case: launch one call a few times on device-drawn inputs (for profilers)")
-    pc.add_argument("--case", choices=["quadratic", "chunked", "mg", "decode", "train"])
+    pc.add_argument("--case", choices=["quadratic", "chunked", "mg", "mg_chunked", "decode", "train"])
     pc.add_argument("--B", type=int, default=8)
     pc.add_argument("--H", type=int, default=16)
     pc.add_argument("--T", type=int, default=2048)
@@ -807,6 +859,21 @@ def roofline_points(res, peaks, cfg):
                                                                                      dc["dv"]),
                              dc["ms"], dc["B"], decode_bytes(dc["B"] * dc["H"], dc["p"], dc["dv"]),
                              cl.get("decode_b64")))
+        # KATA-Mg itself (the metric's name): flash-style at T = 2048 and the
+        # chunked path at T = 2048 and 131072, d = 64 in 2 or 4 groups
+        for name, m in sorted(lg.get("mg", {}).items()):
+            if "P" in m or m.get("summed"):
+                continue
+            wl = "KATA-Mg B=%d H=%d T=%d d=%d groups=%d dv=%d bf16 [%s]" % (m["B"], m["H"], m["T"], m["d"],
+                                                                          m["groups"], m["dv"], m["layout"])
+            if m.get("chunked"):
+                pts.append(hbm_point("mg_chunked", wl, m["ms"], m["B"] * m["T"],
+                                     m["B"] * m["H"] * m["T"] * (2 * m["d"] + 2 * m["dv"]) * 2, cl.get("mg"),
+                                     T=m["T"], groups=m["groups"]))
+            else:
+                pts.append(tensor_point("mg_quadratic", wl, m["ms"], m["B"] * m["T"],
+                                        flash_flops(m["B"] * m["H"], m["T"], m["d"], m["dv"]), cl.get("mg"),
+                                        T=m["T"], groups=m["groups"]))
     return pts
 
 
@@ -894,6 +961,15 @@ def report(args, res, step_ms, e2e_ms, world):
                             m["B"], m["H"], m["d"], m["groups"], m["P"], m["dv"]),
                         "ms": m["ms"], "tokens_per_s": m["B"] / (m["ms"] * 1e-3),
                         "hbm_frac": mb / (m["ms"] * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+                elif m.get("chunked"):
+                    # chunked KATA-Mg: HBM fraction by q, k, v read and o
+                    # written once (2d + 2dv bf16 values per token-head)
+                    cb = m["B"] * m["H"] * m["T"] * (2 * m["d"] + 2 * m["dv"]) * 2
+                    line["mg"][name] = {
+                        "workload": "KATA-Mg chunked B=%d H=%d T=%d d=%d groups=%d dv=%d bf16 [%s]" % (
+                            m["B"], m["H"], m["T"], m["d"], m["groups"], m["dv"], m["layout"]),
+                        "ms": m["ms"], "tokens_per_s": m["B"] * m["T"] / (m["ms"] * 1e-3),
+                        "hbm_frac": cb / (m["ms"] * 1e-3) / 1e9 / peaks["hbm_gbs"]}
                 else:
                     # score flops: d per pair for KATA-Mg, g*d for KATA-Sigma-g
                     # (every query group against every key group)
