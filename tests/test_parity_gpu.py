@@ -129,10 +129,12 @@ def test_empty_sequence_is_a_noop(kata):
 # With 128 (b,h) pairs and T = 700 every pair is one super-chunk (no
 # workspace: the readout starts from S0 and writes the final state); with 2
 # pairs and T = 20000 each spans many, with the state build, the scan and
-# the prefix records in between.
+# the prefix records in between; with 16 pairs and T = 3000 (and the 1900
+# tokens resumed from S0 after 1100) each spans a handful (8 super-chunks of
+# the bf16 p = 16 plan), the regime of the long-context benchmark.
 # p = 32 in bf16 runs the four-block cluster kernels (the state split over
-# four coordinate blocks, one CTA each), with the same two regimes.
-@pytest.mark.parametrize("B,H,T,t0", [(8, 16, 700, 300), (1, 2, 20000, 7000)])
+# four coordinate blocks, one CTA each), with the same regimes.
+@pytest.mark.parametrize("B,H,T,t0", [(8, 16, 700, 300), (1, 2, 20000, 7000), (2, 8, 3000, 1100)])
 @pytest.mark.parametrize("dtype,p", [("f32", 16), ("bf16", 16), ("bf16", 32)])
 def test_chunked_state_in_and_out(kata, dtype, p, B, H, T, t0):
     import torch
