@@ -556,3 +556,108 @@ def test_sigma_g_feature_dimension_matches_state_size_formula(d, g):
     p = d // g
     f = osg.features_sg(rng.standard_normal((3 * p * p, d)), g)
     assert np.linalg.matrix_rank(f) == p * (p + 1) // 2
+
+
+# ---------------------------------------------------------------------------
+# first-order (psi(u) = u) attention: pins of the numpy oracle
+# ---------------------------------------------------------------------------
+
+from oracle import first_order as ofo  # noqa: E402
+
+# Worked example, by hand (d = 1, dv = 1): q = (1, 1, 2), k = (1, 2, -1),
+# v = (3, 5, 7).
+#   t = 0: w = (1)            -> 3 / 1                  = 3
+#   t = 1: w = (1, 2)         -> (3 + 10) / 3           = 13/3
+#   t = 2: w = (2, 4, -2)     -> (6 + 20 - 14) / 4      = 3
+FO_Q, FO_K, FO_V = [1.0, 1.0, 2.0], [1.0, 2.0, -1.0], [3.0, 5.0, 7.0]
+FO_WANT = [3.0, 13.0 / 3.0, 3.0]
+
+
+def _fo_pins_hold(mod) -> bool:
+    """The pin set of the first-order oracle, as one predicate (used on the
+    oracle itself and on copies with planted mistakes)."""
+    ok = True
+    q = np.array(FO_Q).reshape(1, 1, 3, 1)
+    k = np.array(FO_K).reshape(1, 1, 3, 1)
+    v = np.array(FO_V).reshape(1, 1, 3, 1)
+    for fn in (mod.direct_linear, mod.recurrent_linear):
+        ok = ok and np.allclose(fn(q, k, v)[0, 0, :, 0], FO_WANT, rtol=0, atol=1e-13)
+        # zero denominator: q = (1, 1), k = (1, -1) -> D_1 = 0 -> o_1 = 0
+        o = fn(np.ones((1, 1, 2, 1)), np.array([1.0, -1.0]).reshape(1, 1, 2, 1), np.array([2.0, 4.0]).reshape(1, 1, 2, 1))
+        ok = ok and np.allclose(o[0, 0, :, 0], [2.0, 0.0], rtol=0, atol=1e-13)
+        # the first output is the first value whenever q_0 . k_0 != 0, also
+        # when it is negative: q_0 . k_0 = 1*(-3) + 2*1 = -1
+        o = fn(np.array([1.0, 2.0]).reshape(1, 1, 1, 2), np.array([-3.0, 1.0]).reshape(1, 1, 1, 2),
+               np.array([3.0, -4.0]).reshape(1, 1, 1, 2))
+        ok = ok and np.allclose(o[0, 0, 0], [3.0, -4.0], rtol=0, atol=1e-13)
+    # the KATA weight is the first-order weight of the features vec(u u^T):
+    # first-order attention on psi(q), psi(k) is the (independently pinned)
+    # C oracle's KATA attention on q, k
+    q, k, v = _rand(B=1, H=2, T=23, p=3, dv=2, seed=600)
+    psi = lambda u: np.einsum("bhti,bhtj->bhtij", u, u).reshape(u.shape[:3] + (u.shape[3] ** 2,))  # noqa: E731
+    for fn in (mod.direct_linear, mod.recurrent_linear):
+        ok = ok and np.allclose(fn(psi(q), psi(k), v), oracle.direct(q, k, v), rtol=1e-10, atol=1e-12)
+    return bool(ok)
+
+
+def test_first_order_pins():
+    assert _fo_pins_hold(ofo)
+
+
+@pytest.mark.parametrize("shape", [(1, 1, 1, 1, 1), (2, 3, 37, 4, 5), (1, 2, 64, 16, 8)])
+def test_first_order_direct_equals_recurrent(shape):
+    B, H, T, d, dv = shape
+    q, k, v = _rand(B, H, T, d, dv, seed=610 + T)
+    np.testing.assert_allclose(ofo.recurrent_linear(q, k, v), ofo.direct_linear(q, k, v), rtol=1e-9, atol=1e-11)
+
+
+def test_first_order_state_split_and_invariances():
+    q, k, v = _rand(B=2, H=2, T=30, p=4, dv=3, seed=620)
+    o, S, z = ofo.recurrent_linear(q, k, v, return_state=True)
+    # final state closed form: S_T = sum_t k_t v_t^T, z_T = sum_t k_t
+    np.testing.assert_allclose(S, np.einsum("bhtd,bhte->bhde", k, v), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(z, k.sum(axis=2), rtol=1e-12, atol=1e-12)
+    # split and resume from the state after 11 tokens
+    _, S1, z1 = ofo.recurrent_linear(q[:, :, :11], k[:, :, :11], v[:, :, :11], return_state=True)
+    o2 = ofo.recurrent_linear(q[:, :, 11:], k[:, :, 11:], v[:, :, 11:], S0=S1, z0=z1)
+    np.testing.assert_allclose(o2, o[:, :, 11:], rtol=1e-10, atol=1e-12)
+    # o is unchanged by scaling a query, or all keys, by any c != 0 (the
+    # numerator and the denominator scale together), but not by scaling one key
+    for c in (3.0, -0.5):
+        np.testing.assert_allclose(ofo.direct_linear(c * q, k, v), o, rtol=1e-9, atol=1e-11)
+        np.testing.assert_allclose(ofo.direct_linear(q, c * k, v), o, rtol=1e-9, atol=1e-11)
+    k2 = k.copy()
+    k2[:, :, 5] *= 4.0
+    assert np.abs(ofo.direct_linear(q, k2, v) - o)[:, :, 5:].max() > 1e-3
+
+
+MUTATIONS_FO = {
+    "exclusive causal sum": [("np.tril(np.ones((T, T), dtype=bool))", "np.tril(np.ones((T, T), dtype=bool), k=-1)"),
+                             ("    for t in range(T):\n        S += k[:, :, t, :, None] * v[:, :, t, None, :]\n"
+                              "        z += k[:, :, t]\n        N = np.einsum(\"bhd,bhde->bhe\", q[:, :, t], S)\n"
+                              "        D = np.einsum(\"bhd,bhd->bh\", q[:, :, t], z)\n",
+                              "    for t in range(T):\n        N = np.einsum(\"bhd,bhde->bhe\", q[:, :, t], S)\n"
+                              "        D = np.einsum(\"bhd,bhd->bh\", q[:, :, t], z)\n"
+                              "        S += k[:, :, t, :, None] * v[:, :, t, None, :]\n        z += k[:, :, t]\n")],
+    "squared weights": [("W = np.where(np.tril(np.ones((T, T), dtype=bool)), W, 0.0)",
+                         "W = np.where(np.tril(np.ones((T, T), dtype=bool)), W * W, 0.0)"),
+                        ("        z += k[:, :, t]\n", "        z += k[:, :, t] * k[:, :, t]\n")],
+    "no normalisation": [("    return _div(N, W.sum(axis=-1))", "    return N"),
+                         ("        o[:, :, t] = _div(N, D)", "        o[:, :, t] = N")],
+    "query and key swapped": [("\"bhtd,bhsd->bhts\", q, k", "\"bhtd,bhsd->bhts\", k, q"),
+                              ("np.einsum(\"bhd,bhde->bhe\", q[:, :, t], S)", "np.einsum(\"bhd,bhde->bhe\", k[:, :, t], S)")],
+    "negative denominators zeroed": [("    nz = D != 0", "    nz = D > 0")],
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS_FO))
+def test_first_order_pins_catch_planted_mistakes(name):
+    import inspect
+    import types
+    src = inspect.getsource(ofo)
+    for old, new in MUTATIONS_FO[name]:
+        assert src.count(old) == 1, (name, old)
+        src = src.replace(old, new)
+    mutant = types.ModuleType("first_order_mutant")
+    exec(compile(src, "first_order_mutant", "exec"), mutant.__dict__)
+    assert not _fo_pins_hold(mutant), "first-order pin set failed to catch: " + name
