@@ -178,6 +178,48 @@ kata_status_t kata_fwd_chunked_sequential(const void* q, const void* k, const vo
                                           float* S_out, float* z_out, void* stream);
 
 /*
+ * First-order (linear) attention, the feature psi(u) = u: the comparator of
+ * the pages' scan claim ("an associative scan of the first-order feature
+ * lowers the inter-chunk recurrence depth to O(log(T/C)) and averages ~2.4x
+ * the throughput of a matched sequential linear-attention baseline": arXiv
+ * abstract; review page, Figure 3 caption; gist.science sec. 2.3).  For
+ * every (b,h) and t:
+ *   o_t = sum_{s<=t} (q_t . k_s) v_s / sum_{s<=t} (q_t . k_s),
+ * o_t = 0 where the denominator is exactly 0 (it may be negative: the
+ * feature is not sign-constrained).  State: S = S0 + sum_s k_s v_s^T
+ * [d, dv] and z = z0 + sum_s k_s [d].
+ *
+ * kata_fwd_linear_chunked is the chunked form with the associative scan
+ * across super-chunks (state build, scan, readout, as kata_fwd_chunked);
+ * kata_fwd_linear_chunked_sequential is the matched sequential baseline: one
+ * CTA per (b,h) walks all chunks in order, no workspace.  Both run on the
+ * tensor cores and agree up to rounding.
+ *
+ * q, k: [B, H, T, d]; v, o: [B, H, T, dv]; bf16, row-major, 16-byte aligned.
+ * S0/z0 (optional, both or neither) and S_out/z_out (optional, both or
+ * neither): fp32 [B, H, d, dv] / [B, H, d], 16-byte aligned; S_out/z_out
+ * receive the state after token T.  Only d = 16, dv = 64 and
+ * KATA_BF16 are supported (others: KATA_ERR_UNSUPPORTED); C is 64 or 128.
+ * workspace: device memory of at least
+ * kata_fwd_linear_chunked_workspace_size() bytes, 256-byte aligned
+ * (KATA_ERR_WORKSPACE / KATA_ERR_MISALIGNED otherwise; 0 bytes when the
+ * whole sequence fits one super-chunk).  All pointers are owned by the
+ * caller; the calls are asynchronous on `stream`.
+ */
+size_t kata_fwd_linear_chunked_workspace_size(int B, int H, int T, int d, int dv, int C);
+kata_status_t kata_fwd_linear_chunked(const void* q, const void* k, const void* v, void* o,
+                                      int B, int H, int T, int d, int dv, int C,
+                                      kata_dtype_t dtype,
+                                      const float* S0, const float* z0,
+                                      float* S_out, float* z_out,
+                                      void* workspace, size_t workspace_bytes, void* stream);
+kata_status_t kata_fwd_linear_chunked_sequential(const void* q, const void* k, const void* v, void* o,
+                                                 int B, int H, int T, int d, int dv, int C,
+                                                 kata_dtype_t dtype,
+                                                 const float* S0, const float* z0,
+                                                 float* S_out, float* z_out, void* stream);
+
+/*
  * One recurrent decode step for B*H independent streams (constant-time
  * recurrent inference on the fixed-size state; arXiv abstract on aiqbench):
  *   S <- S + psi(k) v^T,  z <- z + psi(k),  o = psi(q)^T S / psi(q)^T z

@@ -31,6 +31,9 @@ SIGNATURES = {
                                           _c_int, _fp, _fp, _fp, _fp, _vp]),
     "kata_fwd_chunked_sequential": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                              _c_int, _fp, _fp, _fp, _fp, _vp]),
+    "kata_fwd_linear_chunked_workspace_size": (_c_size, [_c_int] * 6),
+    "kata_fwd_linear_chunked": (_c_int, [_vp, _vp, _vp, _vp] + [_c_int] * 7 + [_fp, _fp, _fp, _fp, _vp, _c_size, _vp]),
+    "kata_fwd_linear_chunked_sequential": (_c_int, [_vp, _vp, _vp, _vp] + [_c_int] * 7 + [_fp, _fp, _fp, _fp, _vp]),
     "kata_decode_step": (_c_int, [_vp, _vp, _vp, _vp, _fp, _fp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp]),
     "kata_fwd_quadratic_train": (_c_int, [_vp, _vp, _vp, _vp, _fp] + [_c_int] * 6 + [_vp]),
     "kata_bwd_quadratic_workspace_size": (_c_size, [_c_int] * 6),
@@ -198,6 +201,59 @@ def kata_fwd_chunked_sequential(q, k, v, C=64, S0=None, z0=None, return_state=Fa
         z_out = torch.empty((B, H, p * p), dtype=torch.float32, device=dev)
     _check("kata_fwd_chunked_sequential", lib().kata_fwd_chunked_sequential(
         _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), B, H, T, p, dv, C, _dtype_code(q),
+        _opt(S0, "S0"), _opt(z0, "z0"), _opt(S_out, "S_out"), _opt(z_out, "z_out"), _stream_ptr(stream)))
+    if return_state:
+        return o, S_out, z_out
+    return o
+
+
+def kata_fwd_linear_chunked_workspace_size(B, H, T, d, dv, C) -> int:
+    return int(lib().kata_fwd_linear_chunked_workspace_size(B, H, T, d, dv, C))
+
+
+def kata_fwd_linear_chunked(q, k, v, C=64, S0=None, z0=None, return_state=False, o=None, workspace=None,
+                            S_out=None, z_out=None, stream=None):
+    """First-order (psi(u) = u) chunked forward with the associative scan.
+
+    q,k [B,H,T,d], v [B,H,T,dv] (bf16, d=16, dv=64).  Returns o, or
+    (o, S_T, z_T) when return_state is True; S0/z0 ([B,H,d,dv], [B,H,d] fp32)
+    give an initial state.
+    """
+    B, H, T, d = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    if o is None:
+        o = torch.empty((B, H, T, dv), dtype=q.dtype, device=dev)
+    if return_state and S_out is None:
+        S_out = torch.empty((B, H, d, dv), dtype=torch.float32, device=dev)
+        z_out = torch.empty((B, H, d), dtype=torch.float32, device=dev)
+    need = kata_fwd_linear_chunked_workspace_size(B, H, T, d, dv, C)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("kata_fwd_linear_chunked", lib().kata_fwd_linear_chunked(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), B, H, T, d, dv, C, _dtype_code(q),
+        _opt(S0, "S0"), _opt(z0, "z0"), _opt(S_out, "S_out"), _opt(z_out, "z_out"),
+        _opt(workspace, "workspace"), ws_bytes, _stream_ptr(stream)))
+    if return_state:
+        return o, S_out, z_out
+    return o
+
+
+def kata_fwd_linear_chunked_sequential(q, k, v, C=64, S0=None, z0=None, return_state=False, o=None, S_out=None,
+                                       z_out=None, stream=None):
+    """The matched sequential baseline of kata_fwd_linear_chunked: one CTA per
+    (b,h) walks all of its chunks in order (no super-chunk sums, no scan)."""
+    B, H, T, d = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    if o is None:
+        o = torch.empty((B, H, T, dv), dtype=q.dtype, device=dev)
+    if return_state and S_out is None:
+        S_out = torch.empty((B, H, d, dv), dtype=torch.float32, device=dev)
+        z_out = torch.empty((B, H, d), dtype=torch.float32, device=dev)
+    _check("kata_fwd_linear_chunked_sequential", lib().kata_fwd_linear_chunked_sequential(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), B, H, T, d, dv, C, _dtype_code(q),
         _opt(S0, "S0"), _opt(z0, "z0"), _opt(S_out, "S_out"), _opt(z_out, "z_out"), _stream_ptr(stream)))
     if return_state:
         return o, S_out, z_out

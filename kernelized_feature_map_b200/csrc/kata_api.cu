@@ -127,6 +127,17 @@ ChunkPlan make_chunk_plan(int B, int H, int T, int p, int dv, int C, kata_dtype_
   return plan_units(B, H, T, p, dv, C, tc, tc ? cluster_blocks(p, 1) : 1);
 }
 
+ChunkPlan make_linear_plan(int B, int H, int T, int d, int dv, int C) {
+  // the super-chunk split of the tensor-core plan; records in the unpacked
+  // layout (d rows of dv + 4 floats: value columns, then z)
+  ChunkPlan pl = plan_units(B, H, T, d, dv, C, true, 1);
+  pl.P = d;
+  pl.layout = kRecUnpacked;
+  pl.record_floats = (size_t)d * pl.ld;
+  pl.workspace_bytes = pl.G <= 1 ? 0 : (size_t)pl.BH * pl.G * pl.record_floats * sizeof(float);
+  return pl;
+}
+
 ChunkPlan make_cluster_plan(int B, int H, int T, int p, int blocks, int dv, int C) {
   return plan_units(B, H, T, p, dv, C, true, blocks);
 }
@@ -308,6 +319,86 @@ KATA_API kata_status_t kata_fwd_chunked_sequential(const void* q, const void* k,
   plan.workspace_bytes = 0;
   return from_cuda(launch_chunk_readout_sm100(q, k, v, o, nullptr, S0, z0, S_out, z_out, plan, wait_ctl(),
                                               static_cast<cudaStream_t>(stream)));
+}
+
+static kata_status_t check_linear_args(const void* q, const void* k, const void* v, const void* o, int B, int H,
+                                       int T, int d, int dv, int C, kata_dtype_t dtype, const float* S0,
+                                       const float* z0, const float* S_out, const float* z_out) {
+  if (B < 1 || H < 1 || T < 0) return KATA_ERR_INVALID_ARG;
+  if (dtype != KATA_F32 && dtype != KATA_BF16) return KATA_ERR_INVALID_ARG;
+  if (dtype != KATA_BF16 || d != 16 || dv != 64) return KATA_ERR_UNSUPPORTED;
+  if ((long long)T * dv >= (1ll << 31)) return KATA_ERR_UNSUPPORTED;
+  if (!(C == 64 || C == 128)) return KATA_ERR_UNSUPPORTED;
+  if ((S0 == nullptr) != (z0 == nullptr)) return KATA_ERR_INVALID_ARG;
+  if ((S_out == nullptr) != (z_out == nullptr)) return KATA_ERR_INVALID_ARG;
+  for (const void* ptr : {(const void*)S0, (const void*)z0, (const void*)S_out, (const void*)z_out})
+    if (ptr && !aligned16(ptr)) return KATA_ERR_MISALIGNED;
+  if (T == 0) return KATA_OK;
+  if (!q || !k || !v || !o) return KATA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return KATA_ERR_MISALIGNED;
+  return KATA_OK;
+}
+
+// T == 0: the final state is the initial one (or zero)
+static kata_status_t linear_empty(int B, int H, int d, int dv, const float* S0, const float* z0, float* S_out,
+                                  float* z_out, cudaStream_t st) {
+  if (!S_out) return KATA_OK;
+  const size_t BH = (size_t)B * H;
+  cudaError_t e = S0 ? cudaMemcpyAsync(S_out, S0, BH * d * dv * sizeof(float), cudaMemcpyDeviceToDevice, st)
+                     : cudaMemsetAsync(S_out, 0, BH * d * dv * sizeof(float), st);
+  if (e == cudaSuccess)
+    e = S0 ? cudaMemcpyAsync(z_out, z0, BH * d * sizeof(float), cudaMemcpyDeviceToDevice, st)
+           : cudaMemsetAsync(z_out, 0, BH * d * sizeof(float), st);
+  return from_cuda(e);
+}
+
+KATA_API size_t kata_fwd_linear_chunked_workspace_size(int B, int H, int T, int d, int dv, int C) {
+  if (B < 1 || H < 1 || T <= 0 || d != 16 || dv != 64 || !(C == 64 || C == 128)) return 0;
+  return make_linear_plan(B, H, T, d, dv, C).workspace_bytes;
+}
+
+KATA_API kata_status_t kata_fwd_linear_chunked(const void* q, const void* k, const void* v, void* o, int B, int H,
+                                               int T, int d, int dv, int C, kata_dtype_t dtype, const float* S0,
+                                               const float* z0, float* S_out, float* z_out, void* workspace,
+                                               size_t workspace_bytes, void* stream) {
+  kata_status_t s = check_linear_args(q, k, v, o, B, H, T, d, dv, C, dtype, S0, z0, S_out, z_out);
+  if (s != KATA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (T == 0) return linear_empty(B, H, d, dv, S0, z0, S_out, z_out, st);
+  const ChunkPlan plan = make_linear_plan(B, H, T, d, dv, C);
+  if (plan.workspace_bytes > 0) {
+    if (!workspace || workspace_bytes < plan.workspace_bytes) return KATA_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KATA_ERR_MISALIGNED;
+  }
+  float* ws = plan.workspace_bytes > 0 ? static_cast<float*>(workspace) : nullptr;
+  const WaitCtl wc = wait_ctl();
+  // sums of super-chunks 0..G-2, their scan (which adds S0), the readout
+  cudaError_t e = cudaSuccess;
+  if (plan.G > 1) {
+    e = launch_linear_state_sm100(k, v, ws, plan, wc, st);
+    if (e == cudaSuccess) e = launch_state_scan(ws, plan, plan.G - 1, S0, z0, nullptr, nullptr, st);
+  }
+  if (e == cudaSuccess)
+    e = launch_linear_readout_sm100(q, k, v, o, ws, plan.G > 1 ? nullptr : S0, plan.G > 1 ? nullptr : z0, S_out,
+                                    z_out, plan, wc, st);
+  return from_cuda(e);
+}
+
+KATA_API kata_status_t kata_fwd_linear_chunked_sequential(const void* q, const void* k, const void* v, void* o,
+                                                          int B, int H, int T, int d, int dv, int C,
+                                                          kata_dtype_t dtype, const float* S0, const float* z0,
+                                                          float* S_out, float* z_out, void* stream) {
+  kata_status_t s = check_linear_args(q, k, v, o, B, H, T, d, dv, C, dtype, S0, z0, S_out, z_out);
+  if (s != KATA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (T == 0) return linear_empty(B, H, d, dv, S0, z0, S_out, z_out, st);
+  // one super-chunk per (b,h): one CTA walks every chunk of its sequence in
+  // order, carrying the state; no state build, no scan, no workspace
+  ChunkPlan plan = make_linear_plan(B, H, T, d, dv, C);
+  plan.Ls = ((T + 127) / 128) * 128;
+  plan.G = 1;
+  plan.workspace_bytes = 0;
+  return from_cuda(launch_linear_readout_sm100(q, k, v, o, nullptr, S0, z0, S_out, z_out, plan, wait_ctl(), st));
 }
 
 KATA_API kata_status_t kata_decode_step(const void* q, const void* k, const void* v, void* o, float* S, float* z,

@@ -115,6 +115,17 @@ cudaError_t launch_chunk_readout_sm100(const void* q, const void* k, const void*
                                        const float* S0, const float* z0, float* S_out, float* z_out,
                                        const ChunkPlan& pl, const WaitCtl& wc, cudaStream_t st);
 
+// chunk_linear_sm100.cu -- first-order (linear) attention, psi(u) = u, with
+// d = 16 and dv = 64 in bf16: the same three steps with unpacked records
+// (make_linear_plan), the state entering each super-chunk from the scan (or
+// S0/z0 when G == 1), the final state written by the last readout.
+ChunkPlan make_linear_plan(int B, int H, int T, int d, int dv, int C);
+cudaError_t launch_linear_state_sm100(const void* k, const void* v, float* ws, const ChunkPlan& pl, const WaitCtl& wc,
+                                      cudaStream_t st);
+cudaError_t launch_linear_readout_sm100(const void* q, const void* k, const void* v, void* o, const float* ws,
+                                        const float* S0, const float* z0, float* S_out, float* z_out,
+                                        const ChunkPlan& pl, const WaitCtl& wc, cudaStream_t st);
+
 // chunk_cluster_sm100.cu -- the same with the packed state split over the
 // CTAs of a cluster: p = 32 (groups = 1: four blocks) and KATA-Mg over d = 64
 // (groups = 2 of p = 32: eight blocks; groups = 4 of p = 16: four blocks);

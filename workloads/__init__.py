@@ -87,6 +87,18 @@ def normal_qkv(B, H, T, p, dv, seed=0, dtype="bf16"):
     return _cast(q, dtype), _cast(k, dtype), _cast(v, dtype)
 
 
+def nonneg_qkv(B, H, T, p, dv, seed=0, dtype="bf16"):
+    """q, k = |N(0,1)| per coordinate, L2-normalised per token (nonnegative
+    unit vectors, so every q_t . k_s >= 0); v ~ N(0,1).  Inputs for the
+    first-order feature, whose denominators are only sign-definite on such
+    inputs.  Returns float32 arrays."""
+    rng = np.random.default_rng(seed)
+    q = _l2n(np.abs(rng.standard_normal((B, H, T, p), dtype=np.float32)))
+    k = _l2n(np.abs(rng.standard_normal((B, H, T, p), dtype=np.float32)))
+    v = rng.standard_normal((B, H, T, dv), dtype=np.float32)
+    return _cast(q, dtype), _cast(k, dtype), _cast(v, dtype)
+
+
 def recall_qkv(B, H, T, p, dv, seed=0, dtype="bf16", code_size=512, sigma=0.05):
     """Recall-shaped keys (overwrite pattern) and noisy-copy queries."""
     rng = np.random.default_rng(seed)
