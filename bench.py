@@ -395,6 +395,9 @@ def run_ours(args, rank, world, local_rank):
                 t0 = time.time()
                 long["mg"] = run_mg(args, K, torch, dev, stream, flush)
                 windows["mg"] = (t0, time.time())
+                t0 = time.time()
+                long["first_order"] = run_first_order(args, K, torch, dev, stream, flush)
+                windows["first_order"] = (t0, time.time())
                 long["train"] = run_train(args, K, torch, dev, stream, flush)
         t_end = time.time()
         time.sleep(0.15)
@@ -544,6 +547,35 @@ def run_sweep(args, K, torch, dev, stream, flush):
                                         stream, 3, 1),
                   quadratic_ms=_time_call(lambda: K.kata_fwd_quadratic(q, k, v, o=o), flush, stream, 3, 1))
     return grid, recall
+
+
+def run_first_order(args, K, torch, dev, stream, flush):
+    """First-order attention (psi(u) = u, d=16, dv=64, H=16, bf16): the
+    chunked form with the associative scan against the matched sequential
+    baseline (one CTA per sequence) over a batch x length grid, the pages'
+    Figure 3 comparison.  Inputs are drawn on the device: q, k nonnegative
+    unit vectors (|N(0,1)| normalised), v N(0,1)."""
+    bf = torch.bfloat16
+    H, d, dv, C = 16, 16, 64, 64
+    gen = torch.Generator(device=dev)
+    grid = []
+    for B in (1, 4, 16):
+        for T in (2048, 8192, 32768, 131072):
+            gen.manual_seed(2000 * B + T % 991)
+            q = torch.randn((B, H, T, d), generator=gen, device=dev).abs()
+            k = torch.randn((B, H, T, d), generator=gen, device=dev).abs()
+            q = (q / q.norm(dim=-1, keepdim=True)).to(bf)
+            k = (k / k.norm(dim=-1, keepdim=True)).to(bf)
+            v = torch.randn((B, H, T, dv), generator=gen, device=dev).to(bf)
+            o = torch.empty((B, H, T, dv), dtype=bf, device=dev)
+            ws = torch.empty(max(256, K.kata_fwd_linear_chunked_workspace_size(B, H, T, d, dv, C)),
+                             dtype=torch.uint8, device=dev)
+            s_ms = _time_call(lambda: K.kata_fwd_linear_chunked(q, k, v, C=C, o=o, workspace=ws), flush, stream, 3, 1)
+            q_ms = _time_call(lambda: K.kata_fwd_linear_chunked_sequential(q, k, v, C=C, o=o), flush, stream, 3, 1)
+            grid.append(dict(B=B, H=H, T=T, d=d, dv=dv, scan_ms=s_ms, sequential_ms=q_ms))
+            del q, k, v, o, ws
+    torch.cuda.empty_cache()
+    return grid
 
 
 def run_mg(args, K, torch, dev, stream, flush):
@@ -728,6 +760,14 @@ def run_case(args):
             raise SystemExit("--layout bthd is for --case mg")
         elif args.case == "quadratic":
             call = lambda: K.kata_fwd_quadratic(q, k, v, o=o)  # noqa: E731
+        elif args.case == "linear":
+            q, k = q.abs(), k.abs()  # nonnegative unit vectors: sign-definite denominators
+            ws = torch.empty(max(256, K.kata_fwd_linear_chunked_workspace_size(B, H, T, d, dv, args.C)),
+                             dtype=torch.uint8, device=dev)
+            call = lambda: K.kata_fwd_linear_chunked(q, k, v, C=args.C, o=o, workspace=ws)  # noqa: E731
+        elif args.case == "linear_sequential":
+            q, k = q.abs(), k.abs()
+            call = lambda: K.kata_fwd_linear_chunked_sequential(q, k, v, C=args.C, o=o)  # noqa: E731
         elif args.case == "train":
             dO = torch.randn(v.shape, generator=gen, device=dev).to(bf)
             D = torch.empty((B, H, T), dtype=torch.float32, device=dev)
@@ -773,7 +813,8 @@ def main():
     ap.add_argument("--graph", type=int, default=1, help="time the step as a CUDA graph replay (per-path times stay eager)")
     ap.add_argument("--ref-budget", type=float, default=15.0, help="seconds of oracle work per reference step")
     pc = ap.add_argument_group("--case: launch one call a few times on device-drawn inputs (for profilers)")
-    pc.add_argument("--case", choices=["quadratic", "chunked", "mg", "mg_chunked", "decode", "train"])
+    pc.add_argument("--case", choices=["quadratic", "chunked", "mg", "mg_chunked", "decode", "train", "linear",
+                                       "linear_sequential"])
     pc.add_argument("--B", type=int, default=8)
     pc.add_argument("--H", type=int, default=16)
     pc.add_argument("--T", type=int, default=2048)
@@ -874,6 +915,16 @@ def roofline_points(res, peaks, cfg):
                 pts.append(tensor_point("mg_quadratic", wl, m["ms"], m["B"] * m["T"],
                                         flash_flops(m["B"] * m["H"], m["T"], m["d"], m["dv"]), cl.get("mg"),
                                         T=m["T"], groups=m["groups"]))
+        # first-order attention at B1 H16 T131072: both forms
+        for g in lg.get("first_order", []):
+            if g["B"] != 1 or g["T"] != 131072:
+                continue
+            wl = "first-order psi(u)=u B=%d H=%d T=%d d=%d dv=%d bf16" % (g["B"], g["H"], g["T"], g["d"], g["dv"])
+            nbytes = g["B"] * g["H"] * g["T"] * (2 * g["d"] + 2 * g["dv"]) * 2
+            pts.append(hbm_point("first_order_scan", wl, g["scan_ms"], g["B"] * g["T"], nbytes,
+                                 cl.get("first_order"), T=g["T"]))
+            pts.append(hbm_point("first_order_sequential", wl, g["sequential_ms"], g["B"] * g["T"], nbytes,
+                                 cl.get("first_order"), T=g["T"]))
     return pts
 
 
@@ -982,6 +1033,22 @@ def report(args, res, step_ms, e2e_ms, world):
                         "ms": m["ms"], "tokens_per_s": m["B"] * m["T"] / (m["ms"] * 1e-3),
                         "tensor_frac": flash_flops(m["B"] * m["H"], m["T"], width, m["dv"]) / (m["ms"] * 1e-3)
                         / 1e12 / peaks["bf16_tflops"]}
+        if "first_order" in lg:
+            hb = peaks["hbm_gbs"]
+            pts = []
+            for g in lg["first_order"]:
+                nbytes = g["B"] * g["H"] * g["T"] * (2 * g["d"] + 2 * g["dv"]) * 2
+                pts.append({"B": g["B"], "T": g["T"], "scan_ms": g["scan_ms"], "sequential_ms": g["sequential_ms"],
+                            "scan_tokens_per_s": g["B"] * g["T"] / (g["scan_ms"] * 1e-3),
+                            "sequential_tokens_per_s": g["B"] * g["T"] / (g["sequential_ms"] * 1e-3),
+                            "scan_speedup": g["sequential_ms"] / g["scan_ms"],
+                            "scan_hbm_frac": nbytes / (g["scan_ms"] * 1e-3) / 1e9 / hb})
+            sp = np.array([x["scan_speedup"] for x in pts])
+            line["first_order"] = {
+                "workload": "first-order attention psi(u)=u, H=16 d=16 dv=64 bf16, chunked with the associative scan "
+                            "vs the sequential baseline, B x T grid",
+                "grid": pts, "scan_speedup_mean": float(sp.mean()),
+                "scan_speedup_geomean": float(np.exp(np.log(sp).mean()))}
         if "train" in lg:
             tr = lg["train"]
             pairs = tr["B"] * tr["H"] * tr["T"] * (tr["T"] + 1) / 2

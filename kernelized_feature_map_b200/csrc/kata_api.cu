@@ -128,9 +128,22 @@ ChunkPlan make_chunk_plan(int B, int H, int T, int p, int dv, int C, kata_dtype_
 }
 
 ChunkPlan make_linear_plan(int B, int H, int T, int d, int dv, int C) {
-  // the super-chunk split of the tensor-core plan; records in the unpacked
-  // layout (d rows of dv + 4 floats: value columns, then z)
+  // The first-order kernels are bound by HBM, not by the per-chunk work of
+  // the KATA ones: once every SM has a sequence, the readout alone streams
+  // at the HBM rate and a split only adds the state pass's k, v reads.  So
+  // one super-chunk per (b,h) when the sequences fill the SMs, otherwise
+  // enough super-chunks for one wave.  Measured at H16 T131072: B16 one
+  // super-chunk 1814 us against 2245 us with the split of plan_units (4);
+  // B1 nine super-chunks 163.5 us against 862.5 us for one.  Records in the
+  // unpacked layout (d rows of dv + 4 floats: value columns, then z).
   ChunkPlan pl = plan_units(B, H, T, d, dv, C, true, 1);
+  const long long tiles = (T + 127) / 128;
+  long long G = pl.BH * 10 >= (long long)kSMs * 9 ? 1 : kSMs / pl.BH;
+  if (G > tiles) G = tiles;
+  if (G < 1) G = 1;
+  pl.Ls = (int)(((tiles + G - 1) / G) * 128);
+  if (pl.Ls < C) pl.Ls = C;
+  pl.G = T > 0 ? (T + pl.Ls - 1) / pl.Ls : 0;
   pl.P = d;
   pl.layout = kRecUnpacked;
   pl.record_floats = (size_t)d * pl.ld;
