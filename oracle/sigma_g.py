@@ -10,7 +10,8 @@ u = [u^1 | ... | u^g], and the feature is the SUM of the group maps,
 with one value vector and one denominator (arXiv abstract and gist.science
 sec. 2.3 "Varianten": KATA-Sigma-g, summed PSD factors; ai.info summary, Main
 Findings: state (d/g)(d/g+1)/2 * dv, the full map at g = 1).  Two forms: the
-defining double sum, and the recurrence on the explicit p^2 feature.
+defining double sum, and the recurrence on the explicit p^2 feature; and one
+step of that recurrence from a given state (decode).
 """
 from __future__ import annotations
 
@@ -63,3 +64,19 @@ def recurrent_sg(q, k, v, groups: int):
         safe = np.where(den > 0, den, 1.0)
         o[:, :, t] = np.where((den > 0)[..., None], num / safe[..., None], 0.0)
     return o
+
+
+def decode_step_sg(q, k, v, S, z, groups: int):
+    """One recurrent step on the summed-feature state: S' = S + psi_S(k) v^T,
+    z' = z + psi_S(k), o = psi_S(q)^T S' / psi_S(q)^T z' (0 where that is 0).
+
+    q, k [B,H,d]; v [B,H,dv]; S [B,H,p*p,dv], z [B,H,p*p] with p = d/groups
+    (row a*p + b holds sum_j u^j_a u^j_b).  Returns (o, S', z')."""
+    fq, fk = features_sg(q, groups), features_sg(k, groups)
+    v = np.asarray(v, np.float64)
+    S2 = np.asarray(S, np.float64) + fk[..., :, None] * v[..., None, :]
+    z2 = np.asarray(z, np.float64) + fk
+    num = np.einsum("bhp,bhpe->bhe", fq, S2)
+    den = np.einsum("bhp,bhp->bh", fq, z2)
+    safe = np.where(den > 0, den, 1.0)
+    return np.where((den > 0)[..., None], num / safe[..., None], 0.0), S2, z2

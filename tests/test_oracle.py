@@ -661,3 +661,27 @@ def test_first_order_pins_catch_planted_mistakes(name):
     mutant = types.ModuleType("first_order_mutant")
     exec(compile(src, "first_order_mutant", "exec"), mutant.__dict__)
     assert not _fo_pins_hold(mutant), "first-order pin set failed to catch: " + name
+
+
+def test_sigma_g_decode_step_pins():
+    """One decode step from the state after tokens 0..t-1 gives the
+    recurrence's output at token t and its state after t; g = 1 is the C
+    oracle's single-factor step."""
+    q, k, v = _rand_mg(B=2, H=2, T=9, d=8, dv=3, seed=520)
+    for g in (2, 4):
+        p = 8 // g
+        fk = osg.features_sg(k, g)
+        S = np.einsum("bhtp,bhte->bhpe", fk[:, :, :8], v[:, :, :8])
+        z = fk[:, :, :8].sum(axis=2)
+        o, S2, z2 = osg.decode_step_sg(q[:, :, 8], k[:, :, 8], v[:, :, 8], S, z, g)
+        np.testing.assert_allclose(o, osg.recurrent_sg(q, k, v, g)[:, :, 8], rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(S2, np.einsum("bhtp,bhte->bhpe", fk, v), rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(z2, fk.sum(axis=2), rtol=1e-12, atol=1e-12)
+        assert S2.shape == (2, 2, p * p, 3)
+    rng = np.random.default_rng(521)
+    S = rng.standard_normal((2, 2, 64, 3))
+    z = np.abs(rng.standard_normal((2, 2, 64))) + 1.0
+    o1, S1, z1 = osg.decode_step_sg(q[:, :, 0], k[:, :, 0], v[:, :, 0], S, z, 1)
+    o2, S2, z2 = oracle.decode_step(q[:, :, 0], k[:, :, 0], v[:, :, 0], S, z)
+    np.testing.assert_allclose(o1, o2, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(S1, S2, rtol=1e-12, atol=1e-12)
