@@ -637,7 +637,13 @@ def run_mg(args, K, torch, dev, stream, flush):
         o = torch.empty((B, H, dv), dtype=bf, device=dev)
         ms = _time_call(lambda: K.kata_decode_step_mg(q, k, v, S, z, g, o=o), flush, stream, 20, 3)
         out["decode_mg%d_b64" % g] = dict(B=B, H=H, d=d, groups=g, dv=dv, P=P, ms=ms)
-        del q, k, v, S, z, o
+        # KATA-Sigma-g: the summed feature's state has the single factor's
+        # (d/g)^2 rows
+        Ps = (d // g) ** 2
+        Ss, zs = S[:, :, :Ps].contiguous(), z[:, :, :Ps].contiguous()
+        ms = _time_call(lambda: K.kata_decode_step_sg(q, k, v, Ss, zs, g, o=o), flush, stream, 20, 3)
+        out["decode_sg%d_b64" % g] = dict(B=B, H=H, d=d, groups=g, dv=dv, P=Ps, ms=ms, summed=True)
+        del q, k, v, S, z, o, Ss, zs
     return out
 
 
@@ -1008,8 +1014,9 @@ def report(args, res, step_ms, e2e_ms, world):
                 if "P" in m:  # decode step
                     mb = 2 * m["B"] * m["H"] * (m["P"] * m["dv"] + m["P"]) * 4
                     line["mg"][name] = {
-                        "workload": "KATA-Mg decode step B=%d H=%d d=%d groups=%d state [%d x %d] fp32" % (
-                            m["B"], m["H"], m["d"], m["groups"], m["P"], m["dv"]),
+                        "workload": "%s decode step B=%d H=%d d=%d groups=%d state [%d x %d] fp32" % (
+                            "KATA-Sigma-g" if m.get("summed") else "KATA-Mg", m["B"], m["H"], m["d"], m["groups"],
+                            m["P"], m["dv"]),
                         "ms": m["ms"], "tokens_per_s": m["B"] / (m["ms"] * 1e-3),
                         "hbm_frac": mb / (m["ms"] * 1e-3) / 1e9 / peaks["hbm_gbs"]}
                 elif m.get("chunked"):

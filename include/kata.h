@@ -363,6 +363,19 @@ kata_status_t kata_decode_step_mg(const void* q, const void* k, const void* v, v
                                   kata_dtype_t dtype, void* stream);
 
 /*
+ * One KATA-Sigma-g decode step (update with (k, v), then read with q) on
+ * the summed-feature state: psi_S(u) = sum_j vec(u^j u^j^T), so the state
+ * has the single factor's size: S [B,H,p*p,dv] and z [B,H,p*p] fp32
+ * (p = d/groups), read and updated in place, row r = a*p + b holding
+ * sum_j u^j_a u^j_b.  q, k: [B,H,d]; v, o: [B,H,dv] (fp32 or bf16).
+ * Supported (p, groups, dv) as for kata_fwd_sg_quadratic; groups = 1 is
+ * kata_decode_step.  Errors as for kata_decode_step_mg.
+ */
+kata_status_t kata_decode_step_sg(const void* q, const void* k, const void* v, void* o,
+                                  float* S, float* z, int B, int H, int d, int groups, int dv,
+                                  kata_dtype_t dtype, void* stream);
+
+/*
  * Synchronises `stream`, then returns and clears the device-side status word
  * of the current device (KATA_ERR_TIMEOUT if a bounded wait in a kernel ran
  * out since the last call), or KATA_ERR_CUDA if the stream reports an error.

@@ -45,6 +45,7 @@ SIGNATURES = {
     "kata_fwd_mg_chunked": (_c_int, [_vp, _vp, _vp, _vp] + [_c_int] * 9 + [_fp, _fp, _fp, _fp, _vp, _c_size, _vp]),
     "kata_bwd_mg_quadratic": (_c_int, [_vp] * 9 + [_c_int] * 7 + [_vp, _c_size, _vp]),
     "kata_decode_step_mg": (_c_int, [_vp, _vp, _vp, _vp, _fp, _fp] + [_c_int] * 6 + [_vp]),
+    "kata_decode_step_sg": (_c_int, [_vp, _vp, _vp, _vp, _fp, _fp] + [_c_int] * 6 + [_vp]),
     "kata_get_status": (_c_int, [_vp]),
     "kata_status_string": (ctypes.c_char_p, [_c_int]),
     "kata_set_wait_limit": (None, [ctypes.c_longlong]),
@@ -488,6 +489,20 @@ def kata_decode_step_mg(q, k, v, S, z, groups, o=None, stream=None):
     if o is None:
         o = torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
     _check("kata_decode_step_mg", lib().kata_decode_step_mg(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), _dev(S, "S"), _dev(z, "z"), B, H, d, int(groups),
+        dv, _dtype_code(q), _stream_ptr(stream)))
+    return o
+
+
+def kata_decode_step_sg(q, k, v, S, z, groups, o=None, stream=None):
+    """One KATA-Sigma-g decode step: q,k [B,H,d], v [B,H,dv]; S [B,H,p*p,dv]
+    and z [B,H,p*p] (fp32, p = d/groups, the summed feature's state) are
+    updated in place."""
+    B, H, d = q.shape
+    dv = v.shape[-1]
+    if o is None:
+        o = torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
+    _check("kata_decode_step_sg", lib().kata_decode_step_sg(
         _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), _dev(S, "S"), _dev(z, "z"), B, H, d, int(groups),
         dv, _dtype_code(q), _stream_ptr(stream)))
     return o

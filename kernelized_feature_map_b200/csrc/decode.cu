@@ -21,6 +21,10 @@
 // the feature is the concatenation of the G group maps, so the state has
 // G*p*p rows and row r = g*p*p + i*p + j holds the products of coordinates
 // g*p + i and g*p + j; G = 1 is the single-factor step above.
+// KATA-Sigma-g (SUM): the feature is the sum of the G group maps, so the
+// state has the single factor's p*p rows and row r = i*p + j holds
+// sum_g u_{g*p+i} u_{g*p+j} (gist.science sec. 2.3 "Varianten"; ai.info Main
+// Findings, the Sigma-g state (d/g)(d/g+1)/2 * dv, here unpacked).
 #include "kata_common.cuh"
 #include "kata_internal.h"
 
@@ -46,12 +50,32 @@ struct DecodeCfg {
   static constexpr int kMinBlocks = kSmall ? 7 : 1;
 };
 
-template <typename Tin, int p, int DV, int G>
-__global__ void __launch_bounds__((DecodeCfg<G * p * p, DV>::kThreads), (DecodeCfg<G * p * p, DV>::kMinBlocks))
+template <int p, int G, bool SUM>
+constexpr int decode_rows() { return SUM ? p * p : G * p * p; }
+
+// psi_r(u) for state row r of the concatenated (Mg) or summed (Sigma-g)
+// feature, from the row u staged in shared memory
+template <int p, int G, bool SUM>
+__device__ __forceinline__ float decode_feature(const float* u, int r) {
+  if constexpr (SUM) {
+    const int i = r / p, j = r % p;
+    float f = 0.f;
+#pragma unroll
+    for (int g = 0; g < G; ++g) f = fmaf(u[g * p + i], u[g * p + j], f);
+    return f;
+  } else {
+    const int gp = (r / (p * p)) * p, ii = gp + (r % (p * p)) / p, jj = gp + r % p;
+    return u[ii] * u[jj];
+  }
+}
+
+template <typename Tin, int p, int DV, int G, bool SUM>
+__global__ void __launch_bounds__((DecodeCfg<decode_rows<p, G, SUM>(), DV>::kThreads),
+                                  (DecodeCfg<decode_rows<p, G, SUM>(), DV>::kMinBlocks))
     decode_step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
                        Tin* __restrict__ o, float* __restrict__ S, float* __restrict__ z) {
-  constexpr int D = G * p;          // q/k row width
-  constexpr int P = G * p * p;      // state rows
+  constexpr int D = G * p;                       // q/k row width
+  constexpr int P = decode_rows<p, G, SUM>();    // state rows
   constexpr int NT = DecodeCfg<P, DV>::kThreads;
   constexpr int CG = DV / 4;        // 16-byte column groups per state row
   constexpr int RPP = NT / CG;      // rows covered by one pass of the CTA
@@ -103,9 +127,8 @@ __global__ void __launch_bounds__((DecodeCfg<G * p * p, DV>::kThreads), (DecodeC
 #pragma unroll
     for (int i = 0; i < BATCH; ++i) {
       const int r = r0 + (b0 + i) * RPP;
-      const int gp = (r / (p * p)) * p, ii = gp + (r % (p * p)) / p, jj = gp + r % p;
-      const float pk = sk[ii] * sk[jj];
-      const float pq = sq[ii] * sq[jj];
+      const float pk = decode_feature<p, G, SUM>(sk, r);
+      const float pq = decode_feature<p, G, SUM>(sq, r);
       s[i].x = fmaf(pk, vv.x, s[i].x);
       s[i].y = fmaf(pk, vv.y, s[i].y);
       s[i].z = fmaf(pk, vv.z, s[i].z);
@@ -128,10 +151,9 @@ __global__ void __launch_bounds__((DecodeCfg<G * p * p, DV>::kThreads), (DecodeC
   for (int u = 0; u < ZPT; ++u) {
     const int r = tid + NT * u;
     if (r < P) {
-      const int gp = (r / (p * p)) * p, ii = gp + (r % (p * p)) / p, jj = gp + r % p;
-      const float zn = zz[u] + sk[ii] * sk[jj];
+      const float zn = zz[u] + decode_feature<p, G, SUM>(sk, r);
       __stcs(zb + r, zn);
-      den = fmaf(sq[ii] * sq[jj], zn, den);
+      den = fmaf(decode_feature<p, G, SUM>(sq, r), zn, den);
     }
   }
 #pragma unroll
@@ -155,10 +177,10 @@ __global__ void __launch_bounds__((DecodeCfg<G * p * p, DV>::kThreads), (DecodeC
   }
 }
 
-template <typename Tin, int p, int DV, int G>
+template <typename Tin, int p, int DV, int G, bool SUM = false>
 static cudaError_t launch_decode_t(const void* q, const void* k, const void* v, void* o, float* S, float* z,
                                    int BH, cudaStream_t st) {
-  decode_step_kernel<Tin, p, DV, G><<<BH, DecodeCfg<G * p * p, DV>::kThreads, 0, st>>>(
+  decode_step_kernel<Tin, p, DV, G, SUM><<<BH, DecodeCfg<decode_rows<p, G, SUM>(), DV>::kThreads, 0, st>>>(
       (const Tin*)q, (const Tin*)k, (const Tin*)v, (Tin*)o, S, z);
   return cudaGetLastError();
 }
@@ -183,6 +205,23 @@ cudaError_t launch_decode(const void* q, const void* k, const void* v, void* o, 
                           int p, int groups, int dv, kata_dtype_t dt, cudaStream_t st) {
   if (dt == KATA_BF16) return launch_decode_dt<__nv_bfloat16>(q, k, v, o, S, z, BH, p, groups, dv, st);
   return launch_decode_dt<float>(q, k, v, o, S, z, BH, p, groups, dv, st);
+}
+
+template <typename Tin>
+static cudaError_t launch_decode_sg_dt(const void* q, const void* k, const void* v, void* o, float* S, float* z,
+                                       int BH, int p, int groups, int dv, cudaStream_t st) {
+  if (dv == 64) {
+    if (p == 16 && groups == 2) return launch_decode_t<Tin, 16, 64, 2, true>(q, k, v, o, S, z, BH, st);
+    if (p == 16 && groups == 4) return launch_decode_t<Tin, 16, 64, 4, true>(q, k, v, o, S, z, BH, st);
+    if (p == 32 && groups == 2) return launch_decode_t<Tin, 32, 64, 2, true>(q, k, v, o, S, z, BH, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_decode_sg(const void* q, const void* k, const void* v, void* o, float* S, float* z, int BH,
+                             int p, int groups, int dv, kata_dtype_t dt, cudaStream_t st) {
+  if (dt == KATA_BF16) return launch_decode_sg_dt<__nv_bfloat16>(q, k, v, o, S, z, BH, p, groups, dv, st);
+  return launch_decode_sg_dt<float>(q, k, v, o, S, z, BH, p, groups, dv, st);
 }
 
 }  // namespace kata

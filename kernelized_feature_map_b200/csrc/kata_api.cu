@@ -611,6 +611,20 @@ KATA_API kata_status_t kata_bwd_mg_quadratic(const void* q, const void* k, const
   return KATA_OK;
 }
 
+KATA_API kata_status_t kata_decode_step_sg(const void* q, const void* k, const void* v, void* o, float* S, float* z,
+                                           int B, int H, int d, int groups, int dv, kata_dtype_t dtype,
+                                           void* stream) {
+  int p = 0;
+  kata_status_t s = check_mg(B, H, 1, d, groups, dv, dtype, &p);
+  if (s != KATA_OK) return s;
+  if (groups == 1) return kata_decode_step(q, k, v, o, S, z, B, H, p, dv, dtype, stream);
+  if (!q || !k || !v || !o || !S || !z) return KATA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(S) || !aligned16(z))
+    return KATA_ERR_MISALIGNED;
+  return from_cuda(
+      launch_decode_sg(q, k, v, o, S, z, B * H, p, groups, dv, dtype, static_cast<cudaStream_t>(stream)));
+}
+
 KATA_API kata_status_t kata_decode_step_mg(const void* q, const void* k, const void* v, void* o, float* S, float* z,
                                            int B, int H, int d, int groups, int dv, kata_dtype_t dtype,
                                            void* stream) {

@@ -59,6 +59,9 @@ kata_status_t check_chunked_args(const void* q, const void* k, const void* v, co
 // decode.cu -- `groups` PSD factors of width p per head (1: the single-factor step)
 cudaError_t launch_decode(const void* q, const void* k, const void* v, void* o, float* S, float* z,
                           int BH, int p, int groups, int dv, kata_dtype_t dt, cudaStream_t st);
+// the same with the summed (KATA-Sigma-g) feature: p*p state rows
+cudaError_t launch_decode_sg(const void* q, const void* k, const void* v, void* o, float* S, float* z,
+                             int BH, int p, int groups, int dv, kata_dtype_t dt, cudaStream_t st);
 
 // scan.cu -- exclusive prefix over the G records of every (b,h), in place,
 // plus S0 and the final state.  Records g >= G_in hold no data (treated as

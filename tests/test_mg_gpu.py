@@ -285,3 +285,50 @@ def test_mg_chunked_agrees_with_flash(kata):
     a = _run_mg_chunked(kata, q, k, v, g, "bhtd")
     b = _run_mg(kata, q, k, v, g, "bhtd")
     assert row_rel_err(a, b.astype(np.float64), v) <= 2 * TOL["bf16"]
+
+
+# ---------------------------------------------------------------------------
+# KATA-Sigma-g decode: one step on the summed-feature state [p*p, dv]
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dtype,d,g,B,H", [
+    (dt, d, g, 5, 3) for dt in ("f32", "bf16") for d, g in ((64, 4), (64, 2), (32, 2))
+] + [("bf16", 64, 4, 64, 16)])  # and the serving shape, B64 H16
+def test_sg_decode_step(kata, dtype, d, g, B, H):
+    """Against the fp64 Sigma-g step: the state element by element, the
+    output with the per-row metric.  The starting state is random with the
+    structure of a real one (symmetric S, positive-definite z, so the
+    denominator is positive: <psi_S(q), z> with both PSD)."""
+    import torch
+    from oracle import sigma_g as osg
+    p, dv = d // g, 64
+    q, k, v = (x[:, :, 0] for x in workloads.normal_qkv(B, H, 1, d, dv, seed=400 + d + g, dtype=dtype))
+    _, _, _, S, z = workloads.decode_inputs(B, H, p, dv, seed=410 + d + g, dtype=dtype)
+    o_ref, S_ref, z_ref = osg.decode_step_sg(q, k, v, S, z, g)
+    Sd, zd = torch.from_numpy(S).cuda(), torch.from_numpy(z).cuda()
+    o = kata.kata_decode_step_sg(to_dev(q, dtype), to_dev(k, dtype), to_dev(v, dtype), Sd, zd, g)
+    torch.cuda.synchronize()
+    assert kata.kata_get_status() == 0
+    np.testing.assert_allclose(Sd.cpu().numpy(), S_ref, rtol=1e-6, atol=1e-5)
+    np.testing.assert_allclose(zd.cpu().numpy(), z_ref, rtol=1e-6, atol=1e-5)
+    err = row_rel_err(to_np(o)[:, :, None], o_ref[:, :, None], v[:, :, None])
+    assert err <= TOL[dtype], err
+
+
+def test_sg_decode_continues_the_forward(kata):
+    """Decode steps from the Sigma-g oracle's state after T tokens reproduce
+    the flash Sigma-g forward's outputs for the next tokens."""
+    import torch
+    from oracle import sigma_g as osg
+    B, H, T, d, g, dv = 2, 2, 150, 64, 4, 64
+    q, k, v = workloads.normal_qkv(B, H, T + 3, d, dv, seed=420, dtype="bf16")
+    o_fwd = to_np(kata.kata_fwd_sg_quadratic(to_dev(q, "bf16"), to_dev(k, "bf16"), to_dev(v, "bf16"), g))
+    fk = osg.features_sg(k[:, :, :T], g)
+    Sd = torch.from_numpy(np.einsum("bhtp,bhte->bhpe", fk, v[:, :, :T].astype(np.float64)).astype(np.float32)).cuda()
+    zd = torch.from_numpy(fk.sum(axis=2).astype(np.float32)).cuda()
+    outs = []
+    for t in range(T, T + 3):
+        outs.append(to_np(kata.kata_decode_step_sg(to_dev(q[:, :, t], "bf16"), to_dev(k[:, :, t], "bf16"),
+                                                   to_dev(v[:, :, t], "bf16"), Sd, zd, g)))
+    torch.cuda.synchronize()
+    assert row_rel_err(np.stack(outs, axis=2), o_fwd[:, :, T:], v) <= TOL["bf16"]
