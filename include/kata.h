@@ -351,6 +351,25 @@ kata_status_t kata_fwd_sg_quadratic(const void* q, const void* k, const void* v,
                                     kata_layout_t layout, kata_dtype_t dtype, void* stream);
 
 /*
+ * Exact O(T) chunked-state KATA-Sigma-g forward: the three steps of
+ * kata_fwd_chunked on the summed feature psi_S, whose state has the single
+ * factor's size: S [B,H,p*p,dv] and z [B,H,p*p] fp32 (p = d/groups), row
+ * r = a*p + b holding sum_j u^j_a u^j_b, as for kata_decode_step_sg.
+ * q, k: [B,H,T,d]; v, o: [B,H,T,dv] (bf16).  Supported: groups 2 or 4 with
+ * p = 16 (d = 32 or 64), dv = 64, bf16; others KATA_ERR_UNSUPPORTED (groups
+ * < 1 or d not a multiple of groups: KATA_ERR_INVALID_ARG).  C, S0/z0,
+ * S_out/z_out, the workspace (kata_fwd_sg_chunked_workspace_size bytes),
+ * streams and errors as for kata_fwd_chunked.
+ */
+size_t kata_fwd_sg_chunked_workspace_size(int B, int H, int T, int d, int groups, int dv, int C);
+kata_status_t kata_fwd_sg_chunked(const void* q, const void* k, const void* v, void* o,
+                                  int B, int H, int T, int d, int groups, int dv, int C,
+                                  kata_dtype_t dtype,
+                                  const float* S0, const float* z0,
+                                  float* S_out, float* z_out,
+                                  void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * One KATA-Mg decode step (update with (k, v), then read with q):
  * q, k: [B,H,d]; v, o: [B,H,dv] (fp32 or bf16); S: [B,H,groups*p*p,dv] and
  * z: [B,H,groups*p*p] fp32, read and updated in place, with row

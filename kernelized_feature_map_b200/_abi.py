@@ -46,6 +46,8 @@ SIGNATURES = {
     "kata_bwd_mg_quadratic": (_c_int, [_vp] * 9 + [_c_int] * 7 + [_vp, _c_size, _vp]),
     "kata_decode_step_mg": (_c_int, [_vp, _vp, _vp, _vp, _fp, _fp] + [_c_int] * 6 + [_vp]),
     "kata_decode_step_sg": (_c_int, [_vp, _vp, _vp, _vp, _fp, _fp] + [_c_int] * 6 + [_vp]),
+    "kata_fwd_sg_chunked_workspace_size": (_c_size, [_c_int] * 7),
+    "kata_fwd_sg_chunked": (_c_int, [_vp, _vp, _vp, _vp] + [_c_int] * 8 + [_fp, _fp, _fp, _fp, _vp, _c_size, _vp]),
     "kata_get_status": (_c_int, [_vp]),
     "kata_status_string": (ctypes.c_char_p, [_c_int]),
     "kata_set_wait_limit": (None, [ctypes.c_longlong]),
@@ -491,6 +493,37 @@ def kata_decode_step_mg(q, k, v, S, z, groups, o=None, stream=None):
     _check("kata_decode_step_mg", lib().kata_decode_step_mg(
         _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), _dev(S, "S"), _dev(z, "z"), B, H, d, int(groups),
         dv, _dtype_code(q), _stream_ptr(stream)))
+    return o
+
+
+def kata_fwd_sg_chunked_workspace_size(B, H, T, d, groups, dv, C) -> int:
+    return int(lib().kata_fwd_sg_chunked_workspace_size(B, H, T, d, int(groups), dv, C))
+
+
+def kata_fwd_sg_chunked(q, k, v, groups, C=64, S0=None, z0=None, return_state=False, o=None, workspace=None,
+                        S_out=None, z_out=None, stream=None):
+    """KATA-Sigma-g on the exact O(T) chunked path: q,k [B,H,T,d], v [B,H,T,dv]
+    (bf16, d = 16 * groups, groups 2 or 4, dv = 64).  The state ([B,H,p*p,dv],
+    [B,H,p*p] fp32, p = d/groups) is that of the summed feature."""
+    B, H, T, d = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    p = d // int(groups)
+    if o is None:
+        o = torch.empty((B, H, T, dv), dtype=q.dtype, device=dev)
+    if return_state and S_out is None:
+        S_out = torch.empty((B, H, p * p, dv), dtype=torch.float32, device=dev)
+        z_out = torch.empty((B, H, p * p), dtype=torch.float32, device=dev)
+    need = kata_fwd_sg_chunked_workspace_size(B, H, T, d, groups, dv, C)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("kata_fwd_sg_chunked", lib().kata_fwd_sg_chunked(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), B, H, T, d, int(groups), dv, C, _dtype_code(q),
+        _opt(S0, "S0"), _opt(z0, "z0"), _opt(S_out, "S_out"), _opt(z_out, "z_out"),
+        _opt(workspace, "workspace"), ws_bytes, _stream_ptr(stream)))
+    if return_state:
+        return o, S_out, z_out
     return o
 
 

@@ -83,6 +83,57 @@ __device__ __forceinline__ void packed_psi(const __nv_bfloat162 (&u)[8], uint32_
   }
 }
 
+// Row r of a [128 x 16G] bf16 tile as loaded by TMA with the swizzle of its
+// row width (32, 64 or 128 bytes: 16-byte chunk c of row r stored at chunk
+// c ^ ((r >> 2) & 1), c ^ ((r >> 1) & 3) or c ^ (r & 7)); u[8g + e] holds
+// values 16g + 2e, 16g + 2e + 1.
+template <int G>
+__device__ __forceinline__ void load_row_sw(const uint8_t* tile, int r, __nv_bfloat162 (&u)[8 * G]) {
+  static_assert(G == 1 || G == 2 || G == 4, "row widths of 32, 64 or 128 bytes");
+  const uint8_t* row = tile + r * 32 * G;
+  const int x = G == 1 ? (r >> 2) & 1 : G == 2 ? (r >> 1) & 3 : r & 7;
+#pragma unroll
+  for (int c = 0; c < 2 * G; ++c) {
+    const uint4 a = *reinterpret_cast<const uint4*>(row + ((c ^ x) << 4));
+    const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) u[4 * c + e] = *reinterpret_cast<const __nv_bfloat162*>(&w[e]);
+  }
+}
+
+// Half `half` of the packed summed feature psi~_S(u) = sum_g psi~(u^g) of one
+// token with G groups of 16 values (u as from load_row_sw<G>): the words of
+// packed_psi_half, each entry sum_g u^g_i u^g_j accumulated over the groups
+// in fp32 and rounded to bf16 once; key = true applies the factor 2 off the
+// diagonal (exact).
+template <bool key, int half, int G>
+__device__ __forceinline__ void packed_psi_sum_half(const __nv_bfloat162 (&u)[8 * G], uint32_t (&out)[kNPW / 2]) {
+  auto val = [&](int g, int i) {
+    return __bfloat162float((i & 1) ? u[8 * g + (i >> 1)].y : u[8 * g + (i >> 1)].x);
+  };
+  int w = 0;
+#pragma unroll
+  for (int i = (half == 0 ? 0 : 5); i < (half == 0 ? 5 : 16); ++i) {
+    const int npairs = (16 - i + 1) / 2;
+#pragma unroll
+    for (int x = 0; x < npairs; ++x) {
+      const int j0 = i + 2 * x;
+      float a = 0.f, b = 0.f;
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const float ui = val(g, i);
+        a = fmaf(ui, val(g, j0), a);
+        if (j0 + 1 < 16) b = fmaf(ui, val(g, j0 + 1), b);
+      }
+      if (key) {
+        if (x > 0) a *= 2.f;
+        b *= 2.f;
+      }
+      out[w++] = pack_bf16x2(a, b);
+    }
+  }
+}
+
 // Half of the packed psi words of one token: half 0 = runs i = 0..4 (words
 // 0..35), half 1 = runs i = 5..15 (words 36..71); used when two threads
 // share a token.
@@ -148,6 +199,38 @@ __device__ __forceinline__ void store_psi_q_tmem(uint32_t taddr, const uint32_t 
 #pragma unroll
   for (int e = 0; e < 8; ++e) r[e] = w[64 + e];
   tmem_st8(taddr + 64, r);
+}
+
+// Half `half` (words 36 * half ..) of psi~(q) of one query row into TMEM
+// columns [col + 36 * half, col + 36 * half + 36) of this lane; every store
+// starts at a column that is a multiple of its width.
+template <int half>
+__device__ __forceinline__ void store_psi_q_tmem_half(uint32_t taddr, const uint32_t (&w)[kNPW / 2]) {
+  if constexpr (half == 0) {
+    uint32_t a[16], b[16], c[4];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      a[e] = w[e];
+      b[e] = w[16 + e];
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) c[e] = w[32 + e];
+    tmem_st16(taddr, a);
+    tmem_st16(taddr + 16, b);
+    tmem_st4(taddr + 32, c);
+  } else {
+    uint32_t c[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) c[e] = w[e];
+    tmem_st4(taddr + 36, c);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint32_t r[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) r[e] = w[4 + 8 * q + e];
+      tmem_st8(taddr + 40 + 8 * q, r);
+    }
+  }
 }
 
 // --------------------------------------------------------------------------

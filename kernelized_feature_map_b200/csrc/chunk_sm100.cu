@@ -55,32 +55,52 @@ namespace {
 using namespace sm100;
 using namespace chunk;
 
+// G = 1: the single factor psi(u) = vec(u u^T) with p = 16.  G = 2 or 4:
+// KATA-Sigma-g with G groups of 16 (d = 16 G), the summed feature
+// psi_S(u) = sum_j vec(u^j u^j^T) on the same 16 x 16 state (gist.science
+// sec. 2.3 "Varianten"; ai.info Main Findings: state (d/g)(d/g+1)/2 * dv).
+// Its packed entries are summed over the groups in fp32 and rounded to bf16
+// once, and the intra-chunk weights sum_{j,l} (q^j . k^l)^2 are the inner
+// products psi~_S(Q) psi~_S(K)^T (9 MMAs over the 144 packed coordinates)
+// instead of squared Q K^T scores.  The wider Q and K tiles leave room for
+// fewer ring stages.
+template <int G>
+struct ChunkCfg {
+  static constexpr int kD = 16 * G;                    // q, k row width
+  static constexpr int kQKB = kTile * kD * 2;          // one Q or K tile
+  static constexpr int kStateStages = G == 1 ? 6 : 4;
+  static constexpr int kReadStages = G == 4 ? 2 : 3;
+};
+
 // ===========================================================================
 // 1. per-super-chunk state sums
 // ===========================================================================
 constexpr int kStateThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2-9 psi~(k), warps 2-5 record
-constexpr int kStateStages = 6;
 // psi~(K) buffers.  Measured at B1 H16 T131072: 6 stages with 2 buffers
 // 243 us for the whole chunked call, 4 with 3 buffers 252 us, 3 with 4
 // buffers 259 us -- the deeper TMA ring matters more than forming psi~(K)
 // further ahead
 constexpr int kStatePsiBufs = 2;
 
+template <int G>
 struct StateSmem {
-  static constexpr int kStage = kVBytes + kQKBytes;  // [V | K]
+  static constexpr int kStages = ChunkCfg<G>::kStateStages;
+  static constexpr int kStage = kVBytes + ChunkCfg<G>::kQKB;  // [V | K]
   static constexpr int offStage = 0;
-  static constexpr int offOnes = offStage + kStateStages * kStage;  // 1024-aligned
+  static constexpr int offOnes = offStage + kStages * kStage;  // 1024-aligned
   static constexpr int offPsi = offOnes + kOnesBytes;                 // kStatePsiBufs buffers
   static constexpr int offBar = offPsi + kStatePsiBufs * kPsiBytes;
-  static constexpr int kBars = 2 * kStateStages + 2 * kStatePsiBufs + 1;
+  static constexpr int kBars = 2 * kStages + 2 * kStatePsiBufs + 1;
   static constexpr int offMisc = offBar + kBars * 8;
   static constexpr int kBytes = offMisc + 16 + 1024;
 };
 
+template <int NG>
 __global__ void __launch_bounds__(kStateThreads, 1)
     chunk_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                        float* __restrict__ ws, int T, int Ls, int G, long long record_floats, WaitCtl wc) {
-  using L = StateSmem;
+  using L = StateSmem<NG>;
+  constexpr int kStateStages = L::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::offBar);
@@ -181,14 +201,16 @@ __global__ void __launch_bounds__(kStateThreads, 1)
         break;
       }
       if (tid == 0) KATA_TRACE(chunkstate, c, 3);
-      __nv_bfloat162 u[8];
-      load_row_sw32(smem + L::offStage + st * L::kStage + kVBytes, tid, u);
+      __nv_bfloat162 u[8 * NG];
+      load_row_sw<NG>(smem + L::offStage + st * L::kStage + kVBytes, tid, u);
       uint32_t w[kNPW / 2];
       if (half == 0) {
-        packed_psi_half<true, 0>(u, w);
+        if constexpr (NG == 1) packed_psi_half<true, 0>(u, w);
+        else packed_psi_sum_half<true, 0, NG>(u, w);
         store_psi_k_half<0>(smem + L::offPsi + pb * kPsiBytes, tid, w);
       } else {
-        packed_psi_half<true, 1>(u, w);
+        if constexpr (NG == 1) packed_psi_half<true, 1>(u, w);
+        else packed_psi_sum_half<true, 1, NG>(u, w);
         store_psi_k_half<1>(smem + L::offPsi + pb * kPsiBytes, tid, w);
       }
       fence_proxy_async_smem();
@@ -241,17 +263,19 @@ __global__ void __launch_bounds__(kStateThreads, 1)
 // issuing warp costs ~100 cycles in which the tensor pipe drains, so the
 // implied ones are not waited for separately.
 constexpr int kReadThreads = 576;
-constexpr int kReadStages = 3;
 
+template <int G>
 struct ReadSmem {
-  static constexpr int kStage = kVBytes + 2 * kQKBytes;  // [V | Q | K]
+  static constexpr int kStages = ChunkCfg<G>::kReadStages;
+  static constexpr int kQKB = ChunkCfg<G>::kQKB;
+  static constexpr int kStage = kVBytes + 2 * kQKB;  // [V | Q | K]
   static constexpr int offStage = 0;
-  static constexpr int offOnes = offStage + kReadStages * kStage;  // 1024-aligned
+  static constexpr int offOnes = offStage + kStages * kStage;  // 1024-aligned
   static constexpr int offPsi = offOnes + kOnesBytes;  // 2 buffers
   static constexpr int offSB = offPsi + 2 * kPsiBytes;  // one buffer
   static constexpr int offOut = offSB + kSBBytes;      // output staging: 8 boxes [32 x 32], 64B swizzle
   static constexpr int offBar = offOut + kVBytes;
-  static constexpr int kBars = 2 * kReadStages + 8;
+  static constexpr int kBars = 2 * kStages + 8;
   static constexpr int offMisc = offBar + kBars * 8;
   static constexpr int kBytes = offMisc + 16 + 1024;
   // TMEM columns (multiples of 16, 512 in total)
@@ -261,13 +285,15 @@ struct ReadSmem {
   static constexpr uint32_t colS = 384;                                    // scores / weights, 128
 };
 
+template <int NG>
 __global__ void __launch_bounds__(kReadThreads, 1)
     chunk_readout_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                          const float* __restrict__ ws, const float* __restrict__ S0, const float* __restrict__ z0,
                          float* __restrict__ S_out, float* __restrict__ z_out, int T, int Ls, int G,
                          long long record_floats, WaitCtl wc) {
-  using L = ReadSmem;
+  using L = ReadSmem<NG>;
+  constexpr int kReadStages = L::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::offBar);
@@ -331,7 +357,7 @@ __global__ void __launch_bounds__(kReadThreads, 1)
         const int row = t0 + c * kTile;
         tma_load_3d(base, &tm_v, kv_full + st, 0, row, bh);
         tma_load_3d(base + kVBytes, &tm_q, kv_full + st, 0, row, bh);
-        tma_load_3d(base + kVBytes + kQKBytes, &tm_k, kv_full + st, 0, row, bh);
+        tma_load_3d(base + kVBytes + L::kQKB, &tm_k, kv_full + st, 0, row, bh);
         ++issued;
       }
       for (int c = issued - kReadStages < 0 ? 0 : issued - kReadStages; c < issued; ++c)
@@ -341,7 +367,7 @@ __global__ void __launch_bounds__(kReadThreads, 1)
     // ------------------------------------------------------------- MMA
     // the whole warp runs this loop; one elected lane issues (see mma_ts_w)
     {
-      constexpr uint32_t id_qk = idesc_bf16(128, 128, false, false);
+      constexpr uint32_t id_qk = idesc_bf16(128, 128, false, false);  // also psi~_S(Q) (TMEM) psi~_S(K)^T
       constexpr uint32_t id_rd = idesc_bf16(128, 80, false, false);  // A = psi~(Q) (TMEM), B = S~ K-major
       constexpr uint32_t id_wv = idesc_bf16(128, 80, false, true);   // A = W (TMEM), B = [V | 1]
       constexpr uint32_t id_u = idesc_bf16(128, kNP, true, true);    // A = [V | 1]^T, B = psi~(K)
@@ -349,8 +375,9 @@ __global__ void __launch_bounds__(kReadThreads, 1)
       const uint32_t sPsi = smem_u32(smem + L::offPsi), sSB = smem_u32(smem + L::offSB);
       // descriptors built once; stages and K steps are constant offsets
       const uint64_t dq0 = smem_desc(sStage + kVBytes, 16, 256, kSw32);
-      const uint64_t dk0 = smem_desc(sStage + kVBytes + kQKBytes, 16, 256, kSw32);
+      const uint64_t dk0 = smem_desc(sStage + kVBytes + L::kQKB, 16, 256, kSw32);
       const uint64_t dpsi = smem_desc(sPsi, kPsiAtom, 256, kSw32);
+      const uint64_t dpsik = smem_desc(sPsi, 16, 256, kSw32);  // psi~_S(K) as a K-major B operand
       const uint64_t dsb0 = smem_desc(sSB, 16, 256, kSw32);
       for (int c = 0; c < n_chunks; ++c) {
         const int st = c % kReadStages, ob = c & 1;
@@ -362,7 +389,15 @@ __global__ void __launch_bounds__(kReadThreads, 1)
         tc_fence_after();
         // scores of chunk c (overwrite the weights of chunk c-1 only after
         // the intra-chunk MMAs of c-1 issued before them)
-        mma_ss_w(tmem + L::colS, desc_add(dq0, st * L::kStage), desc_add(dk0, st * L::kStage), id_qk, 0);
+        if constexpr (NG == 1) {
+          mma_ss_w(tmem + L::colS, desc_add(dq0, st * L::kStage), desc_add(dk0, st * L::kStage), id_qk, 0);
+        } else {
+          // the Sigma-g weights directly: psi~_S(Q_c) psi~_S(K_c)^T
+#pragma unroll
+          for (int ks = 0; ks < kNP / 16; ++ks)
+            mma_ts_w(tmem + L::colS, tmem + L::colPQ + ks * 8, desc_add(dpsik, (c & 1) * kPsiBytes + ks * kPsiAtom),
+                     id_qk, ks > 0);
+        }
         mma_commit_w(s_full);
         // readout against the bf16 copy of the state entering the chunk (the
         // [O | D] buffer is free: see state_full); first, so that psi~(q_c)
@@ -470,19 +505,29 @@ __global__ void __launch_bounds__(kReadThreads, 1)
           uint32_t r[32];
           tmem_ld32(lane_base + L::colS + 32 * bb, r);
           tmem_wait_ld();
-          // squares on fp32 pairs (each rounded as a scalar multiply)
-          if (bb < quarter) {
+          if constexpr (NG == 1) {
+            // squares on fp32 pairs (each rounded as a scalar multiply)
+            if (bb < quarter) {
 #pragma unroll
-            for (int x = 0; x < 16; ++x) {
-              const uint64_t sq = f32x2_mul(f32x2(r[2 * x], r[2 * x + 1]), f32x2(r[2 * x], r[2 * x + 1]));
-              w[x] = pack_bf16x2(f32x2_lo(sq), f32x2_hi(sq));
+              for (int x = 0; x < 16; ++x) {
+                const uint64_t sq = f32x2_mul(f32x2(r[2 * x], r[2 * x + 1]), f32x2(r[2 * x], r[2 * x + 1]));
+                w[x] = pack_bf16x2(f32x2_lo(sq), f32x2_hi(sq));
+              }
+            } else {
+#pragma unroll
+              for (int x = 0; x < 16; ++x) {
+                const uint32_t a = 2 * x > lane ? 0u : r[2 * x], b = 2 * x + 1 > lane ? 0u : r[2 * x + 1];
+                const uint64_t sq = f32x2_mul(f32x2(a, b), f32x2(a, b));
+                w[x] = pack_bf16x2(f32x2_lo(sq), f32x2_hi(sq));
+              }
             }
           } else {
+            // the Sigma-g weights are the scores themselves
 #pragma unroll
             for (int x = 0; x < 16; ++x) {
-              const uint32_t a = 2 * x > lane ? 0u : r[2 * x], b = 2 * x + 1 > lane ? 0u : r[2 * x + 1];
-              const uint64_t sq = f32x2_mul(f32x2(a, b), f32x2(a, b));
-              w[x] = pack_bf16x2(f32x2_lo(sq), f32x2_hi(sq));
+              const float a = bb == quarter && 2 * x > lane ? 0.f : __uint_as_float(r[2 * x]);
+              const float b = bb == quarter && 2 * x + 1 > lane ? 0.f : __uint_as_float(r[2 * x + 1]);
+              w[x] = pack_bf16x2(a, b);
             }
           }
         }
@@ -510,16 +555,42 @@ __global__ void __launch_bounds__(kReadThreads, 1)
     // psi~(k) of chunk cc into shared-memory buffer cc % 2, or psi~(q) of
     // chunk cc into TMEM, from the chunk's landed stage
     auto psi_k = [&](int cc) {
-      __nv_bfloat162 u[8];
-      uint32_t w[kNPW];
-      load_row_sw32(smem + L::offStage + (cc % kReadStages) * L::kStage + kVBytes + kQKBytes, m, u);
-      packed_psi<true>(u, w);
-      store_psi_k(smem + L::offPsi + (cc & 1) * kPsiBytes, m, w);
+      const uint8_t* tile = smem + L::offStage + (cc % kReadStages) * L::kStage + kVBytes + L::kQKB;
+      uint8_t* dst = smem + L::offPsi + (cc & 1) * kPsiBytes;
+      if constexpr (NG == 1) {
+        __nv_bfloat162 u[8];
+        uint32_t w[kNPW];
+        load_row_sw<1>(tile, m, u);
+        packed_psi<true>(u, w);
+        store_psi_k(dst, m, w);
+      } else {
+        __nv_bfloat162 u[8 * NG];
+        uint32_t w[kNPW / 2];
+        load_row_sw<NG>(tile, m, u);
+        packed_psi_sum_half<true, 0, NG>(u, w);
+        store_psi_k_half<0>(dst, m, w);
+        packed_psi_sum_half<true, 1, NG>(u, w);
+        store_psi_k_half<1>(dst, m, w);
+      }
     };
     auto psi_q_formed = [&](int cc, uint32_t (&w)[kNPW]) {
       __nv_bfloat162 u[8];
-      load_row_sw32(smem + L::offStage + (cc % kReadStages) * L::kStage + kVBytes, m, u);
+      load_row_sw<1>(smem + L::offStage + (cc % kReadStages) * L::kStage + kVBytes, m, u);
       packed_psi<false>(u, w);
+    };
+    // Sigma-g: psi~_S(q) of chunk cc into TMEM one half at a time (the
+    // groups' values and a whole row do not fit in registers together);
+    // `before` runs between forming the first half and storing it
+    auto psi_q_sum_to_tmem = [&](int cc, auto&& before) -> bool {
+      __nv_bfloat162 u[8 * NG];
+      uint32_t w[kNPW / 2];
+      load_row_sw<NG>(smem + L::offStage + (cc % kReadStages) * L::kStage + kVBytes, m, u);
+      packed_psi_sum_half<false, 0, NG>(u, w);
+      if (!before()) return false;
+      store_psi_q_tmem_half<0>(lane_base + L::colPQ, w);
+      packed_psi_sum_half<false, 1, NG>(u, w);
+      store_psi_q_tmem_half<1>(lane_base + L::colPQ, w);
+      return true;
     };
     // running state <- scanned prefix (fp32 into TMEM, bf16 into shared
     // memory); with a single super-chunk there is no workspace and the
@@ -543,10 +614,12 @@ __global__ void __launch_bounds__(kReadThreads, 1)
     if (ok) {
       if (psi_group) {
         psi_k(0);
-      } else {
+      } else if constexpr (NG == 1) {
         uint32_t w[kNPW];
         psi_q_formed(0, w);
         store_psi_q_tmem(lane_base + L::colPQ, w);
+      } else {
+        psi_q_sum_to_tmem(0, [] { return true; });
       }
     }
     tmem_wait_st();
@@ -562,7 +635,7 @@ __global__ void __launch_bounds__(kReadThreads, 1)
         // c-1, which this group saw complete in the previous iteration
         psi_k(c + 1);
         if (m == 0) KATA_TRACE(chunk, c, 11);
-      } else {
+      } else if constexpr (NG == 1) {
         // psi~(q_{c+1}) into TMEM once the readout of chunk c (the first MMAs
         // of the chunk) has read psi~(q_c)
         uint32_t wq[kNPW];
@@ -571,6 +644,16 @@ __global__ void __launch_bounds__(kReadThreads, 1)
         if (m == 0) KATA_TRACE(chunk, c, 19);
         tc_fence_after();
         store_psi_q_tmem(lane_base + L::colPQ, wq);
+        tmem_wait_st();
+      } else {
+        // the same; the readout of chunk c also ends the scores' use of
+        // psi~_S(q_c), issued before it
+        if (!psi_q_sum_to_tmem(c + 1, [&] {
+              if (!mbar_wait_w(rd_done, c & 1, env)) return false;
+              tc_fence_after();
+              return true;
+            }))
+          break;
         tmem_wait_st();
       }
       // the state after chunk c is complete: this group's half of the bf16
@@ -610,41 +693,76 @@ __global__ void __launch_bounds__(kReadThreads, 1)
 
 size_t chunk_record_floats_sm100() { return (size_t)kRecRows * kNP; }
 
-cudaError_t launch_chunk_state_sm100(const void* k, const void* v, float* ws, const ChunkPlan& pl, const WaitCtl& wc,
-                                     cudaStream_t st) {
+namespace {
+
+template <int NG>
+cudaError_t launch_state_t(const void* k, const void* v, float* ws, const ChunkPlan& pl, const WaitCtl& wc,
+                           cudaStream_t st) {
+  using L = StateSmem<NG>;
   if (pl.p != 16 || pl.dv != kDV) return cudaErrorInvalidValue;
   CUtensorMap tk, tv;
-  if (!make_tmap_bf16(&tk, k, 16, pl.T, pl.BH, kTile) || !make_tmap_bf16(&tv, v, kDV, pl.T, pl.BH, kTile))
+  if (!make_tmap_bf16(&tk, k, ChunkCfg<NG>::kD, pl.T, pl.BH, kTile) ||
+      !make_tmap_bf16(&tv, v, kDV, pl.T, pl.BH, kTile))
     return cudaErrorInvalidValue;
-  cudaError_t e =
-      cudaFuncSetAttribute(chunk_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, StateSmem::kBytes);
+  cudaError_t e = cudaFuncSetAttribute(chunk_state_kernel<NG>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
   if (e != cudaSuccess) return e;
   if (pl.G < 2) return cudaSuccess;  // the last super-chunk's sum is never needed
   dim3 grid(pl.G - 1, pl.BH);
-  chunk_state_kernel<<<grid, kStateThreads, StateSmem::kBytes, st>>>(tk, tv, ws, pl.T, pl.Ls, pl.G,
-                                                                      (long long)pl.record_floats, wc);
+  chunk_state_kernel<NG><<<grid, kStateThreads, L::kBytes, st>>>(tk, tv, ws, pl.T, pl.Ls, pl.G,
+                                                                  (long long)pl.record_floats, wc);
   return cudaGetLastError();
+}
+
+template <int NG>
+cudaError_t launch_readout_t(const void* q, const void* k, const void* v, void* o, const float* ws, const float* S0,
+                             const float* z0, float* S_out, float* z_out, const ChunkPlan& pl, const WaitCtl& wc,
+                             cudaStream_t st) {
+  using L = ReadSmem<NG>;
+  if (pl.p != 16 || pl.dv != kDV) return cudaErrorInvalidValue;
+  if (!ws && pl.G != 1) return cudaErrorInvalidValue;
+  constexpr int kD = ChunkCfg<NG>::kD;
+  CUtensorMap tq, tk, tv, to;
+  if (!make_tmap_bf16(&tq, q, kD, pl.T, pl.BH, kTile) || !make_tmap_bf16(&tk, k, kD, pl.T, pl.BH, kTile) ||
+      !make_tmap_bf16(&tv, v, kDV, pl.T, pl.BH, kTile) || !make_tmap_bf16_box(&to, o, kDV, pl.T, pl.BH, 32, 32))
+    return cudaErrorInvalidValue;
+  cudaError_t e =
+      cudaFuncSetAttribute(chunk_readout_kernel<NG>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
+  if (e != cudaSuccess) return e;
+  const dim3 grid(pl.G, pl.BH), block(kReadThreads);
+  if (ws)  // after the state build and scan of this call: launched as the scan's programmatic dependent
+    return launch_pdl(chunk_readout_kernel<NG>, grid, block, (size_t)L::kBytes, st, tq, tk, tv, to,
+                      (const float*)ws, S0, z0, S_out, z_out, pl.T, pl.Ls, pl.G, (long long)pl.record_floats, wc);
+  chunk_readout_kernel<NG><<<grid, block, L::kBytes, st>>>(tq, tk, tv, to, ws, S0, z0, S_out, z_out, pl.T, pl.Ls,
+                                                           pl.G, (long long)pl.record_floats, wc);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_chunk_state_sm100(const void* k, const void* v, float* ws, const ChunkPlan& pl, const WaitCtl& wc,
+                                     cudaStream_t st) {
+  return launch_state_t<1>(k, v, ws, pl, wc, st);
 }
 
 cudaError_t launch_chunk_readout_sm100(const void* q, const void* k, const void* v, void* o, const float* ws,
                                        const float* S0, const float* z0, float* S_out, float* z_out,
                                        const ChunkPlan& pl, const WaitCtl& wc, cudaStream_t st) {
-  if (pl.p != 16 || pl.dv != kDV) return cudaErrorInvalidValue;
-  if (!ws && pl.G != 1) return cudaErrorInvalidValue;
-  CUtensorMap tq, tk, tv, to;
-  if (!make_tmap_bf16(&tq, q, 16, pl.T, pl.BH, kTile) || !make_tmap_bf16(&tk, k, 16, pl.T, pl.BH, kTile) ||
-      !make_tmap_bf16(&tv, v, kDV, pl.T, pl.BH, kTile) || !make_tmap_bf16_box(&to, o, kDV, pl.T, pl.BH, 32, 32))
-    return cudaErrorInvalidValue;
-  cudaError_t e =
-      cudaFuncSetAttribute(chunk_readout_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ReadSmem::kBytes);
-  if (e != cudaSuccess) return e;
-  const dim3 grid(pl.G, pl.BH), block(kReadThreads);
-  if (ws)  // after the state build and scan of this call: launched as the scan's programmatic dependent
-    return launch_pdl(chunk_readout_kernel, grid, block, (size_t)ReadSmem::kBytes, st, tq, tk, tv, to,
-                      (const float*)ws, S0, z0, S_out, z_out, pl.T, pl.Ls, pl.G, (long long)pl.record_floats, wc);
-  chunk_readout_kernel<<<grid, block, ReadSmem::kBytes, st>>>(tq, tk, tv, to, ws, S0, z0, S_out, z_out, pl.T, pl.Ls,
-                                                              pl.G, (long long)pl.record_floats, wc);
-  return cudaGetLastError();
+  return launch_readout_t<1>(q, k, v, o, ws, S0, z0, S_out, z_out, pl, wc, st);
+}
+
+cudaError_t launch_chunk_state_sg(const void* k, const void* v, float* ws, const ChunkPlan& pl, int groups,
+                                  const WaitCtl& wc, cudaStream_t st) {
+  if (groups == 2) return launch_state_t<2>(k, v, ws, pl, wc, st);
+  if (groups == 4) return launch_state_t<4>(k, v, ws, pl, wc, st);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_chunk_readout_sg(const void* q, const void* k, const void* v, void* o, const float* ws,
+                                    const float* S0, const float* z0, float* S_out, float* z_out,
+                                    const ChunkPlan& pl, int groups, const WaitCtl& wc, cudaStream_t st) {
+  if (groups == 2) return launch_readout_t<2>(q, k, v, o, ws, S0, z0, S_out, z_out, pl, wc, st);
+  if (groups == 4) return launch_readout_t<4>(q, k, v, o, ws, S0, z0, S_out, z_out, pl, wc, st);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace kata

@@ -611,6 +611,49 @@ KATA_API kata_status_t kata_bwd_mg_quadratic(const void* q, const void* k, const
   return KATA_OK;
 }
 
+// KATA-Sigma-g on the chunked path: groups of 16 (p = 16), dv = 64, bf16.
+static kata_status_t check_sg_chunked(const void* q, const void* k, const void* v, const void* o, int B, int H,
+                                      int T, int d, int groups, int dv, int C, kata_dtype_t dtype, const float* S0,
+                                      const float* z0, const float* S_out, const float* z_out) {
+  if (groups < 1 || d < 1 || d % groups != 0) return KATA_ERR_INVALID_ARG;
+  if (dtype != KATA_F32 && dtype != KATA_BF16) return KATA_ERR_INVALID_ARG;
+  if (dtype != KATA_BF16 || dv != 64 || d / groups != 16 || !(groups == 2 || groups == 4))
+    return KATA_ERR_UNSUPPORTED;
+  return check_chunked_args(q, k, v, o, B, H, T, 16, dv, C, dtype, S0, z0, S_out, z_out);
+}
+
+KATA_API size_t kata_fwd_sg_chunked_workspace_size(int B, int H, int T, int d, int groups, int dv, int C) {
+  if (groups < 1 || d != 16 * groups) return 0;
+  return kata_fwd_chunked_workspace_size(B, H, T, 16, dv, C, KATA_BF16);
+}
+
+KATA_API kata_status_t kata_fwd_sg_chunked(const void* q, const void* k, const void* v, void* o, int B, int H, int T,
+                                           int d, int groups, int dv, int C, kata_dtype_t dtype, const float* S0,
+                                           const float* z0, float* S_out, float* z_out, void* workspace,
+                                           size_t workspace_bytes, void* stream) {
+  kata_status_t s = check_sg_chunked(q, k, v, o, B, H, T, d, groups, dv, C, dtype, S0, z0, S_out, z_out);
+  if (s != KATA_OK) return s;
+  // T == 0: the state passes through (the p = 16 state of the summed feature)
+  if (T == 0) return kata_fwd_chunked(q, k, v, o, B, H, 0, 16, dv, C, dtype, S0, z0, S_out, z_out, nullptr, 0, stream);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const ChunkPlan plan = make_chunk_plan(B, H, T, 16, dv, C, dtype);
+  if (plan.workspace_bytes > 0) {
+    if (!workspace || workspace_bytes < plan.workspace_bytes) return KATA_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KATA_ERR_MISALIGNED;
+  }
+  float* ws = plan.workspace_bytes > 0 ? static_cast<float*>(workspace) : nullptr;
+  const WaitCtl wc = wait_ctl();
+  cudaError_t e = cudaSuccess;
+  if (plan.G > 1) {
+    e = launch_chunk_state_sg(k, v, ws, plan, groups, wc, st);
+    if (e == cudaSuccess) e = launch_state_scan(ws, plan, plan.G - 1, S0, z0, nullptr, nullptr, st);
+  }
+  if (e == cudaSuccess)
+    e = launch_chunk_readout_sg(q, k, v, o, ws, plan.G > 1 ? nullptr : S0, plan.G > 1 ? nullptr : z0, S_out, z_out,
+                                plan, groups, wc, st);
+  return from_cuda(e);
+}
+
 KATA_API kata_status_t kata_decode_step_sg(const void* q, const void* k, const void* v, void* o, float* S, float* z,
                                            int B, int H, int d, int groups, int dv, kata_dtype_t dtype,
                                            void* stream) {

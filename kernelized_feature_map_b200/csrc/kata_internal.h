@@ -117,6 +117,14 @@ cudaError_t launch_chunk_state_sm100(const void* k, const void* v, float* ws, co
 cudaError_t launch_chunk_readout_sm100(const void* q, const void* k, const void* v, void* o, const float* ws,
                                        const float* S0, const float* z0, float* S_out, float* z_out,
                                        const ChunkPlan& pl, const WaitCtl& wc, cudaStream_t st);
+// The same kernels for KATA-Sigma-g with `groups` (2 or 4) groups of 16
+// (d = 16 * groups): the summed feature on the p = 16 state, the same plan
+// and record layout.
+cudaError_t launch_chunk_state_sg(const void* k, const void* v, float* ws, const ChunkPlan& pl, int groups,
+                                  const WaitCtl& wc, cudaStream_t st);
+cudaError_t launch_chunk_readout_sg(const void* q, const void* k, const void* v, void* o, const float* ws,
+                                    const float* S0, const float* z0, float* S_out, float* z_out,
+                                    const ChunkPlan& pl, int groups, const WaitCtl& wc, cudaStream_t st);
 
 // chunk_linear_sm100.cu -- first-order (linear) attention, psi(u) = u, with
 // d = 16 and dv = 64 in bf16: the same three steps with unpacked records

@@ -332,3 +332,86 @@ def test_sg_decode_continues_the_forward(kata):
                                                    to_dev(v[:, :, t], "bf16"), Sd, zd, g)))
     torch.cuda.synchronize()
     assert row_rel_err(np.stack(outs, axis=2), o_fwd[:, :, T:], v) <= TOL["bf16"]
+
+
+# ---------------------------------------------------------------------------
+# KATA-Sigma-g on the chunked path (groups of 16 on the p = 16 state)
+# ---------------------------------------------------------------------------
+
+def _sg_state(k, v, g):
+    from oracle import sigma_g as osg
+    fk = osg.features_sg(k, g)
+    return (np.einsum("bhtp,bhte->bhpe", fk, np.asarray(v, np.float64)), fk.sum(axis=2))
+
+
+# one super-chunk per (b,h) (B4 H4 T700), several (B2 H4 T3000) and many
+# (B1 H2 T9000: the scan over dozens of records), plus ragged short cases
+@pytest.mark.parametrize("B,H,T", [(2, 3, 77), (1, 2, 129), (4, 4, 700), (2, 4, 3000), (1, 2, 9000)])
+@pytest.mark.parametrize("g", [2, 4])
+def test_sg_chunked_matches_oracle(kata, B, H, T, g):
+    import torch
+    from oracle import sigma_g as osg
+    d, dv = 16 * g, 64
+    q, k, v = workloads.normal_qkv(B, H, T, d, dv, seed=430 + T + g, dtype="bf16")
+    o_ref = osg.recurrent_sg(q, k, v, g)
+    o, S, z = kata.kata_fwd_sg_chunked(to_dev(q, "bf16"), to_dev(k, "bf16"), to_dev(v, "bf16"), g,
+                                       return_state=True)
+    torch.cuda.synchronize()
+    assert kata.kata_get_status() == 0
+    assert row_rel_err(to_np(o), o_ref, v) <= TOL["bf16"]
+    # the final state: every packed entry sum_j k^j_a k^j_b is rounded to bf16
+    # once (2^-9 relative), the T terms summed in fp32
+    S_ref, z_ref = _sg_state(k, v, g)
+    S_abs, z_abs = _sg_state(np.abs(k), np.abs(v), g)
+    eps = 2.0 ** -8 + (T + 4) * 2.0 ** -24
+    assert np.all(np.abs(S.cpu().numpy() - S_ref) <= eps * S_abs + 1e-6)
+    assert np.all(np.abs(z.cpu().numpy() - z_ref) <= eps * z_abs + 1e-6)
+
+
+@pytest.mark.parametrize("g", [2, 4])
+def test_sg_chunked_state_in_and_out_and_agrees_with_flash(kata, g):
+    import torch
+    from oracle import sigma_g as osg
+    B, H, T, t0, d, dv = 2, 4, 3000, 1100, 16 * g, 64
+    q, k, v = workloads.normal_qkv(B, H, T, d, dv, seed=440 + g, dtype="bf16")
+    o_ref = osg.recurrent_sg(q, k, v, g)
+    qd, kd, vd = to_dev(q, "bf16"), to_dev(k, "bf16"), to_dev(v, "bf16")
+    oa, Sa, za = kata.kata_fwd_sg_chunked(qd[:, :, :t0].contiguous(), kd[:, :, :t0].contiguous(),
+                                          vd[:, :, :t0].contiguous(), g, return_state=True)
+    ob = kata.kata_fwd_sg_chunked(qd[:, :, t0:].contiguous(), kd[:, :, t0:].contiguous(),
+                                  vd[:, :, t0:].contiguous(), g, S0=Sa, z0=za)
+    o_flash = kata.kata_fwd_sg_quadratic(qd, kd, vd, g)
+    torch.cuda.synchronize()
+    assert kata.kata_get_status() == 0
+    o_split = np.concatenate([to_np(oa), to_np(ob)], axis=2)
+    assert row_rel_err(o_split, o_ref, v) <= TOL["bf16"]
+    assert row_rel_err(o_split, to_np(o_flash), v) <= TOL["bf16"]
+    # resume from the oracle's state after t0 tokens
+    S1, z1 = _sg_state(k[:, :, :t0], v[:, :, :t0], g)
+    o2 = kata.kata_fwd_sg_chunked(qd[:, :, t0:].contiguous(), kd[:, :, t0:].contiguous(), vd[:, :, t0:].contiguous(),
+                                  g, S0=torch.from_numpy(S1.astype(np.float32)).cuda(),
+                                  z0=torch.from_numpy(z1.astype(np.float32)).cuda())
+    torch.cuda.synchronize()
+    assert row_rel_err(to_np(o2), o_ref[:, :, t0:], v) <= TOL["bf16"]
+
+
+def test_sg_chunked_full_size_sampled_rows(kata):
+    """B1 H16 T131072, d = 64 in 4 groups: sampled rows from the definition."""
+    import torch
+    B, H, T, d, g, dv = 1, 16, 131072, 64, 4, 64
+    q, k, v = workloads.normal_qkv(B, H, T, d, dv, seed=450, dtype="bf16")
+    got = to_np(kata.kata_fwd_sg_chunked(to_dev(q, "bf16"), to_dev(k, "bf16"), to_dev(v, "bf16"), g))
+    torch.cuda.synchronize()
+    assert kata.kata_get_status() == 0
+    rng = np.random.default_rng(451)
+    rows = np.array(sorted(set([0, 1, 127, 128, 129, T // 2, T - 2, T - 1] + rng.integers(0, T, 16).tolist())))
+    for h in (0, 9):
+        qg = q[0, h].astype(np.float64).reshape(T, g, 16)
+        kg = k[0, h].astype(np.float64).reshape(T, g, 16)
+        ref = np.empty((len(rows), dv))
+        for i, t in enumerate(rows):
+            dots = np.einsum("jp,slp->sjl", qg[t], kg[:t + 1])
+            w = (dots * dots).sum(axis=(1, 2))
+            ref[i] = (w @ v[0, h, :t + 1].astype(np.float64)) / w.sum()
+        vmax = np.full(len(rows), np.abs(v[0, h]).max())
+        assert rows_rel_err(got[0, h, rows], ref, vmax) <= TOL["bf16"]
