@@ -622,6 +622,23 @@ def run_mg(args, K, torch, dev, stream, flush):
         out["chunked_mg%d_ctx131k" % g] = dict(B=B, H=H, T=T, d=d, groups=g, dv=dv, layout="bthd", ms=ms_c,
                                                chunked=True)
         del q, k, v, o, ws
+    # KATA-Sigma-g on the chunked path (groups of 16: d = 64 in 4 groups),
+    # [B,H,T,d], at T = 2048 (B = 8) and T = 131072 (B = 1)
+    for B, T in ((8, 2048), (1, 131072)):
+        H, d, g, dv = 16, 64, 4, 64
+        gen_l.manual_seed(600 + B)
+        q = torch.randn((B, H, T, d), generator=gen_l, device=dev)
+        k = torch.randn((B, H, T, d), generator=gen_l, device=dev)
+        q = (q / q.norm(dim=-1, keepdim=True)).to(bf)
+        k = (k / k.norm(dim=-1, keepdim=True)).to(bf)
+        v = torch.randn((B, H, T, dv), generator=gen_l, device=dev).to(bf)
+        o = torch.empty_like(v)
+        ws = torch.empty(max(256, K.kata_fwd_sg_chunked_workspace_size(B, H, T, d, g, dv, 64)), dtype=torch.uint8,
+                         device=dev)
+        ms_c = _time_call(lambda: K.kata_fwd_sg_chunked(q, k, v, g, C=64, o=o, workspace=ws), flush, stream, 5, 2)
+        out["chunked_sg%d_ctx%s" % (g, "2k" if T == 2048 else "131k")] = dict(
+            B=B, H=H, T=T, d=d, groups=g, dv=dv, layout="bhtd", ms=ms_c, chunked=True, summed=True)
+        del q, k, v, o, ws
     # decode step on the concatenated per-group state (B = 64, as for the
     # single-factor decode line): HBM-bound, the state is read and written once
     gen = torch.Generator(device=dev)
@@ -909,7 +926,14 @@ def roofline_points(res, peaks, cfg):
         # KATA-Mg itself (the metric's name): flash-style at T = 2048 and the
         # chunked path at T = 2048 and 131072, d = 64 in 2 or 4 groups
         for name, m in sorted(lg.get("mg", {}).items()):
-            if "P" in m or m.get("summed"):
+            if "P" in m or (m.get("summed") and not m.get("chunked")):
+                continue
+            if m.get("summed"):
+                wl = "KATA-Sigma-g B=%d H=%d T=%d d=%d groups=%d dv=%d bf16" % (m["B"], m["H"], m["T"], m["d"],
+                                                                               m["groups"], m["dv"])
+                pts.append(hbm_point("sg_chunked", wl, m["ms"], m["B"] * m["T"],
+                                     m["B"] * m["H"] * m["T"] * (2 * m["d"] + 2 * m["dv"]) * 2, cl.get("mg"),
+                                     T=m["T"], groups=m["groups"]))
                 continue
             wl = "KATA-Mg B=%d H=%d T=%d d=%d groups=%d dv=%d bf16 [%s]" % (m["B"], m["H"], m["T"], m["d"],
                                                                           m["groups"], m["dv"], m["layout"])
@@ -1024,8 +1048,9 @@ def report(args, res, step_ms, e2e_ms, world):
                     # written once (2d + 2dv bf16 values per token-head)
                     cb = m["B"] * m["H"] * m["T"] * (2 * m["d"] + 2 * m["dv"]) * 2
                     line["mg"][name] = {
-                        "workload": "KATA-Mg chunked B=%d H=%d T=%d d=%d groups=%d dv=%d bf16 [%s]" % (
-                            m["B"], m["H"], m["T"], m["d"], m["groups"], m["dv"], m["layout"]),
+                        "workload": "%s chunked B=%d H=%d T=%d d=%d groups=%d dv=%d bf16 [%s]" % (
+                            "KATA-Sigma-g" if m.get("summed") else "KATA-Mg", m["B"], m["H"], m["T"], m["d"],
+                            m["groups"], m["dv"], m["layout"]),
                         "ms": m["ms"], "tokens_per_s": m["B"] * m["T"] / (m["ms"] * 1e-3),
                         "hbm_frac": cb / (m["ms"] * 1e-3) / 1e9 / peaks["hbm_gbs"]}
                 else:
