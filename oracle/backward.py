@@ -106,3 +106,55 @@ def backward_mg(q, k, v, dO, groups: int):
         dk[..., sl] = np.einsum("bhts,bhtp->bhsp", dSj, q[..., sl])
     dv = np.einsum("bhts,bhte->bhse", W, dN)
     return dq, dk, dv
+
+
+def forward_sg_with_d(q, k, v, groups: int):
+    """KATA-Sigma-g forward (weight sum_{j,l} (q_t^j . k_s^l)^2, every query
+    group against every key group) with its denominators, fp64."""
+    q, k, v = (np.asarray(x, np.float64) for x in (q, k, v))
+    d = q.shape[-1]
+    p = d // groups
+    T = q.shape[2]
+    mask = np.tril(np.ones((T, T), dtype=bool))
+    W = np.zeros(q.shape[:2] + (T, T))
+    for j in range(groups):
+        for l in range(groups):
+            S = np.einsum("bhtp,bhsp->bhts", q[..., j * p:(j + 1) * p], k[..., l * p:(l + 1) * p])
+            W += S * S
+    W = np.where(mask, W, 0.0)
+    N = np.einsum("bhts,bhse->bhte", W, v)
+    D = W.sum(axis=-1)
+    safe = np.where(D > 0, D, 1.0)
+    o = np.where((D > 0)[..., None], N / safe[..., None], 0.0)
+    return o, D
+
+
+def backward_sg(q, k, v, dO, groups: int):
+    """(dq, dk, dv) of the KATA-Sigma-g forward, fp64: the single-factor chain
+    rule with w = sum_{j,l} S_jl^2, S_jl = q^j . k^l, so dS_jl = 2 S_jl dw;
+    dq^j sums over the key groups l, dk^l over the query groups j."""
+    q, k, v, dO = (np.asarray(x, np.float64) for x in (q, k, v, dO))
+    d = q.shape[-1]
+    p = d // groups
+    T = q.shape[2]
+    mask = np.tril(np.ones((T, T), dtype=bool))
+    o, D = forward_sg_with_d(q, k, v, groups)
+    live = D > 0
+    safe = np.where(live, D, 1.0)
+    dN = np.where(live[..., None], dO / safe[..., None], 0.0)
+    dD = np.where(live, -np.einsum("bhte,bhte->bht", dO, o) / safe, 0.0)
+    dW = np.where(mask, np.einsum("bhte,bhse->bhts", dN, v) + dD[..., None], 0.0)
+    W = np.zeros(q.shape[:2] + (T, T))
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    for j in range(groups):
+        sj = slice(j * p, (j + 1) * p)
+        for l in range(groups):
+            sl = slice(l * p, (l + 1) * p)
+            S = np.einsum("bhtp,bhsp->bhts", q[..., sj], k[..., sl])
+            W += np.where(mask, S * S, 0.0)
+            dS = 2.0 * S * dW
+            dq[..., sj] += np.einsum("bhts,bhsp->bhtp", dS, k[..., sl])
+            dk[..., sl] += np.einsum("bhts,bhtp->bhsp", dS, q[..., sj])
+    dv = np.einsum("bhts,bhte->bhse", W, dN)
+    return dq, dk, dv

@@ -685,3 +685,35 @@ def test_sigma_g_decode_step_pins():
     o2, S2, z2 = oracle.decode_step(q[:, :, 0], k[:, :, 0], v[:, :, 0], S, z)
     np.testing.assert_allclose(o1, o2, rtol=1e-11, atol=1e-12)
     np.testing.assert_allclose(S1, S2, rtol=1e-12, atol=1e-12)
+
+
+def test_backward_sg_pins():
+    """KATA-Sigma-g gradients: g = 1 equals the single-factor gradients, the
+    forward equals the Sigma-g oracle, central differences of that oracle
+    match, and scaling a whole query row leaves its output unchanged, so
+    q_t . dq_t = 0 row by row (likewise for a key row only through the
+    normalisation, which is not a pin)."""
+    q, k, v = _rand_mg(B=1, H=1, T=6, d=4, dv=2, seed=490)
+    rng = np.random.default_rng(491)
+    dO = rng.standard_normal(v.shape)
+    for a, b in zip(obw.backward_sg(q, k, v, dO, 1), obw.backward(q, k, v, dO)):
+        np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-13)
+    o, _ = obw.forward_sg_with_d(q, k, v, 2)
+    np.testing.assert_allclose(o, osg.direct_sg(q, k, v, 2), rtol=1e-11, atol=1e-12)
+    dq, dk, dv = obw.backward_sg(q, k, v, dO, 2)
+    h = 1e-6
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        num = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            ap = {"q": q, "k": k, "v": v}
+            am = dict(ap)
+            ap[name], am[name] = xp, xm
+            num[idx] = ((osg.direct_sg(ap["q"], ap["k"], ap["v"], 2) * dO).sum()
+                        - (osg.direct_sg(am["q"], am["k"], am["v"], 2) * dO).sum()) / (2 * h)
+        np.testing.assert_allclose(g, num, rtol=1e-6, atol=1e-7, err_msg=name)
+    q2, k2, v2 = _rand_mg(B=1, H=2, T=30, d=8, dv=3, seed=492)
+    dq2, _, _ = obw.backward_sg(q2, k2, v2, rng.standard_normal(v2.shape), 2)
+    np.testing.assert_allclose(np.einsum("bhtd,bhtd->bht", q2, dq2), 0.0, atol=1e-9)
