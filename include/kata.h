@@ -351,6 +351,27 @@ kata_status_t kata_fwd_sg_quadratic(const void* q, const void* k, const void* v,
                                     kata_layout_t layout, kata_dtype_t dtype, void* stream);
 
 /*
+ * Training with KATA-Sigma-g ([B,H,T,*] layout, bf16, dv = 64, the
+ * (p, groups) of kata_fwd_sg_quadratic with groups > 1): the Sigma-g forward
+ * that also saves D [B,H,T] fp32, and its backward pass.  With
+ * w = sum_{j,l} (q^j . k^l)^2 the gradient is a sum over the (query group,
+ * key group) pairs of the single-factor gradient taken with the pair's
+ * scores and the Sigma-g output's o and D: dq^j sums over l, dk^l over j and
+ * dv over every pair.  The backward runs the single-factor kernels once per
+ * pair on the pair's columns (read and written in place), adding each pass
+ * to the rows the earlier passes wrote (in bf16).  Workspace as
+ * kata_bwd_quadratic (8 bytes per row).
+ */
+kata_status_t kata_fwd_sg_quadratic_train(const void* q, const void* k, const void* v, void* o, float* D,
+                                          int B, int H, int T, int d, int groups, int dv,
+                                          kata_dtype_t dtype, void* stream);
+kata_status_t kata_bwd_sg_quadratic(const void* q, const void* k, const void* v, const void* o,
+                                    const float* D, const void* dO, void* dq, void* dk, void* dv,
+                                    int B, int H, int T, int d, int groups, int dv_width,
+                                    kata_dtype_t dtype, void* workspace, size_t workspace_bytes,
+                                    void* stream);
+
+/*
  * Exact O(T) chunked-state KATA-Sigma-g forward: the three steps of
  * kata_fwd_chunked on the summed feature psi_S, whose state has the single
  * factor's size: S [B,H,p*p,dv] and z [B,H,p*p] fp32 (p = d/groups), row

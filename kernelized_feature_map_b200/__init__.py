@@ -25,6 +25,8 @@ The computation lives in ``libkata.so`` (hand-written CUDA behind the C ABI of
 * :func:`kata_fwd_sg_quadratic`, :func:`kata_fwd_sg_chunked`,
   :func:`kata_decode_step_sg` -- KATA-Sigma-g, summed PSD factors (weight
   sum_{j,l} (q^j . k^l)^2): flash-style and chunked forward, decode;
+  :func:`kata_fwd_sg_quadratic_train`, :func:`kata_bwd_sg_quadratic`,
+  :func:`kata_attention_sg` -- its training forward and backward;
 * :func:`kata_fwd_mg_quadratic_train`, :func:`kata_bwd_mg_quadratic`,
   :func:`kata_attention_mg` -- the same for KATA-Mg ([B,H,T,d]);
 * :func:`kata_fwd_linear_chunked`, :func:`kata_fwd_linear_chunked_sequential`
@@ -37,7 +39,8 @@ from ._abi import (KataError, kata_abi_version, kata_decode_step, kata_fwd_chunk
                    kata_fwd_quadratic_train, kata_bwd_quadratic, kata_attention, KataAttention,
                    kata_fwd_mg_quadratic_train, kata_bwd_mg_quadratic, kata_attention_mg, KataAttentionMg,
                    kata_fwd_sg_quadratic, kata_decode_step_sg, kata_fwd_sg_chunked,
-                   kata_fwd_sg_chunked_workspace_size, kata_fwd_mg_chunked, kata_fwd_mg_chunked_workspace_size,
+                   kata_fwd_sg_chunked_workspace_size, kata_fwd_sg_quadratic_train, kata_bwd_sg_quadratic,
+                   kata_attention_sg, KataAttentionSg, kata_fwd_mg_chunked, kata_fwd_mg_chunked_workspace_size,
                    kata_fwd_linear_chunked, kata_fwd_linear_chunked_sequential,
                    kata_fwd_linear_chunked_workspace_size,
                    kata_get_status, kata_set_wait_limit, lib, status_string)

@@ -47,6 +47,8 @@ SIGNATURES = {
     "kata_decode_step_mg": (_c_int, [_vp, _vp, _vp, _vp, _fp, _fp] + [_c_int] * 6 + [_vp]),
     "kata_decode_step_sg": (_c_int, [_vp, _vp, _vp, _vp, _fp, _fp] + [_c_int] * 6 + [_vp]),
     "kata_fwd_sg_chunked_workspace_size": (_c_size, [_c_int] * 7),
+    "kata_fwd_sg_quadratic_train": (_c_int, [_vp, _vp, _vp, _vp, _fp] + [_c_int] * 7 + [_vp]),
+    "kata_bwd_sg_quadratic": (_c_int, [_vp] * 9 + [_c_int] * 7 + [_vp, _c_size, _vp]),
     "kata_fwd_sg_chunked": (_c_int, [_vp, _vp, _vp, _vp] + [_c_int] * 8 + [_fp, _fp, _fp, _fp, _vp, _c_size, _vp]),
     "kata_get_status": (_c_int, [_vp]),
     "kata_status_string": (ctypes.c_char_p, [_c_int]),
@@ -405,6 +407,60 @@ class KataAttentionMg(torch.autograd.Function):
 def kata_attention_mg(q, k, v, groups):
     """Differentiable KATA-Mg attention, q,k [B,H,T,d], v [B,H,T,dv], groups > 1."""
     return KataAttentionMg.apply(q, k, v, groups)
+
+
+def kata_fwd_sg_quadratic_train(q, k, v, groups, o=None, D=None, stream=None):
+    """KATA-Sigma-g forward ([B,H,T,d], groups > 1) that also returns each row's denominator."""
+    B, H, T, d = q.shape
+    dv = v.shape[-1]
+    if o is None:
+        o = torch.empty((B, H, T, dv), dtype=q.dtype, device=q.device)
+    if D is None:
+        D = torch.empty((B, H, T), dtype=torch.float32, device=q.device)
+    _check("kata_fwd_sg_quadratic_train", lib().kata_fwd_sg_quadratic_train(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), _dev(D, "D"), B, H, T, d, int(groups), dv,
+        _dtype_code(q), _stream_ptr(stream)))
+    return o, D
+
+
+def kata_bwd_sg_quadratic(q, k, v, o, D, dO, groups, workspace=None, stream=None):
+    """Gradients (dq, dk, dv) of the KATA-Sigma-g forward from its o and D."""
+    B, H, T, d = q.shape
+    dvw = v.shape[-1]
+    dq = torch.empty_like(q)
+    dk = torch.empty_like(k)
+    dv = torch.empty_like(v)
+    need = int(lib().kata_bwd_quadratic_workspace_size(B, H, T, d // int(groups), dvw, _dtype_code(q)))
+    if workspace is None:
+        workspace = torch.empty(max(256, need), dtype=torch.uint8, device=q.device)
+    _check("kata_bwd_sg_quadratic", lib().kata_bwd_sg_quadratic(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), _dev(D, "D"), _dev(dO, "dO"), _dev(dq, "dq"),
+        _dev(dk, "dk"), _dev(dv, "dv"), B, H, T, d, int(groups), dvw, _dtype_code(q), _dev(workspace, "workspace"),
+        workspace.numel(), _stream_ptr(stream)))
+    return dq, dk, dv
+
+
+class KataAttentionSg(torch.autograd.Function):
+    """Autograd wrapper of the KATA-Sigma-g forward and backward (marshalling only)."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, groups):
+        q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+        o, D = kata_fwd_sg_quadratic_train(q, k, v, groups)
+        ctx.groups = int(groups)
+        ctx.save_for_backward(q, k, v, o, D)
+        return o
+
+    @staticmethod
+    def backward(ctx, dO):
+        q, k, v, o, D = ctx.saved_tensors
+        dq, dk, dv = kata_bwd_sg_quadratic(q, k, v, o, D, dO.contiguous(), ctx.groups)
+        return dq, dk, dv, None
+
+
+def kata_attention_sg(q, k, v, groups):
+    """Differentiable KATA-Sigma-g attention, q,k [B,H,T,d], v [B,H,T,dv], groups > 1."""
+    return KataAttentionSg.apply(q, k, v, groups)
 
 
 def kata_fwd_mg_quadratic(q, k, v, groups, layout="bhtd", o=None, stream=None):

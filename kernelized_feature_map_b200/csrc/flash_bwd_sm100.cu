@@ -167,6 +167,20 @@ __device__ __forceinline__ void grad_pairs(const uint32_t (&s)[16], const uint32
 }
 
 // 16 fp32 values -> 16 bf16 at dst (32 bytes, 16-byte aligned)
+// The 16 bf16 values at src_row added into the fp32 row r (bf16 -> fp32 is
+// a 16-bit shift, exact): for a gradient another pass has already written
+// part of (KATA-Mg's dV; KATA-Sigma-g's dQ, dK and dV).
+__device__ __forceinline__ void add_row16(const __nv_bfloat16* src_row, uint32_t (&r)[16]) {
+  const uint4* old = reinterpret_cast<const uint4*>(src_row);
+  const uint4 a = old[0], b = old[1];
+  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+  for (int x = 0; x < 8; ++x) {
+    r[2 * x] = __float_as_uint(__uint_as_float(r[2 * x]) + __uint_as_float(w[x] << 16));
+    r[2 * x + 1] = __float_as_uint(__uint_as_float(r[2 * x + 1]) + __uint_as_float(w[x] & 0xffff0000u));
+  }
+}
+
 __device__ __forceinline__ void store_row16(__nv_bfloat16* dst_row, const uint32_t (&r)[16]) {
   uint4* dst = reinterpret_cast<uint4*>(dst_row);
   dst[0] = make_uint4(pack_bf16x2(__uint_as_float(r[0]), __uint_as_float(r[1])),
@@ -200,7 +214,8 @@ template <int p>
 __global__ void __launch_bounds__(kBwThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                  const float2* __restrict__ rowc, __nv_bfloat16* __restrict__ dq, int T, int BH, int ld, WaitCtl wc) {
+                  const float2* __restrict__ rowc, __nv_bfloat16* __restrict__ dq, int T, int BH, int ld,
+                  int dq_accumulate, WaitCtl wc) {
   using C = BwCfg<p>;
   using L = DqSmem<p>;
   extern __shared__ uint8_t smem_raw[];
@@ -422,8 +437,13 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       tc_fence_before();
       mbar_arrive(acc_free);
       if (kq == 0 && row < T) {
-        store_row16(dq + ((size_t)bh * T + row) * ld, r0);
-        if constexpr (p == 32) store_row16(dq + ((size_t)bh * T + row) * ld + 16, r1);
+        __nv_bfloat16* dqr = dq + ((size_t)bh * T + row) * ld;
+        if (dq_accumulate) {
+          add_row16(dqr, r0);
+          if constexpr (p == 32) add_row16(dqr + 16, r1);
+        }
+        store_row16(dqr, r0);
+        if constexpr (p == 32) store_row16(dqr + 16, r1);
       }
       gs += nkv;
     }
@@ -456,7 +476,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const float2* __restrict__ rowc, __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
-                    int T, int BH, int ld, int dv_accumulate, WaitCtl wc) {
+                    int T, int BH, int ld, int dv_accumulate, int dk_accumulate, WaitCtl wc) {
   using C = BwCfg<p>;
   using L = DkvSmem<p>;
   extern __shared__ uint8_t smem_raw[];
@@ -716,18 +736,13 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       if (row < T) {
         const size_t r0 = (size_t)bh * T + row;
         __nv_bfloat16* dvr = dv + r0 * kBwDV + 16 * kq;
-        if (dv_accumulate) {  // another group's dV is already there
-          const uint4* old = reinterpret_cast<const uint4*>(dvr);
-          const uint4 a = old[0], b = old[1];
-          const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-#pragma unroll
-          for (int x = 0; x < 8; ++x) {  // bf16 -> fp32 is a 16-bit shift (exact)
-            rv[2 * x] = __float_as_uint(__uint_as_float(rv[2 * x]) + __uint_as_float(w[x] << 16));
-            rv[2 * x + 1] = __float_as_uint(__uint_as_float(rv[2 * x + 1]) + __uint_as_float(w[x] & 0xffff0000u));
-          }
-        }
+        if (dv_accumulate) add_row16(dvr, rv);  // another pass's dV is already there
         store_row16(dvr, rv);
         if (kq == 0) {
+          if (dk_accumulate) {
+            add_row16(dk + r0 * ld, rk0);
+            if constexpr (p == 32) add_row16(dk + r0 * ld + 16, rk1);
+          }
           store_row16(dk + r0 * ld, rk0);
           if constexpr (p == 32) store_row16(dk + r0 * ld + 16, rk1);
         }
@@ -747,7 +762,8 @@ __global__ void __launch_bounds__(kBwThreads, 1)
 template <int p>
 static cudaError_t launch_bwd_t(const void* q, const void* k, const void* v, const void* o, const float* D,
                                 const void* dO, void* dq, void* dk, void* dv, int BH, int T, int ld, bool rows_ready,
-                                bool dv_accumulate, void* ws, const WaitCtl& wc, cudaStream_t st) {
+                                bool dv_accumulate, bool dq_accumulate, bool dk_accumulate, void* ws,
+                                const WaitCtl& wc, cudaStream_t st) {
   float2* rowc = static_cast<float2*>(ws);
   const long long rows = (long long)BH * T;
   cudaError_t e = cudaSuccess;
@@ -776,11 +792,11 @@ static cudaError_t launch_bwd_t(const void* q, const void* k, const void* v, con
   const long items = (long)grid.x * BH;
   const int pgrid = (int)(items < num_sms ? items : num_sms);
   kq<<<pgrid, kBwThreads, DqSmem<p>::kBytes, st>>>(tq, tk, tv, tdo, rowc, static_cast<__nv_bfloat16*>(dq), T, BH, ld,
-                                                    wc);
+                                                    dq_accumulate ? 1 : 0, wc);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   kkv<<<pgrid, kBwThreads, DkvSmem<p>::kBytes, st>>>(tq, tk, tv, tdo, rowc, static_cast<__nv_bfloat16*>(dk),
                                                       static_cast<__nv_bfloat16*>(dv), T, BH, ld, dv_accumulate ? 1 : 0,
-                                                      wc);
+                                                      dk_accumulate ? 1 : 0, wc);
   return cudaGetLastError();
 }
 
@@ -793,11 +809,14 @@ size_t flash_bwd_workspace_bytes(int BH, int T, int dv) {
 
 cudaError_t launch_flash_bwd_sm100(const void* q, const void* k, const void* v, const void* o, const float* D,
                                    const void* dO, void* dq, void* dk, void* dv, int BH, int T, int p, int ld,
-                                   bool rows_ready, bool dv_accumulate, void* ws, const WaitCtl& wc, cudaStream_t st) {
+                                   bool rows_ready, bool dv_accumulate, bool dq_accumulate, bool dk_accumulate,
+                                   void* ws, const WaitCtl& wc, cudaStream_t st) {
   if (p == 16)
-    return launch_bwd_t<16>(q, k, v, o, D, dO, dq, dk, dv, BH, T, ld, rows_ready, dv_accumulate, ws, wc, st);
+    return launch_bwd_t<16>(q, k, v, o, D, dO, dq, dk, dv, BH, T, ld, rows_ready, dv_accumulate, dq_accumulate,
+                            dk_accumulate, ws, wc, st);
   if (p == 32)
-    return launch_bwd_t<32>(q, k, v, o, D, dO, dq, dk, dv, BH, T, ld, rows_ready, dv_accumulate, ws, wc, st);
+    return launch_bwd_t<32>(q, k, v, o, D, dO, dq, dk, dv, BH, T, ld, rows_ready, dv_accumulate, dq_accumulate,
+                            dk_accumulate, ws, wc, st);
   return cudaErrorInvalidValue;
 }
 

@@ -491,11 +491,11 @@ cudaError_t launch_flash_mg_sm100(const void* q, const void* k, const void* v, v
   return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_flash_sg_sm100(const void* q, const void* k, const void* v, void* o, int B, int H, int T, int p,
-                                  int groups, bool bthd, const WaitCtl& wc, cudaStream_t st) {
-  if (p == 16 && groups == 2) return launch_flash_mg_t<16, 2, true>(q, k, v, o, nullptr, B, H, T, bthd, wc, st);
-  if (p == 16 && groups == 4) return launch_flash_mg_t<16, 4, true>(q, k, v, o, nullptr, B, H, T, bthd, wc, st);
-  if (p == 32 && groups == 2) return launch_flash_mg_t<32, 2, true>(q, k, v, o, nullptr, B, H, T, bthd, wc, st);
+cudaError_t launch_flash_sg_sm100(const void* q, const void* k, const void* v, void* o, float* D_out, int B, int H,
+                                  int T, int p, int groups, bool bthd, const WaitCtl& wc, cudaStream_t st) {
+  if (p == 16 && groups == 2) return launch_flash_mg_t<16, 2, true>(q, k, v, o, D_out, B, H, T, bthd, wc, st);
+  if (p == 16 && groups == 4) return launch_flash_mg_t<16, 4, true>(q, k, v, o, D_out, B, H, T, bthd, wc, st);
+  if (p == 32 && groups == 2) return launch_flash_mg_t<32, 2, true>(q, k, v, o, D_out, B, H, T, bthd, wc, st);
   return cudaErrorInvalidValue;
 }
 

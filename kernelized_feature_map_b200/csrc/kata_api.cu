@@ -461,7 +461,8 @@ KATA_API kata_status_t kata_bwd_quadratic(const void* q, const void* k, const vo
     if (!aligned16(ptr)) return KATA_ERR_MISALIGNED;
   if (!workspace || workspace_bytes < flash_bwd_workspace_bytes(B * H, T, dv_width)) return KATA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return KATA_ERR_MISALIGNED;
-  return from_cuda(launch_flash_bwd_sm100(q, k, v, o, D, dO, dq, dk, dv, B * H, T, p, p, false, false, workspace,
+  return from_cuda(launch_flash_bwd_sm100(q, k, v, o, D, dO, dq, dk, dv, B * H, T, p, p, false, false, false, false,
+                                          workspace,
                                           wait_ctl(), static_cast<cudaStream_t>(stream)));
 }
 
@@ -565,7 +566,7 @@ KATA_API kata_status_t kata_fwd_sg_quadratic(const void* q, const void* k, const
   if (T == 0) return KATA_OK;
   if (!q || !k || !v || !o) return KATA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return KATA_ERR_MISALIGNED;
-  return from_cuda(launch_flash_sg_sm100(q, k, v, o, B, H, T, p, groups, layout == KATA_LAYOUT_BTHD, wait_ctl(),
+  return from_cuda(launch_flash_sg_sm100(q, k, v, o, nullptr, B, H, T, p, groups, layout == KATA_LAYOUT_BTHD, wait_ctl(),
                                          static_cast<cudaStream_t>(stream)));
 }
 
@@ -605,8 +606,55 @@ KATA_API kata_status_t kata_bwd_mg_quadratic(const void* q, const void* k, const
     const size_t off = (size_t)j * p * 2;  // bytes
     cudaError_t e = launch_flash_bwd_sm100(static_cast<const char*>(q) + off, static_cast<const char*>(k) + off, v, o, D,
                                            dO, static_cast<char*>(dq) + off, static_cast<char*>(dk) + off, dv, B * H,
-                                           T, p, d, j > 0, j > 0, workspace, wait_ctl(), st);
+                                           T, p, d, j > 0, j > 0, false, false, workspace, wait_ctl(), st);
     if (e != cudaSuccess) return from_cuda(e);
+  }
+  return KATA_OK;
+}
+
+KATA_API kata_status_t kata_fwd_sg_quadratic_train(const void* q, const void* k, const void* v, void* o, float* D,
+                                                   int B, int H, int T, int d, int groups, int dv,
+                                                   kata_dtype_t dtype, void* stream) {
+  int p = 0;
+  kata_status_t s = check_mg(B, H, T, d, groups, dv, dtype, &p);
+  if (s != KATA_OK) return s;
+  if (dtype != KATA_BF16 || groups < 2) return KATA_ERR_UNSUPPORTED;
+  if (T == 0) return KATA_OK;
+  if (!q || !k || !v || !o || !D) return KATA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(D)) return KATA_ERR_MISALIGNED;
+  return from_cuda(launch_flash_sg_sm100(q, k, v, o, D, B, H, T, p, groups, false, wait_ctl(),
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+KATA_API kata_status_t kata_bwd_sg_quadratic(const void* q, const void* k, const void* v, const void* o,
+                                             const float* D, const void* dO, void* dq, void* dk, void* dv, int B,
+                                             int H, int T, int d, int groups, int dv_width, kata_dtype_t dtype,
+                                             void* workspace, size_t workspace_bytes, void* stream) {
+  int p = 0;
+  kata_status_t s = check_mg(B, H, T, d, groups, dv_width, dtype, &p);
+  if (s != KATA_OK) return s;
+  if (dtype != KATA_BF16 || groups < 2) return KATA_ERR_UNSUPPORTED;
+  if (T == 0) return KATA_OK;
+  for (const void* ptr : {q, k, v, o, (const void*)D, dO, (const void*)dq, (const void*)dk, (const void*)dv})
+    if (!ptr) return KATA_ERR_INVALID_ARG;
+  for (const void* ptr : {q, k, v, o, (const void*)D, dO, (const void*)dq, (const void*)dk, (const void*)dv})
+    if (!aligned16(ptr)) return KATA_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < flash_bwd_workspace_bytes(B * H, T, dv_width)) return KATA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return KATA_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // one pass per (query group j, key group l) with that pair's scores
+  // q^j . k^l: dq^j sums over l, dk^l over j and dv over every pair (the
+  // weight is linear in the pairs' squares); the per-row constants are
+  // computed in the first pass
+  for (int j = 0; j < groups; ++j) {
+    for (int l = 0; l < groups; ++l) {
+      const size_t oj = (size_t)j * p * 2, ol = (size_t)l * p * 2;  // bytes
+      const bool first = j == 0 && l == 0;
+      cudaError_t e = launch_flash_bwd_sm100(static_cast<const char*>(q) + oj, static_cast<const char*>(k) + ol, v, o,
+                                             D, dO, static_cast<char*>(dq) + oj, static_cast<char*>(dk) + ol, dv,
+                                             B * H, T, p, d, !first, !first, l > 0, j > 0, workspace, wait_ctl(), st);
+      if (e != cudaSuccess) return from_cuda(e);
+    }
   }
   return KATA_OK;
 }

@@ -90,11 +90,13 @@ cudaError_t launch_flash_sm100(const void* q, const void* k, const void* v, void
 // denominator [B*H, T] fp32; ws holds flash_bwd_workspace_bytes().
 // q, k, dq and dk rows are ld elements apart (ld = p for [B*H, T, p]; one
 // group of a [B*H, T, d] tensor with ld = d); with rows_ready the per-row
-// constants already in ws are reused; with dv_accumulate dv is added to.
+// constants already in ws are reused; with dv_accumulate (dq_accumulate,
+// dk_accumulate) the pass's dv (dq, dk) is added to what is there.
 size_t flash_bwd_workspace_bytes(int BH, int T, int dv);
 cudaError_t launch_flash_bwd_sm100(const void* q, const void* k, const void* v, const void* o, const float* D,
                                    const void* dO, void* dq, void* dk, void* dv, int BH, int T, int p, int ld,
-                                   bool rows_ready, bool dv_accumulate, void* ws, const WaitCtl& wc, cudaStream_t st);
+                                   bool rows_ready, bool dv_accumulate, bool dq_accumulate, bool dk_accumulate,
+                                   void* ws, const WaitCtl& wc, cudaStream_t st);
 
 // flash_mg_sm100.cu -- tcgen05 flash-style KATA-Mg forward (bf16 inputs,
 // dv = 64) with `groups` PSD factors of width p per head; D_out (nullable,
@@ -102,8 +104,8 @@ cudaError_t launch_flash_bwd_sm100(const void* q, const void* k, const void* v, 
 bool flash_mg_sm100_supports(int p, int groups, int dv);
 // KATA-Sigma-g (summed factors): the same kernel over all (query group, key
 // group) score pairs; the (p, groups, dv) of flash_mg_sm100_supports.
-cudaError_t launch_flash_sg_sm100(const void* q, const void* k, const void* v, void* o, int B, int H, int T, int p,
-                                  int groups, bool bthd, const WaitCtl& wc, cudaStream_t st);
+cudaError_t launch_flash_sg_sm100(const void* q, const void* k, const void* v, void* o, float* D_out, int B, int H,
+                                  int T, int p, int groups, bool bthd, const WaitCtl& wc, cudaStream_t st);
 cudaError_t launch_flash_mg_sm100(const void* q, const void* k, const void* v, void* o, float* D_out, int B, int H, int T,
                                   int p, int groups, bool bthd, const WaitCtl& wc, cudaStream_t st);
 
