@@ -258,6 +258,30 @@ kata_status_t kata_bwd_quadratic(const void* q, const void* k, const void* v, co
                                  void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Training on the chunked path (bf16, p = 16, dv = 64, [B,H,T,*]): an O(T)
+ * forward and backward.  kata_fwd_chunked_train is kata_fwd_chunked (no
+ * initial or final state) that also writes each row's denominator D
+ * [B,H,T] fp32.  kata_bwd_chunked gives the gradients (dq, dk, dv; layouts
+ * of q, k, v; bf16) of the same function as kata_bwd_quadratic, from o, D
+ * and dO: the pairs inside each 128-token chunk with the flash backward
+ * kernels on their diagonal tiles, the pairs across chunks through the
+ * per-chunk states of the forward (S before each chunk) and of the gradient
+ * (sum over later tokens of psi(q_t) [dN_t | dD_t]^T) and their scans, so
+ * that work and memory are linear in T.  Workspace:
+ * kata_bwd_chunked_workspace_size() bytes, 256-byte aligned (8 bytes per row
+ * plus two 65 x 144 fp32 records per 128-token chunk of every (b,h)).
+ * Other sizes: KATA_ERR_UNSUPPORTED.  Streams and errors as above.
+ */
+kata_status_t kata_fwd_chunked_train(const void* q, const void* k, const void* v, void* o, float* D,
+                                     int B, int H, int T, int p, int dv, int C, kata_dtype_t dtype,
+                                     void* workspace, size_t workspace_bytes, void* stream);
+size_t kata_bwd_chunked_workspace_size(int B, int H, int T, int p, int dv, kata_dtype_t dtype);
+kata_status_t kata_bwd_chunked(const void* q, const void* k, const void* v, const void* o,
+                               const float* D, const void* dO, void* dq, void* dk, void* dv,
+                               int B, int H, int T, int p, int dv_width, kata_dtype_t dtype,
+                               void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Training with KATA-Mg ([B,H,T,*] layout, bf16, dv = 64, the (p, groups)
  * of kata_fwd_mg_quadratic with groups > 1): the Mg forward that also saves
  * D [B,H,T] fp32, and its backward pass.  With w = sum_j (q^j . k^j)^2 the

@@ -21,6 +21,8 @@ The computation lives in ``libkata.so`` (hand-written CUDA behind the C ABI of
 * :func:`kata_fwd_quadratic_train`, :func:`kata_bwd_quadratic` -- the forward
   that also returns the denominators, and the backward pass;
   :func:`kata_attention` wraps them as an autograd function;
+  :func:`kata_fwd_chunked_train`, :func:`kata_bwd_chunked`,
+  :func:`kata_attention_chunked` -- the same on the O(T) chunked path;
 * :func:`kata_fwd_mg_chunked` -- KATA-Mg on the exact O(T) chunked path;
 * :func:`kata_fwd_sg_quadratic`, :func:`kata_fwd_sg_chunked`,
   :func:`kata_decode_step_sg` -- KATA-Sigma-g, summed PSD factors (weight
@@ -37,6 +39,7 @@ from ._abi import (KataError, kata_abi_version, kata_decode_step, kata_fwd_chunk
                    kata_fwd_chunked_noalloc, kata_fwd_chunked_sequential, kata_fwd_chunked_workspace_size,
                    kata_fwd_quadratic, kata_fwd_mg_quadratic, kata_decode_step_mg, parallel_kata_attn,
                    kata_fwd_quadratic_train, kata_bwd_quadratic, kata_attention, KataAttention,
+                   kata_fwd_chunked_train, kata_bwd_chunked, kata_attention_chunked, KataAttentionChunked,
                    kata_fwd_mg_quadratic_train, kata_bwd_mg_quadratic, kata_attention_mg, KataAttentionMg,
                    kata_fwd_sg_quadratic, kata_decode_step_sg, kata_fwd_sg_chunked,
                    kata_fwd_sg_chunked_workspace_size, kata_fwd_sg_quadratic_train, kata_bwd_sg_quadratic,

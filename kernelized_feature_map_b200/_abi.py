@@ -39,6 +39,9 @@ SIGNATURES = {
     "kata_bwd_quadratic_workspace_size": (_c_size, [_c_int] * 6),
     "kata_bwd_quadratic": (_c_int, [_vp] * 9 + [_c_int] * 6 + [_vp, _c_size, _vp]),
     "kata_fwd_mg_quadratic": (_c_int, [_vp, _vp, _vp, _vp] + [_c_int] * 8 + [_vp]),
+    "kata_fwd_chunked_train": (_c_int, [_vp, _vp, _vp, _vp, _fp] + [_c_int] * 7 + [_vp, _c_size, _vp]),
+    "kata_bwd_chunked_workspace_size": (_c_size, [_c_int] * 6),
+    "kata_bwd_chunked": (_c_int, [_vp] * 9 + [_c_int] * 6 + [_vp, _c_size, _vp]),
     "kata_fwd_mg_quadratic_train": (_c_int, [_vp, _vp, _vp, _vp, _fp] + [_c_int] * 7 + [_vp]),
     "kata_fwd_sg_quadratic": (_c_int, [_vp, _vp, _vp, _vp] + [_c_int] * 8 + [_vp]),
     "kata_fwd_mg_chunked_workspace_size": (_c_size, [_c_int] * 8),
@@ -353,6 +356,63 @@ def kata_fwd_sg_quadratic(q, k, v, groups, layout="bhtd", o=None, stream=None):
         _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), B, H, T, d, int(groups), dv, code,
         _dtype_code(q), _stream_ptr(stream)))
     return o
+
+
+def kata_fwd_chunked_train(q, k, v, C=64, o=None, D=None, workspace=None, stream=None):
+    """The chunked forward (bf16, p=16, dv=64) that also returns each row's denominator."""
+    B, H, T, p = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    if o is None:
+        o = torch.empty((B, H, T, dv), dtype=q.dtype, device=dev)
+    if D is None:
+        D = torch.empty((B, H, T), dtype=torch.float32, device=dev)
+    need = kata_fwd_chunked_workspace_size(B, H, T, p, dv, C, q.dtype)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("kata_fwd_chunked_train", lib().kata_fwd_chunked_train(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), _dev(D, "D"), B, H, T, p, dv, C, _dtype_code(q),
+        _opt(workspace, "workspace"), ws_bytes, _stream_ptr(stream)))
+    return o, D
+
+
+def kata_bwd_chunked(q, k, v, o, D, dO, workspace=None, stream=None):
+    """Gradients (dq, dk, dv) by the O(T) chunked backward, from o and D."""
+    B, H, T, p = q.shape
+    dvw = v.shape[-1]
+    dq = torch.empty_like(q)
+    dk = torch.empty_like(k)
+    dv = torch.empty_like(v)
+    need = int(lib().kata_bwd_chunked_workspace_size(B, H, T, p, dvw, _dtype_code(q)))
+    if workspace is None:
+        workspace = torch.empty(max(256, need), dtype=torch.uint8, device=q.device)
+    _check("kata_bwd_chunked", lib().kata_bwd_chunked(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), _dev(D, "D"), _dev(dO, "dO"), _dev(dq, "dq"),
+        _dev(dk, "dk"), _dev(dv, "dv"), B, H, T, p, dvw, _dtype_code(q), _dev(workspace, "workspace"),
+        workspace.numel(), _stream_ptr(stream)))
+    return dq, dk, dv
+
+
+class KataAttentionChunked(torch.autograd.Function):
+    """Autograd wrapper of the chunked forward and backward (marshalling only)."""
+
+    @staticmethod
+    def forward(ctx, q, k, v):
+        q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+        o, D = kata_fwd_chunked_train(q, k, v)
+        ctx.save_for_backward(q, k, v, o, D)
+        return o
+
+    @staticmethod
+    def backward(ctx, dO):
+        q, k, v, o, D = ctx.saved_tensors
+        return kata_bwd_chunked(q, k, v, o, D, dO.contiguous())
+
+
+def kata_attention_chunked(q, k, v):
+    """Differentiable KATA attention on the O(T) chunked path, q,k [B,H,T,16], v [B,H,T,64] (bf16)."""
+    return KataAttentionChunked.apply(q, k, v)
 
 
 def kata_fwd_mg_quadratic_train(q, k, v, groups, o=None, D=None, stream=None):

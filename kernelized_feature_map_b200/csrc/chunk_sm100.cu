@@ -290,8 +290,8 @@ __global__ void __launch_bounds__(kReadThreads, 1)
     chunk_readout_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                          const float* __restrict__ ws, const float* __restrict__ S0, const float* __restrict__ z0,
-                         float* __restrict__ S_out, float* __restrict__ z_out, int T, int Ls, int G,
-                         long long record_floats, WaitCtl wc) {
+                         float* __restrict__ S_out, float* __restrict__ z_out, float* __restrict__ D_out, int T,
+                         int Ls, int G, long long record_floats, WaitCtl wc) {
   using L = ReadSmem<NG>;
   constexpr int kReadStages = L::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -458,6 +458,7 @@ __global__ void __launch_bounds__(kReadThreads, 1)
       if (co + 2 < n_chunks) mbar_arrive(state_full);
       if (m == 0) KATA_TRACE(chunk, co, 14);
       const float D = __uint_as_float(db);
+      if (D_out != nullptr && h == 0 && t0 + co * kTile + m < T) D_out[(size_t)bh * T + t0 + co * kTile + m] = D;
       const float inv = D > 0.f ? 1.f / D : 0.f;
       const uint64_t inv2 = f32x2(__float_as_uint(inv), __float_as_uint(inv));
       auto scaled = [&](int k) {
@@ -716,7 +717,7 @@ cudaError_t launch_state_t(const void* k, const void* v, float* ws, const ChunkP
 template <int NG>
 cudaError_t launch_readout_t(const void* q, const void* k, const void* v, void* o, const float* ws, const float* S0,
                              const float* z0, float* S_out, float* z_out, const ChunkPlan& pl, const WaitCtl& wc,
-                             cudaStream_t st) {
+                             cudaStream_t st, float* D_out = nullptr) {
   using L = ReadSmem<NG>;
   if (pl.p != 16 || pl.dv != kDV) return cudaErrorInvalidValue;
   if (!ws && pl.G != 1) return cudaErrorInvalidValue;
@@ -731,9 +732,10 @@ cudaError_t launch_readout_t(const void* q, const void* k, const void* v, void* 
   const dim3 grid(pl.G, pl.BH), block(kReadThreads);
   if (ws)  // after the state build and scan of this call: launched as the scan's programmatic dependent
     return launch_pdl(chunk_readout_kernel<NG>, grid, block, (size_t)L::kBytes, st, tq, tk, tv, to,
-                      (const float*)ws, S0, z0, S_out, z_out, pl.T, pl.Ls, pl.G, (long long)pl.record_floats, wc);
-  chunk_readout_kernel<NG><<<grid, block, L::kBytes, st>>>(tq, tk, tv, to, ws, S0, z0, S_out, z_out, pl.T, pl.Ls,
-                                                           pl.G, (long long)pl.record_floats, wc);
+                      (const float*)ws, S0, z0, S_out, z_out, D_out, pl.T, pl.Ls, pl.G, (long long)pl.record_floats,
+                      wc);
+  chunk_readout_kernel<NG><<<grid, block, L::kBytes, st>>>(tq, tk, tv, to, ws, S0, z0, S_out, z_out, D_out, pl.T,
+                                                           pl.Ls, pl.G, (long long)pl.record_floats, wc);
   return cudaGetLastError();
 }
 
@@ -746,8 +748,8 @@ cudaError_t launch_chunk_state_sm100(const void* k, const void* v, float* ws, co
 
 cudaError_t launch_chunk_readout_sm100(const void* q, const void* k, const void* v, void* o, const float* ws,
                                        const float* S0, const float* z0, float* S_out, float* z_out,
-                                       const ChunkPlan& pl, const WaitCtl& wc, cudaStream_t st) {
-  return launch_readout_t<1>(q, k, v, o, ws, S0, z0, S_out, z_out, pl, wc, st);
+                                       const ChunkPlan& pl, const WaitCtl& wc, cudaStream_t st, float* D_out) {
+  return launch_readout_t<1>(q, k, v, o, ws, S0, z0, S_out, z_out, pl, wc, st, D_out);
 }
 
 cudaError_t launch_chunk_state_sg(const void* k, const void* v, float* ws, const ChunkPlan& pl, int groups,

@@ -215,7 +215,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                   const float2* __restrict__ rowc, __nv_bfloat16* __restrict__ dq, int T, int BH, int ld,
-                  int dq_accumulate, WaitCtl wc) {
+                  int dq_accumulate, int diag_only, WaitCtl wc) {
   using C = BwCfg<p>;
   using L = DqSmem<p>;
   extern __shared__ uint8_t smem_raw[];
@@ -284,7 +284,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         mbar_arrive_expect_tx(q_full + qb, C::kVBytes + C::kQKBytes);
         tma_load_3d(smem + L::offDO + qb * C::kVBytes, &tm_do, q_full + qb, 0, tile * kBw, bh);
         tma_load_3d(smem + L::offQ + qb * C::kQKBytes, &tm_q, q_full + qb, 0, tile * kBw, bh);
-        for (int j = 0; j <= tile; ++j, ++rg) {
+        for (int j = diag_only ? tile : 0; j <= tile; ++j, ++rg) {
           const int st = (int)(rg % kBwStages);
           if (!mbar_wait(kv_empty + st, (int)((rg / kBwStages) & 1) ^ 1, env)) {
             ok = false;
@@ -323,7 +323,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     int nq = 0, acc_cnt = 0;
     bool ok = true;
     for (int it = my_item(nq); ok && it >= 0; it = my_item(++nq)) {
-      const int qb = nq & 1, nkv = item_tile(it) + 1;
+      const int qb = nq & 1, nkv = diag_only ? 1 : item_tile(it) + 1;
       if (!mbar_wait_w(q_full + qb, (nq >> 1) & 1, env) ||
           !mbar_wait_w(kv_full + gs % kBwStages, (gs / kBwStages) & 1, env) ||
           (gs > 0 && !mbar_wait_w(s_read, (gs - 1) & 1, env))) {
@@ -378,7 +378,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     int nq = 0, acc_cnt = 0;
     bool ok = true;
     for (int it = my_item(nq); ok && it >= 0; it = my_item(++nq)) {
-      const int tile = item_tile(it), bh = it % BH, nkv = tile + 1;
+      const int tile = item_tile(it), bh = it % BH, nkv = diag_only ? 1 : tile + 1;
       const int row = tile * kBw + quarter * 32 + lane;
       const float2 rc = row < T ? rowc[(size_t)bh * T + row] : make_float2(0.f, 0.f);  // (-delta, 1/D)
       for (int j = 0; j < nkv; ++j) {
@@ -476,7 +476,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const float2* __restrict__ rowc, __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
-                    int T, int BH, int ld, int dv_accumulate, int dk_accumulate, WaitCtl wc) {
+                    int T, int BH, int ld, int dv_accumulate, int dk_accumulate, int diag_only, WaitCtl wc) {
   using C = BwCfg<p>;
   using L = DkvSmem<p>;
   extern __shared__ uint8_t smem_raw[];
@@ -549,7 +549,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         mbar_arrive_expect_tx(kv_full + kb, C::kVBytes + C::kQKBytes);
         tma_load_3d(smem + L::offV + kb * C::kVBytes, &tm_v, kv_full + kb, 0, tile * kBw, bh);
         tma_load_3d(smem + L::offK + kb * C::kQKBytes, &tm_k, kv_full + kb, 0, tile * kBw, bh);
-        for (int i = tile; i < n_tiles; ++i, ++rg) {
+        for (int i = tile; i < (diag_only ? tile + 1 : n_tiles); ++i, ++rg) {
           const int st = (int)(rg % kBwStages);
           if (!mbar_wait(q_empty + st, (int)((rg / kBwStages) & 1) ^ 1, env)) {
             ok = false;
@@ -589,7 +589,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     int nq = 0, acc_cnt = 0;
     bool ok = true;
     for (int it = my_item(nq); ok && it >= 0; it = my_item(++nq)) {
-      const int tile = it / BH, kb = nq & 1, cnt = n_tiles - tile;
+      const int tile = it / BH, kb = nq & 1, cnt = diag_only ? 1 : n_tiles - tile;
       if (!mbar_wait_w(kv_full + kb, (nq >> 1) & 1, env) ||
           !mbar_wait_w(q_full + gs % kBwStages, (int)((gs / kBwStages) & 1), env) ||
           (gs > 0 && !mbar_wait_w(s_read, (int)((gs - 1) & 1), env))) {
@@ -657,7 +657,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     int nq = 0, acc_cnt = 0;
     bool ok = true;
     for (int it = my_item(nq); ok && it >= 0; it = my_item(++nq)) {
-      const int tile = it / BH, bh = it % BH, cnt = n_tiles - tile;
+      const int tile = it / BH, bh = it % BH, cnt = diag_only ? 1 : n_tiles - tile;
       for (int n = 0; n < cnt; ++n) {
         const int g = gs + n;
         // (-delta, 1/D) of this warp's 32 queries, one per lane (0 past T)
@@ -762,8 +762,8 @@ __global__ void __launch_bounds__(kBwThreads, 1)
 template <int p>
 static cudaError_t launch_bwd_t(const void* q, const void* k, const void* v, const void* o, const float* D,
                                 const void* dO, void* dq, void* dk, void* dv, int BH, int T, int ld, bool rows_ready,
-                                bool dv_accumulate, bool dq_accumulate, bool dk_accumulate, void* ws,
-                                const WaitCtl& wc, cudaStream_t st) {
+                                bool dv_accumulate, bool dq_accumulate, bool dk_accumulate, bool diag_only,
+                                void* ws, const WaitCtl& wc, cudaStream_t st) {
   float2* rowc = static_cast<float2*>(ws);
   const long long rows = (long long)BH * T;
   cudaError_t e = cudaSuccess;
@@ -792,11 +792,11 @@ static cudaError_t launch_bwd_t(const void* q, const void* k, const void* v, con
   const long items = (long)grid.x * BH;
   const int pgrid = (int)(items < num_sms ? items : num_sms);
   kq<<<pgrid, kBwThreads, DqSmem<p>::kBytes, st>>>(tq, tk, tv, tdo, rowc, static_cast<__nv_bfloat16*>(dq), T, BH, ld,
-                                                    dq_accumulate ? 1 : 0, wc);
+                                                    dq_accumulate ? 1 : 0, diag_only ? 1 : 0, wc);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   kkv<<<pgrid, kBwThreads, DkvSmem<p>::kBytes, st>>>(tq, tk, tv, tdo, rowc, static_cast<__nv_bfloat16*>(dk),
                                                       static_cast<__nv_bfloat16*>(dv), T, BH, ld, dv_accumulate ? 1 : 0,
-                                                      dk_accumulate ? 1 : 0, wc);
+                                                      dk_accumulate ? 1 : 0, diag_only ? 1 : 0, wc);
   return cudaGetLastError();
 }
 
@@ -810,13 +810,13 @@ size_t flash_bwd_workspace_bytes(int BH, int T, int dv) {
 cudaError_t launch_flash_bwd_sm100(const void* q, const void* k, const void* v, const void* o, const float* D,
                                    const void* dO, void* dq, void* dk, void* dv, int BH, int T, int p, int ld,
                                    bool rows_ready, bool dv_accumulate, bool dq_accumulate, bool dk_accumulate,
-                                   void* ws, const WaitCtl& wc, cudaStream_t st) {
+                                   void* ws, const WaitCtl& wc, cudaStream_t st, bool diag_only) {
   if (p == 16)
     return launch_bwd_t<16>(q, k, v, o, D, dO, dq, dk, dv, BH, T, ld, rows_ready, dv_accumulate, dq_accumulate,
-                            dk_accumulate, ws, wc, st);
+                            dk_accumulate, diag_only, ws, wc, st);
   if (p == 32)
     return launch_bwd_t<32>(q, k, v, o, D, dO, dq, dk, dv, BH, T, ld, rows_ready, dv_accumulate, dq_accumulate,
-                            dk_accumulate, ws, wc, st);
+                            dk_accumulate, diag_only, ws, wc, st);
   return cudaErrorInvalidValue;
 }
 

@@ -431,6 +431,75 @@ static kata_status_t check_train(int B, int H, int T, int p, int dv, kata_dtype_
   return KATA_OK;
 }
 
+// Training on the chunked path (bf16, p = 16, dv = 64): the forward that
+// also writes D, and the O(T) backward.
+KATA_API kata_status_t kata_fwd_chunked_train(const void* q, const void* k, const void* v, void* o, float* D, int B,
+                                              int H, int T, int p, int dv, int C, kata_dtype_t dtype, void* workspace,
+                                              size_t workspace_bytes, void* stream) {
+  kata_status_t s = check_chunked_args(q, k, v, o, B, H, T, p, dv, C, dtype, nullptr, nullptr, nullptr, nullptr);
+  if (s != KATA_OK) return s;
+  if (dtype != KATA_BF16 || p != 16 || dv != 64) return KATA_ERR_UNSUPPORTED;
+  if (T == 0) return KATA_OK;
+  if (!D) return KATA_ERR_INVALID_ARG;
+  if (!aligned16(D)) return KATA_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const ChunkPlan plan = make_chunk_plan(B, H, T, p, dv, C, dtype);
+  if (plan.workspace_bytes > 0) {
+    if (!workspace || workspace_bytes < plan.workspace_bytes) return KATA_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KATA_ERR_MISALIGNED;
+  }
+  float* ws = plan.workspace_bytes > 0 ? static_cast<float*>(workspace) : nullptr;
+  const WaitCtl wc = wait_ctl();
+  cudaError_t e = cudaSuccess;
+  if (plan.G > 1) {
+    e = launch_chunk_state_sm100(k, v, ws, plan, wc, st);
+    if (e == cudaSuccess) e = launch_state_scan(ws, plan, plan.G - 1, nullptr, nullptr, nullptr, nullptr, st);
+  }
+  if (e == cudaSuccess)
+    e = launch_chunk_readout_sm100(q, k, v, o, ws, nullptr, nullptr, nullptr, nullptr, plan, wc, st, D);
+  return from_cuda(e);
+}
+
+static size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
+KATA_API size_t kata_bwd_chunked_workspace_size(int B, int H, int T, int p, int dv, kata_dtype_t dtype) {
+  if (B < 1 || H < 1 || T <= 0 || p != 16 || dv != 64 || dtype != KATA_BF16) return 0;
+  const int BH = B * H;
+  return round256(flash_bwd_workspace_bytes(BH, T, dv)) + chunk_bwd_records_bytes(BH, T);
+}
+
+KATA_API kata_status_t kata_bwd_chunked(const void* q, const void* k, const void* v, const void* o, const float* D,
+                                        const void* dO, void* dq, void* dk, void* dv, int B, int H, int T, int p,
+                                        int dv_width, kata_dtype_t dtype, void* workspace, size_t workspace_bytes,
+                                        void* stream) {
+  kata_status_t s = check_train(B, H, T, p, dv_width, dtype);
+  if (s != KATA_OK) return s;
+  if (p != 16) return KATA_ERR_UNSUPPORTED;
+  if (T == 0) return KATA_OK;
+  for (const void* ptr : {q, k, v, o, (const void*)D, dO, (const void*)dq, (const void*)dk, (const void*)dv})
+    if (!ptr) return KATA_ERR_INVALID_ARG;
+  for (const void* ptr : {q, k, v, o, (const void*)D, dO, (const void*)dq, (const void*)dk, (const void*)dv})
+    if (!aligned16(ptr)) return KATA_ERR_MISALIGNED;
+  const int BH = B * H;
+  if (!workspace || workspace_bytes < kata_bwd_chunked_workspace_size(B, H, T, p, dv_width, dtype))
+    return KATA_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KATA_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const WaitCtl wc = wait_ctl();
+  // the pairs inside each 128-token chunk: the flash backward on its diagonal
+  // tiles (which also computes the per-row constants); then the pairs across
+  // chunks through the chunk states
+  uint8_t* w8 = static_cast<uint8_t*>(workspace);
+  cudaError_t e = launch_flash_bwd_sm100(q, k, v, o, D, dO, dq, dk, dv, BH, T, p, p, false, false, false, false, w8,
+                                         wc, st, true);
+  if (e == cudaSuccess)
+    e = launch_chunk_bwd_inter_sm100(q, k, v, dO, reinterpret_cast<const float2*>(w8),
+                                     reinterpret_cast<float*>(w8 + round256(flash_bwd_workspace_bytes(BH, T, dv_width))),
+                                     dq, dk, dv, BH, T, wc, st);
+  return from_cuda(e);
+}
+
+
 KATA_API kata_status_t kata_fwd_quadratic_train(const void* q, const void* k, const void* v, void* o, float* D,
                                                 int B, int H, int T, int p, int dv, kata_dtype_t dtype,
                                                 void* stream) {

@@ -91,12 +91,14 @@ cudaError_t launch_flash_sm100(const void* q, const void* k, const void* v, void
 // q, k, dq and dk rows are ld elements apart (ld = p for [B*H, T, p]; one
 // group of a [B*H, T, d] tensor with ld = d); with rows_ready the per-row
 // constants already in ws are reused; with dv_accumulate (dq_accumulate,
-// dk_accumulate) the pass's dv (dq, dk) is added to what is there.
+// dk_accumulate) the pass's dv (dq, dk) is added to what is there; with
+// diag_only only the pairs of each 128-token tile with itself are taken (the
+// intra-chunk part of the chunked backward).
 size_t flash_bwd_workspace_bytes(int BH, int T, int dv);
 cudaError_t launch_flash_bwd_sm100(const void* q, const void* k, const void* v, const void* o, const float* D,
                                    const void* dO, void* dq, void* dk, void* dv, int BH, int T, int p, int ld,
                                    bool rows_ready, bool dv_accumulate, bool dq_accumulate, bool dk_accumulate,
-                                   void* ws, const WaitCtl& wc, cudaStream_t st);
+                                   void* ws, const WaitCtl& wc, cudaStream_t st, bool diag_only = false);
 
 // flash_mg_sm100.cu -- tcgen05 flash-style KATA-Mg forward (bf16 inputs,
 // dv = 64) with `groups` PSD factors of width p per head; D_out (nullable,
@@ -116,9 +118,12 @@ cudaError_t launch_flash_mg_sm100(const void* q, const void* k, const void* v, v
 // of the last super-chunk writes the final state S_out/z_out when non-null.
 cudaError_t launch_chunk_state_sm100(const void* k, const void* v, float* ws, const ChunkPlan& pl, const WaitCtl& wc,
                                      cudaStream_t st);
+// D_out, when not null, receives each row's denominator [B*H, T] fp32 (the
+// training forward of the chunked path).
 cudaError_t launch_chunk_readout_sm100(const void* q, const void* k, const void* v, void* o, const float* ws,
                                        const float* S0, const float* z0, float* S_out, float* z_out,
-                                       const ChunkPlan& pl, const WaitCtl& wc, cudaStream_t st);
+                                       const ChunkPlan& pl, const WaitCtl& wc, cudaStream_t st,
+                                       float* D_out = nullptr);
 // The same kernels for KATA-Sigma-g with `groups` (2 or 4) groups of 16
 // (d = 16 * groups): the summed feature on the p = 16 state, the same plan
 // and record layout.
@@ -127,6 +132,17 @@ cudaError_t launch_chunk_state_sg(const void* k, const void* v, float* ws, const
 cudaError_t launch_chunk_readout_sg(const void* q, const void* k, const void* v, void* o, const float* ws,
                                     const float* S0, const float* z0, float* S_out, float* z_out,
                                     const ChunkPlan& pl, int groups, const WaitCtl& wc, cudaStream_t st);
+
+// chunk_bwd_sm100.cu -- the inter-chunk part of the chunked backward (bf16,
+// p = 16, dv = 64, [B*H, T, *]): per-chunk state sums of the forward and of
+// the gradient, their scans, and the per-chunk gradient terms added to dq,
+// dk, dv (which the diagonal-only flash backward wrote first).  rowc is the
+// flash backward's per-row (-delta, 2/D); records needs
+// chunk_bwd_records_bytes().
+size_t chunk_bwd_records_bytes(int BH, int T);
+cudaError_t launch_chunk_bwd_inter_sm100(const void* q, const void* k, const void* v, const void* dO,
+                                         const float2* rowc, float* records, void* dq, void* dk, void* dv, int BH,
+                                         int T, const WaitCtl& wc, cudaStream_t st);
 
 // chunk_linear_sm100.cu -- first-order (linear) attention, psi(u) = u, with
 // d = 16 and dv = 64 in bf16: the same three steps with unpacked records

@@ -208,3 +208,36 @@ def test_sg_backward_matches_oracle(kata, shape):
     kata.kata_attention_sg(qa, ka, va, g).backward(to_dev(dO, "bf16"))
     torch.cuda.synchronize()
     assert torch.equal(qa.grad, dq) and torch.equal(ka.grad, dk) and torch.equal(va.grad, dv)
+
+
+# ---------------------------------------------------------------------------
+# the O(T) chunked path: forward with D, backward through the chunk states
+# ---------------------------------------------------------------------------
+
+# one chunk (no pair crosses a chunk boundary), a ragged second chunk, several
+# chunks, and enough (b,h) x chunks for many CTA waves
+@pytest.mark.parametrize("B,H,T", [(1, 2, 100), (1, 2, 200), (2, 3, 777), (4, 8, 1000), (1, 1, 4096)])
+def test_chunked_backward_matches_oracle(kata, B, H, T):
+    """Gradients of the chunked training path against the fp64 gradient
+    oracle, with the gate of the flash-path backward; the training forward's
+    o equals kata_fwd_chunked's and its D agrees with the flash forward's."""
+    import torch
+    p = 16
+    q, k, v = workloads.normal_qkv(B, H, T, p, 64, seed=520 + T, dtype="bf16")
+    dO = _dO(v.shape, 521 + T)
+    qd, kd, vd = to_dev(q, "bf16"), to_dev(k, "bf16"), to_dev(v, "bf16")
+    o, D = kata.kata_fwd_chunked_train(qd, kd, vd)
+    assert torch.equal(o, kata.kata_fwd_chunked(qd, kd, vd))
+    _, D_flash = kata.kata_fwd_quadratic_train(qd, kd, vd)
+    torch.cuda.synchronize()
+    np.testing.assert_allclose(D.cpu().numpy(), D_flash.cpu().numpy(), rtol=2e-2, atol=1e-6)
+    dq, dk, dv = kata.kata_bwd_chunked(qd, kd, vd, o, D, to_dev(dO, "bf16"))
+    torch.cuda.synchronize()
+    assert kata.kata_get_status() == 0
+    gq, gk, gv = obw.backward(q, k, v, dO)
+    errs = (_grad_err(to_np(dq), gq), _grad_err(to_np(dk), gk), _grad_err(to_np(dv), gv))
+    assert max(errs) <= GRAD_TOL, errs
+    qa, ka, va = (x.clone().requires_grad_(True) for x in (qd, kd, vd))
+    kata.kata_attention_chunked(qa, ka, va).backward(to_dev(dO, "bf16"))
+    torch.cuda.synchronize()
+    assert torch.equal(qa.grad, dq) and torch.equal(ka.grad, dk) and torch.equal(va.grad, dv)
