@@ -688,7 +688,31 @@ def run_train(args, K, torch, dev, stream, flush):
         K.kata_fwd_quadratic_train(q, k, v, o=o, D=D)
         K.kata_bwd_quadratic(q, k, v, o, D, dO, workspace=ws)
     step_ms = _time_call(step, flush, stream, 10, 3)
-    return dict(B=B, H=H, T=T, p=p, dv=dv, fwd_ms=fwd_ms, bwd_ms=bwd_ms, step_ms=step_ms)
+    out = dict(B=B, H=H, T=T, p=p, dv=dv, fwd_ms=fwd_ms, bwd_ms=bwd_ms, step_ms=step_ms)
+    # the O(T) chunked training path on the same inputs, and alone at the
+    # long context (B1 H16 T131072, where the O(T^2) backward takes seconds)
+    chunked = {}
+    for (Bc, Tc) in ((B, T), (1, 131072)):
+        if (Bc, Tc) != (B, T):
+            gen.manual_seed(98)
+            q = torch.randn((Bc, H, Tc, p), generator=gen, device=dev)
+            k = torch.randn((Bc, H, Tc, p), generator=gen, device=dev)
+            q = (q / q.norm(dim=-1, keepdim=True)).to(bf)
+            k = (k / k.norm(dim=-1, keepdim=True)).to(bf)
+            v = torch.randn((Bc, H, Tc, dv), generator=gen, device=dev).to(bf)
+            dO = torch.randn((Bc, H, Tc, dv), generator=gen, device=dev).to(bf)
+        oc = torch.empty_like(v)
+        Dc = torch.empty((Bc, H, Tc), dtype=torch.float32, device=dev)
+        wsf = torch.empty(max(256, K.kata_fwd_chunked_workspace_size(Bc, H, Tc, p, dv, 64, bf)), dtype=torch.uint8,
+                          device=dev)
+        wsb = torch.empty(max(256, int(K.lib().kata_bwd_chunked_workspace_size(Bc, H, Tc, p, dv, 1))),
+                          dtype=torch.uint8, device=dev)
+        c_fwd = _time_call(lambda: K.kata_fwd_chunked_train(q, k, v, o=oc, D=Dc, workspace=wsf), flush, stream, 5, 2)
+        c_bwd = _time_call(lambda: K.kata_bwd_chunked(q, k, v, oc, Dc, dO, workspace=wsb), flush, stream, 5, 2)
+        chunked["B%d_T%d" % (Bc, Tc)] = dict(B=Bc, H=H, T=Tc, fwd_ms=c_fwd, bwd_ms=c_bwd, step_ms=c_fwd + c_bwd)
+        del oc, Dc, wsf, wsb
+    out["chunked"] = chunked
+    return out
 
 
 # ---------------------------------------------------------------------------
@@ -1092,6 +1116,12 @@ def report(args, res, step_ms, e2e_ms, world):
                 "fwd_ms": tr["fwd_ms"], "bwd_ms": tr["bwd_ms"],
                 "bwd_tensor_frac": bwd_flops / (tr["bwd_ms"] * 1e-3) / 1e12 / peaks["bf16_tflops"],
                 "bwd_algorithmic": "2(3p+2dv) flops per causal pair: S, dP, dV, dQ, dK"}
+            line["train"]["chunked"] = {
+                name: {"workload": "training step of the O(T) chunked path B=%d H=%d T=%d p=%d dv=%d bf16 (forward "
+                                   "saving D, then the chunked backward)" % (c["B"], c["H"], c["T"], tr["p"], tr["dv"]),
+                       "fwd_ms": c["fwd_ms"], "bwd_ms": c["bwd_ms"], "step_ms": c["step_ms"],
+                       "tokens_per_s": c["B"] * c["T"] / (c["step_ms"] * 1e-3)}
+                for name, c in tr.get("chunked", {}).items()}
     line["roofline"]["points"] = roofline_points(res, peaks, cfg)
     if args.cpu_baseline and world == 1:
         cb = time_oracle(cfg)
