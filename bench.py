@@ -807,6 +807,21 @@ def run_case(args):
             raise SystemExit("--layout bthd is for --case mg")
         elif args.case == "quadratic":
             call = lambda: K.kata_fwd_quadratic(q, k, v, o=o)  # noqa: E731
+        elif args.case == "sg_chunked":
+            ws = torch.empty(max(256, K.kata_fwd_sg_chunked_workspace_size(B, H, T, d, g, dv, args.C)),
+                             dtype=torch.uint8, device=dev)
+            call = lambda: K.kata_fwd_sg_chunked(q, k, v, g, C=args.C, o=o, workspace=ws)  # noqa: E731
+        elif args.case == "chunked_train":
+            dO = torch.randn(v.shape, generator=gen, device=dev).to(bf)
+            D = torch.empty((B, H, T), dtype=torch.float32, device=dev)
+            wsf = torch.empty(max(256, K.kata_fwd_chunked_workspace_size(B, H, T, d, dv, args.C, bf)),
+                              dtype=torch.uint8, device=dev)
+            wsb = torch.empty(max(256, int(K.lib().kata_bwd_chunked_workspace_size(B, H, T, d, dv, 1))),
+                              dtype=torch.uint8, device=dev)
+
+            def call():
+                K.kata_fwd_chunked_train(q, k, v, C=args.C, o=o, D=D, workspace=wsf)
+                K.kata_bwd_chunked(q, k, v, o, D, dO, workspace=wsb)
         elif args.case == "linear":
             q, k = q.abs(), k.abs()  # nonnegative unit vectors: sign-definite denominators
             ws = torch.empty(max(256, K.kata_fwd_linear_chunked_workspace_size(B, H, T, d, dv, args.C)),
@@ -861,7 +876,7 @@ def main():
     ap.add_argument("--ref-budget", type=float, default=15.0, help="seconds of oracle work per reference step")
     pc = ap.add_argument_group("--case: launch one call a few times on device-drawn inputs (for profilers)")
     pc.add_argument("--case", choices=["quadratic", "chunked", "mg", "mg_chunked", "decode", "train", "linear",
-                                       "linear_sequential"])
+                                       "linear_sequential", "sg_chunked", "chunked_train"])
     pc.add_argument("--B", type=int, default=8)
     pc.add_argument("--H", type=int, default=16)
     pc.add_argument("--T", type=int, default=2048)

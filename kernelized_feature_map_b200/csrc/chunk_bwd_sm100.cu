@@ -309,15 +309,6 @@ __global__ void __launch_bounds__(kGThreads, 1)
     fence_barrier_init();
   }
   fill_ones(smem + L::offOnes, threadIdx.x, kGThreads);
-  // the copies' rows 65..79 (values past the normaliser) are zero
-  for (int x = threadIdx.x; x < 2 * kTAtom / 16; x += kGThreads) {
-    const int which = x / (kTAtom / 16), y = x % (kTAtom / 16);
-    *reinterpret_cast<uint4*>(smem + (which ? L::offGT : L::offST) + 4 * kTAtom + 16 * y) = make_uint4(0, 0, 0, 0);
-  }
-  for (int x = threadIdx.x; x < 9 * 16 * 2; x += kGThreads) {  // rows 64..79 of each atom, 2 chunks each
-    const int a = x / 32, rr = 64 + (x % 32) / 2, ch = x & 1;
-    *reinterpret_cast<uint4*>(smem + L::offG + a * kSBAtom + rr * 32 + ch * 16) = make_uint4(0, 0, 0, 0);
-  }
   if (warp == 1) tmem_alloc(tmem_holder, 512);
   tc_fence_before();
   __syncthreads();
@@ -373,21 +364,37 @@ __global__ void __launch_bounds__(kGThreads, 1)
     const int m = quarter * 32 + lane;
     const int wt = threadIdx.x - 64;  // 0..255
     // the state before the chunk (record c of wsS) and the state after it
-    // (record n_chunks - 1 - c of wsG) -> bf16 copies
+    // (record n_chunks - 1 - c of wsG) -> bf16 copies, rows past the
+    // normaliser (65..79) zero.  Consecutive threads take consecutive rows of
+    // a copy (16-byte stores 32 bytes apart, conflict-free under the 32-byte
+    // swizzle) and read consecutive record columns.
     const float* recS = wsS + ((size_t)bh * n_chunks + c) * record_floats;
     const float* recG = wsG + ((size_t)bh * n_chunks + (n_chunks - 1 - c)) * record_floats;
-    for (int x = wt; x < kRecRows * (kNP / 4); x += 256) {
-      const int e = x / (kNP / 4), w0 = 4 * (x % (kNP / 4));
-      const float4 s4 = __ldcg(reinterpret_cast<const float4*>(recS + (size_t)e * kNP + w0));
-      const float4 g4 = __ldcg(reinterpret_cast<const float4*>(recG + (size_t)e * kNP + w0));
-      const float sv[4] = {s4.x, s4.y, s4.z, s4.w}, gv[4] = {g4.x, g4.y, g4.z, g4.w};
+    for (int x = wt; x < kNP * 10; x += 256) {  // [144 x 80] copies: row n, values e0..e0+7
+      const int n = x % kNP, e0 = 8 * (x / kNP);
+      float sv[8], gv[8];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        *reinterpret_cast<__nv_bfloat16*>(smem + L::offST + tcopy_offset(w0 + u, e)) = __float2bfloat16_rn(sv[u]);
-        *reinterpret_cast<__nv_bfloat16*>(smem + L::offGT + tcopy_offset(w0 + u, e)) = __float2bfloat16_rn(gv[u]);
+      for (int u = 0; u < 8; ++u) {
+        const bool live = e0 + u < kRecRows;
+        sv[u] = live ? __ldcg(recS + (size_t)(e0 + u) * kNP + n) : 0.f;
+        gv[u] = live ? __ldcg(recG + (size_t)(e0 + u) * kNP + n) : 0.f;
       }
-      *reinterpret_cast<uint2*>(smem + L::offG + copy_offset(e, w0)) =
-          make_uint2(pack_bf16x2(gv[0], gv[1]), pack_bf16x2(gv[2], gv[3]));
+      *reinterpret_cast<uint4*>(smem + L::offST + tcopy_offset(n, e0)) =
+          make_uint4(pack_bf16x2(sv[0], sv[1]), pack_bf16x2(sv[2], sv[3]), pack_bf16x2(sv[4], sv[5]),
+                     pack_bf16x2(sv[6], sv[7]));
+      *reinterpret_cast<uint4*>(smem + L::offGT + tcopy_offset(n, e0)) =
+          make_uint4(pack_bf16x2(gv[0], gv[1]), pack_bf16x2(gv[2], gv[3]), pack_bf16x2(gv[4], gv[5]),
+                     pack_bf16x2(gv[6], gv[7]));
+    }
+    for (int x = wt; x < kSBRows * (kNP / 8); x += 256) {  // [80 x 144] copy: row e, values w0..w0+7
+      const int e = x % kSBRows, w0 = 8 * (x / kSBRows);
+      uint4 val = make_uint4(0, 0, 0, 0);
+      if (e < kRecRows) {
+        const float4 a = __ldcg(reinterpret_cast<const float4*>(recG + (size_t)e * kNP + w0));
+        const float4 b = __ldcg(reinterpret_cast<const float4*>(recG + (size_t)e * kNP + w0 + 4));
+        val = make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
+      }
+      *reinterpret_cast<uint4*>(smem + L::offG + copy_offset(e, w0)) = val;
     }
     bool ok = mbar_wait_w(tiles_full, 0, env);
     const int t = row0 + m;
