@@ -11,22 +11,33 @@
 // forms dPsi of dpsi (the derivative of vec(u u^T)).  Split at the 128-token
 // chunks: the pairs of a chunk with itself are the flash backward kernels'
 // diagonal tiles (launched with diag_only); this file adds the pairs of a
-// token with the chunks before it (dq) or after it (dk, dv) through the
-// chunk states:
-//   1. chunk_grad_sums_kernel: per chunk c the sums
-//        dS~_c^T = [V_c | 1]^T psi~(K_c)     (the forward's state update)
-//        dG~_c^T = [dN_c | dD_c]^T psi~(Q_c)
-//      written as records (dG in reverse chunk order);
-//   2. the scan (scan.cu) over each: record c becomes the state before
-//      chunk c, S_{c-1}, and the reverse one the state after it, G_{c+1};
-//   3. chunk_grad_inter_kernel: per chunk
-//        X = [dN | dD] S~        -> dq_t += 2 dPsi_X q_t
-//        Y = [V | 1]  G~         -> dk_s += 2 dPsi_Y k_s
-//        Z = psi~(K) G~^T        -> dv_s += Z[:, 0:64]
-//      added to the rows the diagonal pass wrote.
+// token with the chunks before it (dq) or after it (dk, dv) through two
+// running states, walked the way the forward's readout walks S~:
+//   1. chunk_grad_sums_kernel (G > 1 super-chunks): per super-chunk the sums
+//        S~^T = sum_c [V_c | 1]^T psi~(K_c)        (the forward's state)
+//        G~^T = sum_c [dN_c | dD_c]^T psi~(Q_c)
+//      over its chunks, written as records (the G~ ones in reverse order);
+//   2. the scan (scan.cu) over both record sequences: the state entering
+//      each super-chunk, S~ from the left and G~ from the right;
+//   3. chunk_grad_walk_kernel: one CTA per (super-chunk, head, direction).
+//      The S walk goes forward through the chunks; per chunk c, against the
+//      bf16 copy of S~ entering it,
+//        X = dN_c S~                   -> dq_t += 2 dPsi(X_t + dD_t z~) q_t
+//      then S~ takes in chunk c.  The G walk goes backward; per chunk c,
+//      against the copy of G~ leaving it,
+//        Y = V_c G~                    -> dk_s += 2 dPsi(Y_s + g~) k_s
+//        Z = psi~(K_c) G~^T            -> dv_s += Z_s
+//      then G~ takes in chunk c.  The gradient terms are added to the rows
+//      the diagonal pass wrote.
 // Packed coordinates as in chunk_common.cuh: the key side of S~ carries the
-// factor 2 off the diagonal, the query side of G~ does not.  Every chunk is
-// independent once the scans are done, so one CTA handles one chunk.
+// factor 2 off the diagonal, the query side of G~ does not.  Row 64 of each
+// state (z~ or g~) is kept in fp32 beside the bf16 copy and added in the
+// epilogue, so no product needs a block of dD or ones for it.
+//
+// The bf16 copy [80 x 144] of a state is the forward's layout: K-major for
+// Z's B operand (K = 144 packed coordinates, N = 64 value rows) and, read
+// with its atoms along N, MN-major for the B operand of X and Y (K = 64 value
+// rows, N = 144), the way psi~ is read as the update's B operand.
 #include <cuda.h>
 
 #include "chunk_common.cuh"
@@ -41,31 +52,15 @@ namespace {
 using namespace sm100;
 using namespace chunk;
 
-constexpr int kGThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2-9 operands and epilogue
+constexpr int kSMCount = 148;
 
-// ---------------------------------------------------------------------------
-// 1. per-chunk sums
-// ---------------------------------------------------------------------------
-struct SumSmem {
-  static constexpr int offV = 0;                      // V tile, 128B swizzle
-  static constexpr int offDN = offV + kVBytes;        // dO tile, scaled to dN in place
-  static constexpr int offOnes = offDN + kVBytes;     // block of ones
-  static constexpr int offAux = offOnes + kOnesBytes; // block of dD (every column of row t)
-  static constexpr int offQ = offAux + kOnesBytes;    // Q tile, 32B swizzle
-  static constexpr int offK = offQ + kQKBytes;        // K tile
-  static constexpr int offPsiK = offK + kQKBytes;     // psi~(K), key side
-  static constexpr int offPsiQ = offPsiK + kPsiBytes; // psi~(Q), query side
-  static constexpr int offBar = offPsiQ + kPsiBytes;
-  static constexpr int offMisc = offBar + 4 * 8;
-  static constexpr int kBytes = offMisc + 16 + 1024;
-};
-
-// Scales the dO row t of a 128B-swizzled [128 x 64] tile by s in place (the
-// swizzle only permutes the row's 16-byte chunks).
-__device__ __forceinline__ void scale_row_sw128(uint8_t* tile, int t, float s) {
+// Scales the bf16 row t of a 128B-swizzled [128 x 64] tile by s in place:
+// physical 16-byte chunks c0 .. c0 + n - 1 (the swizzle only permutes a row's
+// chunks, and the scale is the same for the whole row).
+__device__ __forceinline__ void scale_row_chunks_sw128(uint8_t* tile, int t, float s, int c0, int n) {
   uint4* row = reinterpret_cast<uint4*>(tile + t * 128);
-#pragma unroll
-  for (int c = 0; c < 8; ++c) {
+#pragma unroll 4
+  for (int c = c0; c < c0 + n; ++c) {
     uint4 a = row[c];
     uint32_t* w = reinterpret_cast<uint32_t*>(&a);
 #pragma unroll
@@ -77,117 +72,185 @@ __device__ __forceinline__ void scale_row_sw128(uint8_t* tile, int t, float s) {
   }
 }
 
-// Row t of a [128 x 64] 128B-swizzled block: every value = x (bf16).
-__device__ __forceinline__ void fill_row_sw128(uint8_t* tile, int t, float x) {
-  const uint32_t w = pack_bf16x2(x, x);
-  uint4* row = reinterpret_cast<uint4*>(tile + t * 128);
-#pragma unroll
-  for (int c = 0; c < 8; ++c) row[c] = make_uint4(w, w, w, w);
+// Column 0 of row t of a zeroed 128B-swizzled [128 x 64] block := x (bf16);
+// the rest of the row stays zero.  As the second M atom of the MN-major A
+// operand [dN | block]^T it makes row 64 of the update dD^T psi~(Q).
+__device__ __forceinline__ void set_col0_sw128(uint8_t* blk, int t, float x) {
+  *reinterpret_cast<uint4*>(blk + t * 128 + ((t & 7) << 4)) = make_uint4(pack_bf16x2(x, 0.f), 0u, 0u, 0u);
 }
 
-__global__ void __launch_bounds__(kGThreads, 1)
+__device__ __forceinline__ void zero_block(uint8_t* blk, int tid, int nthreads) {
+  uint4* w = reinterpret_cast<uint4*>(blk);
+  for (int x = tid; x < kOnesBytes / 16; x += nthreads) w[x] = make_uint4(0u, 0u, 0u, 0u);
+}
+
+// (-delta, 2/D) of token t of head bh; zero past T
+__device__ __forceinline__ float2 load_rowc(const float2* rowc, int bh, int T, int t) {
+  return t < T ? rowc[(size_t)bh * T + t] : make_float2(0.f, 0.f);
+}
+
+// ---------------------------------------------------------------------------
+// 1. per-super-chunk sums of both states
+// ---------------------------------------------------------------------------
+constexpr int kSumThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2-9 operands (two threads a token)
+constexpr int kSumStages = 5;
+
+struct SumSmem {
+  static constexpr int kStage = kVBytes + kQKBytes;                 // [V | K] or [dO | Q]
+  static constexpr int offStage = 0;
+  static constexpr int offBlk = offStage + kSumStages * kStage;      // ones, or a dD block per psi~ buffer
+  static constexpr int offPsi = offBlk + 2 * kOnesBytes;             // 2 psi~ buffers
+  static constexpr int offBar = offPsi + 2 * kPsiBytes;
+  static constexpr int kBars = 2 * kSumStages + 4 + 1;
+  static constexpr int offMisc = offBar + kBars * 8;
+  static constexpr int kBytes = offMisc + 16 + 1024;
+};
+
+// blockIdx.z = 0: super-chunk g = blockIdx.x (0 .. G-2), its S~ sum into
+// record (bh, g); blockIdx.z = 1: super-chunk g = blockIdx.x + 1 (1 .. G-1),
+// its G~ sum into record (BH + bh, G - 1 - g).  The last super-chunk's S~ sum
+// and the first one's G~ sum enter no other super-chunk and are not formed.
+__global__ void __launch_bounds__(kSumThreads, 1)
     chunk_grad_sums_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                            const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                           const float2* __restrict__ rowc, float* __restrict__ wsS, float* __restrict__ wsG, int T,
-                           int n_chunks, long long record_floats, WaitCtl wc) {
+                           const float2* __restrict__ rowc, float* __restrict__ ws, int T, int Ls, int G,
+                           long long record_floats, WaitCtl wc) {
   using L = SumSmem;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::offBar);
-  uint64_t* tiles_full = bars;
-  uint64_t* ops_ready = bars + 1;  // operands formed (256)
-  uint64_t* acc_done = bars + 2;
+  uint64_t* kv_full = bars;
+  uint64_t* kv_empty = kv_full + kSumStages;
+  uint64_t* psi_full = kv_empty + kSumStages;  // [2]
+  uint64_t* psi_empty = psi_full + 2;          // [2]
+  uint64_t* acc_done = psi_empty + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::offMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::offMisc + 4);
+
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int c = blockIdx.x, bh = blockIdx.y;
-  const int row0 = c * kTile;
+  const bool grad = blockIdx.z == 1;
+  const int g = grad ? (int)blockIdx.x + 1 : (int)blockIdx.x, bh = blockIdx.y, BH = gridDim.y;
+  const int t0 = g * Ls;
+  const int n_chunks = (min(T, t0 + Ls) - t0 + kTile - 1) / kTile;
 
   if (threadIdx.x == 0) {
-    mbar_init(tiles_full, 1);
-    mbar_init(ops_ready, 256);
+    for (int s = 0; s < kSumStages; ++s) {
+      mbar_init(kv_full + s, 1);
+      mbar_init(kv_empty + s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(psi_full + b, 256);
+      mbar_init(psi_empty + b, 1);
+    }
     mbar_init(acc_done, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  fill_ones(smem + L::offOnes, threadIdx.x, kGThreads);
-  if (warp == 1) tmem_alloc(tmem_holder, 512);
+  if (grad) {
+    zero_block(smem + L::offBlk, threadIdx.x, kSumThreads);
+    zero_block(smem + L::offBlk + kOnesBytes, threadIdx.x, kSumThreads);
+  } else {
+    fill_ones(smem + L::offBlk, threadIdx.x, kSumThreads);
+  }
+  fence_proxy_async_smem();
+  if (warp == 1) tmem_alloc(tmem_holder, 256);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   const WaitEnv env{wc.status, abort_flag, wc.limit};
-  constexpr uint32_t colS = 0, colG = 256;
 
   if (warp == 0) {
     if (lane == 0) {
-      mbar_arrive_expect_tx(tiles_full, 2 * kVBytes + 2 * kQKBytes);
-      tma_load_3d(smem + L::offV, &tm_v, tiles_full, 0, row0, bh);
-      tma_load_3d(smem + L::offDN, &tm_do, tiles_full, 0, row0, bh);
-      tma_load_3d(smem + L::offQ, &tm_q, tiles_full, 0, row0, bh);
-      tma_load_3d(smem + L::offK, &tm_k, tiles_full, 0, row0, bh);
-      mbar_wait_drain(tiles_full, 0);
+      const CUtensorMap* big = grad ? &tm_do : &tm_v;
+      const CUtensorMap* small = grad ? &tm_q : &tm_k;
+      prefetch_tmap(big);
+      prefetch_tmap(small);
+      int issued = 0;
+      for (int c = 0; c < n_chunks; ++c) {
+        const int st = c % kSumStages;
+        if (!mbar_wait(kv_empty + st, ((c / kSumStages) & 1) ^ 1, env)) break;
+        uint8_t* base = smem + L::offStage + st * L::kStage;
+        mbar_arrive_expect_tx(kv_full + st, L::kStage);
+        tma_load_3d(base, big, kv_full + st, 0, t0 + c * kTile, bh);
+        tma_load_3d(base + kVBytes, small, kv_full + st, 0, t0 + c * kTile, bh);
+        ++issued;
+      }
+      for (int c = issued - kSumStages < 0 ? 0 : issued - kSumStages; c < issued; ++c)
+        mbar_wait_drain(kv_full + c % kSumStages, (c / kSumStages) & 1);
     }
   } else if (warp == 1) {
     // whole warp; one elected lane issues
-    bool issued = false;
-    if (mbar_wait_w(ops_ready, 0, env)) {
+    constexpr uint32_t id_u = idesc_bf16(128, kNP, true, true);  // A = [X | w]^T (MN-major), B = psi~ (N-major)
+    const uint32_t sStage = smem_u32(smem + L::offStage), sBlk = smem_u32(smem + L::offBlk);
+    const uint64_t dpsi = smem_desc(smem_u32(smem + L::offPsi), kPsiAtom, 256, kSw32);
+    for (int c = 0; c < n_chunks; ++c) {
+      const int st = c % kSumStages, pb = c & 1;
+      if (!mbar_wait_w(kv_full + st, (c / kSumStages) & 1, env)) break;
+      if (!mbar_wait_w(psi_full + pb, (c >> 1) & 1, env)) break;
       tc_fence_after();
-      constexpr uint32_t id_u = idesc_bf16(128, kNP, true, true);  // A = [X | w]^T (MN-major), B = psi~ (N-major)
-      const uint64_t dvo = desc_vones(smem_u32(smem + L::offV), smem_u32(smem + L::offOnes));
-      const uint64_t dna = desc_vones(smem_u32(smem + L::offDN), smem_u32(smem + L::offAux));
-      const uint64_t dpk = smem_desc(smem_u32(smem + L::offPsiK), kPsiAtom, 256, kSw32);
-      const uint64_t dpq = smem_desc(smem_u32(smem + L::offPsiQ), kPsiAtom, 256, kSw32);
+      const uint64_t da = desc_vones(sStage + st * L::kStage, sBlk + (grad ? pb * kOnesBytes : 0));
+      const uint64_t db = desc_add(dpsi, pb * kPsiBytes);
 #pragma unroll
       for (int ks = 0; ks < kTile / 16; ++ks)
-        mma_ss_w(tmem + colS, desc_add(dvo, ks * 2048), desc_add(dpk, ks * 512), id_u, ks > 0);
-#pragma unroll
-      for (int ks = 0; ks < kTile / 16; ++ks)
-        mma_ss_w(tmem + colG, desc_add(dna, ks * 2048), desc_add(dpq, ks * 512), id_u, ks > 0);
-      mma_commit_w(acc_done);
-      issued = true;
+        mma_ss_w(tmem, desc_add(da, ks * 2048), desc_add(db, ks * 512), id_u, (c > 0 || ks > 0) ? 1u : 0u);
+      mma_commit_w(psi_empty + pb);
+      mma_commit_w(kv_empty + st);
     }
-    if (issued) mbar_wait_drain(acc_done, 0);
+    mma_commit_w(acc_done);
+    mbar_wait_drain(acc_done, 0);
   } else {
-    // warps 2-9: token m of the chunk; warps 2-5 psi~(k_m) and dN_m, warps
-    // 6-9 psi~(q_m) and the dD block
+    // warps 2-9: token (warp - 2) % 4 * 32 + lane, half (warp - 2) / 4 of its
+    // packed psi~ (and, for G~, of its dO row)
+    const int tid = ((warp - 2) & 3) * 32 + lane;
+    const int half = (warp - 2) >> 2;
     const int quarter = warp % 4;
-    const int m = quarter * 32 + lane;
-    const bool kside = warp < 6;
-    bool ok = mbar_wait_w(tiles_full, 0, env);
-    if (ok) {
-      const int t = row0 + m;
-      const float2 rc = t < T ? rowc[(size_t)bh * T + t] : make_float2(0.f, 0.f);  // (-delta, 2/D)
+    const int d = quarter * 32 + lane;  // TMEM lane = record row
+    bool ok = true;
+    float2 rc_next = grad && n_chunks > 0 ? load_rowc(rowc, bh, T, t0 + tid) : make_float2(0.f, 0.f);
+    for (int c = 0; c < n_chunks; ++c) {
+      const int st = c % kSumStages, pb = c & 1;
+      const float2 rc = rc_next;
+      if (grad && c + 1 < n_chunks) rc_next = load_rowc(rowc, bh, T, t0 + (c + 1) * kTile + tid);
+      if (!mbar_wait_w(kv_full + st, (c / kSumStages) & 1, env)) {
+        ok = false;
+        break;
+      }
+      if (c >= 2 && !mbar_wait_w(psi_empty + pb, ((c >> 1) - 1) & 1, env)) {
+        ok = false;
+        break;
+      }
+      uint8_t* stage = smem + L::offStage + st * L::kStage;
       __nv_bfloat162 u[8];
-      uint32_t w[kNPW];
-      if (kside) {
-        load_row_sw<1>(smem + L::offK, m, u);
-        packed_psi<true>(u, w);
-        store_psi_k(smem + L::offPsiK, m, w);
-        scale_row_sw128(smem + L::offDN, m, 0.5f * rc.y);  // dN = dO / D
+      load_row_sw<1>(stage + kVBytes, tid, u);
+      uint32_t w[kNPW / 2];
+      uint8_t* dst = smem + L::offPsi + pb * kPsiBytes;
+      if (half == 0) {
+        if (grad) packed_psi_half<false, 0>(u, w);
+        else packed_psi_half<true, 0>(u, w);
+        store_psi_k_half<0>(dst, tid, w);
       } else {
-        load_row_sw<1>(smem + L::offQ, m, u);
-        packed_psi<false>(u, w);
-        store_psi_k(smem + L::offPsiQ, m, w);
-        fill_row_sw128(smem + L::offAux, m, 0.5f * rc.x * rc.y);  // dD = -delta / D
+        if (grad) packed_psi_half<false, 1>(u, w);
+        else packed_psi_half<true, 1>(u, w);
+        store_psi_k_half<1>(dst, tid, w);
+      }
+      if (grad) {
+        // dN = dO / D in place (this thread's half of the row); dD into
+        // column 0 of the block that follows dN in the A operand
+        scale_row_chunks_sw128(stage, tid, 0.5f * rc.y, 4 * half, 4);
+        if (half == 0) set_col0_sw128(smem + L::offBlk + pb * kOnesBytes, tid, 0.5f * rc.x * rc.y);
       }
       fence_proxy_async_smem();
-      mbar_arrive(ops_ready);
+      mbar_arrive(psi_full + pb);
     }
-    // records: TMEM lanes 0..64 of both sums (quarters 0-2, one warp each)
-    const bool writer = (warp == 2 || warp == 4 || warp == 5 || warp == 6 || warp == 8 || warp == 9);
-    if (ok && writer && mbar_wait_w(acc_done, 0, env)) {
+    // record rows 0..64 live in TMEM lanes 0..64: warps of lane quarters 0-2
+    // load (the load is warp-collective), lanes below 65 store
+    if (ok && warp < 6 && quarter < 3 && n_chunks > 0 && mbar_wait_w(acc_done, 0, env)) {
       tc_fence_after();
-      const int d = quarter * 32 + lane;
-      const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-      if (kside) {
-        float* row = wsS + ((size_t)bh * n_chunks + c) * record_floats + (size_t)min(d, kRecRows - 1) * kNP;
-        state_lane_to_global(lane_base + colS, row, d < kRecRows);
-      } else {
-        float* row = wsG + ((size_t)bh * n_chunks + (n_chunks - 1 - c)) * record_floats +
-                     (size_t)min(d, kRecRows - 1) * kNP;
-        state_lane_to_global(lane_base + colG, row, d < kRecRows);
-      }
+      const size_t seq = grad ? (size_t)BH + bh : (size_t)bh;
+      const int rec = grad ? G - 1 - g : g;
+      float* row = ws + (seq * G + rec) * record_floats + (size_t)min(d, kRecRows - 1) * kNP;
+      state_lane_to_global(tmem + ((uint32_t)(quarter * 32) << 16), row, d < kRecRows);
     }
   }
 
@@ -195,120 +258,232 @@ __global__ void __launch_bounds__(kGThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, 256);
   }
 }
 
 // ---------------------------------------------------------------------------
-// 3. inter-chunk gradients
+// 3. the walks
 // ---------------------------------------------------------------------------
-constexpr int kTAtom = kNP * 32;  // one K step (16 values) of a [144 coordinates x 80] K-major copy
+// Warp roles (448 threads):
+//   warp 0       TMA: [dO | V | K | Q] tiles of each chunk into a 2-stage ring
+//   warp 1       TMEM allocator; MMA issue (the whole warp, one elected lane)
+//   warps 2-5    epilogue: token m = lane quarter * 32 + lane of the chunk
+//   warps 6-9    S walk: psi~(K) into shared memory; G walk: psi~(Q) into
+//                shared memory; then half 0 of the state copy
+//   warps 10-13  dN in place (and for the G walk dD, and psi~(K) into TMEM);
+//                then half 1 of the state copy
+// MMA order per chunk: the products against the copy of the state entering
+// the chunk (X, or Y and Z), then the state update by the chunk.  The copy
+// for the next chunk is refreshed in place once the update has landed (the
+// products, issued before it, have then read it).  Row 64 of the state goes
+// to one of two fp32 vectors, each with its own barrier for the epilogue.
+// TMEM is handed over a chunk at a time: the operand warps read the state
+// (and the G walk stores psi~(K)) only after the epilogue has released the
+// products of the chunk before (acc_free).  With those accesses overlapping
+// the epilogue's reads of the same lane quarter, the epilogue read wrong
+// products for whole lane quarters in some runs (B4 H8 T1000, one
+// super-chunk of 8 chunks per walk); with this hand-over every run is
+// bitwise the same.
+constexpr int kWalkThreads = 448;
+constexpr int kWalkStages = 2;
 
-struct InterSmem {
-  static constexpr int offV = 0;
-  static constexpr int offDN = offV + kVBytes;
-  static constexpr int offOnes = offDN + kVBytes;
-  static constexpr int offAux = offOnes + kOnesBytes;
-  static constexpr int offQ = offAux + kOnesBytes;
-  static constexpr int offK = offQ + kQKBytes;
-  static constexpr int offPsiK = offK + kQKBytes;       // psi~(K), key side (K-major A operand)
-  static constexpr int offST = offPsiK + kPsiBytes;     // S~ as [144 x 80] K-major (5 atoms)
-  static constexpr int offGT = offST + 5 * kTAtom;      // G~ as [144 x 80] K-major
-  static constexpr int offG = offGT + 5 * kTAtom;       // G~ as [80 x 144] K-major (the forward's copy layout)
-  static constexpr int offBar = offG + kSBBytes;
-  static constexpr int offMisc = offBar + 4 * 8;
+struct WalkSmem {
+  static constexpr int kStage = 2 * kVBytes + 2 * kQKBytes;  // [dO | V | K | Q]
+  static constexpr int offStage = 0;
+  static constexpr int offBlk = offStage + kWalkStages * kStage;  // ones (S walk) or 2 dD blocks (G walk)
+  static constexpr int offPsi = offBlk + 2 * kOnesBytes;          // 2 psi~ buffers
+  static constexpr int offSB = offPsi + 2 * kPsiBytes;            // bf16 copy of the state
+  static constexpr int offZ = offSB + kSBBytes;                   // 2 x 144 fp32: row 64 of the state
+  static constexpr int offBar = offZ + 2 * kNP * 4;
+  static constexpr int kBars = 2 * kWalkStages + 8;
+  static constexpr int offMisc = offBar + kBars * 8;
   static constexpr int kBytes = offMisc + 16 + 1024;
-  // TMEM columns
-  static constexpr uint32_t colX = 0;    // [dN | dD] S~, 144
-  static constexpr uint32_t colY = 160;  // [V | 1] G~, 144
-  static constexpr uint32_t colZ = 320;  // psi~(K) G~^T, 80
+  // TMEM columns (512 allocated)
+  static constexpr uint32_t colState = 0;  // S~^T or G~^T, 144
+  static constexpr uint32_t colAcc = 160;  // X or Y, 144
+  static constexpr uint32_t colZ = 320;    // Z, 64
+  static constexpr uint32_t colPK = 384;   // psi~(K) of the G walk, 72
 };
 
-// Element (n, e) of a [144 x 80] K-major bf16 copy (K steps of 16 as 32B-
-// swizzled atoms of [144 rows x 32 B]).
-__device__ __forceinline__ uint32_t tcopy_offset(int n, int e) {
-  return (uint32_t)((e >> 4) * kTAtom + n * 32 + ((((e >> 3) & 1) ^ ((n >> 2) & 1)) << 4) + (e & 7) * 2);
-}
-// Element (e, w) of the forward's [80 x 144] copy layout.
-__device__ __forceinline__ uint32_t copy_offset(int e, int w) {
-  return (uint32_t)((w >> 4) * kSBAtom + e * 32 + ((((w >> 3) & 1) ^ ((e >> 2) & 1)) << 4) + (w & 7) * 2);
+// Half `half` of record row `row` (zeros when row is null) -> TMEM lane; also
+// into bf16 copy row n when `copy`, and as fp32 into zb when zb is not null.
+// Warp-collective (the TMEM stores).
+__device__ __forceinline__ void init_state_half(const float* row, uint32_t taddr, uint8_t* sb, int n, bool copy,
+                                                float* zb, int half) {
+  auto ld4 = [&](int col, uint32_t* r) {
+    float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (row) v4 = *reinterpret_cast<const float4*>(row + col);
+    r[0] = __float_as_uint(v4.x);
+    r[1] = __float_as_uint(v4.y);
+    r[2] = __float_as_uint(v4.z);
+    r[3] = __float_as_uint(v4.w);
+    if (zb) *reinterpret_cast<float4*>(zb + col) = v4;
+  };
+  const int a0 = half == 0 ? 0 : 5;  // first whole atom of the half
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    uint32_t r[16];
+#pragma unroll
+    for (int e = 0; e < 16; e += 4) ld4(16 * (a0 + a) + e, r + e);
+    tmem_st16(taddr + 16 * (a0 + a), r);
+    if (copy) store_state_bf16_atom(sb, n, a0 + a, r);
+  }
+  uint32_t r[8];
+  const int col = half == 0 ? 64 : 72;
+  ld4(col, r);
+  ld4(col + 4, r + 4);
+  tmem_st8(taddr + col, r);
+  if (copy) store_state_bf16_chunk(sb, n, 4, half, r);
 }
 
-// 2 dPsi(u) u for the symmetric p x p form of a packed gradient row held in
-// TMEM columns [taddr, taddr + 144) of this lane: off-diagonal packed entries
-// count f_off times (the entry of one triangle), diagonal ones f_diag times.
-// Warp-collective (the loads).
+// Half `half` of a TMEM lane of the state as fp32 into zb (when `active`).
+// Warp-collective.
+__device__ __forceinline__ void state_half_to_f32(uint32_t taddr, float* zb, bool active, int half) {
+  uint32_t a[32], b[32], c[8];
+  if (half == 0) {
+    tmem_ld32(taddr, a);
+    tmem_ld32(taddr + 32, b);
+    tmem_ld8(taddr + 64, c);
+  } else {
+    tmem_ld8(taddr + 72, c);
+    tmem_ld32(taddr + 80, a);
+    tmem_ld32(taddr + 112, b);
+  }
+  tmem_wait_ld();
+  if (!active) return;
+  auto st4 = [&](int col, const uint32_t* r) {
+    *reinterpret_cast<float4*>(zb + col) =
+        make_float4(__uint_as_float(r[0]), __uint_as_float(r[1]), __uint_as_float(r[2]), __uint_as_float(r[3]));
+  };
+  const int ca = half == 0 ? 0 : 80, cc = half == 0 ? 64 : 72;
+#pragma unroll
+  for (int e = 0; e < 32; e += 4) {
+    st4(ca + e, a + e);
+    st4(ca + 32 + e, b + e);
+  }
+  st4(cc, c);
+  st4(cc + 4, c + 4);
+}
+
+// 2 dPsi(u) u for the symmetric p x p form of the packed gradient row
+// r_w + coef * zb[w], r in TMEM columns [taddr, taddr + 144) of this lane:
+// off-diagonal packed entries count kFOff times (the entry of one triangle),
+// diagonal ones kFDiag times.  Warp-collective (the loads).
 template <int kFDiag, int kFOff>
-__device__ __forceinline__ void packed_grad_times_u(uint32_t taddr, const float (&u)[16], float (&out)[16]) {
+__device__ __forceinline__ void packed_grad_times_u(uint32_t taddr, const float* zb, float coef,
+                                                    const float (&u)[16], float (&out)[16]) {
 #pragma unroll
   for (int i = 0; i < 16; ++i) out[i] = 0.f;
 #pragma unroll
   for (int b = 0; b < 9; ++b) {
     uint32_t r[16];
     tmem_ld16(taddr + 16 * b, r);
+    float zv[16];
+#pragma unroll
+    for (int x = 0; x < 16; x += 4) {
+      const float4 z4 = *reinterpret_cast<const float4*>(zb + 16 * b + x);
+      zv[x] = z4.x;
+      zv[x + 1] = z4.y;
+      zv[x + 2] = z4.z;
+      zv[x + 3] = z4.w;
+    }
     tmem_wait_ld();
 #pragma unroll
     for (int x = 0; x < 16; ++x) {
       const int w = 16 * b + x;
       const int i = packed_i(w), j = packed_j(w);
       if (i < 0) continue;
-      const float g = __uint_as_float(r[x]);
+      const float gr = fmaf(coef, zv[x], __uint_as_float(r[x]));
       if (i == j) {
-        out[i] = fmaf((float)kFDiag * g, u[i], out[i]);
+        out[i] = fmaf((float)kFDiag * gr, u[i], out[i]);
       } else {
-        out[i] = fmaf((float)kFOff * g, u[j], out[i]);
-        out[j] = fmaf((float)kFOff * g, u[i], out[j]);
+        out[i] = fmaf((float)kFOff * gr, u[j], out[i]);
+        out[j] = fmaf((float)kFOff * gr, u[i], out[j]);
       }
     }
   }
 }
 
-// the N bf16 values at row, plus the fp32 values in add, written back
-template <int N>
-__device__ __forceinline__ void add_to_bf16_row(__nv_bfloat16* row, const float (&add)[N]) {
+// Eight bf16 values (one uint4) plus the fp32 values add[0..7], rounded back
+// to bf16 in place
+__device__ __forceinline__ void add_bf16x8(uint4& old, const float* add) {
+  uint32_t* w = reinterpret_cast<uint32_t*>(&old);
 #pragma unroll
-  for (int e = 0; e < N; e += 8) {
-    uint4* p4 = reinterpret_cast<uint4*>(row + e);
-    uint4 a = *p4;
-    uint32_t* w = reinterpret_cast<uint32_t*>(&a);
-#pragma unroll
-    for (int x = 0; x < 4; ++x) {
-      const float lo = __uint_as_float(w[x] << 16) + add[e + 2 * x];
-      const float hi = __uint_as_float(w[x] & 0xffff0000u) + add[e + 2 * x + 1];
-      w[x] = pack_bf16x2(lo, hi);
-    }
-    *p4 = a;
+  for (int x = 0; x < 4; ++x) {
+    const float lo = __uint_as_float(w[x] << 16) + add[2 * x];
+    const float hi = __uint_as_float(w[x] & 0xffff0000u) + add[2 * x + 1];
+    w[x] = pack_bf16x2(lo, hi);
   }
 }
 
-__global__ void __launch_bounds__(kGThreads, 1)
-    chunk_grad_inter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                            const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                            const float2* __restrict__ rowc, const float* __restrict__ wsS,
-                            const float* __restrict__ wsG, __nv_bfloat16* __restrict__ dq,
-                            __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv, int T, int n_chunks,
-                            long long record_floats, WaitCtl wc) {
-  using L = InterSmem;
+template <int N>
+__device__ __forceinline__ void store_bf16_row(__nv_bfloat16* row, const uint4 (&v)[N / 8]) {
+#pragma unroll
+  for (int q = 0; q < N / 8; ++q) reinterpret_cast<uint4*>(row)[q] = v[q];
+}
+
+template <int N>
+__device__ __forceinline__ void load_bf16_row(const __nv_bfloat16* row, uint4 (&out)[N / 8]) {
+#pragma unroll
+  for (int q = 0; q < N / 8; ++q) out[q] = __ldcg(reinterpret_cast<const uint4*>(row) + q);
+}
+
+// blockIdx.z = 0: the S walk of super-chunk blockIdx.x (dq); 1: its G walk
+// (dk, dv).  ws holds the scanned records ([2 BH] sequences of G), null when
+// G = 1 (both walks then start from zero).
+__global__ void __launch_bounds__(kWalkThreads, 1)
+    chunk_grad_walk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                           const float2* __restrict__ rowc, const float* __restrict__ ws,
+                           __nv_bfloat16* __restrict__ dq, __nv_bfloat16* __restrict__ dk,
+                           __nv_bfloat16* __restrict__ dv, int T, int Ls, int G, long long record_floats,
+                           WaitCtl wc) {
+  using L = WalkSmem;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::offBar);
-  uint64_t* tiles_full = bars;
-  uint64_t* ops_ready = bars + 1;  // operands formed (256)
-  uint64_t* acc_done = bars + 2;
+  uint64_t* kv_full = bars;
+  uint64_t* kv_empty = kv_full + kWalkStages;   // MMA commit + 128 epilogue threads
+  uint64_t* ops_full = kv_empty + kWalkStages;  // operands and state copy of the chunk (256)
+  uint64_t* acc_full = ops_full + 1;            // X, or Y and Z, in TMEM
+  uint64_t* acc_free = acc_full + 1;            // the epilogue has read them (128)
+  uint64_t* upd_done = acc_free + 1;            // state updated by the chunk
+  uint64_t* z_ready = upd_done + 1;             // [2] fp32 row 64 of the state (the 64 threads of quarter 2)
+  uint64_t* mma_done = z_ready + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::offMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::offMisc + 4);
+  float* zbuf = reinterpret_cast<float*>(smem + L::offZ);  // [2][144]
+
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int c = blockIdx.x, bh = blockIdx.y;
-  const int row0 = c * kTile;
+  const bool gw = blockIdx.z == 1;  // the G walk
+  const int g = blockIdx.x, bh = blockIdx.y, BH = gridDim.y;
+  const int t0 = g * Ls;
+  const int n_chunks = (min(T, t0 + Ls) - t0 + kTile - 1) / kTile;
+  // the i-th chunk of the walk
+  auto chunk_of = [&](int i) { return gw ? n_chunks - 1 - i : i; };
 
   if (threadIdx.x == 0) {
-    mbar_init(tiles_full, 1);
-    mbar_init(ops_ready, 256);
-    mbar_init(acc_done, 1);
+    for (int s = 0; s < kWalkStages; ++s) {
+      mbar_init(kv_full + s, 1);
+      mbar_init(kv_empty + s, 1 + 128);
+    }
+    mbar_init(ops_full, 256);
+    mbar_init(acc_full, 1);
+    mbar_init(acc_free, 128);
+    mbar_init(upd_done, 1);
+    for (int b = 0; b < 2; ++b) mbar_init(z_ready + b, 64);
+    mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  fill_ones(smem + L::offOnes, threadIdx.x, kGThreads);
+  if (gw) {
+    zero_block(smem + L::offBlk, threadIdx.x, kWalkThreads);
+    zero_block(smem + L::offBlk + kOnesBytes, threadIdx.x, kWalkThreads);
+  } else {
+    fill_ones(smem + L::offBlk, threadIdx.x, kWalkThreads);
+  }
+  fence_proxy_async_smem();
   if (warp == 1) tmem_alloc(tmem_holder, 512);
   tc_fence_before();
   __syncthreads();
@@ -317,142 +492,223 @@ __global__ void __launch_bounds__(kGThreads, 1)
   const WaitEnv env{wc.status, abort_flag, wc.limit};
 
   if (warp == 0) {
+    // ------------------------------------------------------------- TMA
     if (lane == 0) {
-      mbar_arrive_expect_tx(tiles_full, 2 * kVBytes + 2 * kQKBytes);
-      tma_load_3d(smem + L::offV, &tm_v, tiles_full, 0, row0, bh);
-      tma_load_3d(smem + L::offDN, &tm_do, tiles_full, 0, row0, bh);
-      tma_load_3d(smem + L::offQ, &tm_q, tiles_full, 0, row0, bh);
-      tma_load_3d(smem + L::offK, &tm_k, tiles_full, 0, row0, bh);
-      mbar_wait_drain(tiles_full, 0);
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      prefetch_tmap(&tm_do);
+      int issued = 0;
+      for (int i = 0; i < n_chunks; ++i) {
+        const int st = i % kWalkStages;
+        if (!mbar_wait(kv_empty + st, ((i / kWalkStages) & 1) ^ 1, env)) break;
+        uint8_t* base = smem + L::offStage + st * L::kStage;
+        mbar_arrive_expect_tx(kv_full + st, L::kStage);
+        const int row = t0 + chunk_of(i) * kTile;
+        tma_load_3d(base, &tm_do, kv_full + st, 0, row, bh);
+        tma_load_3d(base + kVBytes, &tm_v, kv_full + st, 0, row, bh);
+        tma_load_3d(base + 2 * kVBytes, &tm_k, kv_full + st, 0, row, bh);
+        tma_load_3d(base + 2 * kVBytes + kQKBytes, &tm_q, kv_full + st, 0, row, bh);
+        ++issued;
+      }
+      for (int i = issued - kWalkStages < 0 ? 0 : issued - kWalkStages; i < issued; ++i)
+        mbar_wait_drain(kv_full + i % kWalkStages, (i / kWalkStages) & 1);
     }
   } else if (warp == 1) {
-    bool issued = false;
-    if (mbar_wait_w(ops_ready, 0, env)) {
+    // ------------------------------------------------------------- MMA
+    constexpr uint32_t id_xy = idesc_bf16(128, kNP, false, true);  // A [128 x 64] K-major, B copy MN-major
+    constexpr uint32_t id_z = idesc_bf16(128, kDV, false, false);  // A psi~(K) (TMEM), B copy K-major
+    constexpr uint32_t id_u = idesc_bf16(128, kNP, true, true);    // A [X | w]^T MN-major, B psi~ N-major
+    const uint32_t sStage = smem_u32(smem + L::offStage), sBlk = smem_u32(smem + L::offBlk);
+    const uint32_t sSB = smem_u32(smem + L::offSB);
+    const uint64_t dsb_mn = smem_desc(sSB, kSBAtom, 256, kSw32);  // copy as [K = 64 rows x N = 144]
+    const uint64_t dsb_k = smem_desc(sSB, 16, 256, kSw32);        // copy as [N = 64 rows x K = 144]
+    const uint64_t dpsi = smem_desc(smem_u32(smem + L::offPsi), kPsiAtom, 256, kSw32);
+    for (int i = 0; i < n_chunks; ++i) {
+      const int st = i % kWalkStages, pb = i & 1;
+      const uint32_t sDO = sStage + st * L::kStage, sV = sDO + kVBytes;
+      if (!mbar_wait_w(ops_full, i & 1, env)) break;
+      if (i > 0 && !mbar_wait_w(acc_free, (i - 1) & 1, env)) break;
       tc_fence_after();
-      constexpr uint32_t id_xy = idesc_bf16(128, kNP, false, false);  // A [128 x 80] K-major, B [144 x 80] K-major
-      constexpr uint32_t id_z = idesc_bf16(128, 80, false, false);    // A psi~(K) K-major, B [80 x 144] K-major
-      const uint64_t dV = smem_desc(smem_u32(smem + L::offV), 16, 1024, kSw128);
-      const uint64_t dOnes = smem_desc(smem_u32(smem + L::offOnes), 16, 1024, kSw128);
-      const uint64_t dN = smem_desc(smem_u32(smem + L::offDN), 16, 1024, kSw128);
-      const uint64_t dAux = smem_desc(smem_u32(smem + L::offAux), 16, 1024, kSw128);
-      const uint64_t dST = smem_desc(smem_u32(smem + L::offST), 16, 256, kSw32);
-      const uint64_t dGT = smem_desc(smem_u32(smem + L::offGT), 16, 256, kSw32);
-      const uint64_t dG = smem_desc(smem_u32(smem + L::offG), 16, 256, kSw32);
-      const uint64_t dPK = smem_desc(smem_u32(smem + L::offPsiK), 16, 256, kSw32);
-      // X = [dN | dD] S~ and Y = [V | 1] G~: K = 80 in 5 steps, the fifth
-      // from the dD / ones block
+      // products against the copy of the state entering the chunk
+      const uint64_t da = smem_desc(gw ? sV : sDO, 16, 1024, kSw128);  // V or dN, K-major
 #pragma unroll
-      for (int ks = 0; ks < 5; ++ks) {
-        const uint64_t a = ks < 4 ? desc_add(dN, ks * 32) : dAux;
-        mma_ss_w(tmem + L::colX, a, desc_add(dST, ks * kTAtom), id_xy, ks > 0);
+      for (int ks = 0; ks < kDV / 16; ++ks)
+        mma_ss_w(tmem + L::colAcc, desc_add(da, ks * 32), desc_add(dsb_mn, ks * 512), id_xy, ks > 0);
+      if (gw) {
+#pragma unroll
+        for (int ks = 0; ks < kNP / 16; ++ks)
+          mma_ts_w(tmem + L::colZ, tmem + L::colPK + ks * 8, desc_add(dsb_k, ks * kSBAtom), id_z, ks > 0);
       }
+      mma_commit_w(acc_full);
+      // the state takes in the chunk: S~^T += [V | 1]^T psi~(K), or
+      // G~^T += [dN | dD]^T psi~(Q)
+      const uint64_t du = gw ? desc_vones(sDO, sBlk + pb * kOnesBytes) : desc_vones(sV, sBlk);
+      const uint64_t db = desc_add(dpsi, pb * kPsiBytes);
 #pragma unroll
-      for (int ks = 0; ks < 5; ++ks) {
-        const uint64_t a = ks < 4 ? desc_add(dV, ks * 32) : dOnes;
-        mma_ss_w(tmem + L::colY, a, desc_add(dGT, ks * kTAtom), id_xy, ks > 0);
-      }
-      // Z = psi~(K) G~^T: K = 144 in 9 steps
-#pragma unroll
-      for (int ks = 0; ks < kNP / 16; ++ks)
-        mma_ss_w(tmem + L::colZ, desc_add(dPK, ks * kPsiAtom), desc_add(dG, ks * kSBAtom), id_z, ks > 0);
-      mma_commit_w(acc_done);
-      issued = true;
+      for (int ks = 0; ks < kTile / 16; ++ks)
+        mma_ss_w(tmem + L::colState, desc_add(du, ks * 2048), desc_add(db, ks * 512), id_u, 1);
+      mma_commit_w(upd_done);
+      mma_commit_w(kv_empty + st);
     }
-    if (issued) mbar_wait_drain(acc_done, 0);
-  } else {
+    mma_commit_w(mma_done);
+    mbar_wait_drain(mma_done, 0);
+  } else if (warp < 6) {
+    // ------------------------------------------------------------- epilogue
     const int quarter = warp % 4;
     const int m = quarter * 32 + lane;
-    const int wt = threadIdx.x - 64;  // 0..255
-    // the state before the chunk (record c of wsS) and the state after it
-    // (record n_chunks - 1 - c of wsG) -> bf16 copies, rows past the
-    // normaliser (65..79) zero.  Consecutive threads take consecutive rows of
-    // a copy (16-byte stores 32 bytes apart, conflict-free under the 32-byte
-    // swizzle) and read consecutive record columns.
-    const float* recS = wsS + ((size_t)bh * n_chunks + c) * record_floats;
-    const float* recG = wsG + ((size_t)bh * n_chunks + (n_chunks - 1 - c)) * record_floats;
-    for (int x = wt; x < kNP * 10; x += 256) {  // [144 x 80] copies: row n, values e0..e0+7
-      const int n = x % kNP, e0 = 8 * (x / kNP);
-      float sv[8], gv[8];
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    for (int i = 0; i < n_chunks; ++i) {
+      const int st = i % kWalkStages;
+      const int t = t0 + chunk_of(i) * kTile + m;
+      if (!mbar_wait_w(kv_full + st, (i / kWalkStages) & 1, env)) break;
+      // this token's q (S walk) or k (G walk) row, then the stage may go
+      const uint8_t* tile = smem + L::offStage + st * L::kStage + 2 * kVBytes + (gw ? 0 : kQKBytes);
+      __nv_bfloat162 u2[8];
+      load_row_sw<1>(tile, m, u2);
+      mbar_arrive(kv_empty + st);
+      float u[16];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const bool live = e0 + u < kRecRows;
-        sv[u] = live ? __ldcg(recS + (size_t)(e0 + u) * kNP + n) : 0.f;
-        gv[u] = live ? __ldcg(recG + (size_t)(e0 + u) * kNP + n) : 0.f;
+      for (int x = 0; x < 8; ++x) {
+        u[2 * x] = __low2float(u2[x]);
+        u[2 * x + 1] = __high2float(u2[x]);
       }
-      *reinterpret_cast<uint4*>(smem + L::offST + tcopy_offset(n, e0)) =
-          make_uint4(pack_bf16x2(sv[0], sv[1]), pack_bf16x2(sv[2], sv[3]), pack_bf16x2(sv[4], sv[5]),
-                     pack_bf16x2(sv[6], sv[7]));
-      *reinterpret_cast<uint4*>(smem + L::offGT + tcopy_offset(n, e0)) =
-          make_uint4(pack_bf16x2(gv[0], gv[1]), pack_bf16x2(gv[2], gv[3]), pack_bf16x2(gv[4], gv[5]),
-                     pack_bf16x2(gv[6], gv[7]));
-    }
-    for (int x = wt; x < kSBRows * (kNP / 8); x += 256) {  // [80 x 144] copy: row e, values w0..w0+7
-      const int e = x % kSBRows, w0 = 8 * (x / kSBRows);
-      uint4 val = make_uint4(0, 0, 0, 0);
-      if (e < kRecRows) {
-        const float4 a = __ldcg(reinterpret_cast<const float4*>(recG + (size_t)e * kNP + w0));
-        const float4 b = __ldcg(reinterpret_cast<const float4*>(recG + (size_t)e * kNP + w0 + 4));
-        val = make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
+      const bool live = t < T;
+      const size_t r = (size_t)bh * T + (live ? t : 0);
+      const float* zb = zbuf + (i & 1) * kNP;
+      if (!gw) {
+        const float2 rc = load_rowc(rowc, bh, T, t);
+        uint4 old[2];
+        if (live) load_bf16_row<16>(dq + r * 16, old);
+        if (!mbar_wait_w(z_ready + (i & 1), (i >> 1) & 1, env) || !mbar_wait_w(acc_full, i & 1, env)) break;
+        tc_fence_after();
+        float gq[16];
+        packed_grad_times_u<2, 1>(lane_base + L::colAcc, zb, 0.5f * rc.x * rc.y, u, gq);
+        tc_fence_before();
+        mbar_arrive(acc_free);
+        if (live) {
+          add_bf16x8(old[0], gq);
+          add_bf16x8(old[1], gq + 8);
+          store_bf16_row<16>(dq + r * 16, old);
+        }
+      } else {
+        uint4 oldk[2], oldv[8];
+        if (live) {
+          load_bf16_row<16>(dk + r * 16, oldk);
+          load_bf16_row<kDV>(dv + r * kDV, oldv);
+        }
+        if (!mbar_wait_w(z_ready + (i & 1), (i >> 1) & 1, env) || !mbar_wait_w(acc_full, i & 1, env)) break;
+        tc_fence_after();
+        float gk[16];
+        packed_grad_times_u<2, 2>(lane_base + L::colAcc, zb, 1.f, u, gk);
+        // Z, 32 columns at a time, into the loaded dv row before the
+        // accumulators are released
+#pragma unroll
+        for (int hb = 0; hb < 2; ++hb) {
+          uint32_t za[32];
+          tmem_ld32(lane_base + L::colZ + 32 * hb, za);
+          tmem_wait_ld();
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float zf[8];
+#pragma unroll
+            for (int x = 0; x < 8; ++x) zf[x] = __uint_as_float(za[8 * q + x]);
+            add_bf16x8(oldv[4 * hb + q], zf);
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(acc_free);
+        if (live) {
+          add_bf16x8(oldk[0], gk);
+          add_bf16x8(oldk[1], gk + 8);
+          store_bf16_row<16>(dk + r * 16, oldk);
+          store_bf16_row<kDV>(dv + r * kDV, oldv);
+        }
       }
-      *reinterpret_cast<uint4*>(smem + L::offG + copy_offset(e, w0)) = val;
     }
-    bool ok = mbar_wait_w(tiles_full, 0, env);
-    const int t = row0 + m;
-    const float2 rc = t < T ? rowc[(size_t)bh * T + t] : make_float2(0.f, 0.f);  // (-delta, 2/D)
-    if (ok) {
-      if (warp < 6) {
+  } else {
+    // ------------------------------------------------------------- operands and state copies
+    const bool groupA = warp < 10;
+    const int half = groupA ? 0 : 1;
+    const int quarter = warp % 4;
+    const int m = quarter * 32 + lane;  // token of the chunk / TMEM lane = state row
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    uint8_t* sb = smem + L::offSB;
+    // operands of the i-th chunk of the walk from its landed stage; false if
+    // a wait gave up
+    auto operands = [&](int i) -> bool {
+      const int st = i % kWalkStages, pb = i & 1;
+      uint8_t* stage = smem + L::offStage + st * L::kStage;
+      const uint8_t* ktile = stage + 2 * kVBytes;
+      const uint8_t* qtile = ktile + kQKBytes;
+      if (groupA) {
+        // psi~(K) (S walk, key side) or psi~(Q) (G walk, query side) into
+        // buffer pb, last read by the update by chunk i-2
         __nv_bfloat162 u[8];
         uint32_t w[kNPW];
-        load_row_sw<1>(smem + L::offK, m, u);
-        packed_psi<true>(u, w);
-        store_psi_k(smem + L::offPsiK, m, w);
-      } else {
-        scale_row_sw128(smem + L::offDN, m, 0.5f * rc.y);         // dN = dO / D
-        fill_row_sw128(smem + L::offAux, m, 0.5f * rc.x * rc.y);  // dD = -delta / D
+        load_row_sw<1>(gw ? qtile : ktile, m, u);
+        if (gw) packed_psi<false>(u, w);
+        else packed_psi<true>(u, w);
+        store_psi_k(smem + L::offPsi + pb * kPsiBytes, m, w);
+        return true;
+      }
+      const int t = t0 + chunk_of(i) * kTile + m;
+      const float2 rc = load_rowc(rowc, bh, T, t);
+      scale_row_chunks_sw128(stage, m, 0.5f * rc.y, 0, 8);  // dN = dO / D
+      if (!gw) return true;
+      set_col0_sw128(smem + L::offBlk + pb * kOnesBytes, m, 0.5f * rc.x * rc.y);  // dD
+      // psi~(K) into TMEM once the Z of chunk i-1 has read the previous one
+      // and the epilogue has read the products of chunk i-1
+      __nv_bfloat162 u[8];
+      uint32_t w[kNPW];
+      load_row_sw<1>(ktile, m, u);
+      packed_psi<true>(u, w);
+      if (i > 0) {
+        if (!mbar_wait_w(acc_free, (i - 1) & 1, env)) return false;
+        tc_fence_after();
+      }
+      store_psi_q_tmem(lane_base + L::colPK, w);
+      tmem_wait_st();
+      return true;
+    };
+    // the state entering the walk: the scanned record (rows 0..64) or zero;
+    // rows 0..63 also into the bf16 copy, row 64 (z~ or g~) into zbuf[0].
+    // After the scan this kernel is its programmatic dependent.
+    griddep_wait();
+    if (quarter < 3) {
+      const int d = min(m, kRecRows - 1);
+      const float* row = nullptr;
+      if (ws) {
+        const size_t seq = gw ? (size_t)BH + bh : (size_t)bh;
+        const int rec = gw ? G - 1 - g : g;
+        row = ws + (seq * G + rec) * record_floats + (size_t)d * kNP;
+      }
+      init_state_half(row, lane_base + L::colState, sb, m, m < kDV, m == kDV ? zbuf : nullptr, half);
+    }
+    if (quarter == 2) mbar_arrive(z_ready);
+    bool ok = n_chunks > 0 && mbar_wait_w(kv_full, 0, env) && operands(0);
+    tmem_wait_st();  // the state's TMEM stores land before the first update reads them
+    fence_proxy_async_smem();
+    tc_fence_before();
+    if (ok) mbar_arrive(ops_full);
+    for (int i = 0; ok && i + 1 < n_chunks; ++i) {
+      const int st1 = (i + 1) % kWalkStages;
+      if (!mbar_wait_w(kv_full + st1, ((i + 1) / kWalkStages) & 1, env)) break;
+      if (!operands(i + 1)) break;
+      // the state after chunk i: this group's half of the copy (rows 0..63)
+      // and of row 64 in fp32, for chunk i+1, once the epilogue has read the
+      // products of chunk i out of TMEM (see the class comment)
+      if (!mbar_wait_w(upd_done, i & 1, env) || !mbar_wait_w(acc_free, i & 1, env)) break;
+      tc_fence_after();
+      if (quarter < 2) {
+        state_half_to_bf16(lane_base + L::colState, sb, m, true, half);
+      } else if (quarter == 2) {
+        state_half_to_f32(lane_base + L::colState, zbuf + ((i + 1) & 1) * kNP, lane == 0, half);
+        mbar_arrive(z_ready + ((i + 1) & 1));
       }
       fence_proxy_async_smem();
-      mbar_arrive(ops_ready);
-    }
-    if (ok && mbar_wait_w(acc_done, 0, env)) {
-      tc_fence_after();
-      const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-      if (warp < 6) {
-        // dq_t += 2 dPsi_X q_t (X from the key-side S~: off-diagonal entries
-        // already count both triangles)
-        __nv_bfloat162 u2[8];
-        load_row_sw<1>(smem + L::offQ, m, u2);
-        float u[16], g[16];
-#pragma unroll
-        for (int x = 0; x < 8; ++x) {
-          u[2 * x] = __low2float(u2[x]);
-          u[2 * x + 1] = __high2float(u2[x]);
-        }
-        packed_grad_times_u<2, 1>(lane_base + L::colX, u, g);
-        if (t < T) add_to_bf16_row<16>(dq + ((size_t)bh * T + t) * 16, g);
-      } else {
-        // dk_s += 2 dPsi_Y k_s (Y from the query-side G~: one triangle's
-        // entries) and dv_s += Z[:, 0:64]
-        __nv_bfloat162 u2[8];
-        load_row_sw<1>(smem + L::offK, m, u2);
-        float u[16], g[16];
-#pragma unroll
-        for (int x = 0; x < 8; ++x) {
-          u[2 * x] = __low2float(u2[x]);
-          u[2 * x + 1] = __high2float(u2[x]);
-        }
-        packed_grad_times_u<2, 2>(lane_base + L::colY, u, g);
-        if (t < T) add_to_bf16_row<16>(dk + ((size_t)bh * T + t) * 16, g);
-#pragma unroll
-        for (int b = 0; b < 2; ++b) {
-          uint32_t r[32];
-          tmem_ld32(lane_base + L::colZ + 32 * b, r);
-          tmem_wait_ld();
-          float z[32];
-#pragma unroll
-          for (int x = 0; x < 32; ++x) z[x] = __uint_as_float(r[x]);
-          if (t < T) add_to_bf16_row<32>(dv + ((size_t)bh * T + t) * kDV + 32 * b, z);
-        }
-      }
+      tc_fence_before();
+      mbar_arrive(ops_full);
     }
   }
 
@@ -466,35 +722,12 @@ __global__ void __launch_bounds__(kGThreads, 1)
 
 }  // namespace
 
-size_t chunk_bwd_records_bytes(int BH, int T) {
-  const size_t n_chunks = (size_t)(T + kTile - 1) / kTile;
-  return 2 * (size_t)BH * n_chunks * kRecRows * kNP * sizeof(float);
-}
-
-cudaError_t launch_chunk_bwd_inter_sm100(const void* q, const void* k, const void* v, const void* dO,
-                                         const float2* rowc, float* records, void* dq, void* dk, void* dv, int BH,
-                                         int T, const WaitCtl& wc, cudaStream_t st) {
-  const int n_chunks = (T + kTile - 1) / kTile;
-  if (n_chunks < 2) return cudaSuccess;  // no pair crosses a chunk boundary
-  CUtensorMap tq, tk, tv, tdo;
-  if (!make_tmap_bf16(&tq, q, 16, T, BH, kTile) || !make_tmap_bf16(&tk, k, 16, T, BH, kTile) ||
-      !make_tmap_bf16(&tv, v, kDV, T, BH, kTile) || !make_tmap_bf16(&tdo, dO, kDV, T, BH, kTile))
-    return cudaErrorInvalidValue;
-  const long long rf = (long long)kRecRows * kNP;
-  float* wsS = records;
-  float* wsG = records + (size_t)BH * n_chunks * rf;
-  cudaError_t e =
-      cudaFuncSetAttribute(chunk_grad_sums_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SumSmem::kBytes);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(chunk_grad_inter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             InterSmem::kBytes);
-  if (e != cudaSuccess) return e;
-  const dim3 grid(n_chunks, BH);
-  chunk_grad_sums_kernel<<<grid, kGThreads, SumSmem::kBytes, st>>>(tq, tk, tv, tdo, rowc, wsS, wsG, T, n_chunks, rf,
-                                                                    wc);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  // exclusive prefix over the chunks of each (b,h): S before chunk c, and
-  // (records in reverse order) G after chunk c
+ChunkPlan chunk_bwd_plan(int BH, int T) {
+  // Both walks of every super-chunk run at once, 2 BH G CTAs, one per SM at a
+  // time.  G (at most 16, so that the records scan in registers) is chosen by
+  // a cost in chunk steps on the busiest SM: waves x (chunks per walk + 2 for
+  // a CTA's set-up and drain), plus for G > 1 the sums pass (a sums step costs
+  // about half a walk step) and the scan.
   ChunkPlan pl{};
   pl.BH = BH;
   pl.T = T;
@@ -503,15 +736,67 @@ cudaError_t launch_chunk_bwd_inter_sm100(const void* q, const void* k, const voi
   pl.dv = kDV;
   pl.ld = kDV + 4;
   pl.C = kTile;
-  pl.Ls = kTile;
-  pl.G = n_chunks;
   pl.layout = kRecPackedT;
-  pl.record_floats = (size_t)rf;
-  if ((e = launch_state_scan(wsS, pl, n_chunks, nullptr, nullptr, nullptr, nullptr, st)) != cudaSuccess) return e;
-  if ((e = launch_state_scan(wsG, pl, n_chunks, nullptr, nullptr, nullptr, nullptr, st)) != cudaSuccess) return e;
-  chunk_grad_inter_kernel<<<grid, kGThreads, InterSmem::kBytes, st>>>(
-      tq, tk, tv, tdo, rowc, wsS, wsG, static_cast<__nv_bfloat16*>(dq), static_cast<__nv_bfloat16*>(dk),
-      static_cast<__nv_bfloat16*>(dv), T, n_chunks, rf, wc);
+  pl.record_floats = (size_t)kRecRows * kNP;
+  const long long tiles = (T + kTile - 1) / kTile;
+  auto waves = [](long long units) { return (units + kSMCount - 1) / kSMCount; };
+  long long best = -1, bestG = 1;
+  for (long long Gc = 1; Gc <= 16 && Gc <= (tiles > 0 ? tiles : 1); ++Gc) {
+    const long long per = (tiles + Gc - 1) / Gc;
+    const long long Geff = (tiles + per - 1) / per;
+    long long cost = 2 * waves(2 * (long long)BH * Geff) * (per + 2);  // in half steps
+    if (Geff > 1) cost += waves(2 * (long long)BH * (Geff - 1)) * (per + 4) + 4;
+    if (best < 0 || cost < best) {
+      best = cost;
+      bestG = Gc;
+    }
+  }
+  const long long per = tiles > 0 ? (tiles + bestG - 1) / bestG : 1;
+  pl.Ls = (int)(per * kTile);
+  pl.G = T > 0 ? (T + pl.Ls - 1) / pl.Ls : 0;
+  pl.workspace_bytes = pl.G > 1 ? 2 * (size_t)BH * pl.G * pl.record_floats * sizeof(float) : 0;
+  return pl;
+}
+
+size_t chunk_bwd_records_bytes(int BH, int T) { return chunk_bwd_plan(BH, T).workspace_bytes; }
+
+cudaError_t launch_chunk_bwd_inter_sm100(const void* q, const void* k, const void* v, const void* dO,
+                                         const float2* rowc, float* records, void* dq, void* dk, void* dv, int BH,
+                                         int T, const WaitCtl& wc, cudaStream_t st) {
+  const int n_chunks = (T + kTile - 1) / kTile;
+  if (n_chunks < 2) return cudaSuccess;  // no pair crosses a chunk boundary
+  const ChunkPlan pl = chunk_bwd_plan(BH, T);
+  CUtensorMap tq, tk, tv, tdo;
+  if (!make_tmap_bf16(&tq, q, 16, T, BH, kTile) || !make_tmap_bf16(&tk, k, 16, T, BH, kTile) ||
+      !make_tmap_bf16(&tv, v, kDV, T, BH, kTile) || !make_tmap_bf16(&tdo, dO, kDV, T, BH, kTile))
+    return cudaErrorInvalidValue;
+  cudaError_t e =
+      cudaFuncSetAttribute(chunk_grad_sums_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SumSmem::kBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(chunk_grad_walk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, WalkSmem::kBytes);
+  if (e != cudaSuccess) return e;
+  const long long rf = (long long)pl.record_floats;
+  const dim3 wgrid(pl.G, BH, 2);
+  auto* dqb = static_cast<__nv_bfloat16*>(dq);
+  auto* dkb = static_cast<__nv_bfloat16*>(dk);
+  auto* dvb = static_cast<__nv_bfloat16*>(dv);
+  if (pl.G > 1) {
+    if (!records) return cudaErrorInvalidValue;
+    chunk_grad_sums_kernel<<<dim3(pl.G - 1, BH, 2), kSumThreads, SumSmem::kBytes, st>>>(tq, tk, tv, tdo, rowc,
+                                                                                          records, T, pl.Ls, pl.G,
+                                                                                          rf, wc);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // exclusive prefix over the super-chunks of each of the 2 BH sequences:
+    // S~ entering super-chunk g, and (records in reverse order) G~ leaving it
+    ChunkPlan both = pl;
+    both.BH = 2 * BH;
+    if ((e = launch_state_scan(records, both, pl.G - 1, nullptr, nullptr, nullptr, nullptr, st)) != cudaSuccess)
+      return e;
+    return launch_pdl(chunk_grad_walk_kernel, wgrid, dim3(kWalkThreads), (size_t)WalkSmem::kBytes, st, tq, tk, tv,
+                      tdo, rowc, (const float*)records, dqb, dkb, dvb, T, pl.Ls, pl.G, rf, wc);
+  }
+  chunk_grad_walk_kernel<<<wgrid, kWalkThreads, WalkSmem::kBytes, st>>>(tq, tk, tv, tdo, rowc, nullptr, dqb, dkb,
+                                                                        dvb, T, pl.Ls, pl.G, rf, wc);
   return cudaGetLastError();
 }
 

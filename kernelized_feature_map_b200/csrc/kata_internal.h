@@ -134,11 +134,13 @@ cudaError_t launch_chunk_readout_sg(const void* q, const void* k, const void* v,
                                     const ChunkPlan& pl, int groups, const WaitCtl& wc, cudaStream_t st);
 
 // chunk_bwd_sm100.cu -- the inter-chunk part of the chunked backward (bf16,
-// p = 16, dv = 64, [B*H, T, *]): per-chunk state sums of the forward and of
-// the gradient, their scans, and the per-chunk gradient terms added to dq,
-// dk, dv (which the diagonal-only flash backward wrote first).  rowc is the
-// flash backward's per-row (-delta, 2/D); records needs
-// chunk_bwd_records_bytes().
+// p = 16, dv = 64, [B*H, T, *]): per-super-chunk sums of the forward state and
+// of the gradient state, their scan, and the two walks through each
+// super-chunk's chunks that add the gradient terms to dq, dk, dv (which the
+// diagonal-only flash backward wrote first).  rowc is the flash backward's
+// per-row (-delta, 2/D); records needs chunk_bwd_records_bytes() (0 when a
+// super-chunk spans the whole sequence).
+ChunkPlan chunk_bwd_plan(int BH, int T);
 size_t chunk_bwd_records_bytes(int BH, int T);
 cudaError_t launch_chunk_bwd_inter_sm100(const void* q, const void* k, const void* v, const void* dO,
                                          const float2* rowc, float* records, void* dq, void* dk, void* dv, int BH,

@@ -185,6 +185,24 @@ def test_mg_backward_matches_oracle(kata, shape):
     assert torch.equal(qa.grad, dq) and torch.equal(ka.grad, dk) and torch.equal(va.grad, dv)
 
 
+@pytest.mark.parametrize("B,H,T", [(4, 8, 1000), (1, 2, 5000)])
+def test_chunked_backward_is_deterministic(kata, B, H, T):
+    """Repeated calls give bitwise the same gradients: no role of the walk
+    kernels reads TMEM or shared memory that another role is still writing
+    (one super-chunk of 8 chunks per walk at B4 H8, several at B1 H2)."""
+    import torch
+    q, k, v = workloads.normal_qkv(B, H, T, 16, 64, seed=77 + T, dtype="bf16")
+    dO = np.random.default_rng(T).standard_normal((B, H, T, 64)).astype(np.float32)
+    qd, kd, vd, dOd = (to_dev(x, "bf16") for x in (q, k, v, dO))
+    o, D = kata.kata_fwd_chunked_train(qd, kd, vd)
+    first = [x.clone() for x in kata.kata_bwd_chunked(qd, kd, vd, o, D, dOd)]
+    for _ in range(4):
+        again = kata.kata_bwd_chunked(qd, kd, vd, o, D, dOd)
+        torch.cuda.synchronize()
+        assert all(torch.equal(a, b) for a, b in zip(first, again))
+    assert kata.kata_get_status() == 0
+
+
 @pytest.mark.parametrize("shape", [(2, 2, 700, 64, 4), (1, 3, 385, 32, 2), (1, 2, 256, 64, 2)])
 def test_sg_backward_matches_oracle(kata, shape):
     """KATA-Sigma-g gradients (one single-factor pass per query group x key
@@ -215,8 +233,11 @@ def test_sg_backward_matches_oracle(kata, shape):
 # ---------------------------------------------------------------------------
 
 # one chunk (no pair crosses a chunk boundary), a ragged second chunk, several
-# chunks, and enough (b,h) x chunks for many CTA waves
-@pytest.mark.parametrize("B,H,T", [(1, 2, 100), (1, 2, 200), (2, 3, 777), (4, 8, 1000), (1, 1, 4096)])
+# chunks, and enough (b,h) x chunks for many CTA waves.  The plan walks
+# T = 777 as 7 super-chunks and T = 4096 as 16 (summed and scanned first), the
+# other shapes as one super-chunk per sequence (each walk starts from zero)
+@pytest.mark.parametrize("B,H,T", [(1, 2, 100), (1, 2, 200), (2, 3, 777), (4, 8, 1000), (1, 1, 4096),
+                                   (8, 16, 520)])
 def test_chunked_backward_matches_oracle(kata, B, H, T):
     """Gradients of the chunked training path against the fp64 gradient
     oracle, with the gate of the flash-path backward; the training forward's
