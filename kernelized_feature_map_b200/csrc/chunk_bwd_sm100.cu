@@ -27,8 +27,8 @@
 //      against the copy of G~ leaving it,
 //        Y = V_c G~                    -> dk_s += 2 dPsi(Y_s + g~) k_s
 //        Z = psi~(K_c) G~^T            -> dv_s += Z_s
-//      then G~ takes in chunk c.  The gradient terms are added to the rows
-//      the diagonal pass wrote.
+//      then G~ takes in chunk c.  The walks write dq, dk, dv; the diagonal
+//      pass adds the pairs inside each chunk to them afterwards.
 // Packed coordinates as in chunk_common.cuh: the key side of S~ carries the
 // factor 2 off the diagonal, the query side of G~ does not.  Row 64 of each
 // state (z~ or g~) is kept in fp32 beside the bf16 copy and added in the
@@ -405,28 +405,13 @@ __device__ __forceinline__ void packed_grad_times_u(uint32_t taddr, const float*
   }
 }
 
-// Eight bf16 values (one uint4) plus the fp32 values add[0..7], rounded back
-// to bf16 in place
-__device__ __forceinline__ void add_bf16x8(uint4& old, const float* add) {
-  uint32_t* w = reinterpret_cast<uint32_t*>(&old);
+// 16 fp32 values rounded to bf16 and stored at row (32 bytes)
+__device__ __forceinline__ void store_bf16_row16(__nv_bfloat16* row, const float (&v)[16]) {
+  uint4* p4 = reinterpret_cast<uint4*>(row);
 #pragma unroll
-  for (int x = 0; x < 4; ++x) {
-    const float lo = __uint_as_float(w[x] << 16) + add[2 * x];
-    const float hi = __uint_as_float(w[x] & 0xffff0000u) + add[2 * x + 1];
-    w[x] = pack_bf16x2(lo, hi);
-  }
-}
-
-template <int N>
-__device__ __forceinline__ void store_bf16_row(__nv_bfloat16* row, const uint4 (&v)[N / 8]) {
-#pragma unroll
-  for (int q = 0; q < N / 8; ++q) reinterpret_cast<uint4*>(row)[q] = v[q];
-}
-
-template <int N>
-__device__ __forceinline__ void load_bf16_row(const __nv_bfloat16* row, uint4 (&out)[N / 8]) {
-#pragma unroll
-  for (int q = 0; q < N / 8; ++q) out[q] = __ldcg(reinterpret_cast<const uint4*>(row) + q);
+  for (int q = 0; q < 2; ++q)
+    p4[q] = make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                       pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
 }
 
 // blockIdx.z = 0: the S walk of super-chunk blockIdx.x (dq); 1: its G walk
@@ -555,12 +540,17 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
     mbar_wait_drain(mma_done, 0);
   } else if (warp < 6) {
     // ------------------------------------------------------------- epilogue
+    // writes every row of its walk (the diagonal pass adds to them later);
+    // the S walk's per-row constants are loaded a chunk ahead
     const int quarter = warp % 4;
     const int m = quarter * 32 + lane;
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    float2 rc_next = !gw && n_chunks > 0 ? load_rowc(rowc, bh, T, t0 + chunk_of(0) * kTile + m) : make_float2(0.f, 0.f);
     for (int i = 0; i < n_chunks; ++i) {
       const int st = i % kWalkStages;
       const int t = t0 + chunk_of(i) * kTile + m;
+      const float2 rc = rc_next;
+      if (!gw && i + 1 < n_chunks) rc_next = load_rowc(rowc, bh, T, t0 + chunk_of(i + 1) * kTile + m);
       if (!mbar_wait_w(kv_full + st, (i / kWalkStages) & 1, env)) break;
       // this token's q (S walk) or k (G walk) row, then the stage may go
       const uint8_t* tile = smem + L::offStage + st * L::kStage + 2 * kVBytes + (gw ? 0 : kQKBytes);
@@ -576,53 +566,40 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
       const bool live = t < T;
       const size_t r = (size_t)bh * T + (live ? t : 0);
       const float* zb = zbuf + (i & 1) * kNP;
+      if (!mbar_wait_w(z_ready + (i & 1), (i >> 1) & 1, env) || !mbar_wait_w(acc_full, i & 1, env)) break;
+      tc_fence_after();
+      float gr[16];
       if (!gw) {
-        const float2 rc = load_rowc(rowc, bh, T, t);
-        uint4 old[2];
-        if (live) load_bf16_row<16>(dq + r * 16, old);
-        if (!mbar_wait_w(z_ready + (i & 1), (i >> 1) & 1, env) || !mbar_wait_w(acc_full, i & 1, env)) break;
-        tc_fence_after();
-        float gq[16];
-        packed_grad_times_u<2, 1>(lane_base + L::colAcc, zb, 0.5f * rc.x * rc.y, u, gq);
+        packed_grad_times_u<2, 1>(lane_base + L::colAcc, zb, 0.5f * rc.x * rc.y, u, gr);
         tc_fence_before();
         mbar_arrive(acc_free);
-        if (live) {
-          add_bf16x8(old[0], gq);
-          add_bf16x8(old[1], gq + 8);
-          store_bf16_row<16>(dq + r * 16, old);
-        }
+        if (live) store_bf16_row16(dq + r * 16, gr);
       } else {
-        uint4 oldk[2], oldv[8];
-        if (live) {
-          load_bf16_row<16>(dk + r * 16, oldk);
-          load_bf16_row<kDV>(dv + r * kDV, oldv);
-        }
-        if (!mbar_wait_w(z_ready + (i & 1), (i >> 1) & 1, env) || !mbar_wait_w(acc_full, i & 1, env)) break;
-        tc_fence_after();
-        float gk[16];
-        packed_grad_times_u<2, 2>(lane_base + L::colAcc, zb, 1.f, u, gk);
-        // Z, 32 columns at a time, into the loaded dv row before the
-        // accumulators are released
+        packed_grad_times_u<2, 2>(lane_base + L::colAcc, zb, 1.f, u, gr);
+        // Z, 32 columns at a time, packed to bf16 before the accumulators
+        // are released
+        uint4 zv[8];
 #pragma unroll
         for (int hb = 0; hb < 2; ++hb) {
           uint32_t za[32];
           tmem_ld32(lane_base + L::colZ + 32 * hb, za);
           tmem_wait_ld();
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            float zf[8];
-#pragma unroll
-            for (int x = 0; x < 8; ++x) zf[x] = __uint_as_float(za[8 * q + x]);
-            add_bf16x8(oldv[4 * hb + q], zf);
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const uint32_t* e = za + 8 * q4;
+            zv[4 * hb + q4] = make_uint4(pack_bf16x2(__uint_as_float(e[0]), __uint_as_float(e[1])),
+                                         pack_bf16x2(__uint_as_float(e[2]), __uint_as_float(e[3])),
+                                         pack_bf16x2(__uint_as_float(e[4]), __uint_as_float(e[5])),
+                                         pack_bf16x2(__uint_as_float(e[6]), __uint_as_float(e[7])));
           }
         }
         tc_fence_before();
         mbar_arrive(acc_free);
         if (live) {
-          add_bf16x8(oldk[0], gk);
-          add_bf16x8(oldk[1], gk + 8);
-          store_bf16_row<16>(dk + r * 16, oldk);
-          store_bf16_row<kDV>(dv + r * kDV, oldv);
+          store_bf16_row16(dk + r * 16, gr);
+          uint4* dvr = reinterpret_cast<uint4*>(dv + r * kDV);
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4) dvr[q4] = zv[q4];
         }
       }
     }
@@ -636,7 +613,7 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
     uint8_t* sb = smem + L::offSB;
     // operands of the i-th chunk of the walk from its landed stage; false if
     // a wait gave up
-    auto operands = [&](int i) -> bool {
+    auto operands = [&](int i, float2 rc) -> bool {
       const int st = i % kWalkStages, pb = i & 1;
       uint8_t* stage = smem + L::offStage + st * L::kStage;
       const uint8_t* ktile = stage + 2 * kVBytes;
@@ -652,8 +629,6 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
         store_psi_k(smem + L::offPsi + pb * kPsiBytes, m, w);
         return true;
       }
-      const int t = t0 + chunk_of(i) * kTile + m;
-      const float2 rc = load_rowc(rowc, bh, T, t);
       scale_row_chunks_sw128(stage, m, 0.5f * rc.y, 0, 8);  // dN = dO / D
       if (!gw) return true;
       set_col0_sw128(smem + L::offBlk + pb * kOnesBytes, m, 0.5f * rc.x * rc.y);  // dD
@@ -686,15 +661,22 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
       init_state_half(row, lane_base + L::colState, sb, m, m < kDV, m == kDV ? zbuf : nullptr, half);
     }
     if (quarter == 2) mbar_arrive(z_ready);
-    bool ok = n_chunks > 0 && mbar_wait_w(kv_full, 0, env) && operands(0);
+    // group B's per-row constants, loaded a chunk ahead
+    auto rc_of = [&](int i) {
+      return !groupA && i < n_chunks ? load_rowc(rowc, bh, T, t0 + chunk_of(i) * kTile + m) : make_float2(0.f, 0.f);
+    };
+    float2 rc_cur = rc_of(0), rc_nxt = rc_of(1);
+    bool ok = n_chunks > 0 && mbar_wait_w(kv_full, 0, env) && operands(0, rc_cur);
     tmem_wait_st();  // the state's TMEM stores land before the first update reads them
     fence_proxy_async_smem();
     tc_fence_before();
     if (ok) mbar_arrive(ops_full);
     for (int i = 0; ok && i + 1 < n_chunks; ++i) {
       const int st1 = (i + 1) % kWalkStages;
+      rc_cur = rc_nxt;
+      rc_nxt = rc_of(i + 2);
       if (!mbar_wait_w(kv_full + st1, ((i + 1) / kWalkStages) & 1, env)) break;
-      if (!operands(i + 1)) break;
+      if (!operands(i + 1, rc_cur)) break;
       // the state after chunk i: this group's half of the copy (rows 0..63)
       // and of row 64 in fp32, for chunk i+1, once the epilogue has read the
       // products of chunk i out of TMEM (see the class comment)

@@ -802,6 +802,16 @@ static cudaError_t launch_bwd_t(const void* q, const void* k, const void* v, con
 
 }  // namespace
 
+cudaError_t launch_flash_bwd_rows(const void* dO, const void* o, const float* D, void* ws, int BH, int T,
+                                  cudaStream_t st) {
+  const long long rows = (long long)BH * T;
+  if (rows == 0) return cudaSuccess;
+  bwd_rows_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(dO),
+                                                                 static_cast<const __nv_bfloat16*>(o), D,
+                                                                 static_cast<float2*>(ws), rows);
+  return cudaGetLastError();
+}
+
 size_t flash_bwd_workspace_bytes(int BH, int T, int dv) {
   (void)dv;
   return (size_t)BH * T * sizeof(float2);  // (-delta, 1/D) per row

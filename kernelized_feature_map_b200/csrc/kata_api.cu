@@ -486,16 +486,19 @@ KATA_API kata_status_t kata_bwd_chunked(const void* q, const void* k, const void
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KATA_ERR_MISALIGNED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const WaitCtl wc = wait_ctl();
-  // the pairs inside each 128-token chunk: the flash backward on its diagonal
-  // tiles (which also computes the per-row constants); then the pairs across
-  // chunks through the chunk states
+  // the per-row constants; the pairs across chunks through the chunk states
+  // (written to dq, dk, dv); then the pairs inside each 128-token chunk, the
+  // flash backward on its diagonal tiles, added to them
   uint8_t* w8 = static_cast<uint8_t*>(workspace);
-  cudaError_t e = launch_flash_bwd_sm100(q, k, v, o, D, dO, dq, dk, dv, BH, T, p, p, false, false, false, false, w8,
-                                         wc, st, true);
-  if (e == cudaSuccess)
+  const bool inter = T > 128;  // some pair crosses a chunk boundary
+  cudaError_t e = launch_flash_bwd_rows(dO, o, D, w8, BH, T, st);
+  if (e == cudaSuccess && inter)
     e = launch_chunk_bwd_inter_sm100(q, k, v, dO, reinterpret_cast<const float2*>(w8),
                                      reinterpret_cast<float*>(w8 + round256(flash_bwd_workspace_bytes(BH, T, dv_width))),
                                      dq, dk, dv, BH, T, wc, st);
+  if (e == cudaSuccess)
+    e = launch_flash_bwd_sm100(q, k, v, o, D, dO, dq, dk, dv, BH, T, p, p, true, inter, inter, inter, w8, wc, st,
+                               true);
   return from_cuda(e);
 }
 

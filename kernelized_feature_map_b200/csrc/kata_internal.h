@@ -95,6 +95,10 @@ cudaError_t launch_flash_sm100(const void* q, const void* k, const void* v, void
 // diag_only only the pairs of each 128-token tile with itself are taken (the
 // intra-chunk part of the chunked backward).
 size_t flash_bwd_workspace_bytes(int BH, int T, int dv);
+// The per-row constants (-delta_t, 2/D_t) of the flash backward alone, into
+// the first flash_bwd_workspace_bytes() of ws.
+cudaError_t launch_flash_bwd_rows(const void* dO, const void* o, const float* D, void* ws, int BH, int T,
+                                  cudaStream_t st);
 cudaError_t launch_flash_bwd_sm100(const void* q, const void* k, const void* v, const void* o, const float* D,
                                    const void* dO, void* dq, void* dk, void* dv, int BH, int T, int p, int ld,
                                    bool rows_ready, bool dv_accumulate, bool dq_accumulate, bool dk_accumulate,
@@ -136,10 +140,10 @@ cudaError_t launch_chunk_readout_sg(const void* q, const void* k, const void* v,
 // chunk_bwd_sm100.cu -- the inter-chunk part of the chunked backward (bf16,
 // p = 16, dv = 64, [B*H, T, *]): per-super-chunk sums of the forward state and
 // of the gradient state, their scan, and the two walks through each
-// super-chunk's chunks that add the gradient terms to dq, dk, dv (which the
-// diagonal-only flash backward wrote first).  rowc is the flash backward's
-// per-row (-delta, 2/D); records needs chunk_bwd_records_bytes() (0 when a
-// super-chunk spans the whole sequence).
+// super-chunk's chunks that write the gradient terms to dq, dk, dv (which the
+// diagonal-only flash backward adds to afterwards).  rowc is the flash
+// backward's per-row (-delta, 2/D); records needs chunk_bwd_records_bytes()
+// (0 when a super-chunk spans the whole sequence).
 ChunkPlan chunk_bwd_plan(int BH, int T);
 size_t chunk_bwd_records_bytes(int BH, int T);
 cudaError_t launch_chunk_bwd_inter_sm100(const void* q, const void* k, const void* v, const void* dO,
