@@ -269,8 +269,9 @@ __global__ void __launch_bounds__(kSumThreads, 1)
 //   warp 0       TMA: [dO | V | K | Q] tiles of each chunk into a 2-stage ring
 //   warp 1       TMEM allocator; MMA issue (the whole warp, one elected lane)
 //   warps 2-5    epilogue: token m = lane quarter * 32 + lane of the chunk
-//   warps 6-9    S walk: psi~(K) into shared memory; G walk: psi~(Q) into
-//                shared memory; then half 0 of the state copy
+//   warps 6-9    S walk: psi~(K); G walk: psi~(Q), formed and stored once
+//                the update by the chunk before has read the buffer; then
+//                half 0 of the state copy
 //   warps 10-13  dN in place (and for the G walk dD, and psi~(K) into TMEM);
 //                then half 1 of the state copy
 // MMA order per chunk: the products against the copy of the state entering
@@ -286,14 +287,18 @@ __global__ void __launch_bounds__(kSumThreads, 1)
 // super-chunk of 8 chunks per walk); with this hand-over every run is
 // bitwise the same.
 constexpr int kWalkThreads = 448;
-constexpr int kWalkStages = 2;
+// Three stages of the ring, so that the next chunks' loads are in flight
+// while a chunk is worked on; that leaves room for one psi~ buffer, which the
+// operand warps fill once the update by the chunk before has read it.  Measured at B1 H16 T131072 (backward): 2 stages and 2 psi~
+// buffers 1.99 ms.
+constexpr int kWalkStages = 3;
 
 struct WalkSmem {
   static constexpr int kStage = 2 * kVBytes + 2 * kQKBytes;  // [dO | V | K | Q]
   static constexpr int offStage = 0;
   static constexpr int offBlk = offStage + kWalkStages * kStage;  // ones (S walk) or 2 dD blocks (G walk)
-  static constexpr int offPsi = offBlk + 2 * kOnesBytes;          // 2 psi~ buffers
-  static constexpr int offSB = offPsi + 2 * kPsiBytes;            // bf16 copy of the state
+  static constexpr int offPsi = offBlk + 2 * kOnesBytes;          // psi~ buffer
+  static constexpr int offSB = offPsi + kPsiBytes;                // bf16 copy of the state
   static constexpr int offZ = offSB + kSBBytes;                   // 2 x 144 fp32: row 64 of the state
   static constexpr int offBar = offZ + 2 * kNP * 4;
   static constexpr int kBars = 2 * kWalkStages + 8;
@@ -529,7 +534,7 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
       // the state takes in the chunk: S~^T += [V | 1]^T psi~(K), or
       // G~^T += [dN | dD]^T psi~(Q)
       const uint64_t du = gw ? desc_vones(sDO, sBlk + pb * kOnesBytes) : desc_vones(sV, sBlk);
-      const uint64_t db = desc_add(dpsi, pb * kPsiBytes);
+      const uint64_t db = dpsi;
 #pragma unroll
       for (int ks = 0; ks < kTile / 16; ++ks)
         mma_ss_w(tmem + L::colState, desc_add(du, ks * 2048), desc_add(db, ks * 512), id_u, 1);
@@ -611,24 +616,26 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
     const int m = quarter * 32 + lane;  // token of the chunk / TMEM lane = state row
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
     uint8_t* sb = smem + L::offSB;
-    // operands of the i-th chunk of the walk from its landed stage; false if
-    // a wait gave up
-    auto operands = [&](int i, float2 rc) -> bool {
+    // group A: the row of the i-th chunk of the walk that psi~ is formed from
+    // (k for the S walk, key side; q for the G walk, query side), read from
+    // its landed stage; psi~ is formed and stored once the update by the
+    // chunk before has read the buffer (holding the 72 words across the waits
+    // would spill)
+    __nv_bfloat162 u_psi[8];
+    auto load_psi_row = [&](int i) {
+      const uint8_t* ktile = smem + L::offStage + (i % kWalkStages) * L::kStage + 2 * kVBytes;
+      load_row_sw<1>(gw ? ktile + kQKBytes : ktile, m, u_psi);
+    };
+    auto store_psi = [&]() {
+      uint32_t w[kNPW];
+      if (gw) packed_psi<false>(u_psi, w);
+      else packed_psi<true>(u_psi, w);
+      store_psi_k(smem + L::offPsi, m, w);
+    };
+    // group B: the other operands of the i-th chunk; false if a wait gave up
+    auto operands_b = [&](int i, float2 rc) -> bool {
       const int st = i % kWalkStages, pb = i & 1;
       uint8_t* stage = smem + L::offStage + st * L::kStage;
-      const uint8_t* ktile = stage + 2 * kVBytes;
-      const uint8_t* qtile = ktile + kQKBytes;
-      if (groupA) {
-        // psi~(K) (S walk, key side) or psi~(Q) (G walk, query side) into
-        // buffer pb, last read by the update by chunk i-2
-        __nv_bfloat162 u[8];
-        uint32_t w[kNPW];
-        load_row_sw<1>(gw ? qtile : ktile, m, u);
-        if (gw) packed_psi<false>(u, w);
-        else packed_psi<true>(u, w);
-        store_psi_k(smem + L::offPsi + pb * kPsiBytes, m, w);
-        return true;
-      }
       scale_row_chunks_sw128(stage, m, 0.5f * rc.y, 0, 8);  // dN = dO / D
       if (!gw) return true;
       set_col0_sw128(smem + L::offBlk + pb * kOnesBytes, m, 0.5f * rc.x * rc.y);  // dD
@@ -636,7 +643,7 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
       // and the epilogue has read the products of chunk i-1
       __nv_bfloat162 u[8];
       uint32_t w[kNPW];
-      load_row_sw<1>(ktile, m, u);
+      load_row_sw<1>(stage + 2 * kVBytes, m, u);
       packed_psi<true>(u, w);
       if (i > 0) {
         if (!mbar_wait_w(acc_free, (i - 1) & 1, env)) return false;
@@ -666,7 +673,12 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
       return !groupA && i < n_chunks ? load_rowc(rowc, bh, T, t0 + chunk_of(i) * kTile + m) : make_float2(0.f, 0.f);
     };
     float2 rc_cur = rc_of(0), rc_nxt = rc_of(1);
-    bool ok = n_chunks > 0 && mbar_wait_w(kv_full, 0, env) && operands(0, rc_cur);
+    bool ok = n_chunks > 0 && mbar_wait_w(kv_full, 0, env);
+    if (ok && groupA) {
+      load_psi_row(0);
+      store_psi();
+    }
+    if (ok && !groupA) ok = operands_b(0, rc_cur);
     tmem_wait_st();  // the state's TMEM stores land before the first update reads them
     fence_proxy_async_smem();
     tc_fence_before();
@@ -676,12 +688,15 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
       rc_cur = rc_nxt;
       rc_nxt = rc_of(i + 2);
       if (!mbar_wait_w(kv_full + st1, ((i + 1) / kWalkStages) & 1, env)) break;
-      if (!operands(i + 1, rc_cur)) break;
+      if (groupA) load_psi_row(i + 1);
+      else if (!operands_b(i + 1, rc_cur)) break;
       // the state after chunk i: this group's half of the copy (rows 0..63)
       // and of row 64 in fp32, for chunk i+1, once the epilogue has read the
-      // products of chunk i out of TMEM (see the class comment)
+      // products of chunk i out of TMEM (see the class comment); group A's
+      // psi~ into the buffer the update by chunk i has read
       if (!mbar_wait_w(upd_done, i & 1, env) || !mbar_wait_w(acc_free, i & 1, env)) break;
       tc_fence_after();
+      if (groupA) store_psi();
       if (quarter < 2) {
         state_half_to_bf16(lane_base + L::colState, sb, m, true, half);
       } else if (quarter == 2) {
