@@ -55,12 +55,16 @@ using namespace chunk;
 constexpr int kSMCount = 148;
 
 // Scales the bf16 row t of a 128B-swizzled [128 x 64] tile by s in place:
-// physical 16-byte chunks c0 .. c0 + n - 1 (the swizzle only permutes a row's
-// chunks, and the scale is the same for the whole row).
-__device__ __forceinline__ void scale_row_chunks_sw128(uint8_t* tile, int t, float s, int c0, int n) {
+// n of its physical 16-byte chunks, c0, c0 + step, ... (the swizzle only
+// permutes a row's chunks, and the scale is the same for the whole row).
+// Rows are 128 bytes apart, so the threads of a warp (consecutive rows) start
+// at different chunks (rotated by t): with the same chunk in every row all 32
+// accesses of an instruction fell into the same four banks.
+__device__ __forceinline__ void scale_row_chunks_sw128(uint8_t* tile, int t, float s, int c0, int n, int step) {
   uint4* row = reinterpret_cast<uint4*>(tile + t * 128);
-#pragma unroll 4
-  for (int c = c0; c < c0 + n; ++c) {
+#pragma unroll
+  for (int j = 0; j < n; ++j) {
+    const int c = (c0 + step * (j + t)) & 7;
     uint4 a = row[c];
     uint32_t* w = reinterpret_cast<uint32_t*>(&a);
 #pragma unroll
@@ -237,7 +241,7 @@ __global__ void __launch_bounds__(kSumThreads, 1)
       if (grad) {
         // dN = dO / D in place (this thread's half of the row); dD into
         // column 0 of the block that follows dN in the A operand
-        scale_row_chunks_sw128(stage, tid, 0.5f * rc.y, 4 * half, 4);
+        scale_row_chunks_sw128(stage, tid, 0.5f * rc.y, half, 4, 2);  // chunks of parity `half`
         if (half == 0) set_col0_sw128(smem + L::offBlk + pb * kOnesBytes, tid, 0.5f * rc.x * rc.y);
       }
       fence_proxy_async_smem();
@@ -636,7 +640,7 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
     auto operands_b = [&](int i, float2 rc) -> bool {
       const int st = i % kWalkStages, pb = i & 1;
       uint8_t* stage = smem + L::offStage + st * L::kStage;
-      scale_row_chunks_sw128(stage, m, 0.5f * rc.y, 0, 8);  // dN = dO / D
+      scale_row_chunks_sw128(stage, m, 0.5f * rc.y, 0, 8, 1);  // dN = dO / D
       if (!gw) return true;
       set_col0_sw128(smem + L::offBlk + pb * kOnesBytes, m, 0.5f * rc.x * rc.y);  // dD
       // psi~(K) into TMEM once the Z of chunk i-1 has read the previous one
