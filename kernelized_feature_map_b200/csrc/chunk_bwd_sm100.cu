@@ -384,31 +384,35 @@ __device__ __forceinline__ void packed_grad_times_u(uint32_t taddr, const float*
                                                     const float (&u)[16], float (&out)[16]) {
 #pragma unroll
   for (int i = 0; i < 16; ++i) out[i] = 0.f;
+  // two TMEM loads (32 columns) in flight per wait
 #pragma unroll
-  for (int b = 0; b < 9; ++b) {
-    uint32_t r[16];
-    tmem_ld16(taddr + 16 * b, r);
-    float zv[16];
+  for (int b0 = 0; b0 < 9; b0 += 2) {
+    uint32_t r[2][16];
 #pragma unroll
-    for (int x = 0; x < 16; x += 4) {
-      const float4 z4 = *reinterpret_cast<const float4*>(zb + 16 * b + x);
-      zv[x] = z4.x;
-      zv[x + 1] = z4.y;
-      zv[x + 2] = z4.z;
-      zv[x + 3] = z4.w;
-    }
+    for (int bb = 0; bb < 2; ++bb)
+      if (b0 + bb < 9) tmem_ld16(taddr + 16 * (b0 + bb), r[bb]);
     tmem_wait_ld();
 #pragma unroll
-    for (int x = 0; x < 16; ++x) {
-      const int w = 16 * b + x;
-      const int i = packed_i(w), j = packed_j(w);
-      if (i < 0) continue;
-      const float gr = fmaf(coef, zv[x], __uint_as_float(r[x]));
-      if (i == j) {
-        out[i] = fmaf((float)kFDiag * gr, u[i], out[i]);
-      } else {
-        out[i] = fmaf((float)kFOff * gr, u[j], out[i]);
-        out[j] = fmaf((float)kFOff * gr, u[i], out[j]);
+    for (int bb = 0; bb < 2; ++bb) {
+      const int b = b0 + bb;
+      if (b >= 9) continue;
+#pragma unroll
+      for (int x = 0; x < 16; x += 4) {
+        const float4 z4 = *reinterpret_cast<const float4*>(zb + 16 * b + x);
+        const float zv[4] = {z4.x, z4.y, z4.z, z4.w};
+#pragma unroll
+        for (int y = 0; y < 4; ++y) {
+          const int w = 16 * b + x + y;
+          const int i = packed_i(w), j = packed_j(w);
+          if (i < 0) continue;
+          const float gr = fmaf(coef, zv[y], __uint_as_float(r[bb][x + y]));
+          if (i == j) {
+            out[i] = fmaf((float)kFDiag * gr, u[i], out[i]);
+          } else {
+            out[i] = fmaf((float)kFOff * gr, u[j], out[i]);
+            out[j] = fmaf((float)kFOff * gr, u[i], out[j]);
+          }
+        }
       }
     }
   }
