@@ -49,12 +49,13 @@ METRIC = "KATA-Mg fwd tokens/sec at T=2k and 131k (1 B200); % of roofline"
 UNIT = "tokens/s"
 
 # DRAM bytes (read + write) of one flash_fwd_kernel launch at B8 H16 T2048,
-# from the ncu capture summarised in profiles/flash_fwd_kernel_ctx2k.md.  It
-# is reported only while the kernel's sources are the ones that capture ran.
-FLASH_TRAFFIC_BYTES = 50472704 + 6547712
+# from the ncu capture summarised in profiles/flash_fwd_kernel_ctx2k.md (the
+# traffic recapture).  It is reported only while the kernel's sources are the
+# ones that capture ran.
+FLASH_TRAFFIC_BYTES = 50576640 + 6089984
 FLASH_TRAFFIC_SOURCES = ("kernelized_feature_map_b200/csrc/flash_sm100.cu", "kernelized_feature_map_b200/csrc/sm100.cuh",
                          "kernelized_feature_map_b200/csrc/kata_trace.cuh", "kernelized_feature_map_b200/csrc/kata_common.cuh")
-FLASH_TRAFFIC_SHA256 = "ab7f7563bcf48676323ac1b90d0185ccad44e79b9b632361233c127cf371f620"
+FLASH_TRAFFIC_SHA256 = "7f2726d66afacd6130957ecff278be8d9136251b02fe3e367a30c61ce87e8e25"
 
 
 def flash_traffic(workload):
