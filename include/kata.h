@@ -263,14 +263,18 @@ kata_status_t kata_bwd_quadratic(const void* q, const void* k, const void* v, co
  * initial or final state) that also writes each row's denominator D
  * [B,H,T] fp32.  kata_bwd_chunked gives the gradients (dq, dk, dv; layouts
  * of q, k, v; bf16) of the same function as kata_bwd_quadratic, from o, D
- * and dO: the pairs inside each 128-token chunk with the flash backward
- * kernels on their diagonal tiles, the pairs across chunks through the
- * per-chunk states of the forward (S before each chunk) and of the gradient
- * (sum over later tokens of psi(q_t) [dN_t | dD_t]^T) and their scans, so
- * that work and memory are linear in T.  Workspace:
- * kata_bwd_chunked_workspace_size() bytes, 256-byte aligned (8 bytes per row
- * plus two 65 x 144 fp32 records per 128-token chunk of every (b,h)).
- * Other sizes: KATA_ERR_UNSUPPORTED.  Streams and errors as above.
+ * and dO: the pairs across 128-token chunks through two walks over the
+ * chunks of each super-chunk, one carrying the forward state (S before each
+ * chunk) for dq, one carrying the gradient state (sum over later tokens of
+ * psi(q_t) [dN_t | dD_t]^T) backwards for dk and dv, each entering its
+ * super-chunk from a scan of per-super-chunk sums; then the pairs inside each
+ * chunk with the flash backward kernels on their diagonal tiles, added to
+ * those.  Work and memory are linear in T.  Workspace:
+ * kata_bwd_chunked_workspace_size() bytes, 256-byte aligned (8 bytes per row,
+ * rounded up to 256, plus, when a sequence is split into G > 1 super-chunks,
+ * two 65 x 144 fp32 records per super-chunk of every (b,h)).  Repeated calls
+ * give bitwise the same gradients.  Other sizes: KATA_ERR_UNSUPPORTED.
+ * Streams and errors as above.
  */
 kata_status_t kata_fwd_chunked_train(const void* q, const void* k, const void* v, void* o, float* D,
                                      int B, int H, int T, int p, int dv, int C, kata_dtype_t dtype,

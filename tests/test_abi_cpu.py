@@ -71,6 +71,30 @@ def test_workspace_size_query(L):
     assert sizes == sorted(sizes)
 
 
+def _round256(n):
+    return (n + 255) // 256 * 256
+
+
+def test_chunked_backward_workspace_size(L):
+    """kata_bwd_chunked's workspace: 8 bytes per row (rounded up to 256) and,
+    when the plan splits a sequence into G > 1 super-chunks, two 65 x 144 fp32
+    records (forward and gradient state sums) per super-chunk of every (b,h).
+    The plan keeps one super-chunk when the (b,h) walks alone fill the SMs
+    (B8 H16 T2048: 256 walks of 16 chunks) and splits long sequences so that
+    both walks of every super-chunk run in about two waves (B1 H16 T131072:
+    9 super-chunks, 288 walks of 114 chunks)."""
+    f = L.kata_bwd_chunked_workspace_size
+    rec = 2 * 65 * 144 * 4
+    assert f(8, 16, 2048, 16, 64, 1) == _round256(8 * 16 * 2048 * 8)
+    assert f(1, 16, 131072, 16, 64, 1) == _round256(16 * 131072 * 8) + 16 * 9 * rec
+    # B1 H1 T4096: 32 chunks, walks of 2 chunks in 16 super-chunks (one wave)
+    assert f(1, 1, 4096, 16, 64, 1) == _round256(4096 * 8) + 16 * rec
+    # a single chunk has no pair across chunks, but the row constants remain
+    assert f(1, 2, 100, 16, 64, 1) == _round256(2 * 100 * 8)
+    # other shapes and fp32 are not served
+    assert f(1, 1, 1000, 32, 64, 1) == 0 and f(1, 1, 1000, 16, 16, 1) == 0 and f(1, 1, 1000, 16, 64, 0) == 0
+
+
 VP = ctypes.c_void_p
 
 
