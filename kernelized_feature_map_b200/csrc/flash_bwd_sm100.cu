@@ -209,6 +209,22 @@ __device__ __forceinline__ void add_row16(const __nv_bfloat16* src_row, uint32_t
   }
 }
 
+// The same, from the two 16-byte words of the row loaded earlier.
+__device__ __forceinline__ void add_row16_words(const uint4 (&old)[2], uint32_t (&r)[16]) {
+  const uint32_t w[8] = {old[0].x, old[0].y, old[0].z, old[0].w, old[1].x, old[1].y, old[1].z, old[1].w};
+#pragma unroll
+  for (int x = 0; x < 8; ++x) {
+    r[2 * x] = __float_as_uint(__uint_as_float(r[2 * x]) + __uint_as_float(w[x] << 16));
+    r[2 * x + 1] = __float_as_uint(__uint_as_float(r[2 * x + 1]) + __uint_as_float(w[x] & 0xffff0000u));
+  }
+}
+
+__device__ __forceinline__ void load_row16_words(const __nv_bfloat16* src_row, uint4 (&old)[2]) {
+  const uint4* src = reinterpret_cast<const uint4*>(src_row);
+  old[0] = src[0];
+  old[1] = src[1];
+}
+
 __device__ __forceinline__ void store_row16(__nv_bfloat16* dst_row, const uint32_t (&r)[16]) {
   uint4* dst = reinterpret_cast<uint4*>(dst_row);
   dst[0] = make_uint4(pack_bf16x2(__uint_as_float(r[0]), __uint_as_float(r[1])),
@@ -743,6 +759,16 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         mbar_arrive(p_full);
         if (tslot >= 0) KATA_TRACE(bwd, g, tslot + 3);
       }
+      // rows another pass wrote, loaded before the accumulators are complete
+      // so that their latency overlaps the item's last MMAs
+      const int row = tile * kBw + quarter * 32 + lane;  // this thread's key
+      const size_t r0 = (size_t)bh * T + (row < T ? row : 0);
+      uint4 old_v[2], old_k0[2], old_k1[2];
+      if (dv_accumulate && row < T) load_row16_words(dv + r0 * kBwDV + 16 * kq, old_v);
+      if (dk_accumulate && kq == 0 && row < T) {
+        load_row16_words(dk + r0 * ld, old_k0);
+        if constexpr (p == 32) load_row16_words(dk + r0 * ld + 16, old_k1);
+      }
       if (!ok || !mbar_wait_w(acc_full, acc_cnt & 1, env)) break;
       ++acc_cnt;
       tc_fence_after();
@@ -760,16 +786,14 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       // dV was accumulated with r = 2 / D: halve it (exact)
 #pragma unroll
       for (int x = 0; x < 16; ++x) rv[x] = __float_as_uint(0.5f * __uint_as_float(rv[x]));
-      const int row = tile * kBw + quarter * 32 + lane;  // this thread's key
       if (row < T) {
-        const size_t r0 = (size_t)bh * T + row;
         __nv_bfloat16* dvr = dv + r0 * kBwDV + 16 * kq;
-        if (dv_accumulate) add_row16(dvr, rv);  // another pass's dV is already there
+        if (dv_accumulate) add_row16_words(old_v, rv);  // another pass's dV is already there
         store_row16(dvr, rv);
         if (kq == 0) {
           if (dk_accumulate) {
-            add_row16(dk + r0 * ld, rk0);
-            if constexpr (p == 32) add_row16(dk + r0 * ld + 16, rk1);
+            add_row16_words(old_k0, rk0);
+            if constexpr (p == 32) add_row16_words(old_k1, rk1);
           }
           store_row16(dk + r0 * ld, rk0);
           if constexpr (p == 32) store_row16(dk + r0 * ld + 16, rk1);
