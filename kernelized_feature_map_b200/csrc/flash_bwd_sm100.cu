@@ -467,6 +467,12 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         tc_fence_before();
         mbar_arrive(p_full + (g & 1));
       }
+      // the rows another pass wrote, loaded before the accumulator is
+      // complete so that their latency overlaps the item's last MMAs
+      // (p = 16 only: at p = 32 the registers held across the wait spill)
+      uint4 old0[2];
+      if constexpr (p == 16)
+        if (dq_accumulate && kq == 0 && row < T) load_row16_words(dq + ((size_t)bh * T + row) * ld, old0);
       if (!ok || !mbar_wait_w(acc_full, acc_cnt & 1, env)) break;
       ++acc_cnt;
       tc_fence_after();
@@ -483,8 +489,12 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       if (kq == 0 && row < T) {
         __nv_bfloat16* dqr = dq + ((size_t)bh * T + row) * ld;
         if (dq_accumulate) {
-          add_row16(dqr, r0);
-          if constexpr (p == 32) add_row16(dqr + 16, r1);
+          if constexpr (p == 16) {
+            add_row16_words(old0, r0);
+          } else {
+            add_row16(dqr, r0);
+            add_row16(dqr + 16, r1);
+          }
         }
         store_row16(dqr, r0);
         if constexpr (p == 32) store_row16(dqr + 16, r1);
@@ -763,11 +773,11 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       // so that their latency overlaps the item's last MMAs
       const int row = tile * kBw + quarter * 32 + lane;  // this thread's key
       const size_t r0 = (size_t)bh * T + (row < T ? row : 0);
-      uint4 old_v[2], old_k0[2], old_k1[2];
-      if (dv_accumulate && row < T) load_row16_words(dv + r0 * kBwDV + 16 * kq, old_v);
-      if (dk_accumulate && kq == 0 && row < T) {
-        load_row16_words(dk + r0 * ld, old_k0);
-        if constexpr (p == 32) load_row16_words(dk + r0 * ld + 16, old_k1);
+      // (p = 16 only: at p = 32 the registers held across the wait spill)
+      uint4 old_v[2], old_k0[2];
+      if constexpr (p == 16) {
+        if (dv_accumulate && row < T) load_row16_words(dv + r0 * kBwDV + 16 * kq, old_v);
+        if (dk_accumulate && kq == 0 && row < T) load_row16_words(dk + r0 * ld, old_k0);
       }
       if (!ok || !mbar_wait_w(acc_full, acc_cnt & 1, env)) break;
       ++acc_cnt;
@@ -788,12 +798,19 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       for (int x = 0; x < 16; ++x) rv[x] = __float_as_uint(0.5f * __uint_as_float(rv[x]));
       if (row < T) {
         __nv_bfloat16* dvr = dv + r0 * kBwDV + 16 * kq;
-        if (dv_accumulate) add_row16_words(old_v, rv);  // another pass's dV is already there
+        if (dv_accumulate) {  // another pass's dV is already there
+          if constexpr (p == 16) add_row16_words(old_v, rv);
+          else add_row16(dvr, rv);
+        }
         store_row16(dvr, rv);
         if (kq == 0) {
           if (dk_accumulate) {
-            add_row16_words(old_k0, rk0);
-            if constexpr (p == 32) add_row16_words(old_k1, rk1);
+            if constexpr (p == 16) {
+              add_row16_words(old_k0, rk0);
+            } else {
+              add_row16(dk + r0 * ld, rk0);
+              add_row16(dk + r0 * ld + 16, rk1);
+            }
           }
           store_row16(dk + r0 * ld, rk0);
           if constexpr (p == 32) store_row16(dk + r0 * ld + 16, rk1);
