@@ -103,6 +103,12 @@ def chunked_bytes(BH, T, p, dv, elem=2):
     return BH * T * (2 * p + 2 * dv) * elem
 
 
+def chunked_bwd_bytes(BH, T, p, dv, elem=2):
+    """The chunked backward's HBM work: q, k, v, o, dO and D read once, dq,
+    dk, dv written once: (4p + 4dv) elements and 4 bytes per token-head."""
+    return BH * T * ((4 * p + 4 * dv) * elem + 4)
+
+
 def decode_bytes(BH, p, dv, elem=2):
     """State S (P x dv fp32) and z (P fp32) read and written; q,k,v read, o written."""
     P = p * p
@@ -399,7 +405,9 @@ def run_ours(args, rank, world, local_rank):
                 t0 = time.time()
                 long["first_order"] = run_first_order(args, K, torch, dev, stream, flush)
                 windows["first_order"] = (t0, time.time())
+                t0 = time.time()
                 long["train"] = run_train(args, K, torch, dev, stream, flush)
+                windows["train"] = (t0, time.time())
         t_end = time.time()
         time.sleep(0.15)
         clk.window = (windows["step"][0], windows.get("decode_b64", windows["step"])[1])
@@ -985,6 +993,20 @@ def roofline_points(res, peaks, cfg):
                 pts.append(tensor_point("mg_quadratic", wl, m["ms"], m["B"] * m["T"],
                                         flash_flops(m["B"] * m["H"], m["T"], m["d"], m["dv"]), cl.get("mg"),
                                         T=m["T"], groups=m["groups"]))
+        # the training backward passes: the flash path (tensor, 2(3p+2dv)
+        # flops per causal pair) and the chunked path (HBM, 8p + 8dv + 4
+        # bytes per token-head)
+        tr = lg.get("train")
+        if tr:
+            wt = "backward B=%d H=%d T=%d p=%d dv=%d bf16" % (tr["B"], tr["H"], tr["T"], tr["p"], tr["dv"])
+            pairs = tr["B"] * tr["H"] * tr["T"] * (tr["T"] + 1) / 2
+            pts.append(tensor_point("bwd_quadratic", wt, tr["bwd_ms"], tr["B"] * tr["T"],
+                                    pairs * 2 * (3 * tr["p"] + 2 * tr["dv"]), cl.get("train"), T=tr["T"]))
+            for c in tr.get("chunked", {}).values():
+                wc = "backward B=%d H=%d T=%d p=%d dv=%d bf16" % (c["B"], c["H"], c["T"], tr["p"], tr["dv"])
+                pts.append(hbm_point("bwd_chunked", wc, c["bwd_ms"], c["B"] * c["T"],
+                                     chunked_bwd_bytes(c["B"] * c["H"], c["T"], tr["p"], tr["dv"]), cl.get("train"),
+                                     T=c["T"]))
         # first-order attention at B1 H16 T131072: both forms
         for g in lg.get("first_order", []):
             if g["B"] != 1 or g["T"] != 131072:
@@ -1136,7 +1158,11 @@ def report(args, res, step_ms, e2e_ms, world):
                 name: {"workload": "training step of the O(T) chunked path B=%d H=%d T=%d p=%d dv=%d bf16 (forward "
                                    "saving D, then the chunked backward)" % (c["B"], c["H"], c["T"], tr["p"], tr["dv"]),
                        "fwd_ms": c["fwd_ms"], "bwd_ms": c["bwd_ms"], "step_ms": c["step_ms"],
-                       "tokens_per_s": c["B"] * c["T"] / (c["step_ms"] * 1e-3)}
+                       "tokens_per_s": c["B"] * c["T"] / (c["step_ms"] * 1e-3),
+                       "bwd_hbm_frac": chunked_bwd_bytes(c["B"] * c["H"], c["T"], tr["p"], tr["dv"])
+                       / (c["bwd_ms"] * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                       "bwd_algorithmic": "q, k, v, o, dO, D read and dq, dk, dv written once: 8p + 8dv + 4 bytes "
+                                          "per token-head"}
                 for name, c in tr.get("chunked", {}).items()}
     line["roofline"]["points"] = roofline_points(res, peaks, cfg)
     if args.cpu_baseline and world == 1:
