@@ -17,7 +17,8 @@ def _fake_result():
     long = dict(B=1, H=16, T=131072, p=16, dv=64, chunked_C64_ms=0.235, chunked_C128_ms=0.234, quadratic_ms=29.0,
                 sequential_C64_ms=1.25, decode_b64=dict(B=64, H=16, p=16, dv=64, ms=0.03), sweep=grid,
                 recall=dict(B=4, H=16, T=8192, p=32, dv=64, chunked_ms=13.8, quadratic_ms=0.51), mg=mg,
-                train=dict(B=8, H=16, T=2048, p=16, dv=64, fwd_ms=0.08, bwd_ms=0.36, step_ms=0.43))
+                train=dict(B=8, H=16, T=2048, p=16, dv=64, fwd_ms=0.08, bwd_ms=0.36, step_ms=0.43,
+                           chunked={"B1_T131072": dict(B=1, H=16, T=131072, fwd_ms=0.25, bwd_ms=1.6, step_ms=1.85)}))
     return dict(step_ms=0.116, eager_step_ms=0.125, graph=True, path_ms=[0.081, 0.035, 0.0088], e2e_ms=11.0,
                 h2d=50356224, d2h=67125248, clocks={"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []},
                 timed_s=0.5, long=long, status=0, tokens=8 * 2048, BH=128, T=2048, p=16, dv=64, C=64)
@@ -64,3 +65,23 @@ def test_report_line_has_per_path_points():
     assert ("chunked", 131072, 128) in key and ("quadratic", 131072, None) in key
     assert key[("quadratic", 2048, None)]["bound"] == "tensor" and ("chunked", 2048, 64) in key
     assert any(p["path"] == "decode" for p in pts)
+
+
+def test_backward_passes_are_reported_against_their_rooflines():
+    """The chunked backward's HBM fraction counts q, k, v, o, dO, D read and
+    dq, dk, dv written once (8p + 8dv + 4 bytes per token-head); the flash
+    backward's tensor fraction counts 2(3p + 2dv) flops per causal pair."""
+    args = argparse.Namespace(workload="layer340m_ctx2k", steps=1000, warmup=10, cpu_baseline=0)
+    buf = io.StringIO()
+    with redirect_stdout(buf):
+        bench.report(args, _fake_result(), 0.116, 11.0, 1)
+    line = json.loads(buf.getvalue().strip().splitlines()[-1])
+    assert bench.chunked_bwd_bytes(16, 131072, 16, 64) == 16 * 131072 * 644
+    c = line["train"]["chunked"]["B1_T131072"]
+    assert abs(c["bwd_hbm_frac"] - 16 * 131072 * 644 / 1.6e-3 / 1e9 / 6551.0) < 1e-12
+    pts = {(p["path"], p.get("T")): p for p in line["roofline"]["points"]}
+    assert pts[("bwd_chunked", 131072)]["bound"] == "hbm"
+    assert abs(pts[("bwd_chunked", 131072)]["frac"] - c["bwd_hbm_frac"]) < 1e-12
+    bq = pts[("bwd_quadratic", 2048)]
+    assert bq["bound"] == "tensor"
+    assert abs(bq["achieved"] - 128 * 2048 * 2049 / 2 * 2 * (3 * 16 + 2 * 64) / 0.36e-3 / 1e12) < 1e-6
